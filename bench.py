@@ -1,0 +1,477 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 HSA forward path (landmarks -> top-k selection ->
+chunk attention + fusion), through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step is one pass of the whole path over one prefill sequence of the
+prefill_bf16 workload (B1, T 65536, H32/Hkv8, d128, S64, k16, bf16).  Ranks
+under torchrun each run their own sequence (weak scaling; no data-path
+collective).  The timed region is bracketed by a barrier and a device
+synchronise, and timed with CUDA events on the launching stream.  The reported
+time is the maximum over ranks.  The inputs (Q 512 MiB, K and V 128 MiB each)
+are larger than L2, so no flush is needed between prefill steps.  The decode
+line (decode_1m: batch 8, 1M cached tokens) flushes L2 before every step.
+
+--impl reference times the CPU oracle instead (the task has no other
+reference implementation), on a bounded sample of the same workload.
+Rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HSA prefill tokens/s & decode µs/token at 1M ctx; % of HBM / tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device)
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.read().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.out.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- algorithmic work
+
+def ncand_rows(p) -> np.ndarray:
+    t = np.arange(p.Tq, dtype=np.int64)
+    return np.minimum((p.q_pos0 + t) // p.S, p.C)
+
+
+def work_counts(p, keff_sum: int) -> dict:
+    """Algorithmic work of one forward call (what the method must do: causal
+    candidate chunks only, k_eff chunks of S keys per query head)."""
+    es = 2 if p.dtype == "bf16" else 4
+    lm_bytes = (p.B * p.Tkv * p.Hkv * p.d + p.d * p.d + p.B * p.Hkv * p.C * p.d) * es
+    sel_flops = 2.0 * p.d * p.H * float(ncand_rows(p).sum()) * p.B
+    att_flops = 4.0 * p.S * p.d * p.G * float(keff_sum)
+    att_bytes = (2 * p.B * p.Tq * p.H * p.d) * es + 2 * p.B * p.Tkv * p.Hkv * p.d * es
+    return {"landmarks_bytes": lm_bytes, "select_flops": sel_flops, "attend_flops": att_flops,
+            "attend_bytes": att_bytes}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_b200(args, world, rank, local):
+    import landmark_guided_chunk_b200 as hsa
+    from landmark_guided_chunk_b200.inputs import make_inputs, workload
+
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    p = workload(args.workload)
+    inp = make_inputs(p, seed=args.seed + rank, device=dev)
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau,
+                            torch.bfloat16 if p.dtype == "bf16" else torch.float32)
+    plan = hsa.plan(prob)
+    ws = hsa.alloc_workspace(prob, dev)
+    L = torch.empty(p.B, p.Hkv, p.C, p.d, dtype=Q.dtype, device=dev)
+    O = torch.empty_like(Q)
+    km = hsa.kmax_of(p.k, p.tau)
+    idx = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.int32, device=dev)
+    score = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.float32, device=dev)
+    keff = torch.empty(p.B, p.Tq, p.Hkv, dtype=torch.int32, device=dev)
+    lib = hsa._native.lib()
+    P = hsa._p
+    st = torch.cuda.current_stream(dev)
+    sp = st.cuda_stream
+
+    def stage_landmarks():
+        hsa._native.check(lib.hsa_landmarks(ctypes.byref(prob), P(K), P(W), P(L), sp), "hsa_landmarks")
+
+    def stage_select():
+        hsa._native.check(lib.hsa_select(ctypes.byref(prob), P(Q), P(L), P(idx), P(score), P(keff), P(ws),
+                                         ws.numel(), sp), "hsa_select")
+
+    def stage_attend():
+        hsa._native.check(lib.hsa_attend(ctypes.byref(prob), P(Q), P(K), P(V), P(idx), P(score), P(keff),
+                                         P(O), P(ws), ws.numel(), sp), "hsa_attend")
+
+    stages = [("landmarks", stage_landmarks), ("select", stage_select), ("attend", stage_attend)]
+    for _ in range(args.warmup):
+        for _, f in stages:
+            f()
+    torch.cuda.synchronize(dev)
+    keff_sum = int(keff.sum().item())
+    work = work_counts(p, keff_sum)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for s in range(args.steps):
+        ev[s][0].record(st)
+        for i, (_, f) in enumerate(stages):
+            f()
+            ev[s][i + 1].record(st)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world)
+    total_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
+    stage_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / args.steps
+                for i, (name, _) in enumerate(stages)}
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    tokens_all = p.B * p.Tq * world
+    value = tokens_all / (ms_step * 1e-3)
+
+    # end to end through hsa_forward with host buffers (pinned), copies inside the timed region
+    Qh, Kh, Vh, Wh = (x.cpu().pin_memory() for x in (Q, K, V, W))
+    Oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    Qd, Kd, Vd, Wd = (torch.empty_like(x) for x in (Q, K, V, W))
+    e2e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        for dst, src in ((Qd, Qh), (Kd, Kh), (Vd, Vh), (Wd, Wh)):
+            dst.copy_(src, non_blocking=True)
+        hsa.forward(Qd, Kd, Vd, Wd, p.S, p.k, p.tau, p.q_pos0, L=L, O=O, ws=ws)
+        Oh.copy_(O, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    h2d = sum(x.numel() * x.element_size() for x in (Qh, Kh, Vh, Wh))
+    d2h = Oh.numel() * Oh.element_size()
+    del Qh, Kh, Vh, Wh, Oh, Qd, Kd, Vd, Wd
+
+    # roofline of each stage and of the dominant one
+    stage_rf = {
+        "landmarks": {"bound": "hbm", "work": work["landmarks_bytes"], "unit": "GB/s", "peak": pk["hbm_gbs"]},
+        "select": {"bound": "tensor", "work": work["select_flops"], "unit": "TFLOP/s",
+                   "peak": pk["bf16_tflops_sustained"]},
+        "attend": {"bound": "tensor", "work": work["attend_flops"], "unit": "TFLOP/s",
+                   "peak": pk["bf16_tflops_sustained"]},
+    }
+    stages_out = {}
+    for name, rf in stage_rf.items():
+        ms = stage_ms[name]
+        scale = 1e-9 if rf["unit"] == "GB/s" else 1e-12
+        ach = rf["work"] * scale / (ms * 1e-3)
+        stages_out[name] = {"ms": round(ms, 4), "path": plan[name][0], "kernels": plan[name][1],
+                            "achieved": round(ach, 2), "unit": rf["unit"], "bound": rf["bound"],
+                            "frac": round(ach / rf["peak"], 4)}
+    dom = max(stage_ms, key=stage_ms.get)
+    traffic = dram_traffic(dom, plan[dom][0])
+    roof = {"bound": stage_rf[dom]["bound"], "kernel": f"hsa_{dom} ({plan[dom][0]})",
+            "achieved": stages_out[dom]["achieved"], "peak": stage_rf[dom]["peak"], "unit": stage_rf[dom]["unit"],
+            "frac": stages_out[dom]["frac"], "traffic": traffic,
+            "peak_source": f"{pk['source']} ({'sustained bf16' if stage_rf[dom]['unit'] == 'TFLOP/s' else 'HBM copy'})"}
+    launches = args.steps * (plan["landmarks"][1] + plan["select"][1] + plan["attend"][1])
+
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": f"{p.name}: B{p.B} T{p.Tq} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
+                      "global_batch": p.B * world, "seq_len": p.Tq, "parallelism": f"dp{world} (one sequence per GPU)",
+                      "l2": "inputs larger than L2 (Q 512 MiB, K and V 128 MiB each); no flush"},
+           "e2e": {"value": round(tokens_all / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+           "gpu_launches": launches, "roofline": roof, "stages": stages_out, "clocks": clk,
+           "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3)}
+    del inp, Q, K, V, W, L, O, idx, score, keff, ws
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        out["decode_1m"] = run_decode(args, world, rank, local, pk)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(p, args.seed)
+    return out
+
+
+def run_decode(args, world, rank, local, pk):
+    """Decode step at 1M context (decode_1m): landmarks precomputed, L2 flushed
+    before each step, each step timed alone."""
+    import landmark_guided_chunk_b200 as hsa
+    from landmark_guided_chunk_b200.inputs import make_inputs, workload
+
+    dev = torch.device("cuda", local)
+    p = workload("decode_1m")
+    inp = make_inputs(p, seed=args.seed + rank, device=dev)
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, torch.bfloat16,
+                            hsa._native.HSA_FLAG_LANDMARKS_READY)
+    plan = hsa.plan(prob)
+    ws = hsa.alloc_workspace(prob, dev)
+    O = torch.empty_like(Q)
+    scrub = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+    steps = max(args.steps, 10)
+
+    def step():
+        hsa.forward(Q, K, V, None, p.S, p.k, p.tau, p.q_pos0, L=L, landmarks_ready=True, O=O, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    times = []
+    for _ in range(steps):
+        scrub.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        step()
+        b.record(st)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    us = max_over_ranks(1e3 * statistics.median(times), world)
+    # compulsory HBM bytes of one decode step: the landmark scan plus the k_eff chunks' K and V per (b, kv head)
+    scan = p.B * p.Hkv * p.C * p.d * 2
+    gather = p.B * p.Hkv * p.k * p.S * p.d * 2 * 2
+    gbs = (scan + gather) / (us * 1e-6) * 1e-9
+    res = {"workload": f"decode_1m: B{p.B} ctx {p.Tkv} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
+           "us_per_step": round(us, 2), "us_per_token": round(us / p.B, 3),
+           "tokens_per_s": round(p.B * world / (us * 1e-6), 1),
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / pk["hbm_gbs"], 4), "bytes_per_step": scan + gather},
+           "l2": "512 MiB scrub before every step", "paths": plan,
+           "gpu_launches_per_step": plan["select"][1] + plan["attend"][1]}
+    del inp, Q, K, V, W, L, O, ws, scrub
+    torch.cuda.empty_cache()
+    return res
+
+
+def dram_traffic(stage: str, path: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary,
+    if it was taken on the kernel source that is built now; else None."""
+    f = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(f) as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    ent = d.get(f"{stage}:{path}")
+    if not ent:
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for src in ent.get("sources", []):
+        with open(os.path.join(ROOT, src), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != ent.get("source_hash"):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- CPU baseline (oracle)
+
+def _sample_positions(p, n, seed):
+    rng = np.random.default_rng(seed)
+    edges = np.linspace(0, p.Tq, n + 1).astype(np.int64)
+    return np.array([rng.integers(edges[i], max(edges[i] + 1, edges[i + 1])) for i in range(n)])
+
+
+def cpu_baseline(p, seed, n_tokens=None, budget_s=20.0):
+    """The oracle, as it stands, on a bounded sample of the same workload: the
+    landmarks of every chunk (timed), then selection + attention + fusion for
+    n_tokens positions spread evenly over the sequence (all kv heads).  The
+    throughput is tokens / (time per token of the rows + landmark time per
+    token)."""
+    import oracle
+    from landmark_guided_chunk_b200.inputs import make_inputs
+
+    inp = make_inputs(p, seed=seed, device="cpu")
+    K, W = inp["K"], inp["W_L"]
+    t0 = time.perf_counter()
+    L = oracle.landmarks_stored(K, W, p.S, p.dtype)
+    t_lm = time.perf_counter() - t0
+    if n_tokens is None:
+        # size the row sample from a short probe so the whole baseline stays near budget_s
+        probe = _sample_positions(p, 8, seed)
+        t0 = time.perf_counter()
+        oracle.forward_rows(inp["Q"], K, inp["V"], W, p.S, p.k, p.tau, p.q_pos0, np.zeros(8, int), probe, L=L)
+        per = (time.perf_counter() - t0) / 8
+        n_tokens = int(max(16, min(4096, (budget_s - t_lm) / max(per, 1e-6))))
+    pos = _sample_positions(p, n_tokens, seed + 1)
+    t0 = time.perf_counter()
+    oracle.forward_rows(inp["Q"], K, inp["V"], W, p.S, p.k, p.tau, p.q_pos0, np.zeros(n_tokens, int), pos, L=L)
+    t_rows = time.perf_counter() - t0
+    per_token = t_rows / n_tokens + t_lm / (p.B * p.Tq)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(1.0 / per_token, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"landmarks of all {p.B * p.C} chunks ({t_lm:.2f} s) + selection/attention/fusion of "
+                      f"{n_tokens} positions spread over the sequence, all {p.Hkv} kv heads ({t_rows:.2f} s)"}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step processes S sampled query
+    positions (all kv heads) plus the landmarks of one chunk of keys."""
+    import oracle
+    from landmark_guided_chunk_b200.inputs import make_inputs, workload
+
+    p = workload(args.workload)
+    inp = make_inputs(p, seed=args.seed, device="cpu")
+    K, W = inp["K"], inp["W_L"]
+    L = oracle.landmarks_stored(K, W, p.S, p.dtype)
+    rng = np.random.default_rng(args.seed)
+
+    def step():
+        c = int(rng.integers(0, p.C))
+        oracle.landmarks_stored(K[:, c * p.S:(c + 1) * p.S], W, p.S, p.dtype)
+        pos = np.sort(rng.integers(0, p.Tq, p.S))
+        oracle.forward_rows(inp["Q"], K, inp["V"], W, p.S, p.k, p.tau, p.q_pos0, np.zeros(p.S, int), pos, L=L)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = p.S / dt
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = (f"per step: {p.S} uniformly drawn query positions of {p.name} (all {p.Hkv} kv heads: selection, "
+              f"attention, fusion) + the landmarks of one chunk")
+    return {"metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{p.name}: B{p.B} T{p.Tq} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
+                       "global_batch": p.B, "seq_len": p.Tq, "parallelism": "cpu (oracle, all host cores)"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default="prefill_bf16", choices=["prefill_bf16", "router_bf16", "tiny_f32"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return
+    world, rank, local = dist_setup()
+    out = run_b200(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * hsa.h -- C ABI of the B200 (sm_100a) Hierarchical Sparse Attention forward path.
+ *
+ * Method: "Every Token Counts 16m Context" (HSA summary page), sections Core
+ * Technique and Implementation.  The key sequence is cut into fixed-length,
+ * non-overlapping chunks of S tokens.  Every chunk gets a landmark: the mean of
+ * its keys, projected by a learned d x d matrix W_L.  Every query scores the
+ * landmarks of the chunks strictly before its own and keeps the k best.  It
+ * attends inside each kept chunk with standard softmax attention.  The k chunk
+ * outputs are then fused, weighted by the softmax of their retrieval scores.
+ * The optional gap router (value-of-information router page, abstract) doubles
+ * k for rows whose top-k cut is nearly tied.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor arguments are DEVICE pointers.  The caller allocates them, and
+ *     also the workspace.  The library never allocates, keeps no global
+ *     mutable state, and is safe to call from several host threads on
+ *     different streams, each with its own workspace.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
+ *     the legacy default stream).  Host-side validation runs before any launch.
+ *     An invalid call launches nothing and returns a status.
+ *   - Layouts (row-major, contiguous, every pointer 16-byte aligned):
+ *       Q, O   [B][Tq][H][d]       K, V  [B][Tkv][Hkv][d]
+ *       W_L    [d][d]  (row = input dim: landmark = mean_row * W_L)
+ *       L      [B][Hkv][C][d],  C = floor(Tkv / S)
+ *       idx    [B][Tq][Hkv][kmax] int32   score [B][Tq][Hkv][kmax] float
+ *       keff   [B][Tq][Hkv] int32,        kmax = (tau > 0 ? 2k : k)
+ *     Q, K, V, W_L, L and O all have the problem's dtype.  Scores are fp32 and
+ *     indices int32.
+ *   - Query head h reads kv head floor(h / G), with G = H / Hkv.  One chunk
+ *     selection is made per (batch, query, kv head).  It ranks chunks by the
+ *     sum, over the G query heads, of the raw dot products q_h . L_c.
+ *   - The query at row t sits at absolute position p = q_pos0 + t.  Its
+ *     candidates are the complete chunks c < min(floor(p / S), C).  A trailing
+ *     partial chunk (Tkv mod S tokens) has no landmark and is never a
+ *     candidate.  Prefill: Tq == Tkv and q_pos0 = 0.  Decode: Tq = 1 and
+ *     q_pos0 = Tkv.
+ *   - Ranking: score descending, equal scores to the lower chunk index.
+ *     keff = min(k, #candidates).  With the router on, when #candidates > k
+ *     and (s_k - s_{k+1}) < tau * |s_k|: keff = min(2k, #candidates).
+ *     Unused slots hold idx = -1 and score = -inf.  A row with keff = 0
+ *     outputs zeros.
+ *   - Arithmetic: products of stored values, fp32 accumulation, fp32
+ *     softmax.  L and O are rounded once (to nearest, ties to even) to the
+ *     dtype.
+ *   - Errors are status codes only.  Nothing is thrown across the ABI.  A CUDA
+ *     launch failure maps to HSA_ERR_CUDA.  A kernel whose bounded wait expired
+ *     records HSA_ERR_TIMEOUT in the workspace header.
+ *     hsa_get_device_status() reports it.  Inputs are assumed finite.
+ */
+#ifndef HSA_H_
+#define HSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HSA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define HSA_API __attribute__((visibility("default")))
+#else
+#define HSA_API
+#endif
+
+typedef enum {
+    HSA_OK = 0,
+    HSA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misaligned pointer, bad tau */
+    HSA_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement (d, S, k) */
+    HSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than hsa_workspace_size() */
+    HSA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    HSA_ERR_TIMEOUT = 5        /* a device-side bounded wait expired (read via hsa_get_device_status) */
+} hsa_status_t;
+
+typedef enum { HSA_F32 = 0, HSA_BF16 = 1 } hsa_dtype_t;
+
+/* hsa_problem_t.flags */
+#define HSA_FLAG_LANDMARKS_READY 1u  /* hsa_forward: L already holds the landmarks; skip that stage (W_L may be NULL) */
+
+typedef struct {
+    int32_t B, Tq, Tkv, H, Hkv, d, S, k;
+    int64_t q_pos0;      /* absolute position of query row 0 */
+    float tau;           /* gap-router threshold; 0 disables it, > 0 enables it (then 2k <= 32) */
+    int32_t dtype;       /* hsa_dtype_t */
+    uint32_t flags;      /* HSA_FLAG_* */
+} hsa_problem_t;
+
+/* Supported shapes: d in {64, 128}; S in {32, 64, 128}; 1 <= k <= 32 (2k <= 32 with the
+ * router); H % Hkv == 0 and G = H / Hkv <= 16.  B, Tq or Tkv may be 0 (nothing to do). */
+
+/*
+ * Bytes of device workspace that hsa_select / hsa_attend / hsa_forward need for
+ * problem *p.  The workspace must be 256-byte aligned.  A call may use all of it
+ * and leaves no state in it that a later call depends on, except the
+ * device-status word that hsa_get_device_status() reads and clears.  Calls
+ * that overlap on the GPU must use distinct workspaces.
+ * Returns HSA_ERR_INVALID_ARG / HSA_ERR_UNSUPPORTED for a bad problem.
+ */
+HSA_API hsa_status_t hsa_workspace_size(const hsa_problem_t *p, size_t *bytes);
+
+/*
+ * Landmarks (summary page, Implementation: landmark = encode(mean pool of the
+ * chunk), with encode read as the d x d projection W_L):
+ *   L[b][j][c][:] = ( (1/S) sum_{u<S} K[b][cS+u][j][:] ) * W_L
+ * for every complete chunk c < C.  The mean and the projection are done in
+ * fp32, and the result is rounded once to the dtype.  Needs no workspace.
+ * Q-side fields (Tq, q_pos0, k, tau) are validated but not used.
+ */
+HSA_API hsa_status_t hsa_landmarks(const hsa_problem_t *p, const void *K, const void *W_L, void *L,
+                           void *stream);
+
+/*
+ * Chunk selection (summary page, Core Technique and Implementation: score all
+ * landmarks, keep the top k; router page: gap router).  Writes idx, score and
+ * keff as described above.  score holds the group-summed retrieval score of
+ * each kept chunk (fp32).
+ */
+HSA_API hsa_status_t hsa_select(const hsa_problem_t *p, const void *Q, const void *L, int32_t *idx,
+                        float *score, int32_t *keff, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Chunk attention and fusion (summary page, Implementation: attend to each
+ * selected chunk with standard attention, then fuse the results weighted by
+ * the retrieval scores).  For each (b, t, kv head j) and each head h of the
+ * group:
+ *   w_i  = softmax_{i < keff}(score_i)
+ *   o_i  = softmax_u(q_h . K[c_i S + u] / sqrt(d)) . V[c_i S + u]     (u < S)
+ *   O[h] = sum_i w_i o_i                                              (0 when keff = 0)
+ * idx/score/keff are as hsa_select writes them.  Every idx[i] for i < keff
+ * must be a valid candidate chunk of its row.
+ */
+HSA_API hsa_status_t hsa_attend(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
+                        const int32_t *idx, const float *score, const int32_t *keff, void *O,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The whole path: hsa_landmarks (unless HSA_FLAG_LANDMARKS_READY), then
+ * hsa_select, then hsa_attend.  L is an output (or an input with the flag).
+ * idx, score and keff may each be NULL.  The selection then lives only in the
+ * workspace.
+ */
+HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
+                         const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
+                         void *O, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-status word in the
+ * workspace header.  Returns HSA_OK, HSA_ERR_TIMEOUT (a bounded device wait
+ * expired in an earlier call on this workspace) or HSA_ERR_CUDA.
+ */
+HSA_API hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream);
+
+/* Kernel paths a stage can take (hsa_plan_t.*_path). */
+typedef enum {
+    HSA_PATH_NONE = 0,         /* stage has nothing to do for this problem */
+    HSA_PATH_SIMT_ROWS = 1,    /* CUDA cores, one warp / CTA per selection row */
+    HSA_PATH_SIMT_SPLIT = 2,   /* CUDA cores, each row split over CTAs, then merged */
+    HSA_PATH_TENSOR = 3        /* tcgen05 tensor-core kernel */
+} hsa_path_t;
+
+typedef struct {
+    int32_t landmark_path, select_path, attend_path;        /* hsa_path_t */
+    int32_t landmark_kernels, select_kernels, attend_kernels; /* kernel launches per call of each stage */
+} hsa_plan_t;
+
+/*
+ * Which kernels hsa_landmarks / hsa_select / hsa_attend launch for problem *p
+ * (a pure function of the problem; nothing is launched).  hsa_forward launches
+ * the sum of the three (minus the landmark stage with HSA_FLAG_LANDMARKS_READY).
+ */
+HSA_API hsa_status_t hsa_plan(const hsa_problem_t *p, hsa_plan_t *plan);
+
+/* Static description of a status code. */
+HSA_API const char *hsa_status_string(hsa_status_t s);
+
+/* Detail of the last failing call on this host thread (which argument, which CUDA error). */
+HSA_API const char *hsa_last_error(void);
+
+/* HSA_ABI_VERSION of the loaded library. */
+HSA_API int hsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HSA_H_ */

@@ -1,1 +1,160 @@
-"""B200-native Hierarchical Sparse Attention (HSA) forward path (placeholder; the binding lands with the C-ABI)."""
+"""B200-native Hierarchical Sparse Attention (HSA) forward path.
+
+Method: "Every Token Counts 16m Context" (HSA summary page), Core Technique
+and Implementation.  The sequence is cut into chunks of S tokens, each with a
+landmark (the mean of its keys times W_L).  Each query keeps the top-k
+strictly-past chunks by landmark score, attends inside each kept chunk, and
+fuses the chunk outputs by the softmax of their retrieval scores.  The gap
+router of the value-of-information router page optionally doubles k.
+
+Python surface over the C ABI in include/hsa.h (libhsa_b200.so).  Torch
+supplies device memory and the current stream.  Every step runs in the CUDA
+kernels of that library, and there is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native
+from ._native import HSAError, hsa_problem_t
+
+__all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "attend",
+           "forward", "device_status", "HSAError", "hsa_problem_t", "kmax_of"]
+
+_DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
+
+
+def make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0=0, tau=0.0, dtype=torch.bfloat16, flags=0) -> hsa_problem_t:
+    if dtype not in _DT:
+        raise TypeError(f"dtype {dtype} not supported (float32, bfloat16)")
+    return hsa_problem_t(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, _DT[dtype], flags)
+
+
+def plan(prob: hsa_problem_t) -> dict:
+    """Kernel path and launch count of each stage for this problem (nothing is launched)."""
+    pl = _native.hsa_plan_t()
+    _native.check(_native.lib().hsa_plan(ctypes.byref(prob), ctypes.byref(pl)), "hsa_plan")
+    names = _native.PATH_NAMES
+    return {"landmarks": (names[pl.landmark_path], pl.landmark_kernels),
+            "select": (names[pl.select_path], pl.select_kernels),
+            "attend": (names[pl.attend_path], pl.attend_kernels)}
+
+
+def kmax_of(k: int, tau: float) -> int:
+    return 2 * k if tau > 0 else k
+
+
+def workspace_size(prob: hsa_problem_t) -> int:
+    n = ctypes.c_size_t(0)
+    _native.check(_native.lib().hsa_workspace_size(ctypes.byref(prob), ctypes.byref(n)), "hsa_workspace_size")
+    return int(n.value)
+
+
+def alloc_workspace(prob: hsa_problem_t, device=None) -> torch.Tensor:
+    """A uint8 device buffer of hsa_workspace_size bytes (torch allocations are 256-byte aligned)."""
+    n = max(256, workspace_size(prob))
+    ws = torch.empty(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def landmarks(K: torch.Tensor, W_L: torch.Tensor, S: int, L: torch.Tensor | None = None) -> torch.Tensor:
+    """L [B,Hkv,C,d] = mean of each complete chunk's keys times W_L (rounded once to K's dtype)."""
+    _dev(K, W_L, L)
+    B, Tkv, Hkv, d = K.shape
+    C = Tkv // S
+    if L is None:
+        L = torch.empty(B, Hkv, C, d, dtype=K.dtype, device=K.device)
+    prob = make_problem(B, 0, Tkv, Hkv, Hkv, d, S, 1, 0, 0.0, K.dtype)
+    _native.check(_native.lib().hsa_landmarks(ctypes.byref(prob), _p(K), _p(W_L), _p(L), _stream(K)),
+                  "hsa_landmarks")
+    return L
+
+
+def _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags=0):
+    B, Tq, H, d = Q.shape
+    return make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, Q.dtype, flags)
+
+
+def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None):
+    """Top-k chunk selection.  Returns (idx int32, score fp32 [B,Tq,Hkv,kmax], keff int32 [B,Tq,Hkv])."""
+    _dev(Q, L, ws)
+    B, Tq, H, d = Q.shape
+    Hkv, C = L.shape[1], L.shape[2]
+    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0)
+    km = kmax_of(k, tau)
+    idx = torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device)
+    score = torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device)
+    keff = torch.empty(B, Tq, Hkv, dtype=torch.int32, device=Q.device)
+    if ws is None:
+        ws = alloc_workspace(prob, Q.device)
+    _native.check(_native.lib().hsa_select(ctypes.byref(prob), _p(Q), _p(L), _p(idx), _p(score), _p(keff),
+                                           _p(ws), ws.numel(), _stream(Q)), "hsa_select")
+    return idx, score, keff
+
+
+def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None):
+    """Chunk attention + fusion for a given selection.  Returns O [B,Tq,H,d]."""
+    _dev(Q, K, V, idx, score, keff, O, ws)
+    prob = _prob_from(Q, K.shape[1], K.shape[2], S, k, tau, q_pos0)
+    if O is None:
+        O = torch.empty_like(Q)
+    if ws is None:
+        ws = alloc_workspace(prob, Q.device)
+    _native.check(_native.lib().hsa_attend(ctypes.byref(prob), _p(Q), _p(K), _p(V), _p(idx), _p(score),
+                                           _p(keff), _p(O), _p(ws), ws.numel(), _stream(Q)), "hsa_attend")
+    return O
+
+
+def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False, O=None, ws=None,
+            return_selection=False):
+    """The whole HSA forward.  Returns O, or (O, L, idx, score, keff) with return_selection."""
+    _dev(Q, K, V, W_L, L, O, ws)
+    B, Tq, H, d = Q.shape
+    Tkv, Hkv = K.shape[1], K.shape[2]
+    flags = _native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags)
+    if L is None:
+        if landmarks_ready:
+            raise ValueError("landmarks_ready needs L")
+        L = torch.empty(B, Hkv, Tkv // S, d, dtype=Q.dtype, device=Q.device)
+    if O is None:
+        O = torch.empty_like(Q)
+    if ws is None:
+        ws = alloc_workspace(prob, Q.device)
+    sel = (None, None, None)
+    if return_selection:
+        km = kmax_of(k, tau)
+        sel = (torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device),
+               torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device),
+               torch.empty(B, Tq, Hkv, dtype=torch.int32, device=Q.device))
+    _native.check(_native.lib().hsa_forward(ctypes.byref(prob), _p(Q), _p(K), _p(V), _p(W_L), _p(L),
+                                            _p(sel[0]), _p(sel[1]), _p(sel[2]), _p(O), _p(ws), ws.numel(),
+                                            _stream(Q)), "hsa_forward")
+    if return_selection:
+        return (O, L) + sel
+    return O
+
+
+def device_status(ws: torch.Tensor) -> None:
+    """Synchronise and raise HSAError if a bounded device wait expired on this workspace."""
+    _native.check(_native.lib().hsa_get_device_status(_p(ws), ws.numel(), _stream(ws)),
+                  "hsa_get_device_status")

@@ -1,0 +1,81 @@
+"""ctypes view of libhsa_b200.so (the C ABI in include/hsa.h).
+
+Argument marshalling only.  Every step of the method runs in the CUDA library.
+There is no fallback: if the library is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhsa_b200.so")
+
+HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT = range(6)
+HSA_F32, HSA_BF16 = 0, 1
+HSA_FLAG_LANDMARKS_READY = 1
+
+EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
+            "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version")
+PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor"}
+
+
+class hsa_problem_t(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Tq", ctypes.c_int32), ("Tkv", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("S", ctypes.c_int32), ("k", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
+                ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class hsa_plan_t(ctypes.Structure):
+    _fields_ = [("landmark_path", ctypes.c_int32), ("select_path", ctypes.c_int32),
+                ("attend_path", ctypes.c_int32), ("landmark_kernels", ctypes.c_int32),
+                ("select_kernels", ctypes.c_int32), ("attend_kernels", ctypes.c_int32)]
+
+
+class HSAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {detail}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once.  Raises if it is missing.  There is no other path."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"HSA CUDA library not built: {LIB_PATH} is missing "
+                           "(run landmark_guided_chunk_b200/build.py or __graft_entry__.build())")
+    L = ctypes.CDLL(LIB_PATH)
+    P, Z, I32p, Fp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
+    prob = ctypes.POINTER(hsa_problem_t)
+    L.hsa_workspace_size.argtypes = [prob, ctypes.POINTER(ctypes.c_size_t)]
+    L.hsa_landmarks.argtypes = [prob, P, P, P, P]
+    L.hsa_select.argtypes = [prob, P, P, I32p, Fp, I32p, P, Z, P]
+    L.hsa_attend.argtypes = [prob, P, P, P, I32p, Fp, I32p, P, P, Z, P]
+    L.hsa_forward.argtypes = [prob, P, P, P, P, P, I32p, Fp, I32p, P, P, Z, P]
+    L.hsa_get_device_status.argtypes = [P, Z, P]
+    L.hsa_plan.argtypes = [prob, ctypes.POINTER(hsa_plan_t)]
+    L.hsa_status_string.argtypes = [ctypes.c_int]
+    L.hsa_status_string.restype = ctypes.c_char_p
+    L.hsa_last_error.argtypes = []
+    L.hsa_last_error.restype = ctypes.c_char_p
+    L.hsa_abi_version.argtypes = []
+    L.hsa_abi_version.restype = ctypes.c_int
+    for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
+              "hsa_get_device_status", "hsa_plan"):
+        getattr(L, f).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def check(status: int, where: str) -> None:
+    if status != HSA_OK:
+        L = lib()
+        detail = L.hsa_last_error().decode() or L.hsa_status_string(status).decode()
+        raise HSAError(status, where, f"{L.hsa_status_string(status).decode()} -- {detail}")

@@ -1,0 +1,166 @@
+// common.cuh -- shared device helpers and the internal launch interface of the
+// HSA library.  Host code outside this library never includes it.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "hsa.h"
+
+namespace hsa {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int MAX_KMAX = 32;   // selection slots per row (2k with the router)
+constexpr int MAX_G = 16;      // query heads per kv head
+
+// Validated problem with the derived quantities every stage uses.
+struct Prob {
+    int B, Tq, Tkv, H, Hkv, d, S, k, G, C, kmax, dtype;
+    long long q_pos0;
+    float tau;
+    unsigned flags;
+    long long rows;   // B * Tq * Hkv selection rows
+};
+
+// Byte offsets inside the caller's workspace (all 256-byte aligned).
+struct WsLayout {
+    size_t hdr;          // device-status word (uint32) + padding
+    size_t sel_idx, sel_score, sel_keff;   // selection outputs when hsa_forward gets NULLs
+    size_t split_lists;  // decode split scan: rows x nsplit x kmax (score, id)
+    size_t partials;     // decode split attend: rows x kmax x G x d fp32
+    size_t total;
+    int nsplit, chunks_per_split;
+    bool split_select, split_attend;
+    hsa_plan_t plan;     // kernel paths and launch counts per stage
+};
+
+WsLayout ws_layout(const Prob &p);
+
+// status word values (workspace header)
+constexpr uint32_t DEV_OK = 0;
+constexpr uint32_t DEV_TIMEOUT = 1;
+
+// ---------------------------------------------------------------------------- element access
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Dot product of an fp32 vector in shared memory with one stored row (16-byte aligned),
+// accumulated in fp32 in index order.
+__device__ __forceinline__ float dot_row(const float *__restrict__ q, const float *__restrict__ row, int d) {
+    float acc = 0.f;
+    const float4 *r4 = reinterpret_cast<const float4 *>(row);
+    for (int x = 0; x < d / 4; ++x) {
+        float4 v = __ldg(r4 + x);
+        acc = fmaf(q[4 * x + 0], v.x, acc);
+        acc = fmaf(q[4 * x + 1], v.y, acc);
+        acc = fmaf(q[4 * x + 2], v.z, acc);
+        acc = fmaf(q[4 * x + 3], v.w, acc);
+    }
+    return acc;
+}
+
+__device__ __forceinline__ float dot_row(const float *__restrict__ q, const __nv_bfloat16 *__restrict__ row, int d) {
+    float acc = 0.f;
+    const uint4 *r4 = reinterpret_cast<const uint4 *>(row);
+    for (int x = 0; x < d / 8; ++x) {
+        uint4 u = __ldg(r4 + x);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            float2 f = __bfloat1622float2(h2[y]);
+            acc = fmaf(q[8 * x + 2 * y + 0], f.x, acc);
+            acc = fmaf(q[8 * x + 2 * y + 1], f.y, acc);
+        }
+    }
+    return acc;
+}
+
+// ---------------------------------------------------------------------------- warp top-k list
+// A sorted list of up to kmax (<= 32) entries spread over a warp: lane i holds
+// entry i as (v, id).  Order: v descending, id ascending.  Empty entries are
+// (-inf, INT32_MAX) and rank after every real candidate.
+
+__device__ __forceinline__ bool ranks_before(float v1, int id1, float v2, int id2) {
+    return v1 > v2 || (v1 == v2 && id1 < id2);
+}
+
+__device__ __forceinline__ void list_init(float &v, int &id) {
+    v = -INFINITY;
+    id = INT32_MAX;
+}
+
+// Insert (s, c) (the same on every lane) if it ranks before entry kmax-1.
+__device__ __forceinline__ void list_insert(float &v, int &id, float s, int c, int kmax, int lane) {
+    float vl = __shfl_sync(FULL, v, kmax - 1);
+    int il = __shfl_sync(FULL, id, kmax - 1);
+    if (!ranks_before(s, c, vl, il)) return;
+    unsigned before = __ballot_sync(FULL, lane < kmax && ranks_before(v, id, s, c));
+    int pos = __popc(before);
+    float vu = __shfl_up_sync(FULL, v, 1);
+    int iu = __shfl_up_sync(FULL, id, 1);
+    if (lane < kmax) {
+        if (lane == pos) {
+            v = s;
+            id = c;
+        } else if (lane > pos) {
+            v = vu;
+            id = iu;
+        }
+    }
+}
+
+// Offer one candidate per lane (valid lanes only); inserts those that qualify,
+// in lane order.
+__device__ __forceinline__ void list_offer(float &v, int &id, float s, int c, bool valid, int kmax, int lane) {
+    float vl = __shfl_sync(FULL, v, kmax - 1);
+    int il = __shfl_sync(FULL, id, kmax - 1);
+    unsigned m = __ballot_sync(FULL, valid && ranks_before(s, c, vl, il));
+    while (m) {
+        int src = __ffs(m) - 1;
+        m &= m - 1;
+        float sv = __shfl_sync(FULL, s, src);
+        int cv = __shfl_sync(FULL, c, src);
+        list_insert(v, id, sv, cv, kmax, lane);
+    }
+}
+
+// keff for a row from its sorted list (entries k-1 and k), with the gap router.
+__device__ __forceinline__ int list_keff(float v, int ncand, int k, int kmax, float tau) {
+    int ke = ncand < k ? ncand : k;
+    float sk = __shfl_sync(FULL, v, k - 1);
+    float sk1 = __shfl_sync(FULL, v, kmax > k ? k : k - 1);
+    if (tau > 0.f && ncand > k && (sk - sk1) < tau * fabsf(sk)) ke = ncand < 2 * k ? ncand : 2 * k;
+    return ke;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+
+// ---------------------------------------------------------------------------- launchers
+// Each returns a cudaError_t from the launch; shapes are already validated.
+
+cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
+cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
+                          float *score, int32_t *keff, char *ws, cudaStream_t st);
+cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const void *K, const void *V,
+                          const int32_t *idx, const float *score, const int32_t *keff, void *O, char *ws,
+                          cudaStream_t st);
+
+}  // namespace hsa

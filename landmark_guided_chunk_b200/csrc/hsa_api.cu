@@ -1,0 +1,270 @@
+// hsa_api.cu -- the C ABI declared in include/hsa.h: host-side validation,
+// workspace layout and stage dispatch.  No entry point allocates memory,
+// throws, or keeps global mutable state (the last-error text is per host
+// thread).
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+
+namespace hsa {
+
+static thread_local char g_err[512] = "";
+
+static hsa_status_t fail(hsa_status_t s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+static hsa_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(HSA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const Prob &p) {
+    WsLayout w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t rows = (size_t)p.rows;
+    w.hdr = take(256);
+    w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
+    w.sel_score = take(rows * p.kmax * sizeof(float));
+    w.sel_keff = take(rows * sizeof(int32_t));
+    // Few rows with long scans: split each row's chunk range over CTAs.
+    w.split_select = rows > 0 && rows <= 4096 && p.C >= 2048;
+    if (w.split_select) {
+        const long long target = 148 * 8;
+        long long per_row = (target + (long long)rows - 1) / (long long)rows;
+        long long cps = ((long long)p.C + per_row - 1) / per_row;
+        cps = ((cps + 255) / 256) * 256;
+        if (cps < 256) cps = 256;
+        w.chunks_per_split = (int)cps;
+        w.nsplit = (int)(((long long)p.C + cps - 1) / cps);
+        w.split_lists = take(rows * (size_t)w.nsplit * p.kmax * sizeof(float2));
+    }
+    // Few rows: parallelise the attention over the kept slots too.
+    w.split_attend = rows > 0 && rows <= 2048;
+    if (w.split_attend) w.partials = take(rows * (size_t)p.kmax * p.G * p.d * sizeof(float));
+    w.total = off;
+    const bool has_chunks = (long long)p.B * p.C > 0;
+    w.plan.landmark_path = has_chunks ? HSA_PATH_SIMT_ROWS : HSA_PATH_NONE;
+    w.plan.landmark_kernels = has_chunks ? 1 : 0;
+    w.plan.select_path = rows == 0 ? HSA_PATH_NONE : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
+    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select ? 2 : 1);
+    w.plan.attend_path = rows == 0 ? HSA_PATH_NONE : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
+    w.plan.attend_kernels = rows == 0 ? 0 : (w.split_attend ? 2 : 1);
+    return w;
+}
+
+static hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
+    if (!in) return fail(HSA_ERR_INVALID_ARG, "problem pointer is NULL");
+    if (in->B < 0 || in->Tq < 0 || in->Tkv < 0)
+        return fail(HSA_ERR_INVALID_ARG, "negative size (B=%d Tq=%d Tkv=%d)", in->B, in->Tq, in->Tkv);
+    if (in->H < 1 || in->Hkv < 1 || in->d < 1 || in->S < 1 || in->k < 1)
+        return fail(HSA_ERR_INVALID_ARG, "H, Hkv, d, S, k must be >= 1 (H=%d Hkv=%d d=%d S=%d k=%d)", in->H, in->Hkv,
+                    in->d, in->S, in->k);
+    if (in->H % in->Hkv != 0) return fail(HSA_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", in->H, in->Hkv);
+    if (in->dtype != HSA_F32 && in->dtype != HSA_BF16) return fail(HSA_ERR_INVALID_ARG, "unknown dtype %d", in->dtype);
+    if (!(in->tau >= 0.0f) || isinf(in->tau)) return fail(HSA_ERR_INVALID_ARG, "tau must be finite and >= 0");
+    if (in->q_pos0 < 0) return fail(HSA_ERR_INVALID_ARG, "q_pos0 must be >= 0");
+    if (in->flags & ~HSA_FLAG_LANDMARKS_READY) return fail(HSA_ERR_INVALID_ARG, "unknown flags 0x%x", in->flags);
+    if (in->d != 64 && in->d != 128) return fail(HSA_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", in->d);
+    if (in->S != 32 && in->S != 64 && in->S != 128)
+        return fail(HSA_ERR_UNSUPPORTED, "S=%d (supported: 32, 64, 128)", in->S);
+    const int kmax = in->tau > 0.0f ? 2 * in->k : in->k;
+    if (kmax > MAX_KMAX) return fail(HSA_ERR_UNSUPPORTED, "k=%d gives %d slots (max %d)", in->k, kmax, MAX_KMAX);
+    if (in->H / in->Hkv > MAX_G) return fail(HSA_ERR_UNSUPPORTED, "G=%d (max %d)", in->H / in->Hkv, MAX_G);
+    if (in->B > 65535) return fail(HSA_ERR_UNSUPPORTED, "B=%d (max 65535)", in->B);
+    p->B = in->B;
+    p->Tq = in->Tq;
+    p->Tkv = in->Tkv;
+    p->H = in->H;
+    p->Hkv = in->Hkv;
+    p->d = in->d;
+    p->S = in->S;
+    p->k = in->k;
+    p->G = in->H / in->Hkv;
+    p->C = in->Tkv / in->S;
+    p->kmax = kmax;
+    p->dtype = in->dtype;
+    p->q_pos0 = in->q_pos0;
+    p->tau = in->tau;
+    p->flags = in->flags;
+    p->rows = (long long)in->B * in->Tq * in->Hkv;
+    return HSA_OK;
+}
+
+static bool aligned16(const void *x) { return ((uintptr_t)x & 15u) == 0; }
+
+static hsa_status_t need(const void *x, bool required, const char *name) {
+    if (!required) return HSA_OK;
+    if (!x) return fail(HSA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(x)) return fail(HSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return HSA_OK;
+}
+
+#define HSA_TRY(expr)                       \
+    do {                                    \
+        hsa_status_t s_ = (expr);           \
+        if (s_ != HSA_OK) return s_;        \
+    } while (0)
+
+static hsa_status_t check_ws(const WsLayout &w, void *ws, size_t ws_bytes) {
+    if (ws_bytes < w.total) return fail(HSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, w.total);
+    if (!ws) return fail(HSA_ERR_WORKSPACE, "workspace is NULL");
+    if ((uintptr_t)ws & 255u) return fail(HSA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    return HSA_OK;
+}
+
+static hsa_status_t clear_status(char *ws, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), st);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "clearing the device-status word");
+}
+
+}  // namespace hsa
+
+using namespace hsa;
+
+extern "C" {
+
+int hsa_abi_version(void) { return HSA_ABI_VERSION; }
+
+const char *hsa_last_error(void) { return g_err; }
+
+const char *hsa_status_string(hsa_status_t s) {
+    switch (s) {
+        case HSA_OK: return "HSA_OK";
+        case HSA_ERR_INVALID_ARG: return "HSA_ERR_INVALID_ARG: invalid argument";
+        case HSA_ERR_UNSUPPORTED: return "HSA_ERR_UNSUPPORTED: shape not implemented";
+        case HSA_ERR_WORKSPACE: return "HSA_ERR_WORKSPACE: workspace missing or too small";
+        case HSA_ERR_CUDA: return "HSA_ERR_CUDA: CUDA call failed";
+        case HSA_ERR_TIMEOUT: return "HSA_ERR_TIMEOUT: a device-side wait expired";
+    }
+    return "unknown hsa_status_t";
+}
+
+hsa_status_t hsa_workspace_size(const hsa_problem_t *prob, size_t *bytes) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (!bytes) return fail(HSA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = ws_layout(p).total;
+    return HSA_OK;
+}
+
+hsa_status_t hsa_plan(const hsa_problem_t *prob, hsa_plan_t *plan) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (!plan) return fail(HSA_ERR_INVALID_ARG, "plan is NULL");
+    *plan = ws_layout(p).plan;
+    return HSA_OK;
+}
+
+hsa_status_t hsa_landmarks(const hsa_problem_t *prob, const void *K, const void *W_L, void *L, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    const bool any = (long long)p.B * p.C > 0;
+    HSA_TRY(need(K, any, "K"));
+    HSA_TRY(need(W_L, any, "W_L"));
+    HSA_TRY(need(L, any, "L"));
+    cudaError_t e = launch_landmarks(p, K, W_L, L, (cudaStream_t)stream);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "landmark kernel launch");
+}
+
+hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L, int32_t *idx, float *score,
+                        int32_t *keff, void *ws, size_t ws_bytes, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    const bool rows = p.rows > 0;
+    HSA_TRY(need(Q, rows, "Q"));
+    HSA_TRY(need(L, rows && p.C > 0, "L"));
+    HSA_TRY(need(idx, rows, "idx"));
+    HSA_TRY(need(score, rows, "score"));
+    HSA_TRY(need(keff, rows, "keff"));
+    const WsLayout w = ws_layout(p);
+    HSA_TRY(check_ws(w, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    HSA_TRY(clear_status((char *)ws, st));
+    cudaError_t e = launch_select(p, w, Q, L, idx, score, keff, (char *)ws, st);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "selection kernel launch");
+}
+
+hsa_status_t hsa_attend(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const int32_t *idx,
+                        const float *score, const int32_t *keff, void *O, void *ws, size_t ws_bytes, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    const bool rows = p.rows > 0;
+    HSA_TRY(need(Q, rows, "Q"));
+    HSA_TRY(need(K, rows && p.C > 0, "K"));
+    HSA_TRY(need(V, rows && p.C > 0, "V"));
+    HSA_TRY(need(idx, rows, "idx"));
+    HSA_TRY(need(score, rows, "score"));
+    HSA_TRY(need(keff, rows, "keff"));
+    HSA_TRY(need(O, rows, "O"));
+    const WsLayout w = ws_layout(p);
+    HSA_TRY(check_ws(w, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    HSA_TRY(clear_status((char *)ws, st));
+    cudaError_t e = launch_attend(p, w, Q, K, V, idx, score, keff, O, (char *)ws, st);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "attention kernel launch");
+}
+
+hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const void *W_L,
+                         void *L, int32_t *idx, float *score, int32_t *keff, void *O, void *ws, size_t ws_bytes,
+                         void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    const bool rows = p.rows > 0;
+    const bool ready = (p.flags & HSA_FLAG_LANDMARKS_READY) != 0;
+    const bool chunks = (long long)p.B * p.C > 0;
+    HSA_TRY(need(Q, rows, "Q"));
+    HSA_TRY(need(K, (rows && p.C > 0) || (chunks && !ready), "K"));
+    HSA_TRY(need(V, rows && p.C > 0, "V"));
+    HSA_TRY(need(W_L, chunks && !ready, "W_L"));
+    HSA_TRY(need(L, chunks, "L"));
+    if (idx && !aligned16(idx)) return fail(HSA_ERR_INVALID_ARG, "idx is not 16-byte aligned");
+    if (score && !aligned16(score)) return fail(HSA_ERR_INVALID_ARG, "score is not 16-byte aligned");
+    if (keff && !aligned16(keff)) return fail(HSA_ERR_INVALID_ARG, "keff is not 16-byte aligned");
+    HSA_TRY(need(O, rows, "O"));
+    const WsLayout w = ws_layout(p);
+    HSA_TRY(check_ws(w, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    char *wsb = (char *)ws;
+    HSA_TRY(clear_status(wsb, st));
+    cudaError_t e;
+    if (!ready) {
+        e = launch_landmarks(p, K, W_L, L, st);
+        if (e != cudaSuccess) return cuda_fail(e, "landmark kernel launch");
+    }
+    int32_t *sidx = idx ? idx : reinterpret_cast<int32_t *>(wsb + w.sel_idx);
+    float *ssc = score ? score : reinterpret_cast<float *>(wsb + w.sel_score);
+    int32_t *skf = keff ? keff : reinterpret_cast<int32_t *>(wsb + w.sel_keff);
+    e = launch_select(p, w, Q, L, sidx, ssc, skf, wsb, st);
+    if (e != cudaSuccess) return cuda_fail(e, "selection kernel launch");
+    e = launch_attend(p, w, Q, K, V, sidx, ssc, skf, O, wsb, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+    return HSA_OK;
+}
+
+hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < 256) return fail(HSA_ERR_WORKSPACE, "workspace missing or smaller than its header");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device-status word");
+    if (word == DEV_OK) return HSA_OK;
+    e = cudaMemsetAsync(ws, 0, sizeof word, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device-status word");
+    return fail(HSA_ERR_TIMEOUT, "device-status word 0x%x: a bounded device wait expired", word);
+}
+
+}  // extern "C"

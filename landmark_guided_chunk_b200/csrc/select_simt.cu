@@ -1,0 +1,204 @@
+// select_simt.cu -- chunk selection on CUDA cores (HSA summary page, Core
+// Technique / Implementation: score every landmark of the strictly-past
+// chunks, keep the top k; gap router from the value-of-information router
+// page).  Works for every supported shape and dtype.  fp32 problems always
+// use it, and bf16 problems whose shape the tensor-core kernel does not cover.
+//
+// Score of chunk c for a (b, t, kv head j) row: s_c = sum_{h in group j} q_h . L_c,
+// computed as qbar . L_c with qbar = sum_h q_h formed in fp32 (the same sum,
+// up to fp32 rounding).  Each lane scores its own chunk of a 32-chunk batch.
+// Lanes whose score beats the current k-th entry are inserted, in chunk
+// order, into a warp-distributed sorted list.
+//
+//  * select_rows_kernel   : one warp per row, scans all candidates (prefill).
+//  * select_split_kernel  : (split, row) CTAs, each scanning a chunk range with
+//                           8 warps and emitting one merged list (decode: few
+//                           rows, very long scans).
+//  * select_merge_kernel  : one warp per row merges the split lists.
+#include "common.cuh"
+
+namespace hsa {
+namespace {
+
+struct SelArgs {
+    int Tq, H, Hkv, d, S, C, k, kmax, G;
+    long long q_pos0, rows;
+    float tau;
+};
+
+__device__ __forceinline__ void row_coords(const SelArgs &a, long long row, int &b, int &t, int &j) {
+    j = (int)(row % a.Hkv);
+    long long bt = row / a.Hkv;
+    t = (int)(bt % a.Tq);
+    b = (int)(bt / a.Tq);
+}
+
+__device__ __forceinline__ int row_ncand(const SelArgs &a, int t) {
+    long long n = (a.q_pos0 + t) / a.S;
+    return (int)(n < a.C ? n : a.C);
+}
+
+// qbar[e] = sum over the group's heads of Q[b][t][h][e], into shared memory.
+template <typename T>
+__device__ __forceinline__ void load_qbar(const T *Q, const SelArgs &a, int b, int t, int j, float *qs, int lane) {
+    const T *q = Q + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G) * a.d;
+    for (int e = lane; e < a.d; e += 32) {
+        float s = 0.f;
+        for (int g = 0; g < a.G; ++g) s += to_f32(q[(size_t)g * a.d + e]);
+        qs[e] = s;
+    }
+    __syncwarp();
+}
+
+template <typename T>
+__device__ __forceinline__ void scan_range(const float *qs, const T *Lj, const SelArgs &a, int c0, int c1, int step,
+                                           float &v, int &id, int lane) {
+    for (int base = c0; base < c1; base += step) {
+        int c = base + lane;
+        bool valid = c < c1;
+        float s = valid ? dot_row(qs, Lj + (size_t)c * a.d, a.d) : -INFINITY;
+        list_offer(v, id, s, c, valid, a.kmax, lane);
+    }
+}
+
+__device__ __forceinline__ void write_row(const SelArgs &a, long long row, float v, int id, int ke, int32_t *idx,
+                                          float *score, int32_t *keff, int lane) {
+    if (lane < a.kmax) {
+        idx[row * a.kmax + lane] = lane < ke ? id : -1;
+        score[row * a.kmax + lane] = lane < ke ? v : -INFINITY;
+    }
+    if (lane == 0) keff[row] = ke;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) select_rows_kernel(const T *__restrict__ Q, const T *__restrict__ L,
+                                                          int32_t *__restrict__ idx, float *__restrict__ score,
+                                                          int32_t *__restrict__ keff, SelArgs a) {
+    extern __shared__ float qsm[];   // [8 warps][d]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + warp;
+    if (row >= a.rows) return;
+    int b, t, j;
+    row_coords(a, row, b, t, j);
+    float *qs = qsm + warp * a.d;
+    load_qbar(Q, a, b, t, j, qs, lane);
+    const int ncand = row_ncand(a, t);
+    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * a.d;
+    float v;
+    int id;
+    list_init(v, id);
+    scan_range(qs, Lj, a, 0, ncand, 32, v, id, lane);
+    write_row(a, row, v, id, list_keff(v, ncand, a.k, a.kmax, a.tau), idx, score, keff, lane);
+}
+
+// One CTA = one (split, row).  Warps interleave over 32-chunk batches of the
+// split's range; their lists are merged by warp 0 into the split's list.
+template <typename T>
+__global__ void __launch_bounds__(256) select_split_kernel(const T *__restrict__ Q, const T *__restrict__ L,
+                                                           float2 *__restrict__ lists, SelArgs a, int chunks_per_split,
+                                                           int nsplit) {
+    extern __shared__ float qsm[];   // [d] qbar, then 8 x kmax (v, id) pairs
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = blockIdx.y;
+    const int split = blockIdx.x;
+    int b, t, j;
+    row_coords(a, row, b, t, j);
+    float *qs = qsm;
+    float2 *wl = reinterpret_cast<float2 *>(qsm + a.d);
+    if (warp == 0) load_qbar(Q, a, b, t, j, qs, lane);
+    __syncthreads();
+    const int ncand = row_ncand(a, t);
+    const int c0 = split * chunks_per_split;
+    const int c1 = min(ncand, c0 + chunks_per_split);
+    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * a.d;
+    float v;
+    int id;
+    list_init(v, id);
+    if (c0 < c1) scan_range(qs, Lj, a, c0 + 32 * warp, c1, 256, v, id, lane);
+    if (lane < a.kmax) wl[warp * a.kmax + lane] = make_float2(v, __int_as_float(id));
+    __syncthreads();
+    if (warp == 0) {
+        float mv;
+        int mid;
+        list_init(mv, mid);
+        const int n = 8 * a.kmax;
+        for (int base = 0; base < n; base += 32) {
+            int e = base + lane;
+            float2 x = e < n ? wl[e] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+            int xi = __float_as_int(x.y);
+            list_offer(mv, mid, x.x, xi, xi != INT32_MAX, a.kmax, lane);
+        }
+        if (lane < a.kmax) lists[(row * nsplit + split) * a.kmax + lane] = make_float2(mv, __int_as_float(mid));
+    }
+}
+
+__global__ void __launch_bounds__(256) select_merge_kernel(const float2 *__restrict__ lists, int32_t *__restrict__ idx,
+                                                           float *__restrict__ score, int32_t *__restrict__ keff,
+                                                           SelArgs a, int nsplit) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 8 + warp;
+    if (row >= a.rows) return;
+    int b, t, j;
+    row_coords(a, row, b, t, j);
+    const float2 *src = lists + row * nsplit * a.kmax;
+    const int n = nsplit * a.kmax;
+    float v;
+    int id;
+    list_init(v, id);
+    for (int base = 0; base < n; base += 32) {
+        int e = base + lane;
+        float2 x = e < n ? src[e] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+        int xi = __float_as_int(x.y);
+        list_offer(v, id, x.x, xi, xi != INT32_MAX, a.kmax, lane);
+    }
+    write_row(a, row, v, id, list_keff(v, row_ncand(a, t), a.k, a.kmax, a.tau), idx, score, keff, lane);
+}
+
+SelArgs make_args(const Prob &p) {
+    SelArgs a;
+    a.Tq = p.Tq;
+    a.H = p.H;
+    a.Hkv = p.Hkv;
+    a.d = p.d;
+    a.S = p.S;
+    a.C = p.C;
+    a.k = p.k;
+    a.kmax = p.kmax;
+    a.G = p.G;
+    a.q_pos0 = p.q_pos0;
+    a.rows = p.rows;
+    a.tau = p.tau;
+    return a;
+}
+
+template <typename T>
+cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx, float *score,
+                         int32_t *keff, char *ws, cudaStream_t st) {
+    SelArgs a = make_args(p);
+    if (!w.split_select) {
+        unsigned blocks = (unsigned)((p.rows + 7) / 8);
+        select_rows_kernel<T><<<blocks, 256, 8 * p.d * sizeof(float), st>>>((const T *)Q, (const T *)L, idx, score,
+                                                                            keff, a);
+        return cudaGetLastError();
+    }
+    float2 *lists = reinterpret_cast<float2 *>(ws + w.split_lists);
+    dim3 grid(w.nsplit, (unsigned)p.rows);
+    size_t smem = p.d * sizeof(float) + 8 * p.kmax * sizeof(float2);
+    select_split_kernel<T><<<grid, 256, smem, st>>>((const T *)Q, (const T *)L, lists, a, w.chunks_per_split,
+                                                    w.nsplit);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    select_merge_kernel<<<(unsigned)((p.rows + 7) / 8), 256, 0, st>>>(lists, idx, score, keff, a, w.nsplit);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
+                          float *score, int32_t *keff, char *ws, cudaStream_t st) {
+    if (p.rows == 0) return cudaSuccess;
+    if (p.dtype == HSA_BF16) return launch_typed<__nv_bfloat16>(p, w, Q, L, idx, score, keff, ws, st);
+    return launch_typed<float>(p, w, Q, L, idx, score, keff, ws, st);
+}
+
+}  // namespace hsa

@@ -1,0 +1,107 @@
+"""The C ABI on the host: the library loads, exports every entry point that
+include/hsa.h declares, and rejects bad calls before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import landmark_guided_chunk_b200 as hsa
+from landmark_guided_chunk_b200 import _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "hsa.h")).read()
+    return re.findall(r"HSA_API\s+[\w\s\*]+?\b(hsa_\w+)\s*\(", txt)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 9
+    lib = _native.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_native.EXPORTED)
+    assert lib.hsa_abi_version() == 1
+
+
+def test_status_strings():
+    lib = _native.lib()
+    for s in range(6):
+        assert lib.hsa_status_string(s).startswith(b"HSA_")
+
+
+def _prob(**kw):
+    base = dict(B=1, Tq=128, Tkv=128, H=4, Hkv=2, d=64, S=64, k=4, q_pos0=0, tau=0.0, dtype=torch_bf16(), flags=0)
+    base.update(kw)
+    return hsa.make_problem(**base)
+
+
+def torch_bf16():
+    import torch
+    return torch.bfloat16
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=5), _native.HSA_ERR_INVALID_ARG),
+    (dict(B=-1), _native.HSA_ERR_INVALID_ARG),
+    (dict(k=0), _native.HSA_ERR_INVALID_ARG),
+    (dict(tau=-0.1), _native.HSA_ERR_INVALID_ARG),
+    (dict(tau=float("nan")), _native.HSA_ERR_INVALID_ARG),
+    (dict(tau=float("inf")), _native.HSA_ERR_INVALID_ARG),
+    (dict(q_pos0=-3), _native.HSA_ERR_INVALID_ARG),
+    (dict(flags=8), _native.HSA_ERR_INVALID_ARG),
+    (dict(d=96), _native.HSA_ERR_UNSUPPORTED),
+    (dict(S=48), _native.HSA_ERR_UNSUPPORTED),
+    (dict(k=33), _native.HSA_ERR_UNSUPPORTED),
+    (dict(k=17, tau=0.1), _native.HSA_ERR_UNSUPPORTED),
+    (dict(H=34, Hkv=2), _native.HSA_ERR_UNSUPPORTED),
+])
+def test_workspace_size_rejects_bad_problems(kw, status):
+    with pytest.raises(hsa.HSAError) as e:
+        hsa.workspace_size(_prob(**kw))
+    assert e.value.status == status
+
+
+def test_workspace_size_grows_with_rows_and_is_aligned():
+    a = hsa.workspace_size(_prob(Tq=4096, Tkv=4096))
+    b = hsa.workspace_size(_prob(Tq=8192, Tkv=8192))
+    assert a >= 256 and b > a and a % 256 == 0 and b % 256 == 0
+
+
+def _call_forward(prob, Q=16, K=16, V=16, W=16, L=16, O=16, ws=256, ws_bytes=1 << 30):
+    lib = _native.lib()
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.hsa_forward(ctypes.byref(prob), P(Q), P(K), P(V), P(W), P(L), None, None, None, P(O), P(ws),
+                           ws_bytes, None)
+
+
+def test_forward_validates_pointers_before_launch():
+    """Fake, never-dereferenced addresses: every call below must fail in host validation."""
+    p = _prob()
+    assert _call_forward(p, Q=None) == _native.HSA_ERR_INVALID_ARG
+    assert _call_forward(p, K=24) == _native.HSA_ERR_INVALID_ARG            # misaligned
+    assert _call_forward(p, O=None) == _native.HSA_ERR_INVALID_ARG
+    assert _call_forward(p, W=None) == _native.HSA_ERR_INVALID_ARG
+    assert _call_forward(p, ws=None) == _native.HSA_ERR_WORKSPACE
+    assert _call_forward(p, ws=272) == _native.HSA_ERR_WORKSPACE            # not 256-aligned
+    assert _call_forward(p, ws_bytes=64) == _native.HSA_ERR_WORKSPACE
+    assert b"workspace" in _native.lib().hsa_last_error()
+    ready = _prob(flags=_native.HSA_FLAG_LANDMARKS_READY)
+    assert _call_forward(ready, W=None, L=None) == _native.HSA_ERR_INVALID_ARG   # L is required
+
+
+def test_null_problem_and_status_reader():
+    lib = _native.lib()
+    n = ctypes.c_size_t()
+    assert lib.hsa_workspace_size(None, ctypes.byref(n)) == _native.HSA_ERR_INVALID_ARG
+    assert lib.hsa_get_device_status(None, 0, None) == _native.HSA_ERR_WORKSPACE
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        _native.lib()

@@ -1,0 +1,188 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Small problems are checked on every row.  They span several tiles, with ragged
+tails, both dtypes, d 64/128, S 32/64/128, G 1..8 and the router.  The full
+workloads are checked on sampled rows (prefill) or on every row (decode: the
+oracle rebuilds all landmarks from the cache).
+"""
+import numpy as np
+import pytest
+import torch
+
+import landmark_guided_chunk_b200 as hsa
+import oracle
+from landmark_guided_chunk_b200.inputs import Problem, make_inputs, workload
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _rows_all(p: Problem):
+    return np.repeat(np.arange(p.B), p.Tq), np.tile(np.arange(p.Tq), p.B)
+
+
+def _rows_sampled(p: Problem, n: int, seed: int = 0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, p.S - 1, p.S, 2 * p.S - 1, 2 * p.S, p.Tq // 2, p.Tq - p.S, p.Tq - 1]
+    t = np.array(sorted(set([x for x in fixed if 0 <= x < p.Tq] + list(rng.integers(0, p.Tq, n)))))
+    b = rng.integers(0, p.B, t.size)
+    return b, t
+
+
+def _oracle_L(p: Problem, inp):
+    K, W = inp["K"], inp["W_L"]
+    if K.numel() * K.element_size() > (2 << 30):
+        return oracle.landmarks_stored_sliced(K, W, p.S, p.dtype)
+    return oracle.landmarks_stored(K.cpu(), W.cpu(), p.S, p.dtype)
+
+
+def run_case(p: Problem, rows=None, seed=0, landmarks_first=False):
+    torch.manual_seed(seed)
+    inp = make_inputs(p, seed=seed, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    if landmarks_first:
+        L = hsa.landmarks(K, W, p.S)
+        O, L, idx, score, keff = hsa.forward(Q, K, V, None, p.S, p.k, p.tau, p.q_pos0, L=L,
+                                             landmarks_ready=True, return_selection=True)
+    else:
+        O, L, idx, score, keff = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, p.q_pos0, return_selection=True)
+    torch.cuda.synchronize()
+    L_orc = _oracle_L(p, inp)
+    lm = parity.check_landmarks(L, L_orc)
+    rb, rt = rows if rows is not None else _rows_all(p)
+    tb, tt = torch.as_tensor(rb, device="cuda"), torch.as_tensor(rt, device="cuda")
+    Qr = Q[tb, tt].cpu()
+    orc = oracle.select(Qr, rb, rt + p.q_pos0, L_orc, p.S, p.k, p.tau, p.H, want_all=True)
+    ncand = np.minimum((rt + p.q_pos0) // p.S, p.C)
+    g_idx, g_sc, g_ke = idx[tb, tt].cpu().numpy(), score[tb, tt].cpu().numpy(), keff[tb, tt].cpu().numpy()
+    sel = parity.check_selection(g_idx, g_sc, g_ke, orc, ncand, p.k, p.tau)
+    O_exp = parity.expected_output(Qr, rb, K, V, p.S, orc, g_idx, g_ke, sel["tie_rows"])
+    err = parity.check_output(O[tb, tt], O_exp, Q.dtype)
+    return {"inp": inp, "O": O, "L": L, "idx": idx, "keff": keff, "sel": sel, "lm": lm, "err": err,
+            "orc": orc, "rows": (rb, rt)}
+
+
+SMALL = [
+    workload("tiny_f32"),
+    Problem(B=2, Tq=64 * 40 + 37, Tkv=64 * 40 + 37, H=8, Hkv=2, d=128, S=64, k=16, dtype="bf16", name="bf16_g4"),
+    Problem(B=1, Tq=128 * 24 + 5, Tkv=128 * 24 + 5, H=8, Hkv=2, d=128, S=128, k=8, tau=0.02, dtype="bf16",
+            name="bf16_router"),
+    Problem(B=1, Tq=128 * 24 + 5, Tkv=128 * 24 + 5, H=8, Hkv=2, d=128, S=128, k=8, tau=0.3, dtype="bf16",
+            name="bf16_router_wide"),
+    Problem(B=2, Tq=32 * 50 + 9, Tkv=32 * 50 + 9, H=4, Hkv=4, d=64, S=32, k=5, dtype="bf16", name="bf16_d64_s32"),
+    Problem(B=1, Tq=64 * 30, Tkv=64 * 30, H=16, Hkv=2, d=64, S=64, k=32, dtype="f32", name="f32_g8_k32"),
+    Problem(B=1, Tq=64 * 20 + 63, Tkv=64 * 20 + 63, H=6, Hkv=3, d=128, S=64, k=3, tau=0.05, dtype="f32",
+            name="f32_router"),
+]
+
+
+@pytest.mark.parametrize("p", SMALL, ids=lambda p: p.name)
+def test_small_prefill_all_rows(p):
+    r = run_case(p)
+    assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
+
+
+DECODE_SMALL = [
+    Problem(B=3, Tq=1, Tkv=64 * 3000 + 17, H=8, Hkv=2, d=128, S=64, k=16, q_pos0=64 * 3000 + 17, dtype="bf16",
+            planted=3, name="decode_split"),
+    Problem(B=2, Tq=1, Tkv=64 * 700 + 5, H=4, Hkv=1, d=64, S=64, k=4, q_pos0=64 * 700 + 5, dtype="bf16",
+            planted=2, name="decode_rows"),
+    Problem(B=2, Tq=1, Tkv=128 * 2500, H=8, Hkv=2, d=128, S=128, k=8, tau=0.02, q_pos0=128 * 2500, dtype="bf16",
+            planted=2, name="decode_router"),
+]
+
+
+@pytest.mark.parametrize("p", DECODE_SMALL, ids=lambda p: p.name)
+def test_small_decode(p):
+    r = run_case(p, landmarks_first=True)
+    idx, keff = r["idx"].cpu().numpy(), r["keff"].cpu().numpy()
+    for b in range(p.B):
+        for c in r["inp"]["planted"][b].tolist():
+            for j in range(p.Hkv):
+                assert c in idx[b, 0, j, :keff[b, 0, j]], f"planted chunk {c} missed (b={b}, kv={j})"
+
+
+def test_attend_stage_with_oracle_selection():
+    """hsa_attend alone, fed the oracle's selection: isolates the attention and fusion kernels."""
+    p = Problem(B=2, Tq=64 * 24 + 11, Tkv=64 * 24 + 11, H=8, Hkv=2, d=128, S=64, k=16, dtype="bf16")
+    inp = make_inputs(p, seed=3, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    L = oracle.landmarks_stored(K.cpu(), W.cpu(), p.S, p.dtype)
+    rb, rt = _rows_all(p)
+    Qr = Q.reshape(-1, p.H, p.d).cpu()
+    sel = oracle.select(Qr, rb, rt, L, p.S, p.k, 0.0, p.H)
+    sh = (p.B, p.Tq, p.Hkv)
+    idx = torch.as_tensor(sel["idx"]).reshape(*sh, p.kmax).cuda()
+    sc = torch.as_tensor(sel["score"]).float().reshape(*sh, p.kmax).cuda()
+    ke = torch.as_tensor(sel["keff"]).reshape(*sh).cuda()
+    O = hsa.attend(Q, K, V, idx, sc, ke, p.S, p.k)
+    O_exp = oracle.attend(Qr, rb, K.cpu(), V.cpu(), p.S, sel)
+    parity.check_output(O.reshape(-1, p.H, p.d), O_exp, Q.dtype)
+
+
+def test_select_stage_alone_matches_forward():
+    p = Problem(B=1, Tq=64 * 33, Tkv=64 * 33, H=8, Hkv=2, d=128, S=64, k=16, dtype="bf16")
+    inp = make_inputs(p, seed=4, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    idx, sc, ke = hsa.select(Q, L, p.S, p.k)
+    O, L2, idx2, sc2, ke2 = hsa.forward(Q, K, V, W, p.S, p.k, return_selection=True)
+    assert torch.equal(L, L2) and torch.equal(idx, idx2) and torch.equal(ke, ke2) and torch.equal(sc, sc2)
+
+
+def test_edges_no_chunks_and_short_sequences():
+    for T in (0, 1, 63, 64, 65, 130):
+        p = Problem(B=2, Tq=T, Tkv=T, H=4, Hkv=2, d=64, S=64, k=4, dtype="bf16")
+        inp = make_inputs(p, seed=5, device="cuda")
+        O, L, idx, sc, ke = hsa.forward(inp["Q"], inp["K"], inp["V"], inp["W_L"], 64, 4, return_selection=True)
+        torch.cuda.synchronize()
+        if T == 0:
+            continue
+        t = torch.arange(T, device="cuda")
+        want_ke = torch.clamp(t // 64, max=T // 64).to(torch.int32).view(1, T, 1).expand(2, T, 2)
+        assert torch.equal(ke, torch.minimum(want_ke, torch.tensor(4, device="cuda", dtype=torch.int32)))
+        assert torch.all(O[:, :64] == 0)
+
+
+def test_batch_zero_is_a_no_op():
+    p = hsa.make_problem(0, 5, 5, 4, 2, 64, 64, 4)
+    assert hsa.workspace_size(p) >= 256
+    Q = torch.empty(0, 5, 4, 64, dtype=torch.bfloat16, device="cuda")
+    K = torch.empty(0, 5, 2, 64, dtype=torch.bfloat16, device="cuda")
+    O = hsa.forward(Q, K, K, torch.eye(64, dtype=torch.bfloat16, device="cuda"), 64, 4)
+    assert O.shape == Q.shape
+
+
+def test_device_status_is_clear_after_calls():
+    p = Problem(B=1, Tq=256, Tkv=256, H=4, Hkv=2, d=64, S=64, k=2, dtype="bf16")
+    inp = make_inputs(p, seed=6, device="cuda")
+    prob = hsa.make_problem(1, 256, 256, 4, 2, 64, 64, 2)
+    ws = hsa.alloc_workspace(prob)
+    ws.fill_(0xFF)                      # garbage: every call clears the status word first
+    hsa.forward(inp["Q"], inp["K"], inp["V"], inp["W_L"], 64, 2, ws=ws)
+    hsa.device_status(ws)
+
+
+# ------------------------------------------------------------------- full workloads (sampled rows)
+
+@pytest.mark.parametrize("name", ["prefill_bf16", "router_bf16"])
+def test_full_prefill_workload_sampled_rows(name):
+    p = workload(name)
+    r = run_case(p, rows=_rows_sampled(p, 192))
+    if p.tau > 0:
+        ke = r["keff"].cpu().numpy()
+        frac = float(np.mean(ke[:, p.S * (p.k + 1):] > p.k))
+        assert 0.05 < frac < 0.95, f"router doubled {frac:.3f} of rows"
+
+
+@pytest.mark.parametrize("name", ["decode_1m", "decode_16m"])
+def test_full_decode_workload(name):
+    p = workload(name)
+    r = run_case(p, landmarks_first=True)
+    idx, keff = r["idx"].cpu().numpy(), r["keff"].cpu().numpy()
+    for b in range(p.B):
+        for c in r["inp"]["planted"][b].tolist():
+            for j in range(p.Hkv):
+                assert c in idx[b, 0, j, :keff[b, 0, j]], f"planted chunk {c} missed (b={b}, kv={j})"
+    del r
+    torch.cuda.empty_cache()
