@@ -130,7 +130,9 @@ HSA_API hsa_status_t hsa_select(const hsa_problem_t *p, const void *Q, const voi
  *   o_i  = softmax_u(q_h . K[c_i S + u] / sqrt(d)) . V[c_i S + u]     (u < S)
  *   O[h] = sum_i w_i o_i                                              (0 when keff = 0)
  * idx/score/keff are as hsa_select writes them.  Every idx[i] for i < keff
- * must be a valid candidate chunk of its row.
+ * must be a candidate chunk of its row and keff must lie in [0, kmax].  An
+ * out-of-range value is never dereferenced: its slot is skipped, and
+ * hsa_get_device_status() then reports HSA_ERR_INVALID_ARG.
  */
 HSA_API hsa_status_t hsa_attend(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                         const int32_t *idx, const float *score, const int32_t *keff, void *O,
@@ -148,8 +150,11 @@ HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const vo
 
 /*
  * Synchronises `stream`, then reads and clears the device-status word in the
- * workspace header.  Returns HSA_OK, HSA_ERR_TIMEOUT (a bounded device wait
- * expired in an earlier call on this workspace) or HSA_ERR_CUDA.
+ * workspace header.  Every call that takes a workspace clears that word when it
+ * starts (stream-ordered), so the word describes the latest such call.
+ * Returns HSA_OK, HSA_ERR_TIMEOUT (a bounded device wait expired),
+ * HSA_ERR_INVALID_ARG (hsa_attend skipped an out-of-range chunk index or keff)
+ * or HSA_ERR_CUDA.
  */
 HSA_API hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream);
 

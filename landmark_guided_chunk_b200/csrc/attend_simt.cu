@@ -21,10 +21,30 @@ namespace hsa {
 namespace {
 
 struct AttArgs {
-    int Tq, Tkv, H, Hkv, d, S, kmax, G;
-    long long rows;
-    float scale;   // 1/sqrt(d)
+    int Tq, Tkv, H, Hkv, d, S, C, kmax, G;
+    long long q_pos0, rows;
+    float scale;        // 1/sqrt(d)
+    uint32_t *status;   // workspace status word
 };
+
+// keff and chunk indices come from the caller: out-of-range values are skipped
+// (never dereferenced) and reported through the status word.
+__device__ __forceinline__ int checked_keff(const AttArgs &a, int ke) {
+    if (ke < 0 || ke > a.kmax) {
+        atomicOr(a.status, DEV_BAD_INDEX);
+        return ke < 0 ? 0 : a.kmax;
+    }
+    return ke;
+}
+__device__ __forceinline__ bool valid_chunk(const AttArgs &a, int t, int c) {
+    long long nc = (a.q_pos0 + t) / a.S;
+    if (nc > a.C) nc = a.C;
+    if (c < 0 || c >= nc) {
+        if (threadIdx.x == 0) atomicOr(a.status, DEV_BAD_INDEX);
+        return false;
+    }
+    return true;
+}
 
 constexpr int NT = 128;   // threads per CTA (>= S and >= d)
 
@@ -147,7 +167,7 @@ __global__ void __launch_bounds__(NT) attend_rows_kernel(const T *__restrict__ Q
     const long long row = blockIdx.x;
     int b, t, j;
     row_coords(a, row, b, t, j);
-    const int ke = keff[row];
+    const int ke = checked_keff(a, keff[row]);
     T *out = O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G) * a.d;
     float acc[MAX_G];
 #pragma unroll
@@ -157,6 +177,7 @@ __global__ void __launch_bounds__(NT) attend_rows_kernel(const T *__restrict__ Q
         fusion_weights(score + row * a.kmax, ke, s);
         for (int i = 0; i < ke; ++i) {
             const int c = idx[row * a.kmax + i];
+            if (!valid_chunk(a, t, c)) continue;   // uniform over the block
             __syncthreads();
             stage_chunk(K, V, a, b, j, c, s);
             __syncthreads();
@@ -182,13 +203,18 @@ __global__ void __launch_bounds__(NT) attend_split_kernel(const T *__restrict__ 
     const Smem s = carve(smem, a);
     const int i = blockIdx.x;
     const long long row = blockIdx.y;
-    if (i >= keff[row]) return;
+    if (i >= checked_keff(a, keff[row])) return;
     int b, t, j;
     row_coords(a, row, b, t, j);
-    load_q(Q, a, b, t, j, s);
-    stage_chunk(K, V, a, b, j, idx[row * a.kmax + i], s);
-    __syncthreads();
+    const int c = idx[row * a.kmax + i];
     float *dst = part + (row * a.kmax + i) * (size_t)a.G * a.d;
+    if (!valid_chunk(a, t, c)) {
+        for (int x = threadIdx.x; x < a.G * a.d; x += NT) dst[x] = 0.f;
+        return;
+    }
+    load_q(Q, a, b, t, j, s);
+    stage_chunk(K, V, a, b, j, c, s);
+    __syncthreads();
     for (int g = 0; g < a.G; ++g) {
         const float o = chunk_attention(a, s, g);
         if (threadIdx.x < a.d) dst[(size_t)g * a.d + threadIdx.x] = o;
@@ -205,7 +231,7 @@ __global__ void __launch_bounds__(NT) attend_combine_kernel(const float *__restr
     const long long row = blockIdx.x;
     int b, t, j;
     row_coords(a, row, b, t, j);
-    const int ke = keff[row];
+    const int ke = checked_keff(a, keff[row]);
     fusion_weights(score + row * a.kmax, ke, s);
     __syncthreads();
     T *out = O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G) * a.d;
@@ -228,10 +254,13 @@ cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const 
     a.Hkv = p.Hkv;
     a.d = p.d;
     a.S = p.S;
+    a.C = p.C;
     a.kmax = p.kmax;
     a.G = p.G;
+    a.q_pos0 = p.q_pos0;
     a.rows = p.rows;
     a.scale = 1.0f / sqrtf((float)p.d);
+    a.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
     const size_t smem = smem_bytes(p.G, p.d, p.S, p.kmax);
     if (!w.split_attend) {
         cudaFuncSetAttribute(attend_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -40,7 +40,8 @@ WsLayout ws_layout(const Prob &p);
 
 // status word values (workspace header)
 constexpr uint32_t DEV_OK = 0;
-constexpr uint32_t DEV_TIMEOUT = 1;
+constexpr uint32_t DEV_TIMEOUT = 1;      // a bounded wait expired
+constexpr uint32_t DEV_BAD_INDEX = 2;    // hsa_attend got a chunk index / keff outside its row's range
 
 // ---------------------------------------------------------------------------- element access
 

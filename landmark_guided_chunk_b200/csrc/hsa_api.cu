@@ -264,7 +264,9 @@ hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream) {
     e = cudaMemsetAsync(ws, 0, sizeof word, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device-status word");
-    return fail(HSA_ERR_TIMEOUT, "device-status word 0x%x: a bounded device wait expired", word);
+    if (word & DEV_TIMEOUT) return fail(HSA_ERR_TIMEOUT, "device-status word 0x%x: a bounded device wait expired", word);
+    return fail(HSA_ERR_INVALID_ARG, "device-status word 0x%x: hsa_attend got a keff or chunk index outside "
+                "its row's candidates (those slots were skipped)", word);
 }
 
 }  // extern "C"

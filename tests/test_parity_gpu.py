@@ -186,3 +186,30 @@ def test_full_decode_workload(name):
                 assert c in idx[b, 0, j, :keff[b, 0, j]], f"planted chunk {c} missed (b={b}, kv={j})"
     del r
     torch.cuda.empty_cache()
+
+
+def test_attend_skips_and_reports_out_of_range_selection():
+    """A corrupt caller selection is never dereferenced: the slot is skipped and
+    the status word turns the call into HSA_ERR_INVALID_ARG."""
+    p = Problem(B=1, Tq=64 * 6, Tkv=64 * 6, H=4, Hkv=2, d=64, S=64, k=2, dtype="bf16")
+    inp = make_inputs(p, seed=7, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    idx, sc, ke = hsa.select(Q, L, p.S, p.k)
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k)
+    ws = hsa.alloc_workspace(prob)
+    hsa.attend(Q, K, V, idx, sc, ke, p.S, p.k, ws=ws)
+    hsa.device_status(ws)
+    bad = idx.clone()
+    bad[0, -1, 0, 0] = 1 << 20
+    hsa.attend(Q, K, V, bad, sc, ke, p.S, p.k, ws=ws)
+    with pytest.raises(hsa.HSAError) as e:
+        hsa.device_status(ws)
+    assert e.value.status == hsa._native.HSA_ERR_INVALID_ARG
+    ke2 = ke.clone()
+    ke2[0, -1, 1] = 99
+    hsa.attend(Q, K, V, idx, sc, ke2, p.S, p.k, ws=ws)
+    with pytest.raises(hsa.HSAError):
+        hsa.device_status(ws)
+    hsa.attend(Q, K, V, idx, sc, ke, p.S, p.k, ws=ws)
+    hsa.device_status(ws)
