@@ -79,6 +79,7 @@ typedef enum { HSA_F32 = 0, HSA_BF16 = 1 } hsa_dtype_t;
 
 /* hsa_problem_t.flags */
 #define HSA_FLAG_LANDMARKS_READY 1u  /* hsa_forward: L already holds the landmarks; skip that stage (W_L may be NULL) */
+#define HSA_FLAG_SIMT 2u             /* use the CUDA-core kernels even where a tensor-core kernel exists (testing) */
 
 typedef struct {
     int32_t B, Tq, Tkv, H, Hkv, d, S, k;

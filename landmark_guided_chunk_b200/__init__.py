@@ -94,12 +94,13 @@ def _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags=0):
     return make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, Q.dtype, flags)
 
 
-def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None):
+def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False):
     """Top-k chunk selection.  Returns (idx int32, score fp32 [B,Tq,Hkv,kmax], keff int32 [B,Tq,Hkv])."""
     _dev(Q, L, ws)
     B, Tq, H, d = Q.shape
     Hkv, C = L.shape[1], L.shape[2]
-    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0)
+    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0,
+                      _native.HSA_FLAG_SIMT if force_simt else 0)
     km = kmax_of(k, tau)
     idx = torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device)
     score = torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device)
@@ -111,10 +112,10 @@ def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None):
     return idx, score, keff
 
 
-def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None):
+def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None, force_simt=False):
     """Chunk attention + fusion for a given selection.  Returns O [B,Tq,H,d]."""
     _dev(Q, K, V, idx, score, keff, O, ws)
-    prob = _prob_from(Q, K.shape[1], K.shape[2], S, k, tau, q_pos0)
+    prob = _prob_from(Q, K.shape[1], K.shape[2], S, k, tau, q_pos0, _native.HSA_FLAG_SIMT if force_simt else 0)
     if O is None:
         O = torch.empty_like(Q)
     if ws is None:
@@ -125,12 +126,13 @@ def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None):
 
 
 def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False, O=None, ws=None,
-            return_selection=False):
-    """The whole HSA forward.  Returns O, or (O, L, idx, score, keff) with return_selection."""
+            return_selection=False, force_simt=False):
+    """The whole HSA forward.  Returns O, or (O, L, idx, score, keff) with return_selection.
+    force_simt runs the CUDA-core kernels even where tensor-core ones exist (for A/B tests)."""
     _dev(Q, K, V, W_L, L, O, ws)
     B, Tq, H, d = Q.shape
     Tkv, Hkv = K.shape[1], K.shape[2]
-    flags = _native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0
+    flags = (_native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0) | (_native.HSA_FLAG_SIMT if force_simt else 0)
     prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags)
     if L is None:
         if landmarks_ready:

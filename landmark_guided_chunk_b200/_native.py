@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libhsa_b200.so")
 HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT = range(6)
 HSA_F32, HSA_BF16 = 0, 1
 HSA_FLAG_LANDMARKS_READY = 1
+HSA_FLAG_SIMT = 2
 
 EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version")

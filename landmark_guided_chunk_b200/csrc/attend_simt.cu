@@ -226,8 +226,9 @@ __global__ void __launch_bounds__(NT) attend_combine_kernel(const float *__restr
                                                             const float *__restrict__ score,
                                                             const int32_t *__restrict__ keff, T *__restrict__ O,
                                                             AttArgs a) {
-    extern __shared__ float smem[];
-    const Smem s = carve(smem, a);
+    __shared__ float wbuf[MAX_KMAX];
+    Smem s{};
+    s.w = wbuf;
     const long long row = blockIdx.x;
     int b, t, j;
     row_coords(a, row, b, t, j);
@@ -274,7 +275,7 @@ cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const 
                                                                               (const T *)V, idx, keff, part, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attend_combine_kernel<T><<<(unsigned)p.rows, NT, smem, st>>>(part, score, keff, (T *)O, a);
+    attend_combine_kernel<T><<<(unsigned)p.rows, NT, 0, st>>>(part, score, keff, (T *)O, a);
     return cudaGetLastError();
 }
 

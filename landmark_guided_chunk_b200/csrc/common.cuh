@@ -2,6 +2,7 @@
 // HSA library.  Host code outside this library never includes it.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -32,7 +33,7 @@ struct WsLayout {
     size_t partials;     // decode split attend: rows x kmax x G x d fp32
     size_t total;
     int nsplit, chunks_per_split;
-    bool split_select, split_attend;
+    bool split_select, split_attend, tc_select;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
 };
 
@@ -156,6 +157,16 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 // ---------------------------------------------------------------------------- launchers
 // Each returns a cudaError_t from the launch; shapes are already validated.
+
+// bf16 TMA tensor maps (128-byte swizzle); strides in bytes, box in elements.
+cudaError_t make_tmap_2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                         uint32_t box_outer);
+cudaError_t make_tmap_3d(CUtensorMap *m, const void *base, const uint64_t dims3[3], const uint64_t strides_bytes[2],
+                         const uint32_t box3[3]);
+
+bool select_tc_supported(const Prob &p);
+cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score, int32_t *keff,
+                             uint32_t *status, cudaStream_t st);
 
 cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,

@@ -38,8 +38,10 @@ WsLayout ws_layout(const Prob &p) {
     w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
     w.sel_score = take(rows * p.kmax * sizeof(float));
     w.sel_keff = take(rows * sizeof(int32_t));
-    // Few rows with long scans: split each row's chunk range over CTAs.
-    w.split_select = rows > 0 && rows <= 4096 && p.C >= 2048;
+    // Many rows: tensor-core scoring.  Few rows with long scans: split each
+    // row's chunk range over CTAs.  Otherwise one warp per row.
+    w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(p);
+    w.split_select = !w.tc_select && rows > 0 && rows <= 4096 && p.C >= 2048;
     if (w.split_select) {
         const long long target = 148 * 8;
         long long per_row = (target + (long long)rows - 1) / (long long)rows;
@@ -57,7 +59,9 @@ WsLayout ws_layout(const Prob &p) {
     const bool has_chunks = (long long)p.B * p.C > 0;
     w.plan.landmark_path = has_chunks ? HSA_PATH_SIMT_ROWS : HSA_PATH_NONE;
     w.plan.landmark_kernels = has_chunks ? 1 : 0;
-    w.plan.select_path = rows == 0 ? HSA_PATH_NONE : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
+    w.plan.select_path = rows == 0 ? HSA_PATH_NONE
+                         : w.tc_select  ? HSA_PATH_TENSOR
+                         : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     w.plan.select_kernels = rows == 0 ? 0 : (w.split_select ? 2 : 1);
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     w.plan.attend_kernels = rows == 0 ? 0 : (w.split_attend ? 2 : 1);
@@ -75,7 +79,8 @@ static hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
     if (in->dtype != HSA_F32 && in->dtype != HSA_BF16) return fail(HSA_ERR_INVALID_ARG, "unknown dtype %d", in->dtype);
     if (!(in->tau >= 0.0f) || isinf(in->tau)) return fail(HSA_ERR_INVALID_ARG, "tau must be finite and >= 0");
     if (in->q_pos0 < 0) return fail(HSA_ERR_INVALID_ARG, "q_pos0 must be >= 0");
-    if (in->flags & ~HSA_FLAG_LANDMARKS_READY) return fail(HSA_ERR_INVALID_ARG, "unknown flags 0x%x", in->flags);
+    if (in->flags & ~(HSA_FLAG_LANDMARKS_READY | HSA_FLAG_SIMT))
+        return fail(HSA_ERR_INVALID_ARG, "unknown flags 0x%x", in->flags);
     if (in->d != 64 && in->d != 128) return fail(HSA_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", in->d);
     if (in->S != 32 && in->S != 64 && in->S != 128)
         return fail(HSA_ERR_UNSUPPORTED, "S=%d (supported: 32, 64, 128)", in->S);

@@ -197,6 +197,7 @@ cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const 
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
                           float *score, int32_t *keff, char *ws, cudaStream_t st) {
     if (p.rows == 0) return cudaSuccess;
+    if (w.tc_select) return launch_select_tc(p, Q, L, idx, score, keff, reinterpret_cast<uint32_t *>(ws + w.hdr), st);
     if (p.dtype == HSA_BF16) return launch_typed<__nv_bfloat16>(p, w, Q, L, idx, score, keff, ws, st);
     return launch_typed<float>(p, w, Q, L, idx, score, keff, ws, st);
 }

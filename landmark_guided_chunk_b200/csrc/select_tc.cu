@@ -1,0 +1,326 @@
+// select_tc.cu -- causal landmark scoring on the tcgen05 tensor cores, fused
+// with the per-row top-k and the gap router (HSA summary page, Core Technique
+// and Implementation: score every landmark of the strictly-past chunks, keep
+// the k best; value-of-information router page: double k on a near-tied cut).
+//
+// For one (batch b, kv head j) the group score of query row t and chunk c is
+//     s[t][c] = sum_{h in group j} q_h[t] . L[c]  =  A[t] . Bcat[c]
+// with A[t] = the G*d contiguous values Q[b][t][jG..jG+G-1][:] and Bcat[c] =
+// L[c] repeated G times.  So it is one bf16 GEMM with K = G*d, accumulated
+// in fp32 in TMEM, and the group sum comes out exact up to fp32 rounding.
+// Since B repeats, only the d/64 distinct 64-column blocks of L are staged.
+//
+// Persistent CTAs walk 128-token M-tiles, heaviest (latest) first.  A tile's
+// rows have at most nc_max = floor((q_pos0 + t_last)/S) candidates, so only
+// ceil(nc_max/128) N-slices of 128 chunks are computed.  The causal triangle
+// is skipped at slice granularity, and the last slice's N is trimmed to a
+// multiple of 16.
+//
+//   warp 0      TMA producer: the A tile (G*d/64 boxes of 128 rows x 64 cols)
+//               once per tile, L slices into a 2-stage ring
+//   warp 1      MMA issuer: 4*G*d/64 tcgen05.mma (M128, N<=128, K16) per slice
+//               into one of two TMEM accumulators
+//   warp 2      TMEM allocator (256 columns)
+//   warps 4..7  epilogue: thread = row.  tcgen05.ld 32 scores at a time, mask
+//               c >= ncand(t), threshold-reject, insert into a sorted
+//               register list (score desc, chunk asc: chunks arrive in
+//               increasing order, so a strict > keeps ties on the lower index)
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int TM = 128;        // tokens per M-tile
+constexpr int NT = 128;        // chunks per N-slice
+constexpr int NSTAGE = 2;      // L-slice ring depth
+constexpr int BOX = 64 * 128 * 2;   // one 64-column x 128-row bf16 box (16 KB)
+constexpr uint32_t TMEM_COLS = 2 * NT;
+
+struct TcSelArgs {
+    int B, Tq, Hkv, G, d, S, C, k, kmax;
+    int nkb, dkb;            // G*d/64 and d/64
+    int mtiles, ntiles;
+    long long q_pos0;
+    float tau;
+    uint32_t *status;
+};
+
+struct __align__(8) Bars {
+    uint64_t a_full, a_empty, done;
+    uint64_t b_full[NSTAGE], b_empty[NSTAGE];
+    uint64_t t_full[2], t_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct Tile {
+    int b, j, t0, nc_max, nslices;
+};
+
+__device__ __forceinline__ Tile tile_of(const TcSelArgs &a, int tau) {
+    Tile T;
+    const int bh = a.B * a.Hkv;
+    const int mt = a.mtiles - 1 - tau / bh;   // latest (heaviest) tiles first
+    const int r = tau % bh;
+    T.b = r / a.Hkv;
+    T.j = r % a.Hkv;
+    T.t0 = mt * TM;
+    const int t_last = min(T.t0 + TM - 1, a.Tq - 1);
+    long long nc = (a.q_pos0 + t_last) / a.S;
+    T.nc_max = (int)(nc < a.C ? nc : a.C);
+    T.nslices = (T.nc_max + NT - 1) / NT;
+    return T;
+}
+
+__device__ __forceinline__ int slice_n(const Tile &T, int n) {
+    int w = min(NT, T.nc_max - n * NT);
+    return (w + 15) & ~15;
+}
+
+template <int KL>
+__device__ __forceinline__ void list_push(float (&v)[KL], int (&id)[KL], float x, int xi) {
+#pragma unroll
+    for (int q = 0; q < KL; ++q) {
+        const bool sw = x > v[q];
+        const float tv = v[q];
+        const int ti = id[q];
+        v[q] = sw ? x : tv;
+        id[q] = sw ? xi : ti;
+        x = sw ? tv : x;
+        xi = sw ? ti : xi;
+    }
+}
+
+template <int KL>
+__global__ void __launch_bounds__(256, 1)
+    select_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmL,
+                     int32_t *__restrict__ idx, float *__restrict__ score, int32_t *__restrict__ keff, TcSelArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = base;                                   // nkb boxes
+    uint8_t *sB = base + (size_t)a.nkb * BOX;             // NSTAGE x dkb boxes
+    Bars *bar = reinterpret_cast<Bars *>(sB + (size_t)NSTAGE * a.dkb * BOX);
+    volatile int *abort = &bar->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar->a_full, 1);
+        mbar_init(&bar->a_empty, 1);
+        mbar_init(&bar->done, 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(&bar->b_full[s], 1);
+            mbar_init(&bar->b_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar->t_full[s], 1);
+            mbar_init(&bar->t_empty[s], 4);
+        }
+        bar->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&bar->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmL);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int g = 0, ta = 0;
+            bool ok = true;
+            for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
+                const Tile T = tile_of(a, tau);
+                if (T.nslices == 0) continue;
+                if (ta > 0 && !(ok = mbar_wait(&bar->a_empty, (ta - 1) & 1, abort, a.status))) break;
+                mbar_expect_tx(&bar->a_full, (uint32_t)(a.nkb * BOX));
+                const int y = T.b * a.Tq + T.t0;
+                for (int kb = 0; kb < a.nkb; ++kb)
+                    tma_load_2d(sA + (size_t)kb * BOX, &tmQ, T.j * a.G * a.d + kb * 64, y, &bar->a_full);
+                ++ta;
+                const int ly = (T.b * a.Hkv + T.j) * a.C;
+                for (int n = 0; n < T.nslices; ++n, ++g) {
+                    const int s = g % NSTAGE, i = g / NSTAGE;
+                    if (i > 0 && !(ok = mbar_wait(&bar->b_empty[s], (i - 1) & 1, abort, a.status))) break;
+                    mbar_expect_tx(&bar->b_full[s], (uint32_t)(a.dkb * BOX));
+                    for (int kd = 0; kd < a.dkb; ++kd)
+                        tma_load_2d(sB + (size_t)(s * a.dkb + kd) * BOX, &tmL, kd * 64, ly + n * NT, &bar->b_full[s]);
+                }
+            }
+            // wind down: every load issued has landed before the CTA may exit
+            if (ta > 0) mbar_drain(&bar->a_full, (ta - 1) & 1);
+            for (int s = 0; s < NSTAGE && s < g; ++s) {
+                const int last = (g - 1 - s) / NSTAGE;   // index of the last use of stage s
+                mbar_drain(&bar->b_full[s], last & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int g = 0, ta = 0;
+            bool ok = true;
+            for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
+                const Tile T = tile_of(a, tau);
+                if (T.nslices == 0) continue;
+                if (!(ok = mbar_wait(&bar->a_full, ta & 1, abort, a.status))) break;
+                ++ta;
+                for (int n = 0; n < T.nslices; ++n, ++g) {
+                    const int s = g % NSTAGE, i = g / NSTAGE, buf = g & 1, u = g >> 1;
+                    if (!(ok = mbar_wait(&bar->b_full[s], i & 1, abort, a.status))) break;
+                    if (u > 0 && !(ok = mbar_wait(&bar->t_empty[buf], (u - 1) & 1, abort, a.status))) break;
+                    tc_fence_after();
+                    const uint32_t idesc = idesc_bf16_f32(TM, slice_n(T, n), 0, 0);
+                    const uint32_t d_tmem = tmem + (uint32_t)(buf * NT);
+                    const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB + (size_t)s * a.dkb * BOX);
+                    for (int kb = 0; kb < a.nkb; ++kb) {
+                        const uint32_t aK = aBase + kb * BOX, bK = bBase + (kb % a.dkb) * BOX;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d_tmem, desc_kmajor_sw128(aK + kk * 32), desc_kmajor_sw128(bK + kk * 32), idesc,
+                                      (kb | kk) != 0);
+                    }
+                    umma_commit(&bar->b_empty[s]);
+                    umma_commit(&bar->t_full[buf]);
+                }
+                if (ok) umma_commit(&bar->a_empty);
+            }
+            umma_commit(&bar->done);
+            mbar_drain(&bar->done, 0);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue: thread = row
+        const int ew = warp - 4;
+        const int r = ew * 32 + lane;
+        const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
+        int g = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
+            const Tile T = tile_of(a, tau);
+            const int t = T.t0 + r;
+            const bool valid = t < a.Tq;
+            int nc = 0;
+            if (valid) {
+                long long x = (a.q_pos0 + t) / a.S;
+                nc = (int)(x < a.C ? x : a.C);
+            }
+            float v[KL];
+            int id[KL];
+#pragma unroll
+            for (int q = 0; q < KL; ++q) {
+                v[q] = -INFINITY;
+                id[q] = -1;
+            }
+            for (int n = 0; n < T.nslices; ++n, ++g) {
+                const int buf = g & 1, u = g >> 1;
+                if (!(ok = mbar_wait(&bar->t_full[buf], u & 1, abort, a.status))) break;
+                tc_fence_after();
+                const int nchunks = (slice_n(T, n) + 31) / 32;
+                for (int q = 0; q < nchunks; ++q) {
+                    uint32_t rr[32];
+                    tmem_ld32(lane_base + (uint32_t)(buf * NT + q * 32), rr);
+                    tmem_wait_ld();
+                    const int cb = n * NT + q * 32;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float sv = __uint_as_float(rr[e]);
+                        if (cb + e < nc && sv > v[KL - 1]) list_push<KL>(v, id, sv, cb + e);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar->t_empty[buf]);
+            }
+            if (!ok || !valid) continue;
+            int ke = nc < a.k ? nc : a.k;
+            if (a.tau > 0.f && nc > a.k) {
+                float sk = 0.f, sk1 = 0.f;
+#pragma unroll
+                for (int q = 0; q < KL; ++q) {
+                    if (q == a.k - 1) sk = v[q];
+                    if (q == a.k) sk1 = v[q];
+                }
+                if (sk - sk1 < a.tau * fabsf(sk)) ke = nc < 2 * a.k ? nc : 2 * a.k;
+            }
+            const long long row = ((long long)T.b * a.Tq + t) * a.Hkv + T.j;
+            int32_t *oi = idx + row * a.kmax;
+            float *os = score + row * a.kmax;
+#pragma unroll
+            for (int q = 0; q < KL; ++q) {
+                if (q < a.kmax) {
+                    oi[q] = q < ke ? id[q] : -1;
+                    os[q] = q < ke ? v[q] : -INFINITY;
+                }
+            }
+            keff[row] = ke;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int KL>
+cudaError_t launch_kl(const TcSelArgs &a, const CUtensorMap &mq, const CUtensorMap &ml, int32_t *idx, float *score,
+                      int32_t *keff, int grid, size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(select_tc_kernel<KL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    select_tc_kernel<KL><<<grid, 256, smem, st>>>(mq, ml, idx, score, keff, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool select_tc_supported(const Prob &p) {
+    const int gd = p.G * p.d;
+    return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && gd % 64 == 0 && gd <= 512 && p.Tq >= 64 &&
+           p.C >= 1 && p.kmax <= 32;
+}
+
+cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score, int32_t *keff,
+                             uint32_t *status, cudaStream_t st) {
+    CUtensorMap mq, ml;
+    cudaError_t e = make_tmap_2d(&mq, Q, (uint64_t)p.H * p.d, (uint64_t)p.B * p.Tq, 64, TM);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.C, 64, NT);
+    if (e != cudaSuccess) return e;
+    TcSelArgs a;
+    a.B = p.B;
+    a.Tq = p.Tq;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.d = p.d;
+    a.S = p.S;
+    a.C = p.C;
+    a.k = p.k;
+    a.kmax = p.kmax;
+    a.nkb = p.G * p.d / 64;
+    a.dkb = p.d / 64;
+    a.mtiles = (p.Tq + TM - 1) / TM;
+    a.ntiles = p.B * p.Hkv * a.mtiles;
+    a.q_pos0 = p.q_pos0;
+    a.tau = p.tau;
+    a.status = status;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = a.ntiles < sms ? a.ntiles : sms;
+    const size_t smem = 1024 + (size_t)a.nkb * BOX + (size_t)NSTAGE * a.dkb * BOX + sizeof(Bars);
+    if (p.kmax <= 8) return launch_kl<8>(a, mq, ml, idx, score, keff, grid, smem, st);
+    if (p.kmax <= 16) return launch_kl<16>(a, mq, ml, idx, score, keff, grid, smem, st);
+    return launch_kl<32>(a, mq, ml, idx, score, keff, grid, smem, st);
+}
+
+}  // namespace hsa

@@ -36,16 +36,17 @@ def _oracle_L(p: Problem, inp):
     return oracle.landmarks_stored(K.cpu(), W.cpu(), p.S, p.dtype)
 
 
-def run_case(p: Problem, rows=None, seed=0, landmarks_first=False):
+def run_case(p: Problem, rows=None, seed=0, landmarks_first=False, force_simt=False):
     torch.manual_seed(seed)
     inp = make_inputs(p, seed=seed, device="cuda")
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
     if landmarks_first:
         L = hsa.landmarks(K, W, p.S)
         O, L, idx, score, keff = hsa.forward(Q, K, V, None, p.S, p.k, p.tau, p.q_pos0, L=L,
-                                             landmarks_ready=True, return_selection=True)
+                                             landmarks_ready=True, return_selection=True, force_simt=force_simt)
     else:
-        O, L, idx, score, keff = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, p.q_pos0, return_selection=True)
+        O, L, idx, score, keff = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, p.q_pos0, return_selection=True,
+                                             force_simt=force_simt)
     torch.cuda.synchronize()
     L_orc = _oracle_L(p, inp)
     lm = parity.check_landmarks(L, L_orc)
@@ -76,10 +77,31 @@ SMALL = [
 ]
 
 
+def _plan(p: Problem, simt=False):
+    return hsa.plan(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau,
+                                     torch.bfloat16 if p.dtype == "bf16" else torch.float32,
+                                     hsa._native.HSA_FLAG_SIMT if simt else 0))
+
+
 @pytest.mark.parametrize("p", SMALL, ids=lambda p: p.name)
 def test_small_prefill_all_rows(p):
     r = run_case(p)
     assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
+
+
+@pytest.mark.parametrize("p", [q for q in SMALL if q.dtype == "bf16"], ids=lambda p: p.name)
+def test_small_prefill_cuda_core_path(p):
+    """The same bf16 cases on the CUDA-core kernels (HSA_FLAG_SIMT), so both
+    paths stay pinned to the oracle."""
+    assert _plan(p, simt=True)["select"][0] != "tensor"
+    r = run_case(p, force_simt=True)
+    assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
+
+
+def test_tensor_core_paths_are_the_ones_planned():
+    assert _plan(workload("prefill_bf16"))["select"][0] == "tensor"
+    assert _plan(workload("router_bf16"))["select"][0] == "tensor"
+    assert _plan(SMALL[1])["select"][0] == "tensor"
 
 
 DECODE_SMALL = [
