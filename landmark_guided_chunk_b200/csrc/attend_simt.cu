@@ -285,6 +285,19 @@ cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const
                           const int32_t *idx, const float *score, const int32_t *keff, void *O, char *ws,
                           cudaStream_t st) {
     if (p.rows == 0) return cudaSuccess;
+    if (w.tc_attend) {
+        AttTcBuffers bf;
+        bf.w8 = reinterpret_cast<float *>(ws + w.att_w8);
+        bf.pairs = reinterpret_cast<int32_t *>(ws + w.att_pairs);
+        bf.counters = reinterpret_cast<int32_t *>(ws + w.att_counters);
+        bf.boff = reinterpret_cast<int32_t *>(ws + w.att_boff);
+        bf.btile = reinterpret_cast<int32_t *>(ws + w.att_btile);
+        bf.blk = reinterpret_cast<int32_t *>(ws + w.att_blk);
+        bf.tiles = reinterpret_cast<int2 *>(ws + w.att_tiles);
+        bf.ring = reinterpret_cast<float *>(ws + w.att_ring);
+        bf.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
+        return launch_attend_tc(p, w.att, bf, Q, K, V, idx, score, keff, O, st);
+    }
     if (p.dtype == HSA_BF16) return launch_typed<__nv_bfloat16>(p, w, Q, K, V, idx, score, keff, O, ws, st);
     return launch_typed<float>(p, w, Q, K, V, idx, score, keff, O, ws, st);
 }

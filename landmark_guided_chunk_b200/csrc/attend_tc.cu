@@ -1,0 +1,665 @@
+// attend_tc.cu -- chunk attention + retrieval-weighted fusion on the tcgen05
+// tensor cores, chunk-major (HSA summary page, Implementation: attend to each
+// selected chunk with standard attention, fuse the chunk outputs weighted by
+// the softmax of their retrieval scores).
+//
+// With random selections neighbouring queries share almost no chunks, so a
+// query-major schedule would stream k*S keys per query from memory.  Here
+// the selection is inverted instead: for every (kv head, chunk) we list the
+// (token, slot) pairs that kept it, so K_c and V_c are loaded once per tile of
+// up to TOK = 128/G tokens.  The G heads of each token form the 128-row M
+// operand:
+//     S  = Q_tile . K_c^T / sqrt(d)        tcgen05, M128 x N=S x K=d, TMEM
+//     P  = exp(S - rowmax), l = sum P      epilogue warps, P -> smem (bf16)
+//     O  = P . V_c                          tcgen05, M128 x N=d x K=S, TMEM
+//     O_acc[t][h] += (w_slot / l) * O       fp32 vector reductions
+// Since w is known before the attention, the cross-chunk fusion is linear and
+// needs no rescaling.
+//
+// Accumulators.  The pairs are grouped into phases of TB tokens of one (b, kv
+// head).  Tiles are ordered phase-major, so the active accumulators form a
+// ring of R phase slots that stays resident in L2.  A sub-block of SB tokens
+// is finalised (fp32 -> bf16 into O, slot zeroed) by whichever warp completes
+// its last expected contribution (counter per sub-block).  A tile of phase p
+// waits until phase p-R has been finalised before it reduces into the shared
+// slot.  Persistent CTAs take tiles in increasing order, so that wait always
+// ends.  It is bounded anyway.
+//
+// Helper kernels (before the main kernel): count pairs per (phase, chunk)
+// bucket and compute the fusion weights; two-level exclusive scan of pair
+// and tile counts; tile list; scatter of the pairs into their buckets.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hsa {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;           // head dim of this kernel
+constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
+constexpr int SB = 32;           // tokens per finalisation sub-block
+constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
+constexpr int NT_MAIN = 384;     // 12 warps
+constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
+
+struct AttTcArgs {
+    int B, Tq, Tkv, H, Hkv, G, S, C, kmax, tok;
+    int tb, ntb, nsub, ring, nphase, nbucket, nsq, nskv;
+    long long q_pos0;
+    float scale_log2;            // log2(e) / sqrt(d)
+    const int32_t *idx;
+    const float *score;
+    const int32_t *keff;
+    float *w8;                   // [rows][kmax] fusion weights
+    int32_t *bcount, *bcursor;   // [nbucket]
+    int32_t *boff, *btile;       // [nbucket + 1]
+    int32_t *blk;                // [2 * nblk] first-level block totals
+    int32_t *pairs;              // [rows * kmax]  (t << 5) | slot
+    int2 *tiles;                 // (bucket, first pair)
+    int32_t *sub_need, *sub_done, *phase_done;
+    float *ringbuf;              // [ring][tb][G][D]
+    uint32_t *status;
+};
+
+__device__ __forceinline__ int ncand_of(const AttTcArgs &a, int t) {
+    long long n = (a.q_pos0 + t) / a.S;
+    return (int)(n < a.C ? n : a.C);
+}
+
+__device__ __forceinline__ int phase_of(const AttTcArgs &a, int b, int j, int t) {
+    return (b * a.Hkv + j) * a.ntb + t / a.tb;
+}
+
+// ---------------------------------------------------------------------------- helper kernels
+
+// One thread per selection row: fusion weights, bucket counts, sub-block needs.
+__global__ void att_count_kernel(AttTcArgs a) {
+    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long rows = (long long)a.B * a.Tq * a.Hkv;
+    if (row >= rows) return;
+    const int j = (int)(row % a.Hkv);
+    const long long bt = row / a.Hkv;
+    const int t = (int)(bt % a.Tq), b = (int)(bt / a.Tq);
+    int ke = a.keff[row];
+    if (ke < 0 || ke > a.kmax) {
+        atomicOr(a.status, DEV_BAD_INDEX);
+        ke = ke < 0 ? 0 : a.kmax;
+    }
+    const int nc = ncand_of(a, t);
+    const int p = phase_of(a, b, j, t);
+    const int32_t *ri = a.idx + row * a.kmax;
+    const float *rs = a.score + row * a.kmax;
+    float m = -INFINITY;
+    for (int i = 0; i < ke; ++i) m = fmaxf(m, rs[i]);
+    float z = 0.f;
+    for (int i = 0; i < ke; ++i) z += expf(rs[i] - m);
+    int used = 0;
+    for (int i = 0; i < ke; ++i) {
+        a.w8[row * a.kmax + i] = expf(rs[i] - m) / z;
+        const int c = ri[i];
+        if (c < 0 || c >= nc) {
+            atomicOr(a.status, DEV_BAD_INDEX);
+            continue;
+        }
+        atomicAdd(&a.bcount[(long long)p * a.C + c], 1);
+        ++used;
+    }
+    if (used) atomicAdd(&a.sub_need[p * a.nsub + (t % a.tb) / SB], used);
+}
+
+// First level of the scan: per block of SCAN_BLK buckets, local exclusive
+// prefixes of pair counts (boff) and tile counts (btile), plus block totals.
+__global__ void __launch_bounds__(1024) att_scan1_kernel(AttTcArgs a) {
+    __shared__ int sp[1024], st[1024];
+    const int base = blockIdx.x * SCAN_BLK + threadIdx.x * 4;
+    int np[4], nt[4], sp_, st_;
+    sp_ = st_ = 0;
+    for (int q = 0; q < 4; ++q) {
+        const int u = base + q;
+        const int n = u < a.nbucket ? a.bcount[u] : 0;
+        np[q] = n;
+        nt[q] = (n + a.tok - 1) / a.tok;
+        sp_ += np[q];
+        st_ += nt[q];
+    }
+    sp[threadIdx.x] = sp_;
+    st[threadIdx.x] = st_;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {   // Hillis-Steele inclusive scan
+        int vp = threadIdx.x >= o ? sp[threadIdx.x - o] : 0;
+        int vt = threadIdx.x >= o ? st[threadIdx.x - o] : 0;
+        __syncthreads();
+        sp[threadIdx.x] += vp;
+        st[threadIdx.x] += vt;
+        __syncthreads();
+    }
+    int ep = sp[threadIdx.x] - sp_, et = st[threadIdx.x] - st_;
+    for (int q = 0; q < 4; ++q) {
+        const int u = base + q;
+        if (u < a.nbucket) {
+            a.boff[u] = ep;
+            a.btile[u] = et;
+        }
+        ep += np[q];
+        et += nt[q];
+    }
+    if (threadIdx.x == 1023) {
+        a.blk[2 * blockIdx.x] = sp[1023];
+        a.blk[2 * blockIdx.x + 1] = st[1023];
+    }
+}
+
+// Second level: exclusive scan of the block totals (one block, <= 1024 blocks).
+__global__ void __launch_bounds__(1024) att_scan2_kernel(AttTcArgs a, int nblk) {
+    __shared__ int sp[1024], st[1024];
+    const int i = threadIdx.x;
+    const int vp0 = i < nblk ? a.blk[2 * i] : 0, vt0 = i < nblk ? a.blk[2 * i + 1] : 0;
+    sp[i] = vp0;
+    st[i] = vt0;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        int vp = i >= o ? sp[i - o] : 0;
+        int vt = i >= o ? st[i - o] : 0;
+        __syncthreads();
+        sp[i] += vp;
+        st[i] += vt;
+        __syncthreads();
+    }
+    if (i < nblk) {
+        a.blk[2 * i] = sp[i] - vp0;
+        a.blk[2 * i + 1] = st[i] - vt0;
+    }
+    if (i == 1023) {
+        a.boff[a.nbucket] = sp[1023];
+        a.btile[a.nbucket] = st[1023];
+    }
+}
+
+// Global offsets and the tile list (one thread per bucket).
+__global__ void att_tiles_kernel(AttTcArgs a) {
+    const int u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= a.nbucket) return;
+    const int blk = u / SCAN_BLK;
+    const int op = a.boff[u] + a.blk[2 * blk], ot = a.btile[u] + a.blk[2 * blk + 1];
+    a.boff[u] = op;
+    a.btile[u] = ot;
+    const int n = a.bcount[u];
+    for (int q = 0; q * a.tok < n; ++q) a.tiles[ot + q] = make_int2(u, op + q * a.tok);
+}
+
+// One thread per selection row: place its pairs into their buckets.
+__global__ void att_scatter_kernel(AttTcArgs a) {
+    const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long rows = (long long)a.B * a.Tq * a.Hkv;
+    if (row >= rows) return;
+    const int j = (int)(row % a.Hkv);
+    const long long bt = row / a.Hkv;
+    const int t = (int)(bt % a.Tq), b = (int)(bt / a.Tq);
+    int ke = a.keff[row];
+    ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
+    const int nc = ncand_of(a, t);
+    const int p = phase_of(a, b, j, t);
+    for (int i = 0; i < ke; ++i) {
+        const int c = a.idx[row * a.kmax + i];
+        if (c < 0 || c >= nc) continue;
+        const long long u = (long long)p * a.C + c;
+        const int pos = a.boff[u] + atomicAdd(&a.bcursor[u], 1);
+        a.pairs[pos] = (t << 5) | i;
+    }
+}
+
+// ---------------------------------------------------------------------------- main kernel
+
+struct __align__(8) AttBars {
+    uint64_t q_full[2], q_empty[2], kv_full[2], kv_empty[2];
+    uint64_t s_full, p_full, o_full, o_empty, done;
+    uint32_t tmem_base;
+    int abort;
+    int ntiles;
+};
+
+struct TileInfo {
+    int b, j, c, p, start, n;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const AttTcArgs &a, int tau) {
+    const int2 e = a.tiles[tau];
+    TileInfo T;
+    T.p = e.x / a.C;
+    T.c = e.x % a.C;
+    const int bj = T.p / a.ntb;
+    T.b = bj / a.Hkv;
+    T.j = bj % a.Hkv;
+    T.start = e.y;
+    T.n = min(a.tok, a.boff[e.x + 1] - e.y);
+    return T;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Finalise sub-block sb of phase p with one warp: accumulators -> O (bf16), slot zeroed.
+__device__ void finalize_sub(const AttTcArgs &a, __nv_bfloat16 *O, int p, int sb, bool has_data, int lane) {
+    const int bj = p / a.ntb, tbi = p % a.ntb;
+    const int b = bj / a.Hkv, j = bj % a.Hkv;
+    const int t_begin = tbi * a.tb + sb * SB;
+    const int t_end = min(t_begin + SB, min((tbi + 1) * a.tb, a.Tq));
+    float *slot = a.ringbuf + (size_t)(p % a.ring) * a.tb * a.G * D;
+    for (int t = t_begin; t < t_end; ++t) {
+        for (int g = 0; g < a.G; ++g) {
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 *acc = reinterpret_cast<float4 *>(slot + ((size_t)(t - tbi * a.tb) * a.G + g) * D) + lane;
+            if (has_data) {
+                v = __ldcg(acc);
+                __stcg(acc, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t *>(&lo);
+            pk.y = *reinterpret_cast<uint32_t *>(&hi);
+            reinterpret_cast<uint2 *>(O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + g) * D)[lane] = pk;
+        }
+    }
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(&a.phase_done[p], 1);
+}
+
+__device__ __forceinline__ int nsub_of_phase(const AttTcArgs &a, int p) {
+    const int tbi = p % a.ntb;
+    const int len = min(a.tb, a.Tq - tbi * a.tb);
+    return (len + SB - 1) / SB;
+}
+
+__global__ void __launch_bounds__(NT_MAIN, 1)
+    att_main_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __nv_bfloat16 *__restrict__ Q, __nv_bfloat16 *__restrict__ O, AttTcArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = a.S;
+    const int kv_bytes = S * 128;                         // one 64-column box of S rows
+    uint8_t *sQ = base;                                   // 2 x 32 KB
+    uint8_t *sKV = sQ + 2 * 32768;                        // nskv x (K: 2 boxes, V: 2 boxes)
+    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;    // S/64 x 16 KB
+    float *stg = reinterpret_cast<float *>(sP + (size_t)(S / 64) * 16384);   // 4 warps x 32 x PITCH
+    AttBars *bar = reinterpret_cast<AttBars *>(stg + 4 * 32 * PITCH);
+    volatile int *abort = &bar->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar->q_full[s], 128);
+            mbar_init(&bar->q_empty[s], 1);
+            mbar_init(&bar->kv_full[s], 1);
+            mbar_init(&bar->kv_empty[s], 1);
+        }
+        mbar_init(&bar->s_full, 1);
+        mbar_init(&bar->p_full, 4);
+        mbar_init(&bar->o_full, 1);
+        mbar_init(&bar->o_empty, 4);
+        mbar_init(&bar->done, 1);
+        bar->abort = 0;
+        bar->ntiles = a.btile[a.nbucket];
+        fence_mbar_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(&bar->tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+    const int ntiles = bar->ntiles;
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ producers: Q gather (thread = row), K/V TMA
+        const int r = threadIdx.x;   // 0..127
+        const int m = r / a.G, g = r % a.G;
+        int i = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+            const TileInfo T = tile_info(a, tau);
+            const int sq = i & 1, iq = i >> 1;
+            if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
+            if (warp == 0 && lane == 0) {
+                const int skv = i % a.nskv, ikv = i / a.nskv;
+                if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
+                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
+                uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
+                const int z = T.b * a.Tkv + T.c * S;
+                tma_load_3d(dk, &tmK, 0, T.j, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + kv_bytes, &tmK, 64, T.j, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, T.j, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, T.j, z, &bar->kv_full[skv]);
+            }
+            const bool valid = m < T.n;
+            const char *src = reinterpret_cast<const char *>(Q);
+            if (valid) {
+                const int t = a.pairs[T.start + m] >> 5;
+                src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + g) * D) * 2;
+            }
+            const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const int kb = x >> 3, cx = x & 7;
+                cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
+            }
+            cp_async_arrive(&bar->q_full[sq]);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (warp == 0 && lane == 0) {
+            // wind down: the K/V loads issued have all landed
+            for (int s = 0; s < a.nskv && s < i; ++s) mbar_drain(&bar->kv_full[s], ((i - 1 - s) / a.nskv) & 1);
+        }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t s_tmem = tmem, o_tmem = tmem + 128;
+            const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
+            const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
+            int i = 0;
+            bool ok = true;
+            for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+                const int sq = i & 1, iq = i >> 1, skv = i % a.nskv, ikv = i / a.nskv;
+                if (!(ok = mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status))) break;
+                if (!(ok = mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status))) break;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(sQ + sq * 32768);
+                const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 4 * kv_bytes);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+                    const uint32_t a_addr = qa + (kk >> 2) * 16384 + off;
+                    const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + off;
+                    umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
+                }
+                umma_commit(&bar->s_full);
+                umma_commit(&bar->q_empty[sq]);
+                if (!(ok = mbar_wait(&bar->p_full, i & 1, abort, a.status))) break;
+                if (i > 0 && !(ok = mbar_wait(&bar->o_empty, (i - 1) & 1, abort, a.status))) break;
+                tc_fence_after();
+                const uint32_t pa = smem_u32(sP);
+                const uint32_t vb = kb0 + 2 * kv_bytes;
+                for (int kk = 0; kk < S / 16; ++kk) {
+                    // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it
+                    const uint32_t a_addr = pa + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    // V: MN-major, keys kk*16..+15 = two 8-row groups starting at (kk*16)*128 B;
+                    // the two 64-dim halves are kv_bytes apart
+                    const uint32_t b_addr = vb + kk * 16 * 128;
+                    umma_bf16(o_tmem, desc_kmajor_sw128(a_addr), desc_mnmajor_sw128(b_addr, kv_bytes, 1024), idesc_o,
+                              kk != 0);
+                }
+                umma_commit(&bar->o_full);
+                umma_commit(&bar->kv_empty[skv]);
+            }
+            umma_commit(&bar->done);
+            mbar_drain(&bar->done, 0);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ epilogue: thread = tile row
+        const int ew = warp - 8;
+        const int r = ew * 32 + lane;
+        const int m = r / a.G, g = r % a.G;
+        const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
+        float *wst = stg + ew * 32 * PITCH;
+        // sub-blocks nobody contributes to: write their zeros right away
+        {
+            const int total = a.nphase * a.nsub;
+            for (int e = (blockIdx.x * 4 + ew); e < total; e += gridDim.x * 4) {
+                const int p = e / a.nsub, sb = e % a.nsub;
+                if (sb < nsub_of_phase(a, p) && a.sub_need[e] == 0) finalize_sub(a, O, p, sb, false, lane);
+            }
+        }
+        int i = 0;
+        bool ok = true;
+        for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+            const TileInfo T = tile_info(a, tau);
+            const bool valid = m < T.n;
+            int t = 0, slot = 0;
+            float w = 0.f;
+            if (valid) {
+                const int pr = a.pairs[T.start + m];
+                t = pr >> 5;
+                slot = pr & 31;
+                w = a.w8[(((long long)T.b * a.Tq + t) * a.Hkv + T.j) * a.kmax + slot];
+            }
+            // chunk softmax: S row -> P row (bf16, swizzled), l
+            if (!(ok = mbar_wait(&bar->s_full, i & 1, abort, a.status))) break;
+            tc_fence_after();
+            float l = 0.f;
+            {
+                uint32_t sr[32];
+                float mx = -INFINITY;
+                for (int q = 0; q < S / 32; ++q) {
+                    tmem_ld32(lane_base + q * 32, sr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
+                }
+                for (int q = 0; q < S / 32; ++q) {
+                    tmem_ld32(lane_base + q * 32, sr);
+                    tmem_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = exp2f((__uint_as_float(sr[2 * e]) - mx) * a.scale_log2);
+                        const float p1 = exp2f((__uint_as_float(sr[2 * e + 1]) - mx) * a.scale_log2);
+                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                        // the MMA sees the rounded probabilities: normalise by their sum
+                        const float2 hf = __bfloat1622float2(h);
+                        l += hf.x + hf.y;
+                        pk[e] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    // 32 keys = 4 16-B chunks of the 128-B row of k-block q/2
+                    uint8_t *prow = sP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int cx = (q & 1) * 4 + x;
+                        *reinterpret_cast<uint4 *>(prow + ((cx ^ (r & 7)) << 4)) =
+                            make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->p_full);
+            // ring slot of this phase must be free (phase p - ring finalised)
+            if (T.p >= a.ring) {
+                if (lane == 0) {
+                    const int need = nsub_of_phase(a, T.p - a.ring);
+                    volatile int *pd = a.phase_done + (T.p - a.ring);
+                    const uint64_t t0 = globaltimer_ns();
+                    while (*pd < need) {
+                        if (*abort) break;
+                        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                            *abort = 1;
+                            atomicOr(a.status, DEV_TIMEOUT);
+                            break;
+                        }
+                    }
+                    __threadfence();
+                }
+                __syncwarp();
+            }
+            // O row -> scaled fp32 contributions, reduced into the ring slot 32 columns at a time
+            if (!(ok = mbar_wait(&bar->o_full, i & 1, abort, a.status))) break;
+            tc_fence_after();
+            const float f = valid ? w / l : 0.f;
+            float *acc_slot = a.ringbuf + (size_t)(T.p % a.ring) * a.tb * a.G * D;
+            const int tloc_base = (T.p % a.ntb) * a.tb;
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t orr[32];
+                tmem_ld32(lane_base + 128 + q * 32, orr);
+                tmem_wait_ld();
+                if (q == D / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar->o_empty);
+                }
+                float *mine = wst + lane * PITCH;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(mine + e) =
+                        make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
+                                    __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
+                __syncwarp();
+                // lane -> (row rr*4 + lane/8, 4 floats at column 4*(lane%8))
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int lr = rr * 4 + (lane >> 3);   // row within this warp
+                    const int R = ew * 32 + lr;
+                    const int mm = R / a.G, gg = R % a.G;
+                    const int pr = mm < T.n ? a.pairs[T.start + mm] : -1;
+                    if (pr >= 0) {
+                        const int tt = pr >> 5;
+                        float *dst = acc_slot + ((size_t)(tt - tloc_base) * a.G + gg) * D + q * 32 + 4 * (lane & 7);
+                        const float4 v = *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7));
+                        atomicAdd(reinterpret_cast<float4 *>(dst), v);
+                    }
+                }
+                __syncwarp();
+            }
+            // count the pairs of this warp's tokens; finalise completed sub-blocks
+            __threadfence();
+            __syncwarp();
+            bool fin = false;
+            int fsb = 0;
+            if (valid && g == 0) {
+                fsb = (t - tloc_base) / SB;
+                const int old = atomicAdd(&a.sub_done[T.p * a.nsub + fsb], 1);
+                fin = (old + 1 == a.sub_need[T.p * a.nsub + fsb]);
+                if (fin) __threadfence();
+            }
+            unsigned fm = __ballot_sync(FULL, fin);
+            while (fm) {
+                const int src = __ffs(fm) - 1;
+                fm &= fm - 1;
+                const int sbv = __shfl_sync(FULL, fsb, src);
+                finalize_sub(a, O, T.p, sbv, true, lane);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------- host side
+
+static int att_tb(const Prob &) { return 4096; }
+
+bool attend_tc_supported(const Prob &p) {
+    if (!(p.dtype == HSA_BF16 && p.d == D && (p.S == 64 || p.S == 128) && p.G <= 16 && (32 % p.G) == 0 &&
+          p.C >= 1 && p.Tq >= 1 && p.kmax <= 32 && p.Tq < (1 << 26)))
+        return false;
+    // the second scan level is one block of 1024 threads over SCAN_BLK-bucket blocks
+    const long long ntb = (p.Tq + att_tb(p) - 1) / att_tb(p);
+    const long long nbucket = (long long)p.B * p.Hkv * ntb * p.C;
+    return nbucket <= 1024LL * SCAN_BLK && (long long)p.rows * p.kmax < (1LL << 31);
+}
+static int att_ring() { return 4; }
+
+AttTcLayout attend_tc_layout(const Prob &p) {
+    AttTcLayout L{};
+    L.tb = att_tb(p);
+    L.ntb = (p.Tq + L.tb - 1) / L.tb;
+    L.nsub = L.tb / SB;
+    L.nphase = p.B * p.Hkv * L.ntb;
+    L.nbucket = L.nphase * p.C;
+    L.nblk = (L.nbucket + SCAN_BLK - 1) / SCAN_BLK;
+    L.tok = MROWS / p.G;
+    L.ring = att_ring();
+    const size_t pairs = (size_t)p.rows * p.kmax;
+    L.max_tiles = pairs / L.tok + (size_t)L.nbucket + 1;
+    L.counter_ints = 2 * (size_t)L.nbucket + 2 * (size_t)L.nphase * L.nsub + L.nphase;
+    L.ring_bytes = (size_t)L.ring * L.tb * p.G * D * sizeof(float);
+    return L;
+}
+
+cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,
+                             const void *V, const int32_t *idx, const float *score, const int32_t *keff, void *O,
+                             cudaStream_t st) {
+    AttTcArgs a;
+    a.B = p.B;
+    a.Tq = p.Tq;
+    a.Tkv = p.Tkv;
+    a.H = p.H;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.S = p.S;
+    a.C = p.C;
+    a.kmax = p.kmax;
+    a.tok = L.tok;
+    a.tb = L.tb;
+    a.ntb = L.ntb;
+    a.nsub = L.nsub;
+    a.ring = L.ring;
+    a.nphase = L.nphase;
+    a.nbucket = L.nbucket;
+    a.nsq = 2;
+    a.nskv = p.S <= 64 ? 2 : 1;
+    a.q_pos0 = p.q_pos0;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
+    a.idx = idx;
+    a.score = score;
+    a.keff = keff;
+    a.w8 = bf.w8;
+    a.bcount = bf.counters;
+    a.bcursor = bf.counters + L.nbucket;
+    a.sub_need = bf.counters + 2 * (size_t)L.nbucket;
+    a.sub_done = a.sub_need + (size_t)L.nphase * L.nsub;
+    a.phase_done = a.sub_done + (size_t)L.nphase * L.nsub;
+    a.boff = bf.boff;
+    a.btile = bf.btile;
+    a.blk = bf.blk;
+    a.pairs = bf.pairs;
+    a.tiles = bf.tiles;
+    a.ringbuf = bf.ring;
+    a.status = bf.status;
+
+    // counters and ring slots start at zero on every call
+    cudaError_t e = cudaMemsetAsync(bf.counters, 0, L.counter_ints * sizeof(int32_t), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(bf.ring, 0, L.ring_bytes, st);
+    if (e != cudaSuccess) return e;
+    const int rows_blocks = (int)((p.rows + 255) / 256);
+    att_count_kernel<<<rows_blocks, 256, 0, st>>>(a);
+    att_scan1_kernel<<<L.nblk, 1024, 0, st>>>(a);
+    att_scan2_kernel<<<1, 1024, 0, st>>>(a, L.nblk);
+    att_tiles_kernel<<<(L.nbucket + 255) / 256, 256, 0, st>>>(a);
+    att_scatter_kernel<<<rows_blocks, 256, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    // K and V as 3D (d, Hkv, B*Tkv): box (64, 1, S) = S rows of 128 B
+    CUtensorMap mk, mv;
+    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tkv};
+    const uint64_t strides[2] = {(uint64_t)p.d * 2, (uint64_t)p.Hkv * p.d * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)p.S};
+    if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
+    const int nskv = a.nskv;
+    const size_t smem = 1024 + 2 * 32768 + (size_t)nskv * 4 * p.S * 128 + (size_t)(p.S / 64) * 16384 +
+                        4 * 32 * PITCH * sizeof(float) + sizeof(AttBars);
+    if ((e = cudaFuncSetAttribute(att_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+        cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    att_main_kernel<<<sms, NT_MAIN, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
+    return cudaGetLastError();
+}
+
+}  // namespace hsa

@@ -25,6 +25,20 @@ struct Prob {
     long long rows;   // B * Tq * Hkv selection rows
 };
 
+// Sizes of the chunk-major tensor-core attention's workspace pieces.
+struct AttTcLayout {
+    int tb, ntb, nsub, nphase, nbucket, nblk, tok, ring;
+    size_t max_tiles, counter_ints, ring_bytes;
+};
+
+struct AttTcBuffers {
+    float *w8;
+    int32_t *pairs, *counters, *boff, *btile, *blk;
+    int2 *tiles;
+    float *ring;
+    uint32_t *status;
+};
+
 // Byte offsets inside the caller's workspace (all 256-byte aligned).
 struct WsLayout {
     size_t hdr;          // device-status word (uint32) + padding
@@ -33,7 +47,9 @@ struct WsLayout {
     size_t partials;     // decode split attend: rows x kmax x G x d fp32
     size_t total;
     int nsplit, chunks_per_split;
-    bool split_select, split_attend, tc_select;
+    bool split_select, split_attend, tc_select, tc_attend;
+    AttTcLayout att;
+    size_t att_w8, att_pairs, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
 };
 
@@ -167,6 +183,12 @@ cudaError_t make_tmap_3d(CUtensorMap *m, const void *base, const uint64_t dims3[
 bool select_tc_supported(const Prob &p);
 cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score, int32_t *keff,
                              uint32_t *status, cudaStream_t st);
+
+bool attend_tc_supported(const Prob &p);
+AttTcLayout attend_tc_layout(const Prob &p);
+cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,
+                             const void *V, const int32_t *idx, const float *score, const int32_t *keff, void *O,
+                             cudaStream_t st);
 
 cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,

@@ -52,9 +52,22 @@ WsLayout ws_layout(const Prob &p) {
         w.nsplit = (int)(((long long)p.C + cps - 1) / cps);
         w.split_lists = take(rows * (size_t)w.nsplit * p.kmax * sizeof(float2));
     }
-    // Few rows: parallelise the attention over the kept slots too.
+    // Many rows: chunk-major tensor-core attention.  Few rows: parallelise the
+    // CUDA-core attention over the kept slots too.
     w.split_attend = rows > 0 && rows <= 2048;
+    w.tc_attend = !w.split_attend && rows > 0 && !(p.flags & HSA_FLAG_SIMT) && attend_tc_supported(p);
     if (w.split_attend) w.partials = take(rows * (size_t)p.kmax * p.G * p.d * sizeof(float));
+    if (w.tc_attend) {
+        w.att = attend_tc_layout(p);
+        w.att_w8 = take(rows * p.kmax * sizeof(float));
+        w.att_pairs = take(rows * p.kmax * sizeof(int32_t));
+        w.att_counters = take(w.att.counter_ints * sizeof(int32_t));
+        w.att_boff = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
+        w.att_btile = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
+        w.att_blk = take(2 * (size_t)w.att.nblk * sizeof(int32_t));
+        w.att_tiles = take(w.att.max_tiles * sizeof(int2));
+        w.att_ring = take(w.att.ring_bytes);
+    }
     w.total = off;
     const bool has_chunks = (long long)p.B * p.C > 0;
     w.plan.landmark_path = has_chunks ? HSA_PATH_SIMT_ROWS : HSA_PATH_NONE;
@@ -63,8 +76,11 @@ WsLayout ws_layout(const Prob &p) {
                          : w.tc_select  ? HSA_PATH_TENSOR
                          : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     w.plan.select_kernels = rows == 0 ? 0 : (w.split_select ? 2 : 1);
-    w.plan.attend_path = rows == 0 ? HSA_PATH_NONE : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
-    w.plan.attend_kernels = rows == 0 ? 0 : (w.split_attend ? 2 : 1);
+    w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
+                         : w.tc_attend  ? HSA_PATH_TENSOR
+                         : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
+    // tensor path: count, scan (2 levels), tile list, scatter, main kernel
+    w.plan.attend_kernels = rows == 0 ? 0 : (w.tc_attend ? 6 : (w.split_attend ? 2 : 1));
     return w;
 }
 

@@ -21,10 +21,14 @@
 //   warp 1      MMA issuer: 4*G*d/64 tcgen05.mma (M128, N<=128, K16) per slice
 //               into one of two TMEM accumulators
 //   warp 2      TMEM allocator (256 columns)
-//   warps 4..7  epilogue: thread = row.  tcgen05.ld 32 scores at a time, mask
-//               c >= ncand(t), threshold-reject, insert into a sorted
-//               register list (score desc, chunk asc: chunks arrive in
-//               increasing order, so a strict > keeps ties on the lower index)
+//   warps 4..7  epilogue: thread = row.  tcgen05.ld 32 scores at a time.
+//               Scores of candidate chunks (c < ncand(t)) that beat the
+//               row's current k-th best are appended to a per-thread queue
+//               in shared memory (predicated stores, no divergence).  The
+//               warp then drains the queues in lock-step into sorted
+//               register lists (score desc, chunk asc).  Chunks arrive in
+//               increasing order, so counting the entries >= s gives the
+//               insertion position and keeps ties on the lower index.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -80,17 +84,23 @@ __device__ __forceinline__ int slice_n(const Tile &T, int n) {
     return (w + 15) & ~15;
 }
 
+// Insert (x, xi) into the sorted list; xi is larger than every chunk index
+// already present, so equal scores already in the list stay ahead of it.
 template <int KL>
 __device__ __forceinline__ void list_push(float (&v)[KL], int (&id)[KL], float x, int xi) {
+    int pos = 0;
 #pragma unroll
-    for (int q = 0; q < KL; ++q) {
-        const bool sw = x > v[q];
-        const float tv = v[q];
-        const int ti = id[q];
-        v[q] = sw ? x : tv;
-        id[q] = sw ? xi : ti;
-        x = sw ? tv : x;
-        xi = sw ? ti : xi;
+    for (int q = 0; q < KL; ++q) pos += (v[q] >= x) ? 1 : 0;
+    if (pos >= KL) return;
+#pragma unroll
+    for (int q = KL - 1; q > 0; --q) {
+        const bool sh = q > pos, eq = q == pos;
+        v[q] = sh ? v[q - 1] : (eq ? x : v[q]);
+        id[q] = sh ? id[q - 1] : (eq ? xi : id[q]);
+    }
+    if (pos == 0) {
+        v[0] = x;
+        id[0] = xi;
     }
 }
 
@@ -102,7 +112,9 @@ __global__ void __launch_bounds__(256, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;                                   // nkb boxes
     uint8_t *sB = base + (size_t)a.nkb * BOX;             // NSTAGE x dkb boxes
-    Bars *bar = reinterpret_cast<Bars *>(sB + (size_t)NSTAGE * a.dkb * BOX);
+    float *qv = reinterpret_cast<float *>(sB + (size_t)NSTAGE * a.dkb * BOX);   // [32][128] queued scores
+    int *qi = reinterpret_cast<int *>(qv + 32 * 128);                          // [32][128] queued chunks
+    Bars *bar = reinterpret_cast<Bars *>(qi + 32 * 128);
     volatile int *abort = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -230,11 +242,21 @@ __global__ void __launch_bounds__(256, 1)
                     tmem_ld32(lane_base + (uint32_t)(buf * NT + q * 32), rr);
                     tmem_wait_ld();
                     const int cb = n * NT + q * 32;
+                    const float thr = v[KL - 1];
+                    int cnt = 0;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const float sv = __uint_as_float(rr[e]);
-                        if (cb + e < nc && sv > v[KL - 1]) list_push<KL>(v, id, sv, cb + e);
+                        const bool take = (cb + e < nc) && (sv > thr);
+                        if (take) {
+                            qv[cnt * 128 + r] = sv;
+                            qi[cnt * 128 + r] = cb + e;
+                        }
+                        cnt += take ? 1 : 0;
                     }
+                    const int it_max = __reduce_max_sync(FULL, (unsigned)cnt);
+                    for (int it = 0; it < it_max; ++it)
+                        if (it < cnt) list_push<KL>(v, id, qv[it * 128 + r], qi[it * 128 + r]);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -317,7 +339,7 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = a.ntiles < sms ? a.ntiles : sms;
-    const size_t smem = 1024 + (size_t)a.nkb * BOX + (size_t)NSTAGE * a.dkb * BOX + sizeof(Bars);
+    const size_t smem = 1024 + (size_t)a.nkb * BOX + (size_t)NSTAGE * a.dkb * BOX + 2 * 32 * 128 * 4 + sizeof(Bars);
     if (p.kmax <= 8) return launch_kl<8>(a, mq, ml, idx, score, keff, grid, smem, st);
     if (p.kmax <= 16) return launch_kl<16>(a, mq, ml, idx, score, keff, grid, smem, st);
     return launch_kl<32>(a, mq, ml, idx, score, keff, grid, smem, st);
