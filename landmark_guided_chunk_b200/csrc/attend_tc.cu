@@ -41,7 +41,6 @@ constexpr int D = 128;           // head dim of this kernel
 constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
 constexpr int SB = 32;           // tokens per finalisation sub-block
 constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
-constexpr int NT_MAIN = 384;     // 12 warps
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
 
 struct AttTcArgs {
@@ -212,9 +211,11 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
 
 // ---------------------------------------------------------------------------- main kernel
 
+constexpr int NDEF = 8;   // sub-block counter increments a warp batches behind one fence
+
 struct __align__(8) AttBars {
     uint64_t q_full[2], q_empty[2], kv_full[2], kv_empty[2];
-    uint64_t s_full, p_full, o_full, o_empty, done;
+    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], done;
     uint32_t tmem_base;
     int abort;
     int ntiles;
@@ -243,32 +244,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-
-// Finalise sub-block sb of phase p with one warp: accumulators -> O (bf16), slot zeroed.
-__device__ void finalize_sub(const AttTcArgs &a, __nv_bfloat16 *O, int p, int sb, bool has_data, int lane) {
-    const int bj = p / a.ntb, tbi = p % a.ntb;
-    const int b = bj / a.Hkv, j = bj % a.Hkv;
-    const int t_begin = tbi * a.tb + sb * SB;
-    const int t_end = min(t_begin + SB, min((tbi + 1) * a.tb, a.Tq));
-    float *slot = a.ringbuf + (size_t)(p % a.ring) * a.tb * a.G * D;
-    for (int t = t_begin; t < t_end; ++t) {
-        for (int g = 0; g < a.G; ++g) {
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            float4 *acc = reinterpret_cast<float4 *>(slot + ((size_t)(t - tbi * a.tb) * a.G + g) * D) + lane;
-            if (has_data) {
-                v = __ldcg(acc);
-                __stcg(acc, make_float4(0.f, 0.f, 0.f, 0.f));
-            }
-            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t *>(&lo);
-            pk.y = *reinterpret_cast<uint32_t *>(&hi);
-            reinterpret_cast<uint2 *>(O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + g) * D)[lane] = pk;
-        }
-    }
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(&a.phase_done[p], 1);
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ int nsub_of_phase(const AttTcArgs &a, int p) {
@@ -277,18 +256,91 @@ __device__ __forceinline__ int nsub_of_phase(const AttTcArgs &a, int p) {
     return (len + SB - 1) / SB;
 }
 
-__global__ void __launch_bounds__(NT_MAIN, 1)
+// Finalise sub-block sb of phase p with one warp: accumulators -> O (bf16),
+// slot zeroed.  Rows are independent, so 8 are in flight per step.
+__device__ void finalize_sub(const AttTcArgs &a, __nv_bfloat16 *__restrict__ O, int p, int sb, bool has_data,
+                             int lane) {
+    const int bj = p / a.ntb, tbi = p % a.ntb;
+    const int b = bj / a.Hkv, j = bj % a.Hkv;
+    const int t_begin = tbi * a.tb + sb * SB;
+    const int t_end = min(t_begin + SB, min((tbi + 1) * a.tb, a.Tq));
+    const int nrows = (t_end - t_begin) * a.G;
+    float *__restrict__ slot = a.ringbuf + ((size_t)(p % a.ring) * a.tb + (t_begin - tbi * a.tb)) * a.G * D;
+    __nv_bfloat16 *__restrict__ out = O + (((size_t)b * a.Tq + t_begin) * a.H + (size_t)j * a.G) * D;
+    for (int r0 = 0; r0 < nrows; r0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (has_data && r0 + u < nrows) v[u] = __ldcg(reinterpret_cast<const float4 *>(slot + (size_t)(r0 + u) * D) + lane);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int rr = r0 + u;
+            if (rr >= nrows) break;
+            if (has_data) __stcg(reinterpret_cast<float4 *>(slot + (size_t)rr * D) + lane, make_float4(0.f, 0.f, 0.f, 0.f));
+            const int tt = rr / a.G, gg = rr % a.G;
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y), hi = __floats2bfloat162_rn(v[u].z, v[u].w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t *>(&lo);
+            pk.y = *reinterpret_cast<uint32_t *>(&hi);
+            reinterpret_cast<uint2 *>(out + ((size_t)tt * a.H + gg) * D)[lane] = pk;
+        }
+    }
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(&a.phase_done[p], 1);
+}
+
+// Apply this warp's batched sub-block increments (after one fence) and
+// finalise the sub-blocks they complete.
+__device__ void flush_pending(const AttTcArgs &a, __nv_bfloat16 *O, int *pend, int &npend, int lane) {
+    if (npend == 0) return;
+    __threadfence();
+    __syncwarp();
+    for (int q = 0; q < npend; ++q) {
+        const int e = pend[q * 32 + lane];
+        bool fin = false;
+        if (e >= 0) {
+            const int old = atomicAdd(&a.sub_done[e], 1);
+            fin = (old + 1 == a.sub_need[e]);
+        }
+        unsigned fm = __ballot_sync(FULL, fin);
+        if (fm) __threadfence();
+        while (fm) {
+            const int src = __ffs(fm) - 1;
+            fm &= fm - 1;
+            const int ev = __shfl_sync(FULL, e, src);
+            finalize_sub(a, O, ev / a.nsub, ev % a.nsub, true, lane);
+        }
+    }
+    npend = 0;
+}
+
+// Bounded wait that first flushes the batched increments if it would block.
+__device__ __forceinline__ bool ep_wait(uint64_t *bar, uint32_t parity, const AttTcArgs &a, __nv_bfloat16 *O,
+                                        int *pend, int &npend, int lane, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    flush_pending(a, O, pend, npend, lane);
+    return mbar_wait(bar, parity, abort, a.status);
+}
+
+constexpr int NT_ATT = 416;   // warps 0-3 producers, 4-7 and 8-11 epilogue groups, 12 MMA
+
+__global__ void __launch_bounds__(NT_ATT, 1)
     att_main_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __nv_bfloat16 *__restrict__ Q, __nv_bfloat16 *__restrict__ O, AttTcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.S;
-    const int kv_bytes = S * 128;                         // one 64-column box of S rows
-    uint8_t *sQ = base;                                   // 2 x 32 KB
-    uint8_t *sKV = sQ + 2 * 32768;                        // nskv x (K: 2 boxes, V: 2 boxes)
-    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;    // S/64 x 16 KB
-    float *stg = reinterpret_cast<float *>(sP + (size_t)(S / 64) * 16384);   // 4 warps x 32 x PITCH
-    AttBars *bar = reinterpret_cast<AttBars *>(stg + 4 * 32 * PITCH);
+    const int kv_bytes = S * 128;                          // one 64-column box of S rows
+    const int p_bytes = (S / 64) * 16384;                  // P tile of one group
+    uint8_t *sQ = base;                                    // nsq x 32 KB
+    uint8_t *sKV = sQ + (size_t)a.nsq * 32768;             // nskv x (K: 2 boxes, V: 2 boxes)
+    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 groups x p_bytes
+    float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 warps x 32 x PITCH
+    int *pend_all = reinterpret_cast<int *>(stg + 8 * 32 * PITCH);     // 8 warps x NDEF x 32
+    AttBars *bar = reinterpret_cast<AttBars *>(pend_all + 8 * NDEF * 32);
     volatile int *abort = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -298,18 +350,18 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
             mbar_init(&bar->q_empty[s], 1);
             mbar_init(&bar->kv_full[s], 1);
             mbar_init(&bar->kv_empty[s], 1);
+            mbar_init(&bar->s_full[s], 1);
+            mbar_init(&bar->p_full[s], 4);
+            mbar_init(&bar->o_full[s], 1);
+            mbar_init(&bar->o_empty[s], 4);
         }
-        mbar_init(&bar->s_full, 1);
-        mbar_init(&bar->p_full, 4);
-        mbar_init(&bar->o_full, 1);
-        mbar_init(&bar->o_empty, 4);
         mbar_init(&bar->done, 1);
         bar->abort = 0;
         bar->ntiles = a.btile[a.nbucket];
         fence_mbar_init();
     }
-    if (warp == 4) {
-        tmem_alloc(&bar->tmem_base, 256);
+    if (warp == 12) {
+        tmem_alloc(&bar->tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -326,7 +378,7 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
         bool ok = true;
         for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
             const TileInfo T = tile_info(a, tau);
-            const int sq = i & 1, iq = i >> 1;
+            const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
             if (warp == 0 && lane == 0) {
                 const int skv = i % a.nskv, ikv = i / a.nskv;
@@ -358,16 +410,17 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
             // wind down: the K/V loads issued have all landed
             for (int s = 0; s < a.nskv && s < i; ++s) mbar_drain(&bar->kv_full[s], ((i - 1 - s) / a.nskv) & 1);
         }
-    } else if (warp == 4) {
+    } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t s_tmem = tmem, o_tmem = tmem + 128;
             const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
             int i = 0;
             bool ok = true;
             for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
-                const int sq = i & 1, iq = i >> 1, skv = i % a.nskv, ikv = i / a.nskv;
+                const int sq = i % a.nsq, iq = i / a.nsq, skv = i % a.nskv, ikv = i / a.nskv;
+                const int gsel = i & 1, k = i >> 1;
+                const uint32_t s_tmem = tmem + gsel * 256, o_tmem = s_tmem + 128;
                 if (!(ok = mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status))) break;
                 if (!(ok = mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status))) break;
                 tc_fence_after();
@@ -375,54 +428,58 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
                 const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 4 * kv_bytes);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-                    const uint32_t a_addr = qa + (kk >> 2) * 16384 + off;
-                    const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + off;
+                    const uint32_t a_addr = qa + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + (kk & 3) * 32;
                     umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
                 }
-                umma_commit(&bar->s_full);
+                umma_commit(&bar->s_full[gsel]);
                 umma_commit(&bar->q_empty[sq]);
-                if (!(ok = mbar_wait(&bar->p_full, i & 1, abort, a.status))) break;
-                if (i > 0 && !(ok = mbar_wait(&bar->o_empty, (i - 1) & 1, abort, a.status))) break;
+                if (!(ok = mbar_wait(&bar->p_full[gsel], k & 1, abort, a.status))) break;
+                if (k > 0 && !(ok = mbar_wait(&bar->o_empty[gsel], (k - 1) & 1, abort, a.status))) break;
                 tc_fence_after();
-                const uint32_t pa = smem_u32(sP);
+                const uint32_t pa = smem_u32(sP + gsel * p_bytes);
                 const uint32_t vb = kb0 + 2 * kv_bytes;
                 for (int kk = 0; kk < S / 16; ++kk) {
-                    // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it
+                    // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
+                    // V: MN-major, keys kk*16..+15 are two 8-row groups starting (kk*16)*128 B
+                    // into each 64-dim box; the two boxes are kv_bytes apart.
                     const uint32_t a_addr = pa + (kk >> 2) * 16384 + (kk & 3) * 32;
-                    // V: MN-major, keys kk*16..+15 = two 8-row groups starting at (kk*16)*128 B;
-                    // the two 64-dim halves are kv_bytes apart
                     const uint32_t b_addr = vb + kk * 16 * 128;
                     umma_bf16(o_tmem, desc_kmajor_sw128(a_addr), desc_mnmajor_sw128(b_addr, kv_bytes, 1024), idesc_o,
                               kk != 0);
                 }
-                umma_commit(&bar->o_full);
+                umma_commit(&bar->o_full[gsel]);
                 umma_commit(&bar->kv_empty[skv]);
             }
             umma_commit(&bar->done);
             mbar_drain(&bar->done, 0);
         }
-    } else if (warp >= 8) {
-        // ------------------------------------------------------------ epilogue: thread = tile row
-        const int ew = warp - 8;
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue groups: thread = tile row
+        const int grp = (warp - 4) >> 2;       // tiles i with i % 2 == grp
+        const int ew = (warp - 4) & 3;         // TMEM lane quadrant
         const int r = ew * 32 + lane;
         const int m = r / a.G, g = r % a.G;
-        const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
-        float *wst = stg + ew * 32 * PITCH;
+        const uint32_t lane_base = tmem + grp * 256 + ((uint32_t)(ew * 32) << 16);
+        float *wst = stg + (warp - 4) * 32 * PITCH;
+        int *pend = pend_all + (warp - 4) * NDEF * 32;
+        uint8_t *myP = sP + grp * p_bytes;
+        int npend = 0;
         // sub-blocks nobody contributes to: write their zeros right away
         {
             const int total = a.nphase * a.nsub;
-            for (int e = (blockIdx.x * 4 + ew); e < total; e += gridDim.x * 4) {
+            for (int e = (blockIdx.x * 8 + (warp - 4)); e < total; e += gridDim.x * 8) {
                 const int p = e / a.nsub, sb = e % a.nsub;
                 if (sb < nsub_of_phase(a, p) && a.sub_need[e] == 0) finalize_sub(a, O, p, sb, false, lane);
             }
         }
-        int i = 0;
+        int checked = -1;   // ring phases up to this one are known to be finalised
         bool ok = true;
-        for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+        int i = grp, k = 0;
+        for (int tau = blockIdx.x + grp * gridDim.x; tau < ntiles && ok; tau += 2 * gridDim.x, i += 2, ++k) {
             const TileInfo T = tile_info(a, tau);
             const bool valid = m < T.n;
-            int t = 0, slot = 0;
+            int t = -1, slot = 0;
             float w = 0.f;
             if (valid) {
                 const int pr = a.pairs[T.start + m];
@@ -431,7 +488,7 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
                 w = a.w8[(((long long)T.b * a.Tq + t) * a.Hkv + T.j) * a.kmax + slot];
             }
             // chunk softmax: S row -> P row (bf16, swizzled), l
-            if (!(ok = mbar_wait(&bar->s_full, i & 1, abort, a.status))) break;
+            if (!(ok = ep_wait(&bar->s_full[grp], k & 1, a, O, pend, npend, lane, abort))) break;
             tc_fence_after();
             float l = 0.f;
             {
@@ -457,8 +514,7 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
                         l += hf.x + hf.y;
                         pk[e] = *reinterpret_cast<uint32_t *>(&h);
                     }
-                    // 32 keys = 4 16-B chunks of the 128-B row of k-block q/2
-                    uint8_t *prow = sP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+                    uint8_t *prow = myP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         const int cx = (q & 1) * 4 + x;
@@ -470,31 +526,44 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->p_full);
-            // ring slot of this phase must be free (phase p - ring finalised)
-            if (T.p >= a.ring) {
-                if (lane == 0) {
-                    const int need = nsub_of_phase(a, T.p - a.ring);
-                    volatile int *pd = a.phase_done + (T.p - a.ring);
-                    const uint64_t t0 = globaltimer_ns();
-                    while (*pd < need) {
-                        if (*abort) break;
-                        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-                            *abort = 1;
-                            atomicOr(a.status, DEV_TIMEOUT);
-                            break;
+            if (lane == 0) mbar_arrive(&bar->p_full[grp]);
+            // the ring slot of this phase must be free: phase p - ring finalised
+            if (T.p >= a.ring && T.p - a.ring > checked) {
+                const int need = nsub_of_phase(a, T.p - a.ring);
+                const int *pd = a.phase_done + (T.p - a.ring);
+                if (ld_acquire(pd) < need) {
+                    flush_pending(a, O, pend, npend, lane);
+                    if (lane == 0) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire(pd) < need) {
+                            if (*abort) break;
+                            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                                *abort = 1;
+                                atomicOr(a.status, DEV_TIMEOUT);
+                                break;
+                            }
                         }
                     }
-                    __threadfence();
+                    __syncwarp();
                 }
-                __syncwarp();
+                checked = T.p - a.ring;
             }
-            // O row -> scaled fp32 contributions, reduced into the ring slot 32 columns at a time
-            if (!(ok = mbar_wait(&bar->o_full, i & 1, abort, a.status))) break;
+            // O row -> (w/l) * O, reduced into the ring slot 32 columns at a time
+            if (!(ok = ep_wait(&bar->o_full[grp], k & 1, a, O, pend, npend, lane, abort))) break;
             tc_fence_after();
             const float f = valid ? w / l : 0.f;
-            float *acc_slot = a.ringbuf + (size_t)(T.p % a.ring) * a.tb * a.G * D;
             const int tloc_base = (T.p % a.ntb) * a.tb;
+            float *acc_slot = a.ringbuf + (size_t)(T.p % a.ring) * a.tb * a.G * D;
+            // destination row of each staging row this lane reduces (rows rr*4 + lane/8)
+            float *dstrow[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                const int lr = rr * 4 + (lane >> 3);
+                const int tt = __shfl_sync(FULL, t, lr);
+                const int R = ew * 32 + lr;
+                dstrow[rr] = tt >= 0 ? acc_slot + ((size_t)(tt - tloc_base) * a.G + (R % a.G)) * D + 4 * (lane & 7)
+                                     : nullptr;
+            }
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t orr[32];
                 tmem_ld32(lane_base + 128 + q * 32, orr);
@@ -502,7 +571,7 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
                 if (q == D / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar->o_empty);
+                    if (lane == 0) mbar_arrive(&bar->o_empty[grp]);
                 }
                 float *mine = wst + lane * PITCH;
 #pragma unroll
@@ -511,47 +580,28 @@ __global__ void __launch_bounds__(NT_MAIN, 1)
                         make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
                                     __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
                 __syncwarp();
-                // lane -> (row rr*4 + lane/8, 4 floats at column 4*(lane%8))
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                    const int lr = rr * 4 + (lane >> 3);   // row within this warp
-                    const int R = ew * 32 + lr;
-                    const int mm = R / a.G, gg = R % a.G;
-                    const int pr = mm < T.n ? a.pairs[T.start + mm] : -1;
-                    if (pr >= 0) {
-                        const int tt = pr >> 5;
-                        float *dst = acc_slot + ((size_t)(tt - tloc_base) * a.G + gg) * D + q * 32 + 4 * (lane & 7);
+                    if (dstrow[rr]) {
+                        const int lr = rr * 4 + (lane >> 3);
                         const float4 v = *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7));
-                        atomicAdd(reinterpret_cast<float4 *>(dst), v);
+                        atomicAdd(reinterpret_cast<float4 *>(dstrow[rr] + q * 32), v);
                     }
                 }
                 __syncwarp();
             }
-            // count the pairs of this warp's tokens; finalise completed sub-blocks
-            __threadfence();
-            __syncwarp();
-            bool fin = false;
-            int fsb = 0;
-            if (valid && g == 0) {
-                fsb = (t - tloc_base) / SB;
-                const int old = atomicAdd(&a.sub_done[T.p * a.nsub + fsb], 1);
-                fin = (old + 1 == a.sub_need[T.p * a.nsub + fsb]);
-                if (fin) __threadfence();
-            }
-            unsigned fm = __ballot_sync(FULL, fin);
-            while (fm) {
-                const int src = __ffs(fm) - 1;
-                fm &= fm - 1;
-                const int sbv = __shfl_sync(FULL, fsb, src);
-                finalize_sub(a, O, T.p, sbv, true, lane);
-            }
+            // one pending increment per (token, slot) pair of this warp: its head-0 row's lane
+            pend[npend * 32 + lane] = (valid && g == 0) ? T.p * a.nsub + (t - tloc_base) / SB : -1;
+            ++npend;
+            if (npend == NDEF) flush_pending(a, O, pend, npend, lane);
         }
+        flush_pending(a, O, pend, npend, lane);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 12) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -609,7 +659,8 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.ring = L.ring;
     a.nphase = L.nphase;
     a.nbucket = L.nbucket;
-    a.nsq = 2;
+    // S=64: double-buffered Q and K/V (210 KB of smem); S=128: single (210 KB)
+    a.nsq = p.S <= 64 ? 2 : 1;
     a.nskv = p.S <= 64 ? 2 : 1;
     a.q_pos0 = p.q_pos0;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
@@ -649,16 +700,15 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     const uint32_t box[3] = {64, 1, (uint32_t)p.S};
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
-    const int nskv = a.nskv;
-    const size_t smem = 1024 + 2 * 32768 + (size_t)nskv * 4 * p.S * 128 + (size_t)(p.S / 64) * 16384 +
-                        4 * 32 * PITCH * sizeof(float) + sizeof(AttBars);
+    const size_t smem = 1024 + (size_t)a.nsq * 32768 + (size_t)a.nskv * 4 * p.S * 128 + 2 * (size_t)(p.S / 64) * 16384 +
+                        8 * 32 * PITCH * sizeof(float) + 8 * NDEF * 32 * sizeof(int) + sizeof(AttBars);
     if ((e = cudaFuncSetAttribute(att_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
         return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    att_main_kernel<<<sms, NT_MAIN, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
+    att_main_kernel<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
     return cudaGetLastError();
 }
 
