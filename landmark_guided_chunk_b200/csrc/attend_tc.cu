@@ -12,22 +12,22 @@
 //     S  = Q_tile . K_c^T / sqrt(d)        tcgen05, M128 x N=S x K=d, TMEM
 //     P  = exp(S - rowmax), l = sum P      epilogue warps, P -> smem (bf16)
 //     O  = P . V_c                          tcgen05, M128 x N=d x K=S, TMEM
-//     O_acc[t][h] += (w_slot / l) * O       fp32 vector reductions
+//     O_acc[t][h] += (w_slot / l) * O       fp32 vector reductions (red.v4)
 // Since w is known before the attention, the cross-chunk fusion is linear and
 // needs no rescaling.
 //
 // Accumulators.  The pairs are grouped into phases of TB tokens of one (b, kv
-// head).  Tiles are ordered phase-major, so the active accumulators form a
-// ring of R phase slots that stays resident in L2.  A sub-block of SB tokens
-// is finalised (fp32 -> bf16 into O, slot zeroed) by whichever warp completes
-// its last expected contribution (counter per sub-block).  A tile of phase p
-// waits until phase p-R has been finalised before it reduces into the shared
-// slot.  Persistent CTAs take tiles in increasing order, so that wait always
-// ends.  It is bounded anyway.
+// head), and the tiles are ordered phase-major.  The phases are processed in
+// batches of NB, one kernel launch per batch.  A batch reduces into NB
+// accumulator slots of a ring of 2*NB, which stays resident in L2.  Launch
+// beta first finalises batch beta-1 (its slots -> bf16 O, slots zeroed).  Every
+// warp of every CTA takes a share of that, and then the CTA moves on to the
+// tiles of batch beta, whose slots differ.  The kernel boundary is the only
+// synchronisation, so no CTA ever waits for another.
 //
-// Helper kernels (before the main kernel): count pairs per (phase, chunk)
-// bucket and compute the fusion weights; two-level exclusive scan of pair
-// and tile counts; tile list; scatter of the pairs into their buckets.
+// Helper kernels (before the batches): count pairs per (phase, chunk) bucket
+// and compute the fusion weights; two-level exclusive scan of pair and tile
+// counts; tile list; scatter of the pairs into their buckets.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -39,13 +39,17 @@ using namespace sm100;
 
 constexpr int D = 128;           // head dim of this kernel
 constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
-constexpr int SB = 32;           // tokens per finalisation sub-block
 constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
+constexpr int TB = 4096;         // tokens per phase
+constexpr int NB = 2;            // phases per batch (= per launch)
+constexpr int NT_ATT = 416;      // warps 0-3 producers, 4-7 and 8-11 epilogue groups, 12 MMA
 
 struct AttTcArgs {
     int B, Tq, Tkv, H, Hkv, G, S, C, kmax, tok;
-    int tb, ntb, nsub, ring, nphase, nbucket, nsq, nskv;
+    int ntb, nphase, nbucket, nsq, nskv;
+    int batch;                   // batch processed by this launch (== nbatch: finalise only)
+    int nbatch;
     long long q_pos0;
     float scale_log2;            // log2(e) / sqrt(d)
     const int32_t *idx;
@@ -57,8 +61,7 @@ struct AttTcArgs {
     int32_t *blk;                // [2 * nblk] first-level block totals
     int32_t *pairs;              // [rows * kmax]  (t << 5) | slot
     int2 *tiles;                 // (bucket, first pair)
-    int32_t *sub_need, *sub_done, *phase_done;
-    float *ringbuf;              // [ring][tb][G][D]
+    float *ringbuf;              // [2*NB][TB][G][D]
     uint32_t *status;
 };
 
@@ -68,12 +71,18 @@ __device__ __forceinline__ int ncand_of(const AttTcArgs &a, int t) {
 }
 
 __device__ __forceinline__ int phase_of(const AttTcArgs &a, int b, int j, int t) {
-    return (b * a.Hkv + j) * a.ntb + t / a.tb;
+    return (b * a.Hkv + j) * a.ntb + t / TB;
+}
+
+// ring slot of phase p
+__device__ __forceinline__ float *slot_of(const AttTcArgs &a, int p) {
+    const int s = ((p / NB) & 1) * NB + (p % NB);
+    return a.ringbuf + (size_t)s * TB * a.G * D;
 }
 
 // ---------------------------------------------------------------------------- helper kernels
 
-// One thread per selection row: fusion weights, bucket counts, sub-block needs.
+// One thread per selection row: fusion weights and bucket counts.
 __global__ void att_count_kernel(AttTcArgs a) {
     const long long row = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long rows = (long long)a.B * a.Tq * a.Hkv;
@@ -94,7 +103,6 @@ __global__ void att_count_kernel(AttTcArgs a) {
     for (int i = 0; i < ke; ++i) m = fmaxf(m, rs[i]);
     float z = 0.f;
     for (int i = 0; i < ke; ++i) z += expf(rs[i] - m);
-    int used = 0;
     for (int i = 0; i < ke; ++i) {
         a.w8[row * a.kmax + i] = expf(rs[i] - m) / z;
         const int c = ri[i];
@@ -103,9 +111,7 @@ __global__ void att_count_kernel(AttTcArgs a) {
             continue;
         }
         atomicAdd(&a.bcount[(long long)p * a.C + c], 1);
-        ++used;
     }
-    if (used) atomicAdd(&a.sub_need[p * a.nsub + (t % a.tb) / SB], used);
 }
 
 // First level of the scan: per block of SCAN_BLK buckets, local exclusive
@@ -211,14 +217,12 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
 
 // ---------------------------------------------------------------------------- main kernel
 
-constexpr int NDEF = 8;   // sub-block counter increments a warp batches behind one fence
-
 struct __align__(8) AttBars {
     uint64_t q_full[2], q_empty[2], kv_full[2], kv_empty[2];
     uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], done;
     uint32_t tmem_base;
     int abort;
-    int ntiles;
+    int tile_lo, tile_hi;
 };
 
 struct TileInfo {
@@ -244,88 +248,45 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
+// fp32 vector reduction into global memory with no value returned
+__device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
 }
 
-__device__ __forceinline__ int nsub_of_phase(const AttTcArgs &a, int p) {
-    const int tbi = p % a.ntb;
-    const int len = min(a.tb, a.Tq - tbi * a.tb);
-    return (len + SB - 1) / SB;
-}
-
-// Finalise sub-block sb of phase p with one warp: accumulators -> O (bf16),
-// slot zeroed.  Rows are independent, so 8 are in flight per step.
-__device__ void finalize_sub(const AttTcArgs &a, __nv_bfloat16 *__restrict__ O, int p, int sb, bool has_data,
-                             int lane) {
-    const int bj = p / a.ntb, tbi = p % a.ntb;
-    const int b = bj / a.Hkv, j = bj % a.Hkv;
-    const int t_begin = tbi * a.tb + sb * SB;
-    const int t_end = min(t_begin + SB, min((tbi + 1) * a.tb, a.Tq));
-    const int nrows = (t_end - t_begin) * a.G;
-    float *__restrict__ slot = a.ringbuf + ((size_t)(p % a.ring) * a.tb + (t_begin - tbi * a.tb)) * a.G * D;
-    __nv_bfloat16 *__restrict__ out = O + (((size_t)b * a.Tq + t_begin) * a.H + (size_t)j * a.G) * D;
-    for (int r0 = 0; r0 < nrows; r0 += 8) {
+// Rows (token, head) of the phases in batch `bt`: accumulators -> bf16 O,
+// accumulators zeroed.  Warps of the whole grid take groups of 8 consecutive
+// rows (8 loads in flight per lane).
+__device__ void finalize_batch(const AttTcArgs &a, __nv_bfloat16 *__restrict__ O, int bt, int gwarp, int nwarps,
+                               int lane) {
+    const int p0 = bt * NB, p1 = min(a.nphase, p0 + NB);
+    const int rows_per_phase = TB * a.G;   // a multiple of 8
+    const long long ngroups = (long long)(p1 - p0) * rows_per_phase / 8;
+    for (long long gi = gwarp; gi < ngroups; gi += nwarps) {
+        const long long e0 = gi * 8;
+        const int p = p0 + (int)(e0 / rows_per_phase);
+        const int rr0 = (int)(e0 % rows_per_phase);
+        const int bj = p / a.ntb, tbi = p % a.ntb;
+        const int b = bj / a.Hkv, j = bj % a.Hkv;
+        float4 *acc = reinterpret_cast<float4 *>(slot_of(a, p) + (size_t)rr0 * D) + lane;
         float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (has_data && r0 + u < nrows) v[u] = __ldcg(reinterpret_cast<const float4 *>(slot + (size_t)(r0 + u) * D) + lane);
-        }
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(acc + u * (D / 4));
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int rr = r0 + u;
-            if (rr >= nrows) break;
-            if (has_data) __stcg(reinterpret_cast<float4 *>(slot + (size_t)rr * D) + lane, make_float4(0.f, 0.f, 0.f, 0.f));
-            const int tt = rr / a.G, gg = rr % a.G;
-            __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y), hi = __floats2bfloat162_rn(v[u].z, v[u].w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t *>(&lo);
-            pk.y = *reinterpret_cast<uint32_t *>(&hi);
-            reinterpret_cast<uint2 *>(out + ((size_t)tt * a.H + gg) * D)[lane] = pk;
+            const int rr = rr0 + u;
+            const int t = tbi * TB + rr / a.G, g = rr % a.G;
+            __stcg(acc + u * (D / 4), make_float4(0.f, 0.f, 0.f, 0.f));
+            if (t < a.Tq) {
+                __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y), hi = __floats2bfloat162_rn(v[u].z, v[u].w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t *>(&lo);
+                pk.y = *reinterpret_cast<uint32_t *>(&hi);
+                reinterpret_cast<uint2 *>(O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + g) * D)[lane] = pk;
+            }
         }
     }
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(&a.phase_done[p], 1);
 }
-
-// Apply this warp's batched sub-block increments (after one fence) and
-// finalise the sub-blocks they complete.
-__device__ void flush_pending(const AttTcArgs &a, __nv_bfloat16 *O, int *pend, int &npend, int lane) {
-    if (npend == 0) return;
-    __threadfence();
-    __syncwarp();
-    for (int q = 0; q < npend; ++q) {
-        const int e = pend[q * 32 + lane];
-        bool fin = false;
-        if (e >= 0) {
-            const int old = atomicAdd(&a.sub_done[e], 1);
-            fin = (old + 1 == a.sub_need[e]);
-        }
-        unsigned fm = __ballot_sync(FULL, fin);
-        if (fm) __threadfence();
-        while (fm) {
-            const int src = __ffs(fm) - 1;
-            fm &= fm - 1;
-            const int ev = __shfl_sync(FULL, e, src);
-            finalize_sub(a, O, ev / a.nsub, ev % a.nsub, true, lane);
-        }
-    }
-    npend = 0;
-}
-
-// Bounded wait that first flushes the batched increments if it would block.
-__device__ __forceinline__ bool ep_wait(uint64_t *bar, uint32_t parity, const AttTcArgs &a, __nv_bfloat16 *O,
-                                        int *pend, int &npend, int lane, volatile int *abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    flush_pending(a, O, pend, npend, lane);
-    return mbar_wait(bar, parity, abort, a.status);
-}
-
-constexpr int NT_ATT = 416;   // warps 0-3 producers, 4-7 and 8-11 epilogue groups, 12 MMA
 
 __global__ void __launch_bounds__(NT_ATT, 1)
     att_main_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -339,11 +300,15 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     uint8_t *sKV = sQ + (size_t)a.nsq * 32768;             // nskv x (K: 2 boxes, V: 2 boxes)
     uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 groups x p_bytes
     float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 warps x 32 x PITCH
-    int *pend_all = reinterpret_cast<int *>(stg + 8 * 32 * PITCH);     // 8 warps x NDEF x 32
-    AttBars *bar = reinterpret_cast<AttBars *>(pend_all + 8 * NDEF * 32);
+    AttBars *bar = reinterpret_cast<AttBars *>(stg + 8 * 32 * PITCH);
     volatile int *abort = &bar->abort;
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // finalise the previous batch (its slots are not touched by this batch's tiles)
+    if (a.batch > 0)
+        finalize_batch(a, O, a.batch - 1, blockIdx.x * (NT_ATT / 32) + warp, gridDim.x * (NT_ATT / 32), lane);
+    if (a.batch >= a.nbatch) return;
+
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar->q_full[s], 128);
@@ -357,7 +322,9 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         }
         mbar_init(&bar->done, 1);
         bar->abort = 0;
-        bar->ntiles = a.btile[a.nbucket];
+        const int p0 = a.batch * NB, p1 = min(a.nphase, p0 + NB);
+        bar->tile_lo = a.btile[p0 * a.C];
+        bar->tile_hi = a.btile[p1 * a.C];
         fence_mbar_init();
     }
     if (warp == 12) {
@@ -368,7 +335,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
-    const int ntiles = bar->ntiles;
+    const int tile_lo = bar->tile_lo, tile_hi = bar->tile_hi;
 
     if (warp < 4) {
         // ------------------------------------------------------------ producers: Q gather (thread = row), K/V TMA
@@ -376,7 +343,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         const int m = r / a.G, g = r % a.G;
         int i = 0;
         bool ok = true;
-        for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+        for (int tau = tile_lo + blockIdx.x; tau < tile_hi && ok; tau += gridDim.x, ++i) {
             const TileInfo T = tile_info(a, tau);
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
@@ -417,7 +384,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
             int i = 0;
             bool ok = true;
-            for (int tau = blockIdx.x; tau < ntiles && ok; tau += gridDim.x, ++i) {
+            for (int tau = tile_lo + blockIdx.x; tau < tile_hi && ok; tau += gridDim.x, ++i) {
                 const int sq = i % a.nsq, iq = i / a.nsq, skv = i % a.nskv, ikv = i / a.nskv;
                 const int gsel = i & 1, k = i >> 1;
                 const uint32_t s_tmem = tmem + gsel * 256, o_tmem = s_tmem + 128;
@@ -459,36 +426,24 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         const int grp = (warp - 4) >> 2;       // tiles i with i % 2 == grp
         const int ew = (warp - 4) & 3;         // TMEM lane quadrant
         const int r = ew * 32 + lane;
-        const int m = r / a.G, g = r % a.G;
+        const int m = r / a.G;
         const uint32_t lane_base = tmem + grp * 256 + ((uint32_t)(ew * 32) << 16);
         float *wst = stg + (warp - 4) * 32 * PITCH;
-        int *pend = pend_all + (warp - 4) * NDEF * 32;
         uint8_t *myP = sP + grp * p_bytes;
-        int npend = 0;
-        // sub-blocks nobody contributes to: write their zeros right away
-        {
-            const int total = a.nphase * a.nsub;
-            for (int e = (blockIdx.x * 8 + (warp - 4)); e < total; e += gridDim.x * 8) {
-                const int p = e / a.nsub, sb = e % a.nsub;
-                if (sb < nsub_of_phase(a, p) && a.sub_need[e] == 0) finalize_sub(a, O, p, sb, false, lane);
-            }
-        }
-        int checked = -1;   // ring phases up to this one are known to be finalised
         bool ok = true;
-        int i = grp, k = 0;
-        for (int tau = blockIdx.x + grp * gridDim.x; tau < ntiles && ok; tau += 2 * gridDim.x, i += 2, ++k) {
+        int k = 0;
+        for (int tau = tile_lo + blockIdx.x + grp * gridDim.x; tau < tile_hi && ok; tau += 2 * gridDim.x, ++k) {
             const TileInfo T = tile_info(a, tau);
             const bool valid = m < T.n;
-            int t = -1, slot = 0;
+            int t = -1;
             float w = 0.f;
             if (valid) {
                 const int pr = a.pairs[T.start + m];
                 t = pr >> 5;
-                slot = pr & 31;
-                w = a.w8[(((long long)T.b * a.Tq + t) * a.Hkv + T.j) * a.kmax + slot];
+                w = a.w8[(((long long)T.b * a.Tq + t) * a.Hkv + T.j) * a.kmax + (pr & 31)];
             }
             // chunk softmax: S row -> P row (bf16, swizzled), l
-            if (!(ok = ep_wait(&bar->s_full[grp], k & 1, a, O, pend, npend, lane, abort))) break;
+            if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
             float l = 0.f;
             {
@@ -527,33 +482,12 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->p_full[grp]);
-            // the ring slot of this phase must be free: phase p - ring finalised
-            if (T.p >= a.ring && T.p - a.ring > checked) {
-                const int need = nsub_of_phase(a, T.p - a.ring);
-                const int *pd = a.phase_done + (T.p - a.ring);
-                if (ld_acquire(pd) < need) {
-                    flush_pending(a, O, pend, npend, lane);
-                    if (lane == 0) {
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire(pd) < need) {
-                            if (*abort) break;
-                            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-                                *abort = 1;
-                                atomicOr(a.status, DEV_TIMEOUT);
-                                break;
-                            }
-                        }
-                    }
-                    __syncwarp();
-                }
-                checked = T.p - a.ring;
-            }
-            // O row -> (w/l) * O, reduced into the ring slot 32 columns at a time
-            if (!(ok = ep_wait(&bar->o_full[grp], k & 1, a, O, pend, npend, lane, abort))) break;
+            // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
+            if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
             const float f = valid ? w / l : 0.f;
-            const int tloc_base = (T.p % a.ntb) * a.tb;
-            float *acc_slot = a.ringbuf + (size_t)(T.p % a.ring) * a.tb * a.G * D;
+            const int tloc_base = (T.p % a.ntb) * TB;
+            float *acc_slot = slot_of(a, T.p);
             // destination row of each staging row this lane reduces (rows rr*4 + lane/8)
             float *dstrow[8];
 #pragma unroll
@@ -584,18 +518,12 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 for (int rr = 0; rr < 8; ++rr) {
                     if (dstrow[rr]) {
                         const int lr = rr * 4 + (lane >> 3);
-                        const float4 v = *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7));
-                        atomicAdd(reinterpret_cast<float4 *>(dstrow[rr] + q * 32), v);
+                        red_add_v4(dstrow[rr] + q * 32, *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
                     }
                 }
                 __syncwarp();
             }
-            // one pending increment per (token, slot) pair of this warp: its head-0 row's lane
-            pend[npend * 32 + lane] = (valid && g == 0) ? T.p * a.nsub + (t - tloc_base) / SB : -1;
-            ++npend;
-            if (npend == NDEF) flush_pending(a, O, pend, npend, lane);
         }
-        flush_pending(a, O, pend, npend, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -609,34 +537,36 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 
 // ---------------------------------------------------------------------------- host side
 
-static int att_tb(const Prob &) { return 4096; }
-
 bool attend_tc_supported(const Prob &p) {
     if (!(p.dtype == HSA_BF16 && p.d == D && (p.S == 64 || p.S == 128) && p.G <= 16 && (32 % p.G) == 0 &&
           p.C >= 1 && p.Tq >= 1 && p.kmax <= 32 && p.Tq < (1 << 26)))
         return false;
     // the second scan level is one block of 1024 threads over SCAN_BLK-bucket blocks
-    const long long ntb = (p.Tq + att_tb(p) - 1) / att_tb(p);
+    const long long ntb = (p.Tq + TB - 1) / TB;
     const long long nbucket = (long long)p.B * p.Hkv * ntb * p.C;
     return nbucket <= 1024LL * SCAN_BLK && (long long)p.rows * p.kmax < (1LL << 31);
 }
-static int att_ring() { return 4; }
 
 AttTcLayout attend_tc_layout(const Prob &p) {
     AttTcLayout L{};
-    L.tb = att_tb(p);
-    L.ntb = (p.Tq + L.tb - 1) / L.tb;
-    L.nsub = L.tb / SB;
+    L.tb = TB;
+    L.ntb = (p.Tq + TB - 1) / TB;
+    L.nsub = 0;
     L.nphase = p.B * p.Hkv * L.ntb;
     L.nbucket = L.nphase * p.C;
     L.nblk = (L.nbucket + SCAN_BLK - 1) / SCAN_BLK;
     L.tok = MROWS / p.G;
-    L.ring = att_ring();
+    L.ring = 2 * NB;
     const size_t pairs = (size_t)p.rows * p.kmax;
     L.max_tiles = pairs / L.tok + (size_t)L.nbucket + 1;
-    L.counter_ints = 2 * (size_t)L.nbucket + 2 * (size_t)L.nphase * L.nsub + L.nphase;
-    L.ring_bytes = (size_t)L.ring * L.tb * p.G * D * sizeof(float);
+    L.counter_ints = 2 * (size_t)L.nbucket;
+    L.ring_bytes = (size_t)L.ring * TB * p.G * D * sizeof(float);
     return L;
+}
+
+int attend_tc_launches(const AttTcLayout &L) {
+    const int nbatch = (L.nphase + NB - 1) / NB;
+    return 5 + nbatch + 1;   // count, scan1, scan2, tiles, scatter, one per batch, final finalise
 }
 
 cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,
@@ -653,15 +583,13 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.C = p.C;
     a.kmax = p.kmax;
     a.tok = L.tok;
-    a.tb = L.tb;
     a.ntb = L.ntb;
-    a.nsub = L.nsub;
-    a.ring = L.ring;
     a.nphase = L.nphase;
     a.nbucket = L.nbucket;
-    // S=64: double-buffered Q and K/V (210 KB of smem); S=128: single (210 KB)
+    // S=64: double-buffered Q and K/V (~200 KB of smem); S=128: single
     a.nsq = p.S <= 64 ? 2 : 1;
     a.nskv = p.S <= 64 ? 2 : 1;
+    a.nbatch = (L.nphase + NB - 1) / NB;
     a.q_pos0 = p.q_pos0;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
     a.idx = idx;
@@ -670,9 +598,6 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.w8 = bf.w8;
     a.bcount = bf.counters;
     a.bcursor = bf.counters + L.nbucket;
-    a.sub_need = bf.counters + 2 * (size_t)L.nbucket;
-    a.sub_done = a.sub_need + (size_t)L.nphase * L.nsub;
-    a.phase_done = a.sub_done + (size_t)L.nphase * L.nsub;
     a.boff = bf.boff;
     a.btile = bf.btile;
     a.blk = bf.blk;
@@ -681,7 +606,7 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.ringbuf = bf.ring;
     a.status = bf.status;
 
-    // counters and ring slots start at zero on every call
+    // bucket counters and the accumulator ring start at zero on every call
     cudaError_t e = cudaMemsetAsync(bf.counters, 0, L.counter_ints * sizeof(int32_t), st);
     if (e == cudaSuccess) e = cudaMemsetAsync(bf.ring, 0, L.ring_bytes, st);
     if (e != cudaSuccess) return e;
@@ -701,15 +626,19 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
     const size_t smem = 1024 + (size_t)a.nsq * 32768 + (size_t)a.nskv * 4 * p.S * 128 + 2 * (size_t)(p.S / 64) * 16384 +
-                        8 * 32 * PITCH * sizeof(float) + 8 * NDEF * 32 * sizeof(int) + sizeof(AttBars);
+                        8 * 32 * PITCH * sizeof(float) + sizeof(AttBars);
     if ((e = cudaFuncSetAttribute(att_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
         return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    att_main_kernel<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
-    return cudaGetLastError();
+    for (int bt = 0; bt <= a.nbatch; ++bt) {
+        a.batch = bt;
+        att_main_kernel<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace hsa

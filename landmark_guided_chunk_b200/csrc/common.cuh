@@ -186,6 +186,7 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
 
 bool attend_tc_supported(const Prob &p);
 AttTcLayout attend_tc_layout(const Prob &p);
+int attend_tc_launches(const AttTcLayout &L);
 cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,
                              const void *V, const int32_t *idx, const float *score, const int32_t *keff, void *O,
                              cudaStream_t st);

@@ -79,8 +79,8 @@ WsLayout ws_layout(const Prob &p) {
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_attend  ? HSA_PATH_TENSOR
                          : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
-    // tensor path: count, scan (2 levels), tile list, scatter, main kernel
-    w.plan.attend_kernels = rows == 0 ? 0 : (w.tc_attend ? 6 : (w.split_attend ? 2 : 1));
+    // tensor path: count, scan (2 levels), tile list, scatter, one main kernel per phase batch + 1
+    w.plan.attend_kernels = rows == 0 ? 0 : (w.tc_attend ? attend_tc_launches(w.att) : (w.split_attend ? 2 : 1));
     return w;
 }
 
