@@ -343,8 +343,13 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         const int m = r / a.G, g = r % a.G;
         int i = 0;
         bool ok = true;
-        for (int tau = tile_lo + blockIdx.x; tau < tile_hi && ok; tau += gridDim.x, ++i) {
-            const TileInfo T = tile_info(a, tau);
+        int tau = tile_lo + blockIdx.x;
+        TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
+        int pr = (tau < tile_hi && m < T.n) ? a.pairs[T.start + m] : 0;
+        for (; tau < tile_hi && ok; ++i) {
+            // prefetch the next tile while this one is issued
+            const int tau_n = tau + gridDim.x;
+            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
             if (warp == 0 && lane == 0) {
@@ -361,7 +366,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             const bool valid = m < T.n;
             const char *src = reinterpret_cast<const char *>(Q);
             if (valid) {
-                const int t = a.pairs[T.start + m] >> 5;
+                const int t = pr >> 5;
                 src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + g) * D) * 2;
             }
             const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
@@ -371,6 +376,9 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
             }
             cp_async_arrive(&bar->q_full[sq]);
+            pr = (tau_n < tile_hi && m < Tn.n) ? a.pairs[Tn.start + m] : 0;
+            T = Tn;
+            tau = tau_n;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (warp == 0 && lane == 0) {
@@ -379,18 +387,20 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         }
     } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
+        // With two K/V stages QK(i+1) is issued before PV(i), so the two epilogue
+        // groups' softmaxes overlap; with one stage the order is QK(i), PV(i), ...
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
-            int i = 0;
-            bool ok = true;
-            for (int tau = tile_lo + blockIdx.x; tau < tile_hi && ok; tau += gridDim.x, ++i) {
+            const int n_mine = tile_lo + (int)blockIdx.x < tile_hi
+                                   ? (tile_hi - tile_lo - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                                   : 0;
+            auto issue_qk = [&](int i) -> bool {
                 const int sq = i % a.nsq, iq = i / a.nsq, skv = i % a.nskv, ikv = i / a.nskv;
-                const int gsel = i & 1, k = i >> 1;
-                const uint32_t s_tmem = tmem + gsel * 256, o_tmem = s_tmem + 128;
-                if (!(ok = mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status))) break;
-                if (!(ok = mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status))) break;
+                if (!mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status)) return false;
+                if (!mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status)) return false;
                 tc_fence_after();
+                const uint32_t s_tmem = tmem + (i & 1) * 256;
                 const uint32_t qa = smem_u32(sQ + sq * 32768);
                 const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 4 * kv_bytes);
 #pragma unroll
@@ -399,13 +409,21 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                     const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + (kk & 3) * 32;
                     umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
                 }
-                umma_commit(&bar->s_full[gsel]);
+                umma_commit(&bar->s_full[i & 1]);
                 umma_commit(&bar->q_empty[sq]);
+                return true;
+            };
+            const bool early = a.nskv >= 2;
+            bool ok = n_mine > 0 ? issue_qk(0) : true;
+            for (int i = 0; i < n_mine && ok; ++i) {
+                const int skv = i % a.nskv, gsel = i & 1, k = i >> 1;
+                if (early && i + 1 < n_mine && !(ok = issue_qk(i + 1))) break;
                 if (!(ok = mbar_wait(&bar->p_full[gsel], k & 1, abort, a.status))) break;
                 if (k > 0 && !(ok = mbar_wait(&bar->o_empty[gsel], (k - 1) & 1, abort, a.status))) break;
                 tc_fence_after();
+                const uint32_t o_tmem = tmem + gsel * 256 + 128;
                 const uint32_t pa = smem_u32(sP + gsel * p_bytes);
-                const uint32_t vb = kb0 + 2 * kv_bytes;
+                const uint32_t vb = smem_u32(sKV + (size_t)skv * 4 * kv_bytes) + 2 * kv_bytes;
                 for (int kk = 0; kk < S / 16; ++kk) {
                     // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
                     // V: MN-major, keys kk*16..+15 are two 8-row groups starting (kk*16)*128 B
@@ -417,6 +435,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 }
                 umma_commit(&bar->o_full[gsel]);
                 umma_commit(&bar->kv_empty[skv]);
+                if (!early && i + 1 < n_mine && !(ok = issue_qk(i + 1))) break;
             }
             umma_commit(&bar->done);
             mbar_drain(&bar->done, 0);
@@ -432,16 +451,23 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         uint8_t *myP = sP + grp * p_bytes;
         bool ok = true;
         int k = 0;
-        for (int tau = tile_lo + blockIdx.x + grp * gridDim.x; tau < tile_hi && ok; tau += 2 * gridDim.x, ++k) {
-            const TileInfo T = tile_info(a, tau);
-            const bool valid = m < T.n;
-            int t = -1;
-            float w = 0.f;
-            if (valid) {
-                const int pr = a.pairs[T.start + m];
-                t = pr >> 5;
-                w = a.w8[(((long long)T.b * a.Tq + t) * a.Hkv + T.j) * a.kmax + (pr & 31)];
+        auto row_info = [&](const TileInfo &X, int &tt, float &ww) {
+            tt = -1;
+            ww = 0.f;
+            if (m < X.n) {
+                const int pr = a.pairs[X.start + m];
+                tt = pr >> 5;
+                ww = a.w8[(((long long)X.b * a.Tq + tt) * a.Hkv + X.j) * a.kmax + (pr & 31)];
             }
+        };
+        int tau = tile_lo + blockIdx.x + grp * gridDim.x;
+        TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
+        int t;
+        float w;
+        row_info(T, t, w);
+        for (; tau < tile_hi && ok; ++k) {
+            const bool valid = m < T.n;
+            const int tau_n = tau + 2 * gridDim.x;
             // chunk softmax: S row -> P row (bf16, swizzled), l
             if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -482,6 +508,11 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->p_full[grp]);
+            // next tile's descriptor, pair and weight: their latency hides behind this tile's PV and reductions
+            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
+            int t_n;
+            float w_n;
+            row_info(Tn, t_n, w_n);
             // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
             if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -523,6 +554,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 }
                 __syncwarp();
             }
+            T = Tn;
+            t = t_n;
+            w = w_n;
+            tau = tau_n;
         }
     }
     tc_fence_before();
