@@ -289,11 +289,12 @@ cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const
         AttTcBuffers bf;
         bf.w8 = reinterpret_cast<float *>(ws + w.att_w8);
         bf.pairs = reinterpret_cast<int32_t *>(ws + w.att_pairs);
+        bf.pair_w = reinterpret_cast<float *>(ws + w.att_pair_w);
         bf.counters = reinterpret_cast<int32_t *>(ws + w.att_counters);
         bf.boff = reinterpret_cast<int32_t *>(ws + w.att_boff);
         bf.btile = reinterpret_cast<int32_t *>(ws + w.att_btile);
         bf.blk = reinterpret_cast<int32_t *>(ws + w.att_blk);
-        bf.tiles = reinterpret_cast<int2 *>(ws + w.att_tiles);
+        bf.tiles = reinterpret_cast<int4 *>(ws + w.att_tiles);
         bf.ring = reinterpret_cast<float *>(ws + w.att_ring);
         bf.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
         return launch_attend_tc(p, w.att, bf, Q, K, V, idx, score, keff, O, st);

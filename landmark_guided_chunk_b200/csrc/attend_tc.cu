@@ -60,7 +60,8 @@ struct AttTcArgs {
     int32_t *boff, *btile;       // [nbucket + 1]
     int32_t *blk;                // [2 * nblk] first-level block totals
     int32_t *pairs;              // [rows * kmax]  (t << 5) | slot
-    int2 *tiles;                 // (bucket, first pair)
+    float *pair_w;               // [rows * kmax]  fusion weight of each pair
+    int4 *tiles;                 // (phase, chunk, first pair, pairs in tile)
     float *ringbuf;              // [2*NB][TB][G][D]
     uint32_t *status;
 };
@@ -191,7 +192,8 @@ __global__ void att_tiles_kernel(AttTcArgs a) {
     a.boff[u] = op;
     a.btile[u] = ot;
     const int n = a.bcount[u];
-    for (int q = 0; q * a.tok < n; ++q) a.tiles[ot + q] = make_int2(u, op + q * a.tok);
+    for (int q = 0; q * a.tok < n; ++q)
+        a.tiles[ot + q] = make_int4(u / a.C, u % a.C, op + q * a.tok, min(a.tok, n - q * a.tok));
 }
 
 // One thread per selection row: place its pairs into their buckets.
@@ -212,6 +214,7 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
         const long long u = (long long)p * a.C + c;
         const int pos = a.boff[u] + atomicAdd(&a.bcursor[u], 1);
         a.pairs[pos] = (t << 5) | i;
+        a.pair_w[pos] = a.w8[row * a.kmax + i];
     }
 }
 
@@ -230,15 +233,15 @@ struct TileInfo {
 };
 
 __device__ __forceinline__ TileInfo tile_info(const AttTcArgs &a, int tau) {
-    const int2 e = a.tiles[tau];
+    const int4 e = a.tiles[tau];
     TileInfo T;
-    T.p = e.x / a.C;
-    T.c = e.x % a.C;
+    T.p = e.x;
+    T.c = e.y;
     const int bj = T.p / a.ntb;
     T.b = bj / a.Hkv;
     T.j = bj % a.Hkv;
-    T.start = e.y;
-    T.n = min(a.tok, a.boff[e.x + 1] - e.y);
+    T.start = e.z;
+    T.n = e.w;
     return T;
 }
 
@@ -455,9 +458,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             tt = -1;
             ww = 0.f;
             if (m < X.n) {
-                const int pr = a.pairs[X.start + m];
-                tt = pr >> 5;
-                ww = a.w8[(((long long)X.b * a.Tq + tt) * a.Hkv + X.j) * a.kmax + (pr & 31)];
+                tt = a.pairs[X.start + m] >> 5;
+                ww = a.pair_w[X.start + m];
             }
         };
         int tau = tile_lo + blockIdx.x + grp * gridDim.x;
@@ -468,6 +470,11 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         for (; tau < tile_hi && ok; ++k) {
             const bool valid = m < T.n;
             const int tau_n = tau + 2 * gridDim.x;
+            // next tile's descriptor, pair and weight: two dependent loads whose latency hides behind this tile
+            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
+            int t_n;
+            float w_n;
+            row_info(Tn, t_n, w_n);
             // chunk softmax: S row -> P row (bf16, swizzled), l
             if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -508,11 +515,6 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->p_full[grp]);
-            // next tile's descriptor, pair and weight: their latency hides behind this tile's PV and reductions
-            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
-            int t_n;
-            float w_n;
-            row_info(Tn, t_n, w_n);
             // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
             if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -637,6 +639,7 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.btile = bf.btile;
     a.blk = bf.blk;
     a.pairs = bf.pairs;
+    a.pair_w = bf.pair_w;
     a.tiles = bf.tiles;
     a.ringbuf = bf.ring;
     a.status = bf.status;

@@ -32,9 +32,9 @@ struct AttTcLayout {
 };
 
 struct AttTcBuffers {
-    float *w8;
+    float *w8, *pair_w;
     int32_t *pairs, *counters, *boff, *btile, *blk;
-    int2 *tiles;
+    int4 *tiles;
     float *ring;
     uint32_t *status;
 };
@@ -49,7 +49,7 @@ struct WsLayout {
     int nsplit, chunks_per_split;
     bool split_select, split_attend, tc_select, tc_attend;
     AttTcLayout att;
-    size_t att_w8, att_pairs, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
+    size_t att_w8, att_pairs, att_pair_w, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
 };
 

@@ -61,11 +61,12 @@ WsLayout ws_layout(const Prob &p) {
         w.att = attend_tc_layout(p);
         w.att_w8 = take(rows * p.kmax * sizeof(float));
         w.att_pairs = take(rows * p.kmax * sizeof(int32_t));
+        w.att_pair_w = take(rows * p.kmax * sizeof(float));
         w.att_counters = take(w.att.counter_ints * sizeof(int32_t));
         w.att_boff = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
         w.att_btile = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
         w.att_blk = take(2 * (size_t)w.att.nblk * sizeof(int32_t));
-        w.att_tiles = take(w.att.max_tiles * sizeof(int2));
+        w.att_tiles = take(w.att.max_tiles * sizeof(int4));
         w.att_ring = take(w.att.ring_bytes);
     }
     w.total = off;
