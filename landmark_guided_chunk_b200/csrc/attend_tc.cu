@@ -338,33 +338,44 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
-    const int tile_lo = bar->tile_lo, tile_hi = bar->tile_hi;
+    // each CTA takes a contiguous range of the batch's tiles, so the tiles of one
+    // bucket (same chunk) mostly stay together and share one K/V load
+    const int per = (bar->tile_hi - bar->tile_lo + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int tile_lo = min(bar->tile_hi, bar->tile_lo + (int)blockIdx.x * per);
+    const int tile_hi = min(bar->tile_hi, tile_lo + per);
 
     if (warp < 4) {
         // ------------------------------------------------------------ producers: Q gather (thread = row), K/V TMA
         const int r = threadIdx.x;   // 0..127
         const int m = r / a.G, g = r % a.G;
-        int i = 0;
+        int i = 0, nload = 0;
         bool ok = true;
-        int tau = tile_lo + blockIdx.x;
+        int tau = tile_lo;
         TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
         int pr = (tau < tile_hi && m < T.n) ? a.pairs[T.start + m] : 0;
+        int prev_p = -1, prev_c = -1;
         for (; tau < tile_hi && ok; ++i) {
             // prefetch the next tile while this one is issued
-            const int tau_n = tau + gridDim.x;
+            const int tau_n = tau + 1;
             TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
-            if (warp == 0 && lane == 0) {
-                const int skv = i % a.nskv, ikv = i / a.nskv;
-                if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
-                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
-                uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
-                const int z = T.b * a.Tkv + T.c * S;
-                tma_load_3d(dk, &tmK, 0, T.j, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + kv_bytes, &tmK, 64, T.j, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, T.j, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, T.j, z, &bar->kv_full[skv]);
+            const bool newkv = T.p != prev_p || T.c != prev_c;
+            if (newkv) {
+                if (warp == 0 && lane == 0) {
+                    const int skv = nload % a.nskv, ikv = nload / a.nskv;
+                    if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
+                    mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
+                    uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
+                    const int z = T.b * a.Tkv + T.c * S;
+                    tma_load_3d(dk, &tmK, 0, T.j, z, &bar->kv_full[skv]);
+                    tma_load_3d(dk + kv_bytes, &tmK, 64, T.j, z, &bar->kv_full[skv]);
+                    tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, T.j, z, &bar->kv_full[skv]);
+                    tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, T.j, z, &bar->kv_full[skv]);
+                }
+                ++nload;
+                prev_p = T.p;
+                prev_c = T.c;
             }
             const bool valid = m < T.n;
             const char *src = reinterpret_cast<const char *>(Q);
@@ -386,7 +397,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (warp == 0 && lane == 0) {
             // wind down: the K/V loads issued have all landed
-            for (int s = 0; s < a.nskv && s < i; ++s) mbar_drain(&bar->kv_full[s], ((i - 1 - s) / a.nskv) & 1);
+            for (int s = 0; s < a.nskv && s < nload; ++s)
+                mbar_drain(&bar->kv_full[s], ((nload - 1 - s) / a.nskv) & 1);
         }
     } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
@@ -395,13 +407,26 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
-            const int n_mine = tile_lo + (int)blockIdx.x < tile_hi
-                                   ? (tile_hi - tile_lo - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
-                                   : 0;
-            auto issue_qk = [&](int i) -> bool {
-                const int sq = i % a.nsq, iq = i / a.nsq, skv = i % a.nskv, ikv = i / a.nskv;
+            const int n_mine = tile_hi - tile_lo;
+            // K/V load index of each tile, derived from the tile records exactly as the producer does
+            int key_p = -1, key_c = -1, nload = 0;
+            auto load_of = [&](int i) -> int {   // call with i = 0, 1, 2, ... in order
+                const int4 e = a.tiles[tile_lo + i];
+                if (e.x != key_p || e.y != key_c) {
+                    key_p = e.x;
+                    key_c = e.y;
+                    ++nload;
+                }
+                return nload - 1;
+            };
+            int waited_load = -1;   // last load whose kv_full has been waited on
+            auto issue_qk = [&](int i, int li) -> bool {
+                const int sq = i % a.nsq, iq = i / a.nsq, skv = li % a.nskv, ikv = li / a.nskv;
                 if (!mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status)) return false;
-                if (!mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status)) return false;
+                if (li != waited_load) {
+                    if (!mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status)) return false;
+                    waited_load = li;
+                }
                 tc_fence_after();
                 const uint32_t s_tmem = tmem + (i & 1) * 256;
                 const uint32_t qa = smem_u32(sQ + sq * 32768);
@@ -417,13 +442,16 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 return true;
             };
             const bool early = a.nskv >= 2;
-            bool ok = n_mine > 0 ? issue_qk(0) : true;
+            int li = n_mine > 0 ? load_of(0) : 0;
+            bool ok = n_mine > 0 ? issue_qk(0, li) : true;
             for (int i = 0; i < n_mine && ok; ++i) {
-                const int skv = i % a.nskv, gsel = i & 1, k = i >> 1;
-                if (early && i + 1 < n_mine && !(ok = issue_qk(i + 1))) break;
+                const int gsel = i & 1, k = i >> 1;
+                const int li_next = i + 1 < n_mine ? load_of(i + 1) : -1;
+                if (early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
                 if (!(ok = mbar_wait(&bar->p_full[gsel], k & 1, abort, a.status))) break;
                 if (k > 0 && !(ok = mbar_wait(&bar->o_empty[gsel], (k - 1) & 1, abort, a.status))) break;
                 tc_fence_after();
+                const int skv = li % a.nskv;
                 const uint32_t o_tmem = tmem + gsel * 256 + 128;
                 const uint32_t pa = smem_u32(sP + gsel * p_bytes);
                 const uint32_t vb = smem_u32(sKV + (size_t)skv * 4 * kv_bytes) + 2 * kv_bytes;
@@ -437,8 +465,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                               kk != 0);
                 }
                 umma_commit(&bar->o_full[gsel]);
-                umma_commit(&bar->kv_empty[skv]);
-                if (!early && i + 1 < n_mine && !(ok = issue_qk(i + 1))) break;
+                // the K/V stage is free once the last tile of its load is done
+                if (li_next != li) umma_commit(&bar->kv_empty[skv]);
+                if (!early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
+                li = li_next;
             }
             umma_commit(&bar->done);
             mbar_drain(&bar->done, 0);
@@ -462,14 +492,14 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 ww = a.pair_w[X.start + m];
             }
         };
-        int tau = tile_lo + blockIdx.x + grp * gridDim.x;
+        int tau = tile_lo + grp;
         TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
         int t;
         float w;
         row_info(T, t, w);
         for (; tau < tile_hi && ok; ++k) {
             const bool valid = m < T.n;
-            const int tau_n = tau + 2 * gridDim.x;
+            const int tau_n = tau + 2;
             // next tile's descriptor, pair and weight: two dependent loads whose latency hides behind this tile
             TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
             int t_n;
