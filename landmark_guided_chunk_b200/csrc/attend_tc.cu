@@ -220,9 +220,18 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
 
 // ---------------------------------------------------------------------------- main kernel
 
+constexpr int NINFO = 4;   // tiles of row info (token, weight) the producers may run ahead
+
+struct TileRows {            // one tile's row info, written by the producers, read by the epilogue
+    int p, n;
+    int t[MROWS];            // token of each row (-1: padding row)
+    float w[MROWS];          // fusion weight of each row's (token, slot) pair
+};
+
 struct __align__(8) AttBars {
     uint64_t q_full[2], q_empty[2], kv_full[2], kv_empty[2];
     uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], done;
+    uint64_t info_full[NINFO], info_empty[NINFO];
     uint32_t tmem_base;
     int abort;
     int tile_lo, tile_hi;
@@ -303,7 +312,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     uint8_t *sKV = sQ + (size_t)a.nsq * 32768;             // nskv x (K: 2 boxes, V: 2 boxes)
     uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 groups x p_bytes
     float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 warps x 32 x PITCH
-    AttBars *bar = reinterpret_cast<AttBars *>(stg + 8 * 32 * PITCH);
+    TileRows *info = reinterpret_cast<TileRows *>(stg + 8 * 32 * PITCH);      // NINFO stages
+    AttBars *bar = reinterpret_cast<AttBars *>(info + NINFO);
     volatile int *abort = &bar->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -322,6 +332,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             mbar_init(&bar->p_full[s], 4);
             mbar_init(&bar->o_full[s], 1);
             mbar_init(&bar->o_empty[s], 4);
+        }
+        for (int s = 0; s < NINFO; ++s) {
+            mbar_init(&bar->info_full[s], 128);
+            mbar_init(&bar->info_empty[s], 4);
         }
         mbar_init(&bar->done, 1);
         bar->abort = 0;
@@ -353,6 +367,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         int tau = tile_lo;
         TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
         int pr = (tau < tile_hi && m < T.n) ? a.pairs[T.start + m] : 0;
+        float pw = (tau < tile_hi && m < T.n) ? a.pair_w[T.start + m] : 0.f;
         int prev_p = -1, prev_c = -1;
         for (; tau < tile_hi && ok; ++i) {
             // prefetch the next tile while this one is issued
@@ -390,7 +405,21 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
             }
             cp_async_arrive(&bar->q_full[sq]);
+            // row info for the epilogue
+            {
+                const int si = i % NINFO, ii = i / NINFO;
+                if (ii > 0 && !(ok = mbar_wait(&bar->info_empty[si], (ii - 1) & 1, abort, a.status))) break;
+                TileRows &ri = info[si];
+                if (r == 0) {
+                    ri.p = T.p;
+                    ri.n = T.n;
+                }
+                ri.t[r] = valid ? (pr >> 5) : -1;
+                ri.w[r] = valid ? pw : 0.f;
+                mbar_arrive(&bar->info_full[si]);
+            }
             pr = (tau_n < tile_hi && m < Tn.n) ? a.pairs[Tn.start + m] : 0;
+            pw = (tau_n < tile_hi && m < Tn.n) ? a.pair_w[Tn.start + m] : 0.f;
             T = Tn;
             tau = tau_n;
         }
@@ -478,33 +507,22 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         const int grp = (warp - 4) >> 2;       // tiles i with i % 2 == grp
         const int ew = (warp - 4) & 3;         // TMEM lane quadrant
         const int r = ew * 32 + lane;
-        const int m = r / a.G;
         const uint32_t lane_base = tmem + grp * 256 + ((uint32_t)(ew * 32) << 16);
         float *wst = stg + (warp - 4) * 32 * PITCH;
         uint8_t *myP = sP + grp * p_bytes;
         bool ok = true;
         int k = 0;
-        auto row_info = [&](const TileInfo &X, int &tt, float &ww) {
-            tt = -1;
-            ww = 0.f;
-            if (m < X.n) {
-                tt = a.pairs[X.start + m] >> 5;
-                ww = a.pair_w[X.start + m];
-            }
-        };
         int tau = tile_lo + grp;
-        TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
-        int t;
-        float w;
-        row_info(T, t, w);
-        for (; tau < tile_hi && ok; ++k) {
-            const bool valid = m < T.n;
-            const int tau_n = tau + 2;
-            // next tile's descriptor, pair and weight: two dependent loads whose latency hides behind this tile
-            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
-            int t_n;
-            float w_n;
-            row_info(Tn, t_n, w_n);
+        for (; tau < tile_hi && ok; ++k, tau += 2) {
+            const int i = tau - tile_lo;
+            const int si = i % NINFO;
+            if (!(ok = mbar_wait(&bar->info_full[si], (i / NINFO) & 1, abort, a.status))) break;
+            const int Tp = info[si].p;
+            const int t = info[si].t[r];
+            const float w = info[si].w[r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->info_empty[si]);
+            const bool valid = t >= 0;
             // chunk softmax: S row -> P row (bf16, swizzled), l
             if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -549,8 +567,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
             const float f = valid ? w / l : 0.f;
-            const int tloc_base = (T.p % a.ntb) * TB;
-            float *acc_slot = slot_of(a, T.p);
+            const int tloc_base = (Tp % a.ntb) * TB;
+            float *acc_slot = slot_of(a, Tp);
             // destination row of each staging row this lane reduces (rows rr*4 + lane/8)
             float *dstrow[8];
 #pragma unroll
@@ -586,10 +604,6 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 }
                 __syncwarp();
             }
-            T = Tn;
-            t = t_n;
-            w = w_n;
-            tau = tau_n;
         }
     }
     tc_fence_before();
@@ -694,7 +708,7 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
     const size_t smem = 1024 + (size_t)a.nsq * 32768 + (size_t)a.nskv * 4 * p.S * 128 + 2 * (size_t)(p.S / 64) * 16384 +
-                        8 * 32 * PITCH * sizeof(float) + sizeof(AttBars);
+                        8 * 32 * PITCH * sizeof(float) + NINFO * sizeof(TileRows) + sizeof(AttBars);
     if ((e = cudaFuncSetAttribute(att_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
         cudaSuccess)
         return e;
