@@ -140,6 +140,32 @@ HSA_API hsa_status_t hsa_attend(const hsa_problem_t *p, const void *Q, const voi
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * hsa_select without a workspace, for callers that cannot allocate device
+ * memory at the point of the call: code that runs under an allocator that
+ * must not be re-entered, a runtime whose memory pool is already carved up, or
+ * an embedding that only owns the tensors it passes in.  It computes exactly
+ * what hsa_select computes; the paper has no counterpart for this entry point.
+ *   - Its scratch (the status word and, for few rows with long scans, the
+ *     per-split candidate lists) is a 1 MiB array inside the library.  Every
+ *     GPU that loads the library holds that array until the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress), so make that first call before any stream
+ *     capture.  Later calls reuse the address.
+ *   - Problems whose scratch would exceed 1 MiB are rejected with
+ *     HSA_ERR_WORKSPACE before anything is launched (e.g. 64 decode rows over
+ *     16384 chunks with k = 16 need ~0.13 MiB; prefill problems need only the
+ *     status word; 4096 decode rows with 32 slots each need just over 1 MiB).
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents: calls that overlap on the GPU (other streams, other
+ *     host threads) race on it and must be serialised by the caller.  A
+ *     device-side timeout of this call is recorded in that array, not in any
+ *     workspace, so hsa_get_device_status() cannot report it.
+ */
+HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *p, const void *Q, const void *L, int32_t *idx,
+                                        float *score, int32_t *keff, void *stream);
+
+/*
  * The whole path: hsa_landmarks (unless HSA_FLAG_LANDMARKS_READY), then
  * hsa_select, then hsa_attend.  L is an output (or an input with the flag).
  * idx, score and keff may each be NULL.  The selection then lives only in the

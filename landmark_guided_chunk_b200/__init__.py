@@ -20,7 +20,7 @@ import torch
 from . import _native
 from ._native import HSAError, hsa_problem_t
 
-__all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "attend",
+__all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "select_noalloc", "attend",
            "forward", "device_status", "HSAError", "hsa_problem_t", "kmax_of"]
 
 _DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
@@ -109,6 +109,27 @@ def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False):
         ws = alloc_workspace(prob, Q.device)
     _native.check(_native.lib().hsa_select(ctypes.byref(prob), _p(Q), _p(L), _p(idx), _p(score), _p(keff),
                                            _p(ws), ws.numel(), _stream(Q)), "hsa_select")
+    return idx, score, keff
+
+
+def select_noalloc(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, out=None):
+    """hsa_select without a workspace: the library's own fixed 1 MiB device
+    scratch is used instead (see include/hsa.h for who needs this and its
+    limits).  out, if given, is (idx, score, keff) to fill; they are allocated
+    here otherwise."""
+    _dev(Q, L)
+    B, Tq, H, d = Q.shape
+    Hkv, C = L.shape[1], L.shape[2]
+    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0)
+    km = kmax_of(k, tau)
+    if out is None:
+        out = (torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device),
+               torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device),
+               torch.empty(B, Tq, Hkv, dtype=torch.int32, device=Q.device))
+    idx, score, keff = out
+    _dev(idx, score, keff)
+    _native.check(_native.lib().hsa_select_noalloc(ctypes.byref(prob), _p(Q), _p(L), _p(idx), _p(score), _p(keff),
+                                                   _stream(Q)), "hsa_select_noalloc")
     return idx, score, keff
 
 

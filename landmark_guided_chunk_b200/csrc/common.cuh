@@ -55,6 +55,13 @@ struct WsLayout {
 
 WsLayout ws_layout(const Prob &p);
 
+// Host-side helpers of the entry points (hsa_api.cu): record the detail for
+// hsa_last_error() and return the status; validate a problem; check a pointer.
+hsa_status_t fail(hsa_status_t s, const char *fmt, ...);
+hsa_status_t cuda_fail(cudaError_t e, const char *what);
+hsa_status_t validate(const hsa_problem_t *in, Prob *p);
+hsa_status_t need(const void *x, bool required, const char *name);
+
 // status word values (workspace header)
 constexpr uint32_t DEV_OK = 0;
 constexpr uint32_t DEV_TIMEOUT = 1;      // a bounded wait expired

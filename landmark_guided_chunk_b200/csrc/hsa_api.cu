@@ -11,7 +11,7 @@ namespace hsa {
 
 static thread_local char g_err[512] = "";
 
-static hsa_status_t fail(hsa_status_t s, const char *fmt, ...) {
+hsa_status_t fail(hsa_status_t s, const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
     vsnprintf(g_err, sizeof g_err, fmt, ap);
@@ -19,7 +19,7 @@ static hsa_status_t fail(hsa_status_t s, const char *fmt, ...) {
     return s;
 }
 
-static hsa_status_t cuda_fail(cudaError_t e, const char *what) {
+hsa_status_t cuda_fail(cudaError_t e, const char *what) {
     return fail(HSA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
@@ -85,7 +85,7 @@ WsLayout ws_layout(const Prob &p) {
     return w;
 }
 
-static hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
+hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
     if (!in) return fail(HSA_ERR_INVALID_ARG, "problem pointer is NULL");
     if (in->B < 0 || in->Tq < 0 || in->Tkv < 0)
         return fail(HSA_ERR_INVALID_ARG, "negative size (B=%d Tq=%d Tkv=%d)", in->B, in->Tq, in->Tkv);
@@ -126,7 +126,7 @@ static hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
 
 static bool aligned16(const void *x) { return ((uintptr_t)x & 15u) == 0; }
 
-static hsa_status_t need(const void *x, bool required, const char *name) {
+hsa_status_t need(const void *x, bool required, const char *name) {
     if (!required) return HSA_OK;
     if (!x) return fail(HSA_ERR_INVALID_ARG, "%s is NULL", name);
     if (!aligned16(x)) return fail(HSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
