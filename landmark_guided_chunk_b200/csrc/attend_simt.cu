@@ -100,16 +100,28 @@ __device__ __forceinline__ void row_coords(const AttArgs &a, long long row, int 
     b = (int)(bt / a.Tq);
 }
 
-// Stage chunk c of kv head j (batch b) into shared memory as fp32.
+// Stage chunk c of kv head j (batch b) into shared memory as fp32, reading
+// the S rows of K and V with 16-byte loads.
 template <typename T>
 __device__ __forceinline__ void stage_chunk(const T *K, const T *V, const AttArgs &a, int b, int j, int c,
                                             const Smem &s) {
+    constexpr int EPS = 16 / (int)sizeof(T);
+    const int segs = a.d / EPS;
     const size_t row0 = ((size_t)b * a.Tkv + (size_t)c * a.S) * a.Hkv + j;
-    for (int i = threadIdx.x; i < a.S * a.d; i += NT) {
-        const int u = i / a.d, e = i - u * a.d;
-        const size_t off = (row0 + (size_t)u * a.Hkv) * a.d + e;
-        s.Ks[u * (a.d + 1) + e] = to_f32(K[off]);
-        s.Vs[u * a.d + e] = to_f32(V[off]);
+    for (int i = threadIdx.x; i < a.S * segs; i += NT) {
+        const int u = i / segs, sg = i - u * segs;
+        const size_t off = (row0 + (size_t)u * a.Hkv) * a.d + (size_t)sg * EPS;
+        const uint4 kk = __ldg(reinterpret_cast<const uint4 *>(K + off));
+        const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(V + off));
+        const T *kt = reinterpret_cast<const T *>(&kk);
+        const T *vt = reinterpret_cast<const T *>(&vv);
+        float *kd = s.Ks + u * (a.d + 1) + sg * EPS;
+        float *vd = s.Vs + u * a.d + sg * EPS;
+#pragma unroll
+        for (int e = 0; e < EPS; ++e) {
+            kd[e] = to_f32(kt[e]);
+            vd[e] = to_f32(vt[e]);
+        }
     }
 }
 

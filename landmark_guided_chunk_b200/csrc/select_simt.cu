@@ -61,6 +61,62 @@ __device__ __forceinline__ void scan_range(const float *qs, const T *Lj, const S
     }
 }
 
+// Same scan, but with a row of L spread over SEGS lanes (16 bytes each), so a
+// warp's load instruction covers 32/SEGS whole rows contiguously.  The
+// partial dots are summed with xor-shuffles, and each score is handed to the
+// lane that owns its chunk in the 32-chunk batch offered to the list.
+template <typename T, int SEGS>
+__device__ __forceinline__ void scan_range_rows(const float *qs, const T *Lj, const SelArgs &a, int c0, int c1,
+                                                int step, float &v, int &id, int lane) {
+    constexpr int EPS = 16 / (int)sizeof(T);   // elements per 16-byte segment
+    constexpr int CPR = 32 / SEGS;             // rows per load instruction
+    const int seg = lane % SEGS, sub = lane / SEGS;
+    float qv[EPS];
+#pragma unroll
+    for (int e = 0; e < EPS; ++e) qv[e] = qs[seg * EPS + e];
+    for (int base = c0; base < c1; base += step) {
+        float mine = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < 32 / CPR; ++r) {
+            const int c = base + r * CPR + sub;
+            float part = 0.f;
+            if (c < c1) {
+                const uint4 u = __ldg(reinterpret_cast<const uint4 *>(Lj + (size_t)c * a.d) + seg);
+                if (sizeof(T) == 2) {
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        part = fmaf(qv[2 * e], f.x, part);
+                        part = fmaf(qv[2 * e + 1], f.y, part);
+                    }
+                } else {
+                    const float *f = reinterpret_cast<const float *>(&u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) part = fmaf(qv[e], f[e], part);
+                }
+            }
+#pragma unroll
+            for (int o = SEGS / 2; o > 0; o >>= 1) part += __shfl_xor_sync(FULL, part, o);
+            // the score of row r*CPR + x sits in lanes x*SEGS .. x*SEGS+SEGS-1
+            const float got = __shfl_sync(FULL, part, (lane % CPR) * SEGS);
+            if (lane / CPR == r) mine = got;
+        }
+        const int c = base + lane;
+        list_offer(v, id, mine, c, c < c1, a.kmax, lane);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void scan_range_fast(const float *qs, const T *Lj, const SelArgs &a, int c0, int c1,
+                                                int step, float &v, int &id, int lane) {
+    const int segs = a.d * (int)sizeof(T) / 16;
+    if (segs == 16) scan_range_rows<T, 16>(qs, Lj, a, c0, c1, step, v, id, lane);
+    else if (segs == 8) scan_range_rows<T, 8>(qs, Lj, a, c0, c1, step, v, id, lane);
+    else if (segs == 32) scan_range_rows<T, 32>(qs, Lj, a, c0, c1, step, v, id, lane);
+    else scan_range(qs, Lj, a, c0, c1, step, v, id, lane);
+}
+
 __device__ __forceinline__ void write_row(const SelArgs &a, long long row, float v, int id, int ke, int32_t *idx,
                                           float *score, int32_t *keff, int lane) {
     if (lane < a.kmax) {
@@ -114,7 +170,7 @@ __global__ void __launch_bounds__(256) select_split_kernel(const T *__restrict__
     float v;
     int id;
     list_init(v, id);
-    if (c0 < c1) scan_range(qs, Lj, a, c0 + 32 * warp, c1, 256, v, id, lane);
+    if (c0 < c1) scan_range_fast(qs, Lj, a, c0 + 32 * warp, c1, 256, v, id, lane);
     if (lane < a.kmax) wl[warp * a.kmax + lane] = make_float2(v, __int_as_float(id));
     __syncthreads();
     if (warp == 0) {

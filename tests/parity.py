@@ -1,8 +1,11 @@
 """Comparison rules between the CUDA path and the CPU oracle.
 
-* Landmarks: bf16 values may differ from the oracle's by at most one bf16 ulp
-  (the GPU sums in fp32, the oracle in fp64, so a value next to a rounding
-  boundary can land on either side).  fp32 values must be within 1e-5.
+* Landmarks: bf16 values may differ from the oracle's by one bf16 ulp plus
+  the fp32 accumulation error of the d-term projection, bounded here by
+  2^-17 * max|L| (the GPU sums in fp32, the oracle in fp64).  So a value next
+  to a rounding boundary may land on either side, and a value that cancels to
+  nearly zero (whose bf16 ulp is tiny) may differ by the absolute fp32 error.
+  fp32 values must be within 1e-5.
 * Selection: chunk indices are bit-exact, except where the oracle's scores
   around the cut lie within REL = 1e-3 (relative) of each other.  There, any
   GPU set that differs from the oracle's only among such near-tied chunks is
@@ -36,8 +39,10 @@ def check_landmarks(L_gpu: torch.Tensor, L_orc: np.ndarray) -> dict:
     g = L_gpu.double().cpu().numpy()
     diff = np.abs(g - L_orc)
     if L_gpu.dtype == torch.bfloat16:
-        bad = diff > bf16_ulp(L_orc) * 1.0000001
-        assert not bad.any(), f"{bad.sum()} landmark values differ by more than one bf16 ulp (max diff {diff.max()})"
+        atol = 2.0 ** -17 * float(np.abs(L_orc).max()) if L_orc.size else 0.0
+        bad = diff > bf16_ulp(L_orc) * 1.0000001 + atol
+        assert not bad.any(), (f"{bad.sum()} landmark values differ by more than one bf16 ulp + {atol:.2e} "
+                               f"(worst: gpu {g[bad][:3]} oracle {L_orc[bad][:3]})")
         return {"flips": int((diff > 0).sum()), "n": diff.size}
     assert diff.max() <= 1e-5, f"fp32 landmark max diff {diff.max()}"
     return {"flips": 0, "n": diff.size, "max_diff": float(diff.max())}
