@@ -265,12 +265,12 @@ __global__ void __launch_bounds__(256, 1)
             if (!ok || !valid) continue;
             int ke = nc < a.k ? nc : a.k;
             if (a.tau > 0.f && nc > a.k) {
-                float sk = 0.f, sk1 = 0.f;
+                // entries k-1 and k (k < kmax <= KL) through this thread's column of the
+                // drained queue: selecting them from registers by a runtime index would
+                // move the whole list into local memory
 #pragma unroll
-                for (int q = 0; q < KL; ++q) {
-                    if (q == a.k - 1) sk = v[q];
-                    if (q == a.k) sk1 = v[q];
-                }
+                for (int q = 0; q < KL; ++q) qv[q * 128 + r] = v[q];
+                const float sk = qv[(a.k - 1) * 128 + r], sk1 = qv[a.k * 128 + r];
                 if (sk - sk1 < a.tau * fabsf(sk)) ke = nc < 2 * a.k ? nc : 2 * a.k;
             }
             const long long row = ((long long)T.b * a.Tq + t) * a.Hkv + T.j;
