@@ -17,18 +17,25 @@
 // multiple of 16.
 //
 //   warp 0      TMA producer: the A tile (G*d/64 boxes of 128 rows x 64 cols)
-//               once per tile, L slices into a 2-stage ring
+//               once per tile, each box reloaded for the next tile as soon as
+//               the last slice's MMAs have read it; L slices into a 2-stage ring
 //   warp 1      MMA issuer: 4*G*d/64 tcgen05.mma (M128, N<=128, K16) per slice
 //               into one of two TMEM accumulators
 //   warp 2      TMEM allocator (256 columns)
-//   warps 4..7  epilogue: thread = row.  tcgen05.ld 32 scores at a time.
+//   warps 4..7  epilogue: thread = row.  tcgen05.ld 16 scores at a time.
 //               Scores of candidate chunks (c < ncand(t)) that beat the
-//               row's current k-th best are appended to a per-thread queue
-//               in shared memory (predicated stores, no divergence).  The
-//               warp then drains the queues in lock-step into sorted
-//               register lists (score desc, chunk asc).  Chunks arrive in
-//               increasing order, so counting the entries >= s gives the
-//               insertion position and keeps ties on the lower index.
+//               row's current k-th best are appended to the row's FIFO (a
+//               ring of 32 entries in shared memory, predicated stores).
+//               The warp then pops entries in lock-step into sorted register
+//               lists (score desc, chunk asc): as many pops as the warp's mean
+//               FIFO length, and more if a FIFO could overflow on the next 16
+//               columns; everything at the row's end.  Draining by the mean
+//               rather than the longest FIFO keeps most lanes busy; an entry
+//               that went stale while queued is a no-op push.  Chunks arrive
+//               in increasing order, so an entry that equals a listed score
+//               goes behind it, which keeps ties on the lower index.
+//               The accumulator is released as soon as its last columns are
+//               in registers, before that chunk's pops.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -42,6 +49,7 @@ constexpr int NT = 128;        // chunks per N-slice
 constexpr int NSTAGE = 2;      // L-slice ring depth
 constexpr int BOX = 64 * 128 * 2;   // one 64-column x 128-row bf16 box (16 KB)
 constexpr uint32_t TMEM_COLS = 2 * NT;
+constexpr int MAX_KB = 8;      // G*d <= 512
 
 struct TcSelArgs {
     int B, Tq, Hkv, G, d, S, C, k, kmax;
@@ -53,7 +61,7 @@ struct TcSelArgs {
 };
 
 struct __align__(8) Bars {
-    uint64_t a_full, a_empty, done;
+    uint64_t a_full[MAX_KB], a_empty[MAX_KB], done;
     uint64_t b_full[NSTAGE], b_empty[NSTAGE];
     uint64_t t_full[2], t_empty[2];
     uint32_t tmem_base;
@@ -86,22 +94,29 @@ __device__ __forceinline__ int slice_n(const Tile &T, int n) {
 
 // Insert (x, xi) into the sorted list; xi is larger than every chunk index
 // already present, so equal scores already in the list stay ahead of it.
+// Entry q keeps its value when v[q] >= x; otherwise it takes x if v[q-1] >= x
+// (x lands at q) and v[q-1] otherwise (shifted down).  Going from the tail up,
+// v[q-1] still holds its old value when entry q reads it.  x = -inf changes nothing.
 template <int KL>
 __device__ __forceinline__ void list_push(float (&v)[KL], int (&id)[KL], float x, int xi) {
-    int pos = 0;
 #pragma unroll
-    for (int q = 0; q < KL; ++q) pos += (v[q] >= x) ? 1 : 0;
-    if (pos >= KL) return;
-#pragma unroll
-    for (int q = KL - 1; q > 0; --q) {
-        const bool sh = q > pos, eq = q == pos;
-        v[q] = sh ? v[q - 1] : (eq ? x : v[q]);
-        id[q] = sh ? id[q - 1] : (eq ? xi : id[q]);
+    for (int q = KL - 1; q >= 1; --q) {
+        const bool keep = v[q] >= x, here = v[q - 1] >= x;
+        v[q] = keep ? v[q] : (here ? x : v[q - 1]);
+        id[q] = keep ? id[q] : (here ? xi : id[q - 1]);
     }
-    if (pos == 0) {
-        v[0] = x;
-        id[0] = xi;
-    }
+    const bool keep0 = v[0] >= x;
+    v[0] = keep0 ? v[0] : x;
+    id[0] = keep0 ? id[0] : xi;
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
 }
 
 template <int KL>
@@ -119,8 +134,10 @@ __global__ void __launch_bounds__(256, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        mbar_init(&bar->a_full, 1);
-        mbar_init(&bar->a_empty, 1);
+        for (int kb = 0; kb < MAX_KB; ++kb) {
+            mbar_init(&bar->a_full[kb], 1);
+            mbar_init(&bar->a_empty[kb], 1);
+        }
         mbar_init(&bar->done, 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bar->b_full[s], 1);
@@ -149,17 +166,21 @@ __global__ void __launch_bounds__(256, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int g = 0, ta = 0;
+            int g = 0, ta = 0, kb_part = 0;   // kb_part: boxes issued of a tile cut short
             bool ok = true;
             for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
                 const Tile T = tile_of(a, tau);
                 if (T.nslices == 0) continue;
-                if (ta > 0 && !(ok = mbar_wait(&bar->a_empty, (ta - 1) & 1, abort, a.status))) break;
-                mbar_expect_tx(&bar->a_full, (uint32_t)(a.nkb * BOX));
                 const int y = T.b * a.Tq + T.t0;
-                for (int kb = 0; kb < a.nkb; ++kb)
-                    tma_load_2d(sA + (size_t)kb * BOX, &tmQ, T.j * a.G * a.d + kb * 64, y, &bar->a_full);
+                for (int kb = 0; kb < a.nkb; ++kb) {
+                    if (ta > 0 && !(ok = mbar_wait(&bar->a_empty[kb], (ta - 1) & 1, abort, a.status))) break;
+                    mbar_expect_tx(&bar->a_full[kb], (uint32_t)BOX);
+                    tma_load_2d(sA + (size_t)kb * BOX, &tmQ, T.j * a.G * a.d + kb * 64, y, &bar->a_full[kb]);
+                    kb_part = kb + 1;
+                }
+                if (!ok) break;
                 ++ta;
+                kb_part = 0;
                 const int ly = (T.b * a.Hkv + T.j) * a.C;
                 for (int n = 0; n < T.nslices; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE;
@@ -170,7 +191,10 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             // wind down: every load issued has landed before the CTA may exit
-            if (ta > 0) mbar_drain(&bar->a_full, (ta - 1) & 1);
+            for (int kb = 0; kb < a.nkb; ++kb) {
+                const int nload = ta + (kb < kb_part ? 1 : 0);   // loads issued into box kb
+                if (nload > 0) mbar_drain(&bar->a_full[kb], (nload - 1) & 1);
+            }
             for (int s = 0; s < NSTAGE && s < g; ++s) {
                 const int last = (g - 1 - s) / NSTAGE;   // index of the last use of stage s
                 mbar_drain(&bar->b_full[s], last & 1);
@@ -184,9 +208,9 @@ __global__ void __launch_bounds__(256, 1)
             for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
                 const Tile T = tile_of(a, tau);
                 if (T.nslices == 0) continue;
-                if (!(ok = mbar_wait(&bar->a_full, ta & 1, abort, a.status))) break;
+                const uint32_t pa = ta & 1;
                 ++ta;
-                for (int n = 0; n < T.nslices; ++n, ++g) {
+                for (int n = 0; n < T.nslices && ok; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE, buf = g & 1, u = g >> 1;
                     if (!(ok = mbar_wait(&bar->b_full[s], i & 1, abort, a.status))) break;
                     if (u > 0 && !(ok = mbar_wait(&bar->t_empty[buf], (u - 1) & 1, abort, a.status))) break;
@@ -194,17 +218,23 @@ __global__ void __launch_bounds__(256, 1)
                     const uint32_t idesc = idesc_bf16_f32(TM, slice_n(T, n), 0, 0);
                     const uint32_t d_tmem = tmem + (uint32_t)(buf * NT);
                     const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB + (size_t)s * a.dkb * BOX);
+                    const bool last = n == T.nslices - 1;
                     for (int kb = 0; kb < a.nkb; ++kb) {
+                        if (n == 0) {
+                            if (!(ok = mbar_wait(&bar->a_full[kb], pa, abort, a.status))) break;
+                            tc_fence_after();
+                        }
                         const uint32_t aK = aBase + kb * BOX, bK = bBase + (kb % a.dkb) * BOX;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_bf16(d_tmem, desc_kmajor_sw128(aK + kk * 32), desc_kmajor_sw128(bK + kk * 32), idesc,
                                       (kb | kk) != 0);
+                        if (last) umma_commit(&bar->a_empty[kb]);   // box kb may be refilled
                     }
+                    if (!ok) break;
                     umma_commit(&bar->b_empty[s]);
                     umma_commit(&bar->t_full[buf]);
                 }
-                if (ok) umma_commit(&bar->a_empty);
             }
             umma_commit(&bar->done);
             mbar_drain(&bar->done, 0);
@@ -232,35 +262,51 @@ __global__ void __launch_bounds__(256, 1)
                 v[q] = -INFINITY;
                 id[q] = -1;
             }
+            int head = 0, tail = 0;   // this row's FIFO of pending (score, chunk): ring of 32 in qv/qi
             for (int n = 0; n < T.nslices; ++n, ++g) {
                 const int buf = g & 1, u = g >> 1;
                 if (!(ok = mbar_wait(&bar->t_full[buf], u & 1, abort, a.status))) break;
                 tc_fence_after();
-                const int nchunks = (slice_n(T, n) + 31) / 32;
-                for (int q = 0; q < nchunks; ++q) {
-                    uint32_t rr[32];
-                    tmem_ld32(lane_base + (uint32_t)(buf * NT + q * 32), rr);
+                const int nch = slice_n(T, n) / 16;
+                const bool last_slice = n == T.nslices - 1;
+                for (int q = 0; q < nch; ++q) {
+                    uint32_t rr[16];
+                    tmem_ld16(lane_base + (uint32_t)(buf * NT + q * 16), rr);
                     tmem_wait_ld();
-                    const int cb = n * NT + q * 32;
+                    if (q == nch - 1) {   // the accumulator may be overwritten from here on
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar->t_empty[buf]);
+                    }
+                    const int cb = n * NT + q * 16;
                     const float thr = v[KL - 1];
-                    int cnt = 0;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 16; ++e) {
                         const float sv = __uint_as_float(rr[e]);
                         const bool take = (cb + e < nc) && (sv > thr);
+                        const int slot = (tail & 31) * 128 + r;
                         if (take) {
-                            qv[cnt * 128 + r] = sv;
-                            qi[cnt * 128 + r] = cb + e;
+                            qv[slot] = sv;
+                            qi[slot] = cb + e;
                         }
-                        cnt += take ? 1 : 0;
+                        tail += take ? 1 : 0;
                     }
-                    const int it_max = __reduce_max_sync(FULL, (unsigned)cnt);
-                    for (int it = 0; it < it_max; ++it)
-                        if (it < cnt) list_push<KL>(v, id, qv[it * 128 + r], qi[it * 128 + r]);
+                    const int len = tail - head;
+                    const int mx = (int)__reduce_max_sync(FULL, (unsigned)len);
+                    int dn = mx;
+                    if (!(last_slice && q == nch - 1)) {
+                        const int sum = (int)__reduce_add_sync(FULL, (unsigned)len);
+                        dn = max((sum + 31) >> 5, mx - 16);   // leaves room for the next 16 columns
+                    }
+                    for (int it = 0; it < dn; ++it) {
+                        const bool has = head < tail;
+                        const int slot = (head & 31) * 128 + r;
+                        const float x = has ? qv[slot] : -INFINITY;
+                        const int xi = has ? qi[slot] : 0;
+                        head += has ? 1 : 0;
+                        list_push<KL>(v, id, x, xi);
+                    }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->t_empty[buf]);
             }
             if (!ok || !valid) continue;
             int ke = nc < a.k ? nc : a.k;

@@ -55,7 +55,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended in hardware for up to
+// `suspend_ns` while the phase is still open, instead of returning at once:
+// a waiting warp then issues almost nothing.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s: far beyond any legitimate wait here
+constexpr uint32_t SUSPEND_NS = 200000u;             // longest single suspension inside a wait (0.2 ms)
 
 // Wait until the phase with `parity` of *bar has completed.  Returns false (and
 // leaves *abort set) if the CTA is aborting or the limit expired.
@@ -63,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity, SUSPEND_NS)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
             *abort = 1;
@@ -76,7 +92,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // Bounded wait used only while winding down (ignores the abort flag).
 __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
+    while (!mbar_try_wait_suspend(bar, parity, SUSPEND_NS))
         if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
     return true;
 }
