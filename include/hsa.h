@@ -181,7 +181,8 @@ HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const vo
  * starts (stream-ordered), so the word describes the latest such call.
  * Returns HSA_OK, HSA_ERR_TIMEOUT (a bounded device wait expired),
  * HSA_ERR_INVALID_ARG (hsa_attend skipped an out-of-range chunk index or keff)
- * or HSA_ERR_CUDA.
+ * or HSA_ERR_CUDA (a CUDA call failed, or a kernel's own index check failed and
+ * skipped the access, leaving that call's results incomplete).
  */
 HSA_API hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream);
 

@@ -311,6 +311,10 @@ cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const
         bf.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
         return launch_attend_tc(p, w.att, bf, Q, K, V, idx, score, keff, O, st);
     }
+    if (w.gather_attend)
+        return launch_attend_gather(p, Q, K, V, idx, score, keff, O, reinterpret_cast<float *>(ws + w.att_acc),
+                                    reinterpret_cast<int32_t *>(ws + w.att_cnt), reinterpret_cast<uint32_t *>(ws + w.hdr),
+                                    st);
     if (p.dtype == HSA_BF16) return launch_typed<__nv_bfloat16>(p, w, Q, K, V, idx, score, keff, O, ws, st);
     return launch_typed<float>(p, w, Q, K, V, idx, score, keff, O, ws, st);
 }

@@ -45,9 +45,13 @@ struct WsLayout {
     size_t sel_idx, sel_score, sel_keff;   // selection outputs when hsa_forward gets NULLs
     size_t split_lists;  // decode split scan: rows x nsplit x kmax (score, id)
     size_t partials;     // decode split attend: rows x kmax x G x d fp32
+    size_t sel_cnt;      // split select (tensor-core scan): per-row completion counters, right after the header
+    size_t att_cnt;      // gather attend: per-row completion counters, right after the header
+    size_t att_acc;      // gather attend: per-row fp32 accumulators (rows x G x d), right after the counters
+    size_t clear_bytes;  // bytes from the workspace start zeroed before every call (status word, counters)
     size_t total;
     int nsplit, chunks_per_split;
-    bool split_select, split_attend, tc_select, tc_attend;
+    bool split_select, mma_select, split_attend, gather_attend, tc_select, tc_attend;
     AttTcLayout att;
     size_t att_w8, att_pairs, att_pair_w, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
@@ -66,6 +70,7 @@ hsa_status_t need(const void *x, bool required, const char *name);
 constexpr uint32_t DEV_OK = 0;
 constexpr uint32_t DEV_TIMEOUT = 1;      // a bounded wait expired
 constexpr uint32_t DEV_BAD_INDEX = 2;    // hsa_attend got a chunk index / keff outside its row's range
+constexpr uint32_t DEV_INTERNAL = 4;     // a kernel's own slot/index check failed; the access was skipped
 
 // ---------------------------------------------------------------------------- element access
 
@@ -158,6 +163,74 @@ __device__ __forceinline__ void list_offer(float &v, int &id, float s, int c, bo
     }
 }
 
+// ---- bitonic forms of the same list (kmax <= 16).  One (v, id) per lane;
+// "better" is ranks_before; sentinels (-inf, INT32_MAX) rank last.
+
+// Compare-exchange with the lane at distance `stride`: the lower lane of the
+// pair keeps the better entry when `desc` holds for it, the worse otherwise.
+__device__ __forceinline__ void bitonic_step(float &v, int &id, int stride, bool desc, int lane) {
+    const float pv = __shfl_xor_sync(FULL, v, stride);
+    const int pid = __shfl_xor_sync(FULL, id, stride);
+    const bool lower = (lane & stride) == 0;
+    const bool take = (lower == desc) ? ranks_before(pv, pid, v, id) : ranks_before(v, id, pv, pid);
+    if (take) {
+        v = pv;
+        id = pid;
+    }
+}
+
+// Sort the 32 lanes' entries, best first.
+__device__ __forceinline__ void bitonic_sort32(float &v, int &id, int lane) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+        const bool desc = (lane & size) == 0;   // direction of this lane's block
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) bitonic_step(v, id, stride, desc, lane);
+    }
+}
+
+// Lanes 0..15 hold a sorted list A (best first), lanes 16..31 a sorted list B
+// in reverse (worst first): the sequence is bitonic; afterwards all 32 lanes
+// are sorted best first, so lanes 0..15 hold the best 16 of A and B.
+__device__ __forceinline__ void bitonic_merge32(float &v, int &id, int lane) {
+#pragma unroll
+    for (int stride = 16; stride > 0; stride >>= 1) bitonic_step(v, id, stride, true, lane);
+}
+
+// Merge a sorted list held the same way (lane < kmax <= 16: entry lane) into
+// the warp list.
+__device__ __forceinline__ void list_merge16(float &v, int &id, float bv, int bid, int kmax, int lane) {
+    // lane 16 + i takes B's entry 15 - i
+    const float rv = __shfl_sync(FULL, bv, 31 - lane);
+    const int rid = __shfl_sync(FULL, bid, 31 - lane);
+    float x = lane < 16 ? (lane < kmax ? v : -INFINITY) : (31 - lane < kmax ? rv : -INFINITY);
+    int xi = lane < 16 ? (lane < kmax ? id : INT32_MAX) : (31 - lane < kmax ? rid : INT32_MAX);
+    bitonic_merge32(x, xi, lane);
+    v = lane < kmax ? x : -INFINITY;
+    id = lane < kmax ? xi : INT32_MAX;
+}
+
+// Offer one candidate per lane (valid lanes only), kmax <= 16: few qualifying
+// candidates are inserted one by one; many are sorted as a batch and merged.
+__device__ __forceinline__ void list_offer16(float &v, int &id, float s, int c, bool valid, int kmax, int lane) {
+    const float vl = __shfl_sync(FULL, v, kmax - 1);
+    const int il = __shfl_sync(FULL, id, kmax - 1);
+    const bool pass = valid && ranks_before(s, c, vl, il);
+    unsigned m = __ballot_sync(FULL, pass);
+    if (__popc(m) <= 3) {
+        while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            list_insert(v, id, __shfl_sync(FULL, s, src), __shfl_sync(FULL, c, src), kmax, lane);
+        }
+        return;
+    }
+    float x = pass ? s : -INFINITY;
+    int xi = pass ? c : INT32_MAX;
+    bitonic_sort32(x, xi, lane);
+    list_merge16(v, id, x, xi, kmax, lane);
+}
+
 // keff for a row from its sorted list (entries k-1 and k), with the gap router.
 __device__ __forceinline__ int list_keff(float v, int ncand, int k, int kmax, float tau) {
     int ke = ncand < k ? ncand : k;
@@ -192,6 +265,11 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
                              uint32_t *status, cudaStream_t st);
 
 bool attend_tc_supported(const Prob &p);
+bool attend_gather_supported(const Prob &p);
+bool select_mma_supported(const Prob &p);
+cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
+                                 const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
+                                 uint32_t *status, cudaStream_t st);
 AttTcLayout attend_tc_layout(const Prob &p);
 int attend_tc_launches(const AttTcLayout &L);
 cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,

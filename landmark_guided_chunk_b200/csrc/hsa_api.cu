@@ -25,6 +25,7 @@ hsa_status_t cuda_fail(cudaError_t e, const char *what) {
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+
 WsLayout ws_layout(const Prob &p) {
     WsLayout w{};
     size_t off = 0;
@@ -35,13 +36,29 @@ WsLayout ws_layout(const Prob &p) {
     };
     const size_t rows = (size_t)p.rows;
     w.hdr = take(256);
+    // Many rows: tensor-core scoring.  Few rows with long scans: split each
+    // row's chunk range over CTAs (in bf16 with G <= 8, with tensor-core tile
+    // scores and the merge folded into the scan kernel).  Otherwise one warp
+    // per row.
+    w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(p);
+    w.split_select = !w.tc_select && rows > 0 && rows <= 4096 && p.C >= 2048;
+    w.mma_select = w.split_select && !(p.flags & HSA_FLAG_SIMT) && select_mma_supported(p);
+    // Few rows: the kept slots are spread over CTAs too (split attend); in bf16
+    // the gather kernel does it in one launch.
+    w.split_attend = rows > 0 && rows <= 2048;
+    w.gather_attend = w.split_attend && !(p.flags & HSA_FLAG_SIMT) && attend_gather_supported(p);
+    // Per-row completion counters and fp32 accumulators of those single-launch
+    // kernels sit right after the header, so that the one memset of the status
+    // word that starts every call clears them too.
+    if (w.mma_select) w.sel_cnt = take(rows * sizeof(int32_t));
+    if (w.gather_attend) {
+        w.att_cnt = take(rows * sizeof(int32_t));
+        w.att_acc = take(rows * (size_t)p.G * p.d * sizeof(float));
+    }
+    w.clear_bytes = off > 256 ? off : sizeof(uint32_t);
     w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
     w.sel_score = take(rows * p.kmax * sizeof(float));
     w.sel_keff = take(rows * sizeof(int32_t));
-    // Many rows: tensor-core scoring.  Few rows with long scans: split each
-    // row's chunk range over CTAs.  Otherwise one warp per row.
-    w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(p);
-    w.split_select = !w.tc_select && rows > 0 && rows <= 4096 && p.C >= 2048;
     if (w.split_select) {
         const long long target = 148 * 8;
         long long per_row = (target + (long long)rows - 1) / (long long)rows;
@@ -52,11 +69,9 @@ WsLayout ws_layout(const Prob &p) {
         w.nsplit = (int)(((long long)p.C + cps - 1) / cps);
         w.split_lists = take(rows * (size_t)w.nsplit * p.kmax * sizeof(float2));
     }
-    // Many rows: chunk-major tensor-core attention.  Few rows: parallelise the
-    // CUDA-core attention over the kept slots too.
-    w.split_attend = rows > 0 && rows <= 2048;
+    // Many rows: chunk-major tensor-core attention.
     w.tc_attend = !w.split_attend && rows > 0 && !(p.flags & HSA_FLAG_SIMT) && attend_tc_supported(p);
-    if (w.split_attend) w.partials = take(rows * (size_t)p.kmax * p.G * p.d * sizeof(float));
+    if (w.split_attend && !w.gather_attend) w.partials = take(rows * (size_t)p.kmax * p.G * p.d * sizeof(float));
     if (w.tc_attend) {
         w.att = attend_tc_layout(p);
         w.att_w8 = take(rows * p.kmax * sizeof(float));
@@ -76,12 +91,14 @@ WsLayout ws_layout(const Prob &p) {
     w.plan.select_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_select  ? HSA_PATH_TENSOR
                          : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
-    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select ? 2 : 1);
+    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select ? 2 : 1);
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_attend  ? HSA_PATH_TENSOR
                          : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     // tensor path: count, scan (2 levels), tile list, scatter, one main kernel per phase batch + 1
-    w.plan.attend_kernels = rows == 0 ? 0 : (w.tc_attend ? attend_tc_launches(w.att) : (w.split_attend ? 2 : 1));
+    w.plan.attend_kernels = rows == 0 ? 0
+                            : w.tc_attend ? attend_tc_launches(w.att)
+                                          : (w.split_attend && !w.gather_attend ? 2 : 1);
     return w;
 }
 
@@ -146,8 +163,8 @@ static hsa_status_t check_ws(const WsLayout &w, void *ws, size_t ws_bytes) {
     return HSA_OK;
 }
 
-static hsa_status_t clear_status(char *ws, cudaStream_t st) {
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), st);
+static hsa_status_t clear_status(char *ws, const WsLayout &w, cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, w.clear_bytes, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "clearing the device-status word");
 }
 
@@ -213,7 +230,7 @@ hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L,
     const WsLayout w = ws_layout(p);
     HSA_TRY(check_ws(w, ws, ws_bytes));
     cudaStream_t st = (cudaStream_t)stream;
-    HSA_TRY(clear_status((char *)ws, st));
+    HSA_TRY(clear_status((char *)ws, w, st));
     cudaError_t e = launch_select(p, w, Q, L, idx, score, keff, (char *)ws, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "selection kernel launch");
 }
@@ -233,7 +250,7 @@ hsa_status_t hsa_attend(const hsa_problem_t *prob, const void *Q, const void *K,
     const WsLayout w = ws_layout(p);
     HSA_TRY(check_ws(w, ws, ws_bytes));
     cudaStream_t st = (cudaStream_t)stream;
-    HSA_TRY(clear_status((char *)ws, st));
+    HSA_TRY(clear_status((char *)ws, w, st));
     cudaError_t e = launch_attend(p, w, Q, K, V, idx, score, keff, O, (char *)ws, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "attention kernel launch");
 }
@@ -259,7 +276,7 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     HSA_TRY(check_ws(w, ws, ws_bytes));
     cudaStream_t st = (cudaStream_t)stream;
     char *wsb = (char *)ws;
-    HSA_TRY(clear_status(wsb, st));
+    HSA_TRY(clear_status(wsb, w, st));
     cudaError_t e;
     if (!ready) {
         e = launch_landmarks(p, K, W_L, L, st);
@@ -287,6 +304,9 @@ hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device-status word");
     if (word & DEV_TIMEOUT) return fail(HSA_ERR_TIMEOUT, "device-status word 0x%x: a bounded device wait expired", word);
+    if (word & DEV_INTERNAL)
+        return fail(HSA_ERR_CUDA, "device-status word 0x%x: a kernel's internal index check failed (the access was "
+                    "skipped; results of that call are incomplete)", word);
     return fail(HSA_ERR_INVALID_ARG, "device-status word 0x%x: hsa_attend got a keff or chunk index outside "
                 "its row's candidates (those slots were skipped)", word);
 }

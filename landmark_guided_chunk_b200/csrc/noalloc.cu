@@ -54,17 +54,24 @@ extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, co
     if ((s = need(score, rows, "score")) != HSA_OK) return s;
     if ((s = need(keff, rows, "keff")) != HSA_OK) return s;
     // The selection stage needs the status word and, on the split path, the
-    // per-split candidate lists; nothing else of the full workspace layout.
+    // per-row counters of the tensor-core scan and the per-split candidate
+    // lists; nothing else of the full workspace layout.
     const WsLayout full = ws_layout(p);
     WsLayout w{};
     w.tc_select = full.tc_select;
     w.split_select = full.split_select;
+    w.mma_select = full.mma_select;
     w.nsplit = full.nsplit;
     w.chunks_per_split = full.chunks_per_split;
     w.hdr = 0;
-    w.split_lists = 256;
+    // after the status word: the per-row counters of the split scan (zeroed
+    // with it), then the per-split candidate lists
+    const size_t counters =
+        w.mma_select ? (((size_t)p.rows * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
+    w.sel_cnt = 256;
+    w.split_lists = 256 + counters;
     const size_t lists = w.split_select ? (size_t)p.rows * w.nsplit * p.kmax * sizeof(float2) : 0;
-    const size_t needed = 256 + lists;
+    const size_t needed = 256 + counters + lists;
     if (needed > NOALLOC_BYTES)
         return fail(HSA_ERR_WORKSPACE,
                     "hsa_select_noalloc: this problem needs %zu bytes of scratch; the static scratch holds %zu "
@@ -74,7 +81,8 @@ extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, co
     void *scratch = nullptr;
     if ((s = scratch_on_current_device(&scratch)) != HSA_OK) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(uint32_t), st);   // status word starts clear
+    // status word (and the split scan's counters) start clear
+    cudaError_t e = cudaMemsetAsync(scratch, 0, counters ? 256 + counters : sizeof(uint32_t), st);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch status word");
     e = launch_select(p, w, Q, L, idx, score, keff, (char *)scratch, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "selection kernel launch");

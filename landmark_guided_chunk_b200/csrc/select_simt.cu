@@ -15,6 +15,10 @@
 //                           8 warps and emitting one merged list (decode: few
 //                           rows, very long scans).
 //  * select_merge_kernel  : one warp per row merges the split lists.
+//  * select_split_mma_kernel : the split scan for bf16 with G <= 8, scoring 16
+//                           chunks per tensor-core instruction; the CTA that
+//                           completes a row's last split merges the row, so
+//                           there is no separate merge launch.
 #include "common.cuh"
 
 namespace hsa {
@@ -117,6 +121,74 @@ __device__ __forceinline__ void scan_range_fast(const float *qs, const T *Lj, co
     else scan_range(qs, Lj, a, c0, c1, step, v, id, lane);
 }
 
+// ---------------------------------------------------------------------------- tensor-core scan (bf16)
+// Scores of 16 consecutive chunks for the whole GQA group with mma.sync
+// m16n8k16: A = 16 landmark rows (M = chunk, K = d), B = the group's query
+// heads (K = d, N = head, G <= 8 of the 8 columns; the others zero), fp32
+// accumulation.  Each product is exact, and the group score is the fp32 sum
+// of a row's head columns.  Because the contraction runs over d in any order,
+// the k index is permuted so that every fragment a lane needs is one 16-byte
+// piece of a row: lane (r, q) = (lane/4, lane%4) reads d = 32p + 8q .. +7 of
+// landmark rows r and r+8 (A) and of head r (B) for k-steps 2p and 2p+1.
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Group scores of chunks cb .. cb+15 of Lj (rows >= c_end read as zero): on
+// return every lane of quad r holds chunk cb+r in s0 and chunk cb+r+8 in s1.
+template <int D>
+__device__ __forceinline__ void tile_scores(const __nv_bfloat16 *Lj, int cb, int c_end, const uint4 (&bq)[D / 32],
+                                            float &s0, float &s1) {
+    const int lane = threadIdx.x & 31, r = lane >> 2, q = lane & 3;
+    const bool ra = cb + r < c_end, rb = cb + r + 8 < c_end;
+    uint4 ua[D / 32], ub[D / 32];
+#pragma unroll
+    for (int p = 0; p < D / 32; ++p) {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        ua[p] = ra ? __ldg(reinterpret_cast<const uint4 *>(Lj + (size_t)(cb + r) * D + 32 * p + 8 * q)) : z;
+        ub[p] = rb ? __ldg(reinterpret_cast<const uint4 *>(Lj + (size_t)(cb + r + 8) * D + 32 * p + 8 * q)) : z;
+    }
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int p = 0; p < D / 32; ++p) {
+        mma_16816(c, ua[p].x, ub[p].x, ua[p].y, ub[p].y, bq[p].x, bq[p].y);
+        mma_16816(c, ua[p].z, ub[p].z, ua[p].w, ub[p].w, bq[p].z, bq[p].w);
+    }
+    s0 = c[0] + c[1];
+    s1 = c[2] + c[3];
+    s0 += __shfl_xor_sync(FULL, s0, 1);
+    s1 += __shfl_xor_sync(FULL, s1, 1);
+    s0 += __shfl_xor_sync(FULL, s0, 2);
+    s1 += __shfl_xor_sync(FULL, s1, 2);
+}
+
+// Scan chunks [c0, c1) of Lj into the warp list, 32 chunks per offer.
+template <int D>
+__device__ __forceinline__ void scan_range_mma(const uint4 (&bq)[D / 32], const __nv_bfloat16 *Lj, const SelArgs &a,
+                                               int c0, int c1, float &v, int &id, int lane) {
+    for (int base = c0; base < c1; base += 32) {
+        float s00, s01, s10, s11;
+        tile_scores<D>(Lj, base, c1, bq, s00, s01);
+        tile_scores<D>(Lj, base + 16, c1, bq, s10, s11);
+        // chunk base + lane: tile lane/16, half (lane/8)&1, row lane%8, held by lane 4*(lane%8)
+        const int src = 4 * (lane & 7);
+        const float x00 = __shfl_sync(FULL, s00, src), x01 = __shfl_sync(FULL, s01, src);
+        const float x10 = __shfl_sync(FULL, s10, src), x11 = __shfl_sync(FULL, s11, src);
+        const float mine = lane < 16 ? (lane < 8 ? x00 : x01) : (lane < 24 ? x10 : x11);
+        const int c = base + lane;
+        if (a.kmax <= 16)
+            list_offer16(v, id, mine, c, c < c1, a.kmax, lane);
+        else
+            list_offer(v, id, mine, c, c < c1, a.kmax, lane);
+    }
+}
+
 __device__ __forceinline__ void write_row(const SelArgs &a, long long row, float v, int id, int ke, int32_t *idx,
                                           float *score, int32_t *keff, int lane) {
     if (lane < a.kmax) {
@@ -188,6 +260,100 @@ __global__ void __launch_bounds__(256) select_split_kernel(const T *__restrict__
     }
 }
 
+// Merge a warp-list set: n entries (v, id) from src (global, read through L2)
+// into the warp list, then write the row (lane k < kmax holds entry k).
+__device__ __forceinline__ void merge_lists_to_row(const float2 *src, int n, const SelArgs &a, long long row,
+                                                   int ncand, int32_t *idx, float *score, int32_t *keff, int lane) {
+    float v;
+    int id;
+    list_init(v, id);
+    if (a.kmax <= 16) {   // n / kmax sorted lists: bitonic merges, one list at a time
+        for (int base = 0; base < n; base += a.kmax) {
+            const float2 x = lane < a.kmax ? __ldcg(src + base + lane) : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+            list_merge16(v, id, x.x, __float_as_int(x.y), a.kmax, lane);
+        }
+        write_row(a, row, v, id, list_keff(v, ncand, a.k, a.kmax, a.tau), idx, score, keff, lane);
+        return;
+    }
+    for (int base = 0; base < n; base += 32) {
+        const int e = base + lane;
+        const float2 x = e < n ? __ldcg(src + e) : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+        const int xi = __float_as_int(x.y);
+        list_offer(v, id, x.x, xi, xi != INT32_MAX, a.kmax, lane);
+    }
+    write_row(a, row, v, id, list_keff(v, ncand, a.k, a.kmax, a.tau), idx, score, keff, lane);
+}
+
+// Decode scan, bf16, G <= 8: one CTA = one (split, row); each warp scans a
+// contiguous part of the split's range with the tensor-core tile scores, the
+// warp lists are merged into the split's list, and the CTA that completes the
+// row's last split (per-row counter, zeroed with the status word) merges the
+// row's split lists and writes the row's selection.
+template <int D>
+__global__ void __launch_bounds__(256) select_split_mma_kernel(const __nv_bfloat16 *__restrict__ Q,
+                                                               const __nv_bfloat16 *__restrict__ L,
+                                                               float2 *__restrict__ lists, int32_t *__restrict__ idx,
+                                                               float *__restrict__ score, int32_t *__restrict__ keff,
+                                                               int32_t *__restrict__ cnt, SelArgs a,
+                                                               int chunks_per_split, int nsplit) {
+    __shared__ float2 wl[8 * MAX_KMAX];
+    __shared__ int s_last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = blockIdx.y;
+    const int split = blockIdx.x;
+    int b, t, j;
+    row_coords(a, row, b, t, j);
+    const int ncand = row_ncand(a, t);
+    const int c0 = split * chunks_per_split;
+    const int c1 = min(ncand, c0 + chunks_per_split);
+    float v;
+    int id;
+    list_init(v, id);
+    if (c0 < c1) {
+        // the group's query heads as B fragments (head lane/4; heads >= G are zero)
+        uint4 bq[D / 32];
+        const int hr = lane >> 2, q = lane & 3;
+        const __nv_bfloat16 *qh = Q + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + hr) * D;
+#pragma unroll
+        for (int p = 0; p < D / 32; ++p)
+            bq[p] = hr < a.G ? __ldg(reinterpret_cast<const uint4 *>(qh + 32 * p + 8 * q)) : make_uint4(0u, 0u, 0u, 0u);
+        const int per = ((c1 - c0 + 8 * 32 - 1) / (8 * 32)) * 32;   // a multiple of 32 per warp
+        const int w0 = c0 + warp * per, w1 = min(c1, w0 + per);
+        const __nv_bfloat16 *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * D;
+        if (w0 < w1) scan_range_mma<D>(bq, Lj, a, w0, w1, v, id, lane);
+    }
+    if (lane < a.kmax) wl[warp * a.kmax + lane] = make_float2(v, __int_as_float(id));
+    __syncthreads();
+    if (warp == 0) {
+        float mv;
+        int mid;
+        list_init(mv, mid);
+        const int n = 8 * a.kmax;
+        if (a.kmax <= 16) {   // eight sorted lists: bitonic merges
+            for (int w2 = 0; w2 < 8; ++w2) {
+                const float2 x = lane < a.kmax ? wl[w2 * a.kmax + lane] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+                list_merge16(mv, mid, x.x, __float_as_int(x.y), a.kmax, lane);
+            }
+        } else {
+            for (int base = 0; base < n; base += 32) {
+                const int e = base + lane;
+                const float2 x = e < n ? wl[e] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+                const int xi = __float_as_int(x.y);
+                list_offer(mv, mid, x.x, xi, xi != INT32_MAX, a.kmax, lane);
+            }
+        }
+        if (lane < a.kmax) lists[(row * nsplit + split) * a.kmax + lane] = make_float2(mv, __int_as_float(mid));
+        __threadfence();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&cnt[row], 1) == nsplit - 1;
+    __syncthreads();
+    if (s_last && warp == 0) {
+        __threadfence();
+        merge_lists_to_row(lists + row * nsplit * a.kmax, nsplit * a.kmax, a, row, ncand, idx, score, keff, lane);
+    }
+}
+
 __global__ void __launch_bounds__(256) select_merge_kernel(const float2 *__restrict__ lists, int32_t *__restrict__ idx,
                                                            float *__restrict__ score, int32_t *__restrict__ keff,
                                                            SelArgs a, int nsplit) {
@@ -231,6 +397,18 @@ template <typename T>
 cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx, float *score,
                          int32_t *keff, char *ws, cudaStream_t st) {
     SelArgs a = make_args(p);
+    if (w.split_select && w.mma_select) {
+        float2 *lists = reinterpret_cast<float2 *>(ws + w.split_lists);
+        int32_t *cnt = reinterpret_cast<int32_t *>(ws + w.sel_cnt);
+        dim3 grid(w.nsplit, (unsigned)p.rows);
+        if (p.d == 128)
+            select_split_mma_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)L, lists,
+                                                               idx, score, keff, cnt, a, w.chunks_per_split, w.nsplit);
+        else
+            select_split_mma_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)L, lists,
+                                                              idx, score, keff, cnt, a, w.chunks_per_split, w.nsplit);
+        return cudaGetLastError();
+    }
     if (!w.split_select) {
         unsigned blocks = (unsigned)((p.rows + 7) / 8);
         select_rows_kernel<T><<<blocks, 256, 8 * p.d * sizeof(float), st>>>((const T *)Q, (const T *)L, idx, score,
@@ -249,6 +427,10 @@ cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const 
 }
 
 }  // namespace
+
+bool select_mma_supported(const Prob &p) {
+    return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && p.G <= 8 && p.kmax <= MAX_KMAX;
+}
 
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
                           float *score, int32_t *keff, char *ws, cudaStream_t st) {

@@ -102,6 +102,11 @@ def test_tensor_core_paths_are_the_ones_planned():
     assert _plan(workload("prefill_bf16"))["select"][0] == "tensor"
     assert _plan(workload("router_bf16"))["select"][0] == "tensor"
     assert _plan(SMALL[1])["select"][0] == "tensor"
+    # few rows in bf16: the single-launch slot-parallel gather kernel
+    assert tuple(_plan(workload("decode_1m"))["attend"]) == ("simt_split", 1)
+    # long decode scans in bf16: split tensor-core scan with the merge folded in
+    assert tuple(_plan(workload("decode_1m"))["select"]) == ("simt_split", 1)
+    assert tuple(_plan(DECODE_SMALL[3])["select"]) == ("simt_split", 1)
 
 
 DECODE_SMALL = [
@@ -111,7 +116,27 @@ DECODE_SMALL = [
             planted=2, name="decode_rows"),
     Problem(B=2, Tq=1, Tkv=128 * 2500, H=8, Hkv=2, d=128, S=128, k=8, tau=0.02, q_pos0=128 * 2500, dtype="bf16",
             planted=2, name="decode_router"),
+    Problem(B=2, Tq=1, Tkv=32 * 2400 + 31, H=16, Hkv=2, d=64, S=32, k=12, q_pos0=32 * 2400 + 31, dtype="bf16",
+            planted=2, name="decode_s32_g8"),
+    Problem(B=2, Tq=1, Tkv=64 * 2200 + 9, H=8, Hkv=2, d=128, S=64, k=24, q_pos0=64 * 2200 + 9, dtype="bf16",
+            planted=2, name="decode_k24"),
 ]
+
+
+# few rows (<= 2048) with Tq > 1: the slot-parallel attention, with every
+# supported (d, S) and group sizes up to 16
+FEW_ROWS = [
+    Problem(B=1, Tq=32 * 30 + 7, Tkv=32 * 30 + 7, H=16, Hkv=1, d=64, S=32, k=6, dtype="bf16", name="few_d64_s32_g16"),
+    Problem(B=2, Tq=128 * 6 + 3, Tkv=128 * 6 + 3, H=6, Hkv=1, d=128, S=128, k=3, tau=0.1, dtype="bf16",
+            name="few_d128_s128_g6"),
+    Problem(B=1, Tq=64 * 12, Tkv=64 * 12, H=8, Hkv=2, d=64, S=64, k=16, dtype="bf16", name="few_d64_s64_k_all"),
+]
+
+
+@pytest.mark.parametrize("p", FEW_ROWS, ids=lambda p: p.name)
+def test_few_rows_slot_parallel_attention(p):
+    assert p.B * p.Tq * p.Hkv <= 2048
+    run_case(p)
 
 
 @pytest.mark.parametrize("p", DECODE_SMALL, ids=lambda p: p.name)
