@@ -51,7 +51,8 @@ struct WsLayout {
     size_t clear_bytes;  // bytes from the workspace start zeroed before every call (status word, counters)
     size_t total;
     int nsplit, chunks_per_split;
-    bool split_select, mma_select, split_attend, gather_attend, tc_select, tc_attend;
+    bool split_select, mma_select, stream_select, split_attend, gather_attend, tc_select, tc_attend;
+    int stream_grid, stream_maxe;   // stream scan: CTAs and list slots per row
     AttTcLayout att;
     size_t att_w8, att_pairs, att_pair_w, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
@@ -267,6 +268,11 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
 bool attend_tc_supported(const Prob &p);
 bool attend_gather_supported(const Prob &p);
 bool select_mma_supported(const Prob &p);
+bool select_stream_supported(const Prob &p);
+void select_stream_shape(const Prob &p, int sms, int *grid, int *maxe);
+cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
+                                 int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
+                                 cudaStream_t st);
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
                                  const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
                                  uint32_t *status, cudaStream_t st);

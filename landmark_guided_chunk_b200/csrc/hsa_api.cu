@@ -25,6 +25,18 @@ hsa_status_t cuda_fail(cudaError_t e, const char *what) {
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// SMs of the current device (148 if it cannot be queried); kernels sized by it
+// and their workspace layouts use the same value.
+static int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return sms;
+}
+
 
 WsLayout ws_layout(const Prob &p) {
     WsLayout w{};
@@ -37,12 +49,15 @@ WsLayout ws_layout(const Prob &p) {
     const size_t rows = (size_t)p.rows;
     w.hdr = take(256);
     // Many rows: tensor-core scoring.  Few rows with long scans: split each
-    // row's chunk range over CTAs (in bf16 with G <= 8, with tensor-core tile
-    // scores and the merge folded into the scan kernel).  Otherwise one warp
-    // per row.
+    // row's chunk range over CTAs -- for decode in bf16 (one query per row,
+    // G <= 8, kmax <= 16) one CTA per SM streams its share of all rows' landmarks
+    // through a TMA ring; otherwise in bf16 with G <= 8 (split) CTAs score with
+    // the tensor cores and fold the merge in.  Otherwise one warp per row.
     w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(p);
     w.split_select = !w.tc_select && rows > 0 && rows <= 4096 && p.C >= 2048;
-    w.mma_select = w.split_select && !(p.flags & HSA_FLAG_SIMT) && select_mma_supported(p);
+    w.stream_select = w.split_select && !(p.flags & HSA_FLAG_SIMT) && select_stream_supported(p);
+    w.mma_select = w.split_select && !w.stream_select && !(p.flags & HSA_FLAG_SIMT) && select_mma_supported(p);
+    if (w.stream_select) select_stream_shape(p, device_sms(), &w.stream_grid, &w.stream_maxe);
     // Few rows: the kept slots are spread over CTAs too (split attend); in bf16
     // the gather kernel does it in one launch.
     w.split_attend = rows > 0 && rows <= 2048;
@@ -50,7 +65,7 @@ WsLayout ws_layout(const Prob &p) {
     // Per-row completion counters and fp32 accumulators of those single-launch
     // kernels sit right after the header, so that the one memset of the status
     // word that starts every call clears them too.
-    if (w.mma_select) w.sel_cnt = take(rows * sizeof(int32_t));
+    if (w.mma_select || w.stream_select) w.sel_cnt = take(rows * sizeof(int32_t));
     if (w.gather_attend) {
         w.att_cnt = take(rows * sizeof(int32_t));
         w.att_acc = take(rows * (size_t)p.G * p.d * sizeof(float));
@@ -67,7 +82,8 @@ WsLayout ws_layout(const Prob &p) {
         if (cps < 256) cps = 256;
         w.chunks_per_split = (int)cps;
         w.nsplit = (int)(((long long)p.C + cps - 1) / cps);
-        w.split_lists = take(rows * (size_t)w.nsplit * p.kmax * sizeof(float2));
+        const size_t slots = w.stream_select ? (size_t)w.stream_maxe : (size_t)w.nsplit;
+        w.split_lists = take(rows * slots * p.kmax * sizeof(float2));
     }
     // Many rows: chunk-major tensor-core attention.
     w.tc_attend = !w.split_attend && rows > 0 && !(p.flags & HSA_FLAG_SIMT) && attend_tc_supported(p);
@@ -91,7 +107,7 @@ WsLayout ws_layout(const Prob &p) {
     w.plan.select_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_select  ? HSA_PATH_TENSOR
                          : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
-    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select ? 2 : 1);
+    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select && !w.stream_select ? 2 : 1);
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_attend  ? HSA_PATH_TENSOR
                          : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);

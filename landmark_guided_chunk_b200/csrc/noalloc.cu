@@ -61,16 +61,20 @@ extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, co
     w.tc_select = full.tc_select;
     w.split_select = full.split_select;
     w.mma_select = full.mma_select;
+    w.stream_select = full.stream_select;
+    w.stream_grid = full.stream_grid;
+    w.stream_maxe = full.stream_maxe;
     w.nsplit = full.nsplit;
     w.chunks_per_split = full.chunks_per_split;
     w.hdr = 0;
     // after the status word: the per-row counters of the split scan (zeroed
     // with it), then the per-split candidate lists
     const size_t counters =
-        w.mma_select ? (((size_t)p.rows * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
+        (w.mma_select || w.stream_select) ? (((size_t)p.rows * sizeof(int32_t) + 255) & ~(size_t)255) : 0;
     w.sel_cnt = 256;
     w.split_lists = 256 + counters;
-    const size_t lists = w.split_select ? (size_t)p.rows * w.nsplit * p.kmax * sizeof(float2) : 0;
+    const size_t slots = w.stream_select ? (size_t)w.stream_maxe : (size_t)w.nsplit;
+    const size_t lists = w.split_select ? (size_t)p.rows * slots * p.kmax * sizeof(float2) : 0;
     const size_t needed = 256 + counters + lists;
     if (needed > NOALLOC_BYTES)
         return fail(HSA_ERR_WORKSPACE,

@@ -436,6 +436,10 @@ cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const
                           float *score, int32_t *keff, char *ws, cudaStream_t st) {
     if (p.rows == 0) return cudaSuccess;
     if (w.tc_select) return launch_select_tc(p, Q, L, idx, score, keff, reinterpret_cast<uint32_t *>(ws + w.hdr), st);
+    if (w.stream_select)
+        return launch_select_stream(p, Q, L, idx, score, keff, reinterpret_cast<float2 *>(ws + w.split_lists),
+                                    reinterpret_cast<int32_t *>(ws + w.sel_cnt), reinterpret_cast<uint32_t *>(ws + w.hdr),
+                                    w.stream_grid, w.stream_maxe, st);
     if (p.dtype == HSA_BF16) return launch_typed<__nv_bfloat16>(p, w, Q, L, idx, score, keff, ws, st);
     return launch_typed<float>(p, w, Q, L, idx, score, keff, ws, st);
 }

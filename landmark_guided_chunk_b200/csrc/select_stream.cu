@@ -1,0 +1,307 @@
+// select_stream.cu -- chunk selection for decode (one query per sequence over
+// a long cached context), bf16 (HSA summary page, Core Technique /
+// Implementation: score every landmark of the strictly-past chunks, keep the
+// top k; gap router from the value-of-information router page).
+//
+// The rows (b, kv head j) all have the same candidates, ncand = min(q_pos0/S, C),
+// so their landmarks form rows * ceil(ncand/64) tiles of 64 chunks.  Each
+// persistent CTA (one per SM) takes a contiguous range of those tiles:
+//   warp 6     TMA producer: streams the range's tiles (64 landmark rows x d,
+//              boxes of 64 columns with the 128-byte swizzle) through a ring
+//              of NST stages, so ~190 KB per SM are always in flight
+//   warps 0-5  consumers, tile k -> warp k % 6 (stage k % 12, so each stage
+//              has one consumer warp): the group score of 16 chunks
+//              per mma.sync m16n8k16 (A = landmark rows via ldmatrix, B = the
+//              group's query heads as columns, fp32 accumulate; the products
+//              are exact and the group score is the fp32 sum of the head
+//              columns), then a warp-wide top-k list per row: a batch of 32
+//              candidates with few qualifiers is inserted one by one, one with
+//              many is sorted by a bitonic network and merged
+// At the end each CTA merges its warps' lists per row (bitonic merges), writes
+// one list per (row, CTA), and the CTA that completes a row (per-row counter,
+// zeroed with the status word) merges the row's lists and writes its
+// selection, with the router's k_eff.
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace hsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int TCH = 64;    // chunks per tile
+constexpr int NCW = 6;     // consumer warps
+constexpr int NST = 12;    // ring stages
+constexpr int RMAX = 4;    // rows one CTA may touch
+// Tile k goes to warp k % NCW and stage k % NST.  With NST a multiple of NCW
+// every stage has a single consumer warp, which waits for the stage's phases
+// in order.  (Two warps waiting on one stage for consecutive phases would let
+// the later one see the earlier phase's parity as complete.)
+static_assert(NST % NCW == 0, "each ring stage must belong to one consumer warp");
+
+struct StreamArgs {
+    int Tq, H, Hkv, G, S, C, k, kmax;
+    int ncand, tpr;       // candidates of every row; tiles per row
+    long long total;      // rows * tpr
+    int grid, maxe;       // CTAs; list slots per row
+    float tau;
+    uint32_t *status;
+};
+
+struct __align__(8) StreamBars {
+    uint64_t full[NST], empty[NST];
+    int abort;
+};
+
+// A slot or index outside its range (which the grid sizing rules out) is
+// recorded in the status word and the access skipped.
+__device__ __forceinline__ bool in_range(long long x, long long n, uint32_t *status) {
+    if (x >= 0 && x < n) return true;
+    atomicOr(status, DEV_INTERNAL);
+    return false;
+}
+
+__device__ __forceinline__ long long cta_lo(const StreamArgs &a, int x) { return (long long)x * a.total / a.grid; }
+// the CTA whose range holds tile T
+__device__ __forceinline__ int cta_of(const StreamArgs &a, long long T) {
+    return (int)(((T + 1) * a.grid - 1) / a.total);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// 16-byte chunk j of row u in a box of 128-byte rows written with the 128-byte swizzle
+__device__ __forceinline__ uint32_t swz(uint32_t box, int u, int j) {
+    return box + (uint32_t)u * 128u + ((uint32_t)(j ^ (u & 7)) << 4);
+}
+
+template <int D>
+__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+    select_stream_kernel(const __grid_constant__ CUtensorMap tmL, const __nv_bfloat16 *__restrict__ Q,
+                         float2 *__restrict__ lists, int32_t *__restrict__ idx, float *__restrict__ score,
+                         int32_t *__restrict__ keff, int32_t *__restrict__ cnt, StreamArgs a) {
+    constexpr int NB = D / 64;          // boxes per tile
+    constexpr int BOXB = TCH * 128;     // bytes of one box
+    constexpr int STB = NB * BOXB;      // bytes of one stage
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ StreamBars bar;
+    __shared__ float2 wl[RMAX][NCW][16];   // each consumer warp's list per row slot
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int x = (int)blockIdx.x;
+    const long long lo = cta_lo(a, x), hi = cta_lo(a, x + 1);
+    const int ntile = (int)(hi - lo);
+    const long long r_lo = lo / a.tpr;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&bar.full[s], 1);
+            mbar_init(&bar.empty[s], 1);
+        }
+        bar.abort = 0;
+        fence_mbar_init();
+    }
+    for (int e = threadIdx.x; e < RMAX * NCW * 16; e += blockDim.x)
+        (&wl[0][0][0])[e] = make_float2(-INFINITY, __int_as_float(INT32_MAX));
+    __syncthreads();
+
+    if (warp == NCW) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int k = 0;
+            for (; k < ntile; ++k) {
+                const int s = k % NST, u = k / NST;
+                if (u > 0 && !(ok = mbar_wait(&bar.empty[s], (u - 1) & 1, &bar.abort, a.status))) break;
+                const long long T = lo + k, row = T / a.tpr;
+                const int y = (int)(row * a.C + (T % a.tpr) * TCH);
+                mbar_expect_tx(&bar.full[s], (uint32_t)STB);
+#pragma unroll
+                for (int kb = 0; kb < NB; ++kb)
+                    tma_load_2d(base + (size_t)s * STB + kb * BOXB, &tmL, 64 * kb, y, &bar.full[s]);
+            }
+            // every load issued has landed before the CTA may exit
+            for (int s = 0; s < NST && s < k; ++s) mbar_drain(&bar.full[s], ((k - 1 - s) / NST) & 1);
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const int r4 = lane >> 2, q2 = 2 * (lane & 3);
+        const int mi = lane >> 3, r8 = lane & 7;   // ldmatrix: this lane addresses row r8 of matrix mi
+        uint32_t bq[D / 16][2];
+        long long cur = -1;
+        float v;
+        int id;
+        list_init(v, id);
+        for (int k = warp; k < ntile; k += NCW) {
+            const int s = k % NST, u = k / NST;
+            const long long T = lo + k, row = T / a.tpr;
+            const int kt = (int)(T % a.tpr);
+            if (row != cur) {
+                if (cur >= 0 && lane < 16 && in_range(cur - r_lo, RMAX, a.status))
+                    wl[cur - r_lo][warp][lane] = make_float2(v, __int_as_float(id));
+                list_init(v, id);
+                cur = row;
+                // the group's query heads as B columns (head lane/4; heads >= G are zero)
+                const int j = (int)(row % a.Hkv), b = (int)(row / a.Hkv);
+                const __nv_bfloat16 *qh = Q + (((size_t)b * a.Tq) * a.H + (size_t)j * a.G + r4) * D;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    bq[ks][0] = r4 < a.G ? *reinterpret_cast<const uint32_t *>(qh + 16 * ks + q2) : 0u;
+                    bq[ks][1] = r4 < a.G ? *reinterpret_cast<const uint32_t *>(qh + 16 * ks + 8 + q2) : 0u;
+                }
+            }
+            if (!mbar_wait(&bar.full[s], u & 1, &bar.abort, a.status)) break;
+            const uint32_t st = smem_u32(base + (size_t)s * STB);
+            float sc[TCH / 16][2];
+#pragma unroll
+            for (int mt = 0; mt < TCH / 16; ++mt) {
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(swz(st + (uint32_t)(ks / 4) * BOXB, 16 * mt + 8 * (mi & 1) + r8, 2 * (ks % 4) + (mi >> 1)),
+                            a0, a1, a2, a3);
+                    mma16816(c, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+                }
+                float s0 = c[0] + c[1], s1 = c[2] + c[3];
+                s0 += __shfl_xor_sync(FULL, s0, 1);
+                s1 += __shfl_xor_sync(FULL, s1, 1);
+                s0 += __shfl_xor_sync(FULL, s0, 2);
+                s1 += __shfl_xor_sync(FULL, s1, 2);
+                sc[mt][0] = s0;   // chunk 16*mt + r4
+                sc[mt][1] = s1;   // chunk 16*mt + r4 + 8
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.empty[s]);   // the stage may be refilled
+            // two offers of 32 chunks: chunk 32h + L sits in m-tile 2h + L/16, half (L/8)&1, quad L%8
+            const int src = 4 * (lane & 7);
+#pragma unroll
+            for (int h = 0; h < TCH / 32; ++h) {
+                const float x0 = __shfl_sync(FULL, sc[2 * h][0], src), x1 = __shfl_sync(FULL, sc[2 * h][1], src);
+                const float x2 = __shfl_sync(FULL, sc[2 * h + 1][0], src), x3 = __shfl_sync(FULL, sc[2 * h + 1][1], src);
+                const float mine = lane < 16 ? (lane < 8 ? x0 : x1) : (lane < 24 ? x2 : x3);
+                const int c = kt * TCH + 32 * h + lane;
+                list_offer16(v, id, mine, c, c < a.ncand, a.kmax, lane);
+            }
+        }
+        if (cur >= 0 && lane < 16 && in_range(cur - r_lo, RMAX, a.status))
+            wl[cur - r_lo][warp][lane] = make_float2(v, __int_as_float(id));
+    }
+    __syncthreads();
+
+    // ---- per row slot: merge the consumer warps' lists, publish the CTA's list;
+    // the CTA that completes the row merges the row's lists and writes the row
+    if (ntile == 0 || bar.abort) return;
+    const int nrows = (int)((hi - 1) / a.tpr - r_lo + 1);
+    if (warp >= nrows || !in_range(warp, RMAX, a.status)) return;
+    const long long row = r_lo + warp;
+    float v = lane < 16 ? wl[warp][0][lane].x : -INFINITY;
+    int id = lane < 16 ? __float_as_int(wl[warp][0][lane].y) : INT32_MAX;
+    if (lane >= a.kmax) {
+        v = -INFINITY;
+        id = INT32_MAX;
+    }
+    for (int w2 = 1; w2 < NCW; ++w2) {
+        const float2 e = lane < 16 ? wl[warp][w2][lane] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+        list_merge16(v, id, e.x, __float_as_int(e.y), a.kmax, lane);
+    }
+    const long long T0 = row * a.tpr;
+    const int x0 = cta_of(a, T0), x1 = cta_of(a, T0 + a.tpr - 1);
+    float2 *rl = lists + row * (long long)a.maxe * a.kmax;
+    if (!in_range(x - x0, a.maxe, a.status) || !in_range(x1 - x0, a.maxe, a.status)) return;
+    if (lane < a.kmax) rl[(x - x0) * a.kmax + lane] = make_float2(v, __int_as_float(id));
+    __threadfence();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&cnt[row], 1) == x1 - x0;
+    if (!__shfl_sync(FULL, last, 0)) return;
+    __threadfence();
+    list_init(v, id);
+    for (int e = 0; e <= x1 - x0; ++e) {
+        const float2 f = lane < a.kmax ? __ldcg(rl + e * a.kmax + lane) : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+        list_merge16(v, id, f.x, __float_as_int(f.y), a.kmax, lane);
+    }
+    const int ke = list_keff(v, a.ncand, a.k, a.kmax, a.tau);
+    if (lane < a.kmax) {
+        idx[row * a.kmax + lane] = lane < ke ? id : -1;
+        score[row * a.kmax + lane] = lane < ke ? v : -INFINITY;
+    }
+    if (lane == 0) keff[row] = ke;
+}
+
+}  // namespace
+
+// Decode-shaped problems (one query per sequence) with long contexts.
+bool select_stream_supported(const Prob &p) {
+    const long long ncand = std::min<long long>(p.q_pos0 / p.S, p.C);
+    return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && p.Tq == 1 && p.G <= 8 && p.kmax <= 16 &&
+           ncand >= 2048 && (long long)p.B * p.Hkv * p.C < (1ll << 31);
+}
+
+// Grid and list slots of the stream scan (also sizes its workspace).
+void select_stream_shape(const Prob &p, int sms, int *grid, int *maxe) {
+    const long long ncand = std::min<long long>(p.q_pos0 / p.S, p.C);
+    const long long tpr = (ncand + TCH - 1) / TCH, total = p.rows * tpr;
+    long long g = sms;
+    // a CTA's range may touch at most RMAX rows: at most (RMAX - 1) * tpr + 1 tiles
+    const long long need = (total + (RMAX - 1) * tpr) / ((RMAX - 1) * tpr + 1);
+    if (g < need) g = need;
+    if (g > total) g = total;
+    const long long minn = total / g;   // tiles of the smallest range (>= 1)
+    long long e = tpr / minn + 2;
+    if (e > g) e = g;
+    *grid = (int)g;
+    *maxe = (int)e;
+}
+
+cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
+                                 int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
+                                 cudaStream_t st) {
+    StreamArgs a;
+    a.Tq = p.Tq;
+    a.H = p.H;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.S = p.S;
+    a.C = p.C;
+    a.k = p.k;
+    a.kmax = p.kmax;
+    a.ncand = (int)std::min<long long>(p.q_pos0 / p.S, p.C);
+    a.tpr = (a.ncand + TCH - 1) / TCH;
+    a.total = p.rows * (long long)a.tpr;
+    a.grid = grid;
+    a.maxe = maxe;
+    a.tau = p.tau;
+    a.status = status;
+    CUtensorMap ml;
+    cudaError_t e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.C, 64, TCH);
+    if (e != cudaSuccess) return e;
+    const size_t smem = 1024 + (size_t)NST * (p.d / 64) * TCH * 128;
+    if (p.d == 128) {
+        if ((e = cudaFuncSetAttribute(select_stream_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        select_stream_kernel<128><<<grid, (NCW + 1) * 32, smem, st>>>(ml, (const __nv_bfloat16 *)Q, lists, idx, score,
+                                                                      keff, cnt, a);
+    } else {
+        if ((e = cudaFuncSetAttribute(select_stream_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        select_stream_kernel<64><<<grid, (NCW + 1) * 32, smem, st>>>(ml, (const __nv_bfloat16 *)Q, lists, idx, score,
+                                                                     keff, cnt, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace hsa
