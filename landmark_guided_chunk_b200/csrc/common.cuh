@@ -213,10 +213,13 @@ __device__ __forceinline__ void list_merge16(float &v, int &id, float bv, int bi
 
 // Offer one candidate per lane (valid lanes only), kmax <= 16: few qualifying
 // candidates are inserted one by one; many are sorted as a batch and merged.
-__device__ __forceinline__ void list_offer16(float &v, int &id, float s, int c, bool valid, int kmax, int lane) {
+// `floor`: candidates scoring below it are known to be out of the row's top k
+// (another list already holds k entries at or above it), so they are skipped.
+__device__ __forceinline__ void list_offer16(float &v, int &id, float s, int c, bool valid, int kmax, int lane,
+                                             float floor = -INFINITY) {
     const float vl = __shfl_sync(FULL, v, kmax - 1);
     const int il = __shfl_sync(FULL, id, kmax - 1);
-    const bool pass = valid && ranks_before(s, c, vl, il);
+    const bool pass = valid && s >= floor && ranks_before(s, c, vl, il);
     unsigned m = __ballot_sync(FULL, pass);
     if (__popc(m) <= 3) {
         while (m) {

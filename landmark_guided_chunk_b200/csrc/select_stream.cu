@@ -63,6 +63,15 @@ __device__ __forceinline__ bool in_range(long long x, long long n, uint32_t *sta
     return false;
 }
 
+// Order-preserving unsigned code of a float (for atomicMax on scores).
+__device__ __forceinline__ unsigned ord_enc(float x) {
+    const unsigned u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_dec(unsigned e) {
+    return __uint_as_float((e & 0x80000000u) ? (e & 0x7fffffffu) : ~e);
+}
+
 __device__ __forceinline__ long long cta_lo(const StreamArgs &a, int x) { return (long long)x * a.total / a.grid; }
 // the CTA whose range holds tile T
 __device__ __forceinline__ int cta_of(const StreamArgs &a, long long T) {
@@ -99,6 +108,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ StreamBars bar;
     __shared__ float2 wl[RMAX][NCW][16];   // each consumer warp's list per row slot
+    __shared__ unsigned s_floor[RMAX];     // best k-th score any warp's list has reached, per row slot
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int x = (int)blockIdx.x;
     const long long lo = cta_lo(a, x), hi = cta_lo(a, x + 1);
@@ -115,6 +125,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     }
     for (int e = threadIdx.x; e < RMAX * NCW * 16; e += blockDim.x)
         (&wl[0][0][0])[e] = make_float2(-INFINITY, __int_as_float(INT32_MAX));
+    if (threadIdx.x < RMAX) s_floor[threadIdx.x] = 0x007fffffu;   // the code of -inf
     __syncthreads();
 
     if (warp == NCW) {
@@ -185,7 +196,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar.empty[s]);   // the stage may be refilled
-            // two offers of 32 chunks: chunk 32h + L sits in m-tile 2h + L/16, half (L/8)&1, quad L%8
+            // two offers of 32 chunks: chunk 32h + L sits in m-tile 2h + L/16, half (L/8)&1, quad L%8.
+            // A candidate below another warp's k-th best for this row cannot make the row's top k.
+            const int rs = (int)(cur - r_lo);
+            const float floor = (rs >= 0 && rs < RMAX) ? ord_dec(*(volatile unsigned *)&s_floor[rs]) : -INFINITY;
             const int src = 4 * (lane & 7);
 #pragma unroll
             for (int h = 0; h < TCH / 32; ++h) {
@@ -193,8 +207,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 const float x2 = __shfl_sync(FULL, sc[2 * h + 1][0], src), x3 = __shfl_sync(FULL, sc[2 * h + 1][1], src);
                 const float mine = lane < 16 ? (lane < 8 ? x0 : x1) : (lane < 24 ? x2 : x3);
                 const int c = kt * TCH + 32 * h + lane;
-                list_offer16(v, id, mine, c, c < a.ncand, a.kmax, lane);
+                list_offer16(v, id, mine, c, c < a.ncand, a.kmax, lane, floor);
             }
+            // publish this list's k-th best once it holds k entries
+            const float vk = __shfl_sync(FULL, v, a.kmax - 1);
+            if (lane == 0 && vk != -INFINITY && rs >= 0 && rs < RMAX) atomicMax(&s_floor[rs], ord_enc(vk));
         }
         if (cur >= 0 && lane < 16 && in_range(cur - r_lo, RMAX, a.status))
             wl[cur - r_lo][warp][lane] = make_float2(v, __int_as_float(id));
