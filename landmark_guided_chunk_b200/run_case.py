@@ -4,6 +4,11 @@ Used to drive profilers on a single, small, reproducible case:
 
     python -m landmark_guided_chunk_b200.run_case --workload prefill_bf16 --T 16384 --iters 3
     python -m landmark_guided_chunk_b200.run_case --workload decode_1m --B 2 --ctx 262144 --iters 3
+    python -m landmark_guided_chunk_b200.run_case --workload decode_1m --select-only --iters 3
+
+--select-only runs the selection stage alone on the workload's query shapes and
+random landmarks, with no K/V allocated (the decode_1m selection then needs
+0.25 GiB on the device instead of 32 GiB).
 
 Prints the per-stage kernel paths and the wall time of the last iteration.
 """
@@ -18,6 +23,24 @@ import landmark_guided_chunk_b200 as hsa
 from landmark_guided_chunk_b200.inputs import make_inputs, workload
 
 
+def select_only(p, args):
+    g = torch.Generator(device="cuda").manual_seed(0)
+    dt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+    Q = torch.randn(p.B, p.Tq, p.H, p.d, device="cuda", generator=g).to(dt)
+    L = (torch.randn(p.B, p.Hkv, p.C, p.d, device="cuda", generator=g) / 8).to(dt)
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, dt,
+                            hsa._native.HSA_FLAG_SIMT if args.simt else 0)
+    ws = hsa.alloc_workspace(prob)
+    for _ in range(args.iters):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        hsa.select(Q, L, p.S, p.k, p.tau, p.q_pos0, Tkv=p.Tkv, ws=ws, force_simt=args.simt)
+        torch.cuda.synchronize()
+        dt_s = time.perf_counter() - t0
+    hsa.device_status(ws)
+    print(f"{p.name} (select only): B{p.B} Tq{p.Tq} Tkv{p.Tkv} plan={hsa.plan(prob)} last={dt_s * 1e3:.3f} ms")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="prefill_bf16")
@@ -26,6 +49,7 @@ def main():
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--simt", action="store_true", help="CUDA-core kernels only")
+    ap.add_argument("--select-only", action="store_true", help="selection stage only, random landmarks, no K/V")
     args = ap.parse_args()
     p = workload(args.workload)
     if args.B is not None:
@@ -35,6 +59,9 @@ def main():
     if args.ctx is not None:
         p = p.with_(Tkv=args.ctx, q_pos0=args.ctx)
     torch.cuda.set_device(0)
+    if args.select_only:
+        select_only(p, args)
+        return
     inp = make_inputs(p, seed=0, device="cuda")
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
     ready = p.is_decode
