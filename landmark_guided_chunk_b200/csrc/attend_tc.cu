@@ -224,7 +224,7 @@ constexpr int NINFO = 4;   // tiles of row info (token, weight) the producers ma
 
 struct TileRows {            // one tile's row info, written by the producers, read by the epilogue
     int p, n;
-    int t[MROWS];            // token of each row (-1: padding row)
+    int off[MROWS];          // row's float offset in its phase's accumulator slot (-1: padding row)
     float w[MROWS];          // fusion weight of each row's (token, slot) pair
 };
 
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                     ri.p = T.p;
                     ri.n = T.n;
                 }
-                ri.t[r] = valid ? (pr >> 5) : -1;
+                ri.off[r] = valid ? (((pr >> 5) - (T.p % a.ntb) * TB) * a.G + g) * D : -1;
                 ri.w[r] = valid ? pw : 0.f;
                 mbar_arrive(&bar->info_full[si]);
             }
@@ -518,11 +518,15 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             const int si = i % NINFO;
             if (!(ok = mbar_wait(&bar->info_full[si], (i / NINFO) & 1, abort, a.status))) break;
             const int Tp = info[si].p;
-            const int t = info[si].t[r];
+            const int myoff = info[si].off[r];
             const float w = info[si].w[r];
+            // destinations of the staging rows this lane will reduce (rows rr*4 + lane/8 of the warp)
+            int dstoff[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) dstoff[rr] = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->info_empty[si]);
-            const bool valid = t >= 0;
+            const bool valid = myoff >= 0;
             // chunk softmax: S row -> P row (bf16, swizzled), l
             if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
@@ -567,18 +571,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
             tc_fence_after();
             const float f = valid ? w / l : 0.f;
-            const int tloc_base = (Tp % a.ntb) * TB;
-            float *acc_slot = slot_of(a, Tp);
-            // destination row of each staging row this lane reduces (rows rr*4 + lane/8)
-            float *dstrow[8];
-#pragma unroll
-            for (int rr = 0; rr < 8; ++rr) {
-                const int lr = rr * 4 + (lane >> 3);
-                const int tt = __shfl_sync(FULL, t, lr);
-                const int R = ew * 32 + lr;
-                dstrow[rr] = tt >= 0 ? acc_slot + ((size_t)(tt - tloc_base) * a.G + (R % a.G)) * D + 4 * (lane & 7)
-                                     : nullptr;
-            }
+            float *acc_slot = slot_of(a, Tp) + 4 * (lane & 7);
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t orr[32];
                 tmem_ld32(lane_base + 128 + q * 32, orr);
@@ -597,9 +590,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 __syncwarp();
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                    if (dstrow[rr]) {
+                    if (dstoff[rr] >= 0) {
                         const int lr = rr * 4 + (lane >> 3);
-                        red_add_v4(dstrow[rr] + q * 32, *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
+                        red_add_v4(acc_slot + dstoff[rr] + q * 32,
+                                   *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
                     }
                 }
                 __syncwarp();
