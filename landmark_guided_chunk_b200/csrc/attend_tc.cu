@@ -10,9 +10,15 @@
 // up to TOK = 128/G tokens.  The G heads of each token form the 128-row M
 // operand:
 //     S  = Q_tile . K_c^T / sqrt(d)        tcgen05, M128 x N=S x K=d, TMEM
-//     P  = exp(S - rowmax), l = sum P      epilogue warps, P -> smem (bf16)
+//     P  = exp(S - rowmax), l = sum P      softmax warps, P -> smem (bf16)
 //     O  = P . V_c                          tcgen05, M128 x N=d x K=S, TMEM
-//     O_acc[t][h] += (w_slot / l) * O       fp32 vector reductions (red.v4)
+//     O_acc[t][h] += (w_slot / l) * O       O-drain warps, fp32 vector reductions (red.v4)
+// Roles (16 warps, 4 per SM sub-partition so each may hold 128 registers):
+// two producer warps gather the tile's Q rows (cp.async) and issue the K/V TMA
+// loads, one thread issues the MMAs, four softmax warps (one per TMEM lane
+// quadrant) and eight O-drain warps (two per quadrant, 64 columns each) take
+// every tile.  S, P and O are double-buffered by tile parity, so the drain of
+// tile i overlaps the softmax of tile i+1 and the QK product of tile i+2.
 // Since w is known before the attention, the cross-chunk fusion is linear and
 // needs no rescaling.
 //
@@ -43,7 +49,8 @@ constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
 constexpr int TB = 4096;         // tokens per phase
 constexpr int NB = 2;            // phases per batch (= per launch)
-constexpr int NT_ATT = 416;      // warps 0-3 producers, 4-7 and 8-11 epilogue groups, 12 MMA
+constexpr int NT_ATT = 512;      // warps 0-1 producers, 2 MMA, 3 idle, 4-7 softmax, 8-15 O drain
+constexpr int NPROD = 64;        // producer threads (two tile rows each)
 
 struct AttTcArgs {
     int B, Tq, Tkv, H, Hkv, G, S, C, kmax, tok;
@@ -230,8 +237,9 @@ struct TileRows {            // one tile's row info, written by the producers, r
 
 struct __align__(8) AttBars {
     uint64_t q_full[2], q_empty[2], kv_full[2], kv_empty[2];
-    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2], done;
+    uint64_t s_full[2], p_full[2], p_empty[2], o_full[2], o_empty[2], l_full[2], l_empty[2], done;
     uint64_t info_full[NINFO], info_empty[NINFO];
+    float l[2][MROWS];           // softmax row sums of the tiles in the two TMEM/P buffers
     uint32_t tmem_base;
     int abort;
     int tile_lo, tile_hi;
@@ -307,11 +315,11 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.S;
     const int kv_bytes = S * 128;                          // one 64-column box of S rows
-    const int p_bytes = (S / 64) * 16384;                  // P tile of one group
+    const int p_bytes = (S / 64) * 16384;                  // one P tile
     uint8_t *sQ = base;                                    // nsq x 32 KB
     uint8_t *sKV = sQ + (size_t)a.nsq * 32768;             // nskv x (K: 2 boxes, V: 2 boxes)
-    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 groups x p_bytes
-    float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 warps x 32 x PITCH
+    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 P buffers x p_bytes
+    float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 O warps x 32 x PITCH
     TileRows *info = reinterpret_cast<TileRows *>(stg + 8 * 32 * PITCH);      // NINFO stages
     AttBars *bar = reinterpret_cast<AttBars *>(info + NINFO);
     volatile int *abort = &bar->abort;
@@ -324,18 +332,21 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar->q_full[s], 128);
+            mbar_init(&bar->q_full[s], NPROD);
             mbar_init(&bar->q_empty[s], 1);
             mbar_init(&bar->kv_full[s], 1);
             mbar_init(&bar->kv_empty[s], 1);
             mbar_init(&bar->s_full[s], 1);
             mbar_init(&bar->p_full[s], 4);
+            mbar_init(&bar->p_empty[s], 1);
             mbar_init(&bar->o_full[s], 1);
-            mbar_init(&bar->o_empty[s], 4);
+            mbar_init(&bar->o_empty[s], 8);
+            mbar_init(&bar->l_full[s], 4);
+            mbar_init(&bar->l_empty[s], 8);
         }
         for (int s = 0; s < NINFO; ++s) {
-            mbar_init(&bar->info_full[s], 128);
-            mbar_init(&bar->info_empty[s], 4);
+            mbar_init(&bar->info_full[s], NPROD);
+            mbar_init(&bar->info_empty[s], 8);
         }
         mbar_init(&bar->done, 1);
         bar->abort = 0;
@@ -344,7 +355,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
         bar->tile_hi = a.btile[p1 * a.C];
         fence_mbar_init();
     }
-    if (warp == 12) {
+    if (warp == 2) {
         tmem_alloc(&bar->tmem_base, 512);
         tmem_relinquish();
     }
@@ -352,32 +363,60 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+    // TMEM columns: S buffers at 0 and 128, O buffers at 256 and 384 (buffer = tile index & 1)
     // each CTA takes a contiguous range of the batch's tiles, so the tiles of one
     // bucket (same chunk) mostly stay together and share one K/V load
     const int per = (bar->tile_hi - bar->tile_lo + (int)gridDim.x - 1) / (int)gridDim.x;
     const int tile_lo = min(bar->tile_hi, bar->tile_lo + (int)blockIdx.x * per);
     const int tile_hi = min(bar->tile_hi, tile_lo + per);
 
-    if (warp < 4) {
-        // ------------------------------------------------------------ producers: Q gather (thread = row), K/V TMA
-        const int r = threadIdx.x;   // 0..127
-        const int m = r / a.G, g = r % a.G;
+    if (warp < 2) {
+        // ------------------------------------------------------------ producers: Q gather (rows r, r+64), K/V TMA
+        int rr[2], mm[2], gg[2], pr[2];
+        float pw[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            rr[h] = threadIdx.x + h * NPROD;
+            mm[h] = rr[h] / a.G;
+            gg[h] = rr[h] % a.G;
+        }
         int i = 0, nload = 0;
         bool ok = true;
         int tau = tile_lo;
         TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
-        int pr = (tau < tile_hi && m < T.n) ? a.pairs[T.start + m] : 0;
-        float pw = (tau < tile_hi && m < T.n) ? a.pair_w[T.start + m] : 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const bool v = tau < tile_hi && mm[h] < T.n;
+            pr[h] = v ? a.pairs[T.start + mm[h]] : 0;
+            pw[h] = v ? a.pair_w[T.start + mm[h]] : 0.f;
+        }
         int prev_p = -1, prev_c = -1;
         for (; tau < tile_hi && ok; ++i) {
             // prefetch the next tile while this one is issued
             const int tau_n = tau + 1;
             TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
+            // row info for the O drain (its slot is free once the drain of tile i - NINFO read it)
+            {
+                const int si = i % NINFO, ii = i / NINFO;
+                if (ii > 0 && !(ok = mbar_wait(&bar->info_empty[si], (ii - 1) & 1, abort, a.status))) break;
+                TileRows &ri = info[si];
+                if (threadIdx.x == 0) {
+                    ri.p = T.p;
+                    ri.n = T.n;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const bool v = mm[h] < T.n;
+                    ri.off[rr[h]] = v ? (((pr[h] >> 5) - (T.p % a.ntb) * TB) * a.G + gg[h]) * D : -1;
+                    ri.w[rr[h]] = v ? pw[h] : 0.f;
+                }
+                mbar_arrive(&bar->info_full[si]);
+            }
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
             const bool newkv = T.p != prev_p || T.c != prev_c;
             if (newkv) {
-                if (warp == 0 && lane == 0) {
+                if (threadIdx.x == 0) {
                     const int skv = nload % a.nskv, ikv = nload / a.nskv;
                     if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
                     mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
@@ -392,47 +431,42 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 prev_p = T.p;
                 prev_c = T.c;
             }
-            const bool valid = m < T.n;
-            const char *src = reinterpret_cast<const char *>(Q);
-            if (valid) {
-                const int t = pr >> 5;
-                src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + g) * D) * 2;
-            }
-            const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                const int kb = x >> 3, cx = x & 7;
-                cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
+            for (int h = 0; h < 2; ++h) {
+                const int r = rr[h];
+                const bool valid = mm[h] < T.n;
+                const char *src = reinterpret_cast<const char *>(Q);
+                if (valid) {
+                    const int t = pr[h] >> 5;
+                    src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
+                }
+                const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const int kb = x >> 3, cx = x & 7;
+                    cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
+                }
             }
             cp_async_arrive(&bar->q_full[sq]);
-            // row info for the epilogue
-            {
-                const int si = i % NINFO, ii = i / NINFO;
-                if (ii > 0 && !(ok = mbar_wait(&bar->info_empty[si], (ii - 1) & 1, abort, a.status))) break;
-                TileRows &ri = info[si];
-                if (r == 0) {
-                    ri.p = T.p;
-                    ri.n = T.n;
-                }
-                ri.off[r] = valid ? (((pr >> 5) - (T.p % a.ntb) * TB) * a.G + g) * D : -1;
-                ri.w[r] = valid ? pw : 0.f;
-                mbar_arrive(&bar->info_full[si]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const bool v = tau_n < tile_hi && mm[h] < Tn.n;
+                pr[h] = v ? a.pairs[Tn.start + mm[h]] : 0;
+                pw[h] = v ? a.pair_w[Tn.start + mm[h]] : 0.f;
             }
-            pr = (tau_n < tile_hi && m < Tn.n) ? a.pairs[Tn.start + m] : 0;
-            pw = (tau_n < tile_hi && m < Tn.n) ? a.pair_w[Tn.start + m] : 0.f;
             T = Tn;
             tau = tau_n;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-        if (warp == 0 && lane == 0) {
+        if (threadIdx.x == 0) {
             // wind down: the K/V loads issued have all landed
             for (int s = 0; s < a.nskv && s < nload; ++s)
                 mbar_drain(&bar->kv_full[s], ((nload - 1 - s) / a.nskv) & 1);
         }
-    } else if (warp == 12) {
+    } else if (warp == 2) {
         // ------------------------------------------------------------ MMA issuer
-        // With two K/V stages QK(i+1) is issued before PV(i), so the two epilogue
-        // groups' softmaxes overlap; with one stage the order is QK(i), PV(i), ...
+        // With two K/V stages QK(i+1) is issued before PV(i), so the next tile's softmax
+        // overlaps this one's PV; with one stage the order is QK(i), PV(i), ...
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
@@ -449,6 +483,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 return nload - 1;
             };
             int waited_load = -1;   // last load whose kv_full has been waited on
+            // QK(i) writes S buffer i & 1, whose previous tile (i - 2) the softmax has released
+            // through p_full before PV(i - 2) was issued, which precedes this call.
             auto issue_qk = [&](int i, int li) -> bool {
                 const int sq = i % a.nsq, iq = i / a.nsq, skv = li % a.nskv, ikv = li / a.nskv;
                 if (!mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status)) return false;
@@ -457,7 +493,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                     waited_load = li;
                 }
                 tc_fence_after();
-                const uint32_t s_tmem = tmem + (i & 1) * 256;
+                const uint32_t s_tmem = tmem + (i & 1) * 128;
                 const uint32_t qa = smem_u32(sQ + sq * 32768);
                 const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 4 * kv_bytes);
 #pragma unroll
@@ -474,15 +510,15 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             int li = n_mine > 0 ? load_of(0) : 0;
             bool ok = n_mine > 0 ? issue_qk(0, li) : true;
             for (int i = 0; i < n_mine && ok; ++i) {
-                const int gsel = i & 1, k = i >> 1;
+                const int b = i & 1, k = i >> 1;
                 const int li_next = i + 1 < n_mine ? load_of(i + 1) : -1;
                 if (early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
-                if (!(ok = mbar_wait(&bar->p_full[gsel], k & 1, abort, a.status))) break;
-                if (k > 0 && !(ok = mbar_wait(&bar->o_empty[gsel], (k - 1) & 1, abort, a.status))) break;
+                if (!(ok = mbar_wait(&bar->p_full[b], k & 1, abort, a.status))) break;
+                if (k > 0 && !(ok = mbar_wait(&bar->o_empty[b], (k - 1) & 1, abort, a.status))) break;
                 tc_fence_after();
                 const int skv = li % a.nskv;
-                const uint32_t o_tmem = tmem + gsel * 256 + 128;
-                const uint32_t pa = smem_u32(sP + gsel * p_bytes);
+                const uint32_t o_tmem = tmem + 256 + b * 128;
+                const uint32_t pa = smem_u32(sP + b * p_bytes);
                 const uint32_t vb = smem_u32(sKV + (size_t)skv * 4 * kv_bytes) + 2 * kv_bytes;
                 for (int kk = 0; kk < S / 16; ++kk) {
                     // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
@@ -493,7 +529,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                     umma_bf16(o_tmem, desc_kmajor_sw128(a_addr), desc_mnmajor_sw128(b_addr, kv_bytes, 1024), idesc_o,
                               kk != 0);
                 }
-                umma_commit(&bar->o_full[gsel]);
+                umma_commit(&bar->o_full[b]);
+                umma_commit(&bar->p_empty[b]);
                 // the K/V stage is free once the last tile of its load is done
                 if (li_next != li) umma_commit(&bar->kv_empty[skv]);
                 if (!early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
@@ -502,19 +539,71 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             umma_commit(&bar->done);
             mbar_drain(&bar->done, 0);
         }
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ epilogue groups: thread = tile row
-        const int grp = (warp - 4) >> 2;       // tiles i with i % 2 == grp
-        const int ew = (warp - 4) & 3;         // TMEM lane quadrant
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ softmax: thread = tile row, every tile
+        const int ew = warp & 3;               // TMEM lane quadrant
         const int r = ew * 32 + lane;
-        const uint32_t lane_base = tmem + grp * 256 + ((uint32_t)(ew * 32) << 16);
-        float *wst = stg + (warp - 4) * 32 * PITCH;
-        uint8_t *myP = sP + grp * p_bytes;
+        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
         bool ok = true;
-        int k = 0;
-        int tau = tile_lo + grp;
-        for (; tau < tile_hi && ok; ++k, tau += 2) {
-            const int i = tau - tile_lo;
+        for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
+            const int b = i & 1, k = i >> 1;
+            if (!(ok = mbar_wait(&bar->s_full[b], k & 1, abort, a.status))) break;
+            tc_fence_after();
+            const uint32_t s_base = tmem + lane_off + b * 128;
+            uint8_t *myP = sP + b * p_bytes;
+            float l = 0.f;
+            uint32_t sr[32];
+            float mx = -INFINITY;
+            for (int q = 0; q < S / 32; ++q) {
+                tmem_ld32(s_base + q * 32, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
+            }
+            // P buffer b is free once PV(i - 2) has read it
+            if (k > 0 && !(ok = mbar_wait(&bar->p_empty[b], (k - 1) & 1, abort, a.status))) break;
+            for (int q = 0; q < S / 32; ++q) {
+                tmem_ld32(s_base + q * 32, sr);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = exp2f((__uint_as_float(sr[2 * e]) - mx) * a.scale_log2);
+                    const float p1 = exp2f((__uint_as_float(sr[2 * e + 1]) - mx) * a.scale_log2);
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    // the MMA sees the rounded probabilities: normalise by their sum
+                    const float2 hf = __bfloat1622float2(h);
+                    l += hf.x + hf.y;
+                    pk[e] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                uint8_t *prow = myP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int cx = (q & 1) * 4 + x;
+                    *reinterpret_cast<uint4 *>(prow + ((cx ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->p_full[b]);
+            // row sum for the O drain of this tile
+            if (k > 0 && !(ok = mbar_wait(&bar->l_empty[b], (k - 1) & 1, abort, a.status))) break;
+            bar->l[b][r] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->l_full[b]);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ O drain: thread = tile row, 64 of its columns
+        const int ew = warp & 3;               // TMEM lane quadrant
+        const int hf = (warp - 8) >> 2;        // column half
+        const int r = ew * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
+        float *wst = stg + (warp - 8) * 32 * PITCH;
+        bool ok = true;
+        for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
+            const int b = i & 1, k = i >> 1;
             const int si = i % NINFO;
             if (!(ok = mbar_wait(&bar->info_full[si], (i / NINFO) & 1, abort, a.status))) break;
             const int Tp = info[si].p;
@@ -526,60 +615,24 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             for (int rr = 0; rr < 8; ++rr) dstoff[rr] = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->info_empty[si]);
-            const bool valid = myoff >= 0;
-            // chunk softmax: S row -> P row (bf16, swizzled), l
-            if (!(ok = mbar_wait(&bar->s_full[grp], k & 1, abort, a.status))) break;
-            tc_fence_after();
-            float l = 0.f;
-            {
-                uint32_t sr[32];
-                float mx = -INFINITY;
-                for (int q = 0; q < S / 32; ++q) {
-                    tmem_ld32(lane_base + q * 32, sr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
-                }
-                for (int q = 0; q < S / 32; ++q) {
-                    tmem_ld32(lane_base + q * 32, sr);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = exp2f((__uint_as_float(sr[2 * e]) - mx) * a.scale_log2);
-                        const float p1 = exp2f((__uint_as_float(sr[2 * e + 1]) - mx) * a.scale_log2);
-                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        // the MMA sees the rounded probabilities: normalise by their sum
-                        const float2 hf = __bfloat1622float2(h);
-                        l += hf.x + hf.y;
-                        pk[e] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                    uint8_t *prow = myP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const int cx = (q & 1) * 4 + x;
-                        *reinterpret_cast<uint4 *>(prow + ((cx ^ (r & 7)) << 4)) =
-                            make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
+            if (!(ok = mbar_wait(&bar->l_full[b], k & 1, abort, a.status))) break;
+            const float l = bar->l[b][r];
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->p_full[grp]);
+            if (lane == 0) mbar_arrive(&bar->l_empty[b]);
+            const float f = myoff >= 0 ? w / l : 0.f;
             // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
-            if (!(ok = mbar_wait(&bar->o_full[grp], k & 1, abort, a.status))) break;
+            if (!(ok = mbar_wait(&bar->o_full[b], k & 1, abort, a.status))) break;
             tc_fence_after();
-            const float f = valid ? w / l : 0.f;
             float *acc_slot = slot_of(a, Tp) + 4 * (lane & 7);
-            for (int q = 0; q < D / 32; ++q) {
+            const uint32_t o_base = tmem + lane_off + 256 + b * 128 + hf * 64;
+            for (int q = 0; q < 2; ++q) {
                 uint32_t orr[32];
-                tmem_ld32(lane_base + 128 + q * 32, orr);
+                tmem_ld32(o_base + q * 32, orr);
                 tmem_wait_ld();
-                if (q == D / 32 - 1) {
+                if (q == 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar->o_empty[grp]);
+                    if (lane == 0) mbar_arrive(&bar->o_empty[b]);
                 }
                 float *mine = wst + lane * PITCH;
 #pragma unroll
@@ -588,11 +641,12 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                         make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
                                     __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
                 __syncwarp();
+                const int col = hf * 64 + q * 32;
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
                     if (dstoff[rr] >= 0) {
                         const int lr = rr * 4 + (lane >> 3);
-                        red_add_v4(acc_slot + dstoff[rr] + q * 32,
+                        red_add_v4(acc_slot + dstoff[rr] + col,
                                    *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
                     }
                 }
@@ -602,7 +656,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
