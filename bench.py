@@ -11,7 +11,8 @@ collective).  The timed region is bracketed by a barrier and a device
 synchronise, and timed with CUDA events on the launching stream.  The reported
 time is the maximum over ranks.  The inputs (Q 512 MiB, K and V 128 MiB each)
 are larger than L2, so no flush is needed between prefill steps.  The decode
-line (decode_1m: batch 8, 1M cached tokens) flushes L2 before every step.
+lines (decode_1m: batch 8, 1M cached tokens; decode_16m: batch 1, 16M cached
+tokens) flush L2 before every step.
 
 --impl reference times the CPU oracle instead (the task has no other
 reference implementation), on a bounded sample of the same workload.
@@ -318,19 +319,22 @@ def run_b200(args, world, rank, local):
     torch.cuda.empty_cache()
     if not args.no_decode:
         out["decode_1m"] = run_decode(args, world, rank, local, pk)
+        if not args.no_decode_16m:
+            out["decode_16m"] = run_decode(args, world, rank, local, pk, "decode_16m")
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(p, args.seed)
     return out
 
 
-def run_decode(args, world, rank, local, pk):
-    """Decode step at 1M context (decode_1m): landmarks precomputed, L2 flushed
-    before each step, each step timed alone."""
+def run_decode(args, world, rank, local, pk, name="decode_1m"):
+    """One decode step (decode_1m: batch 8 at 1M context; decode_16m: batch 1 at
+    16M context): landmarks precomputed, L2 flushed before each step, each step
+    timed alone."""
     import landmark_guided_chunk_b200 as hsa
     from landmark_guided_chunk_b200.inputs import make_inputs, workload
 
     dev = torch.device("cuda", local)
-    p = workload("decode_1m")
+    p = workload(name)
     inp = make_inputs(p, seed=args.seed + rank, device=dev)
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
     L = hsa.landmarks(K, W, p.S)
@@ -419,7 +423,7 @@ def run_decode(args, world, rank, local, pk):
                    "single_call_us": round(att_us, 2),
                    "single_call_timing": "one call after an L2 flush, incl. its status memset and launch"},
     }
-    res = {"workload": f"decode_1m: B{p.B} ctx {p.Tkv} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
+    res = {"workload": f"{name}: B{p.B} ctx {p.Tkv} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
            "us_per_step": round(us, 2), "us_per_token": round(us / p.B, 3),
            "tokens_per_s": round(p.B * world / (us * 1e-6), 1),
            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -541,6 +545,7 @@ def main():
     ap.add_argument("--workload", default="prefill_bf16", choices=["prefill_bf16", "router_bf16", "tiny_f32"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-decode-16m", action="store_true", help="skip the 16M-context decode line (64 GiB cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
