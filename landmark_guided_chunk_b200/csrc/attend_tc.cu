@@ -49,7 +49,7 @@ constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
 constexpr int TB = 4096;         // tokens per phase
 constexpr int NB = 2;            // phases per batch (= per launch)
-constexpr int NT_ATT = 512;      // warps 0-1 producers, 2 MMA, 3 idle, 4-7 softmax, 8-15 O drain
+constexpr int NT_ATT = 512;      // warps 0-1 Q producers, 2 MMA, 3 K/V loader, 4-7 softmax, 8-15 O drain
 constexpr int NPROD = 64;        // producer threads (two tile rows each)
 
 struct AttTcArgs {
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             mm[h] = rr[h] / a.G;
             gg[h] = rr[h] % a.G;
         }
-        int i = 0, nload = 0;
+        int i = 0;
         bool ok = true;
         int tau = tile_lo;
         TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
@@ -390,7 +390,6 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             pr[h] = v ? a.pairs[T.start + mm[h]] : 0;
             pw[h] = v ? a.pair_w[T.start + mm[h]] : 0.f;
         }
-        int prev_p = -1, prev_c = -1;
         for (; tau < tile_hi && ok; ++i) {
             // prefetch the next tile while this one is issued
             const int tau_n = tau + 1;
@@ -414,23 +413,6 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             }
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
-            const bool newkv = T.p != prev_p || T.c != prev_c;
-            if (newkv) {
-                if (threadIdx.x == 0) {
-                    const int skv = nload % a.nskv, ikv = nload / a.nskv;
-                    if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
-                    mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
-                    uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
-                    const int z = T.b * a.Tkv + T.c * S;
-                    tma_load_3d(dk, &tmK, 0, T.j, z, &bar->kv_full[skv]);
-                    tma_load_3d(dk + kv_bytes, &tmK, 64, T.j, z, &bar->kv_full[skv]);
-                    tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, T.j, z, &bar->kv_full[skv]);
-                    tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, T.j, z, &bar->kv_full[skv]);
-                }
-                ++nload;
-                prev_p = T.p;
-                prev_c = T.c;
-            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int r = rr[h];
@@ -458,7 +440,29 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             tau = tau_n;
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
-        if (threadIdx.x == 0) {
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ K/V loader: one TMA load per bucket run
+        // (consecutive tiles of one (phase, chunk) share a load), as far ahead as the stages allow
+        if (lane == 0) {
+            int nload = 0, prev_p = -1, prev_c = -1;
+            bool ok = true;
+            for (int tau = tile_lo; tau < tile_hi && ok; ++tau) {
+                const int4 e = a.tiles[tau];
+                if (e.x == prev_p && e.y == prev_c) continue;
+                prev_p = e.x;
+                prev_c = e.y;
+                const int bj = e.x / a.ntb, Tb = bj / a.Hkv, Tj = bj % a.Hkv;
+                const int skv = nload % a.nskv, ikv = nload / a.nskv;
+                if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
+                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
+                uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
+                const int z = Tb * a.Tkv + e.y * S;
+                tma_load_3d(dk, &tmK, 0, Tj, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + kv_bytes, &tmK, 64, Tj, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, Tj, z, &bar->kv_full[skv]);
+                tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, Tj, z, &bar->kv_full[skv]);
+                ++nload;
+            }
             // wind down: the K/V loads issued have all landed
             for (int s = 0; s < a.nskv && s < nload; ++s)
                 mbar_drain(&bar->kv_full[s], ((nload - 1 - s) / a.nskv) & 1);
