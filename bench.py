@@ -431,9 +431,52 @@ def run_decode(args, world, rank, local, pk, name="decode_1m"):
            "stages": stages,
            "l2": "512 MiB written then read before every step and before each stage timed alone", "paths": plan,
            "gpu_launches_per_step": plan["select"][1] + plan["attend"][1]}
+    if name == "decode_1m":
+        res["loop"] = decode_loop(p, hsa, Q, K, V, W, L, O, ws, st, world)
     del inp, Q, K, V, W, L, O, ws, scrub, qs, sels, outs
     torch.cuda.empty_cache()
     return res
+
+
+def decode_loop(p, hsa, Q, K, V, W, L, O, ws, st, world):
+    """A generation loop over the cache's last chunk: the cache starts S tokens short,
+    and each step appends one token per sequence (hsa_decode_append; the S-th append
+    completes the chunk and computes its landmark) and runs the forward of the next
+    query on Tkv + 1 cached tokens.  The appended rows are the cache's own, so every
+    step reads the same data as the one-step measurement.  Timed back to back (a
+    running loop's steady state, no flush): whole steps, then the same forwards alone."""
+    T0 = p.Tkv - p.S
+    kn = [K[:, t].contiguous() for t in range(T0, p.Tkv)]
+    vn = [V[:, t].contiguous() for t in range(T0, p.Tkv)]
+
+    def run(append):
+        for i in range(p.S):
+            kv = T0 + i
+            if append:
+                hsa.decode_append(K, V, kn[i], vn[i], kv, p.S, W, L)
+            hsa.forward(Q, K, V, None, p.S, p.k, p.tau, kv + 1, L=L, landmarks_ready=True, O=O, ws=ws,
+                        kv_len=kv + 1)
+
+    run(True)
+    torch.cuda.synchronize()
+    times = {}
+    for label, app in (("step", True), ("forward", False)):
+        ts = []
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            run(app)
+            b.record(st)
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / p.S)
+        times[label] = max_over_ranks(statistics.median(ts), world)
+    hsa.device_status(ws)
+    return {"us_per_step": round(times["step"], 2), "steps": p.S,
+            "forward_only_us_per_step": round(times["forward"], 2),
+            "append_us_per_step": round(times["step"] - times["forward"], 2),
+            "timing": f"{p.S} steps back to back (no flush between them), median of 3 runs: append + forward, "
+                      "then the same forwards alone; the append's cost is the difference (it includes the "
+                      "one step in S that computes the completed chunk's landmark)"}
 
 
 def dram_traffic(stage: str, path: str):

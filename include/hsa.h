@@ -20,9 +20,13 @@
  *     the legacy default stream).  Host-side validation runs before any launch.
  *     An invalid call launches nothing and returns a status.
  *   - Layouts (row-major, contiguous, every pointer 16-byte aligned):
- *       Q, O   [B][Tq][H][d]       K, V  [B][Tkv][Hkv][d]
+ *       Q, O   [B][Tq][H][d]       K, V  [B][Tcap][Hkv][d]
  *       W_L    [d][d]  (row = input dim: landmark = mean_row * W_L)
- *       L      [B][Hkv][C][d],  C = floor(Tkv / S)
+ *       L      [B][Hkv][Ccap][d],  C = floor(Tkv / S) of them valid
+ *     Tkv is the number of cached tokens; Tcap >= Tkv (hsa_problem_t.kv_cap,
+ *     0 = Tkv) the tokens the K/V buffers hold per sequence, and
+ *     Ccap = floor(Tcap / S) the chunks L holds per (b, kv head).  A decode
+ *     loop keeps Tcap fixed while Tkv grows (hsa_decode_append).
  *       idx    [B][Tq][Hkv][kmax] int32   score [B][Tq][Hkv][kmax] float
  *       keff   [B][Tq][Hkv] int32,        kmax = (tau > 0 ? 2k : k)
  *     Q, K, V, W_L, L and O all have the problem's dtype.  Scores are fp32 and
@@ -58,7 +62,7 @@
 extern "C" {
 #endif
 
-#define HSA_ABI_VERSION 1
+#define HSA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define HSA_API __attribute__((visibility("default")))
@@ -87,6 +91,7 @@ typedef struct {
     float tau;           /* gap-router threshold; 0 disables it, > 0 enables it (then 2k <= 32) */
     int32_t dtype;       /* hsa_dtype_t */
     uint32_t flags;      /* HSA_FLAG_* */
+    int32_t kv_cap;      /* Tcap: tokens per sequence the K/V buffers hold (0 = Tkv; else >= Tkv) */
 } hsa_problem_t;
 
 /* Supported shapes: d in {64, 128}; S in {32, 64, 128}; 1 <= k <= 32 (2k <= 32 with the
@@ -112,6 +117,23 @@ HSA_API hsa_status_t hsa_workspace_size(const hsa_problem_t *p, size_t *bytes);
  */
 HSA_API hsa_status_t hsa_landmarks(const hsa_problem_t *p, const void *K, const void *W_L, void *L,
                            void *stream);
+
+/*
+ * One step of a decode loop on a cache that grows in place (summary page,
+ * Implementation: every chunk gets its landmark; a decode step that completes
+ * a chunk therefore has to produce that chunk's landmark before a later query
+ * can retrieve it).  With Tkv = the tokens cached before the step (< Tcap):
+ *   K[b][Tkv][:][:] = k_new[b][:][:],  V[b][Tkv][:][:] = v_new[b][:][:]
+ * for every sequence b (k_new, v_new are [B][Hkv][d]), and, if Tkv + 1 is a
+ * multiple of S, the landmark of the chunk c = (Tkv + 1) / S - 1 that the new
+ * token completes is written to L[b][:][c][:] exactly as hsa_landmarks
+ * computes it (the same kernel code, so the two agree bit for bit).  The next
+ * step's problem has Tkv + 1 (and, for its query, q_pos0 = Tkv + 1).  Only
+ * B, Tkv, Hkv, d, S, dtype and kv_cap are used; Tkv must be < Tcap.  One
+ * launch; needs no workspace.  W_L and L may be NULL when no chunk completes.
+ */
+HSA_API hsa_status_t hsa_decode_append(const hsa_problem_t *p, const void *k_new, const void *v_new, void *K,
+                                       void *V, const void *W_L, void *L, void *stream);
 
 /*
  * Chunk selection (summary page, Core Technique and Implementation: score all

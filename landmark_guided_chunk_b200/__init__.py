@@ -21,15 +21,17 @@ from . import _native
 from ._native import HSAError, hsa_problem_t
 
 __all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "select_noalloc", "attend",
-           "forward", "device_status", "HSAError", "hsa_problem_t", "kmax_of"]
+           "forward", "decode_append", "device_status", "HSAError", "hsa_problem_t", "kmax_of"]
 
 _DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
 
 
-def make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0=0, tau=0.0, dtype=torch.bfloat16, flags=0) -> hsa_problem_t:
+def make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0=0, tau=0.0, dtype=torch.bfloat16, flags=0,
+                 kv_cap=0) -> hsa_problem_t:
+    """Tkv = cached tokens; kv_cap = tokens the K/V buffers hold per sequence (0 = Tkv)."""
     if dtype not in _DT:
         raise TypeError(f"dtype {dtype} not supported (float32, bfloat16)")
-    return hsa_problem_t(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, _DT[dtype], flags)
+    return hsa_problem_t(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, _DT[dtype], flags, kv_cap)
 
 
 def plan(prob: hsa_problem_t) -> dict:
@@ -76,22 +78,29 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def landmarks(K: torch.Tensor, W_L: torch.Tensor, S: int, L: torch.Tensor | None = None) -> torch.Tensor:
-    """L [B,Hkv,C,d] = mean of each complete chunk's keys times W_L (rounded once to K's dtype)."""
+def landmarks(K: torch.Tensor, W_L: torch.Tensor, S: int, L: torch.Tensor | None = None,
+              kv_len: int | None = None) -> torch.Tensor:
+    """L [B,Hkv,Tcap//S,d] = mean of each complete chunk's keys times W_L (rounded once to K's
+    dtype), for the chunks of the first kv_len tokens (default: all Tcap = K.shape[1])."""
     _dev(K, W_L, L)
-    B, Tkv, Hkv, d = K.shape
-    C = Tkv // S
+    B, Tcap, Hkv, d = K.shape
+    Tkv = Tcap if kv_len is None else kv_len
     if L is None:
-        L = torch.empty(B, Hkv, C, d, dtype=K.dtype, device=K.device)
-    prob = make_problem(B, 0, Tkv, Hkv, Hkv, d, S, 1, 0, 0.0, K.dtype)
+        L = torch.empty(B, Hkv, Tcap // S, d, dtype=K.dtype, device=K.device)
+    prob = make_problem(B, 0, Tkv, Hkv, Hkv, d, S, 1, 0, 0.0, K.dtype, kv_cap=Tcap)
     _native.check(_native.lib().hsa_landmarks(ctypes.byref(prob), _p(K), _p(W_L), _p(L), _stream(K)),
                   "hsa_landmarks")
     return L
 
 
-def _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags=0):
+def _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags=0, kv_cap=0):
     B, Tq, H, d = Q.shape
-    return make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, Q.dtype, flags)
+    return make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, Q.dtype, flags, kv_cap)
+
+
+def _l_cap(Tkv, Ccap, S):
+    """kv_cap whose chunk stride is L's Ccap (L may hold more chunks than Tkv has)."""
+    return max(Tkv, Ccap * S)
 
 
 def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False):
@@ -99,8 +108,8 @@ def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False):
     _dev(Q, L, ws)
     B, Tq, H, d = Q.shape
     Hkv, C = L.shape[1], L.shape[2]
-    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0,
-                      _native.HSA_FLAG_SIMT if force_simt else 0)
+    Tkv = Tkv if Tkv is not None else C * S
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, _native.HSA_FLAG_SIMT if force_simt else 0, _l_cap(Tkv, C, S))
     km = kmax_of(k, tau)
     idx = torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device)
     score = torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device)
@@ -120,7 +129,8 @@ def select_noalloc(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, out=None):
     _dev(Q, L)
     B, Tq, H, d = Q.shape
     Hkv, C = L.shape[1], L.shape[2]
-    prob = _prob_from(Q, Tkv if Tkv is not None else C * S, Hkv, S, k, tau, q_pos0)
+    Tkv = Tkv if Tkv is not None else C * S
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, 0, _l_cap(Tkv, C, S))
     km = kmax_of(k, tau)
     if out is None:
         out = (torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device),
@@ -133,10 +143,13 @@ def select_noalloc(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, out=None):
     return idx, score, keff
 
 
-def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None, force_simt=False):
-    """Chunk attention + fusion for a given selection.  Returns O [B,Tq,H,d]."""
+def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None, force_simt=False, kv_len=None):
+    """Chunk attention + fusion for a given selection.  Returns O [B,Tq,H,d].  kv_len: cached
+    tokens when the K/V buffers hold more (default: all of K.shape[1])."""
     _dev(Q, K, V, idx, score, keff, O, ws)
-    prob = _prob_from(Q, K.shape[1], K.shape[2], S, k, tau, q_pos0, _native.HSA_FLAG_SIMT if force_simt else 0)
+    Tcap = K.shape[1]
+    prob = _prob_from(Q, Tcap if kv_len is None else kv_len, K.shape[2], S, k, tau, q_pos0,
+                      _native.HSA_FLAG_SIMT if force_simt else 0, Tcap)
     if O is None:
         O = torch.empty_like(Q)
     if ws is None:
@@ -147,18 +160,21 @@ def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None, 
 
 
 def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False, O=None, ws=None,
-            return_selection=False, force_simt=False):
+            return_selection=False, force_simt=False, kv_len=None):
     """The whole HSA forward.  Returns O, or (O, L, idx, score, keff) with return_selection.
-    force_simt runs the CUDA-core kernels even where tensor-core ones exist (for A/B tests)."""
+    force_simt runs the CUDA-core kernels even where tensor-core ones exist (for A/B tests).
+    kv_len: cached tokens when the K/V buffers (and L) hold more, as in a decode loop (default:
+    all of K.shape[1]); L is then [B, Hkv, K.shape[1] // S, d]."""
     _dev(Q, K, V, W_L, L, O, ws)
     B, Tq, H, d = Q.shape
-    Tkv, Hkv = K.shape[1], K.shape[2]
+    Tcap, Hkv = K.shape[1], K.shape[2]
+    Tkv = Tcap if kv_len is None else kv_len
     flags = (_native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0) | (_native.HSA_FLAG_SIMT if force_simt else 0)
-    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags)
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags, Tcap)
     if L is None:
         if landmarks_ready:
             raise ValueError("landmarks_ready needs L")
-        L = torch.empty(B, Hkv, Tkv // S, d, dtype=Q.dtype, device=Q.device)
+        L = torch.empty(B, Hkv, Tcap // S, d, dtype=Q.dtype, device=Q.device)
     if O is None:
         O = torch.empty_like(Q)
     if ws is None:
@@ -175,6 +191,19 @@ def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False
     if return_selection:
         return (O, L) + sel
     return O
+
+
+def decode_append(K, V, k_new, v_new, kv_len, S, W_L=None, L=None) -> bool:
+    """One decode step's cache update: K[:, kv_len] = k_new and V[:, kv_len] = v_new
+    (k_new, v_new [B, Hkv, d]; K, V [B, Tcap, Hkv, d] with kv_len < Tcap), and, when that
+    completes a chunk, its landmark into L [B, Hkv, Tcap // S, d].  Returns whether a chunk
+    was completed (W_L and L are needed then)."""
+    _dev(K, V, k_new, v_new, W_L, L)
+    B, Tcap, Hkv, d = K.shape
+    prob = make_problem(B, 1, kv_len, Hkv, Hkv, d, S, 1, kv_len, 0.0, K.dtype, 0, Tcap)
+    _native.check(_native.lib().hsa_decode_append(ctypes.byref(prob), _p(k_new), _p(v_new), _p(K), _p(V),
+                                                   _p(W_L), _p(L), _stream(K)), "hsa_decode_append")
+    return (kv_len + 1) % S == 0
 
 
 def device_status(ws: torch.Tensor) -> None:

@@ -19,7 +19,7 @@ HSA_FLAG_SIMT = 2
 
 EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version",
-            "hsa_select_noalloc")
+            "hsa_select_noalloc", "hsa_decode_append")
 PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor"}
 
 
@@ -27,7 +27,8 @@ class hsa_problem_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Tq", ctypes.c_int32), ("Tkv", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("S", ctypes.c_int32), ("k", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
-                ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+                ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("flags", ctypes.c_uint32),
+                ("kv_cap", ctypes.c_int32)]
 
 
 class hsa_plan_t(ctypes.Structure):
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
     L.hsa_get_device_status.argtypes = [P, Z, P]
     L.hsa_plan.argtypes = [prob, ctypes.POINTER(hsa_plan_t)]
     L.hsa_select_noalloc.argtypes = [prob, P, P, I32p, Fp, I32p, P]
+    L.hsa_decode_append.argtypes = [prob, P, P, P, P, P, P, P]
     L.hsa_status_string.argtypes = [ctypes.c_int]
     L.hsa_status_string.restype = ctypes.c_char_p
     L.hsa_last_error.argtypes = []
@@ -71,7 +73,7 @@ def lib() -> ctypes.CDLL:
     L.hsa_abi_version.argtypes = []
     L.hsa_abi_version.restype = ctypes.c_int
     for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
-              "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc"):
+              "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc", "hsa_decode_append"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

@@ -181,7 +181,7 @@ constexpr int MAXW = 8;    // worker warps (= chunk stages) per CTA at most
 constexpr int MAXU = 32;   // units per worker at most (the grid is sized for it)
 
 struct GatherArgs {
-    int B, Tq, Tkv, H, Hkv, S, C, kmax, G;
+    int B, Tq, Tcap, H, Hkv, S, C, kmax, G;
     int nunits, nw;     // units = rows * kmax (slot-major within a row); worker warps per CTA
     long long q_pos0;
     float scale;        // 1/sqrt(d)
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
         if (c >= 0 && !s_abort) {
             issued = true;
             if (lane == 0) {
-                const int z = b * a.Tkv + c * S;
+                const int z = b * a.Tcap + c * S;
                 mbar_expect_tx(mbk, (uint32_t)(NB * BOX));
                 mbar_expect_tx(mbv, (uint32_t)(NB * BOX));
 #pragma unroll
@@ -379,7 +379,7 @@ cudaError_t launch_d(const Prob &p, const GatherArgs &a, const CUtensorMap &mk, 
 
 bool attend_gather_supported(const Prob &p) {
     return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && (p.S == 32 || p.S == 64 || p.S == 128) &&
-           p.G <= 16 && p.kmax <= 32 && (long long)p.B * p.Tkv < (1ll << 31) && p.rows * p.kmax < (1ll << 31);
+           p.G <= 16 && p.kmax <= 32 && (long long)p.B * p.Tcap < (1ll << 31) && p.rows * p.kmax < (1ll << 31);
 }
 
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
@@ -388,7 +388,7 @@ cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, co
     GatherArgs a;
     a.B = p.B;
     a.Tq = p.Tq;
-    a.Tkv = p.Tkv;
+    a.Tcap = p.Tcap;
     a.H = p.H;
     a.Hkv = p.Hkv;
     a.S = p.S;
@@ -400,9 +400,9 @@ cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, co
     a.q_pos0 = p.q_pos0;
     a.scale = 1.0f / sqrtf((float)p.d);
     a.status = status;
-    // K and V as 3D (d, Hkv, B*Tkv): box (64, 1, S) = S rows of 128 bytes, 128-byte swizzle
+    // K and V as 3D (d, Hkv, B*Tcap): box (64, 1, S) = S rows of 128 bytes, 128-byte swizzle
     CUtensorMap mk, mv;
-    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tkv};
+    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tcap};
     const uint64_t strides[2] = {(uint64_t)p.d * 2, (uint64_t)p.Hkv * p.d * 2};
     const uint32_t box[3] = {64, 1, (uint32_t)p.S};
     cudaError_t e;

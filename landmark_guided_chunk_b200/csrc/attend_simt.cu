@@ -21,7 +21,7 @@ namespace hsa {
 namespace {
 
 struct AttArgs {
-    int Tq, Tkv, H, Hkv, d, S, C, kmax, G;
+    int Tq, Tcap, H, Hkv, d, S, C, kmax, G;
     long long q_pos0, rows;
     float scale;        // 1/sqrt(d)
     uint32_t *status;   // workspace status word
@@ -107,7 +107,7 @@ __device__ __forceinline__ void stage_chunk(const T *K, const T *V, const AttArg
                                             const Smem &s) {
     constexpr int EPS = 16 / (int)sizeof(T);
     const int segs = a.d / EPS;
-    const size_t row0 = ((size_t)b * a.Tkv + (size_t)c * a.S) * a.Hkv + j;
+    const size_t row0 = ((size_t)b * a.Tcap + (size_t)c * a.S) * a.Hkv + j;
     for (int i = threadIdx.x; i < a.S * segs; i += NT) {
         const int u = i / segs, sg = i - u * segs;
         const size_t off = (row0 + (size_t)u * a.Hkv) * a.d + (size_t)sg * EPS;
@@ -262,7 +262,7 @@ cudaError_t launch_typed(const Prob &p, const WsLayout &w, const void *Q, const 
                          cudaStream_t st) {
     AttArgs a;
     a.Tq = p.Tq;
-    a.Tkv = p.Tkv;
+    a.Tcap = p.Tcap;
     a.H = p.H;
     a.Hkv = p.Hkv;
     a.d = p.d;

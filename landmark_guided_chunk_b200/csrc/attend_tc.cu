@@ -53,7 +53,7 @@ constexpr int NT_ATT = 512;      // warps 0-1 Q producers, 2 MMA, 3 K/V loader, 
 constexpr int NPROD = 64;        // producer threads (two tile rows each)
 
 struct AttTcArgs {
-    int B, Tq, Tkv, H, Hkv, G, S, C, kmax, tok;
+    int B, Tq, Tcap, H, Hkv, G, S, C, kmax, tok;
     int ntb, nphase, nbucket, nsq, nskv;
     int batch;                   // batch processed by this launch (== nbatch: finalise only)
     int nbatch;
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
                 mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
                 uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
-                const int z = Tb * a.Tkv + e.y * S;
+                const int z = Tb * a.Tcap + e.y * S;
                 tma_load_3d(dk, &tmK, 0, Tj, z, &bar->kv_full[skv]);
                 tma_load_3d(dk + kv_bytes, &tmK, 64, Tj, z, &bar->kv_full[skv]);
                 tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, Tj, z, &bar->kv_full[skv]);
@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 
 bool attend_tc_supported(const Prob &p) {
     if (!(p.dtype == HSA_BF16 && p.d == D && (p.S == 64 || p.S == 128) && p.G <= 16 && (32 % p.G) == 0 &&
-          p.C >= 1 && p.Tq >= 1 && p.kmax <= 32 && p.Tq < (1 << 26)))
+          p.C >= 1 && p.Tq >= 1 && p.kmax <= 32 && p.Tq < (1 << 26) && (long long)p.B * p.Tcap < (1ll << 31)))
         return false;
     // the second scan level is one block of 1024 threads over SCAN_BLK-bucket blocks
     const long long ntb = (p.Tq + TB - 1) / TB;
@@ -708,7 +708,7 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     AttTcArgs a;
     a.B = p.B;
     a.Tq = p.Tq;
-    a.Tkv = p.Tkv;
+    a.Tcap = p.Tcap;
     a.H = p.H;
     a.Hkv = p.Hkv;
     a.G = p.G;
@@ -752,9 +752,9 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     att_scatter_kernel<<<rows_blocks, 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    // K and V as 3D (d, Hkv, B*Tkv): box (64, 1, S) = S rows of 128 B
+    // K and V as 3D (d, Hkv, B*Tcap): box (64, 1, S) = S rows of 128 B
     CUtensorMap mk, mv;
-    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tkv};
+    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tcap};
     const uint64_t strides[2] = {(uint64_t)p.d * 2, (uint64_t)p.Hkv * p.d * 2};
     const uint32_t box[3] = {64, 1, (uint32_t)p.S};
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;

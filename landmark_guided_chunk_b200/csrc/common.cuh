@@ -19,6 +19,8 @@ constexpr int MAX_G = 16;      // query heads per kv head
 // Validated problem with the derived quantities every stage uses.
 struct Prob {
     int B, Tq, Tkv, H, Hkv, d, S, k, G, C, kmax, dtype;
+    int Tcap;         // K/V token stride: tokens each sequence's buffers hold (>= Tkv)
+    int Lc;           // L chunk stride: floor(Tcap / S) (>= C)
     long long q_pos0;
     float tau;
     unsigned flags;
@@ -286,6 +288,8 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
                              cudaStream_t st);
 
 cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
+cudaError_t launch_decode_append(const Prob &p, const void *knew, const void *vnew, void *K, void *V, const void *W,
+                                 void *L, cudaStream_t st);
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
                           float *score, int32_t *keff, char *ws, cudaStream_t st);
 cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const void *K, const void *V,

@@ -138,6 +138,8 @@ hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
     if (kmax > MAX_KMAX) return fail(HSA_ERR_UNSUPPORTED, "k=%d gives %d slots (max %d)", in->k, kmax, MAX_KMAX);
     if (in->H / in->Hkv > MAX_G) return fail(HSA_ERR_UNSUPPORTED, "G=%d (max %d)", in->H / in->Hkv, MAX_G);
     if (in->B > 65535) return fail(HSA_ERR_UNSUPPORTED, "B=%d (max 65535)", in->B);
+    if (in->kv_cap != 0 && in->kv_cap < in->Tkv)
+        return fail(HSA_ERR_INVALID_ARG, "kv_cap=%d is below Tkv=%d", in->kv_cap, in->Tkv);
     p->B = in->B;
     p->Tq = in->Tq;
     p->Tkv = in->Tkv;
@@ -148,6 +150,8 @@ hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
     p->k = in->k;
     p->G = in->H / in->Hkv;
     p->C = in->Tkv / in->S;
+    p->Tcap = in->kv_cap != 0 ? in->kv_cap : in->Tkv;
+    p->Lc = p->Tcap / in->S;
     p->kmax = kmax;
     p->dtype = in->dtype;
     p->q_pos0 = in->q_pos0;
@@ -231,6 +235,24 @@ hsa_status_t hsa_landmarks(const hsa_problem_t *prob, const void *K, const void 
     HSA_TRY(need(L, any, "L"));
     cudaError_t e = launch_landmarks(p, K, W_L, L, (cudaStream_t)stream);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "landmark kernel launch");
+}
+
+hsa_status_t hsa_decode_append(const hsa_problem_t *prob, const void *k_new, const void *v_new, void *K, void *V,
+                               const void *W_L, void *L, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (p.B > 0 && p.Tkv >= p.Tcap)
+        return fail(HSA_ERR_INVALID_ARG, "no room to append: Tkv=%d, kv_cap=%d", p.Tkv, p.Tcap);
+    const bool any = p.B > 0;
+    const bool completes = any && (p.Tkv + 1) % p.S == 0;
+    HSA_TRY(need(k_new, any, "k_new"));
+    HSA_TRY(need(v_new, any, "v_new"));
+    HSA_TRY(need(K, any, "K"));
+    HSA_TRY(need(V, any, "V"));
+    HSA_TRY(need(W_L, completes, "W_L"));
+    HSA_TRY(need(L, completes, "L"));
+    cudaError_t e = launch_decode_append(p, k_new, v_new, K, V, W_L, L, (cudaStream_t)stream);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "decode append kernel launch");
 }
 
 hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L, int32_t *idx, float *score,

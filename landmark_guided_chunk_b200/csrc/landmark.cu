@@ -79,12 +79,20 @@ __host__ __device__ __forceinline__ size_t landmark_smem(int n, int d, int nv, i
     return (size_t)d * d * tsize + sizeof(float) * ((size_t)n * row_groups(n / nv) + (size_t)NT / (d / 4) * JB * d);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(NT, 2) landmark_kernel(const T *__restrict__ K, const T *__restrict__ W,
-                                                         T *__restrict__ L, int Tkv, int Hkv, int d, int S, int C) {
-    extern __shared__ __align__(16) unsigned char sm[];
+// A row of K as 16-byte vectors: through the read-only path, or (for a chunk this
+// kernel itself has just completed) with ordinary loads, which see this CTA's writes.
+template <bool NC> __device__ __forceinline__ uint4 ld_row(const uint4 *p) {
+    if constexpr (NC) return __ldg(p);
+    else return *p;
+}
+
+// The landmark of chunk c of sequence b, computed by the whole CTA (NT threads; the
+// dynamic shared memory is laid out as landmark_smem describes).
+template <typename T, bool NC>
+__device__ __forceinline__ void landmark_chunk(unsigned char *sm, const T *__restrict__ K, const T *__restrict__ W,
+                                               T *__restrict__ L, int b, int c, int Tcap, int Hkv, int d, int S,
+                                               int Lc) {
     constexpr int NV = Vec<T>::N;
-    const int c = blockIdx.x, b = blockIdx.y;
     const int n = Hkv * d;              // channels of one token row
     const int nvr = n / NV;             // 16-byte vectors of one token row
     const int R = row_groups(nvr);
@@ -102,7 +110,7 @@ __global__ void __launch_bounds__(NT, 2) landmark_kernel(const T *__restrict__ K
     asm volatile("cp.async.commit_group;" ::: "memory");
 
     // Pooling: group grp sums rows grp, grp + R, ... with eight rows' loads in flight.
-    const T *chunk = K + ((size_t)b * Tkv + (size_t)c * S) * n;
+    const T *chunk = K + ((size_t)b * Tcap + (size_t)c * S) * n;
     const float inv = 1.0f / (float)S;
     if ((int)threadIdx.x < R * nvr || R == 1) {
         const int grp = R == 1 ? 0 : (int)threadIdx.x / nvr;
@@ -117,11 +125,11 @@ __global__ void __launch_bounds__(NT, 2) landmark_kernel(const T *__restrict__ K
             for (; u + (RB - 1) * R < S; u += RB * R) {
                 uint4 x[RB];
 #pragma unroll
-                for (int k = 0; k < RB; ++k) x[k] = __ldg(src + (size_t)(u + k * R) * nvr);
+                for (int k = 0; k < RB; ++k) x[k] = ld_row<NC>(src + (size_t)(u + k * R) * nvr);
 #pragma unroll
                 for (int k = 0; k < RB; ++k) Vec<T>::add(acc, x[k]);
             }
-            for (; u < S; u += R) Vec<T>::add(acc, __ldg(src + (size_t)u * nvr));
+            for (; u < S; u += R) Vec<T>::add(acc, ld_row<NC>(src + (size_t)u * nvr));
             const float scl = R == 1 ? inv : 1.0f;
 #pragma unroll
             for (int i = 0; i < NV; ++i) part[grp * n + v * NV + i] = acc[i] * scl;
@@ -178,10 +186,40 @@ __global__ void __launch_bounds__(NT, 2) landmark_kernel(const T *__restrict__ K
                 sum.z += x.z;
                 sum.w += x.w;
             }
-            store4<T>(L + (((size_t)b * Hkv + j0 + jj) * C + c) * d + 4 * f4, sum);
+            store4<T>(L + (((size_t)b * Hkv + j0 + jj) * Lc + c) * d + 4 * f4, sum);
         }
         __syncthreads();
     }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT, 2) landmark_kernel(const T *__restrict__ K, const T *__restrict__ W,
+                                                         T *__restrict__ L, int Tcap, int Hkv, int d, int S, int Lc) {
+    extern __shared__ __align__(16) unsigned char sm[];
+    landmark_chunk<T, true>(sm, K, W, L, blockIdx.y, blockIdx.x, Tcap, Hkv, d, S, Lc);
+}
+
+// One decode step's cache update, one CTA per sequence b: the new token's K and V
+// rows go to position Tkv, and if that completes a chunk, its landmark follows.
+template <typename T>
+__global__ void __launch_bounds__(NT, 2) decode_append_kernel(const T *__restrict__ knew, const T *__restrict__ vnew,
+                                                              T *__restrict__ K, T *__restrict__ V,
+                                                              const T *__restrict__ W, T *__restrict__ L, int Tkv,
+                                                              int Tcap, int Hkv, int d, int S, int Lc, int complete) {
+    extern __shared__ __align__(16) unsigned char sm[];
+    const int b = blockIdx.x;
+    const int n = Hkv * d, nv16 = n * (int)sizeof(T) / 16;
+    const uint4 *ks = reinterpret_cast<const uint4 *>(knew + (size_t)b * n);
+    const uint4 *vs = reinterpret_cast<const uint4 *>(vnew + (size_t)b * n);
+    uint4 *kd = reinterpret_cast<uint4 *>(K + ((size_t)b * Tcap + Tkv) * n);
+    uint4 *vd = reinterpret_cast<uint4 *>(V + ((size_t)b * Tcap + Tkv) * n);
+    for (int v = threadIdx.x; v < nv16; v += NT) {
+        kd[v] = ks[v];
+        vd[v] = vs[v];
+    }
+    if (!complete) return;
+    __syncthreads();   // the chunk's last row, written above, is read back by the whole CTA
+    landmark_chunk<T, false>(sm, K, W, L, b, (Tkv + 1) / S - 1, Tcap, Hkv, d, S, Lc);
 }
 
 }  // namespace
@@ -195,12 +233,35 @@ cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(landmark_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         landmark_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(
-            (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)W, (__nv_bfloat16 *)L, p.Tkv, p.Hkv, p.d, p.S, p.C);
+            (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)W, (__nv_bfloat16 *)L, p.Tcap, p.Hkv, p.d, p.S, p.Lc);
     } else {
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(landmark_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        landmark_kernel<float><<<grid, NT, smem, st>>>((const float *)K, (const float *)W, (float *)L, p.Tkv,
-                                                         p.Hkv, p.d, p.S, p.C);
+        landmark_kernel<float><<<grid, NT, smem, st>>>((const float *)K, (const float *)W, (float *)L, p.Tcap,
+                                                         p.Hkv, p.d, p.S, p.Lc);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append(const Prob &p, const void *knew, const void *vnew, void *K, void *V, const void *W,
+                                 void *L, cudaStream_t st) {
+    if (p.B == 0) return cudaSuccess;
+    const int complete = (p.Tkv + 1) % p.S == 0 ? 1 : 0;
+    const bool bf = p.dtype == HSA_BF16;
+    const size_t smem = complete ? landmark_smem(p.Hkv * p.d, p.d, bf ? 8 : 4, bf ? 2 : 4) : 0;
+    if (bf) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(decode_append_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        decode_append_kernel<__nv_bfloat16><<<p.B, NT, smem, st>>>(
+            (const __nv_bfloat16 *)knew, (const __nv_bfloat16 *)vnew, (__nv_bfloat16 *)K, (__nv_bfloat16 *)V,
+            (const __nv_bfloat16 *)W, (__nv_bfloat16 *)L, p.Tkv, p.Tcap, p.Hkv, p.d, p.S, p.Lc, complete);
+    } else {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(decode_append_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        decode_append_kernel<float><<<p.B, NT, smem, st>>>((const float *)knew, (const float *)vnew, (float *)K,
+                                                           (float *)V, (const float *)W, (float *)L, p.Tkv, p.Tcap,
+                                                           p.Hkv, p.d, p.S, p.Lc, complete);
     }
     return cudaGetLastError();
 }

@@ -26,6 +26,7 @@ namespace {
 
 struct SelArgs {
     int Tq, H, Hkv, d, S, C, k, kmax, G;
+    int Lc;               // chunks per (b, kv head) in L's layout
     long long q_pos0, rows;
     float tau;
 };
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(const T *__restrict__ 
     float *qs = qsm + warp * a.d;
     load_qbar(Q, a, b, t, j, qs, lane);
     const int ncand = row_ncand(a, t);
-    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * a.d;
+    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.Lc * a.d;
     float v;
     int id;
     list_init(v, id);
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(256) select_split_kernel(const T *__restrict__
     const int ncand = row_ncand(a, t);
     const int c0 = split * chunks_per_split;
     const int c1 = min(ncand, c0 + chunks_per_split);
-    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * a.d;
+    const T *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.Lc * a.d;
     float v;
     int id;
     list_init(v, id);
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(256) select_split_mma_kernel(const __nv_bfloat
             bq[p] = hr < a.G ? __ldg(reinterpret_cast<const uint4 *>(qh + 32 * p + 8 * q)) : make_uint4(0u, 0u, 0u, 0u);
         const int per = ((c1 - c0 + 8 * 32 - 1) / (8 * 32)) * 32;   // a multiple of 32 per warp
         const int w0 = c0 + warp * per, w1 = min(c1, w0 + per);
-        const __nv_bfloat16 *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.C * D;
+        const __nv_bfloat16 *Lj = L + ((size_t)b * a.Hkv + j) * (size_t)a.Lc * D;
         if (w0 < w1) scan_range_mma<D>(bq, Lj, a, w0, w1, v, id, lane);
     }
     if (lane < a.kmax) wl[warp * a.kmax + lane] = make_float2(v, __int_as_float(id));
@@ -384,6 +385,7 @@ SelArgs make_args(const Prob &p) {
     a.d = p.d;
     a.S = p.S;
     a.C = p.C;
+    a.Lc = p.Lc;
     a.k = p.k;
     a.kmax = p.kmax;
     a.G = p.G;

@@ -43,6 +43,7 @@ static_assert(NST % NCW == 0, "each ring stage must belong to one consumer warp"
 
 struct StreamArgs {
     int Tq, H, Hkv, G, S, C, k, kmax;
+    int Lc;               // chunks per (b, kv head) in L's layout
     int ncand, tpr;       // candidates of every row; tiles per row
     long long total;      // rows * tpr
     int grid, maxe;       // CTAs; list slots per row
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 const int s = k % NST, u = k / NST;
                 if (u > 0 && !(ok = mbar_wait(&bar.empty[s], (u - 1) & 1, &bar.abort, a.status))) break;
                 const long long T = lo + k, row = T / a.tpr;
-                const int y = (int)(row * a.C + (T % a.tpr) * TCH);
+                const int y = (int)(row * a.Lc + (T % a.tpr) * TCH);
                 mbar_expect_tx(&bar.full[s], (uint32_t)STB);
 #pragma unroll
                 for (int kb = 0; kb < NB; ++kb)
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 bool select_stream_supported(const Prob &p) {
     const long long ncand = std::min<long long>(p.q_pos0 / p.S, p.C);
     return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && p.Tq == 1 && p.G <= 8 && p.kmax <= 16 &&
-           ncand >= 2048 && (long long)p.B * p.Hkv * p.C < (1ll << 31);
+           ncand >= 2048 && (long long)p.B * p.Hkv * p.Lc < (1ll << 31);
 }
 
 // Grid and list slots of the stream scan (also sizes its workspace).
@@ -292,6 +293,7 @@ cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, in
     a.G = p.G;
     a.S = p.S;
     a.C = p.C;
+    a.Lc = p.Lc;
     a.k = p.k;
     a.kmax = p.kmax;
     a.ncand = (int)std::min<long long>(p.q_pos0 / p.S, p.C);
@@ -302,7 +304,7 @@ cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, in
     a.tau = p.tau;
     a.status = status;
     CUtensorMap ml;
-    cudaError_t e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.C, 64, TCH);
+    cudaError_t e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, TCH);
     if (e != cudaSuccess) return e;
     const size_t smem = 1024 + (size_t)NST * (p.d / 64) * TCH * 128;
     if (p.d == 128) {

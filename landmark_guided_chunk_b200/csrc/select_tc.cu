@@ -53,6 +53,7 @@ constexpr int MAX_KB = 8;      // G*d <= 512
 
 struct TcSelArgs {
     int B, Tq, Hkv, G, d, S, C, k, kmax;
+    int Lc;                  // chunks per (b, kv head) in L's layout
     int nkb, dkb;            // G*d/64 and d/64
     int mtiles, ntiles;
     long long q_pos0;
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(256, 1)
                 if (!ok) break;
                 ++ta;
                 kb_part = 0;
-                const int ly = (T.b * a.Hkv + T.j) * a.C;
+                const int ly = (T.b * a.Hkv + T.j) * a.Lc;
                 for (int n = 0; n < T.nslices; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE;
                     if (i > 0 && !(ok = mbar_wait(&bar->b_empty[s], (i - 1) & 1, abort, a.status))) break;
@@ -362,7 +363,7 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
     CUtensorMap mq, ml;
     cudaError_t e = make_tmap_2d(&mq, Q, (uint64_t)p.H * p.d, (uint64_t)p.B * p.Tq, 64, TM);
     if (e != cudaSuccess) return e;
-    e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.C, 64, NT);
+    e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, NT);
     if (e != cudaSuccess) return e;
     TcSelArgs a;
     a.B = p.B;
@@ -372,6 +373,7 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
     a.d = p.d;
     a.S = p.S;
     a.C = p.C;
+    a.Lc = p.Lc;
     a.k = p.k;
     a.kmax = p.kmax;
     a.nkb = p.G * p.d / 64;

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.EXPORTED)
-    assert lib.hsa_abi_version() == 1
+    assert lib.hsa_abi_version() == 2
 
 
 def test_status_strings():
@@ -58,6 +58,7 @@ def torch_bf16():
     (dict(k=33), _native.HSA_ERR_UNSUPPORTED),
     (dict(k=17, tau=0.1), _native.HSA_ERR_UNSUPPORTED),
     (dict(H=34, Hkv=2), _native.HSA_ERR_UNSUPPORTED),
+    (dict(Tkv=128, kv_cap=127), _native.HSA_ERR_INVALID_ARG),
 ])
 def test_workspace_size_rejects_bad_problems(kw, status):
     with pytest.raises(hsa.HSAError) as e:
@@ -91,6 +92,26 @@ def test_forward_validates_pointers_before_launch():
     assert b"workspace" in _native.lib().hsa_last_error()
     ready = _prob(flags=_native.HSA_FLAG_LANDMARKS_READY)
     assert _call_forward(ready, W=None, L=None) == _native.HSA_ERR_INVALID_ARG   # L is required
+
+
+def _call_append(prob, kn=16, vn=16, K=16, V=16, W=16, L=16):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return _native.lib().hsa_decode_append(ctypes.byref(prob), P(kn), P(vn), P(K), P(V), P(W), P(L), None)
+
+
+def test_decode_append_validates_before_launch():
+    """Fake, never-dereferenced addresses: every call below must fail in host validation."""
+    full = _prob(Tq=1, Tkv=256, kv_cap=256, q_pos0=256)
+    assert _call_append(full) == _native.HSA_ERR_INVALID_ARG                # no room to append
+    assert b"no room" in _native.lib().hsa_last_error()
+    tight = _prob(Tq=1, Tkv=130, kv_cap=0, q_pos0=130)                      # kv_cap 0 = Tkv: full too
+    assert _call_append(tight) == _native.HSA_ERR_INVALID_ARG
+    p = _prob(Tq=1, Tkv=130, kv_cap=256, q_pos0=130)
+    assert _call_append(p, kn=None) == _native.HSA_ERR_INVALID_ARG
+    assert _call_append(p, V=24) == _native.HSA_ERR_INVALID_ARG              # misaligned
+    completes = _prob(Tq=1, Tkv=127, kv_cap=256, q_pos0=127)                 # token 127 completes chunk 1
+    assert _call_append(completes, W=None) == _native.HSA_ERR_INVALID_ARG
+    assert _call_append(completes, L=None) == _native.HSA_ERR_INVALID_ARG
 
 
 def test_null_problem_and_status_reader():
