@@ -80,7 +80,8 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -433,9 +434,69 @@ def run_decode(args, world, rank, local, pk, name="decode_1m"):
            "gpu_launches_per_step": plan["select"][1] + plan["attend"][1]}
     if name == "decode_1m":
         res["loop"] = decode_loop(p, hsa, Q, K, V, W, L, O, ws, st, world)
+    if name == "decode_16m" and p.B == 1:
+        res["sharded_8"] = sharded_share(p, hsa, Q, K, V, L, flush_l2, st, world)
     del inp, Q, K, V, W, L, O, ws, scrub, qs, sels, outs
     torch.cuda.empty_cache()
     return res
+
+
+def sharded_share(p, hsa, Q, K, V, L, flush_l2, st, world, nshard=8):
+    """One rank's share of a context-sharded decode step with the context split
+    8 ways (landmark_guided_chunk_b200.sharded): the local selection and partial
+    outputs over 1/8 of the cache, then the merge of 8 ranks' partials (this
+    rank's, re-indexed as 8 disjoint chunk ranges).  The all-gather between them
+    is not part of it: one GPU per run here."""
+    from landmark_guided_chunk_b200 import sharded
+    C = p.C
+    c1 = C // nshard
+    Kg, Vg = K[:, :c1 * p.S], V[:, :c1 * p.S]            # contiguous: B = 1
+    Lg = L[:, :, :c1].contiguous()
+    prob = hsa.make_problem(p.B, 1, c1 * p.S, p.H, p.Hkv, p.d, p.S, hsa.kmax_of(p.k, p.tau), c1 * p.S, 0.0,
+                            torch.bfloat16)
+    wsg = hsa.alloc_workspace(prob, Q.device)
+    parts = sharded.shard_partials(Q, Kg, Vg, Lg, p.S, p.k, p.tau, p.Tkv, 0, ws=wsg)
+    sc, gi, ke, o = parts
+    stacked = (sc.unsqueeze(0).repeat(nshard, 1, 1, 1, 1),
+               torch.stack([torch.where(gi >= 0, gi + s * c1, gi) for s in range(nshard)]),
+               ke.unsqueeze(0).repeat(nshard, 1, 1, 1), o.unsqueeze(0).repeat(nshard, 1, 1, 1, 1, 1, 1))
+    ts = {"local": [], "merge": []}
+    for _ in range(10):
+        flush_l2()
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(st)
+        sharded.shard_partials(Q, Kg, Vg, Lg, p.S, p.k, p.tau, p.Tkv, 0, ws=wsg)
+        b.record(st)
+        hsa.merge_partials(*stacked, p.S, p.k, p.tau, dtype=Q.dtype)
+        c.record(st)
+        c.synchronize()
+        ts["local"].append(a.elapsed_time(b) * 1e3)
+        ts["merge"].append(b.elapsed_time(c) * 1e3)
+    # back to back: the host's launches run ahead of the device, so this is device time
+    NB = 10
+    bb = []
+    for _ in range(3):
+        flush_l2()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(NB):
+            sharded.shard_partials(Q, Kg, Vg, Lg, p.S, p.k, p.tau, p.Tkv, 0, ws=wsg)
+            hsa.merge_partials(*stacked, p.S, p.k, p.tau, dtype=Q.dtype)
+        b.record(st)
+        b.synchronize()
+        bb.append(a.elapsed_time(b) * 1e3 / NB)
+    hsa.device_status(wsg)
+    loc = max_over_ranks(statistics.median(ts["local"]), world)
+    mrg = max_over_ranks(statistics.median(ts["merge"]), world)
+    b2b = max_over_ranks(statistics.median(bb), world)
+    return {"nshard": nshard, "shard_tokens": c1 * p.S, "us_per_step_per_rank": round(b2b, 2),
+            "single_local_us": round(loc, 2), "single_merge_us": round(mrg, 2),
+            "exchange": f"not measured (one GPU per run): an all-gather of {nshard} x "
+                        f"{(sc.numel() * 8 + ke.numel() * 4 + o.numel() * 4) // 1024} KiB",
+            "timing": f"us_per_step_per_rank: mean of {NB} back-to-back (local + merge) after one L2 flush, median "
+                      "of 3; single_*: one call each after an L2 flush, host launch latency included.  local = "
+                      "selection (k = kmax, router off) + partial outputs over 1/8 of the chunks; merge = 8 ranks' "
+                      "partials into O"}
 
 
 def decode_loop(p, hsa, Q, K, V, W, L, O, ws, st, world):

@@ -193,6 +193,42 @@ HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *p, const void *Q, c
  * idx, score and keff may each be NULL.  The selection then lives only in the
  * workspace.
  */
+/*
+ * Context-sharded decode, per shard (summary page, Implementation: the
+ * retrieval scores rank the chunks and weight their outputs).  The chunks of
+ * a sequence may be split into contiguous ranges held by different devices
+ * (shards): each shard selects its own top kmax chunks (hsa_select with
+ * k = kmax and tau = 0, so its list is never cut by the router) and computes
+ * here, for every selection row and kept slot i < keff, the chunk's attention
+ * output for each of the G query heads, without the fusion weight:
+ *   o_part[b][t][j][i][g][:] = softmax_u(q_{jG+g} . K[c_i S + u] / sqrt(d)) . V[c_i S + u]
+ * (fp32, [B][Tq][Hkv][kmax][G][d]; slots i >= keff are not written).  idx holds
+ * the shard's local chunk indices.  bf16 only, d 64/128; the rows' chunks are
+ * all gathered at once, which suits decode (few rows).  Uses the workspace's
+ * status word only (hsa_workspace_size of the same problem suffices).
+ */
+HSA_API hsa_status_t hsa_attend_partials(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
+                                         const int32_t *idx, const int32_t *keff, float *o_part, void *ws,
+                                         size_t ws_bytes, void *stream);
+
+/*
+ * Context-sharded decode, the merge: from the nshard shards' selections and
+ * partial outputs, concatenated shard-major as an all-gather leaves them --
+ *   score, idx [nshard][B][Tq][Hkv][kmax] (idx: GLOBAL chunk indices),
+ *   keff [nshard][B][Tq][Hkv], o_part [nshard][B][Tq][Hkv][kmax][G][d] --
+ * the rows' selection over the whole context (the top kmax of the union, same
+ * order and ties as hsa_select; then keff = min(k, #kept), doubled by the gap
+ * router as in hsa_select) and the output
+ *   O[b][t][jG+g][:] = sum_{i < keff} softmax_i(score_i) o_part[shard_i][b][t][j][slot_i][g][:].
+ * The problem describes one shard's rows (B, Tq, H, Hkv, d, k, tau, dtype);
+ * its Tkv is not used.  idx_out, score_out ([B][Tq][Hkv][kmax]) and keff_out
+ * may each be NULL.  Needs nshard * kmax <= 256 and G * d <= 2048.  No
+ * workspace.
+ */
+HSA_API hsa_status_t hsa_merge_partials(const hsa_problem_t *p, int nshard, const float *score,
+                                        const int32_t *idx, const int32_t *keff, const float *o_part, void *O,
+                                        int32_t *idx_out, float *score_out, int32_t *keff_out, void *stream);
+
 HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                          const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
                          void *O, void *ws, size_t ws_bytes, void *stream);

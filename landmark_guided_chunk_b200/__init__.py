@@ -21,7 +21,8 @@ from . import _native
 from ._native import HSAError, hsa_problem_t
 
 __all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "select_noalloc", "attend",
-           "forward", "decode_append", "device_status", "HSAError", "hsa_problem_t", "kmax_of"]
+           "forward", "decode_append", "attend_partials", "merge_partials", "device_status", "HSAError",
+           "hsa_problem_t", "kmax_of"]
 
 _DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
 
@@ -204,6 +205,50 @@ def decode_append(K, V, k_new, v_new, kv_len, S, W_L=None, L=None) -> bool:
     _native.check(_native.lib().hsa_decode_append(ctypes.byref(prob), _p(k_new), _p(v_new), _p(K), _p(V),
                                                    _p(W_L), _p(L), _stream(K)), "hsa_decode_append")
     return (kv_len + 1) % S == 0
+
+
+def attend_partials(Q, K, V, idx, keff, S, k, tau=0.0, q_pos0=0, kv_len=None, out=None, ws=None):
+    """One shard's chunk outputs for its selection, without fusion: o [B,Tq,Hkv,kmax,G,d] fp32,
+    o[b,t,j,i,g] = softmax(q_{jG+g} K_{c_i}^T / sqrt(d)) V_{c_i} for i < keff (others unwritten).
+    idx holds the shard's local chunk indices."""
+    _dev(Q, K, V, idx, keff, out, ws)
+    B, Tq, H, d = Q.shape
+    Tcap, Hkv = K.shape[1], K.shape[2]
+    prob = _prob_from(Q, Tcap if kv_len is None else kv_len, Hkv, S, k, tau, q_pos0, 0, Tcap)
+    km = kmax_of(k, tau)
+    if out is None:
+        out = torch.empty(B, Tq, Hkv, km, H // Hkv, d, dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = alloc_workspace(prob, Q.device)
+    _native.check(_native.lib().hsa_attend_partials(ctypes.byref(prob), _p(Q), _p(K), _p(V), _p(idx), _p(keff),
+                                                    _p(out), _p(ws), ws.numel(), _stream(Q)),
+                  "hsa_attend_partials")
+    return out
+
+
+def merge_partials(score, idx, keff, o_part, S, k, tau=0.0, dtype=torch.bfloat16, O=None,
+                   return_selection=False):
+    """Merge of nshard shards' selections and partial outputs, concatenated shard-major
+    (score, idx [P,B,Tq,Hkv,kmax] with global chunk indices, keff [P,B,Tq,Hkv],
+    o_part [P,B,Tq,Hkv,kmax,G,d]) into O [B,Tq,H,d] of dtype, and with return_selection
+    also the merged (idx, score, keff)."""
+    _dev(score, idx, keff, o_part, O)
+    P, B, Tq, Hkv, km, G, d = o_part.shape
+    if km != kmax_of(k, tau):
+        raise ValueError(f"partials hold {km} slots per row, but k={k}, tau={tau} merge into {kmax_of(k, tau)}")
+    H = Hkv * G
+    prob = make_problem(B, Tq, 0, H, Hkv, d, S, k, 0, tau, dtype)
+    if O is None:
+        O = torch.empty(B, Tq, H, d, dtype=dtype, device=o_part.device)
+    sel = (None, None, None)
+    if return_selection:
+        sel = (torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=o_part.device),
+               torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=o_part.device),
+               torch.empty(B, Tq, Hkv, dtype=torch.int32, device=o_part.device))
+    _native.check(_native.lib().hsa_merge_partials(ctypes.byref(prob), P, _p(score), _p(idx), _p(keff), _p(o_part),
+                                                   _p(O), _p(sel[0]), _p(sel[1]), _p(sel[2]), _stream(o_part)),
+                  "hsa_merge_partials")
+    return (O,) + sel if return_selection else O
 
 
 def device_status(ws: torch.Tensor) -> None:

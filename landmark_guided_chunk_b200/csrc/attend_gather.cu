@@ -88,13 +88,14 @@ __device__ __forceinline__ void red_add2(float *addr, float x, float y) {
 }
 
 // One staged chunk (K boxes at sK, V boxes at sV): the group's attention
-// output, times w / (softmax denominator), added into acc[g][d0..d0+DW) for
-// g < G.  wait_v() is called between the softmax and the PV product (V may
-// still be landing while the scores are computed); if it returns false the
-// product is skipped and the function returns false.
-template <int D, int S, int DW, typename WaitV>
+// output, times w / (softmax denominator), handed to emit(g, col, x, y) for
+// the column pair (col, col+1) of head g < G, columns [d0, d0+DW).  wait_v()
+// is called between the softmax and the PV product (V may still be landing
+// while the scores are computed); if it returns false the product is skipped
+// and the function returns false.
+template <int D, int S, int DW, typename WaitV, typename Emit>
 __device__ __forceinline__ bool chunk_unit(uint32_t sK, uint32_t sV, const uint32_t (&qa)[D / 16][4], int G,
-                                           float scale, float w, int d0, float *acc, WaitV wait_v) {
+                                           float scale, float w, int d0, Emit emit, WaitV wait_v) {
     constexpr int BOX = S * 128;     // bytes per box
     constexpr int KS = D / 16;       // k-steps of the score MMA
     constexpr int QN = S / 8;        // n-tiles of the score tile
@@ -171,8 +172,8 @@ __device__ __forceinline__ bool chunk_unit(uint32_t sK, uint32_t sV, const uint3
 #pragma unroll
     for (int n = 0; n < ON; ++n) {
         const int col = d0 + 8 * n + q2;
-        if (g0 < G) red_add2(acc + (size_t)g0 * D + col, o[n][0] * f0, o[n][1] * f0);
-        if (g1 < G) red_add2(acc + (size_t)g1 * D + col, o[n][2] * f1, o[n][3] * f1);
+        if (g0 < G) emit(g0, col, o[n][0] * f0, o[n][1] * f0);
+        if (g1 < G) emit(g1, col, o[n][2] * f1, o[n][3] * f1);
     }
     return true;
 }
@@ -186,6 +187,7 @@ struct GatherArgs {
     long long q_pos0;
     float scale;        // 1/sqrt(d)
     uint32_t *status;   // workspace status word
+    float *part;        // partial mode: o_i of every (row, slot) [rows][kmax][G][D], unweighted; else null
 };
 
 // Every warp is an independent worker with one chunk stage of its own; a CTA is
@@ -198,7 +200,7 @@ struct GatherArgs {
 // row's fp32 accumulator.  The per-row completion counters are bumped after
 // all of the worker's additions, behind a single fence; the warp that
 // completes a row converts its accumulator to bf16 O.
-template <int D, int S>
+template <int D, int S, bool PART>
 __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                   const __grid_constant__ CUtensorMap tmV,
                                                                   const __nv_bfloat16 *__restrict__ Q,
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
             ke = keff[row];
             c = idx[(size_t)row * a.kmax + i];
         }
-        const float sv = lane < a.kmax ? score[(size_t)row * a.kmax + lane] : -INFINITY;
+        const float sv = (!PART && lane < a.kmax) ? score[(size_t)row * a.kmax + lane] : -INFINITY;
         uint32_t qa[D / 16][4];
         load_q_frags<D>(Q + qrow, a.G, qa);
         ke = __shfl_sync(FULL, ke, 0);
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
             pend_k = pend_v = true;
         }
         if (c == -2) {
-            if (ke == 0 && i == 0)   // no candidates: the output is zero
+            if (ke == 0 && i == 0 && !PART)   // no candidates: the output is zero
                 for (int e = lane; e < a.G * D; e += 32) O[qrow + e] = __float2bfloat16(0.f);
             continue;
         }
@@ -303,7 +305,19 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
                 if (v) pend_v = false;
                 return __all_sync(FULL, v) && !s_abort;
             };
-            chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, w, 0, acc + (size_t)row * a.G * D, wait_v);
+            if constexpr (!PART) {
+                float *racc = acc + (size_t)row * a.G * D;
+                chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, w, 0,
+                                    [&](int g, int col, float x, float y) { red_add2(racc + (size_t)g * D + col, x, y); },
+                                    wait_v);
+            } else {   // partial output of this slot: o_i unweighted, plain stores
+                float *po = a.part + ((size_t)row * a.kmax + i) * a.G * D;
+                chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, 1.0f, 0,
+                                    [&](int g, int col, float x, float y) {
+                                        *reinterpret_cast<float2 *>(po + (size_t)g * D + col) = make_float2(x, y);
+                                    },
+                                    wait_v);
+            }
         }
         if (issued && !pend_k && !pend_v) phase ^= 1u;   // both copies consumed (after an expired wait they stay pending)
         __syncwarp();   // the stage is free for the next unit
@@ -311,8 +325,8 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
 
     // completion counters, behind one fence for all of this worker's additions;
     // whoever completes a row's last slot converts the row's accumulator to O
-    __threadfence();
-    for (int r = 0; r < nr; ++r) {
+    if (!PART) __threadfence();
+    for (int r = 0; r < nr && !PART; ++r) {
         const int row = __shfl_sync(FULL, m_row, r), ke = __shfl_sync(FULL, m_ke, r), c = __shfl_sync(FULL, m_c, r);
         if (c == -2) continue;
         int last = 0;
@@ -335,7 +349,7 @@ __global__ void __launch_bounds__(MAXW * 32) attend_gather_kernel(const __grid_c
     if (lane == 0 && pend_v) mbar_drain(mbv, phase);
 }
 
-template <int D, int S>
+template <int D, int S, bool PART>
 cudaError_t launch_ds(const Prob &p, GatherArgs a, const CUtensorMap &mk, const CUtensorMap &mv, const void *Q,
                       const int32_t *idx, const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
                       cudaStream_t st) {
@@ -344,12 +358,13 @@ cudaError_t launch_ds(const Prob &p, GatherArgs a, const CUtensorMap &mk, const 
     a.nw = nw < 1 ? 1 : (nw > MAXW ? MAXW : nw);
     const size_t smem = 1024 + (size_t)a.nw * STAGE;
     cudaError_t e =
-        cudaFuncSetAttribute(attend_gather_kernel<D, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(attend_gather_kernel<D, S, PART>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148, per_sm = 1;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attend_gather_kernel<D, S>, a.nw * 32, smem)) !=
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attend_gather_kernel<D, S, PART>, a.nw * 32,
+                                                           smem)) !=
         cudaSuccess)
         return e;
     if (per_sm < 1) per_sm = 1;
@@ -358,19 +373,19 @@ cudaError_t launch_ds(const Prob &p, GatherArgs a, const CUtensorMap &mk, const 
     if (grid < min_grid) grid = min_grid;
     const long long max_grid = (a.nunits + a.nw - 1) / a.nw;   // no CTA without units
     if (grid > max_grid) grid = max_grid;
-    attend_gather_kernel<D, S><<<(unsigned)grid, a.nw * 32, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, idx, score,
-                                                                       keff, (__nv_bfloat16 *)O, acc, cnt, a);
+    attend_gather_kernel<D, S, PART><<<(unsigned)grid, a.nw * 32, smem, st>>>(
+        mk, mv, (const __nv_bfloat16 *)Q, idx, score, keff, (__nv_bfloat16 *)O, acc, cnt, a);
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool PART>
 cudaError_t launch_d(const Prob &p, const GatherArgs &a, const CUtensorMap &mk, const CUtensorMap &mv, const void *Q,
                      const int32_t *idx, const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
                      cudaStream_t st) {
     switch (p.S) {
-        case 32: return launch_ds<D, 32>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
-        case 64: return launch_ds<D, 64>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
-        case 128: return launch_ds<D, 128>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+        case 32: return launch_ds<D, 32, PART>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+        case 64: return launch_ds<D, 64, PART>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+        case 128: return launch_ds<D, 128, PART>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -384,8 +399,9 @@ bool attend_gather_supported(const Prob &p) {
 
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
                                  const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
-                                 uint32_t *status, cudaStream_t st) {
+                                 uint32_t *status, cudaStream_t st, float *part) {
     GatherArgs a;
+    a.part = part;
     a.B = p.B;
     a.Tq = p.Tq;
     a.Tcap = p.Tcap;
@@ -408,8 +424,12 @@ cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, co
     cudaError_t e;
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
-    if (p.d == 128) return launch_d<128>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
-    return launch_d<64>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+    if (part != nullptr) {
+        if (p.d == 128) return launch_d<128, true>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+        return launch_d<64, true>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+    }
+    if (p.d == 128) return launch_d<128, false>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
+    return launch_d<64, false>(p, a, mk, mv, Q, idx, score, keff, O, acc, cnt, st);
 }
 
 }  // namespace hsa

@@ -278,9 +278,15 @@ void select_stream_shape(const Prob &p, int sms, int *grid, int *maxe);
 cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
                                  int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
                                  cudaStream_t st);
+// part != null: partial mode (o_i of every (row, slot) into part [rows][kmax][G][d]; no fusion, O unused)
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
                                  const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,
-                                 uint32_t *status, cudaStream_t st);
+                                 uint32_t *status, cudaStream_t st, float *part = nullptr);
+// The merge of per-shard selections and partial outputs into one row's output (merge.cu).
+cudaError_t launch_merge_partials(const Prob &p, int nshard, const float *score, const int32_t *idx,
+                                  const int32_t *keff, const float *part, void *O, int32_t *idx_out, float *score_out,
+                                  int32_t *keff_out, cudaStream_t st);
+bool merge_supported(const Prob &p, int nshard);
 AttTcLayout attend_tc_layout(const Prob &p);
 int attend_tc_launches(const AttTcLayout &L);
 cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuffers &bf, const void *Q, const void *K,

@@ -293,6 +293,50 @@ hsa_status_t hsa_attend(const hsa_problem_t *prob, const void *Q, const void *K,
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "attention kernel launch");
 }
 
+hsa_status_t hsa_attend_partials(const hsa_problem_t *prob, const void *Q, const void *K, const void *V,
+                                 const int32_t *idx, const int32_t *keff, float *o_part, void *ws, size_t ws_bytes,
+                                 void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (p.rows > 0 && !attend_gather_supported(p))
+        return fail(HSA_ERR_UNSUPPORTED, "partial outputs need the chunk-gather path (bf16, d 64/128, G <= 16)");
+    const bool rows = p.rows > 0;
+    HSA_TRY(need(Q, rows, "Q"));
+    HSA_TRY(need(K, rows && p.C > 0, "K"));
+    HSA_TRY(need(V, rows && p.C > 0, "V"));
+    HSA_TRY(need(idx, rows, "idx"));
+    HSA_TRY(need(keff, rows, "keff"));
+    HSA_TRY(need(o_part, rows, "o_part"));
+    const WsLayout w = ws_layout(p);
+    HSA_TRY(check_ws(w, ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    HSA_TRY(clear_status((char *)ws, w, st));
+    if (!rows || p.C == 0) return HSA_OK;
+    cudaError_t e = launch_attend_gather(p, Q, K, V, idx, nullptr, keff, nullptr, nullptr, nullptr,
+                                         reinterpret_cast<uint32_t *>((char *)ws + w.hdr), st, o_part);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "partial attention kernel launch");
+}
+
+hsa_status_t hsa_merge_partials(const hsa_problem_t *prob, int nshard, const float *score, const int32_t *idx,
+                                const int32_t *keff, const float *o_part, void *O, int32_t *idx_out,
+                                float *score_out, int32_t *keff_out, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (nshard < 1) return fail(HSA_ERR_INVALID_ARG, "nshard=%d", nshard);
+    if (!merge_supported(p, nshard))
+        return fail(HSA_ERR_UNSUPPORTED, "merge of %d shards x %d slots, G*d=%d (max 256 candidates, G*d <= 2048)",
+                    nshard, p.kmax, p.G * p.d);
+    const bool rows = p.rows > 0;
+    HSA_TRY(need(score, rows, "score"));
+    HSA_TRY(need(idx, rows, "idx"));
+    HSA_TRY(need(keff, rows, "keff"));
+    HSA_TRY(need(o_part, rows, "o_part"));
+    HSA_TRY(need(O, rows, "O"));
+    cudaError_t e = launch_merge_partials(p, nshard, score, idx, keff, o_part, O, idx_out, score_out, keff_out,
+                                          (cudaStream_t)stream);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "merge kernel launch");
+}
+
 hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const void *W_L,
                          void *L, int32_t *idx, float *score, int32_t *keff, void *O, void *ws, size_t ws_bytes,
                          void *stream) {

@@ -246,9 +246,17 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     if (!__shfl_sync(FULL, last, 0)) return;
     __threadfence();
     list_init(v, id);
-    for (int e = 0; e <= x1 - x0; ++e) {
-        const float2 f = lane < a.kmax ? __ldcg(rl + e * a.kmax + lane) : make_float2(-INFINITY, __int_as_float(INT32_MAX));
-        list_merge16(v, id, f.x, __float_as_int(f.y), a.kmax, lane);
+    // the row's lists, eight in flight per round trip (then merged in order)
+    const int ne = x1 - x0 + 1;
+    for (int e0 = 0; e0 < ne; e0 += 8) {
+        float2 f[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            f[u] = (e0 + u < ne && lane < a.kmax) ? __ldcg(rl + (e0 + u) * a.kmax + lane)
+                                                  : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (e0 + u < ne) list_merge16(v, id, f[u].x, __float_as_int(f[u].y), a.kmax, lane);
     }
     const int ke = list_keff(v, a.ncand, a.k, a.kmax, a.tau);
     if (lane < a.kmax) {
