@@ -128,9 +128,9 @@ __global__ void __launch_bounds__(256, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;                                   // nkb boxes
     uint8_t *sB = base + (size_t)a.nkb * BOX;             // NSTAGE x dkb boxes
-    float *qv = reinterpret_cast<float *>(sB + (size_t)NSTAGE * a.dkb * BOX);   // [32][128] queued scores
-    int *qi = reinterpret_cast<int *>(qv + 32 * 128);                          // [32][128] queued chunks
-    Bars *bar = reinterpret_cast<Bars *>(qi + 32 * 128);
+    // [32][128] queued (score, chunk as int bits): one 8-byte store per queued candidate
+    float2 *qvi = reinterpret_cast<float2 *>(sB + (size_t)NSTAGE * a.dkb * BOX);
+    Bars *bar = reinterpret_cast<Bars *>(qvi + 32 * 128);
     volatile int *abort = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(256, 1)
                 v[q] = -INFINITY;
                 id[q] = -1;
             }
-            int head = 0, tail = 0;   // this row's FIFO of pending (score, chunk): ring of 32 in qv/qi
+            int head = 0, tail = 0;   // this row's FIFO of pending (score, chunk): ring of 32 in qvi
             for (int n = 0; n < T.nslices; ++n, ++g) {
                 const int buf = g & 1, u = g >> 1;
                 if (!(ok = mbar_wait(&bar->t_full[buf], u & 1, abort, a.status))) break;
@@ -287,8 +287,7 @@ __global__ void __launch_bounds__(256, 1)
                         const bool take = (cb + e < nc) && (sv > thr);
                         const int slot = (tail & 31) * 128 + r;
                         if (take) {
-                            qv[slot] = sv;
-                            qi[slot] = cb + e;
+                            qvi[slot] = make_float2(sv, __int_as_float(cb + e));
                         }
                         tail += take ? 1 : 0;
                     }
@@ -302,8 +301,9 @@ __global__ void __launch_bounds__(256, 1)
                     for (int it = 0; it < dn; ++it) {
                         const bool has = head < tail;
                         const int slot = (head & 31) * 128 + r;
-                        const float x = has ? qv[slot] : -INFINITY;
-                        const int xi = has ? qi[slot] : 0;
+                        const float2 qe = has ? qvi[slot] : make_float2(-INFINITY, 0.f);
+                        const float x = qe.x;
+                        const int xi = __float_as_int(qe.y);
                         head += has ? 1 : 0;
                         list_push<KL>(v, id, x, xi);
                     }
@@ -316,8 +316,8 @@ __global__ void __launch_bounds__(256, 1)
                 // drained queue: selecting them from registers by a runtime index would
                 // move the whole list into local memory
 #pragma unroll
-                for (int q = 0; q < KL; ++q) qv[q * 128 + r] = v[q];
-                const float sk = qv[(a.k - 1) * 128 + r], sk1 = qv[a.k * 128 + r];
+                for (int q = 0; q < KL; ++q) qvi[q * 128 + r].x = v[q];
+                const float sk = qvi[(a.k - 1) * 128 + r].x, sk1 = qvi[a.k * 128 + r].x;
                 if (sk - sk1 < a.tau * fabsf(sk)) ke = nc < 2 * a.k ? nc : 2 * a.k;
             }
             const long long row = ((long long)T.b * a.Tq + t) * a.Hkv + T.j;
