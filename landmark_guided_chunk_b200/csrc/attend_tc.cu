@@ -475,10 +475,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
             const int n_mine = tile_hi - tile_lo;
-            // K/V load index of each tile, derived from the tile records exactly as the producer does
+            // K/V load index of each tile, derived from the tile records exactly as the loader does;
+            // the records come four tiles ahead, so their L2 round trips stay off this loop
             int key_p = -1, key_c = -1, nload = 0;
-            auto load_of = [&](int i) -> int {   // call with i = 0, 1, 2, ... in order
-                const int4 e = a.tiles[tile_lo + i];
+            auto load_of = [&](int4 e) -> int {   // call with the records of tiles 0, 1, 2, ... in order
                 if (e.x != key_p || e.y != key_c) {
                     key_p = e.x;
                     key_c = e.y;
@@ -486,6 +486,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 }
                 return nload - 1;
             };
+            auto rec = [&](int t) -> int4 { return t < n_mine ? a.tiles[tile_lo + t] : make_int4(-1, -1, 0, 0); };
+            int4 w1 = rec(1), w2 = rec(2), w3 = rec(3), w4 = rec(4);
             int waited_load = -1;   // last load whose kv_full has been waited on
             // QK(i) writes S buffer i & 1, whose previous tile (i - 2) the softmax has released
             // through p_full before PV(i - 2) was issued, which precedes this call.
@@ -511,11 +513,15 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 return true;
             };
             const bool early = a.nskv >= 2;
-            int li = n_mine > 0 ? load_of(0) : 0;
+            int li = n_mine > 0 ? load_of(rec(0)) : 0;
             bool ok = n_mine > 0 ? issue_qk(0, li) : true;
             for (int i = 0; i < n_mine && ok; ++i) {
                 const int b = i & 1, k = i >> 1;
-                const int li_next = i + 1 < n_mine ? load_of(i + 1) : -1;
+                const int li_next = i + 1 < n_mine ? load_of(w1) : -1;
+                w1 = w2;
+                w2 = w3;
+                w3 = w4;
+                w4 = rec(i + 5);
                 if (early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
                 if (!(ok = mbar_wait(&bar->p_full[b], k & 1, abort, a.status))) break;
                 if (k > 0 && !(ok = mbar_wait(&bar->o_empty[b], (k - 1) & 1, abort, a.status))) break;
