@@ -14,7 +14,9 @@ conversion; landmarks against numpy chunk means (W_L = I), a one-hot W_L
 brute force with ties, the strict-past candidate rule, the group sum and the
 router limits; attention against closed forms (constant-V chunks, V = 1, a
 two-chunk sigmoid, a single aligned key), convexity, torch SDPA for single
-candidate rows, and the exhaustive limit k >= #candidates.
+candidate rows, and the exhaustive limit k >= #candidates; the backward against
+central finite differences of the forward above (selection held fixed) and the
+closed forms of its sums (sum_u dV_u, the per-chunk sum of dK, sum_i ds_i = 0).
 """
 from __future__ import annotations
 
@@ -39,8 +41,10 @@ def _load():
         lib.hsa_oracle_landmarks.argtypes = [I, I, LL, I, I, I, P, P, P]
         lib.hsa_oracle_select.argtypes = [I, I, I, I, I, LL, I, D, I, LL, P, P, P, P, P, P, P, P]
         lib.hsa_oracle_attend.argtypes = [I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P]
+        lib.hsa_oracle_backward.argtypes = [I, I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P, P,
+                                            P, P, P, P, P]
         for f in (lib.hsa_oracle_round, lib.hsa_oracle_landmarks, lib.hsa_oracle_select,
-                  lib.hsa_oracle_attend):
+                  lib.hsa_oracle_attend, lib.hsa_oracle_backward):
             f.restype = None
         _lib = lib
     return _lib
@@ -201,5 +205,36 @@ def forward_rows(Q, K, V, W_L, S: int, k: int, tau: float, q_pos0: int, rows_b, 
     return {"L": L, "sel": sel, "O": O}
 
 
+def backward(Qr, row_b, K, V, W_L, L, S: int, sel: dict, dO) -> dict:
+    """Gradients of the method for rows Qr [n,H,d] (batches row_b) with the
+    selection ``sel`` (idx, keff; chunk indices into K, V [B,Tkv,Hkv,d]) held
+    fixed.  L [B,Hkv,C,d] holds the landmarks the scores are taken from; dO
+    [n,H,d] is the output gradient.  Returns fp64 dQ [n,H,d], dK, dV
+    [B,Tkv,Hkv,d], dW [d,d] and dL [B,Hkv,C,d]."""
+    dq, Qa = _buf(Qr)
+    dk, Ka = _buf(K)
+    dv, Va = _buf(V)
+    dw, Wa = _buf(W_L)
+    if not (dq == dk == dv == dw):
+        raise TypeError("Q, K, V, W_L must share a dtype")
+    n, H, d = Qa.shape
+    B, Tkv, Hkv, _ = Ka.shape
+    L = np.ascontiguousarray(L, dtype=np.float64)
+    if L.shape != (B, Hkv, Tkv // S, d):
+        raise ValueError(f"L has shape {L.shape}, expected {(B, Hkv, Tkv // S, d)}")
+    idx = np.ascontiguousarray(sel["idx"], dtype=np.int32)
+    keff = np.ascontiguousarray(sel["keff"], dtype=np.int32)
+    kmax = idx.shape[-1]
+    rb = np.ascontiguousarray(row_b, dtype=np.int32)
+    g = np.ascontiguousarray(dO.detach().cpu().double().numpy() if isinstance(dO, torch.Tensor) else dO,
+                             dtype=np.float64)
+    out = {"dQ": np.empty((n, H, d)), "dK": np.empty((B, Tkv, Hkv, d)), "dV": np.empty((B, Tkv, Hkv, d)),
+           "dW": np.empty((d, d)), "dL": np.empty((B, Hkv, L.shape[2], d))}
+    _load().hsa_oracle_backward(dq, B, Tkv, H, Hkv, d, S, kmax, n, _ptr(rb), _ptr(Qa), _ptr(Ka), _ptr(Va),
+                                _ptr(Wa), _ptr(L), _ptr(idx), _ptr(keff), _ptr(g), _ptr(out["dQ"]),
+                                _ptr(out["dK"]), _ptr(out["dV"]), _ptr(out["dW"]), _ptr(out["dL"]))
+    return out
+
+
 __all__ = ["round_to", "landmarks", "landmarks_stored", "landmarks_stored_sliced", "select", "attend",
-           "attend_gathered", "forward_rows"]
+           "attend_gathered", "forward_rows", "backward"]

@@ -224,3 +224,167 @@ void hsa_oracle_attend(int dt, long long Tkv, int H, int Hkv, int d, int S, int 
         free(w); free(a); free(o);
     }
 }
+
+/*
+ * Gradients of the method with the selection held fixed (the chunk choice is a
+ * discrete decision: it has no gradient, and the kept chunks' scores still
+ * carry one through the fusion weights).  The forward this differentiates,
+ * for the rows given and kv head j, each head h of its group and kept slot i:
+ *   s_i  = sum_{h in group} q_h . L[c_i]          (L = mean-pooled keys * W_L)
+ *   w    = softmax_i(s)                           (i < keff)
+ *   a_iu = softmax_u(q_h . K[c_i S + u] / sqrt(d)),  o_hi = sum_u a_iu V[c_i S + u]
+ *   O_h  = sum_i w_i o_hi
+ * Given dO [n][H][d] (double), the chain rule gives, in this order:
+ *   e_hi  = dO_h . o_hi,   dw_i = sum_h e_hi,   ds_i = w_i (dw_i - sum_i' w_i' dw_i')
+ *   dq_h += sum_i ds_i L[c_i],                  dL[c_i] += ds_i q_h
+ *   with g = w_i dO_h:  dV_u += a_iu g,  dz_u = a_iu (g . V_u - g . o_hi),
+ *                       dq_h += (1/sqrt d) sum_u dz_u K_u,  dK_u += (1/sqrt d) dz_u q_h
+ * and, through the landmark of every complete chunk c (m_c = its key mean):
+ *   dW_L += m_c^T dL[c],   dK_u += (dL[c] W_L^T) / S   for the S keys of chunk c.
+ * Inputs: Qr [n][H][d] (dt), row_b [n], K, V [B][Tkv][Hkv][d] (dt), W [d][d]
+ * (dt), L [B][Hkv][C][d] (double: the landmarks the scores are taken from),
+ * idx, keff as from hsa_oracle_select.  Outputs, all double and OVERWRITTEN:
+ * dQ [n][H][d], dK, dV [B][Tkv][Hkv][d], dW [d][d], dL [B][Hkv][C][d].
+ * L enters the scores as given, so rounding it to a storage dtype is taken as
+ * the identity in the chain rule (the rounding has no useful derivative).
+ */
+void hsa_oracle_backward(int dt, int B, long long Tkv, int H, int Hkv, int d, int S, int kmax,
+                         long long n, const int *row_b, const void *Qr, const void *K,
+                         const void *V, const void *W, const double *L, const int *idx,
+                         const int *keff, const double *dO, double *dQ, double *dK,
+                         double *dV, double *dW, double *dL)
+{
+    int G = H / Hkv;
+    long long C = Tkv / S;
+    double scale = 1.0 / sqrt((double)d);
+    memset(dQ, 0, sizeof(double) * (size_t)n * H * d);
+    memset(dK, 0, sizeof(double) * (size_t)B * Tkv * Hkv * d);
+    memset(dV, 0, sizeof(double) * (size_t)B * Tkv * Hkv * d);
+    memset(dW, 0, sizeof(double) * (size_t)d * d);
+    memset(dL, 0, sizeof(double) * (size_t)B * Hkv * C * d);
+    /* kv heads touch disjoint parts of dQ, dK, dV and dL: one thread per head */
+#pragma omp parallel for schedule(static)
+    for (int j = 0; j < Hkv; ++j) {
+        double *w = (double *)malloc(sizeof(double) * (size_t)kmax);
+        double *dw = (double *)malloc(sizeof(double) * (size_t)kmax);
+        double *e = (double *)malloc(sizeof(double) * (size_t)kmax * G);
+        double *a = (double *)malloc(sizeof(double) * (size_t)kmax * G * S);   /* a[(i*G+g)*S+u] */
+        double *o = (double *)malloc(sizeof(double) * (size_t)kmax * G * d);   /* o[(i*G+g)*d+x] */
+        for (long long r = 0; r < n; ++r) {
+            size_t b = (size_t)row_b[r];
+            size_t so = ((size_t)r * Hkv + j) * kmax;
+            int ke = keff[(size_t)r * Hkv + j];
+            if (ke <= 0) continue;
+            const double *Lj = L + (b * Hkv + j) * (size_t)C * d;
+            /* scores and fusion weights */
+            double m = -INFINITY, z = 0.0;
+            for (int i = 0; i < ke; ++i) {
+                double s = 0.0;
+                for (int g = 0; g < G; ++g)
+                    for (int x = 0; x < d; ++x)
+                        s += load(Qr, ((size_t)r * H + j * G + g) * d + x, dt) * Lj[(size_t)idx[so + i] * d + x];
+                w[i] = s;
+                if (s > m) m = s;
+            }
+            for (int i = 0; i < ke; ++i) { w[i] = exp(w[i] - m); z += w[i]; }
+            for (int i = 0; i < ke; ++i) w[i] /= z;
+            /* in-chunk attention of every (slot, head) and e = dO . o */
+            for (int i = 0; i < ke; ++i) {
+                size_t c = (size_t)idx[so + i];
+                for (int g = 0; g < G; ++g) {
+                    size_t qh = ((size_t)r * H + j * G + g) * d;
+                    double *ai = a + ((size_t)i * G + g) * S, *oi = o + ((size_t)i * G + g) * d;
+                    double amax = -INFINITY, l = 0.0;
+                    for (int u = 0; u < S; ++u) {
+                        size_t kr = ((b * (size_t)Tkv + c * S + u) * Hkv + j) * (size_t)d;
+                        double dot = 0.0;
+                        for (int x = 0; x < d; ++x) dot += load(Qr, qh + x, dt) * load(K, kr + x, dt);
+                        ai[u] = dot * scale;
+                        if (ai[u] > amax) amax = ai[u];
+                    }
+                    for (int u = 0; u < S; ++u) { ai[u] = exp(ai[u] - amax); l += ai[u]; }
+                    for (int u = 0; u < S; ++u) ai[u] /= l;
+                    for (int x = 0; x < d; ++x) oi[x] = 0.0;
+                    for (int u = 0; u < S; ++u) {
+                        size_t vr = ((b * (size_t)Tkv + c * S + u) * Hkv + j) * (size_t)d;
+                        for (int x = 0; x < d; ++x) oi[x] += ai[u] * load(V, vr + x, dt);
+                    }
+                    double ev = 0.0;
+                    for (int x = 0; x < d; ++x) ev += dO[qh + x] * oi[x];
+                    e[(size_t)i * G + g] = ev;
+                }
+            }
+            /* fusion softmax: dw, then ds */
+            double wdw = 0.0;
+            for (int i = 0; i < ke; ++i) {
+                dw[i] = 0.0;
+                for (int g = 0; g < G; ++g) dw[i] += e[(size_t)i * G + g];
+                wdw += w[i] * dw[i];
+            }
+            for (int i = 0; i < ke; ++i) {
+                double ds = w[i] * (dw[i] - wdw);
+                size_t c = (size_t)idx[so + i];
+                double *dLc = dL + ((b * Hkv + j) * (size_t)C + c) * d;
+                for (int g = 0; g < G; ++g) {
+                    size_t qh = ((size_t)r * H + j * G + g) * d;
+                    for (int x = 0; x < d; ++x) {
+                        dQ[qh + x] += ds * Lj[c * d + x];
+                        dLc[x] += ds * load(Qr, qh + x, dt);
+                    }
+                }
+            }
+            /* in-chunk attention backward with the output gradient w_i dO_h */
+            for (int i = 0; i < ke; ++i) {
+                size_t c = (size_t)idx[so + i];
+                for (int g = 0; g < G; ++g) {
+                    size_t qh = ((size_t)r * H + j * G + g) * d;
+                    const double *ai = a + ((size_t)i * G + g) * S, *oi = o + ((size_t)i * G + g) * d;
+                    double go = 0.0;
+                    for (int x = 0; x < d; ++x) go += w[i] * dO[qh + x] * oi[x];
+                    for (int u = 0; u < S; ++u) {
+                        size_t kr = ((b * (size_t)Tkv + c * S + u) * Hkv + j) * (size_t)d;
+                        double gv = 0.0;
+                        for (int x = 0; x < d; ++x) {
+                            double gx = w[i] * dO[qh + x];
+                            dV[kr + x] += ai[u] * gx;
+                            gv += gx * load(V, kr + x, dt);
+                        }
+                        double dz = ai[u] * (gv - go) * scale;
+                        for (int x = 0; x < d; ++x) {
+                            dQ[qh + x] += dz * load(K, kr + x, dt);
+                            dK[kr + x] += dz * load(Qr, qh + x, dt);
+                        }
+                    }
+                }
+            }
+        }
+        free(w); free(dw); free(e); free(a); free(o);
+    }
+    /* landmark backward: dW_L and the keys' share through the chunk mean */
+    double *mean = (double *)malloc(sizeof(double) * (size_t)d);
+    double *dm = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int b = 0; b < B; ++b)
+        for (int j = 0; j < Hkv; ++j)
+            for (long long c = 0; c < C; ++c) {
+                const double *dLc = dL + (((size_t)b * Hkv + j) * (size_t)C + (size_t)c) * d;
+                for (int x = 0; x < d; ++x) mean[x] = 0.0;
+                for (int u = 0; u < S; ++u) {
+                    size_t kr = (((size_t)b * Tkv + (size_t)(c * S + u)) * Hkv + j) * (size_t)d;
+                    for (int x = 0; x < d; ++x) mean[x] += load(K, kr + x, dt);
+                }
+                for (int x = 0; x < d; ++x) mean[x] /= (double)S;
+                for (int x = 0; x < d; ++x) {
+                    double acc = 0.0;
+                    for (int f = 0; f < d; ++f) {
+                        dW[(size_t)x * d + f] += mean[x] * dLc[f];
+                        acc += dLc[f] * load(W, (size_t)x * d + f, dt);
+                    }
+                    dm[x] = acc / (double)S;
+                }
+                for (int u = 0; u < S; ++u) {
+                    size_t kr = (((size_t)b * Tkv + (size_t)(c * S + u)) * Hkv + j) * (size_t)d;
+                    for (int x = 0; x < d; ++x) dK[kr + x] += dm[x];
+                }
+            }
+    free(mean); free(dm);
+}
