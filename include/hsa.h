@@ -1,5 +1,5 @@
 /*
- * hsa.h -- C ABI of the B200 (sm_100a) Hierarchical Sparse Attention forward path.
+ * hsa.h -- C ABI of the B200 (sm_100a) Hierarchical Sparse Attention forward path and its backward.
  *
  * Method: "Every Token Counts 16m Context" (HSA summary page), sections Core
  * Technique and Implementation.  The key sequence is cut into fixed-length,
@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define HSA_ABI_VERSION 2
+#define HSA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define HSA_API __attribute__((visibility("default")))
@@ -232,6 +232,38 @@ HSA_API hsa_status_t hsa_merge_partials(const hsa_problem_t *p, int nshard, cons
 HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                          const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
                          void *O, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Backward pass: gradients of the method with respect to Q, K, V and W_L,
+ * with the forward's chunk selection held fixed (HSA summary page,
+ * Implementation: the kept chunks' retrieval scores weight their outputs, so
+ * the scores carry a gradient; which chunks are kept is a discrete choice and
+ * has none).  With w = softmax(score) over the kept slots of a selection row,
+ * a the in-chunk attention probabilities and o the per-chunk outputs, it
+ * returns the exact gradients of O = sum_i w_i o_i, for the upstream gradient
+ * dO, through the in-chunk softmax attention, the fusion softmax, the group
+ * scores s_i = sum_h q_h . L_ci, and the landmarks L_c = mean(K of chunk c) W_L.
+ *
+ * Inputs (the problem's dtype unless noted): Q, K, V, W_L and L as given to
+ * hsa_forward (L: the landmarks the scores were taken from); idx, score, keff:
+ * the selection the forward returned (score fp32: it sets the fusion
+ * weights); dO [B][Tq][H][d].
+ * Outputs, fp32, OVERWRITTEN (the call zeroes them first): dQ [B][Tq][H][d],
+ * dK and dV [B][Tcap][Hkv][d] (the K/V layout; tokens past Tkv, and those of a
+ * trailing partial chunk, get 0), dW_L [d][d].
+ * L enters the scores as stored: its rounding to the dtype counts as the
+ * identity in the chain rule.  A chunk index or keff outside its row's
+ * candidates is skipped and recorded in the status word (HSA_ERR_INVALID_ARG
+ * from hsa_get_device_status).  Workspace: hsa_backward_workspace_size (its
+ * header is the status word).  The adds into dQ, dK, dV and dW_L are fp32
+ * atomic reductions, so their order, and the last bits of the result, vary
+ * from call to call.
+ */
+HSA_API hsa_status_t hsa_backward_workspace_size(const hsa_problem_t *p, size_t *bytes);
+HSA_API hsa_status_t hsa_backward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
+                                  const void *W_L, const void *L, const int32_t *idx, const float *score,
+                                  const int32_t *keff, const void *dO, float *dQ, float *dK, float *dV,
+                                  float *dW_L, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device-status word in the

@@ -22,7 +22,7 @@ from ._native import HSAError, hsa_problem_t
 
 __all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "select_noalloc", "attend",
            "forward", "decode_append", "attend_partials", "merge_partials", "device_status", "HSAError",
-           "hsa_problem_t", "kmax_of"]
+           "hsa_problem_t", "kmax_of", "backward", "backward_workspace_size"]
 
 _DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
 
@@ -249,6 +249,39 @@ def merge_partials(score, idx, keff, o_part, S, k, tau=0.0, dtype=torch.bfloat16
                                                    _p(O), _p(sel[0]), _p(sel[1]), _p(sel[2]), _stream(o_part)),
                   "hsa_merge_partials")
     return (O,) + sel if return_selection else O
+
+
+def backward_workspace_size(prob: hsa_problem_t) -> int:
+    n = ctypes.c_size_t()
+    _native.check(_native.lib().hsa_backward_workspace_size(ctypes.byref(prob), ctypes.byref(n)),
+                  "hsa_backward_workspace_size")
+    return int(n.value)
+
+
+def backward(Q, K, V, W_L, L, idx, score, keff, dO, S, k, tau=0.0, q_pos0=0, kv_len=None, out=None, ws=None):
+    """Gradients (dQ, dK, dV, dW_L), fp32, of the forward with its selection (idx, score,
+    keff) held fixed, for the output gradient dO [B,Tq,H,d].  L: the landmarks the forward
+    scored ([B, Hkv, K.shape[1] // S, d]).  kv_len as in forward.  out: optional preallocated
+    (dQ, dK, dV, dW_L); ws: optional workspace (uint8, 256-byte aligned)."""
+    _dev(Q, K, V, W_L, L, idx, score, keff, dO, ws)
+    B, Tq, H, d = Q.shape
+    Tcap, Hkv = K.shape[1], K.shape[2]
+    Tkv = Tcap if kv_len is None else kv_len
+    if dO.shape != Q.shape or dO.dtype != Q.dtype:
+        raise ValueError(f"dO must match Q ({tuple(Q.shape)}, {Q.dtype}); got {tuple(dO.shape)}, {dO.dtype}")
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, 0, Tcap)
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=Q.device)
+        out = (torch.empty(B, Tq, H, d, **f32), torch.empty(B, Tcap, Hkv, d, **f32),
+               torch.empty(B, Tcap, Hkv, d, **f32), torch.empty(d, d, **f32))
+    dQ, dK, dV, dW = out
+    _dev(dQ, dK, dV, dW)
+    if ws is None:
+        ws = torch.empty(max(256, backward_workspace_size(prob)), dtype=torch.uint8, device=Q.device)
+    _native.check(_native.lib().hsa_backward(ctypes.byref(prob), _p(Q), _p(K), _p(V), _p(W_L), _p(L), _p(idx),
+                                             _p(score), _p(keff), _p(dO), _p(dQ), _p(dK), _p(dV), _p(dW), _p(ws),
+                                             ws.numel(), _stream(Q)), "hsa_backward")
+    return dQ, dK, dV, dW
 
 
 def device_status(ws: torch.Tensor) -> None:

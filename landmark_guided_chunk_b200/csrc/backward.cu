@@ -1,0 +1,717 @@
+// backward.cu -- gradients of the method with respect to Q, K, V and W_L, with
+// the chunk selection of the forward held fixed (HSA summary page,
+// Implementation: the retrieval scores weight the chunk outputs, so they carry
+// a gradient into the queries and, through the landmarks, into the keys and
+// W_L; which chunks are kept is a discrete choice with no gradient).
+//
+// For a selection row (b, t, kv head j) with kept chunks c_i, fusion weights
+// w = softmax(s) and in-chunk probabilities a_hiu of its heads h:
+//   e_hi  = dO_h . o_hi = sum_u a_hiu (dO_h . V_u)
+//   dz_hiu = w_i a_hiu (dO_h . V_u - e_hi) / sqrt(d)         (in-chunk softmax)
+//   dQ_h += sum_u dz_hiu K_u,  dK_u += dz_hiu q_h,  dV_u += w_i a_hiu dO_h
+//   ds_i  = w_i (dw_i - sum_i' w_i' dw_i'),  dw_i = sum_h e_hi (fusion softmax)
+//   dQ_h += sum_i ds_i L_ci,   dL_ci += ds_i sum_h q_h       (s_i = sum_h q_h . L_ci)
+// and through every landmark L_c = mean(K of chunk c) W_L:
+//   dW_L += mean_c^T dL_c,     dK_u += (dL_c W_L^T) / S for the S keys of chunk c.
+//
+// Stages (all on the caller's stream):
+//   prep     one thread per selection row: fusion weights, pair count per
+//            (b, j, c) bucket, checks of keff and the chunk indices;
+//   scan     one CTA: exclusive scans of the bucket counts (pairs) and of
+//            their tile counts, the tile list, the scatter cursors;
+//   scatter  one thread per selection row: its (row, slot) pairs -> buckets;
+//   attend   chunk-major, one CTA per SM over a contiguous range of tiles.  A
+//            tile holds up to RT query-head rows that kept one chunk.  K_c and
+//            V_c are staged once per bucket run; the CTA keeps dK_c and dV_c in
+//            registers until the bucket changes and then adds them to memory
+//            with vector reductions.  Per tile: Z = q K^T, GV = dO V^T (one
+//            pass over d), row softmax and e in one warp per row, then dQ =
+//            dZ K and the dK/dV updates.  e goes to the workspace.
+//   fuse     one warp per selection row: dw, ds, the score path into dQ and dL;
+//   landmark one pass over all complete chunks: chunk means, dW_L partials per
+//            CTA, and dL W_L^T / S added to the chunk's key gradients.
+// All arithmetic is fp32 on CUDA cores (the gradients are fp32 buffers); the
+// stored inputs (fp32 or bf16) are read exactly.
+#include "common.cuh"
+
+namespace hsa {
+namespace {
+
+constexpr int RT = 32;          // query-head rows per tile
+constexpr int NT_BWD = 512;     // threads of the attend kernel (16 warps)
+constexpr int NT_SCAN = 1024;
+
+struct BwdArgs {
+    int B, Tq, Tcap, H, Hkv, G, d, S, C, kmax, pt;   // pt: pairs per tile = RT / G
+    long long q_pos0, rows;
+    long long nbucket;
+    float scale;                // 1/sqrt(d)
+    const int32_t *idx, *keff;
+    const float *score;
+    float *w;                   // [rows][kmax] fusion weights
+    float *e;                   // [rows][kmax][G]  dO_h . o_hi
+    int32_t *bcount;            // [nbucket] pair counts, then scatter cursors
+    int32_t *boff;              // [nbucket + 1] first pair of each bucket
+    int32_t *pairs;             // [rows * kmax] row * kmax + slot, bucket-major
+    int4 *tiles;                // (bucket, first pair, pairs, 0)
+    int32_t *ntiles;            // number of tiles (written by the scan)
+    float *dL;                  // [B][Hkv][C][d] landmark gradients
+    uint32_t *status;
+};
+
+__device__ __forceinline__ void red_add4(float *p, float4 v) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void red_add2(float *p, float2 v) {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v.x), "f"(v.y) : "memory");
+}
+
+// number of candidate chunks of a query row
+__device__ __forceinline__ long long ncand_of(const BwdArgs &a, int t) {
+    long long nc = (a.q_pos0 + t) / a.S;
+    return nc > a.C ? a.C : nc;
+}
+
+// ---------------------------------------------------------------------------- prep, scan, scatter
+
+__global__ void bwd_prep_kernel(BwdArgs a) {
+    const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= a.rows) return;
+    const int j = (int)(r % a.Hkv);
+    const long long bt = r / a.Hkv;
+    const int t = (int)(bt % a.Tq), b = (int)(bt / a.Tq);
+    int ke = a.keff[r];
+    if (ke < 0 || ke > a.kmax) {
+        atomicOr(a.status, DEV_BAD_INDEX);
+        ke = ke < 0 ? 0 : a.kmax;
+    }
+    const float *sc = a.score + r * a.kmax;
+    float m = -INFINITY;
+    for (int i = 0; i < ke; ++i) m = fmaxf(m, sc[i]);
+    float z = 0.f;
+    for (int i = 0; i < ke; ++i) z += expf(sc[i] - m);
+    const long long nc = ncand_of(a, t);
+    for (int i = 0; i < a.kmax; ++i) {
+        const float wi = i < ke ? expf(sc[i] - m) / z : 0.f;
+        a.w[r * a.kmax + i] = wi;
+        if (i >= ke) continue;
+        const int c = a.idx[r * a.kmax + i];
+        if (c < 0 || c >= nc) {
+            atomicOr(a.status, DEV_BAD_INDEX);
+            continue;
+        }
+        atomicAdd(a.bcount + ((long long)b * a.Hkv + j) * a.C + c, 1);
+    }
+}
+
+// Exclusive scans of pair counts and tile counts over the buckets, in blocks
+// of NT_SCAN with a running carry; each bucket also writes its tile records
+// and turns its count into the scatter cursor.
+__global__ void __launch_bounds__(NT_SCAN) bwd_scan_kernel(BwdArgs a) {
+    __shared__ int wp[NT_SCAN / 32], wt[NT_SCAN / 32];
+    __shared__ int carry_p, carry_t;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        carry_p = 0;
+        carry_t = 0;
+    }
+    __syncthreads();
+    for (long long base = 0; base < a.nbucket; base += NT_SCAN) {
+        const long long i = base + threadIdx.x;
+        const int cnt = i < a.nbucket ? a.bcount[i] : 0;
+        const int nt = (cnt + a.pt - 1) / a.pt;
+        int ip = cnt, it = nt;   // inclusive warp scans
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int xp = __shfl_up_sync(FULL, ip, o), xt = __shfl_up_sync(FULL, it, o);
+            if (lane >= o) {
+                ip += xp;
+                it += xt;
+            }
+        }
+        if (lane == 31) {
+            wp[warp] = ip;
+            wt[warp] = it;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int sp = wp[lane], st = wt[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int xp = __shfl_up_sync(FULL, sp, o), xt = __shfl_up_sync(FULL, st, o);
+                if (lane >= o) {
+                    sp += xp;
+                    st += xt;
+                }
+            }
+            wp[lane] = sp;   // inclusive prefix over warps
+            wt[lane] = st;
+        }
+        __syncthreads();
+        const int ep = carry_p + (warp ? wp[warp - 1] : 0) + ip - cnt;
+        const int et = carry_t + (warp ? wt[warp - 1] : 0) + it - nt;
+        if (i < a.nbucket) {
+            a.boff[i] = ep;
+            a.bcount[i] = ep;   // scatter cursor
+            for (int q = 0; q < nt; ++q)
+                a.tiles[et + q] = make_int4((int)i, ep + q * a.pt, min(a.pt, cnt - q * a.pt), 0);
+        }
+        __syncthreads();
+        if (threadIdx.x == NT_SCAN - 1) {
+            carry_p = ep + cnt;
+            carry_t = et + nt;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        a.boff[a.nbucket] = carry_p;
+        *a.ntiles = carry_t;
+    }
+}
+
+__global__ void bwd_scatter_kernel(BwdArgs a) {
+    const long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= a.rows) return;
+    const int j = (int)(r % a.Hkv);
+    const long long bt = r / a.Hkv;
+    const int t = (int)(bt % a.Tq), b = (int)(bt / a.Tq);
+    int ke = a.keff[r];
+    ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
+    const long long nc = ncand_of(a, t);
+    for (int i = 0; i < ke; ++i) {
+        const int c = a.idx[r * a.kmax + i];
+        if (c < 0 || c >= nc) continue;
+        const int pos = atomicAdd(a.bcount + ((long long)b * a.Hkv + j) * a.C + c, 1);
+        a.pairs[pos] = (int)(r * a.kmax + i);
+    }
+}
+
+// ---------------------------------------------------------------------------- chunk-major attention backward
+
+// 16 bytes of stored values -> fp32 in shared memory
+__device__ __forceinline__ void cvt16(const float *src, float *dst) {
+    *reinterpret_cast<float4 *>(dst) = __ldg(reinterpret_cast<const float4 *>(src));
+}
+__device__ __forceinline__ void cvt16(const __nv_bfloat16 *src, float *dst) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src));
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+    reinterpret_cast<float4 *>(dst)[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+    reinterpret_cast<float4 *>(dst)[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+}
+
+template <int CPL> struct Cols;   // CPL consecutive fp32 values of one lane
+template <> struct Cols<4> {
+    float v[4];
+    __device__ __forceinline__ void load(const float *p) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    }
+    __device__ __forceinline__ void red(float *p) const { red_add4(p, make_float4(v[0], v[1], v[2], v[3])); }
+};
+template <> struct Cols<2> {
+    float v[2];
+    __device__ __forceinline__ void load(const float *p) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x; v[1] = x.y;
+    }
+    __device__ __forceinline__ void red(float *p) const { red_add2(p, make_float2(v[0], v[1])); }
+};
+
+template <int S, int D> struct BwdShape {
+    static constexpr int KP = D + 4;       // K, V, q, dO row pitch (floats): float4 rows, conflict-free
+    static constexpr int SP = S + 4;       // dZ, w*P row pitch
+    static constexpr int KPT = S / 32;     // keys per lane in the row pass
+    static constexpr int UPW = S / 16;     // keys per warp in the dK/dV pass
+    static constexpr int CPL = D / 32;     // columns per lane
+    static constexpr size_t smem = sizeof(float) * (2 * (size_t)S * KP + 2 * (size_t)RT * KP + 2 * (size_t)RT * SP) +
+                                   RT * (sizeof(long long) + sizeof(float) + sizeof(int));
+};
+
+template <typename T, int S, int D>
+__global__ void __launch_bounds__(NT_BWD, 1)
+    bwd_attend_kernel(BwdArgs a, const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
+                      const T *__restrict__ dO, float *__restrict__ dQ, float *__restrict__ dK,
+                      float *__restrict__ dV) {
+    using SH = BwdShape<S, D>;
+    constexpr int KP = SH::KP, SP = SH::SP, KPT = SH::KPT, UPW = SH::UPW, CPL = SH::CPL;
+    constexpr int EPS = 16 / (int)sizeof(T);   // stored elements per 16-byte load
+    constexpr int SEGS = D / EPS;
+    extern __shared__ float4 smem4[];
+    float *sK = reinterpret_cast<float *>(smem4);
+    float *sV = sK + S * KP;
+    float *sq = sV + S * KP;
+    float *sg = sq + RT * KP;
+    float *sZ = sg + RT * KP;     // dZ (scaled in-chunk softmax gradient)
+    float *sPw = sZ + RT * SP;    // w * P
+    long long *s_qoff = reinterpret_cast<long long *>(sPw + RT * SP);
+    float *s_w = reinterpret_cast<float *>(s_qoff + RT);
+    int *s_e = reinterpret_cast<int *>(s_w + RT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = *a.ntiles;
+    const int lo = (int)((long long)ntiles * blockIdx.x / gridDim.x);
+    const int hi = (int)((long long)ntiles * (blockIdx.x + 1) / gridDim.x);
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+
+    float accK[UPW][CPL], accV[UPW][CPL];   // keys warp + 16 m, columns lane * CPL + x
+#pragma unroll
+    for (int m = 0; m < UPW; ++m)
+#pragma unroll
+        for (int x = 0; x < CPL; ++x) accK[m][x] = accV[m][x] = 0.f;
+    int cur = -1, cb = 0, cj = 0, cc = 0;
+
+    auto flush = [&]() {
+#pragma unroll
+        for (int m = 0; m < UPW; ++m) {
+            const int u = warp + 16 * m;
+            const long long off = (((long long)cb * a.Tcap + (long long)cc * S + u) * a.Hkv + cj) * D + lane * CPL;
+            Cols<CPL> k, v;
+#pragma unroll
+            for (int x = 0; x < CPL; ++x) {
+                k.v[x] = accK[m][x];
+                v.v[x] = accV[m][x];
+                accK[m][x] = accV[m][x] = 0.f;
+            }
+            k.red(dK + off);
+            v.red(dV + off);
+        }
+    };
+
+    for (int ti = lo; ti < hi; ++ti) {
+        const int4 tr = a.tiles[ti];
+        const int nrow = tr.z * a.G;
+        if (tr.x != cur) {
+            if (cur >= 0) flush();
+            cur = tr.x;
+            cc = cur % a.C;
+            const int bj = cur / a.C;
+            cj = bj % a.Hkv;
+            cb = bj / a.Hkv;
+            const long long row0 = ((long long)cb * a.Tcap + (long long)cc * S) * a.Hkv + cj;
+            for (int i = threadIdx.x; i < S * SEGS; i += NT_BWD) {
+                const int u = i / SEGS, sgm = i - u * SEGS;
+                const long long off = (row0 + (long long)u * a.Hkv) * D + sgm * EPS;
+                cvt16(K + off, sK + u * KP + sgm * EPS);
+                cvt16(V + off, sV + u * KP + sgm * EPS);
+            }
+        }
+        if (threadIdx.x < RT) {
+            const int rr = threadIdx.x;
+            if (rr < nrow) {
+                const int pc = a.pairs[tr.y + rr / a.G], g = rr % a.G;
+                const long long bt = (long long)(pc / a.kmax) / a.Hkv;
+                s_qoff[rr] = (bt * a.H + (long long)cj * a.G + g) * D;
+                s_w[rr] = a.w[pc];
+                s_e[rr] = pc * a.G + g;
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < RT * SEGS; i += NT_BWD) {
+            const int rr = i / SEGS, sgm = i - rr * SEGS;
+            float *qd = sq + rr * KP + sgm * EPS, *gd = sg + rr * KP + sgm * EPS;
+            if (rr < nrow) {
+                cvt16(Q + s_qoff[rr] + sgm * EPS, qd);
+                cvt16(dO + s_qoff[rr] + sgm * EPS, gd);
+            } else {
+#pragma unroll
+                for (int x = 0; x < EPS; ++x) qd[x] = gd[x] = 0.f;
+            }
+        }
+        __syncthreads();
+
+        // ---- rows warp and warp + 16: Z = q K^T and GV = dO V^T over keys lane + 32 m
+        if (warp < nrow) {
+            float z0[KPT], z1[KPT], v0[KPT], v1[KPT];
+#pragma unroll
+            for (int m = 0; m < KPT; ++m) z0[m] = z1[m] = v0[m] = v1[m] = 0.f;
+            const float *qa = sq + warp * KP, *qb = sq + (warp + 16) * KP;
+            const float *ga = sg + warp * KP, *gb = sg + (warp + 16) * KP;
+#pragma unroll 4
+            for (int x = 0; x < D; x += 4) {
+                const float4 q0 = *reinterpret_cast<const float4 *>(qa + x);
+                const float4 q1 = *reinterpret_cast<const float4 *>(qb + x);
+                const float4 g0 = *reinterpret_cast<const float4 *>(ga + x);
+                const float4 g1 = *reinterpret_cast<const float4 *>(gb + x);
+#pragma unroll
+                for (int m = 0; m < KPT; ++m) {
+                    const float4 k = *reinterpret_cast<const float4 *>(sK + (lane + 32 * m) * KP + x);
+                    const float4 v = *reinterpret_cast<const float4 *>(sV + (lane + 32 * m) * KP + x);
+                    z0[m] = fmaf(q0.x, k.x, fmaf(q0.y, k.y, fmaf(q0.z, k.z, fmaf(q0.w, k.w, z0[m]))));
+                    z1[m] = fmaf(q1.x, k.x, fmaf(q1.y, k.y, fmaf(q1.z, k.z, fmaf(q1.w, k.w, z1[m]))));
+                    v0[m] = fmaf(g0.x, v.x, fmaf(g0.y, v.y, fmaf(g0.z, v.z, fmaf(g0.w, v.w, v0[m]))));
+                    v1[m] = fmaf(g1.x, v.x, fmaf(g1.y, v.y, fmaf(g1.z, v.z, fmaf(g1.w, v.w, v1[m]))));
+                }
+            }
+            // softmax over the chunk's keys, e = sum_u P_u GV_u, dZ and w P of one row
+            auto finish = [&](float (&z)[KPT], const float (&gv)[KPT], int rr) {
+                float mx = z[0];
+#pragma unroll
+                for (int m = 1; m < KPT; ++m) mx = fmaxf(mx, z[m]);
+                mx = warp_max(mx);
+                float l = 0.f;
+#pragma unroll
+                for (int m = 0; m < KPT; ++m) {
+                    z[m] = exp2f((z[m] - mx) * scale_log2);
+                    l += z[m];
+                }
+                const float inv = 1.f / warp_sum(l);
+                float ev = 0.f;
+#pragma unroll
+                for (int m = 0; m < KPT; ++m) {
+                    z[m] *= inv;
+                    ev = fmaf(z[m], gv[m], ev);
+                }
+                ev = warp_sum(ev);
+                const float w = s_w[rr], ws = w * a.scale;
+#pragma unroll
+                for (int m = 0; m < KPT; ++m) {
+                    sZ[rr * SP + lane + 32 * m] = ws * z[m] * (gv[m] - ev);
+                    sPw[rr * SP + lane + 32 * m] = w * z[m];
+                }
+                if (lane == 0) a.e[s_e[rr]] = ev;
+            };
+            finish(z0, v0, warp);
+            if (warp + 16 < nrow) finish(z1, v1, warp + 16);
+        }
+        __syncthreads();
+
+        // ---- dQ of rows warp, warp + 16 (columns lane * CPL ..)
+        if (warp < nrow) {
+            float d0[CPL], d1[CPL];
+#pragma unroll
+            for (int x = 0; x < CPL; ++x) d0[x] = d1[x] = 0.f;
+            const bool two = warp + 16 < nrow;
+#pragma unroll 4
+            for (int u = 0; u < S; ++u) {
+                Cols<CPL> k;
+                k.load(sK + u * KP + lane * CPL);
+                const float za = sZ[warp * SP + u], zb = two ? sZ[(warp + 16) * SP + u] : 0.f;
+#pragma unroll
+                for (int x = 0; x < CPL; ++x) {
+                    d0[x] = fmaf(za, k.v[x], d0[x]);
+                    d1[x] = fmaf(zb, k.v[x], d1[x]);
+                }
+            }
+            Cols<CPL> o;
+#pragma unroll
+            for (int x = 0; x < CPL; ++x) o.v[x] = d0[x];
+            o.red(dQ + s_qoff[warp] + lane * CPL);
+            if (two) {
+#pragma unroll
+                for (int x = 0; x < CPL; ++x) o.v[x] = d1[x];
+                o.red(dQ + s_qoff[warp + 16] + lane * CPL);
+            }
+        }
+        // ---- dK_u += sum_r dZ[r][u] q_r, dV_u += sum_r wP[r][u] dO_r  (keys warp + 16 m)
+        for (int rr = 0; rr < nrow; ++rr) {
+            Cols<CPL> qv, gv;
+            qv.load(sq + rr * KP + lane * CPL);
+            gv.load(sg + rr * KP + lane * CPL);
+#pragma unroll
+            for (int m = 0; m < UPW; ++m) {
+                const float zz = sZ[rr * SP + warp + 16 * m], pw = sPw[rr * SP + warp + 16 * m];
+#pragma unroll
+                for (int x = 0; x < CPL; ++x) {
+                    accK[m][x] = fmaf(zz, qv.v[x], accK[m][x]);
+                    accV[m][x] = fmaf(pw, gv.v[x], accV[m][x]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+    if (cur >= 0) flush();
+}
+
+// ---------------------------------------------------------------------------- fusion softmax backward
+
+constexpr int NT_FUSE = 256;   // 8 warps, one selection row each
+
+// Per selection row: dw_i = sum_h e_hi, ds_i = w_i (dw_i - sum w dw); then
+// dQ_h += sum_i ds_i L_ci for every head of the group, dL_ci += ds_i sum_h q_h.
+template <typename T, int D>
+__global__ void __launch_bounds__(NT_FUSE) bwd_fuse_kernel(BwdArgs a, int Lc, const T *__restrict__ Q,
+                                                           const T *__restrict__ L, float *__restrict__ dQ) {
+    constexpr int CPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    const long long r = (long long)blockIdx.x * (NT_FUSE / 32) + (threadIdx.x >> 5);
+    if (r >= a.rows) return;
+    const int j = (int)(r % a.Hkv);
+    const long long bt = r / a.Hkv;
+    const int t = (int)(bt % a.Tq), b = (int)(bt / a.Tq);
+    int ke = a.keff[r];
+    ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
+    if (ke == 0) return;
+    const long long nc = ncand_of(a, t);
+    float w = 0.f, dw = 0.f;
+    int c = -1;
+    if (lane < ke) {
+        c = a.idx[r * a.kmax + lane];
+        if (c >= 0 && c < nc) {
+            w = a.w[r * a.kmax + lane];
+            const float *e = a.e + (r * a.kmax + lane) * a.G;
+            for (int g = 0; g < a.G; ++g) dw += e[g];
+        } else {
+            c = -1;
+        }
+    }
+    const float wdw = warp_sum(w * dw);
+    const float ds = w * (dw - wdw);
+    // sum of the group's query rows, this lane's columns
+    float qs[CPL];
+#pragma unroll
+    for (int x = 0; x < CPL; ++x) qs[x] = 0.f;
+    const T *qrow = Q + (bt * a.H + (long long)j * a.G) * D + lane * CPL;
+    for (int g = 0; g < a.G; ++g)
+#pragma unroll
+        for (int x = 0; x < CPL; ++x) qs[x] += to_f32(qrow[(long long)g * D + x]);
+    float dq[CPL];
+#pragma unroll
+    for (int x = 0; x < CPL; ++x) dq[x] = 0.f;
+    for (int i = 0; i < ke; ++i) {
+        const float dsi = __shfl_sync(FULL, ds, i);
+        const int ci = __shfl_sync(FULL, c, i);
+        if (ci < 0) continue;   // warp-uniform
+        const T *lrow = L + (((long long)b * a.Hkv + j) * Lc + ci) * D + lane * CPL;
+        Cols<CPL> o;
+#pragma unroll
+        for (int x = 0; x < CPL; ++x) {
+            dq[x] = fmaf(dsi, to_f32(lrow[x]), dq[x]);
+            o.v[x] = dsi * qs[x];
+        }
+        o.red(a.dL + (((long long)b * a.Hkv + j) * a.C + ci) * D + lane * CPL);
+    }
+    Cols<CPL> o;
+#pragma unroll
+    for (int x = 0; x < CPL; ++x) o.v[x] = dq[x];
+    for (int g = 0; g < a.G; ++g) o.red(dQ + (bt * a.H + (long long)j * a.G + g) * D + lane * CPL);
+}
+
+// ---------------------------------------------------------------------------- landmark backward
+
+constexpr int NT_LM = 256;
+
+template <int D> struct LmShape {
+    static constexpr int WP = D + 1;   // W_L row pitch in shared memory (conflict-free column walks)
+    static constexpr int PARTS = NT_LM / D;
+    static constexpr size_t smem = sizeof(float) * ((size_t)D * WP + 3 * (size_t)D + (size_t)PARTS * D);
+};
+
+// Every complete chunk (b, j, c) with a nonzero landmark gradient: its key
+// mean m_c, dW_L += m_c^T dL_c (a per-CTA partial in registers, added once),
+// and dL_c W_L^T / S added to the gradients of its S keys.  Each chunk has one
+// CTA, and the attention kernels that also add into dK have finished, so the
+// key gradients are updated with plain loads and stores.
+template <typename T, int D>
+__global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T *__restrict__ K,
+                                                             const T *__restrict__ W, float *__restrict__ dK,
+                                                             float *__restrict__ dW) {
+    using SH = LmShape<D>;
+    constexpr int WP = SH::WP, PARTS = SH::PARTS, CPL = D / 32, XPW = D / (NT_LM / 32);
+    extern __shared__ float4 smem4[];
+    float *sW = reinterpret_cast<float *>(smem4);
+    float *sdl = sW + D * WP;
+    float *sm = sdl + D;
+    float *sdm = sm + D;
+    float *spart = sdm + D;   // [PARTS][D]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < D * D; i += NT_LM) sW[(i / D) * WP + (i % D)] = to_f32(W[i]);
+    float acc[XPW][CPL];   // dW_L rows warp + 8 a, columns lane * CPL + x
+#pragma unroll
+    for (int q = 0; q < XPW; ++q)
+#pragma unroll
+        for (int x = 0; x < CPL; ++x) acc[q][x] = 0.f;
+    const long long nch = (long long)a.B * a.Hkv * a.C;
+    const long long lo = nch * blockIdx.x / gridDim.x, hi = nch * (blockIdx.x + 1) / gridDim.x;
+    const int xcol = threadIdx.x % D, part = threadIdx.x / D;
+    __syncthreads();
+    for (long long ch = lo; ch < hi; ++ch) {
+        const int c = (int)(ch % a.C);
+        const long long bj = ch / a.C;
+        const int j = (int)(bj % a.Hkv), b = (int)(bj / a.Hkv);
+        float v = 0.f;
+        if (threadIdx.x < D) {
+            v = a.dL[ch * D + threadIdx.x];
+            sdl[threadIdx.x] = v;
+        }
+        if (!__syncthreads_or(v != 0.f)) continue;   // never kept by any row: nothing to add
+        const long long row0 = ((long long)b * a.Tcap + (long long)c * a.S) * a.Hkv + j;
+        float ps = 0.f, pm = 0.f;
+        for (int u = part; u < a.S; u += PARTS) ps += to_f32(K[(row0 + (long long)u * a.Hkv) * D + xcol]);
+        for (int f = part; f < D; f += PARTS) pm = fmaf(sdl[f], sW[xcol * WP + f], pm);
+        spart[part * D + xcol] = ps;
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float m = 0.f;
+            for (int q = 0; q < PARTS; ++q) m += spart[q * D + threadIdx.x];
+            sm[threadIdx.x] = m / (float)a.S;
+        }
+        __syncthreads();
+        spart[part * D + xcol] = pm;
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float m = 0.f;
+            for (int q = 0; q < PARTS; ++q) m += spart[q * D + threadIdx.x];
+            sdm[threadIdx.x] = m / (float)a.S;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < a.S * D; i += NT_LM) {
+            const int u = i / D, x = i - u * D;
+            float *p = dK + (row0 + (long long)u * a.Hkv) * D + x;
+            *p += sdm[x];
+        }
+#pragma unroll
+        for (int q = 0; q < XPW; ++q) {
+            const float mx = sm[warp + 8 * q];
+#pragma unroll
+            for (int x = 0; x < CPL; ++x) acc[q][x] = fmaf(mx, sdl[lane * CPL + x], acc[q][x]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int q = 0; q < XPW; ++q) {
+        Cols<CPL> o;
+#pragma unroll
+        for (int x = 0; x < CPL; ++x) o.v[x] = acc[q][x];
+        o.red(dW + (long long)(warp + 8 * q) * D + lane * CPL);
+    }
+}
+
+template <typename T, int S, int D>
+cudaError_t launch_attend_t(const BwdArgs &a, int grid, const void *Q, const void *K, const void *V, const void *dO,
+                            float *dQ, float *dK, float *dV, cudaStream_t st) {
+    const size_t smem = BwdShape<S, D>::smem;
+    cudaError_t e = cudaFuncSetAttribute(bwd_attend_kernel<T, S, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_attend_kernel<T, S, D><<<grid, NT_BWD, smem, st>>>(a, (const T *)Q, (const T *)K, (const T *)V,
+                                                            (const T *)dO, dQ, dK, dV);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_attend_s(const BwdArgs &a, int grid, const void *Q, const void *K, const void *V, const void *dO,
+                            float *dQ, float *dK, float *dV, cudaStream_t st) {
+    switch (a.S) {
+        case 32: return launch_attend_t<T, 32, D>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
+        case 64: return launch_attend_t<T, 64, D>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
+        default: return launch_attend_t<T, 128, D>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_tail_t(const BwdArgs &a, int Lc, int lm_grid, const void *Q, const void *K, const void *W,
+                          const void *L, float *dQ, float *dK, float *dW, cudaStream_t st) {
+    const unsigned fuse_grid = (unsigned)((a.rows + NT_FUSE / 32 - 1) / (NT_FUSE / 32));
+    bwd_fuse_kernel<T, D><<<fuse_grid, NT_FUSE, 0, st>>>(a, Lc, (const T *)Q, (const T *)L, dQ);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = LmShape<D>::smem;
+    e = cudaFuncSetAttribute(bwd_landmark_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_landmark_kernel<T, D><<<lm_grid, NT_LM, smem, st>>>(a, (const T *)K, (const T *)W, dK, dW);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+BwdLayout backward_layout(const Prob &p) {
+    BwdLayout w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return o;
+    };
+    const size_t pairs = (size_t)p.rows * p.kmax;
+    w.pt = RT / p.G;
+    w.nbucket = (long long)p.B * p.Hkv * p.C;
+    w.max_tiles = (long long)((pairs + w.pt - 1) / w.pt) + w.nbucket;
+    w.hdr = take(256);   // status word at 0, tile count at 16
+    w.bcount = take((size_t)w.nbucket * sizeof(int32_t));
+    w.dL = take((size_t)w.nbucket * p.d * sizeof(float));
+    w.clear_bytes = off;
+    w.w = take(pairs * sizeof(float));
+    w.e = take(pairs * p.G * sizeof(float));
+    w.boff = take(((size_t)w.nbucket + 1) * sizeof(int32_t));
+    w.pairs = take(pairs * sizeof(int32_t));
+    w.tiles = take((size_t)w.max_tiles * sizeof(int4));
+    w.total = off;
+    return w;
+}
+
+bool backward_supported(const Prob &p) {
+    const BwdLayout w = backward_layout(p);
+    return (long long)p.rows * p.kmax * p.G < (1ll << 31) && w.max_tiles < (1ll << 31) && p.G <= RT;
+}
+
+int backward_launches(const Prob &p) { return p.rows > 0 && p.C > 0 ? 6 : 0; }
+
+cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms, const void *Q, const void *K,
+                            const void *V, const void *W, const void *L, const int32_t *idx, const float *score,
+                            const int32_t *keff, const void *dO, float *dQ, float *dK, float *dV, float *dW,
+                            cudaStream_t st) {
+    cudaError_t e;
+    const size_t kv_bytes = (size_t)p.B * p.Tcap * p.Hkv * p.d * sizeof(float);
+    const size_t q_bytes = (size_t)p.B * p.Tq * p.H * p.d * sizeof(float);
+    if (q_bytes && (e = cudaMemsetAsync(dQ, 0, q_bytes, st)) != cudaSuccess) return e;
+    if (kv_bytes && (e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
+    if (kv_bytes && (e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dW, 0, (size_t)p.d * p.d * sizeof(float), st)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(ws, 0, w.clear_bytes, st)) != cudaSuccess) return e;
+    if (p.rows == 0 || p.C == 0) return cudaSuccess;
+    BwdArgs a;
+    a.B = p.B;
+    a.Tq = p.Tq;
+    a.Tcap = p.Tcap;
+    a.H = p.H;
+    a.Hkv = p.Hkv;
+    a.G = p.G;
+    a.d = p.d;
+    a.S = p.S;
+    a.C = p.C;
+    a.kmax = p.kmax;
+    a.pt = w.pt;
+    a.q_pos0 = p.q_pos0;
+    a.rows = p.rows;
+    a.nbucket = w.nbucket;
+    a.scale = 1.f / sqrtf((float)p.d);
+    a.idx = idx;
+    a.keff = keff;
+    a.score = score;
+    a.w = reinterpret_cast<float *>(ws + w.w);
+    a.e = reinterpret_cast<float *>(ws + w.e);
+    a.bcount = reinterpret_cast<int32_t *>(ws + w.bcount);
+    a.boff = reinterpret_cast<int32_t *>(ws + w.boff);
+    a.pairs = reinterpret_cast<int32_t *>(ws + w.pairs);
+    a.tiles = reinterpret_cast<int4 *>(ws + w.tiles);
+    a.ntiles = reinterpret_cast<int32_t *>(ws + w.hdr + 16);
+    a.dL = reinterpret_cast<float *>(ws + w.dL);
+    a.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
+    const unsigned row_grid = (unsigned)((p.rows + 255) / 256);
+    bwd_prep_kernel<<<row_grid, 256, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_scan_kernel<<<1, NT_SCAN, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_scatter_kernel<<<row_grid, 256, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int grid = (int)(w.max_tiles < sms ? w.max_tiles : sms);
+    const bool bf = p.dtype == HSA_BF16;
+    if (p.d == 64)
+        e = bf ? launch_attend_s<__nv_bfloat16, 64>(a, grid, Q, K, V, dO, dQ, dK, dV, st)
+               : launch_attend_s<float, 64>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
+    else
+        e = bf ? launch_attend_s<__nv_bfloat16, 128>(a, grid, Q, K, V, dO, dQ, dK, dV, st)
+               : launch_attend_s<float, 128>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
+    if (e != cudaSuccess) return e;
+    const long long nch = w.nbucket;
+    const int lm_grid = (int)(nch < 2ll * sms ? nch : 2ll * sms);
+    if (p.d == 64)
+        return bf ? launch_tail_t<__nv_bfloat16, 64>(a, p.Lc, lm_grid, Q, K, W, L, dQ, dK, dW, st)
+                  : launch_tail_t<float, 64>(a, p.Lc, lm_grid, Q, K, W, L, dQ, dK, dW, st);
+    return bf ? launch_tail_t<__nv_bfloat16, 128>(a, p.Lc, lm_grid, Q, K, W, L, dQ, dK, dW, st)
+              : launch_tail_t<float, 128>(a, p.Lc, lm_grid, Q, K, W, L, dQ, dK, dW, st);
+}
+
+}  // namespace hsa

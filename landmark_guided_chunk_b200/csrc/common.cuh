@@ -294,6 +294,20 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
                              cudaStream_t st);
 
 cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
+
+// Backward (backward.cu): workspace layout, support check, kernel count, launch.
+struct BwdLayout {
+    size_t hdr, bcount, dL, clear_bytes, w, e, boff, pairs, tiles, total;
+    long long nbucket, max_tiles;
+    int pt;
+};
+BwdLayout backward_layout(const Prob &p);
+bool backward_supported(const Prob &p);
+int backward_launches(const Prob &p);
+cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms, const void *Q, const void *K,
+                            const void *V, const void *W, const void *L, const int32_t *idx, const float *score,
+                            const int32_t *keff, const void *dO, float *dQ, float *dK, float *dV, float *dW,
+                            cudaStream_t st);
 cudaError_t launch_decode_append(const Prob &p, const void *knew, const void *vnew, void *K, void *V, const void *W,
                                  void *L, cudaStream_t st);
 cudaError_t launch_select(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,

@@ -374,6 +374,46 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     return HSA_OK;
 }
 
+hsa_status_t hsa_backward_workspace_size(const hsa_problem_t *prob, size_t *bytes) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (!bytes) return fail(HSA_ERR_INVALID_ARG, "bytes is NULL");
+    if (!backward_supported(p)) return fail(HSA_ERR_UNSUPPORTED, "backward: problem too large for 32-bit pair indices");
+    *bytes = backward_layout(p).total;
+    return HSA_OK;
+}
+
+hsa_status_t hsa_backward(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const void *W_L,
+                          const void *L, const int32_t *idx, const float *score, const int32_t *keff, const void *dO,
+                          float *dQ, float *dK, float *dV, float *dW_L, void *ws, size_t ws_bytes, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (!backward_supported(p)) return fail(HSA_ERR_UNSUPPORTED, "backward: problem too large for 32-bit pair indices");
+    const bool rows = p.rows > 0;
+    const bool work = rows && p.C > 0;
+    const bool kv = (long long)p.B * p.Tcap > 0;
+    HSA_TRY(need(Q, rows, "Q"));
+    HSA_TRY(need(K, work, "K"));
+    HSA_TRY(need(V, work, "V"));
+    HSA_TRY(need(W_L, work, "W_L"));
+    HSA_TRY(need(L, work, "L"));
+    HSA_TRY(need(idx, work, "idx"));
+    HSA_TRY(need(score, work, "score"));
+    HSA_TRY(need(keff, work, "keff"));
+    HSA_TRY(need(dO, rows, "dO"));
+    HSA_TRY(need(dQ, rows, "dQ"));
+    HSA_TRY(need(dK, kv, "dK"));
+    HSA_TRY(need(dV, kv, "dV"));
+    HSA_TRY(need(dW_L, true, "dW_L"));
+    const BwdLayout w = backward_layout(p);
+    if (ws_bytes < w.total) return fail(HSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, w.total);
+    if (!ws) return fail(HSA_ERR_WORKSPACE, "workspace is NULL");
+    if ((uintptr_t)ws & 255u) return fail(HSA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    cudaError_t e = launch_backward(p, w, (char *)ws, device_sms(), Q, K, V, W_L, L, idx, score, keff, dO, dQ, dK,
+                                    dV, dW_L, (cudaStream_t)stream);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "backward kernel launch");
+}
+
 hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream) {
     if (!ws || ws_bytes < 256) return fail(HSA_ERR_WORKSPACE, "workspace missing or smaller than its header");
     cudaStream_t st = (cudaStream_t)stream;

@@ -28,7 +28,7 @@ from dataclasses import dataclass, field, replace
 
 import torch
 
-__all__ = ["Problem", "WORKLOADS", "workload", "make_inputs", "torch_dtype"]
+__all__ = ["Problem", "WORKLOADS", "workload", "make_inputs", "make_output_grad", "torch_dtype"]
 
 
 @dataclass(frozen=True)
@@ -137,6 +137,17 @@ def make_inputs(p: Problem, seed: int = 0, device: str | torch.device = "cpu") -
     if p.planted > 0:
         out["planted"] = plant_chunks(p, Q, K, gen)
     return out
+
+
+def make_output_grad(p: Problem, seed: int = 0, device: str | torch.device = "cpu") -> torch.Tensor:
+    """An upstream gradient dO [B,Tq,H,d] ~ N(0, 1) in p.dtype for the backward
+    (its own generator, so the forward inputs of the same seed are unchanged)."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    dO = torch.empty(p.B, p.Tq, p.H, p.d, dtype=torch_dtype(p.dtype), device=dev)
+    _randn_into(dO, gen)
+    return dO
 
 
 def plant_chunks(p: Problem, Q: torch.Tensor, K: torch.Tensor, gen: torch.Generator) -> torch.Tensor:

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.EXPORTED)
-    assert lib.hsa_abi_version() == 2
+    assert lib.hsa_abi_version() == 3
 
 
 def test_status_strings():
@@ -126,3 +126,29 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         _native.lib()
+
+
+def _call_backward(prob, ws_bytes=1 << 20, **ptrs):
+    names = ("Q", "K", "V", "W", "L", "idx", "score", "keff", "dO", "dQ", "dK", "dV", "dW", "ws")
+    vals = {n: 256 for n in names}
+    vals.update(ptrs)
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    return _native.lib().hsa_backward(ctypes.byref(prob), *[P(vals[n]) for n in names[:-1]], P(vals["ws"]),
+                                      ws_bytes, None)
+
+
+def test_backward_workspace_and_validation_before_launch():
+    """hsa_backward_workspace_size is host arithmetic; every call below fails in host
+    validation (fake, never-dereferenced addresses)."""
+    p = _prob()
+    n = ctypes.c_size_t()
+    assert _native.lib().hsa_backward_workspace_size(ctypes.byref(p), ctypes.byref(n)) == _native.HSA_OK
+    rows, kmax, G, C = 128 * 2, 4, 2, 2
+    assert n.value >= rows * kmax * (4 + 4 * G + 4) + 2 * C * 64 * 4
+    assert _call_backward(p, dO=None) == _native.HSA_ERR_INVALID_ARG
+    assert b"dO" in _native.lib().hsa_last_error()
+    assert _call_backward(p, dK=24) == _native.HSA_ERR_INVALID_ARG             # misaligned
+    assert _call_backward(p, ws=None) == _native.HSA_ERR_WORKSPACE
+    assert _call_backward(p, ws_bytes=16) == _native.HSA_ERR_WORKSPACE
+    assert _call_backward(p, ws=256 + 16) == _native.HSA_ERR_WORKSPACE        # not 256-byte aligned
+    assert _call_backward(_prob(H=5)) == _native.HSA_ERR_INVALID_ARG
