@@ -316,6 +316,8 @@ def run_b200(args, world, rank, local):
                                  "overlapping the previous and next step's compute (double-buffered device tensors)"},
            "gpu_launches": launches, "roofline": roof, "stages": stages_out, "clocks": clk,
            "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3)}
+    if not args.no_backward:
+        out["backward"] = run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, world)
     del inp, Q, K, V, W, L, O, idx, score, keff, ws
     torch.cuda.empty_cache()
     if not args.no_decode:
@@ -325,6 +327,51 @@ def run_b200(args, world, rank, local):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(p, args.seed)
     return out
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz (clocks.max.sm)
+FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, world):
+    """hsa_backward on the forward's selection: dQ, dK, dV, dW_L (fp32) for a
+    seeded upstream gradient dO.  Algorithmic work: the five S x d contractions
+    per kept (query head, chunk) pair (Q K^T, dO V^T, dZ K, dZ^T Q, (wP)^T dO),
+    2 S d FLOPs each."""
+    from landmark_guided_chunk_b200.inputs import make_output_grad
+    dev = Q.device
+    dO = make_output_grad(p, seed=args.seed + 1000, device=dev)
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, Q.dtype)
+    ws = torch.empty(hsa.backward_workspace_size(prob), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = (torch.empty(Q.shape, **f32), torch.empty(K.shape, **f32), torch.empty(K.shape, **f32),
+           torch.empty(p.d, p.d, **f32))
+
+    def step():
+        hsa.backward(Q, K, V, W, L, idx, score, keff, dO, p.S, p.k, p.tau, q_pos0=p.q_pos0, out=out, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    nsteps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(nsteps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / nsteps, world)
+    flops = 10.0 * p.S * p.d * p.G * float(keff_sum)
+    ach = flops / (ms * 1e-3) / 1e12
+    del ws, out, dO
+    return {"ms": round(ms, 3), "steps": nsteps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
+            "kernels": 6, "dtype": "f32 arithmetic on bf16 inputs" if p.dtype == "bf16" else "f32",
+            "roofline": {"bound": "alu", "achieved": round(ach, 2), "unit": "TFLOP/s",
+                         "peak": round(FFMA_PEAK_TFLOPS, 1), "frac": round(ach / FFMA_PEAK_TFLOPS, 4),
+                         "peak_source": "fp32 FMA lanes x clocks.max.sm (CUDA cores; the backward does not use "
+                                        "the tensor cores yet)"}}
 
 
 def run_decode(args, world, rank, local, pk, name="decode_1m"):
@@ -651,6 +698,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-decode-16m", action="store_true", help="skip the 16M-context decode line (64 GiB cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -258,18 +258,20 @@ def backward_workspace_size(prob: hsa_problem_t) -> int:
     return int(n.value)
 
 
-def backward(Q, K, V, W_L, L, idx, score, keff, dO, S, k, tau=0.0, q_pos0=0, kv_len=None, out=None, ws=None):
+def backward(Q, K, V, W_L, L, idx, score, keff, dO, S, k, tau=0.0, q_pos0=0, kv_len=None, out=None, ws=None,
+             force_simt=False):
     """Gradients (dQ, dK, dV, dW_L), fp32, of the forward with its selection (idx, score,
     keff) held fixed, for the output gradient dO [B,Tq,H,d].  L: the landmarks the forward
     scored ([B, Hkv, K.shape[1] // S, d]).  kv_len as in forward.  out: optional preallocated
-    (dQ, dK, dV, dW_L); ws: optional workspace (uint8, 256-byte aligned)."""
+    (dQ, dK, dV, dW_L); ws: optional workspace (uint8, 256-byte aligned).  force_simt runs the
+    fp32 CUDA-core attention backward where the tensor-core one would apply (bf16, d 128)."""
     _dev(Q, K, V, W_L, L, idx, score, keff, dO, ws)
     B, Tq, H, d = Q.shape
     Tcap, Hkv = K.shape[1], K.shape[2]
     Tkv = Tcap if kv_len is None else kv_len
     if dO.shape != Q.shape or dO.dtype != Q.dtype:
         raise ValueError(f"dO must match Q ({tuple(Q.shape)}, {Q.dtype}); got {tuple(dO.shape)}, {dO.dtype}")
-    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, 0, Tcap)
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, _native.HSA_FLAG_SIMT if force_simt else 0, Tcap)
     if out is None:
         f32 = dict(dtype=torch.float32, device=Q.device)
         out = (torch.empty(B, Tq, H, d, **f32), torch.empty(B, Tcap, Hkv, d, **f32),

@@ -33,6 +33,7 @@
 // All arithmetic is fp32 on CUDA cores (the gradients are fp32 buffers); the
 // stored inputs (fp32 or bf16) are read exactly.
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace hsa {
 namespace {
@@ -578,6 +579,332 @@ __global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T 
     }
 }
 
+// ---------------------------------------------------------------------------- tensor-core attention backward
+//
+// bf16, d = 128, S = 64 or 128.  One CTA of 128 threads per SM; thread r is
+// tile row r and TMEM lane r.  A tile is up to 128 query-head rows that kept
+// one chunk (128 / G pairs).  Per tile, issued by thread 0 on tcgen05 with
+// fp32 accumulators in TMEM:
+//   Z   = Q K^T,  GV = dO V^T          M128 x N=S x K=d   (both operands K-major)
+//   (threads: P = softmax(Z / sqrt d), e = P . GV, dZ = w P (GV - e) / sqrt d, wP;
+//    dZ and wP rounded to bf16 into shared memory, as P is in the forward)
+//   dQ   = dZ K                        M128 x N=d x K=S   (dZ K-major, K MN-major)
+//   dK^T += Q^T dZ,  dV^T += dO^T wP   M=d x N=S x K=128 rows (both MN-major: the
+//                                      same swizzled tiles read transposed)
+// dK^T and dV^T stay in TMEM for a bucket's run of tiles and are added to
+// memory (fp32 reductions, one key per column) when the bucket changes; dQ
+// is added per tile through a staging buffer so each reduction covers whole
+// 128-byte row segments.  TMEM columns: Z [0, S), GV [S, 2S), dQ [0, 128)
+// (over Z and GV, which are read before dQ is issued), dK^T [2S, 3S), dV^T
+// [3S, 4S).  Shared tiles use the 128-byte swizzle of the forward kernel
+// (rows of 64 bf16, 8-row groups 1024 B apart, 16-byte chunk c of row r at
+// c ^ (r & 7)); Q and dO are double-buffered for S = 64 so the next tile's
+// gather overlaps this tile's MMAs.
+
+constexpr int BT_ROWS = 128;
+constexpr int BT_PITCH = 36;   // dQ staging pitch (floats)
+
+struct BwdTcBars {
+    uint64_t zg, mma2, done;
+    uint32_t tmem;
+    int abort;
+};
+
+template <int S> struct BwdTcShape {
+    static constexpr int NQB = S == 64 ? 2 : 1;   // Q / dO buffers
+    static constexpr int KVB = S * 128;           // one 64-column box of S rows
+    static constexpr int PB = (S / 64) * 16384;   // one [128][S] bf16 tile
+    static constexpr int TMEM_COLS = 4 * S;
+    static constexpr size_t smem = 1024 + (size_t)NQB * 2 * 32768 + 4 * (size_t)KVB + 2 * (size_t)PB +
+                                   4 * 32 * BT_PITCH * sizeof(float) + (size_t)NQB * BT_ROWS * sizeof(long long) +
+                                   sizeof(BwdTcBars);
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int S>
+__global__ void __launch_bounds__(BT_ROWS, 1)
+    bwd_tc_kernel(BwdArgs a, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                  const __nv_bfloat16 *__restrict__ V, const __nv_bfloat16 *__restrict__ dO,
+                  float *__restrict__ dQ, float *__restrict__ dK, float *__restrict__ dV) {
+    using namespace sm100;
+    using SH = BwdTcShape<S>;
+    constexpr int NQB = SH::NQB, KVB = SH::KVB, PB = SH::PB, D = 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                       // NQB x 32 KB: two 64-dim boxes of 128 rows
+    uint8_t *sG = sQ + NQB * 32768;           // dO, same layout
+    uint8_t *sK = sG + NQB * 32768;           // two boxes of S rows
+    uint8_t *sV = sK + 2 * KVB;
+    uint8_t *sZ = sV + 2 * KVB;               // dZ, bf16 [128][S]
+    uint8_t *sP = sZ + PB;                    // w P, bf16 [128][S]
+    float *stg = reinterpret_cast<float *>(sP + PB);                          // 4 warps x 32 x BT_PITCH
+    long long *s_qoff = reinterpret_cast<long long *>(stg + 4 * 32 * BT_PITCH);   // [NQB][128]
+    BwdTcBars *bar = reinterpret_cast<BwdTcBars *>(s_qoff + NQB * BT_ROWS);
+    volatile int *abort = &bar->abort;
+    const int r = threadIdx.x, warp = r >> 5, lane = r & 31;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const int ntiles = *a.ntiles;
+    const int lo = (int)((long long)ntiles * blockIdx.x / gridDim.x);
+    const int hi = (int)((long long)ntiles * (blockIdx.x + 1) / gridDim.x);
+    if (lo >= hi) return;
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+
+    if (r == 0) {
+        mbar_init(&bar->zg, 1);
+        mbar_init(&bar->mma2, 1);
+        mbar_init(&bar->done, 1);
+        bar->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&bar->tmem, SH::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem;
+
+    // this thread's row of tile ti: Q / dO rows into buffer qb (zero rows past the tile), its
+    // fusion weight and e slot
+    auto gather = [&](int ti, int qb, float &w_o, int &e_o) {
+        const int4 tr = a.tiles[ti];
+        const int nrow = tr.z * a.G;
+        const int j = (tr.x / a.C) % a.Hkv;
+        const char *srcq = reinterpret_cast<const char *>(Q), *srcg = reinterpret_cast<const char *>(dO);
+        long long qoff = -1;
+        w_o = 0.f;
+        e_o = -1;
+        if (r < nrow) {
+            const int pc = a.pairs[tr.y + r / a.G], g = r % a.G;
+            const long long bt = (long long)(pc / a.kmax) / a.Hkv;
+            qoff = (bt * a.H + (long long)j * a.G + g) * D;
+            w_o = a.w[pc];
+            e_o = pc * a.G + g;
+            srcq += qoff * 2;
+            srcg += qoff * 2;
+        }
+        s_qoff[qb * BT_ROWS + r] = qoff;
+        const uint32_t nb = r < nrow ? 16u : 0u;
+        const uint32_t dq = smem_u32(sQ + qb * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t dg = smem_u32(sG + qb * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+            const uint32_t o = (x >> 3) * 16384 + (((x & 7) ^ (r & 7)) << 4);
+            cp_async16(dq + o, srcq + (nb ? x * 16 : 0), nb);
+            cp_async16(dg + o, srcg + (nb ? x * 16 : 0), nb);
+        }
+    };
+    // K_c and V_c of a bucket into the two box pairs
+    auto load_kv = [&](int bucket) {
+        const int c = bucket % a.C, bj = bucket / a.C, j = bj % a.Hkv, b = bj / a.Hkv;
+        const long long row0 = ((long long)b * a.Tcap + (long long)c * S) * a.Hkv + j;
+        for (int i = r; i < S * 16; i += BT_ROWS) {
+            const int u = i >> 4, x = i & 15;
+            const uint32_t o = (x >> 3) * KVB + (u >> 3) * 1024 + (u & 7) * 128 + (((x & 7) ^ (u & 7)) << 4);
+            const long long src = (row0 + (long long)u * a.Hkv) * D + x * 8;
+            cp_async16(smem_u32(sK) + o, K + src, 16u);
+            cp_async16(smem_u32(sV) + o, V + src, 16u);
+        }
+    };
+    // dK^T and dV^T of the finished bucket -> memory (lane r = dimension r; one key per column)
+    auto drain_kv = [&](int bucket) {
+        const int c = bucket % a.C, bj = bucket / a.C, j = bj % a.Hkv, b = bj / a.Hkv;
+        const long long row0 = ((long long)b * a.Tcap + (long long)c * S) * a.Hkv + j;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float *dst = h ? dV : dK;
+#pragma unroll 1
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + (2 + h) * S + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    float *pd = dst + (row0 + (long long)(q * 32 + e) * a.Hkv) * D + r;
+                    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(pd), "f"(__uint_as_float(v[e])) : "memory");
+                }
+            }
+        }
+    };
+
+    const uint32_t idesc_zg = idesc_bf16_f32(128, S, 0, 0);
+    const uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t idesc_kv = idesc_bf16_f32(128, S, 1, 1);
+    float w_c, w_n = 0.f;
+    int e_c, e_n = -1;
+    int bucket = a.tiles[lo].x;
+    load_kv(bucket);
+    gather(lo, 0, w_c, e_c);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+    bool first = true;   // first tile of the bucket run: dK^T / dV^T start from zero
+    int i = 0;
+    for (int ti = lo; ti < hi; ++ti, ++i) {
+        const int qb = NQB == 2 ? (i & 1) : 0;
+        const bool has_next = ti + 1 < hi;
+        const int nbucket = has_next ? a.tiles[ti + 1].x : -1;
+        // ---- Z = Q K^T, GV = dO V^T
+        if (r == 0) {
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ + qb * 32768), ga = smem_u32(sG + qb * 32768);
+            const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32, bo = (kk >> 2) * KVB + (kk & 3) * 32;
+                umma_bf16(tmem, desc_kmajor_sw128(qa + ao), desc_kmajor_sw128(kb + bo), idesc_zg, kk != 0);
+                umma_bf16(tmem + S, desc_kmajor_sw128(ga + ao), desc_kmajor_sw128(vb + bo), idesc_zg, kk != 0);
+            }
+            umma_commit(&bar->zg);
+        }
+        if (NQB == 2 && has_next) gather(ti + 1, qb ^ 1, w_n, e_n);
+        if (!__syncthreads_and(mbar_wait(&bar->zg, i & 1, abort, a.status))) break;
+        tc_fence_after();
+        // ---- row softmax, e, dZ and w P (this thread's row)
+        {
+            float p[S];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    p[q * 32 + e] = __uint_as_float(v[e]);
+                    mx = fmaxf(mx, p[q * 32 + e]);
+                }
+            }
+            float l = 0.f;
+#pragma unroll
+            for (int u = 0; u < S; ++u) {
+                p[u] = exp2f((p[u] - mx) * scale_log2);
+                l += p[u];
+            }
+            const float inv = 1.f / l;
+            float ev = 0.f;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + S + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    p[q * 32 + e] *= inv;
+                    ev = fmaf(p[q * 32 + e], __uint_as_float(v[e]), ev);
+                }
+            }
+            if (e_c >= 0) a.e[e_c] = ev;
+            const float ws = w_c * a.scale;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + S + q * 32, v);
+                tmem_wait_ld();
+                uint32_t zk[16], pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = p[q * 32 + 2 * e], p1 = p[q * 32 + 2 * e + 1];
+                    __nv_bfloat162 hz = __floats2bfloat162_rn(ws * p0 * (__uint_as_float(v[2 * e]) - ev),
+                                                              ws * p1 * (__uint_as_float(v[2 * e + 1]) - ev));
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(w_c * p0, w_c * p1);
+                    zk[e] = *reinterpret_cast<uint32_t *>(&hz);
+                    pk[e] = *reinterpret_cast<uint32_t *>(&hp);
+                }
+                const int ro = (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int cx = (q & 1) * 4 + x, o = ro + ((cx ^ (r & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(sZ + o) = make_uint4(zk[4 * x], zk[4 * x + 1], zk[4 * x + 2], zk[4 * x + 3]);
+                    *reinterpret_cast<uint4 *>(sP + o) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- dQ = dZ K, dK^T += Q^T dZ, dV^T += dO^T wP
+        if (r == 0) {
+            tc_fence_after();
+            const uint32_t za = smem_u32(sZ), pa = smem_u32(sP), kb = smem_u32(sK);
+            const uint32_t qa = smem_u32(sQ + qb * 32768), ga = smem_u32(sG + qb * 32768);
+#pragma unroll
+            for (int kk = 0; kk < S / 16; ++kk)
+                umma_bf16(tmem, desc_kmajor_sw128(za + (kk >> 2) * 16384 + (kk & 3) * 32),
+                          desc_mnmajor_sw128(kb + kk * 2048, KVB, 1024), idesc_dq, kk != 0);
+#pragma unroll
+            for (int kk = 0; kk < BT_ROWS / 16; ++kk) {
+                const uint32_t acc = (kk != 0 || !first) ? 1u : 0u;
+                umma_bf16(tmem + 2 * S, desc_mnmajor_sw128(qa + kk * 2048, 16384, 1024),
+                          desc_mnmajor_sw128(za + kk * 2048, 16384, 1024), idesc_kv, acc);
+                umma_bf16(tmem + 3 * S, desc_mnmajor_sw128(ga + kk * 2048, 16384, 1024),
+                          desc_mnmajor_sw128(pa + kk * 2048, 16384, 1024), idesc_kv, acc);
+            }
+            umma_commit(&bar->mma2);
+        }
+        if (!__syncthreads_and(mbar_wait(&bar->mma2, i & 1, abort, a.status))) break;
+        tc_fence_after();
+        // ---- dQ rows -> memory, 32 columns at a time through the warp's staging rows
+        {
+            float *wst = stg + warp * 32 * BT_PITCH;
+            long long dst[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) dst[rr] = s_qoff[qb * BT_ROWS + warp * 32 + rr * 4 + (lane >> 3)];
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + q * 32, v);
+                tmem_wait_ld();
+                float *mine = wst + lane * BT_PITCH;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(mine + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    if (dst[rr] >= 0) {
+                        const int lr = rr * 4 + (lane >> 3);
+                        red_add4(dQ + dst[rr] + q * 32 + 4 * (lane & 7),
+                                 *reinterpret_cast<const float4 *>(wst + lr * BT_PITCH + 4 * (lane & 7)));
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        first = nbucket != bucket;
+        if (first) drain_kv(bucket);
+        if (has_next) {
+            if (NQB == 1) gather(ti + 1, 0, w_n, e_n);
+            if (nbucket != bucket) load_kv(nbucket);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        bucket = nbucket;
+        w_c = w_n;
+        e_c = e_n;
+    }
+    cp_async_wait_all();
+    // wind down: every MMA issued has completed before TMEM is released
+    if (r == 0) {
+        umma_commit(&bar->done);
+        mbar_drain(&bar->done, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, SH::TMEM_COLS);
+    }
+}
+
 template <typename T, int S, int D>
 cudaError_t launch_attend_t(const BwdArgs &a, int grid, const void *Q, const void *K, const void *V, const void *dO,
                             float *dQ, float *dK, float *dV, cudaStream_t st) {
@@ -625,7 +952,8 @@ BwdLayout backward_layout(const Prob &p) {
         return o;
     };
     const size_t pairs = (size_t)p.rows * p.kmax;
-    w.pt = RT / p.G;
+    w.tc = p.dtype == HSA_BF16 && p.d == 128 && (p.S == 64 || p.S == 128) && !(p.flags & HSA_FLAG_SIMT);
+    w.pt = (w.tc ? BT_ROWS : RT) / p.G;
     w.nbucket = (long long)p.B * p.Hkv * p.C;
     w.max_tiles = (long long)((pairs + w.pt - 1) / w.pt) + w.nbucket;
     w.hdr = take(256);   // status word at 0, tile count at 16
@@ -698,7 +1026,23 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int grid = (int)(w.max_tiles < sms ? w.max_tiles : sms);
     const bool bf = p.dtype == HSA_BF16;
-    if (p.d == 64)
+    if (w.tc) {
+        const size_t smem = p.S == 64 ? BwdTcShape<64>::smem : BwdTcShape<128>::smem;
+        if (p.S == 64) {
+            e = cudaFuncSetAttribute(bwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess)
+                bwd_tc_kernel<64><<<grid, BT_ROWS, smem, st>>>(a, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                                                               (const __nv_bfloat16 *)V, (const __nv_bfloat16 *)dO,
+                                                               dQ, dK, dV);
+        } else {
+            e = cudaFuncSetAttribute(bwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e == cudaSuccess)
+                bwd_tc_kernel<128><<<grid, BT_ROWS, smem, st>>>(a, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                                                                (const __nv_bfloat16 *)V, (const __nv_bfloat16 *)dO,
+                                                                dQ, dK, dV);
+        }
+        if (e == cudaSuccess) e = cudaGetLastError();
+    } else if (p.d == 64)
         e = bf ? launch_attend_s<__nv_bfloat16, 64>(a, grid, Q, K, V, dO, dQ, dK, dV, st)
                : launch_attend_s<float, 64>(a, grid, Q, K, V, dO, dQ, dK, dV, st);
     else

@@ -299,7 +299,8 @@ cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *
 struct BwdLayout {
     size_t hdr, bcount, dL, clear_bytes, w, e, boff, pairs, tiles, total;
     long long nbucket, max_tiles;
-    int pt;
+    int pt;    // pairs per tile
+    bool tc;   // tensor-core attention backward (bf16, d 128, S 64 / 128)
 };
 BwdLayout backward_layout(const Prob &p);
 bool backward_supported(const Prob &p);

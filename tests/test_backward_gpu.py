@@ -8,13 +8,20 @@ differentiates the same selection on the same stored inputs, scoring on the
 landmarks the library stored (their rounding counts as the identity on both
 sides).
 
-Tolerance, per gradient tensor: max |gpu - oracle| <= 1e-4 * max |oracle|.  Both
-sides read the same stored values; the GPU accumulates in fp32 (its fusion
-weights come from the forward's fp32 scores, relative error ~1e-6; every sum
-it forms has fp32 rounding ~6e-8 relative to its terms' magnitude, and the
-largest sums have a few thousand terms), so 1e-4 of the tensor's scale covers
-the accumulated rounding with a wide margin while a dropped term or wrong
-factor (the oracle pins show those move a gradient by O(1) of its scale) fails.
+Tolerance, per gradient tensor, as max |gpu - oracle| / max |oracle|:
+  * CUDA-core path (fp32, and bf16 with HSA_FLAG_SIMT or d = 64): 1e-4.  Both
+    sides read the same stored values; the GPU accumulates in fp32 (its fusion
+    weights come from the forward's fp32 scores, relative error ~1e-6; every
+    sum has fp32 rounding ~6e-8 relative to its terms, a few thousand terms at
+    most), measured 2e-7 .. 1e-6.
+  * tensor-core path (bf16, d = 128, S 64 / 128): 1e-2.  dZ and w P are rounded
+    once to bf16 (relative error <= 2^-9 = 1.95e-3) before the dQ, dK and dV
+    contractions, as P is in the forward; every term of those sums carries
+    one such factor, and the measured worst is 2.6e-3 of the tensor's scale.
+    1e-2 (about 5 x 2^-9) bounds that with margin; e, the score path and dW_L
+    stay fp32 (measured ~1e-6).
+A dropped term or a wrong factor moves a gradient by O(1) of its scale (the
+oracle pins show that), so both bounds still catch one.
 """
 import numpy as np
 import pytest
@@ -27,17 +34,22 @@ from landmark_guided_chunk_b200.inputs import Problem, make_inputs, make_output_
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-4
+TOL_TC = 1e-2
 
 
-def _close(name, got, ref):
+def _tc_path(p: Problem, force_simt=False) -> bool:
+    return p.dtype == "bf16" and p.d == 128 and p.S in (64, 128) and not force_simt
+
+
+def _close(name, got, ref, tol=TOL):
     got = got.double().cpu().numpy() if isinstance(got, torch.Tensor) else got
     scale = float(np.abs(ref).max()) if ref.size else 0.0
     err = float(np.abs(got - ref).max()) if ref.size else 0.0
-    assert err <= TOL * max(scale, 1e-30), f"{name}: max error {err:.3g} vs scale {scale:.3g}"
+    assert err <= tol * max(scale, 1e-30), f"{name}: max error {err:.3g} vs scale {scale:.3g} (tol {tol:g})"
     return err / max(scale, 1e-30)
 
 
-def _run(p: Problem, seed: int, kv_len=None, W_random=True):
+def _run(p: Problem, seed: int, kv_len=None, W_random=True, force_simt=False):
     inp = make_inputs(p, seed=seed, device="cuda")
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
     if W_random and p.is_decode:
@@ -47,7 +59,8 @@ def _run(p: Problem, seed: int, kv_len=None, W_random=True):
     n = K.shape[1] if kv_len is None else kv_len
     O, L, idx, sc, ke = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, q_pos0=p.q_pos0, return_selection=True,
                                     kv_len=kv_len)
-    dQ, dK, dV, dW = hsa.backward(Q, K, V, W, L, idx, sc, ke, dO, p.S, p.k, p.tau, q_pos0=p.q_pos0, kv_len=kv_len)
+    dQ, dK, dV, dW = hsa.backward(Q, K, V, W, L, idx, sc, ke, dO, p.S, p.k, p.tau, q_pos0=p.q_pos0, kv_len=kv_len,
+                                  force_simt=force_simt)
     torch.cuda.synchronize()
     return dict(Q=Q, K=K, V=V, W=W, dO=dO, L=L, idx=idx, sc=sc, ke=ke, dQ=dQ, dK=dK, dV=dV, dW=dW, n=n)
 
@@ -66,53 +79,54 @@ def _oracle_rows(r, p, rows_b, rows_t):
     return oracle.backward(Qr, np.asarray(rows_b), K, V, r["W"].cpu(), L, p.S, sel, dOr)
 
 
-def _full_check(p, r):
+def _full_check(p, r, tol):
     B, Tq = p.B, p.Tq
     rows_b = np.repeat(np.arange(B), Tq)
     rows_t = np.tile(np.arange(Tq), B)
     g = _oracle_rows(r, p, rows_b, rows_t)
     n = r["n"]
-    errs = {"dQ": _close("dQ", r["dQ"].reshape(B * Tq, p.H, p.d), g["dQ"]),
-            "dK": _close("dK", r["dK"][:, :n], g["dK"]),
-            "dV": _close("dV", r["dV"][:, :n], g["dV"]),
-            "dW": _close("dW", r["dW"], g["dW"])}
+    errs = {"dQ": _close("dQ", r["dQ"].reshape(B * Tq, p.H, p.d), g["dQ"], tol),
+            "dK": _close("dK", r["dK"][:, :n], g["dK"], tol),
+            "dV": _close("dV", r["dV"][:, :n], g["dV"], tol),
+            "dW": _close("dW", r["dW"], g["dW"], tol)}
     # tokens past the complete chunks (trailing partial chunk, spare capacity) get exactly 0
     c_end = (n // p.S) * p.S
     assert torch.all(r["dK"][:, c_end:] == 0) and torch.all(r["dV"][:, c_end:] == 0)
     return errs
 
 
-@pytest.mark.parametrize("case", [
-    "tiny_f32",
-    "bf16_gqa4_S64",
-    "bf16_router_S128",
-    "f32_G16_S32_capacity",
-    "bf16_decode_rows",
-])
+CASES = {
+    "tiny_f32": (workload("tiny_f32"), None, False),
+    "bf16_gqa4_S64": (Problem(B=2, Tq=64 * 12 + 37, Tkv=64 * 12 + 37, H=8, Hkv=2, d=128, S=64, k=4, dtype="bf16"),
+                      None, False),
+    "bf16_gqa4_S64_simt": (Problem(B=2, Tq=64 * 12 + 37, Tkv=64 * 12 + 37, H=8, Hkv=2, d=128, S=64, k=4,
+                                   dtype="bf16"), None, True),
+    "bf16_router_S128_d64": (Problem(B=1, Tq=128 * 9 + 5, Tkv=128 * 9 + 5, H=4, Hkv=2, d=64, S=128, k=3, tau=0.05,
+                                     dtype="bf16"), None, False),
+    "bf16_router_S128_d128": (Problem(B=1, Tq=128 * 9 + 5, Tkv=128 * 9 + 5, H=8, Hkv=2, d=128, S=128, k=3,
+                                      tau=0.05, dtype="bf16"), None, False),
+    "bf16_G1_S64": (Problem(B=1, Tq=64 * 10 + 3, Tkv=64 * 10 + 3, H=2, Hkv=2, d=128, S=64, k=6, dtype="bf16"),
+                    None, False),
+    "bf16_G16_S128": (Problem(B=1, Tq=128 * 6 + 9, Tkv=128 * 6 + 9, H=16, Hkv=1, d=128, S=128, k=2, dtype="bf16"),
+                      None, False),
+    "f32_G16_S32_capacity": (Problem(B=1, Tq=32 * 20 + 7, Tkv=32 * 20 + 7 + 45, H=16, Hkv=1, d=64, S=32, k=5,
+                                     dtype="f32"), 32 * 20 + 7, False),
+    "bf16_capacity_S64": (Problem(B=2, Tq=64 * 9 + 20, Tkv=64 * 9 + 20 + 100, H=8, Hkv=2, d=128, S=64, k=3,
+                                  dtype="bf16"), 64 * 9 + 20, False),
+    "bf16_decode_rows": (Problem(B=3, Tq=1, Tkv=64 * 50 + 9, H=8, Hkv=2, d=128, S=64, k=8, q_pos0=64 * 50 + 9,
+                                 dtype="bf16"), None, False),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
 def test_backward_matches_oracle(case):
-    kv_len = None
-    if case == "tiny_f32":
-        p = workload("tiny_f32")
-    elif case == "bf16_gqa4_S64":
-        p = Problem(B=2, Tq=64 * 12 + 37, Tkv=64 * 12 + 37, H=8, Hkv=2, d=128, S=64, k=4, dtype="bf16")
-    elif case == "bf16_router_S128":
-        p = Problem(B=1, Tq=128 * 9 + 5, Tkv=128 * 9 + 5, H=4, Hkv=2, d=64, S=128, k=3, tau=0.05, dtype="bf16")
-    elif case == "f32_G16_S32_capacity":
-        T = 32 * 20 + 7
-        p = Problem(B=1, Tq=T, Tkv=T + 45, H=16, Hkv=1, d=64, S=32, k=5, dtype="f32")
-        kv_len = T
-    else:
-        T = 64 * 50 + 9
-        p = Problem(B=3, Tq=1, Tkv=T, H=8, Hkv=2, d=128, S=64, k=8, q_pos0=T, dtype="bf16")
+    p, kv_len, simt = CASES[case]
+    r = _run(p, seed=40, kv_len=kv_len, force_simt=simt)
     if kv_len is not None:
-        inp_p = p
-        r = _run(inp_p, seed=40, kv_len=kv_len)
         p = p.with_(Tkv=kv_len)
-    else:
-        r = _run(p, seed=40)
     if p.tau > 0:
         assert int((r["ke"] > p.k).sum()) > 0, "the router case must double some rows"
-    _full_check(p, r)
+    _full_check(p, r, TOL_TC if _tc_path(p, simt) else TOL)
 
 
 def test_backward_without_candidates_is_zero():
@@ -135,13 +149,17 @@ def test_backward_prefill_full_size_sampled_rows():
     rows_t = np.sort(np.concatenate([rng.choice(p.Tq, 24, replace=False), [p.S, p.Tq - 1]]))
     rows_b = np.zeros_like(rows_t)
     g = _oracle_rows(r, p, rows_b, rows_t)
-    _close("dQ (sampled rows)", r["dQ"][0, torch.as_tensor(rows_t)], g["dQ"])
+    _close("dQ (sampled rows)", r["dQ"][0, torch.as_tensor(rows_t)], g["dQ"], TOL_TC)
     dO = r["dO"].double()
     kept = (r["ke"] > 0).double()                                       # [B,Tq,Hkv]
     dOg = dO.view(p.B, p.Tq, p.Hkv, p.G, p.d).sum(3)                     # [B,Tq,Hkv,d]
     expect = (dOg * kept.unsqueeze(-1)).sum(1)                           # [B,Hkv,d]
     got = r["dV"].double().sum(1)
-    scale = float(r["dV"].double().abs().sum(1).max())
-    assert float((got - expect).abs().max()) <= 1e-5 * scale
+    # w P is rounded to bf16 before the dV contraction: each kept row's share is off by at most
+    # 2^-9 of its |dO| (its weights and probabilities sum to 1)
+    bound = 2.0 ** -9 * (dOg.abs() * kept.unsqueeze(-1)).sum(1) + 1e-5 * float(r["dV"].double().abs().sum(1).max())
+    assert bool(((got - expect).abs() <= bound).all())
+    # dZ is rounded to bf16 as well: the per-chunk sums of its entries are zero only up to those
+    # independent roundings, whose total grows like the square root of their count
     kscale = float(r["dK"].double().abs().sum(1).max())
-    assert float(r["dK"].double().sum(1).abs().max()) <= 1e-5 * kscale
+    assert float(r["dK"].double().sum(1).abs().max()) <= 2.0 ** -9 * kscale
