@@ -366,12 +366,17 @@ def run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, wo
     flops = 10.0 * p.S * p.d * p.G * float(keff_sum)
     ach = flops / (ms * 1e-3) / 1e12
     del ws, out, dO
+    tc = p.dtype == "bf16" and p.d == 128 and p.S in (64, 128)
+    pk = peaks()
+    roof = ({"bound": "tensor", "achieved": round(ach, 2), "unit": "TFLOP/s", "peak": pk["bf16_tflops_sustained"],
+             "frac": round(ach / pk["bf16_tflops_sustained"], 4),
+             "peak_source": f"{pk['source']} (sustained bf16); whole backward call, 6 kernels"} if tc else
+            {"bound": "alu", "achieved": round(ach, 2), "unit": "TFLOP/s", "peak": round(FFMA_PEAK_TFLOPS, 1),
+             "frac": round(ach / FFMA_PEAK_TFLOPS, 4),
+             "peak_source": "fp32 FMA lanes x clocks.max.sm (CUDA-core path)"})
     return {"ms": round(ms, 3), "steps": nsteps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
-            "kernels": 6, "dtype": "f32 arithmetic on bf16 inputs" if p.dtype == "bf16" else "f32",
-            "roofline": {"bound": "alu", "achieved": round(ach, 2), "unit": "TFLOP/s",
-                         "peak": round(FFMA_PEAK_TFLOPS, 1), "frac": round(ach / FFMA_PEAK_TFLOPS, 4),
-                         "peak_source": "fp32 FMA lanes x clocks.max.sm (CUDA cores; the backward does not use "
-                                        "the tensor cores yet)"}}
+            "kernels": 6, "path": "tensor" if tc else "simt",
+            "dtype": "bf16 operands, fp32 accumulation" if tc else "f32", "roofline": roof}
 
 
 def run_decode(args, world, rank, local, pk, name="decode_1m"):

@@ -115,6 +115,9 @@ CASES = {
                                   dtype="bf16"), 64 * 9 + 20, False),
     "bf16_decode_rows": (Problem(B=3, Tq=1, Tkv=64 * 50 + 9, H=8, Hkv=2, d=128, S=64, k=8, q_pos0=64 * 50 + 9,
                                  dtype="bf16"), None, False),
+    # G = 16 over 73 chunks: tiles of 8 pairs, many tiles per chunk
+    "bf16_G16_long": (Problem(B=1, Tq=4096 + 600, Tkv=4096 + 600, H=32, Hkv=2, d=128, S=64, k=2, dtype="bf16"),
+                      None, False),
 }
 
 
