@@ -669,13 +669,14 @@ __global__ void __launch_bounds__(BT_ROWS, 1)
     tc_fence_after();
     const uint32_t tmem = bar->tmem;
 
-    // this thread's row of tile ti: Q / dO rows into buffer qb (zero rows past the tile), its
-    // fusion weight and e slot
+    // Tile ti's Q / dO rows into buffer qb (zero rows past the tile).  Each thread first looks up
+    // its own row (and keeps that row's fusion weight and e slot); then the copies are dealt so
+    // that 16 consecutive lanes copy one row's 256 contiguous bytes, two rows per warp
+    // instruction, instead of one row per lane.
     auto gather = [&](int ti, int qb, float &w_o, int &e_o) {
         const int4 tr = a.tiles[ti];
         const int nrow = tr.z * a.G;
         const int j = (tr.x / a.C) % a.Hkv;
-        const char *srcq = reinterpret_cast<const char *>(Q), *srcg = reinterpret_cast<const char *>(dO);
         long long qoff = -1;
         w_o = 0.f;
         e_o = -1;
@@ -685,18 +686,20 @@ __global__ void __launch_bounds__(BT_ROWS, 1)
             qoff = (bt * a.H + (long long)j * a.G + g) * D;
             w_o = a.w[pc];
             e_o = pc * a.G + g;
-            srcq += qoff * 2;
-            srcg += qoff * 2;
         }
         s_qoff[qb * BT_ROWS + r] = qoff;
-        const uint32_t nb = r < nrow ? 16u : 0u;
-        const uint32_t dq = smem_u32(sQ + qb * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
-        const uint32_t dg = smem_u32(sG + qb * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-            const uint32_t o = (x >> 3) * 16384 + (((x & 7) ^ (r & 7)) << 4);
-            cp_async16(dq + o, srcq + (nb ? x * 16 : 0), nb);
-            cp_async16(dg + o, srcg + (nb ? x * 16 : 0), nb);
+        __syncthreads();
+        const char *q8 = reinterpret_cast<const char *>(Q), *g8 = reinterpret_cast<const char *>(dO);
+        const uint32_t bq = smem_u32(sQ + qb * 32768), bg = smem_u32(sG + qb * 32768);
+#pragma unroll 4
+        for (int k = 0; k < 16; ++k) {
+            const int idx = r + BT_ROWS * k, row = idx >> 4, x = idx & 15;
+            const long long off = s_qoff[qb * BT_ROWS + row];
+            const uint32_t nb = off >= 0 ? 16u : 0u;
+            const long long src = off >= 0 ? off * 2 + x * 16 : 0;
+            const uint32_t o = (x >> 3) * 16384 + (row >> 3) * 1024 + (row & 7) * 128 + (((x & 7) ^ (row & 7)) << 4);
+            cp_async16(bq + o, q8 + src, nb);
+            cp_async16(bg + o, g8 + src, nb);
         }
     };
     // K_c and V_c of a bucket into the two box pairs
