@@ -624,6 +624,23 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// arrive on *bar once this thread's earlier cp.async copies have landed (no pending-count increment)
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(sm100::smem_u32(bar)) : "memory");
+}
+
+// (batch, kv head, chunk) of a bucket index (b * Hkv + j) * C + c
+struct BucketPos {
+    int b, j, c;
+};
+__device__ __forceinline__ BucketPos bucket_pos(const BwdArgs &a, int bucket) {
+    BucketPos q;
+    q.c = bucket % a.C;
+    const int bj = bucket / a.C;
+    q.j = bj % a.Hkv;
+    q.b = bj / a.Hkv;
+    return q;
+}
 
 template <int S>
 __global__ void __launch_bounds__(BT_ROWS, 1)
@@ -908,6 +925,370 @@ __global__ void __launch_bounds__(BT_ROWS, 1)
     }
 }
 
+// ---------------------------------------------------------------------------- warp-specialized tensor-core backward (S = 64)
+//
+// The tile steps of bwd_tc_kernel, with roles that overlap from tile to tile:
+//   warps 0-3   producers: each tile's row info (query offset, fusion weight, e slot) into a ring
+//               of NWI slots, the Q / dO rows into one of two buffers (16 lanes per 256-byte row),
+//               and K / V once per chunk run
+//   warps 4-7   softmax: P, e, dZ and w P of tile i (thread = TMEM lane = row)
+//   warps 8-11  drain: dQ of every tile through the staging rows, dK^T / dV^T at a run's end
+//   warp 12     one thread issues the MMAs
+// TMEM: Z / GV of tile parity b at [128 b, 128 b + 64) / [128 b + 64, 128 b + 128), dQ [256, 384),
+// dK^T [384, 448), dV^T [448, 512).  So the softmax of tile i+1 runs while the drain of tile i
+// reduces its dQ, and the producers gather tile i+2.  Each barrier has one group of waiters that
+// waits its phases in order, and every wait is bounded.
+
+constexpr int NW_P = 4, NW_S = 4, NW_D = 4;
+constexpr int NT_W = 32 * (NW_P + NW_S + NW_D + 1);
+constexpr int NWI = 4;   // row-info ring slots
+
+struct BwInfo {
+    long long qoff[BT_ROWS];
+    float w[BT_ROWS];
+    int e[BT_ROWS];
+};
+
+struct BwBars {
+    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, zg_full[2], zg_empty[2], ds_full, ds_empty, dq_full, dq_empty;
+    uint64_t info_full[NWI], info_empty[NWI], done;
+    uint32_t tmem;
+    int abort;
+};
+
+constexpr size_t BW_SMEM = 1024 + 4 * 32768 + 4 * 8192 + 2 * 16384 + NW_D * 32 * BT_PITCH * sizeof(float) +
+                           NWI * sizeof(BwInfo) + sizeof(BwBars);
+
+__global__ void __launch_bounds__(NT_W, 1)
+    bwd_tcw_kernel(BwdArgs a, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                   const __nv_bfloat16 *__restrict__ V, const __nv_bfloat16 *__restrict__ dO,
+                   float *__restrict__ dQ, float *__restrict__ dK, float *__restrict__ dV) {
+    using namespace sm100;
+    constexpr int S = 64, D = 128, KVB = S * 128;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = base;                    // 2 x 32 KB
+    uint8_t *sG = sQ + 2 * 32768;          // 2 x 32 KB
+    uint8_t *sK = sG + 2 * 32768;          // two boxes of S rows
+    uint8_t *sV = sK + 2 * KVB;
+    uint8_t *sZ = sV + 2 * KVB;            // dZ, bf16 [128][64]
+    uint8_t *sP = sZ + 16384;              // w P
+    float *stg = reinterpret_cast<float *>(sP + 16384);
+    BwInfo *info = reinterpret_cast<BwInfo *>(stg + NW_D * 32 * BT_PITCH);
+    BwBars *bar = reinterpret_cast<BwBars *>(info + NWI);
+    volatile int *abort = &bar->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = *a.ntiles;
+    const int lo = (int)((long long)ntiles * blockIdx.x / gridDim.x);
+    const int hi = (int)((long long)ntiles * (blockIdx.x + 1) / gridDim.x);
+    const int n = hi - lo;
+    if (n <= 0) return;
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+
+    if (threadIdx.x == 0) {
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&bar->q_full[q], 32 * NW_P);
+            mbar_init(&bar->q_empty[q], 1);
+            mbar_init(&bar->zg_full[q], 1);
+            mbar_init(&bar->zg_empty[q], NW_S);
+        }
+        mbar_init(&bar->kv_full, 32 * NW_P);
+        mbar_init(&bar->kv_empty, 1);
+        mbar_init(&bar->ds_full, NW_S);
+        mbar_init(&bar->ds_empty, 1);
+        mbar_init(&bar->dq_full, 1);
+        mbar_init(&bar->dq_empty, NW_D);
+        for (int q = 0; q < NWI; ++q) {
+            mbar_init(&bar->info_full[q], NW_P);
+            mbar_init(&bar->info_empty[q], NW_D);
+        }
+        mbar_init(&bar->done, 1);
+        bar->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == NW_P + NW_S + NW_D) {
+        tmem_alloc(&bar->tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem;
+    auto bucket_at = [&](int i) -> int { return i < n ? a.tiles[lo + i].x : -1; };
+    auto wait_all = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(FULL, mbar_wait(b, par, abort, a.status) ? 1 : 0) != 0;
+    };
+
+    if (warp < NW_P) {
+        // ------------------------------------------------------------ producers
+        const int pr = threadIdx.x;   // this thread's row of each tile
+        int prev = -1, nload = 0;
+        for (int i = 0; i < n; ++i) {
+            const int b = i & 1, si = i % NWI;
+            const int4 tr = a.tiles[lo + i];
+            if (tr.x != prev) {
+                // K / V of a new chunk run, once the previous run's last MMAs have released them
+                if (nload > 0 && !wait_all(&bar->kv_empty, (nload - 1) & 1)) break;
+                const BucketPos bp = bucket_pos(a, tr.x);
+                const long long row0 = ((long long)bp.b * a.Tcap + (long long)bp.c * S) * a.Hkv + bp.j;
+                for (int q = pr; q < S * 16; q += 32 * NW_P) {
+                    const int u = q >> 4, x = q & 15;
+                    const uint32_t o = (x >> 3) * KVB + (u >> 3) * 1024 + (u & 7) * 128 + (((x & 7) ^ (u & 7)) << 4);
+                    const long long src = (row0 + (long long)u * a.Hkv) * D + x * 8;
+                    cp_async16(smem_u32(sK) + o, K + src, 16u);
+                    cp_async16(smem_u32(sV) + o, V + src, 16u);
+                }
+                cp_async_arrive(&bar->kv_full);
+                ++nload;
+                prev = tr.x;
+            }
+            if (i >= 2 && !wait_all(&bar->q_empty[b], ((i >> 1) - 1) & 1)) break;
+            if (i >= NWI && !wait_all(&bar->info_empty[si], ((i / NWI) - 1) & 1)) break;
+            long long qoff = -1;
+            float w = 0.f;
+            int e = -1;
+            if (pr < tr.z * a.G) {
+                const int pc = a.pairs[tr.y + pr / a.G], g = pr % a.G;
+                const long long bt = (long long)(pc / a.kmax) / a.Hkv;
+                qoff = (bt * a.H + (long long)bucket_pos(a, tr.x).j * a.G + g) * D;
+                w = a.w[pc];
+                e = pc * a.G + g;
+            }
+            info[si].qoff[pr] = qoff;
+            info[si].w[pr] = w;
+            info[si].e[pr] = e;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->info_full[si]);
+            // this warp's 32 rows, 16 lanes per row
+            const char *q8 = reinterpret_cast<const char *>(Q), *g8 = reinterpret_cast<const char *>(dO);
+            const uint32_t bq = smem_u32(sQ + b * 32768), bg = smem_u32(sG + b * 32768);
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int rr = 2 * k + (lane >> 4), x = lane & 15;
+                const long long off = __shfl_sync(FULL, qoff, rr);
+                const int row = warp * 32 + rr;
+                const uint32_t nb = off >= 0 ? 16u : 0u;
+                const long long src = off >= 0 ? off * 2 + x * 16 : 0;
+                const uint32_t o = (x >> 3) * 16384 + (row >> 3) * 1024 + (row & 7) * 128 + (((x & 7) ^ (row & 7)) << 4);
+                cp_async16(bq + o, q8 + src, nb);
+                cp_async16(bg + o, g8 + src, nb);
+            }
+            cp_async_arrive(&bar->q_full[b]);
+        }
+        cp_async_wait_all();
+    } else if (warp < NW_P + NW_S) {
+        // ------------------------------------------------------------ softmax
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        for (int i = 0; i < n; ++i) {
+            const int b = i & 1, si = i % NWI;
+            if (!wait_all(&bar->info_full[si], (i / NWI) & 1)) break;
+            const float w = info[si].w[row];
+            const int eslot = info[si].e[row];
+            if (!wait_all(&bar->zg_full[b], (i >> 1) & 1)) break;
+            tc_fence_after();
+            const uint32_t zt = tmem + lane_off + b * 128, gt = zt + 64;
+            float p[S];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(zt + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    p[q * 32 + x] = __uint_as_float(v[x]);
+                    mx = fmaxf(mx, p[q * 32 + x]);
+                }
+            }
+            float l = 0.f;
+#pragma unroll
+            for (int u = 0; u < S; ++u) {
+                p[u] = exp2f((p[u] - mx) * scale_log2);
+                l += p[u];
+            }
+            const float inv = 1.f / l;
+            float ev = 0.f;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(gt + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    p[q * 32 + x] *= inv;
+                    ev = fmaf(p[q * 32 + x], __uint_as_float(v[x]), ev);
+                }
+            }
+            if (eslot >= 0) a.e[eslot] = ev;
+            // dZ / w P buffer: free once the previous tile's MMAs have read it
+            if (i >= 1 && !wait_all(&bar->ds_empty, (i - 1) & 1)) break;
+            const float ws = w * a.scale;
+#pragma unroll
+            for (int q = 0; q < S / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(gt + q * 32, v);
+                tmem_wait_ld();
+                uint32_t zk[16], pk[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const float p0 = p[q * 32 + 2 * x], p1 = p[q * 32 + 2 * x + 1];
+                    __nv_bfloat162 hz = __floats2bfloat162_rn(ws * p0 * (__uint_as_float(v[2 * x]) - ev),
+                                                              ws * p1 * (__uint_as_float(v[2 * x + 1]) - ev));
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(w * p0, w * p1);
+                    zk[x] = *reinterpret_cast<uint32_t *>(&hz);
+                    pk[x] = *reinterpret_cast<uint32_t *>(&hp);
+                }
+                const int ro = (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int cx = q * 4 + x, o = ro + ((cx ^ (row & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(sZ + o) = make_uint4(zk[4 * x], zk[4 * x + 1], zk[4 * x + 2], zk[4 * x + 3]);
+                    *reinterpret_cast<uint4 *>(sP + o) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar->zg_empty[b]);
+                mbar_arrive(&bar->ds_full);
+            }
+        }
+    } else if (warp < NW_P + NW_S + NW_D) {
+        // ------------------------------------------------------------ drain
+        const int quad = warp & 3;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float *wst = stg + quad * 32 * BT_PITCH;
+        int bk_next = bucket_at(0);
+        for (int i = 0; i < n; ++i) {
+            const int si = i % NWI, bk = bk_next;
+            bk_next = bucket_at(i + 1);
+            if (!wait_all(&bar->info_full[si], (i / NWI) & 1)) break;
+            long long dst[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) dst[rr] = info[si].qoff[quad * 32 + rr * 4 + (lane >> 3)];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->info_empty[si]);
+            if (!wait_all(&bar->dq_full, i & 1)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int q = 0; q < D / 32; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + 256 + q * 32, v);
+                tmem_wait_ld();
+                float *mine = wst + lane * BT_PITCH;
+#pragma unroll
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4 *>(mine + x) = make_float4(__uint_as_float(v[x]), __uint_as_float(v[x + 1]),
+                                                                        __uint_as_float(v[x + 2]), __uint_as_float(v[x + 3]));
+                __syncwarp();
+#pragma unroll
+                for (int rr = 0; rr < 8; ++rr) {
+                    if (dst[rr] >= 0) {
+                        const int lr = rr * 4 + (lane >> 3);
+                        red_add4(dQ + dst[rr] + q * 32 + 4 * (lane & 7),
+                                 *reinterpret_cast<const float4 *>(wst + lr * BT_PITCH + 4 * (lane & 7)));
+                    }
+                }
+                __syncwarp();
+            }
+            if (bk_next != bk) {
+                // end of this CTA's run of the chunk: dK^T / dV^T (lane = dimension) -> memory
+                const BucketPos bp = bucket_pos(a, bk);
+                const long long row0 = ((long long)bp.b * a.Tcap + (long long)bp.c * S) * a.Hkv + bp.j;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    float *dstp = h ? dV : dK;
+#pragma unroll 1
+                    for (int q = 0; q < S / 32; ++q) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + lane_off + 384 + h * 64 + q * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) {
+                            float *pd = dstp + (row0 + (long long)(q * 32 + x) * a.Hkv) * D + quad * 32 + lane;
+                            asm volatile("red.global.add.f32 [%0], %1;" ::"l"(pd), "f"(__uint_as_float(v[x])) : "memory");
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->dq_empty);
+        }
+    } else if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t idesc_zg = idesc_bf16_f32(128, S, 0, 0);
+        const uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
+        const uint32_t idesc_kv = idesc_bf16_f32(128, S, 1, 1);
+        const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), za = smem_u32(sZ), pa = smem_u32(sP);
+        auto mma1 = [&](int i, bool newc, int li) -> bool {
+            const int b = i & 1;
+            if (!mbar_wait(&bar->q_full[b], (i >> 1) & 1, abort, a.status)) return false;
+            if (newc && !mbar_wait(&bar->kv_full, li & 1, abort, a.status)) return false;
+            if (i >= 2 && !mbar_wait(&bar->zg_empty[b], ((i >> 1) - 1) & 1, abort, a.status)) return false;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ + b * 32768), ga = smem_u32(sG + b * 32768);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32, bo = (kk >> 2) * KVB + (kk & 3) * 32;
+                umma_bf16(tmem + b * 128, desc_kmajor_sw128(qa + ao), desc_kmajor_sw128(kb + bo), idesc_zg, kk != 0);
+                umma_bf16(tmem + b * 128 + 64, desc_kmajor_sw128(ga + ao), desc_kmajor_sw128(vb + bo), idesc_zg, kk != 0);
+            }
+            umma_commit(&bar->zg_full[b]);
+            return true;
+        };
+        auto mma2 = [&](int i, bool first, bool endc) -> bool {
+            if (!mbar_wait(&bar->ds_full, i & 1, abort, a.status)) return false;
+            if (i >= 1 && !mbar_wait(&bar->dq_empty, (i - 1) & 1, abort, a.status)) return false;
+            tc_fence_after();
+            const uint32_t qa = smem_u32(sQ + (i & 1) * 32768), ga = smem_u32(sG + (i & 1) * 32768);
+#pragma unroll
+            for (int kk = 0; kk < S / 16; ++kk)
+                umma_bf16(tmem + 256, desc_kmajor_sw128(za + (kk & 3) * 32), desc_mnmajor_sw128(kb + kk * 2048, KVB, 1024),
+                          idesc_dq, kk != 0);
+#pragma unroll
+            for (int kk = 0; kk < BT_ROWS / 16; ++kk) {
+                const uint32_t acc = (kk != 0 || !first) ? 1u : 0u;
+                umma_bf16(tmem + 384, desc_mnmajor_sw128(qa + kk * 2048, 16384, 1024),
+                          desc_mnmajor_sw128(za + kk * 2048, 16384, 1024), idesc_kv, acc);
+                umma_bf16(tmem + 448, desc_mnmajor_sw128(ga + kk * 2048, 16384, 1024),
+                          desc_mnmajor_sw128(pa + kk * 2048, 16384, 1024), idesc_kv, acc);
+            }
+            umma_commit(&bar->dq_full);
+            umma_commit(&bar->ds_empty);
+            umma_commit(&bar->q_empty[i & 1]);
+            if (endc) umma_commit(&bar->kv_empty);
+            return true;
+        };
+        bool ok = true, first_prev = false, end_prev = false;
+        int prev = -1, li = -1, bk_next = bucket_at(0);
+        for (int i = 0; i < n && ok; ++i) {
+            const int bk = bk_next;
+            bk_next = bucket_at(i + 1);
+            const bool newc = bk != prev, endc = bk_next != bk;
+            if (newc) ++li;
+            // at a run boundary the previous tile's MMAs release K / V before the new run's land
+            if (i >= 1 && newc) ok = mma2(i - 1, first_prev, end_prev);
+            if (ok) ok = mma1(i, newc, li);
+            if (ok && i >= 1 && !newc) ok = mma2(i - 1, first_prev, end_prev);
+            first_prev = newc;
+            end_prev = endc;
+            prev = bk;
+        }
+        if (ok) mma2(n - 1, first_prev, end_prev);
+        umma_commit(&bar->done);
+        mbar_drain(&bar->done, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == NW_P + NW_S + NW_D) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 template <typename T, int S, int D>
 cudaError_t launch_attend_t(const BwdArgs &a, int grid, const void *Q, const void *K, const void *V, const void *dO,
                             float *dQ, float *dK, float *dV, cudaStream_t st) {
@@ -1030,13 +1411,13 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     const int grid = (int)(w.max_tiles < sms ? w.max_tiles : sms);
     const bool bf = p.dtype == HSA_BF16;
     if (w.tc) {
-        const size_t smem = p.S == 64 ? BwdTcShape<64>::smem : BwdTcShape<128>::smem;
+        const size_t smem = p.S == 64 ? BW_SMEM : BwdTcShape<128>::smem;
         if (p.S == 64) {
-            e = cudaFuncSetAttribute(bwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            e = cudaFuncSetAttribute(bwd_tcw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e == cudaSuccess)
-                bwd_tc_kernel<64><<<grid, BT_ROWS, smem, st>>>(a, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
-                                                               (const __nv_bfloat16 *)V, (const __nv_bfloat16 *)dO,
-                                                               dQ, dK, dV);
+                bwd_tcw_kernel<<<grid, NT_W, smem, st>>>(a, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                                                         (const __nv_bfloat16 *)V, (const __nv_bfloat16 *)dO, dQ, dK,
+                                                         dV);
         } else {
             e = cudaFuncSetAttribute(bwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e == cudaSuccess)
