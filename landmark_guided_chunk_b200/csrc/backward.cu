@@ -54,6 +54,7 @@ struct BwdArgs {
     int32_t *bcount;            // [nbucket] pair counts, then scatter cursors
     int32_t *boff;              // [nbucket + 1] first pair of each bucket
     int32_t *pairs;             // [rows * kmax] row * kmax + slot, bucket-major
+    float *pair_w;              // [rows * kmax] fusion weight of each pair, bucket-major
     int4 *tiles;                // (bucket, first pair, pairs, 0)
     int32_t *ntiles;            // number of tiles (written by the scan)
     float *dL;                  // [B][Hkv][C][d] landmark gradients
@@ -185,6 +186,7 @@ __global__ void bwd_scatter_kernel(BwdArgs a) {
         if (c < 0 || c >= nc) continue;
         const int pos = atomicAdd(a.bcount + ((long long)b * a.Hkv + j) * a.C + c, 1);
         a.pairs[pos] = (int)(r * a.kmax + i);
+        a.pair_w[pos] = a.w[r * a.kmax + i];
     }
 }
 
@@ -934,10 +936,11 @@ __global__ void __launch_bounds__(BT_ROWS, 1)
 //   warps 4-7   softmax: P, e, dZ and w P of tile i (thread = TMEM lane = row)
 //   warps 8-11  drain: dQ of every tile through the staging rows, dK^T / dV^T at a run's end
 //   warp 12     one thread issues the MMAs
-// TMEM: Z / GV of tile parity b at [128 b, 128 b + 64) / [128 b + 64, 128 b + 128), dQ [256, 384),
-// dK^T [384, 448), dV^T [448, 512).  So the softmax of tile i+1 runs while the drain of tile i
-// reduces its dQ, and the producers gather tile i+2.  Each barrier has one group of waiters that
-// waits its phases in order, and every wait is bounded.
+// TMEM: Z [0, 64), GV [64, 128), dQ of tile parity b at [128 + 128 b, 256 + 128 b), dK^T
+// [384, 448), dV^T [448, 512).  dQ is double-buffered, so the MMAs of tile i+1 need not wait for
+// the drain of tile i: the softmax of tile i+1 runs while the drain reduces dQ of tile i and the
+// producers gather tile i+2.  Each barrier has one group of waiters that waits its phases in
+// order, and every wait is bounded.
 
 constexpr int NW_P = 4, NW_S = 4, NW_D = 4;
 constexpr int NT_W = 32 * (NW_P + NW_S + NW_D + 1);
@@ -950,7 +953,7 @@ struct BwInfo {
 };
 
 struct BwBars {
-    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, zg_full[2], zg_empty[2], ds_full, ds_empty, dq_full, dq_empty;
+    uint64_t q_full[2], q_empty[2], kv_full, kv_empty, zg_full, zg_empty, ds_full, ds_empty, dq_full[2], dq_empty[2];
     uint64_t info_full[NWI], info_empty[NWI], done;
     uint32_t tmem;
     int abort;
@@ -989,15 +992,15 @@ __global__ void __launch_bounds__(NT_W, 1)
         for (int q = 0; q < 2; ++q) {
             mbar_init(&bar->q_full[q], 32 * NW_P);
             mbar_init(&bar->q_empty[q], 1);
-            mbar_init(&bar->zg_full[q], 1);
-            mbar_init(&bar->zg_empty[q], NW_S);
+            mbar_init(&bar->dq_full[q], 1);
+            mbar_init(&bar->dq_empty[q], NW_D);
         }
+        mbar_init(&bar->zg_full, 1);
+        mbar_init(&bar->zg_empty, NW_S);
         mbar_init(&bar->kv_full, 32 * NW_P);
         mbar_init(&bar->kv_empty, 1);
         mbar_init(&bar->ds_full, NW_S);
         mbar_init(&bar->ds_empty, 1);
-        mbar_init(&bar->dq_full, 1);
-        mbar_init(&bar->dq_empty, NW_D);
         for (int q = 0; q < NWI; ++q) {
             mbar_init(&bar->info_full[q], NW_P);
             mbar_init(&bar->info_empty[q], NW_D);
@@ -1023,9 +1026,11 @@ __global__ void __launch_bounds__(NT_W, 1)
         // ------------------------------------------------------------ producers
         const int pr = threadIdx.x;   // this thread's row of each tile
         int prev = -1, nload = 0;
+        int4 tr_next = a.tiles[lo];
         for (int i = 0; i < n; ++i) {
             const int b = i & 1, si = i % NWI;
-            const int4 tr = a.tiles[lo + i];
+            const int4 tr = tr_next;
+            if (i + 1 < n) tr_next = a.tiles[lo + i + 1];   // read a tile ahead
             if (tr.x != prev) {
                 // K / V of a new chunk run, once the previous run's last MMAs have released them
                 if (nload > 0 && !wait_all(&bar->kv_empty, (nload - 1) & 1)) break;
@@ -1049,9 +1054,9 @@ __global__ void __launch_bounds__(NT_W, 1)
             int e = -1;
             if (pr < tr.z * a.G) {
                 const int pc = a.pairs[tr.y + pr / a.G], g = pr % a.G;
+                w = a.pair_w[tr.y + pr / a.G];
                 const long long bt = (long long)(pc / a.kmax) / a.Hkv;
                 qoff = (bt * a.H + (long long)bucket_pos(a, tr.x).j * a.G + g) * D;
-                w = a.w[pc];
                 e = pc * a.G + g;
             }
             info[si].qoff[pr] = qoff;
@@ -1085,20 +1090,21 @@ __global__ void __launch_bounds__(NT_W, 1)
             if (!wait_all(&bar->info_full[si], (i / NWI) & 1)) break;
             const float w = info[si].w[row];
             const int eslot = info[si].e[row];
-            if (!wait_all(&bar->zg_full[b], (i >> 1) & 1)) break;
+            if (!wait_all(&bar->zg_full, i & 1)) break;
             tc_fence_after();
-            const uint32_t zt = tmem + lane_off + b * 128, gt = zt + 64;
+            const uint32_t zt = tmem + lane_off, gt = zt + 64;
             float p[S];
             float mx = -INFINITY;
-#pragma unroll
-            for (int q = 0; q < S / 32; ++q) {
-                uint32_t v[32];
-                tmem_ld32(zt + q * 32, v);
+            {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(zt, v0);
+                tmem_ld32(zt + 32, v1);
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
-                    p[q * 32 + x] = __uint_as_float(v[x]);
-                    mx = fmaxf(mx, p[q * 32 + x]);
+                    p[x] = __uint_as_float(v0[x]);
+                    p[32 + x] = __uint_as_float(v1[x]);
+                    mx = fmaxf(mx, fmaxf(p[x], p[32 + x]));
                 }
             }
             float l = 0.f;
@@ -1109,15 +1115,17 @@ __global__ void __launch_bounds__(NT_W, 1)
             }
             const float inv = 1.f / l;
             float ev = 0.f;
-#pragma unroll
-            for (int q = 0; q < S / 32; ++q) {
-                uint32_t v[32];
-                tmem_ld32(gt + q * 32, v);
+            {
+                uint32_t v0[32], v1[32];
+                tmem_ld32(gt, v0);
+                tmem_ld32(gt + 32, v1);
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 32; ++x) {
-                    p[q * 32 + x] *= inv;
-                    ev = fmaf(p[q * 32 + x], __uint_as_float(v[x]), ev);
+                    p[x] *= inv;
+                    p[32 + x] *= inv;
+                    ev = fmaf(p[x], __uint_as_float(v0[x]), ev);
+                    ev = fmaf(p[32 + x], __uint_as_float(v1[x]), ev);
                 }
             }
             if (eslot >= 0) a.e[eslot] = ev;
@@ -1151,7 +1159,7 @@ __global__ void __launch_bounds__(NT_W, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bar->zg_empty[b]);
+                mbar_arrive(&bar->zg_empty);
                 mbar_arrive(&bar->ds_full);
             }
         }
@@ -1170,12 +1178,12 @@ __global__ void __launch_bounds__(NT_W, 1)
             for (int rr = 0; rr < 8; ++rr) dst[rr] = info[si].qoff[quad * 32 + rr * 4 + (lane >> 3)];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->info_empty[si]);
-            if (!wait_all(&bar->dq_full, i & 1)) break;
+            if (!wait_all(&bar->dq_full[i & 1], (i >> 1) & 1)) break;
             tc_fence_after();
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_off + 256 + q * 32, v);
+                tmem_ld32(tmem + lane_off + 128 + 128 * (i & 1) + q * 32, v);
                 tmem_wait_ld();
                 float *mine = wst + lane * BT_PITCH;
 #pragma unroll
@@ -1215,7 +1223,7 @@ __global__ void __launch_bounds__(NT_W, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->dq_empty);
+            if (lane == 0) mbar_arrive(&bar->dq_empty[i & 1]);
         }
     } else if (lane == 0) {
         // ------------------------------------------------------------ MMA issuer
@@ -1227,27 +1235,28 @@ __global__ void __launch_bounds__(NT_W, 1)
             const int b = i & 1;
             if (!mbar_wait(&bar->q_full[b], (i >> 1) & 1, abort, a.status)) return false;
             if (newc && !mbar_wait(&bar->kv_full, li & 1, abort, a.status)) return false;
-            if (i >= 2 && !mbar_wait(&bar->zg_empty[b], ((i >> 1) - 1) & 1, abort, a.status)) return false;
+            if (i >= 1 && !mbar_wait(&bar->zg_empty, (i - 1) & 1, abort, a.status)) return false;
             tc_fence_after();
             const uint32_t qa = smem_u32(sQ + b * 32768), ga = smem_u32(sG + b * 32768);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32, bo = (kk >> 2) * KVB + (kk & 3) * 32;
-                umma_bf16(tmem + b * 128, desc_kmajor_sw128(qa + ao), desc_kmajor_sw128(kb + bo), idesc_zg, kk != 0);
-                umma_bf16(tmem + b * 128 + 64, desc_kmajor_sw128(ga + ao), desc_kmajor_sw128(vb + bo), idesc_zg, kk != 0);
+                umma_bf16(tmem, desc_kmajor_sw128(qa + ao), desc_kmajor_sw128(kb + bo), idesc_zg, kk != 0);
+                umma_bf16(tmem + 64, desc_kmajor_sw128(ga + ao), desc_kmajor_sw128(vb + bo), idesc_zg, kk != 0);
             }
-            umma_commit(&bar->zg_full[b]);
+            umma_commit(&bar->zg_full);
             return true;
         };
         auto mma2 = [&](int i, bool first, bool endc) -> bool {
+            const int b = i & 1;
             if (!mbar_wait(&bar->ds_full, i & 1, abort, a.status)) return false;
-            if (i >= 1 && !mbar_wait(&bar->dq_empty, (i - 1) & 1, abort, a.status)) return false;
+            if (i >= 2 && !mbar_wait(&bar->dq_empty[b], ((i >> 1) - 1) & 1, abort, a.status)) return false;
             tc_fence_after();
-            const uint32_t qa = smem_u32(sQ + (i & 1) * 32768), ga = smem_u32(sG + (i & 1) * 32768);
+            const uint32_t qa = smem_u32(sQ + b * 32768), ga = smem_u32(sG + b * 32768);
 #pragma unroll
             for (int kk = 0; kk < S / 16; ++kk)
-                umma_bf16(tmem + 256, desc_kmajor_sw128(za + (kk & 3) * 32), desc_mnmajor_sw128(kb + kk * 2048, KVB, 1024),
-                          idesc_dq, kk != 0);
+                umma_bf16(tmem + 128 + 128 * b, desc_kmajor_sw128(za + (kk & 3) * 32),
+                          desc_mnmajor_sw128(kb + kk * 2048, KVB, 1024), idesc_dq, kk != 0);
 #pragma unroll
             for (int kk = 0; kk < BT_ROWS / 16; ++kk) {
                 const uint32_t acc = (kk != 0 || !first) ? 1u : 0u;
@@ -1256,17 +1265,18 @@ __global__ void __launch_bounds__(NT_W, 1)
                 umma_bf16(tmem + 448, desc_mnmajor_sw128(ga + kk * 2048, 16384, 1024),
                           desc_mnmajor_sw128(pa + kk * 2048, 16384, 1024), idesc_kv, acc);
             }
-            umma_commit(&bar->dq_full);
+            umma_commit(&bar->dq_full[b]);
             umma_commit(&bar->ds_empty);
-            umma_commit(&bar->q_empty[i & 1]);
+            umma_commit(&bar->q_empty[b]);
             if (endc) umma_commit(&bar->kv_empty);
             return true;
         };
         bool ok = true, first_prev = false, end_prev = false;
-        int prev = -1, li = -1, bk_next = bucket_at(0);
+        int prev = -1, li = -1, bk_next = bucket_at(0), bk_next2 = bucket_at(1);
         for (int i = 0; i < n && ok; ++i) {
             const int bk = bk_next;
-            bk_next = bucket_at(i + 1);
+            bk_next = bk_next2;
+            bk_next2 = bucket_at(i + 2);   // read two tiles ahead
             const bool newc = bk != prev, endc = bk_next != bk;
             if (newc) ++li;
             // at a run boundary the previous tile's MMAs release K / V before the new run's land
@@ -1348,6 +1358,7 @@ BwdLayout backward_layout(const Prob &p) {
     w.e = take(pairs * p.G * sizeof(float));
     w.boff = take(((size_t)w.nbucket + 1) * sizeof(int32_t));
     w.pairs = take(pairs * sizeof(int32_t));
+    w.pair_w = take(pairs * sizeof(float));
     w.tiles = take((size_t)w.max_tiles * sizeof(int4));
     w.total = off;
     return w;
@@ -1397,6 +1408,7 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     a.bcount = reinterpret_cast<int32_t *>(ws + w.bcount);
     a.boff = reinterpret_cast<int32_t *>(ws + w.boff);
     a.pairs = reinterpret_cast<int32_t *>(ws + w.pairs);
+    a.pair_w = reinterpret_cast<float *>(ws + w.pair_w);
     a.tiles = reinterpret_cast<int4 *>(ws + w.tiles);
     a.ntiles = reinterpret_cast<int32_t *>(ws + w.hdr + 16);
     a.dL = reinterpret_cast<float *>(ws + w.dL);

@@ -297,7 +297,7 @@ cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *
 
 // Backward (backward.cu): workspace layout, support check, kernel count, launch.
 struct BwdLayout {
-    size_t hdr, bcount, dL, clear_bytes, w, e, boff, pairs, tiles, total;
+    size_t hdr, bcount, dL, clear_bytes, w, e, boff, pairs, pair_w, tiles, total;
     long long nbucket, max_tiles;
     int pt;    // pairs per tile
     bool tc;   // tensor-core attention backward (bf16, d 128, S 64 / 128)
