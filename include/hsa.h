@@ -258,6 +258,11 @@ HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const vo
  * header is the status word).  The adds into dQ, dK, dV and dW_L are fp32
  * atomic reductions, so their order, and the last bits of the result, vary
  * from call to call.
+ * Paths: bf16 with d = 128 and S = 64 or 128 uses the tcgen05 tensor cores,
+ * with dZ (the in-chunk softmax gradient) and w P rounded to bf16 before the
+ * dQ, dK and dV products; fp32, d = 64, S = 32, or HSA_FLAG_SIMT in p->flags
+ * use fp32 CUDA-core arithmetic throughout.  Six kernel launches (plus the
+ * zeroing of the outputs), all on `stream`.
  */
 HSA_API hsa_status_t hsa_backward_workspace_size(const hsa_problem_t *p, size_t *bytes);
 HSA_API hsa_status_t hsa_backward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,

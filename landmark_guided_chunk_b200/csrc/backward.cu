@@ -20,18 +20,21 @@
 //   scan     one CTA: exclusive scans of the bucket counts (pairs) and of
 //            their tile counts, the tile list, the scatter cursors;
 //   scatter  one thread per selection row: its (row, slot) pairs -> buckets;
-//   attend   chunk-major, one CTA per SM over a contiguous range of tiles.  A
-//            tile holds up to RT query-head rows that kept one chunk.  K_c and
-//            V_c are staged once per bucket run; the CTA keeps dK_c and dV_c in
-//            registers until the bucket changes and then adds them to memory
-//            with vector reductions.  Per tile: Z = q K^T, GV = dO V^T (one
-//            pass over d), row softmax and e in one warp per row, then dQ =
-//            dZ K and the dK/dV updates.  e goes to the workspace.
+//   attend   chunk-major, one CTA per SM over a contiguous range of tiles of
+//            query-head rows that kept one chunk; K_c and V_c are staged once
+//            per bucket run and dK_c, dV_c stay on chip until the bucket
+//            changes.  Per tile: Z = q K^T, GV = dO V^T, the row softmax and
+//            e, then dQ = dZ K and the dK/dV updates; e goes to the
+//            workspace.  bf16 with d = 128 runs on tcgen05 (bwd_tcw_kernel
+//            for S = 64, bwd_tc_kernel for S = 128); everything else, and any
+//            problem with HSA_FLAG_SIMT, on CUDA cores (bwd_attend_kernel).
 //   fuse     one warp per selection row: dw, ds, the score path into dQ and dL;
 //   landmark one pass over all complete chunks: chunk means, dW_L partials per
 //            CTA, and dL W_L^T / S added to the chunk's key gradients.
-// All arithmetic is fp32 on CUDA cores (the gradients are fp32 buffers); the
-// stored inputs (fp32 or bf16) are read exactly.
+// Accumulation is fp32 everywhere and the gradients are fp32 buffers; the
+// stored inputs (fp32 or bf16) are read exactly.  The tensor-core kernels
+// round dZ and w P to bf16 before the dQ, dK and dV products, as the forward
+// rounds P; the CUDA-core kernel rounds nothing.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -583,7 +586,8 @@ __global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T 
 
 // ---------------------------------------------------------------------------- tensor-core attention backward
 //
-// bf16, d = 128, S = 64 or 128.  One CTA of 128 threads per SM; thread r is
+// bf16, d = 128, used for S = 128 (S = 64 runs the warp-specialized bwd_tcw_kernel below, which
+// needs TMEM columns this one spends on S = 128).  One CTA of 128 threads per SM; thread r is
 // tile row r and TMEM lane r.  A tile is up to 128 query-head rows that kept
 // one chunk (128 / G pairs).  Per tile, issued by thread 0 on tcgen05 with
 // fp32 accumulators in TMEM:
@@ -600,8 +604,8 @@ __global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T 
 // (over Z and GV, which are read before dQ is issued), dK^T [2S, 3S), dV^T
 // [3S, 4S).  Shared tiles use the 128-byte swizzle of the forward kernel
 // (rows of 64 bf16, 8-row groups 1024 B apart, 16-byte chunk c of row r at
-// c ^ (r & 7)); Q and dO are double-buffered for S = 64 so the next tile's
-// gather overlaps this tile's MMAs.
+// c ^ (r & 7)).  With one Q / dO buffer (S = 128) the next tile is gathered
+// after this tile's MMAs have read its rows.
 
 constexpr int BT_ROWS = 128;
 constexpr int BT_PITCH = 36;   // dQ staging pitch (floats)
