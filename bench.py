@@ -347,8 +347,11 @@ def run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, wo
     out = (torch.empty(Q.shape, **f32), torch.empty(K.shape, **f32), torch.empty(K.shape, **f32),
            torch.empty(p.d, p.d, **f32))
 
+    from landmark_guided_chunk_b200 import dp
+
     def step():
-        hsa.backward(Q, K, V, W, L, idx, score, keff, dO, p.S, p.k, p.tau, q_pos0=p.q_pos0, out=out, ws=ws)
+        # each rank differentiates its own sequence; W_L's gradient is summed over the ranks
+        dp.backward_dp(Q, K, V, W, L, idx, score, keff, dO, p.S, p.k, p.tau, q_pos0=p.q_pos0, out=out, ws=ws)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -376,6 +379,7 @@ def run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, wo
              "peak_source": "fp32 FMA lanes x clocks.max.sm (CUDA-core path)"})
     return {"ms": round(ms, 3), "steps": nsteps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
             "kernels": 6, "path": "tensor" if tc else "simt",
+            "exchange": "all-reduce (sum) of dW_L, d x d fp32, over the ranks" if world > 1 else "none (one rank)",
             "dtype": "bf16 operands, fp32 accumulation" if tc else "f32", "roofline": roof}
 
 

@@ -2,6 +2,10 @@
 
 * bench.py's rank helpers: the reported time is the maximum over ranks, and
   every rank takes the same barrier.
+* The data-parallel backward's exchange (landmark_guided_chunk_b200.dp): each
+  rank differentiates its own sequence (the oracle's backward stands in for the
+  kernels), and after allreduce_param_grads every rank holds the W_L gradient of
+  the whole batch -- the oracle's backward over both sequences at once.
 * Context-sharded decode (landmark_guided_chunk_b200.sharded), the method
   itself: each rank holds a contiguous range of a sequence's chunks, keeps its
   local top kmax with the router off (its candidates counted from
@@ -146,3 +150,46 @@ def test_sharded_decode_method_two_ranks():
 
 def test_sharded_decode_method_two_ranks_router():
     mp.spawn(_sharded_method, args=(_free_port(), 3, 0.3), nprocs=WORLD, join=True)
+
+
+def _dp_problem():
+    rng = np.random.default_rng(91)
+    B, T, H, Hkv, d, S = WORLD, 32 * 6 + 9, 4, 2, 16, 32
+    Q = torch.tensor(rng.standard_normal((B, T, H, d)))
+    K = torch.tensor(rng.standard_normal((B, T, Hkv, d)))
+    V = torch.tensor(rng.standard_normal((B, T, Hkv, d)))
+    W = torch.tensor(rng.standard_normal((d, d)) / d ** 0.5)
+    dO = rng.standard_normal((B, T, H, d))
+    return Q, K, V, W, dO, S
+
+
+def _oracle_backward(Q, K, V, W, dO, S, k):
+    B, T = Q.shape[:2]
+    rb, rp = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+    Qr = Q.reshape(B * T, *Q.shape[2:])
+    L = oracle.landmarks(K, W, S)
+    sel = oracle.select(Qr, rb, rp, L, S, k, 0.0, Q.shape[2])
+    return oracle.backward(Qr, rb, K, V, W, L, S, sel, dO.reshape(B * T, *dO.shape[2:]))
+
+
+def _dp_backward(rank, port):
+    _init(rank, port)
+    try:
+        from landmark_guided_chunk_b200 import dp
+        Q, K, V, W, dO, S = _dp_problem()
+        mine = _oracle_backward(Q[rank:rank + 1], K[rank:rank + 1], V[rank:rank + 1], W, dO[rank:rank + 1], S, 3)
+        dW = torch.tensor(mine["dW"])
+        dp.allreduce_param_grads(dW)
+        whole = _oracle_backward(Q, K, V, W, dO, S, 3)
+        assert np.allclose(dW.numpy(), whole["dW"], atol=1e-12, rtol=0)
+        # the per-sequence gradients need no exchange: this rank's rows of the whole batch
+        T = Q.shape[1]
+        assert np.allclose(mine["dQ"], whole["dQ"][rank * T:(rank + 1) * T], atol=1e-12)
+        assert np.allclose(mine["dK"][0], whole["dK"][rank], atol=1e-12)
+        assert np.allclose(mine["dV"][0], whole["dV"][rank], atol=1e-12)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_backward_exchange_two_ranks():
+    mp.spawn(_dp_backward, args=(_free_port(),), nprocs=WORLD, join=True)
