@@ -115,6 +115,14 @@ CASES = {
                                   dtype="bf16"), 64 * 9 + 20, False),
     "bf16_decode_rows": (Problem(B=3, Tq=1, Tkv=64 * 50 + 9, H=8, Hkv=2, d=128, S=64, k=8, q_pos0=64 * 50 + 9,
                                  dtype="bf16"), None, False),
+    # the CUDA-core kernel's other shapes: fp32 at S = 128, d = 128; bf16 at S = 32 (no tensor-core
+    # path) and at S = 128, d = 128 forced onto the CUDA cores
+    "f32_S128_d128": (Problem(B=1, Tq=128 * 5 + 17, Tkv=128 * 5 + 17, H=4, Hkv=2, d=128, S=128, k=2, dtype="f32"),
+                      None, False),
+    "bf16_S32_d128": (Problem(B=1, Tq=32 * 20 + 7, Tkv=32 * 20 + 7, H=8, Hkv=2, d=128, S=32, k=4, dtype="bf16"),
+                      None, False),
+    "bf16_S128_d128_simt": (Problem(B=1, Tq=128 * 6 + 3, Tkv=128 * 6 + 3, H=4, Hkv=2, d=128, S=128, k=3,
+                                    dtype="bf16"), None, True),
     # G = 16 over 73 chunks: tiles of 8 pairs, many tiles per chunk
     "bf16_G16_long": (Problem(B=1, Tq=4096 + 600, Tkv=4096 + 600, H=32, Hkv=2, d=128, S=64, k=2, dtype="bf16"),
                       None, False),
@@ -137,6 +145,26 @@ def test_backward_without_candidates_is_zero():
     r = _run(p, seed=3)
     for name in ("dQ", "dK", "dV", "dW"):
         assert torch.all(r[name] == 0), name
+
+
+def test_backward_empty_batch():
+    """B = 0: nothing to differentiate; dW_L (always allocated) comes back zeroed."""
+    p = Problem(B=0, Tq=70, Tkv=70, H=4, Hkv=2, d=64, S=32, k=2, dtype="bf16")
+    dt = torch.bfloat16
+    Q = torch.empty(0, 70, 4, 64, dtype=dt, device="cuda")
+    K = torch.empty(0, 70, 2, 64, dtype=dt, device="cuda")
+    V = torch.empty_like(K)
+    W = torch.randn(64, 64, device="cuda").to(dt)
+    L = torch.empty(0, 2, 2, 64, dtype=dt, device="cuda")
+    idx = torch.empty(0, 70, 2, 2, dtype=torch.int32, device="cuda")
+    sc = torch.empty(0, 70, 2, 2, dtype=torch.float32, device="cuda")
+    ke = torch.empty(0, 70, 2, dtype=torch.int32, device="cuda")
+    dW = torch.full((64, 64), 7.0, device="cuda")
+    out = (torch.empty(0, 70, 4, 64, device="cuda"), torch.empty(0, 70, 2, 64, device="cuda"),
+           torch.empty(0, 70, 2, 64, device="cuda"), dW)
+    hsa.backward(Q, K, V, W, L, idx, sc, ke, torch.empty_like(Q), p.S, p.k, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(dW == 0)
 
 
 def test_backward_prefill_full_size_sampled_rows():
