@@ -31,22 +31,25 @@ _F32, _BF16, _F64 = 0, 1, 2
 _lib = None
 
 
+def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the argument types of the oracle's C entry points on a loaded library."""
+    P, I, LL, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_double
+    lib.hsa_oracle_round.argtypes = [I, P, LL, P]
+    lib.hsa_oracle_landmarks.argtypes = [I, I, LL, I, I, I, P, P, P]
+    lib.hsa_oracle_select.argtypes = [I, I, I, I, I, LL, I, D, I, LL, P, P, P, P, P, P, P, P]
+    lib.hsa_oracle_attend.argtypes = [I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P]
+    lib.hsa_oracle_backward.argtypes = [I, I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P, P,
+                                        P, P, P, P, P]
+    for f in (lib.hsa_oracle_round, lib.hsa_oracle_landmarks, lib.hsa_oracle_select,
+              lib.hsa_oracle_attend, lib.hsa_oracle_backward):
+        f.restype = None
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        P, I, LL, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_double
-        lib.hsa_oracle_round.argtypes = [I, P, LL, P]
-        lib.hsa_oracle_landmarks.argtypes = [I, I, LL, I, I, I, P, P, P]
-        lib.hsa_oracle_select.argtypes = [I, I, I, I, I, LL, I, D, I, LL, P, P, P, P, P, P, P, P]
-        lib.hsa_oracle_attend.argtypes = [I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P]
-        lib.hsa_oracle_backward.argtypes = [I, I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P, P,
-                                            P, P, P, P, P]
-        for f in (lib.hsa_oracle_round, lib.hsa_oracle_landmarks, lib.hsa_oracle_select,
-                  lib.hsa_oracle_attend, lib.hsa_oracle_backward):
-            f.restype = None
-        _lib = lib
+        _lib = _bind(ctypes.CDLL(_build.build()))
     return _lib
 
 
