@@ -5,7 +5,8 @@ in a temporary directory), builds it, binds it in place of the real oracle
 library, and runs the pin tests that should notice: at least one of them must
 fail.  The mistakes are the ones an implementation of the method could make:
 a wrong chunk mean, W_L applied transposed, the query's own chunk among its
-candidates, ties broken the wrong way, the router's comparison reversed,
+candidates, a group score from one head, bf16 rounding with ties away from
+zero, ties between chunks broken the wrong way, the router's comparison reversed,
 uniform fusion weights, the in-chunk softmax without its 1/sqrt(d), and in
 the backward a dropped softmax term, a missing landmark share, a missing e
 term and a sign error.
@@ -36,6 +37,14 @@ MUTANTS = {
         "long long ncand = row_p[r] / S + 1;",
         [pins.test_decode_position_sees_all_complete_chunks,
          lambda: pins.test_select_matches_exact_integer_brute_force(0.0)]),
+    "group score from one head": (
+        "                for (int h = j * G; h < (j + 1) * G; ++h) {\n                    double dot = 0.0;",
+        "                for (int h = j * G; h < j * G + 1; ++h) {\n                    double dot = 0.0;",
+        [pins.test_select_group_sum_decides]),
+    "bf16 rounding ties away from zero": (
+        "double r = nearbyint(x / ulp) * ulp;",
+        "double r = round(x / ulp) * ulp;",
+        [pins.test_round_bf16_ties_to_even]),
     "ties to the higher chunk": (
         "return (x->c > y->c) - (x->c < y->c);",
         "return (x->c < y->c) - (x->c > y->c);",
