@@ -9,9 +9,10 @@ asynchronous completions are the producers' cp.async arrivals, the TMA loads
 and the tcgen05 commits.  This model replays each role with the kernel's phase
 formulas for both stage configurations (S = 64: nsq = nskv = 2; S = 128: one
 each), under random interleavings and completion delays, over random tile
-sequences, and checks that every role finishes, that no waiter tests a
-barrier two phases past the one it waits for (a parity-only wait would
-misread it), and the one hand-off with no barrier: QK of tile i overwrites
+sequences, and checks that every role finishes, that every waiter tests its
+barrier only while it has completed the awaited phase or the one before (a
+parity-only wait misreads anything else), and the one hand-off with no
+barrier: QK of tile i overwrites
 the S buffer of tile i-2, so the softmax must have read that tile by then
 (it has, through p_full, before PV(i-2) is issued).  A change to the
 kernel's barriers, counts or phase arithmetic has to be mirrored here.
@@ -153,7 +154,8 @@ def run(tiles, nsq, nskv, seed):
         if waiting[r] is None:
             return True
         bar, ph = waiting[r]
-        assert bar.phase <= ph + 1, f"{bar.name}: waiter for phase {ph} sees phase {bar.phase} (parity alias)"
+        # a parity wait is right only while the barrier has completed ph or ph + 1 phases
+        assert ph <= bar.phase <= ph + 1, f"{bar.name}: waiter for phase {ph} sees phase {bar.phase} (parity alias)"
         return bar.phase > ph
 
     steps = 0

@@ -9,9 +9,10 @@ order, once the MMAs before them are done).  This model replays every role's
 loop with the kernel's phase formulas, under random interleavings and random
 completion delays, over random sequences of chunk runs, and checks that:
   * every role finishes (no wait that can never be satisfied), and
-  * no waiter tests a barrier that has already completed two phases past the
-    one it waits for (an mbarrier wait compares parity only, so that would be
-    misread as an open phase).
+  * every waiter tests its barrier only while the barrier has completed the
+    phase it waits for or the one before (an mbarrier wait compares parity
+    only: two phases further on reads as open, one phase short reads the
+    previous phase as this one).
 A change to the kernel's barriers, counts or phase arithmetic has to be
 mirrored here.
 """
@@ -134,7 +135,8 @@ def run(buckets, seed):
         if waiting[r] is None:
             return True
         bar, ph = waiting[r]
-        assert bar.phase <= ph + 1, f"{bar.name}: waiter for phase {ph} sees phase {bar.phase} (parity alias)"
+        # a parity wait is right only while the barrier has completed ph or ph + 1 phases
+        assert ph <= bar.phase <= ph + 1, f"{bar.name}: waiter for phase {ph} sees phase {bar.phase} (parity alias)"
         return bar.phase > ph
 
     steps = 0
