@@ -159,66 +159,140 @@ def work_counts(p, keff_sum: int) -> dict:
 
 # --------------------------------------------------------------------------- our arm
 
+class PrefillSetup:
+    """Inputs, outputs and the three stage calls (landmarks, select, attend) of
+    one prefill workload, each a direct call of the C ABI on one stream."""
+
+    def __init__(self, name, seed, dev):
+        import landmark_guided_chunk_b200 as hsa
+        from landmark_guided_chunk_b200.inputs import make_inputs, workload
+
+        self.hsa = hsa
+        self.dev = dev
+        self.p = p = workload(name)
+        self.inp = make_inputs(p, seed=seed, device=dev)
+        self.Q, self.K, self.V, self.W = (self.inp[x] for x in ("Q", "K", "V", "W_L"))
+        self.prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau,
+                                     torch.bfloat16 if p.dtype == "bf16" else torch.float32)
+        self.plan = hsa.plan(self.prob)
+        self.ws = hsa.alloc_workspace(self.prob, dev)
+        self.L = torch.empty(p.B, p.Hkv, p.C, p.d, dtype=self.Q.dtype, device=dev)
+        self.O = torch.empty_like(self.Q)
+        km = hsa.kmax_of(p.k, p.tau)
+        self.idx = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.int32, device=dev)
+        self.score = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.float32, device=dev)
+        self.keff = torch.empty(p.B, p.Tq, p.Hkv, dtype=torch.int32, device=dev)
+        self.st = torch.cuda.current_stream(dev)
+        lib, P, sp, prob = hsa._native.lib(), hsa._p, self.st.cuda_stream, self.prob
+        Q, K, V, W, L, O = self.Q, self.K, self.V, self.W, self.L, self.O
+        idx, score, keff, ws = self.idx, self.score, self.keff, self.ws
+
+        def stage_landmarks():
+            hsa._native.check(lib.hsa_landmarks(ctypes.byref(prob), P(K), P(W), P(L), sp), "hsa_landmarks")
+
+        def stage_select():
+            hsa._native.check(lib.hsa_select(ctypes.byref(prob), P(Q), P(L), P(idx), P(score), P(keff), P(ws),
+                                             ws.numel(), sp), "hsa_select")
+
+        def stage_attend():
+            hsa._native.check(lib.hsa_attend(ctypes.byref(prob), P(Q), P(K), P(V), P(idx), P(score), P(keff),
+                                             P(O), P(ws), ws.numel(), sp), "hsa_attend")
+
+        self.stages = [("landmarks", stage_landmarks), ("select", stage_select), ("attend", stage_attend)]
+
+    def time_stages(self, steps, warmup, world, clocks=None):
+        """Warm-up, then `steps` forwards back to back, each stage bracketed by
+        CUDA events on the launching stream.  Returns (ms per forward, max over
+        ranks; mean ms of each stage; keff sum; clock record)."""
+        for _ in range(warmup):
+            for _, f in self.stages:
+                f()
+        torch.cuda.synchronize(self.dev)
+        keff_sum = int(self.keff.sum().item())
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize(self.dev)
+        if clocks is not None:
+            clocks.start()
+        for s in range(steps):
+            ev[s][0].record(self.st)
+            for i, (_, f) in enumerate(self.stages):
+                f()
+                ev[s][i + 1].record(self.st)
+        torch.cuda.synchronize(self.dev)
+        clk = clocks.stop() if clocks is not None else None
+        barrier(world)
+        total_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
+        stage_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps
+                    for i, (name, _) in enumerate(self.stages)}
+        return max_over_ranks(total_ms / steps, world), stage_ms, keff_sum, clk
+
+    def roofline(self, stage_ms, keff_sum, pk):
+        """Each stage's achieved rate against the measured peaks, and the
+        dominant stage's roofline object.  The stages are timed inside a
+        forward of a few ms, so the burst bf16 peak applies; the fraction of
+        the sustained peak is given beside it."""
+        p, work = self.p, work_counts(self.p, keff_sum)
+        stage_rf = {
+            "landmarks": {"bound": "hbm", "work": work["landmarks_bytes"], "unit": "GB/s", "peak": pk["hbm_gbs"]},
+            "select": {"bound": "tensor", "work": work["select_flops"], "unit": "TFLOP/s", "peak": pk["bf16_tflops"]},
+            "attend": {"bound": "tensor", "work": work["attend_flops"], "unit": "TFLOP/s", "peak": pk["bf16_tflops"]},
+        }
+        stages_out = {}
+        for name, rf in stage_rf.items():
+            ms = stage_ms[name]
+            scale = 1e-9 if rf["unit"] == "GB/s" else 1e-12
+            ach = rf["work"] * scale / (ms * 1e-3)
+            stages_out[name] = {"ms": round(ms, 4), "path": self.plan[name][0], "kernels": self.plan[name][1],
+                                "achieved": round(ach, 2), "unit": rf["unit"], "bound": rf["bound"],
+                                "frac": round(ach / rf["peak"], 4)}
+            if rf["unit"] == "TFLOP/s":
+                stages_out[name]["frac_of_sustained"] = round(ach / pk["bf16_tflops_sustained"], 4)
+        dom = max(stage_ms, key=stage_ms.get)
+        traffic = dram_traffic(f"{dom}:{p.name}", self.plan[dom][0])
+        roof = {"bound": stage_rf[dom]["bound"], "kernel": f"hsa_{dom} ({self.plan[dom][0]})",
+                "achieved": stages_out[dom]["achieved"], "peak": stage_rf[dom]["peak"],
+                "unit": stage_rf[dom]["unit"], "frac": stages_out[dom]["frac"], "traffic": traffic,
+                "peak_source": f"{pk['source']} ({'burst bf16' if stage_rf[dom]['unit'] == 'TFLOP/s' else 'HBM copy'})"}
+        return stages_out, roof
+
+
+def run_router(args, world, rank, local, pk):
+    """The gap-router prefill workload (router_bf16: B1, T 131072, S 128, k 8
+    doubled to 16 where the normalised top-k gap is below tau = 0.02): forward
+    time per stage, tokens/s, the mean k_eff and the measured fraction of
+    selection rows the router doubled."""
+    dev = torch.device("cuda", local)
+    ps = PrefillSetup("router_bf16", args.seed + rank, dev)
+    p = ps.p
+    steps = max(1, min(args.steps, 10))
+    ms, stage_ms, keff_sum, _ = ps.time_stages(steps, args.warmup, world)
+    stages_out, roof = ps.roofline(stage_ms, keff_sum, pk)
+    nc = torch.as_tensor(ncand_rows(p), device=dev).view(1, -1, 1)
+    eligible = (nc > p.k).expand_as(ps.keff)
+    doubled = (ps.keff > p.k) & eligible
+    frac = float(doubled.sum().item()) / max(1, int(eligible.sum().item()))
+    out = {"workload": f"{p.name}: B{p.B} T{p.Tq} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}->{2 * p.k} tau{p.tau}",
+           "ms_per_forward": round(ms, 4), "steps": steps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
+           "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3), "doubled_fraction": round(frac, 4),
+           "stages": stages_out, "roofline": roof,
+           "gpu_launches": steps * sum(ps.plan[x][1] for x in ("landmarks", "select", "attend"))}
+    del ps
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_b200(args, world, rank, local):
     import landmark_guided_chunk_b200 as hsa
-    from landmark_guided_chunk_b200.inputs import make_inputs, workload
 
     dev = torch.device("cuda", local)
     pk = peaks()
-    p = workload(args.workload)
-    inp = make_inputs(p, seed=args.seed + rank, device=dev)
-    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
-    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau,
-                            torch.bfloat16 if p.dtype == "bf16" else torch.float32)
-    plan = hsa.plan(prob)
-    ws = hsa.alloc_workspace(prob, dev)
-    L = torch.empty(p.B, p.Hkv, p.C, p.d, dtype=Q.dtype, device=dev)
-    O = torch.empty_like(Q)
-    km = hsa.kmax_of(p.k, p.tau)
-    idx = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.int32, device=dev)
-    score = torch.empty(p.B, p.Tq, p.Hkv, km, dtype=torch.float32, device=dev)
-    keff = torch.empty(p.B, p.Tq, p.Hkv, dtype=torch.int32, device=dev)
-    lib = hsa._native.lib()
-    P = hsa._p
-    st = torch.cuda.current_stream(dev)
-    sp = st.cuda_stream
-
-    def stage_landmarks():
-        hsa._native.check(lib.hsa_landmarks(ctypes.byref(prob), P(K), P(W), P(L), sp), "hsa_landmarks")
-
-    def stage_select():
-        hsa._native.check(lib.hsa_select(ctypes.byref(prob), P(Q), P(L), P(idx), P(score), P(keff), P(ws),
-                                         ws.numel(), sp), "hsa_select")
-
-    def stage_attend():
-        hsa._native.check(lib.hsa_attend(ctypes.byref(prob), P(Q), P(K), P(V), P(idx), P(score), P(keff),
-                                         P(O), P(ws), ws.numel(), sp), "hsa_attend")
-
-    stages = [("landmarks", stage_landmarks), ("select", stage_select), ("attend", stage_attend)]
-    for _ in range(args.warmup):
-        for _, f in stages:
-            f()
-    torch.cuda.synchronize(dev)
-    keff_sum = int(keff.sum().item())
-    work = work_counts(p, keff_sum)
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ps = PrefillSetup(args.workload, args.seed + rank, dev)
+    p, prob, plan, ws = ps.p, ps.prob, ps.plan, ps.ws
+    Q, K, V, W, L, O = ps.Q, ps.K, ps.V, ps.W, ps.L, ps.O
+    idx, score, keff, st = ps.idx, ps.score, ps.keff, ps.st
     clocks = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    for s in range(args.steps):
-        ev[s][0].record(st)
-        for i, (_, f) in enumerate(stages):
-            f()
-            ev[s][i + 1].record(st)
-    torch.cuda.synchronize(dev)
-    clk = clocks.stop()
-    barrier(world)
-    total_ms = sum(e[0].elapsed_time(e[3]) for e in ev)
-    stage_ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / args.steps
-                for i, (name, _) in enumerate(stages)}
-    ms_step = max_over_ranks(total_ms / args.steps, world)
+    ms_step, stage_ms, keff_sum, clk = ps.time_stages(args.steps, args.warmup, world, clocks)
     tokens_all = p.B * p.Tq * world
     value = tokens_all / (ms_step * 1e-3)
 
@@ -280,28 +354,7 @@ def run_b200(args, world, rank, local):
     d2h = Oh.numel() * Oh.element_size()
     del Qh, Kh, Vh, Wh, Oh, dev_in, dev_out
 
-    # roofline of each stage and of the dominant one
-    stage_rf = {
-        "landmarks": {"bound": "hbm", "work": work["landmarks_bytes"], "unit": "GB/s", "peak": pk["hbm_gbs"]},
-        "select": {"bound": "tensor", "work": work["select_flops"], "unit": "TFLOP/s",
-                   "peak": pk["bf16_tflops_sustained"]},
-        "attend": {"bound": "tensor", "work": work["attend_flops"], "unit": "TFLOP/s",
-                   "peak": pk["bf16_tflops_sustained"]},
-    }
-    stages_out = {}
-    for name, rf in stage_rf.items():
-        ms = stage_ms[name]
-        scale = 1e-9 if rf["unit"] == "GB/s" else 1e-12
-        ach = rf["work"] * scale / (ms * 1e-3)
-        stages_out[name] = {"ms": round(ms, 4), "path": plan[name][0], "kernels": plan[name][1],
-                            "achieved": round(ach, 2), "unit": rf["unit"], "bound": rf["bound"],
-                            "frac": round(ach / rf["peak"], 4)}
-    dom = max(stage_ms, key=stage_ms.get)
-    traffic = dram_traffic(dom, plan[dom][0])
-    roof = {"bound": stage_rf[dom]["bound"], "kernel": f"hsa_{dom} ({plan[dom][0]})",
-            "achieved": stages_out[dom]["achieved"], "peak": stage_rf[dom]["peak"], "unit": stage_rf[dom]["unit"],
-            "frac": stages_out[dom]["frac"], "traffic": traffic,
-            "peak_source": f"{pk['source']} ({'sustained bf16' if stage_rf[dom]['unit'] == 'TFLOP/s' else 'HBM copy'})"}
+    stages_out, roof = ps.roofline(stage_ms, keff_sum, pk)
     launches = args.steps * (plan["landmarks"][1] + plan["select"][1] + plan["attend"][1])
 
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -318,8 +371,10 @@ def run_b200(args, world, rank, local):
            "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3)}
     if not args.no_backward:
         out["backward"] = run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, world)
-    del inp, Q, K, V, W, L, O, idx, score, keff, ws
+    del ps, Q, K, V, W, L, O, idx, score, keff, ws
     torch.cuda.empty_cache()
+    if not args.no_router and args.workload == "prefill_bf16":
+        out["router_bf16"] = run_router(args, world, rank, local, pk)
     if not args.no_decode:
         out["decode_1m"] = run_decode(args, world, rank, local, pk)
         if not args.no_decode_16m:
@@ -696,19 +751,109 @@ def run_reference(args, world, rank):
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+
+# --------------------------------------------------------------------------- single-case driver for profilers
+
+def run_case(args):
+    """One workload (optionally resized) run --iters times through the public
+    API, for profiler captures of a small, reproducible case:
+      --T N         prefill length (Tq = Tkv = N)
+      --ctx N       decode context length
+      --B N         batch
+      --select-only selection stage alone on the workload's query shapes and
+                    random landmarks, no K/V allocated
+      --backward    one forward (with its selection), then the backward --iters times
+      --simt        CUDA-core kernels only (HSA_FLAG_SIMT)
+    Prints the kernel path of each stage and the wall time of the last iteration."""
+    import landmark_guided_chunk_b200 as hsa
+    from landmark_guided_chunk_b200.inputs import make_inputs, make_output_grad, workload
+
+    p = workload(args.workload)
+    if args.B is not None:
+        p = p.with_(B=args.B)
+    if args.T is not None:
+        p = p.with_(Tq=args.T, Tkv=args.T)
+    if args.ctx is not None:
+        p = p.with_(Tkv=args.ctx, q_pos0=args.ctx)
+    torch.cuda.set_device(0)
+    dt = torch.bfloat16 if p.dtype == "bf16" else torch.float32
+    simt = hsa._native.HSA_FLAG_SIMT if args.simt else 0
+
+    def timed(f):
+        for _ in range(args.iters):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            f()
+            torch.cuda.synchronize()
+            last = time.perf_counter() - t0
+        return last * 1e3
+
+    if args.select_only:
+        g = torch.Generator(device="cuda").manual_seed(0)
+        Q = torch.randn(p.B, p.Tq, p.H, p.d, device="cuda", generator=g).to(dt)
+        L = (torch.randn(p.B, p.Hkv, p.C, p.d, device="cuda", generator=g) / 8).to(dt)
+        prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, dt, simt)
+        ws = hsa.alloc_workspace(prob)
+        ms = timed(lambda: hsa.select(Q, L, p.S, p.k, p.tau, p.q_pos0, Tkv=p.Tkv, ws=ws, force_simt=args.simt))
+        hsa.device_status(ws)
+        print(f"{p.name} (select only): B{p.B} Tq{p.Tq} Tkv{p.Tkv} plan={hsa.plan(prob)} last={ms:.3f} ms")
+        return
+    inp = make_inputs(p, seed=0, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    if args.backward:
+        O, L, idx, sc, ke = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, p.q_pos0, return_selection=True)
+        dO = make_output_grad(p, seed=1, device="cuda")
+        prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, dt, simt)
+        ws = torch.empty(hsa.backward_workspace_size(prob), dtype=torch.uint8, device="cuda")
+        f32 = dict(dtype=torch.float32, device="cuda")
+        out = (torch.empty(Q.shape, **f32), torch.empty(K.shape, **f32), torch.empty(K.shape, **f32),
+               torch.empty(p.d, p.d, **f32))
+        ms = timed(lambda: hsa.backward(Q, K, V, W, L, idx, sc, ke, dO, p.S, p.k, p.tau, p.q_pos0, out=out, ws=ws,
+                                        force_simt=args.simt))
+        hsa.device_status(ws)
+        print(f"{p.name} backward: B{p.B} Tq{p.Tq} Tkv{p.Tkv} simt={args.simt} last={ms:.3f} ms")
+        return
+    ready = p.is_decode
+    L = hsa.landmarks(K, W, p.S) if ready else None
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, dt,
+                            (hsa._native.HSA_FLAG_LANDMARKS_READY if ready else 0) | simt)
+    ws = hsa.alloc_workspace(prob)
+    O = torch.empty_like(Q)
+    ms = timed(lambda: hsa.forward(Q, K, V, None if ready else W, p.S, p.k, p.tau, p.q_pos0, L=L,
+                                   landmarks_ready=ready, O=O, ws=ws, force_simt=args.simt))
+    hsa.device_status(ws)
+    print(f"{p.name}: B{p.B} Tq{p.Tq} Tkv{p.Tkv} plan={hsa.plan(prob)} last={ms:.3f} ms")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", default="prefill_bf16", choices=["prefill_bf16", "router_bf16", "tiny_f32"])
+    ap.add_argument("--workload", default="prefill_bf16",
+                    help="prefill_bf16 | router_bf16 | tiny_f32 (with --case also decode_1m, decode_16m)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-decode-16m", action="store_true", help="skip the 16M-context decode line (64 GiB cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass line")
+    ap.add_argument("--no-router", action="store_true", help="skip the gap-router prefill line (router_bf16)")
+    ap.add_argument("--case", action="store_true",
+                    help="single-case driver for profiler captures (see run_case); prints no JSON line")
+    ap.add_argument("--iters", type=int, default=3, help="--case: iterations")
+    ap.add_argument("--T", type=int, default=None, help="--case: prefill length (Tq = Tkv)")
+    ap.add_argument("--ctx", type=int, default=None, help="--case: decode context length")
+    ap.add_argument("--B", type=int, default=None, help="--case: batch")
+    ap.add_argument("--simt", action="store_true", help="--case: CUDA-core kernels only")
+    ap.add_argument("--select-only", action="store_true", help="--case: selection stage only, random landmarks")
+    ap.add_argument("--backward", action="store_true", help="--case: one forward, then the backward --iters times")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
+    if args.workload not in ("prefill_bf16", "router_bf16", "tiny_f32"):
+        ap.error(f"--workload {args.workload} is a --case workload; the bench line runs a prefill workload")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define HSA_ABI_VERSION 3
+#define HSA_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define HSA_API __attribute__((visibility("default")))
@@ -182,17 +182,21 @@ HSA_API hsa_status_t hsa_attend(const hsa_problem_t *p, const void *Q, const voi
  *     call's contents: calls that overlap on the GPU (other streams, other
  *     host threads) race on it and must be serialised by the caller.  A
  *     device-side timeout of this call is recorded in that array, not in any
- *     workspace, so hsa_get_device_status() cannot report it.
+ *     workspace: hsa_noalloc_status() reports it.
  */
 HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *p, const void *Q, const void *L, int32_t *idx,
                                         float *score, int32_t *keff, void *stream);
 
 /*
- * The whole path: hsa_landmarks (unless HSA_FLAG_LANDMARKS_READY), then
- * hsa_select, then hsa_attend.  L is an output (or an input with the flag).
- * idx, score and keff may each be NULL.  The selection then lives only in the
- * workspace.
+ * Device status of the latest hsa_select_noalloc call on the current device:
+ * synchronises `stream`, then reads and clears the status word at the start of
+ * the library's static scratch (every hsa_select_noalloc call clears it when it
+ * starts).  Returns HSA_OK, HSA_ERR_TIMEOUT (a bounded device wait expired; the
+ * call's idx/score/keff are incomplete) or HSA_ERR_CUDA (a kernel's own index
+ * check failed and skipped the access).  Allocates nothing.
  */
+HSA_API hsa_status_t hsa_noalloc_status(void *stream);
+
 /*
  * Context-sharded decode, per shard (summary page, Implementation: the
  * retrieval scores rank the chunks and weight their outputs).  The chunks of
@@ -229,6 +233,12 @@ HSA_API hsa_status_t hsa_merge_partials(const hsa_problem_t *p, int nshard, cons
                                         const int32_t *idx, const int32_t *keff, const float *o_part, void *O,
                                         int32_t *idx_out, float *score_out, int32_t *keff_out, void *stream);
 
+/*
+ * The whole path: hsa_landmarks (unless HSA_FLAG_LANDMARKS_READY), then
+ * hsa_select, then hsa_attend.  L is an output (or an input with the flag).
+ * idx, score and keff may each be NULL.  The selection then lives only in the
+ * workspace.
+ */
 HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                          const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
                          void *O, void *ws, size_t ws_bytes, void *stream);
@@ -284,9 +294,11 @@ HSA_API hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stre
 /* Kernel paths a stage can take (hsa_plan_t.*_path). */
 typedef enum {
     HSA_PATH_NONE = 0,         /* stage has nothing to do for this problem */
-    HSA_PATH_SIMT_ROWS = 1,    /* CUDA cores, one warp / CTA per selection row */
+    HSA_PATH_SIMT_ROWS = 1,    /* CUDA cores, one warp / CTA per selection row (landmarks: per chunk) */
     HSA_PATH_SIMT_SPLIT = 2,   /* CUDA cores, each row split over CTAs, then merged */
-    HSA_PATH_TENSOR = 3        /* tcgen05 tensor-core kernel */
+    HSA_PATH_TENSOR = 3,       /* tcgen05 tensor-core kernel (TMEM accumulators), many rows per tile */
+    HSA_PATH_MMA_SPLIT = 4     /* warp-level mma.sync tensor-core kernel for few rows: each row's chunks
+                                  split over CTAs (decode scan, chunk gather), merged in the same launch */
 } hsa_path_t;
 
 typedef struct {

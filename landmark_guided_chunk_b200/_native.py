@@ -20,8 +20,8 @@ HSA_FLAG_SIMT = 2
 EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version",
             "hsa_select_noalloc", "hsa_decode_append", "hsa_attend_partials", "hsa_merge_partials",
-            "hsa_backward_workspace_size", "hsa_backward")
-PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor"}
+            "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status")
+PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor", 4: "mma_split"}
 
 
 class hsa_problem_t(ctypes.Structure):
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
     L.hsa_decode_append.argtypes = [prob, P, P, P, P, P, P, P]
     L.hsa_attend_partials.argtypes = [prob, P, P, P, I32p, I32p, Fp, P, Z, P]
     L.hsa_merge_partials.argtypes = [prob, ctypes.c_int, Fp, I32p, I32p, Fp, P, I32p, Fp, I32p, P]
+    L.hsa_noalloc_status.argtypes = [P]
     L.hsa_backward_workspace_size.argtypes = [prob, ctypes.POINTER(ctypes.c_size_t)]
     L.hsa_backward.argtypes = [prob, P, P, P, P, P, I32p, Fp, I32p, P, Fp, Fp, Fp, Fp, P, Z, P]
     L.hsa_status_string.argtypes = [ctypes.c_int]
@@ -79,7 +80,8 @@ def lib() -> ctypes.CDLL:
     L.hsa_abi_version.restype = ctypes.c_int
     for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
               "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc", "hsa_decode_append",
-              "hsa_attend_partials", "hsa_merge_partials", "hsa_backward_workspace_size", "hsa_backward"):
+              "hsa_attend_partials", "hsa_merge_partials", "hsa_backward_workspace_size", "hsa_backward",
+              "hsa_noalloc_status"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

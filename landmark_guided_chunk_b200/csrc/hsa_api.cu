@@ -106,10 +106,12 @@ WsLayout ws_layout(const Prob &p) {
     w.plan.landmark_kernels = has_chunks ? 1 : 0;
     w.plan.select_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_select  ? HSA_PATH_TENSOR
+                         : (w.stream_select || w.mma_select) ? HSA_PATH_MMA_SPLIT
                          : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select && !w.stream_select ? 2 : 1);
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_attend  ? HSA_PATH_TENSOR
+                         : w.gather_attend ? HSA_PATH_MMA_SPLIT
                          : (w.split_attend ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
     // tensor path: count, scan (2 levels), tile list, scatter, one main kernel per phase batch + 1
     w.plan.attend_kernels = rows == 0 ? 0

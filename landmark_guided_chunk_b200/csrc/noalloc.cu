@@ -91,3 +91,23 @@ extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, co
     e = launch_select(p, w, Q, L, idx, score, keff, (char *)scratch, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "selection kernel launch");
 }
+
+// Status of the latest hsa_select_noalloc call on the current device: the word
+// at the start of the static scratch, read and cleared after `stream` drains.
+extern "C" HSA_API hsa_status_t hsa_noalloc_status(void *stream) {
+    void *scratch = nullptr;
+    hsa_status_t s = scratch_on_current_device(&scratch);
+    if (s != HSA_OK) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, scratch, sizeof word, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the static scratch status word");
+    if (word == DEV_OK) return HSA_OK;
+    e = cudaMemsetAsync(scratch, 0, sizeof word, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch status word");
+    if (word & DEV_TIMEOUT)
+        return fail(HSA_ERR_TIMEOUT, "static scratch status word 0x%x: a bounded device wait expired", word);
+    return fail(HSA_ERR_CUDA, "static scratch status word 0x%x: a kernel's internal index check failed", word);
+}

@@ -10,8 +10,9 @@
  * projection of the mean-pooled chunk; scores = similarity(query, landmarks);
  * keep the k best; attend inside each kept chunk with standard attention; fuse
  * the chunk outputs weighted by their retrieval scores) and the gap router of
- * the value-of-information router page ("double the kept set where the k-th /
- * (k+1)-th gap is smallest").  Readings where the pages are silent:
+ * the value-of-information router page (abstract: rows whose top-k cut is
+ * nearly tied, a small gap between the k-th and (k+1)-th scores, keep twice
+ * as many chunks).  Readings where the pages are silent:
  *   - the landmark is mean(keys of the chunk) times a d x d matrix W_L
  *     (row vector times W_L, W_L[e_in][e_out]), no refiner layer;
  *   - the similarity is the raw dot product; with grouped-query attention a

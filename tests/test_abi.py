@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.EXPORTED)
-    assert lib.hsa_abi_version() == 3
+    assert lib.hsa_abi_version() == 4
 
 
 def test_status_strings():

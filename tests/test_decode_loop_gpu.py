@@ -134,7 +134,7 @@ def test_decode_with_capacity_on_the_streaming_path():
     L = hsa.landmarks(K, W, p.S, kv_len=p.Tkv)
     prob = hsa.make_problem(p.B, 1, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.Tkv, 0.0, torch.bfloat16,
                             hsa._native.HSA_FLAG_LANDMARKS_READY, cap)
-    assert hsa.plan(prob)["attend"] == ("simt_split", 1)
+    assert hsa.plan(prob)["attend"] == ("mma_split", 1)
     O, _, idx, sc, ke = hsa.forward(Q, K, V, None, p.S, p.k, q_pos0=p.Tkv, L=L, landmarks_ready=True,
                                     return_selection=True, kv_len=p.Tkv)
     Kt, Vt = _tight(K, p.Tkv), _tight(V, p.Tkv)

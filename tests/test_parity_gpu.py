@@ -104,14 +104,16 @@ def test_small_prefill_cuda_core_path(p):
 
 
 def test_tensor_core_paths_are_the_ones_planned():
-    assert _plan(workload("prefill_bf16"))["select"][0] == "tensor"
-    assert _plan(workload("router_bf16"))["select"][0] == "tensor"
+    # many rows in bf16: tcgen05 scoring and chunk-major tcgen05 attention
+    for name in ("prefill_bf16", "router_bf16"):
+        assert _plan(workload(name))["select"][0] == "tensor"
+        assert _plan(workload(name))["attend"][0] == "tensor"
     assert _plan(SMALL[1])["select"][0] == "tensor"
-    # few rows in bf16: the single-launch slot-parallel gather kernel
-    assert tuple(_plan(workload("decode_1m"))["attend"]) == ("simt_split", 1)
-    # long decode scans in bf16: split tensor-core scan with the merge folded in
-    assert tuple(_plan(workload("decode_1m"))["select"]) == ("simt_split", 1)
-    assert tuple(_plan(DECODE_SMALL[3])["select"]) == ("simt_split", 1)
+    # few rows in bf16: the single-launch gather kernel (TMA + mma.sync)
+    assert tuple(_plan(workload("decode_1m"))["attend"]) == ("mma_split", 1)
+    # long decode scans in bf16: the streaming mma.sync scan with the merge folded in
+    assert tuple(_plan(workload("decode_1m"))["select"]) == ("mma_split", 1)
+    assert tuple(_plan(DECODE_SMALL[3])["select"]) == ("mma_split", 1)
 
 
 DECODE_SMALL = [

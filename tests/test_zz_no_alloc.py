@@ -46,6 +46,8 @@ def test_noalloc_select_equals_workspace_select_twice(p):
     for _ in range(2):
         out = (torch.full_like(ref_idx, -7), torch.full_like(ref_score, 7.0), torch.full_like(ref_keff, -7))
         assert _noalloc_call(p, Q, L, out) == _native.HSA_OK
+        # the call's device-status word (in the static scratch) reports a clean run
+        assert _native.lib().hsa_noalloc_status(torch.cuda.current_stream().cuda_stream) == _native.HSA_OK
         torch.cuda.synchronize()
         assert torch.equal(out[0], ref_idx)
         assert torch.equal(out[2], ref_keff)
@@ -57,7 +59,7 @@ def test_noalloc_select_rejects_a_problem_beyond_its_scratch():
     # 4096 decode rows x 32 slots (k = 16 with the router): the candidate lists need 1 MiB + the status word
     p = Problem(B=2048, Tq=1, Tkv=64 * 4096, H=2, Hkv=2, d=64, S=64, k=16, q_pos0=64 * 4096, tau=0.5, dtype="bf16")
     assert hsa.plan(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau))["select"][0] \
-        == "simt_split"
+        == "mma_split"
     prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau)
     fake = ctypes.c_void_p(256)   # never dereferenced: the size check comes first
     rc = _native.lib().hsa_select_noalloc(ctypes.byref(prob), fake, fake, fake, fake, fake, None)
