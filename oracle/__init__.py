@@ -17,6 +17,10 @@ two-chunk sigmoid, a single aligned key), convexity, torch SDPA for single
 candidate rows, and the exhaustive limit k >= #candidates; the backward against
 central finite differences of the forward above (selection held fixed) and the
 closed forms of its sums (sum_u dV_u, the per-chunk sum of dK, sum_i ds_i = 0).
+Selection variants (tests/test_oracle_variant_pins.py): the landmark refiner
+against torch SDPA, W_v = 0, W_q = 0 and constant chunks; Quest scoring against
+its upper-bound property, equality for single-key and constant chunks, the
+sign cases, numpy's channel max/min, and brute-force ranking.
 """
 from __future__ import annotations
 
@@ -40,8 +44,12 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.hsa_oracle_attend.argtypes = [I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P]
     lib.hsa_oracle_backward.argtypes = [I, I, LL, I, I, I, I, I, LL, P, P, P, P, P, P, P, P, P,
                                         P, P, P, P, P]
+    lib.hsa_oracle_landmarks_refined.argtypes = [I, I, LL, I, I, I, P, P, P, P, P, P]
+    lib.hsa_oracle_quest_summaries.argtypes = [I, I, LL, I, I, I, P, P]
+    lib.hsa_oracle_select_quest.argtypes = [I, I, I, I, I, LL, I, D, I, LL, P, P, P, P, P, P, P, P]
     for f in (lib.hsa_oracle_round, lib.hsa_oracle_landmarks, lib.hsa_oracle_select,
-              lib.hsa_oracle_attend, lib.hsa_oracle_backward):
+              lib.hsa_oracle_attend, lib.hsa_oracle_backward, lib.hsa_oracle_landmarks_refined,
+              lib.hsa_oracle_quest_summaries, lib.hsa_oracle_select_quest):
         f.restype = None
     return lib
 
@@ -115,6 +123,63 @@ def landmarks_stored_sliced(K, W_L, S: int, dtype: str, chunks_per_slice: int = 
             Ks = K[b:b + 1, c0 * S:c1 * S].cpu()
             L[b:b + 1, :, c0:c1] = landmarks_stored(Ks, W, S, dtype)
     return L
+
+
+def landmarks_refined(K, W_L, W_q, W_k, W_v, S: int) -> np.ndarray:
+    """fp64 refined landmarks [B,Hkv,C,d]: the pooled landmark mean(K) W_L plus
+    one head of cross-attention from it (query L0 W_q) to the chunk's keys
+    (keys K W_k, values K W_v, scale 1/sqrt(d))."""
+    dk, Ka = _buf(K)
+    ws = [_buf(w) for w in (W_L, W_q, W_k, W_v)]
+    if any(dw != dk for dw, _ in ws):
+        raise TypeError("K and the weights must share a dtype")
+    B, T, Hkv, d = Ka.shape
+    C = T // S
+    L = np.zeros((B, Hkv, C, d), dtype=np.float64)
+    _load().hsa_oracle_landmarks_refined(dk, B, T, Hkv, d, S, _ptr(Ka), *(_ptr(a) for _, a in ws), _ptr(L))
+    return L
+
+
+def landmarks_refined_stored(K, W_L, W_q, W_k, W_v, S: int, dtype: str) -> np.ndarray:
+    """Refined landmarks as the library stores them: rounded once to dtype."""
+    return round_to(dtype, landmarks_refined(K, W_L, W_q, W_k, W_v, S))
+
+
+def quest_summaries(K, S: int) -> np.ndarray:
+    """Quest chunk summaries [B,Hkv,C,2d] (fp64 holding stored values): the
+    channel-wise max of each complete chunk's keys, then the channel-wise min."""
+    dk, Ka = _buf(K)
+    B, T, Hkv, d = Ka.shape
+    C = T // S
+    Lq = np.zeros((B, Hkv, C, 2 * d), dtype=np.float64)
+    _load().hsa_oracle_quest_summaries(dk, B, T, Hkv, d, S, _ptr(Ka), _ptr(Lq))
+    return Lq
+
+
+def select_quest(Qr, row_b, row_p, Lq: np.ndarray, S: int, k: int, tau: float, H: int,
+                 want_all: bool = False) -> dict:
+    """Top-k selection by Quest's criticality bound for query rows Qr [n,H,d]
+    against chunk summaries Lq [B,Hkv,C,2d]; same outputs as :func:`select`."""
+    dq, Qa = _buf(Qr)
+    Lq = np.ascontiguousarray(Lq, dtype=np.float64)
+    n, Hq, d = Qa.shape
+    assert Hq == H
+    B, Hkv, C, d2 = Lq.shape
+    assert d2 == 2 * d and H % Hkv == 0
+    kmax = 2 * k if tau > 0 else k
+    rb = np.ascontiguousarray(row_b, dtype=np.int32)
+    rp = np.ascontiguousarray(row_p, dtype=np.int64)
+    idx = np.empty((n, Hkv, kmax), dtype=np.int32)
+    score = np.empty((n, Hkv, kmax), dtype=np.float64)
+    keff = np.empty((n, Hkv), dtype=np.int32)
+    alls = np.empty((n, Hkv, C), dtype=np.float64) if want_all else None
+    _load().hsa_oracle_select_quest(dq, H, Hkv, d, S, C, k, float(tau), kmax, n, _ptr(rb), _ptr(rp),
+                                    _ptr(Qa), _ptr(Lq), _ptr(idx), _ptr(score), _ptr(keff),
+                                    _ptr(alls) if alls is not None else None)
+    out = {"idx": idx, "score": score, "keff": keff}
+    if want_all:
+        out["allscores"] = alls
+    return out
 
 
 def select(Qr, row_b, row_p, L: np.ndarray, S: int, k: int, tau: float, H: int,

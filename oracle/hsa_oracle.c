@@ -389,3 +389,175 @@ void hsa_oracle_backward(int dt, int B, long long Tkv, int H, int Hkv, int d, in
             }
     free(mean); free(dm);
 }
+
+/* ------------------------------------------------------------------------
+ * Selection variants.
+ *
+ * Landmark refiner (HSA summary page, Implementation: a learned layer with
+ * cross-attention refines the mean-pooled landmark).  Reading: one head of
+ * cross-attention whose query is the pooled landmark and whose keys and
+ * values are the chunk's own S keys, added back to the landmark:
+ *   L0  = mean_u(K_u) W_L
+ *   q   = L0 W_q,     kap_u = K_u W_k,     nu_u = K_u W_v
+ *   a   = softmax_u(q . kap_u / sqrt(d))
+ *   L   = L0 + sum_u a_u nu_u
+ * W_L, W_q, W_k, W_v: d x d, row = input dim, dtype dt.  L: double, NOT
+ * rounded to the storage dtype.
+ */
+void hsa_oracle_landmarks_refined(int dt, int B, long long T, int Hkv, int d, int S,
+                                  const void *K, const void *WL, const void *Wq,
+                                  const void *Wk, const void *Wv, double *L)
+{
+    long long C = T / S;
+    double scale = 1.0 / sqrt((double)d);
+#pragma omp parallel for collapse(2) schedule(dynamic, 4)
+    for (int b = 0; b < B; ++b) {
+        for (long long c = 0; c < C; ++c) {
+            double *mean = (double *)malloc(sizeof(double) * (size_t)d);
+            double *l0 = (double *)malloc(sizeof(double) * (size_t)d);
+            double *q = (double *)malloc(sizeof(double) * (size_t)d);
+            double *kap = (double *)malloc(sizeof(double) * (size_t)d);
+            double *nu = (double *)malloc(sizeof(double) * (size_t)d);
+            double *logit = (double *)malloc(sizeof(double) * (size_t)S);
+            double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+            for (int j = 0; j < Hkv; ++j) {
+                size_t row0 = (((size_t)b * (size_t)T + (size_t)(c * S)) * Hkv + j) * (size_t)d;
+                size_t rstride = (size_t)Hkv * d;
+                for (int e = 0; e < d; ++e) mean[e] = 0.0;
+                for (int u = 0; u < S; ++u)
+                    for (int e = 0; e < d; ++e) mean[e] += load(K, row0 + u * rstride + e, dt);
+                for (int e = 0; e < d; ++e) mean[e] = mean[e] / (double)S;
+                for (int f = 0; f < d; ++f) {
+                    double s = 0.0;
+                    for (int e = 0; e < d; ++e) s += mean[e] * load(WL, (size_t)e * d + f, dt);
+                    l0[f] = s;
+                }
+                for (int f = 0; f < d; ++f) {
+                    double s = 0.0;
+                    for (int e = 0; e < d; ++e) s += l0[e] * load(Wq, (size_t)e * d + f, dt);
+                    q[f] = s;
+                }
+                /* logits of the landmark query against every key of the chunk */
+                double mx = -INFINITY;
+                for (int u = 0; u < S; ++u) {
+                    for (int f = 0; f < d; ++f) {
+                        double s = 0.0;
+                        for (int e = 0; e < d; ++e)
+                            s += load(K, row0 + u * rstride + e, dt) * load(Wk, (size_t)e * d + f, dt);
+                        kap[f] = s;
+                    }
+                    double dot = 0.0;
+                    for (int f = 0; f < d; ++f) dot += q[f] * kap[f];
+                    logit[u] = dot * scale;
+                    if (logit[u] > mx) mx = logit[u];
+                }
+                double z = 0.0;
+                for (int u = 0; u < S; ++u) { logit[u] = exp(logit[u] - mx); z += logit[u]; }
+                for (int f = 0; f < d; ++f) acc[f] = 0.0;
+                for (int u = 0; u < S; ++u) {
+                    double a = logit[u] / z;
+                    for (int f = 0; f < d; ++f) {
+                        double s = 0.0;
+                        for (int e = 0; e < d; ++e)
+                            s += load(K, row0 + u * rstride + e, dt) * load(Wv, (size_t)e * d + f, dt);
+                        nu[f] = s;
+                    }
+                    for (int f = 0; f < d; ++f) acc[f] += a * nu[f];
+                }
+                double *out = L + (((size_t)b * Hkv + j) * (size_t)C + (size_t)c) * (size_t)d;
+                for (int f = 0; f < d; ++f) out[f] = l0[f] + acc[f];
+            }
+            free(mean); free(l0); free(q); free(kap); free(nu); free(logit); free(acc);
+        }
+    }
+}
+
+/*
+ * Quest-style chunk summaries (value-of-information router page, abstract:
+ * the router stacks on block-scoring methods such as Quest).  Reading: Quest's
+ * page summary with the chunk as the page -- per complete chunk and kv head,
+ * the channel-wise maximum and minimum of its S keys:
+ *   Lq[b][j][c][e] = max_u K[b][cS+u][j][e],   Lq[b][j][c][d + e] = min_u K[b][cS+u][j][e]
+ * Lq [B][Hkv][C][2d] double (the values are stored values: no rounding).
+ */
+void hsa_oracle_quest_summaries(int dt, int B, long long T, int Hkv, int d, int S,
+                                const void *K, double *Lq)
+{
+    long long C = T / S;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (long long c = 0; c < C; ++c) {
+            for (int j = 0; j < Hkv; ++j) {
+                double *out = Lq + (((size_t)b * Hkv + j) * (size_t)C + (size_t)c) * (size_t)(2 * d);
+                for (int e = 0; e < d; ++e) { out[e] = -INFINITY; out[d + e] = INFINITY; }
+                for (int u = 0; u < S; ++u) {
+                    size_t row = (((size_t)b * (size_t)T + (size_t)(c * S + u)) * Hkv + j) * (size_t)d;
+                    for (int e = 0; e < d; ++e) {
+                        double x = load(K, row + e, dt);
+                        if (x > out[e]) out[e] = x;
+                        if (x < out[d + e]) out[d + e] = x;
+                    }
+                }
+            }
+        }
+    }
+}
+
+/*
+ * Top-k selection with Quest's criticality score in place of the landmark dot
+ * product.  For chunk c and a query row's kv head j:
+ *   s_c = sum_{h in group j} sum_e max(q_h[e] * Lq_c[e], q_h[e] * Lq_c[d + e])
+ * -- for each head the largest value any key of the chunk could give each
+ * product q_h[e] k[e], summed: an upper bound of sum_h max_u q_h . K_u.  The
+ * candidates, ranking, ties, keff and router are those of hsa_oracle_select.
+ *   Lq [B][Hkv][C][2d] double; other arguments as hsa_oracle_select.
+ */
+void hsa_oracle_select_quest(int dt_q, int H, int Hkv, int d, int S, long long C, int k,
+                             double tau, int kmax, long long n, const int *row_b,
+                             const long long *row_p, const void *Qr, const double *Lq,
+                             int *idx, double *score, int *keff, double *allscores)
+{
+    int G = H / Hkv;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (long long r = 0; r < n; ++r) {
+        long long ncand = row_p[r] / (long long)S;
+        if (ncand > C) ncand = C;
+        if (ncand < 0) ncand = 0;
+        cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * (size_t)(ncand > 0 ? ncand : 1));
+        for (int j = 0; j < Hkv; ++j) {
+            const double *Lj = Lq + ((size_t)row_b[r] * Hkv + j) * (size_t)C * (size_t)(2 * d);
+            for (long long c = 0; c < ncand; ++c) {
+                const double *mx = Lj + (size_t)c * (2 * d), *mn = mx + d;
+                double s = 0.0;
+                for (int h = j * G; h < (j + 1) * G; ++h) {
+                    double bound = 0.0;
+                    for (int e = 0; e < d; ++e) {
+                        double qe = load(Qr, ((size_t)r * H + h) * d + e, dt_q);
+                        double hi = qe * mx[e], lo = qe * mn[e];
+                        bound += hi > lo ? hi : lo;
+                    }
+                    s += bound;
+                }
+                cand[c].s = s;
+                cand[c].c = c;
+                if (allscores) allscores[((size_t)r * Hkv + j) * (size_t)C + c] = s;
+            }
+            if (allscores)
+                for (long long c = ncand; c < C; ++c)
+                    allscores[((size_t)r * Hkv + j) * (size_t)C + c] = -INFINITY;
+            qsort(cand, (size_t)ncand, sizeof(cand_t), cand_order);
+            long long ke = ncand < k ? ncand : k;
+            if (tau > 0.0 && ncand > k) {
+                double gap = cand[k - 1].s - cand[k].s;
+                if (gap < tau * fabs(cand[k - 1].s)) ke = ncand < 2 * k ? ncand : 2 * k;
+            }
+            size_t o = ((size_t)r * Hkv + j) * kmax;
+            for (int i = 0; i < kmax; ++i) {
+                idx[o + i] = i < ke ? (int)cand[i].c : -1;
+                score[o + i] = i < ke ? cand[i].s : -INFINITY;
+            }
+            keff[(size_t)r * Hkv + j] = (int)ke;
+        }
+        free(cand);
+    }
+}

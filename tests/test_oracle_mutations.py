@@ -9,7 +9,10 @@ candidates, a group score from one head, bf16 rounding with ties away from
 zero, ties between chunks broken the wrong way, the router's comparison reversed,
 uniform fusion weights, the in-chunk softmax without its 1/sqrt(d), and in
 the backward a dropped softmax term, a missing landmark share, a missing e
-term and a sign error.
+term and a sign error; in the selection variants a refiner without its
+1/sqrt(d), without its residual or with W_k transposed, and a Quest score
+that takes the smaller product, starts the channel minimum at 0 or reads one
+head of the group.
 """
 import ctypes
 import os
@@ -20,6 +23,7 @@ import pytest
 import oracle
 from tests import test_oracle_backward_pins as bw
 from tests import test_oracle_pins as pins
+from tests import test_oracle_variant_pins as vp
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "hsa_oracle.c")
 
@@ -77,6 +81,30 @@ MUTANTS = {
         "dLc[x] += ds * load(Qr, qh + x, dt);",
         "dLc[x] -= ds * load(Qr, qh + x, dt);",
         [lambda: bw.test_backward_matches_central_finite_differences(2, 0.0, 1)]),
+    "refiner: no 1/sqrt(d)": (
+        "logit[u] = dot * scale;",
+        "logit[u] = dot;",
+        [lambda: vp.test_refiner_matches_sdpa(vp.torch.float32, 16, 8)]),
+    "refiner: residual dropped": (
+        "for (int f = 0; f < d; ++f) out[f] = l0[f] + acc[f];",
+        "for (int f = 0; f < d; ++f) out[f] = acc[f];",
+        [vp.test_refiner_without_value_path_is_the_plain_landmark]),
+    "refiner: W_k transposed": (
+        "s += load(K, row0 + u * rstride + e, dt) * load(Wk, (size_t)e * d + f, dt);",
+        "s += load(K, row0 + u * rstride + e, dt) * load(Wk, (size_t)f * d + e, dt);",
+        [lambda: vp.test_refiner_matches_sdpa(vp.torch.float32, 16, 8)]),
+    "quest: smaller product taken": (
+        "bound += hi > lo ? hi : lo;",
+        "bound += hi < lo ? hi : lo;",
+        [vp.test_quest_score_bounds_every_key]),
+    "quest: channel minimum starts at 0": (
+        "for (int e = 0; e < d; ++e) { out[e] = -INFINITY; out[d + e] = INFINITY; }",
+        "for (int e = 0; e < d; ++e) { out[e] = -INFINITY; out[d + e] = 0.0; }",
+        [vp.test_quest_summaries_are_channel_max_and_min]),
+    "quest: one head of the group": (
+        "                for (int h = j * G; h < (j + 1) * G; ++h) {\n                    double bound = 0.0;",
+        "                for (int h = j * G; h < j * G + 1; ++h) {\n                    double bound = 0.0;",
+        [lambda: vp.test_quest_score_is_exact_when_the_chunk_has_one_key_value("single_key")]),
 }
 
 
