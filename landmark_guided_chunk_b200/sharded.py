@@ -1,4 +1,19 @@
-"""Context-sharded decode (HSA summary page, Implementation: the retrieval
+"""Multi-device HSA: the (batch, kv head) split of prefill and the
+context-sharded decode.
+
+Prefill split (``prefill_shard_range``, ``sharded_prefill``).  Each kv head's
+landmarks, selection, chunk attention and fusion read only that kv head's K, V
+and its G query heads (HSA summary page, Implementation: one selection per
+query, attention inside the kept chunks; the GQA group shares it), and each
+sequence is independent.  So the (b, kv head) units split over devices with no
+exchange at all: a rank holds the Q, K, V of its units -- the layout a
+head-parallel model already has -- and computes their O.  With Hkv divisible
+by the world size the ranks take contiguous blocks of Hkv / world kv heads
+(this shortens one long sequence's prefill); otherwise, with B divisible, they
+take contiguous blocks of sequences.  The only collective is optional: an
+all-gather that assembles the whole O on every rank.
+
+Context-sharded decode (HSA summary page, Implementation: the retrieval
 scores rank the chunks and weight their outputs).
 
 A long context's chunks are split into contiguous ranges, one per device: each
@@ -27,9 +42,56 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import attend_partials, kmax_of, merge_partials, select
+from . import attend_partials, forward, kmax_of, merge_partials, select
 
-__all__ = ["local_q_pos", "shard_partials", "gather_shards", "sharded_decode"]
+__all__ = ["local_q_pos", "shard_partials", "gather_shards", "sharded_decode", "prefill_shard_range",
+           "shard_inputs", "sharded_prefill"]
+
+
+def _world_rank(group):
+    if group is None and not dist.is_initialized():
+        return 1, 0
+    return dist.get_world_size(group), dist.get_rank(group)
+
+
+def prefill_shard_range(B: int, Hkv: int, world: int, rank: int):
+    """This rank's units of the (b, kv head) split: ("heads", j0, j1) -- kv
+    heads j0..j1-1 of every sequence -- when world divides Hkv, else
+    ("batch", b0, b1) -- sequences b0..b1-1 -- when it divides B."""
+    if Hkv % world == 0:
+        n = Hkv // world
+        return "heads", rank * n, (rank + 1) * n
+    if B % world == 0:
+        n = B // world
+        return "batch", rank * n, (rank + 1) * n
+    raise ValueError(f"neither Hkv={Hkv} nor B={B} is divisible by the world size {world}")
+
+
+def shard_inputs(Q, K, V, world: int, rank: int):
+    """This rank's part of Q [B,T,H,d], K and V [B,T,Hkv,d] under the (b, kv
+    head) split, as contiguous copies (a head-parallel model holds them this way
+    already).  Returns (kind, Q, K, V) with kind "heads" or "batch"."""
+    B, Hkv = K.shape[0], K.shape[2]
+    G = Q.shape[2] // Hkv
+    kind, a, b = prefill_shard_range(B, Hkv, world, rank)
+    if kind == "heads":
+        return kind, Q[:, :, a * G:b * G].contiguous(), K[:, :, a:b].contiguous(), V[:, :, a:b].contiguous()
+    return kind, Q[a:b].contiguous(), K[a:b].contiguous(), V[a:b].contiguous()
+
+
+def sharded_prefill(Q, K, V, W_L, S, k, tau=0.0, kind="heads", group=None, gather=False, forward_fn=forward):
+    """The (b, kv head) split of a prefill on this rank.  Q, K, V are this
+    rank's shard and kind its split (``shard_inputs``); W_L is shared.  Returns
+    this rank's O, or with gather=True the whole O [B, T, H, d] on every rank,
+    assembled by one all-gather (ranks concatenated along the heads or the
+    batch).  forward_fn computes one shard (the CUDA path by default)."""
+    O = forward_fn(Q, K, V, W_L, S, k, tau)
+    world, _ = _world_rank(group)
+    if not gather or world == 1:
+        return O
+    parts = [torch.empty_like(O) for _ in range(world)]
+    dist.all_gather(parts, O.contiguous(), group=group)
+    return torch.cat(parts, dim=2 if kind == "heads" else 0)
 
 
 def local_q_pos(q_pos0: int, chunk0: int, S: int) -> int:

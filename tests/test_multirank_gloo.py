@@ -193,3 +193,48 @@ def _dp_backward(rank, port):
 
 def test_data_parallel_backward_exchange_two_ranks():
     mp.spawn(_dp_backward, args=(_free_port(),), nprocs=WORLD, join=True)
+
+
+def _oracle_forward(Q, K, V, W, S, k, tau):
+    B, T, H, d = Q.shape
+    rb, rt = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+    out = oracle.forward_rows(Q, K, V, W, S, k, tau, 0, rb, rt)
+    return torch.tensor(out["O"]).reshape(B, T, H, d)
+
+
+def _sharded_prefill(rank, port, B, Hkv, expect_kind):
+    """The (b, kv head) split of a prefill: each rank computes its shard (the
+    oracle stands in for the kernels) and one all-gather assembles O; it must
+    equal the oracle over the whole problem, bit for bit (the units share nothing)."""
+    _init(rank, port)
+    try:
+        from landmark_guided_chunk_b200 import sharded
+        rng = np.random.default_rng(5)
+        T, G, d, S, k = 32 * 7 + 5, 2, 16, 32, 3
+        H = Hkv * G
+        Q = torch.tensor(rng.standard_normal((B, T, H, d)), dtype=torch.float32)
+        K = torch.tensor(rng.standard_normal((B, T, Hkv, d)), dtype=torch.float32)
+        V = torch.tensor(rng.standard_normal((B, T, Hkv, d)), dtype=torch.float32)
+        W = torch.tensor(rng.standard_normal((d, d)) / d ** 0.5, dtype=torch.float32)
+        kind, Qr, Kr, Vr = sharded.shard_inputs(Q, K, V, WORLD, rank)
+        assert kind == expect_kind
+        O = sharded.sharded_prefill(Qr, Kr, Vr, W, S, k, 0.0, kind=kind, gather=True, forward_fn=_oracle_forward)
+        ref = _oracle_forward(Q, K, V, W, S, k, 0.0)
+        assert O.shape == ref.shape
+        assert torch.equal(O, ref)
+        mine = sharded.sharded_prefill(Qr, Kr, Vr, W, S, k, 0.0, kind=kind, forward_fn=_oracle_forward)
+        a = rank * (Hkv // WORLD) * G if kind == "heads" else 0
+        if kind == "heads":
+            assert torch.equal(mine, ref[:, :, a:a + Qr.shape[2]])
+        else:
+            assert torch.equal(mine, ref[rank * (B // WORLD):(rank + 1) * (B // WORLD)])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_prefill_kv_head_split_two_ranks():
+    mp.spawn(_sharded_prefill, args=(_free_port(), 1, 4, "heads"), nprocs=WORLD, join=True)
+
+
+def test_sharded_prefill_batch_split_two_ranks():
+    mp.spawn(_sharded_prefill, args=(_free_port(), 2, 3, "batch"), nprocs=WORLD, join=True)

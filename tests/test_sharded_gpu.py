@@ -80,3 +80,36 @@ def test_merge_rejects_mismatched_slots():
     ke = torch.zeros(2, 1, 1, 2, dtype=torch.int32, device="cuda")
     with pytest.raises(ValueError):
         hsa.merge_partials(sc, ix, ke, o, 64, 8, tau=0.05)   # the router doubles k: 16 slots expected
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_prefill_kv_head_shards_match_the_oracle(world):
+    """The (b, kv head) split of one prefill sequence: every rank's shard, run
+    through the CUDA forward on this device, against the oracle on that shard's
+    rows (its kv heads' landmarks, selection and output)."""
+    from landmark_guided_chunk_b200 import sharded
+    p = Problem(B=1, Tq=64 * 20 + 13, Tkv=64 * 20 + 13, H=16, Hkv=4, d=128, S=64, k=8, dtype="bf16")
+    inp = make_inputs(p, seed=9, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    outs = []
+    for r in range(world):
+        kind, Qr, Kr, Vr = sharded.shard_inputs(Q, K, V, world, r)
+        assert kind == "heads"
+        O, L, idx, sc, ke = hsa.forward(Qr, Kr, Vr, W, p.S, p.k, return_selection=True)
+        torch.cuda.synchronize()
+        B, T, Hr, d = Qr.shape
+        rb, rt = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+        Lr = L.double().cpu().numpy()
+        parity.check_landmarks(L, oracle.landmarks_stored(Kr.cpu(), W.cpu(), p.S, "bf16"))
+        orc = oracle.select(Qr.cpu().reshape(B * T, Hr, d), rb, rt, Lr, p.S, p.k, 0.0, Hr, want_all=True)
+        ncand = np.minimum(rt // p.S, p.C)
+        sel = parity.check_selection(idx.reshape(-1, Kr.shape[2], p.k).cpu().numpy(),
+                                     sc.reshape(-1, Kr.shape[2], p.k).cpu().numpy(),
+                                     ke.reshape(-1, Kr.shape[2]).cpu().numpy(), orc, ncand, p.k, 0.0)
+        O_exp = parity.expected_output(Qr.cpu().reshape(B * T, Hr, d), rb, Kr, Vr, p.S, orc,
+                                       idx.reshape(-1, Kr.shape[2], p.k).cpu().numpy(),
+                                       ke.reshape(-1, Kr.shape[2]).cpu().numpy(), sel["tie_rows"])
+        parity.check_output(O.reshape(B * T, Hr, d), O_exp, torch.bfloat16)
+        outs.append(O)
+    # the shards tile the heads: together they are the single-device result's layout
+    assert torch.cat(outs, dim=2).shape == Q.shape
