@@ -23,6 +23,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -282,6 +283,105 @@ def run_router(args, world, rank, local, pk):
     return out
 
 
+def run_variants(args, world, rank, local, pk):
+    """The two selection variants on the prefill_bf16 shapes, each stage timed
+    with CUDA events over back-to-back forwards: Quest block scoring
+    (summaries -> Quest selection -> attention) and the landmark refiner
+    (refined landmarks -> selection -> attention)."""
+    import landmark_guided_chunk_b200 as hsa
+
+    dev = torch.device("cuda", local)
+    ps = PrefillSetup(args.workload, args.seed + rank, dev)
+    p, Q, K, V, W = ps.p, ps.Q, ps.K, ps.V, ps.W
+    lib, P, sp = hsa._native.lib(), hsa._p, ps.st.cuda_stream
+    g = torch.Generator(device=dev).manual_seed(args.seed + 7)
+    Wq, Wk, Wv = ((torch.randn(p.d, p.d, device=dev, generator=g) / math.sqrt(p.d)).to(Q.dtype) for _ in range(3))
+    steps = max(1, min(args.steps, 10))
+    out = {}
+    es = 2 if p.dtype == "bf16" else 4
+    k_bytes = p.B * p.Tkv * p.Hkv * p.d * es
+
+    def timed(stages):
+        for _ in range(args.warmup):
+            for _, f in stages:
+                f()
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(steps)]
+        barrier(world)
+        for s in range(steps):
+            ev[s][0].record(ps.st)
+            for i, (_, f) in enumerate(stages):
+                f()
+                ev[s][i + 1].record(ps.st)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ms = {name: sum(e[i].elapsed_time(e[i + 1]) for e in ev) / steps for i, (name, _) in enumerate(stages)}
+        return ms, max_over_ranks(sum(ms.values()), world)
+
+    # Quest block scoring
+    qprob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, Q.dtype,
+                             hsa._native.HSA_FLAG_QUEST)
+    qplan = hsa.plan(qprob)
+    qws = hsa.alloc_workspace(qprob, dev)
+    Lq = torch.empty(p.B, p.Hkv, p.C, 2 * p.d, dtype=Q.dtype, device=dev)
+    idx, score, keff, O = ps.idx, ps.score, ps.keff, ps.O
+    stages = [
+        ("summaries", lambda: hsa._native.check(lib.hsa_landmarks(ctypes.byref(qprob), P(K), None, P(Lq), sp),
+                                                "hsa_landmarks")),
+        ("select", lambda: hsa._native.check(lib.hsa_select(ctypes.byref(qprob), P(Q), P(Lq), P(idx), P(score),
+                                                            P(keff), P(qws), qws.numel(), sp), "hsa_select")),
+        ("attend", lambda: hsa._native.check(lib.hsa_attend(ctypes.byref(qprob), P(Q), P(K), P(V), P(idx),
+                                                            P(score), P(keff), P(O), P(qws), qws.numel(), sp),
+                                             "hsa_attend")),
+    ]
+    ms, total = timed(stages)
+    keff_sum = int(keff.sum().item())
+    work = work_counts(p, keff_sum)
+    # the selection kernels contract [P | N] (hi and lo parts) with [Mx | Mn]: 4d per (token, kv head, candidate)
+    sel_flops = 2.0 * 4 * p.d * p.Hkv * float(ncand_rows(p).sum()) * p.B
+    sum_bytes = k_bytes + p.B * p.Hkv * p.C * 2 * p.d * es
+    out["quest"] = {
+        "ms_per_forward": round(total, 4), "tokens_per_s": round(p.B * p.Tq * world / (total * 1e-3), 1),
+        "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3), "plan": {k2: list(v) for k2, v in qplan.items()},
+        "stages": {
+            "summaries": {"ms": round(ms["summaries"], 4), "bound": "hbm", "unit": "GB/s",
+                          "achieved": round(sum_bytes / (ms["summaries"] * 1e-3) / 1e9, 1),
+                          "frac": round(sum_bytes / (ms["summaries"] * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+            "select": {"ms": round(ms["select"], 4), "bound": "tensor", "unit": "TFLOP/s",
+                       "achieved": round(sel_flops / (ms["select"] * 1e-3) / 1e12, 2),
+                       "frac": round(sel_flops / (ms["select"] * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+                       "note": "query transform + tcgen05 scoring of the width-4d contraction with fused top-k"},
+            "attend": {"ms": round(ms["attend"], 4), "bound": "tensor", "unit": "TFLOP/s",
+                       "achieved": round(work["attend_flops"] / (ms["attend"] * 1e-3) / 1e12, 2),
+                       "frac": round(work["attend_flops"] / (ms["attend"] * 1e-3) / 1e12 / pk["bf16_tflops"], 4)}},
+        "gpu_launches": steps * sum(qplan[x][1] for x in ("landmarks", "select", "attend"))}
+    del qws, Lq
+
+    # landmark refiner
+    L = ps.L
+
+    def refine():
+        hsa._native.check(lib.hsa_landmarks_refined(ctypes.byref(ps.prob), P(K), P(W), P(Wq), P(Wk), P(Wv), P(L), sp),
+                          "hsa_landmarks_refined")
+
+    stages = [("refined_landmarks", refine)] + ps.stages[1:]
+    ms, total = timed(stages)
+    keff_sum = int(keff.sum().item())
+    lm_bytes = k_bytes + p.B * p.Hkv * p.C * p.d * es + 4 * p.d * p.d * es
+    out["refine"] = {
+        "ms_per_forward": round(total, 4), "tokens_per_s": round(p.B * p.Tq * world / (total * 1e-3), 1),
+        "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3),
+        "stages": {"refined_landmarks": {"ms": round(ms["refined_landmarks"], 4), "bound": "hbm", "unit": "GB/s",
+                                         "achieved": round(lm_bytes / (ms["refined_landmarks"] * 1e-3) / 1e9, 1),
+                                         "frac": round(lm_bytes / (ms["refined_landmarks"] * 1e-3) / 1e9
+                                                       / pk["hbm_gbs"], 4)},
+                   "select": {"ms": round(ms["select"], 4)}, "attend": {"ms": round(ms["attend"], 4)}},
+        "gpu_launches": steps * (1 + ps.plan["select"][1] + ps.plan["attend"][1])}
+    del ps
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_b200(args, world, rank, local):
     import landmark_guided_chunk_b200 as hsa
 
@@ -375,6 +475,8 @@ def run_b200(args, world, rank, local):
     torch.cuda.empty_cache()
     if not args.no_router and args.workload == "prefill_bf16":
         out["router_bf16"] = run_router(args, world, rank, local, pk)
+    if not args.no_variants and args.workload == "prefill_bf16":
+        out["variants"] = run_variants(args, world, rank, local, pk)
     if not args.no_decode:
         out["decode_1m"] = run_decode(args, world, rank, local, pk)
         if not args.no_decode_16m:
@@ -839,6 +941,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass line")
     ap.add_argument("--no-router", action="store_true", help="skip the gap-router prefill line (router_bf16)")
+    ap.add_argument("--no-variants", action="store_true", help="skip the selection-variant lines (Quest, refiner)")
     ap.add_argument("--case", action="store_true",
                     help="single-case driver for profiler captures (see run_case); prints no JSON line")
     ap.add_argument("--iters", type=int, default=3, help="--case: iterations")

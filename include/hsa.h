@@ -84,6 +84,22 @@ typedef enum { HSA_F32 = 0, HSA_BF16 = 1 } hsa_dtype_t;
 /* hsa_problem_t.flags */
 #define HSA_FLAG_LANDMARKS_READY 1u  /* hsa_forward: L already holds the landmarks; skip that stage (W_L may be NULL) */
 #define HSA_FLAG_SIMT 2u             /* use the CUDA-core kernels even where a tensor-core kernel exists (testing) */
+/* Testing only: the tcgen05 scoring kernel (hsa_select on the HSA_PATH_TENSOR select path;
+ * other paths ignore the flag) runs with a 0.1 ms wait limit, and its epilogue first waits on a
+ * barrier that nothing arrives on.  That wait expires, every role of the kernel winds down
+ * (in-flight loads drained, MMAs committed, TMEM freed) and the call's status word records
+ * HSA_ERR_TIMEOUT; idx/score/keff are left incomplete.  It exercises the failure path that a
+ * real stall would take, without faulting or hanging the device. */
+#define HSA_FLAG_TEST_STALL 4u
+/* Quest block scoring in place of the landmark dot product (value-of-information router page,
+ * abstract: the router stacks on block scorers such as Quest).  "Landmarks" are then the Quest
+ * chunk summaries Lq [B][Hkv][Ccap][2d]: the channel-wise max of the chunk's keys, then the
+ * channel-wise min (exact stored values; hsa_landmarks computes them and takes no W_L).  A query
+ * row's score of chunk c is sum_{h in group} sum_e max(q_h[e] Lq_c[e], q_h[e] Lq_c[d + e]);
+ * candidates, ranking, ties, keff, router and the fusion weights (softmax of these scores) are
+ * unchanged.  Honoured by hsa_landmarks, hsa_decode_append, hsa_select, hsa_forward and
+ * hsa_workspace_size; hsa_backward and hsa_select_noalloc return HSA_ERR_UNSUPPORTED. */
+#define HSA_FLAG_QUEST 8u
 
 typedef struct {
     int32_t B, Tq, Tkv, H, Hkv, d, S, k;
@@ -117,6 +133,23 @@ HSA_API hsa_status_t hsa_workspace_size(const hsa_problem_t *p, size_t *bytes);
  */
 HSA_API hsa_status_t hsa_landmarks(const hsa_problem_t *p, const void *K, const void *W_L, void *L,
                            void *stream);
+
+/*
+ * Refined landmarks (HSA summary page, Implementation: a learned layer with
+ * cross-attention refines the mean-pooled landmark).  For every complete chunk
+ * c and kv head j, one head of cross-attention whose query is the pooled
+ * landmark and whose keys and values are the chunk's own keys, added back:
+ *   L0 = ( (1/S) sum_{u<S} K[b][cS+u][j][:] ) * W_L
+ *   a_u = softmax_u( (L0 W_q) . (K[b][cS+u][j][:] W_k) / sqrt(d) )
+ *   L[b][j][c][:] = L0 + sum_u a_u K[b][cS+u][j][:] W_v
+ * W_L, W_q, W_k, W_v are d x d (row = input dim) in the dtype.  fp32 throughout,
+ * one rounding of L to the dtype.  The result replaces hsa_landmarks' output:
+ * pass it to hsa_select / hsa_forward (HSA_FLAG_LANDMARKS_READY).  Needs no
+ * workspace; one launch.  HSA_FLAG_QUEST is rejected (HSA_ERR_INVALID_ARG).
+ * hsa_backward differentiates the plain landmark only and does not apply.
+ */
+HSA_API hsa_status_t hsa_landmarks_refined(const hsa_problem_t *p, const void *K, const void *W_L, const void *W_q,
+                                           const void *W_k, const void *W_v, void *L, void *stream);
 
 /*
  * One step of a decode loop on a cache that grows in place (summary page,

@@ -20,7 +20,8 @@ import torch
 from . import _native
 from ._native import HSAError, hsa_problem_t
 
-__all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "select", "select_noalloc", "attend",
+__all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "landmarks_refined",
+           "quest_summaries", "select", "select_noalloc", "attend",
            "forward", "decode_append", "attend_partials", "merge_partials", "device_status", "HSAError",
            "hsa_problem_t", "kmax_of", "backward", "backward_workspace_size"]
 
@@ -94,6 +95,34 @@ def landmarks(K: torch.Tensor, W_L: torch.Tensor, S: int, L: torch.Tensor | None
     return L
 
 
+def landmarks_refined(K: torch.Tensor, W_L: torch.Tensor, W_q: torch.Tensor, W_k: torch.Tensor, W_v: torch.Tensor,
+                      S: int, L: torch.Tensor | None = None, kv_len: int | None = None) -> torch.Tensor:
+    """Refined landmarks [B,Hkv,Tcap//S,d]: the pooled landmark L0 = mean(K_c) W_L plus one head of
+    cross-attention from it to the chunk's keys, softmax((L0 W_q)(K_c W_k)^T / sqrt(d)) K_c W_v."""
+    _dev(K, W_L, W_q, W_k, W_v, L)
+    B, Tcap, Hkv, d = K.shape
+    Tkv = Tcap if kv_len is None else kv_len
+    if L is None:
+        L = torch.empty(B, Hkv, Tcap // S, d, dtype=K.dtype, device=K.device)
+    prob = make_problem(B, 0, Tkv, Hkv, Hkv, d, S, 1, 0, 0.0, K.dtype, kv_cap=Tcap)
+    _native.check(_native.lib().hsa_landmarks_refined(ctypes.byref(prob), _p(K), _p(W_L), _p(W_q), _p(W_k), _p(W_v),
+                                                      _p(L), _stream(K)), "hsa_landmarks_refined")
+    return L
+
+
+def quest_summaries(K: torch.Tensor, S: int, Lq: torch.Tensor | None = None, kv_len: int | None = None) -> torch.Tensor:
+    """Quest chunk summaries Lq [B,Hkv,Tcap//S,2d]: the channel-wise max of each complete chunk's
+    keys, then the channel-wise min (hsa_landmarks under HSA_FLAG_QUEST)."""
+    _dev(K, Lq)
+    B, Tcap, Hkv, d = K.shape
+    Tkv = Tcap if kv_len is None else kv_len
+    if Lq is None:
+        Lq = torch.empty(B, Hkv, Tcap // S, 2 * d, dtype=K.dtype, device=K.device)
+    prob = make_problem(B, 0, Tkv, Hkv, Hkv, d, S, 1, 0, 0.0, K.dtype, _native.HSA_FLAG_QUEST, kv_cap=Tcap)
+    _native.check(_native.lib().hsa_landmarks(ctypes.byref(prob), _p(K), None, _p(Lq), _stream(K)), "hsa_landmarks")
+    return Lq
+
+
 def _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags=0, kv_cap=0):
     B, Tq, H, d = Q.shape
     return make_problem(B, Tq, Tkv, H, Hkv, d, S, k, q_pos0, tau, Q.dtype, flags, kv_cap)
@@ -104,13 +133,15 @@ def _l_cap(Tkv, Ccap, S):
     return max(Tkv, Ccap * S)
 
 
-def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False):
-    """Top-k chunk selection.  Returns (idx int32, score fp32 [B,Tq,Hkv,kmax], keff int32 [B,Tq,Hkv])."""
+def select(Q, L, S, k, tau=0.0, q_pos0=0, Tkv=None, ws=None, force_simt=False, quest=False):
+    """Top-k chunk selection.  Returns (idx int32, score fp32 [B,Tq,Hkv,kmax], keff int32 [B,Tq,Hkv]).
+    quest: L holds Quest chunk summaries [B,Hkv,C,2d] and the scores are Quest's bounds."""
     _dev(Q, L, ws)
     B, Tq, H, d = Q.shape
     Hkv, C = L.shape[1], L.shape[2]
     Tkv = Tkv if Tkv is not None else C * S
-    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, _native.HSA_FLAG_SIMT if force_simt else 0, _l_cap(Tkv, C, S))
+    flags = (_native.HSA_FLAG_SIMT if force_simt else 0) | (_native.HSA_FLAG_QUEST if quest else 0)
+    prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags, _l_cap(Tkv, C, S))
     km = kmax_of(k, tau)
     idx = torch.empty(B, Tq, Hkv, km, dtype=torch.int32, device=Q.device)
     score = torch.empty(B, Tq, Hkv, km, dtype=torch.float32, device=Q.device)
@@ -161,21 +192,30 @@ def attend(Q, K, V, idx, score, keff, S, k, tau=0.0, q_pos0=0, O=None, ws=None, 
 
 
 def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False, O=None, ws=None,
-            return_selection=False, force_simt=False, kv_len=None):
+            return_selection=False, force_simt=False, kv_len=None, quest=False, refine=None):
     """The whole HSA forward.  Returns O, or (O, L, idx, score, keff) with return_selection.
     force_simt runs the CUDA-core kernels even where tensor-core ones exist (for A/B tests).
     kv_len: cached tokens when the K/V buffers (and L) hold more, as in a decode loop (default:
-    all of K.shape[1]); L is then [B, Hkv, K.shape[1] // S, d]."""
+    all of K.shape[1]); L is then [B, Hkv, K.shape[1] // S, d].
+    quest: Quest block scoring (L = chunk summaries [.., 2d], W_L unused).
+    refine: (W_q, W_k, W_v) -- the landmarks are the refined ones (hsa_landmarks_refined), then
+    the forward runs on them."""
     _dev(Q, K, V, W_L, L, O, ws)
     B, Tq, H, d = Q.shape
     Tcap, Hkv = K.shape[1], K.shape[2]
     Tkv = Tcap if kv_len is None else kv_len
-    flags = (_native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0) | (_native.HSA_FLAG_SIMT if force_simt else 0)
+    if refine is not None:
+        if quest or landmarks_ready:
+            raise ValueError("refine makes the landmarks: not with quest or landmarks_ready")
+        L = landmarks_refined(K, W_L, *refine, S, L=L, kv_len=kv_len)
+        landmarks_ready = True
+    flags = ((_native.HSA_FLAG_LANDMARKS_READY if landmarks_ready else 0) |
+             (_native.HSA_FLAG_SIMT if force_simt else 0) | (_native.HSA_FLAG_QUEST if quest else 0))
     prob = _prob_from(Q, Tkv, Hkv, S, k, tau, q_pos0, flags, Tcap)
     if L is None:
         if landmarks_ready:
             raise ValueError("landmarks_ready needs L")
-        L = torch.empty(B, Hkv, Tcap // S, d, dtype=Q.dtype, device=Q.device)
+        L = torch.empty(B, Hkv, Tcap // S, 2 * d if quest else d, dtype=Q.dtype, device=Q.device)
     if O is None:
         O = torch.empty_like(Q)
     if ws is None:
@@ -194,14 +234,16 @@ def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False
     return O
 
 
-def decode_append(K, V, k_new, v_new, kv_len, S, W_L=None, L=None) -> bool:
+def decode_append(K, V, k_new, v_new, kv_len, S, W_L=None, L=None, quest=False) -> bool:
     """One decode step's cache update: K[:, kv_len] = k_new and V[:, kv_len] = v_new
     (k_new, v_new [B, Hkv, d]; K, V [B, Tcap, Hkv, d] with kv_len < Tcap), and, when that
-    completes a chunk, its landmark into L [B, Hkv, Tcap // S, d].  Returns whether a chunk
-    was completed (W_L and L are needed then)."""
+    completes a chunk, its landmark into L [B, Hkv, Tcap // S, d] (quest: its Quest summary
+    into L [B, Hkv, Tcap // S, 2d]).  Returns whether a chunk was completed (L, and W_L unless
+    quest, are needed then)."""
     _dev(K, V, k_new, v_new, W_L, L)
     B, Tcap, Hkv, d = K.shape
-    prob = make_problem(B, 1, kv_len, Hkv, Hkv, d, S, 1, kv_len, 0.0, K.dtype, 0, Tcap)
+    prob = make_problem(B, 1, kv_len, Hkv, Hkv, d, S, 1, kv_len, 0.0, K.dtype,
+                        _native.HSA_FLAG_QUEST if quest else 0, Tcap)
     _native.check(_native.lib().hsa_decode_append(ctypes.byref(prob), _p(k_new), _p(v_new), _p(K), _p(V),
                                                    _p(W_L), _p(L), _stream(K)), "hsa_decode_append")
     return (kv_len + 1) % S == 0

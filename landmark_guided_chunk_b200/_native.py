@@ -16,11 +16,13 @@ HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_WORKSPACE, HSA_ERR_CUD
 HSA_F32, HSA_BF16 = 0, 1
 HSA_FLAG_LANDMARKS_READY = 1
 HSA_FLAG_SIMT = 2
+HSA_FLAG_TEST_STALL = 4
+HSA_FLAG_QUEST = 8
 
 EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version",
             "hsa_select_noalloc", "hsa_decode_append", "hsa_attend_partials", "hsa_merge_partials",
-            "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status")
+            "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status", "hsa_landmarks_refined")
 PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor", 4: "mma_split"}
 
 
@@ -70,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.hsa_attend_partials.argtypes = [prob, P, P, P, I32p, I32p, Fp, P, Z, P]
     L.hsa_merge_partials.argtypes = [prob, ctypes.c_int, Fp, I32p, I32p, Fp, P, I32p, Fp, I32p, P]
     L.hsa_noalloc_status.argtypes = [P]
+    L.hsa_landmarks_refined.argtypes = [prob, P, P, P, P, P, P, P]
     L.hsa_backward_workspace_size.argtypes = [prob, ctypes.POINTER(ctypes.c_size_t)]
     L.hsa_backward.argtypes = [prob, P, P, P, P, P, I32p, Fp, I32p, P, Fp, Fp, Fp, Fp, P, Z, P]
     L.hsa_status_string.argtypes = [ctypes.c_int]
@@ -81,7 +84,7 @@ def lib() -> ctypes.CDLL:
     for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
               "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc", "hsa_decode_append",
               "hsa_attend_partials", "hsa_merge_partials", "hsa_backward_workspace_size", "hsa_backward",
-              "hsa_noalloc_status"):
+              "hsa_noalloc_status", "hsa_landmarks_refined"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

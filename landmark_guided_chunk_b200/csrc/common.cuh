@@ -56,6 +56,8 @@ struct WsLayout {
     bool split_select, mma_select, stream_select, split_attend, gather_attend, tc_select, tc_attend;
     int stream_grid, stream_maxe;   // stream scan: CTAs and list slots per row
     AttTcLayout att;
+    bool quest;          // Quest scoring: the select fields above describe quest_select_view(p)
+    size_t quest_q;      // Quest scoring: the transformed query rows (quest_qprep_bytes)
     size_t att_w8, att_pairs, att_pair_w, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
 };
@@ -294,6 +296,16 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
                              cudaStream_t st);
 
 cudaError_t launch_landmarks(const Prob &p, const void *K, const void *W, void *L, cudaStream_t st);
+
+// Selection variants (variants.cu): the landmark refiner and Quest scoring.
+cudaError_t launch_landmarks_refined(const Prob &p, const void *K, const void *WL, const void *Wq, const void *Wk,
+                                     const void *Wv, void *L, cudaStream_t st);
+cudaError_t launch_quest_summaries(const Prob &p, const void *K, void *Lq, cudaStream_t st);
+cudaError_t launch_quest_summary_chunk(const Prob &p, const void *K, void *Lq, int c, cudaStream_t st);
+// The problem the selection kernels see under Quest scoring: d' = 2d, G' = 2 (bf16) or 1 (fp32).
+Prob quest_select_view(const Prob &p);
+size_t quest_qprep_bytes(const Prob &p);
+cudaError_t launch_quest_qprep(const Prob &p, const void *Q, void *Qp, cudaStream_t st);
 
 // Backward (backward.cu): workspace layout, support check, kernel count, launch.
 struct BwdLayout {

@@ -40,6 +40,11 @@ static int device_sms() {
 
 WsLayout ws_layout(const Prob &p) {
     WsLayout w{};
+    // Under Quest scoring the selection kernels run on a transformed problem
+    // (query rows [P | N], landmarks = chunk summaries, width 2d); every select
+    // decision below is taken on that view.
+    w.quest = (p.flags & HSA_FLAG_QUEST) != 0;
+    const Prob ps = w.quest ? quest_select_view(p) : p;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -53,11 +58,11 @@ WsLayout ws_layout(const Prob &p) {
     // G <= 8, kmax <= 16) one CTA per SM streams its share of all rows' landmarks
     // through a TMA ring; otherwise in bf16 with G <= 8 (split) CTAs score with
     // the tensor cores and fold the merge in.  Otherwise one warp per row.
-    w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(p);
+    w.tc_select = rows > 0 && !(p.flags & HSA_FLAG_SIMT) && select_tc_supported(ps);
     w.split_select = !w.tc_select && rows > 0 && rows <= 4096 && p.C >= 2048;
-    w.stream_select = w.split_select && !(p.flags & HSA_FLAG_SIMT) && select_stream_supported(p);
-    w.mma_select = w.split_select && !w.stream_select && !(p.flags & HSA_FLAG_SIMT) && select_mma_supported(p);
-    if (w.stream_select) select_stream_shape(p, device_sms(), &w.stream_grid, &w.stream_maxe);
+    w.stream_select = w.split_select && !(p.flags & HSA_FLAG_SIMT) && select_stream_supported(ps);
+    w.mma_select = w.split_select && !w.stream_select && !(p.flags & HSA_FLAG_SIMT) && select_mma_supported(ps);
+    if (w.stream_select) select_stream_shape(ps, device_sms(), &w.stream_grid, &w.stream_maxe);
     // Few rows: the kept slots are spread over CTAs too (split attend); in bf16
     // the gather kernel does it in one launch.
     w.split_attend = rows > 0 && rows <= 2048;
@@ -74,6 +79,7 @@ WsLayout ws_layout(const Prob &p) {
     w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
     w.sel_score = take(rows * p.kmax * sizeof(float));
     w.sel_keff = take(rows * sizeof(int32_t));
+    if (w.quest) w.quest_q = take(quest_qprep_bytes(p));
     if (w.split_select) {
         const long long target = 148 * 8;
         long long per_row = (target + (long long)rows - 1) / (long long)rows;
@@ -108,7 +114,7 @@ WsLayout ws_layout(const Prob &p) {
                          : w.tc_select  ? HSA_PATH_TENSOR
                          : (w.stream_select || w.mma_select) ? HSA_PATH_MMA_SPLIT
                          : (w.split_select ? HSA_PATH_SIMT_SPLIT : HSA_PATH_SIMT_ROWS);
-    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select && !w.stream_select ? 2 : 1);
+    w.plan.select_kernels = rows == 0 ? 0 : (w.split_select && !w.mma_select && !w.stream_select ? 2 : 1) + (w.quest ? 1 : 0);
     w.plan.attend_path = rows == 0 ? HSA_PATH_NONE
                          : w.tc_attend  ? HSA_PATH_TENSOR
                          : w.gather_attend ? HSA_PATH_MMA_SPLIT
@@ -131,7 +137,7 @@ hsa_status_t validate(const hsa_problem_t *in, Prob *p) {
     if (in->dtype != HSA_F32 && in->dtype != HSA_BF16) return fail(HSA_ERR_INVALID_ARG, "unknown dtype %d", in->dtype);
     if (!(in->tau >= 0.0f) || isinf(in->tau)) return fail(HSA_ERR_INVALID_ARG, "tau must be finite and >= 0");
     if (in->q_pos0 < 0) return fail(HSA_ERR_INVALID_ARG, "q_pos0 must be >= 0");
-    if (in->flags & ~(HSA_FLAG_LANDMARKS_READY | HSA_FLAG_SIMT))
+    if (in->flags & ~(HSA_FLAG_LANDMARKS_READY | HSA_FLAG_SIMT | HSA_FLAG_TEST_STALL | HSA_FLAG_QUEST))
         return fail(HSA_ERR_INVALID_ARG, "unknown flags 0x%x", in->flags);
     if (in->d != 64 && in->d != 128) return fail(HSA_ERR_UNSUPPORTED, "d=%d (supported: 64, 128)", in->d);
     if (in->S != 32 && in->S != 64 && in->S != 128)
@@ -185,6 +191,25 @@ static hsa_status_t check_ws(const WsLayout &w, void *ws, size_t ws_bytes) {
     return HSA_OK;
 }
 
+// The selection stage as the caller's problem asks: under Quest scoring the
+// query rows are transformed into the workspace first and the selection
+// kernels run on the transformed problem.
+static cudaError_t run_selection(const Prob &p, const WsLayout &w, const void *Q, const void *L, int32_t *idx,
+                                 float *score, int32_t *keff, char *ws, cudaStream_t st) {
+    if (!w.quest) return launch_select(p, w, Q, L, idx, score, keff, ws, st);
+    if (p.rows == 0) return cudaSuccess;
+    void *Qp = ws + w.quest_q;
+    cudaError_t e = launch_quest_qprep(p, Q, Qp, st);
+    if (e != cudaSuccess) return e;
+    return launch_select(quest_select_view(p), w, Qp, L, idx, score, keff, ws, st);
+}
+
+// Landmarks, or the Quest chunk summaries under HSA_FLAG_QUEST.
+static cudaError_t run_landmarks(const Prob &p, const void *K, const void *W_L, void *L, cudaStream_t st) {
+    if (p.flags & HSA_FLAG_QUEST) return launch_quest_summaries(p, K, L, st);
+    return launch_landmarks(p, K, W_L, L, st);
+}
+
 static hsa_status_t clear_status(char *ws, const WsLayout &w, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(ws, 0, w.clear_bytes, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "clearing the device-status word");
@@ -233,10 +258,26 @@ hsa_status_t hsa_landmarks(const hsa_problem_t *prob, const void *K, const void 
     HSA_TRY(validate(prob, &p));
     const bool any = (long long)p.B * p.C > 0;
     HSA_TRY(need(K, any, "K"));
-    HSA_TRY(need(W_L, any, "W_L"));
+    HSA_TRY(need(W_L, any && !(p.flags & HSA_FLAG_QUEST), "W_L"));
     HSA_TRY(need(L, any, "L"));
-    cudaError_t e = launch_landmarks(p, K, W_L, L, (cudaStream_t)stream);
+    cudaError_t e = run_landmarks(p, K, W_L, L, (cudaStream_t)stream);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "landmark kernel launch");
+}
+
+hsa_status_t hsa_landmarks_refined(const hsa_problem_t *prob, const void *K, const void *W_L, const void *W_q,
+                                   const void *W_k, const void *W_v, void *L, void *stream) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (p.flags & HSA_FLAG_QUEST) return fail(HSA_ERR_INVALID_ARG, "the refiner makes landmarks, not Quest summaries");
+    const bool any = (long long)p.B * p.C > 0;
+    HSA_TRY(need(K, any, "K"));
+    HSA_TRY(need(W_L, any, "W_L"));
+    HSA_TRY(need(W_q, any, "W_q"));
+    HSA_TRY(need(W_k, any, "W_k"));
+    HSA_TRY(need(W_v, any, "W_v"));
+    HSA_TRY(need(L, any, "L"));
+    cudaError_t e = launch_landmarks_refined(p, K, W_L, W_q, W_k, W_v, L, (cudaStream_t)stream);
+    return e == cudaSuccess ? HSA_OK : cuda_fail(e, "refined landmark kernel launch");
 }
 
 hsa_status_t hsa_decode_append(const hsa_problem_t *prob, const void *k_new, const void *v_new, void *K, void *V,
@@ -251,9 +292,19 @@ hsa_status_t hsa_decode_append(const hsa_problem_t *prob, const void *k_new, con
     HSA_TRY(need(v_new, any, "v_new"));
     HSA_TRY(need(K, any, "K"));
     HSA_TRY(need(V, any, "V"));
-    HSA_TRY(need(W_L, completes, "W_L"));
+    const bool quest = (p.flags & HSA_FLAG_QUEST) != 0;
+    HSA_TRY(need(W_L, completes && !quest, "W_L"));
     HSA_TRY(need(L, completes, "L"));
-    cudaError_t e = launch_decode_append(p, k_new, v_new, K, V, W_L, L, (cudaStream_t)stream);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (quest) {
+        // the append alone, then the completed chunk's summary (stream-ordered after the append)
+        Prob pa = p;
+        pa.S = p.Tcap + 1;   // no chunk completes for the append kernel
+        cudaError_t e = launch_decode_append(pa, k_new, v_new, K, V, nullptr, nullptr, st);
+        if (e == cudaSuccess && completes) e = launch_quest_summary_chunk(p, K, L, (p.Tkv + 1) / p.S - 1, st);
+        return e == cudaSuccess ? HSA_OK : cuda_fail(e, "decode append kernel launch");
+    }
+    cudaError_t e = launch_decode_append(p, k_new, v_new, K, V, W_L, L, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "decode append kernel launch");
 }
 
@@ -271,7 +322,7 @@ hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L,
     HSA_TRY(check_ws(w, ws, ws_bytes));
     cudaStream_t st = (cudaStream_t)stream;
     HSA_TRY(clear_status((char *)ws, w, st));
-    cudaError_t e = launch_select(p, w, Q, L, idx, score, keff, (char *)ws, st);
+    cudaError_t e = run_selection(p, w, Q, L, idx, score, keff, (char *)ws, st);
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "selection kernel launch");
 }
 
@@ -350,7 +401,7 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     HSA_TRY(need(Q, rows, "Q"));
     HSA_TRY(need(K, (rows && p.C > 0) || (chunks && !ready), "K"));
     HSA_TRY(need(V, rows && p.C > 0, "V"));
-    HSA_TRY(need(W_L, chunks && !ready, "W_L"));
+    HSA_TRY(need(W_L, chunks && !ready && !(p.flags & HSA_FLAG_QUEST), "W_L"));
     HSA_TRY(need(L, chunks, "L"));
     if (idx && !aligned16(idx)) return fail(HSA_ERR_INVALID_ARG, "idx is not 16-byte aligned");
     if (score && !aligned16(score)) return fail(HSA_ERR_INVALID_ARG, "score is not 16-byte aligned");
@@ -363,13 +414,13 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     HSA_TRY(clear_status(wsb, w, st));
     cudaError_t e;
     if (!ready) {
-        e = launch_landmarks(p, K, W_L, L, st);
+        e = run_landmarks(p, K, W_L, L, st);
         if (e != cudaSuccess) return cuda_fail(e, "landmark kernel launch");
     }
     int32_t *sidx = idx ? idx : reinterpret_cast<int32_t *>(wsb + w.sel_idx);
     float *ssc = score ? score : reinterpret_cast<float *>(wsb + w.sel_score);
     int32_t *skf = keff ? keff : reinterpret_cast<int32_t *>(wsb + w.sel_keff);
-    e = launch_select(p, w, Q, L, sidx, ssc, skf, wsb, st);
+    e = run_selection(p, w, Q, L, sidx, ssc, skf, wsb, st);
     if (e != cudaSuccess) return cuda_fail(e, "selection kernel launch");
     e = launch_attend(p, w, Q, K, V, sidx, ssc, skf, O, wsb, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
@@ -379,6 +430,7 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
 hsa_status_t hsa_backward_workspace_size(const hsa_problem_t *prob, size_t *bytes) {
     Prob p;
     HSA_TRY(validate(prob, &p));
+    if (p.flags & HSA_FLAG_QUEST) return fail(HSA_ERR_UNSUPPORTED, "backward of Quest scoring is not implemented");
     if (!bytes) return fail(HSA_ERR_INVALID_ARG, "bytes is NULL");
     if (!backward_supported(p)) return fail(HSA_ERR_UNSUPPORTED, "backward: problem too large for 32-bit pair indices");
     *bytes = backward_layout(p).total;
@@ -390,6 +442,7 @@ hsa_status_t hsa_backward(const hsa_problem_t *prob, const void *Q, const void *
                           float *dQ, float *dK, float *dV, float *dW_L, void *ws, size_t ws_bytes, void *stream) {
     Prob p;
     HSA_TRY(validate(prob, &p));
+    if (p.flags & HSA_FLAG_QUEST) return fail(HSA_ERR_UNSUPPORTED, "backward of Quest scoring is not implemented");
     if (!backward_supported(p)) return fail(HSA_ERR_UNSUPPORTED, "backward: problem too large for 32-bit pair indices");
     const bool rows = p.rows > 0;
     const bool work = rows && p.C > 0;

@@ -47,6 +47,8 @@ extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, co
     Prob p;
     hsa_status_t s = validate(prob, &p);
     if (s != HSA_OK) return s;
+    if (p.flags & HSA_FLAG_QUEST)
+        return fail(HSA_ERR_UNSUPPORTED, "hsa_select_noalloc: Quest scoring needs a caller workspace (use hsa_select)");
     const bool rows = p.rows > 0;
     if ((s = need(Q, rows, "Q")) != HSA_OK) return s;
     if ((s = need(L, rows && p.C > 0, "L")) != HSA_OK) return s;

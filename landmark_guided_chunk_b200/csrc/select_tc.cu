@@ -45,11 +45,12 @@ namespace {
 using namespace sm100;
 
 constexpr int TM = 128;        // tokens per M-tile
-constexpr int NT = 128;        // chunks per N-slice
 constexpr int NSTAGE = 2;      // L-slice ring depth
-constexpr int BOX = 64 * 128 * 2;   // one 64-column x 128-row bf16 box (16 KB)
-constexpr uint32_t TMEM_COLS = 2 * NT;
+constexpr int BOX = 64 * 128 * 2;   // one 64-column x 128-row bf16 box of the query tile (16 KB)
 constexpr int MAX_KB = 8;      // G*d <= 512
+// Chunks per N-slice (NT): 128, or 64 when a landmark row has 256 columns, so
+// that the query tile and two slices still fit in shared memory.
+constexpr uint64_t TEST_STALL_WAIT_NS = 100000ull;   // wait limit under HSA_FLAG_TEST_STALL (0.1 ms)
 
 struct TcSelArgs {
     int B, Tq, Hkv, G, d, S, C, k, kmax;
@@ -59,10 +60,12 @@ struct TcSelArgs {
     long long q_pos0;
     float tau;
     uint32_t *status;
+    uint64_t wait_ns;        // limit of every bounded wait
+    int stall;               // test hook: the epilogue first waits on a barrier nothing arrives on
 };
 
 struct __align__(8) Bars {
-    uint64_t a_full[MAX_KB], a_empty[MAX_KB], done;
+    uint64_t a_full[MAX_KB], a_empty[MAX_KB], done, never;
     uint64_t b_full[NSTAGE], b_empty[NSTAGE];
     uint64_t t_full[2], t_empty[2];
     uint32_t tmem_base;
@@ -73,6 +76,7 @@ struct Tile {
     int b, j, t0, nc_max, nslices;
 };
 
+template <int NT>
 __device__ __forceinline__ Tile tile_of(const TcSelArgs &a, int tau) {
     Tile T;
     const int bh = a.B * a.Hkv;
@@ -88,6 +92,7 @@ __device__ __forceinline__ Tile tile_of(const TcSelArgs &a, int tau) {
     return T;
 }
 
+template <int NT>
 __device__ __forceinline__ int slice_n(const Tile &T, int n) {
     int w = min(NT, T.nc_max - n * NT);
     return (w + 15) & ~15;
@@ -120,16 +125,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
-template <int KL>
+template <int KL, int NT>
 __global__ void __launch_bounds__(256, 1)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmL,
                      int32_t *__restrict__ idx, float *__restrict__ score, int32_t *__restrict__ keff, TcSelArgs a) {
+    constexpr int BOXB = 64 * NT * 2;                     // one 64-column x NT-row box of a landmark slice
+    constexpr uint32_t TMEM_COLS = 2 * NT;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;                                   // nkb boxes
     uint8_t *sB = base + (size_t)a.nkb * BOX;             // NSTAGE x dkb boxes
     // [32][128] queued (score, chunk as int bits): one 8-byte store per queued candidate
-    float2 *qvi = reinterpret_cast<float2 *>(sB + (size_t)NSTAGE * a.dkb * BOX);
+    float2 *qvi = reinterpret_cast<float2 *>(sB + (size_t)NSTAGE * a.dkb * BOXB);
     Bars *bar = reinterpret_cast<Bars *>(qvi + 32 * 128);
     volatile int *abort = &bar->abort;
 
@@ -140,6 +147,7 @@ __global__ void __launch_bounds__(256, 1)
             mbar_init(&bar->a_empty[kb], 1);
         }
         mbar_init(&bar->done, 1);
+        mbar_init(&bar->never, 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bar->b_full[s], 1);
             mbar_init(&bar->b_empty[s], 1);
@@ -170,11 +178,11 @@ __global__ void __launch_bounds__(256, 1)
             int g = 0, ta = 0, kb_part = 0;   // kb_part: boxes issued of a tile cut short
             bool ok = true;
             for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
-                const Tile T = tile_of(a, tau);
+                const Tile T = tile_of<NT>(a, tau);
                 if (T.nslices == 0) continue;
                 const int y = T.b * a.Tq + T.t0;
                 for (int kb = 0; kb < a.nkb; ++kb) {
-                    if (ta > 0 && !(ok = mbar_wait(&bar->a_empty[kb], (ta - 1) & 1, abort, a.status))) break;
+                    if (ta > 0 && !(ok = mbar_wait(&bar->a_empty[kb], (ta - 1) & 1, abort, a.status, a.wait_ns))) break;
                     mbar_expect_tx(&bar->a_full[kb], (uint32_t)BOX);
                     tma_load_2d(sA + (size_t)kb * BOX, &tmQ, T.j * a.G * a.d + kb * 64, y, &bar->a_full[kb]);
                     kb_part = kb + 1;
@@ -185,10 +193,10 @@ __global__ void __launch_bounds__(256, 1)
                 const int ly = (T.b * a.Hkv + T.j) * a.Lc;
                 for (int n = 0; n < T.nslices; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE;
-                    if (i > 0 && !(ok = mbar_wait(&bar->b_empty[s], (i - 1) & 1, abort, a.status))) break;
-                    mbar_expect_tx(&bar->b_full[s], (uint32_t)(a.dkb * BOX));
+                    if (i > 0 && !(ok = mbar_wait(&bar->b_empty[s], (i - 1) & 1, abort, a.status, a.wait_ns))) break;
+                    mbar_expect_tx(&bar->b_full[s], (uint32_t)(a.dkb * BOXB));
                     for (int kd = 0; kd < a.dkb; ++kd)
-                        tma_load_2d(sB + (size_t)(s * a.dkb + kd) * BOX, &tmL, kd * 64, ly + n * NT, &bar->b_full[s]);
+                        tma_load_2d(sB + (size_t)(s * a.dkb + kd) * BOXB, &tmL, kd * 64, ly + n * NT, &bar->b_full[s]);
                 }
             }
             // wind down: every load issued has landed before the CTA may exit
@@ -207,25 +215,25 @@ __global__ void __launch_bounds__(256, 1)
             int g = 0, ta = 0;
             bool ok = true;
             for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
-                const Tile T = tile_of(a, tau);
+                const Tile T = tile_of<NT>(a, tau);
                 if (T.nslices == 0) continue;
                 const uint32_t pa = ta & 1;
                 ++ta;
                 for (int n = 0; n < T.nslices && ok; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE, buf = g & 1, u = g >> 1;
-                    if (!(ok = mbar_wait(&bar->b_full[s], i & 1, abort, a.status))) break;
-                    if (u > 0 && !(ok = mbar_wait(&bar->t_empty[buf], (u - 1) & 1, abort, a.status))) break;
+                    if (!(ok = mbar_wait(&bar->b_full[s], i & 1, abort, a.status, a.wait_ns))) break;
+                    if (u > 0 && !(ok = mbar_wait(&bar->t_empty[buf], (u - 1) & 1, abort, a.status, a.wait_ns))) break;
                     tc_fence_after();
-                    const uint32_t idesc = idesc_bf16_f32(TM, slice_n(T, n), 0, 0);
+                    const uint32_t idesc = idesc_bf16_f32(TM, slice_n<NT>(T, n), 0, 0);
                     const uint32_t d_tmem = tmem + (uint32_t)(buf * NT);
-                    const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB + (size_t)s * a.dkb * BOX);
+                    const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB + (size_t)s * a.dkb * BOXB);
                     const bool last = n == T.nslices - 1;
                     for (int kb = 0; kb < a.nkb; ++kb) {
                         if (n == 0) {
-                            if (!(ok = mbar_wait(&bar->a_full[kb], pa, abort, a.status))) break;
+                            if (!(ok = mbar_wait(&bar->a_full[kb], pa, abort, a.status, a.wait_ns))) break;
                             tc_fence_after();
                         }
-                        const uint32_t aK = aBase + kb * BOX, bK = bBase + (kb % a.dkb) * BOX;
+                        const uint32_t aK = aBase + kb * BOX, bK = bBase + (kb % a.dkb) * BOXB;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_bf16(d_tmem, desc_kmajor_sw128(aK + kk * 32), desc_kmajor_sw128(bK + kk * 32), idesc,
@@ -246,9 +254,11 @@ __global__ void __launch_bounds__(256, 1)
         const int r = ew * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(ew * 32) << 16);
         int g = 0;
-        bool ok = true;
+        // test hook: a wait that runs out (nothing arrives on `never`), so the
+        // expiry, abort and wind-down of every role run as they would on a stall
+        bool ok = !a.stall || mbar_wait(&bar->never, 0, abort, a.status, a.wait_ns);
         for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
-            const Tile T = tile_of(a, tau);
+            const Tile T = tile_of<NT>(a, tau);
             const int t = T.t0 + r;
             const bool valid = t < a.Tq;
             int nc = 0;
@@ -266,9 +276,9 @@ __global__ void __launch_bounds__(256, 1)
             int head = 0, tail = 0;   // this row's FIFO of pending (score, chunk): ring of 32 in qvi
             for (int n = 0; n < T.nslices; ++n, ++g) {
                 const int buf = g & 1, u = g >> 1;
-                if (!(ok = mbar_wait(&bar->t_full[buf], u & 1, abort, a.status))) break;
+                if (!(ok = mbar_wait(&bar->t_full[buf], u & 1, abort, a.status, a.wait_ns))) break;
                 tc_fence_after();
-                const int nch = slice_n(T, n) / 16;
+                const int nch = slice_n<NT>(T, n) / 16;
                 const bool last_slice = n == T.nslices - 1;
                 for (int q = 0; q < nch; ++q) {
                     uint32_t rr[16];
@@ -341,21 +351,32 @@ __global__ void __launch_bounds__(256, 1)
     }
 }
 
-template <int KL>
+template <int KL, int NT>
 cudaError_t launch_kl(const TcSelArgs &a, const CUtensorMap &mq, const CUtensorMap &ml, int32_t *idx, float *score,
                       int32_t *keff, int grid, size_t smem, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(select_tc_kernel<KL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(select_tc_kernel<KL, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    select_tc_kernel<KL><<<grid, 256, smem, st>>>(mq, ml, idx, score, keff, a);
+    select_tc_kernel<KL, NT><<<grid, 256, smem, st>>>(mq, ml, idx, score, keff, a);
     return cudaGetLastError();
+}
+
+template <int NT>
+cudaError_t launch_nt(const Prob &p, const TcSelArgs &a, const CUtensorMap &mq, const CUtensorMap &ml, int32_t *idx,
+                      float *score, int32_t *keff, int grid, cudaStream_t st) {
+    const size_t smem =
+        1024 + (size_t)a.nkb * BOX + (size_t)NSTAGE * a.dkb * (64 * NT * 2) + 2 * 32 * 128 * 4 + sizeof(Bars);
+    if (p.kmax <= 8) return launch_kl<8, NT>(a, mq, ml, idx, score, keff, grid, smem, st);
+    if (p.kmax <= 16) return launch_kl<16, NT>(a, mq, ml, idx, score, keff, grid, smem, st);
+    return launch_kl<32, NT>(a, mq, ml, idx, score, keff, grid, smem, st);
 }
 
 }  // namespace
 
 bool select_tc_supported(const Prob &p) {
     const int gd = p.G * p.d;
-    return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && gd % 64 == 0 && gd <= 512 && p.Tq >= 64 &&
-           p.C >= 1 && p.kmax <= 32;
+    return p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128 || p.d == 256) && gd % 64 == 0 && gd <= 512 &&
+           p.Tq >= 64 && p.C >= 1 && p.kmax <= 32;
 }
 
 cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score, int32_t *keff,
@@ -363,7 +384,8 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
     CUtensorMap mq, ml;
     cudaError_t e = make_tmap_2d(&mq, Q, (uint64_t)p.H * p.d, (uint64_t)p.B * p.Tq, 64, TM);
     if (e != cudaSuccess) return e;
-    e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, NT);
+    const int nt = p.d > 128 ? 64 : 128;   // chunks per N-slice
+    e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, (uint32_t)nt);
     if (e != cudaSuccess) return e;
     TcSelArgs a;
     a.B = p.B;
@@ -383,14 +405,14 @@ cudaError_t launch_select_tc(const Prob &p, const void *Q, const void *L, int32_
     a.q_pos0 = p.q_pos0;
     a.tau = p.tau;
     a.status = status;
+    a.stall = (p.flags & HSA_FLAG_TEST_STALL) ? 1 : 0;
+    a.wait_ns = a.stall ? TEST_STALL_WAIT_NS : WAIT_LIMIT_NS;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = a.ntiles < sms ? a.ntiles : sms;
-    const size_t smem = 1024 + (size_t)a.nkb * BOX + (size_t)NSTAGE * a.dkb * BOX + 2 * 32 * 128 * 4 + sizeof(Bars);
-    if (p.kmax <= 8) return launch_kl<8>(a, mq, ml, idx, score, keff, grid, smem, st);
-    if (p.kmax <= 16) return launch_kl<16>(a, mq, ml, idx, score, keff, grid, smem, st);
-    return launch_kl<32>(a, mq, ml, idx, score, keff, grid, smem, st);
+    if (nt == 64) return launch_nt<64>(p, a, mq, ml, idx, score, keff, grid, st);
+    return launch_nt<128>(p, a, mq, ml, idx, score, keff, grid, st);
 }
 
 }  // namespace hsa

@@ -74,14 +74,16 @@ constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s: far beyond any legit
 constexpr uint32_t SUSPEND_NS = 200000u;             // longest single suspension inside a wait (0.2 ms)
 
 // Wait until the phase with `parity` of *bar has completed.  Returns false (and
-// leaves *abort set) if the CTA is aborting or the limit expired.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+// leaves *abort set) if the CTA is aborting or `limit_ns` expired (the check
+// runs between suspensions, so the limit is rounded up to SUSPEND_NS).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status,
+                                          uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_suspend(bar, parity, SUSPEND_NS)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort = 1;
             atomicOr(status, DEV_TIMEOUT);
             return false;

@@ -101,6 +101,20 @@ def check_selection(idx, score, keff, orc_sel: dict, ncand: np.ndarray, k: int, 
     return {"exact": exact, "ties": ties, "tie_rows": tie_rows}
 
 
+def selection_mismatch_rate(idx, keff, orc_sel) -> float:
+    """Fraction of (row, kv head) selections whose kept SET differs from the
+    oracle's (idx/keff: GPU outputs flattened to [n, Hkv, kmax] / [n, Hkv])."""
+    idx, keff = np.asarray(idx), np.asarray(keff)
+    n, Hkv, _ = idx.shape
+    bad = 0
+    for r in range(n):
+        for j in range(Hkv):
+            ke, oke = int(keff[r, j]), int(orc_sel["keff"][r, j])
+            if ke != oke or set(idx[r, j, :ke].tolist()) != set(orc_sel["idx"][r, j, :oke].tolist()):
+                bad += 1
+    return bad / max(1, n * Hkv)
+
+
 def expected_output(Qr, row_b, K, V, S, orc_sel, idx, keff, tie_rows):
     """Oracle output for the oracle selection, with the validated GPU selection
     substituted in the near-tie rows."""

@@ -52,7 +52,7 @@ def torch_bf16():
     (dict(tau=float("nan")), _native.HSA_ERR_INVALID_ARG),
     (dict(tau=float("inf")), _native.HSA_ERR_INVALID_ARG),
     (dict(q_pos0=-3), _native.HSA_ERR_INVALID_ARG),
-    (dict(flags=8), _native.HSA_ERR_INVALID_ARG),
+    (dict(flags=64), _native.HSA_ERR_INVALID_ARG),
     (dict(d=96), _native.HSA_ERR_UNSUPPORTED),
     (dict(S=48), _native.HSA_ERR_UNSUPPORTED),
     (dict(k=33), _native.HSA_ERR_UNSUPPORTED),
@@ -152,3 +152,22 @@ def test_backward_workspace_and_validation_before_launch():
     assert _call_backward(p, ws_bytes=16) == _native.HSA_ERR_WORKSPACE
     assert _call_backward(p, ws=256 + 16) == _native.HSA_ERR_WORKSPACE        # not 256-byte aligned
     assert _call_backward(_prob(H=5)) == _native.HSA_ERR_INVALID_ARG
+
+
+def test_quest_flag_host_rules():
+    """Quest scoring: the workspace holds the transformed query rows, the plan adds
+    their kernel, and the calls that do not implement it refuse before launching."""
+    plain, quest = _prob(), _prob(flags=_native.HSA_FLAG_QUEST)
+    assert hsa.workspace_size(quest) >= hsa.workspace_size(plain) + 128 * 2 * 2 * 2 * 64 * 2
+    assert hsa.plan(quest)["select"][1] == hsa.plan(plain)["select"][1] + 1
+    n = ctypes.c_size_t(0)
+    assert _native.lib().hsa_backward_workspace_size(ctypes.byref(quest), ctypes.byref(n)) == \
+        _native.HSA_ERR_UNSUPPORTED
+    fake = ctypes.c_void_p(256)
+    assert _native.lib().hsa_select_noalloc(ctypes.byref(quest), fake, fake, fake, fake, fake, None) == \
+        _native.HSA_ERR_UNSUPPORTED
+    assert _native.lib().hsa_landmarks_refined(ctypes.byref(quest), fake, fake, fake, fake, fake, fake, None) == \
+        _native.HSA_ERR_INVALID_ARG
+    # the refiner needs every weight
+    assert _native.lib().hsa_landmarks_refined(ctypes.byref(plain), fake, fake, fake, None, fake, fake, None) == \
+        _native.HSA_ERR_INVALID_ARG

@@ -65,3 +65,29 @@ def test_noalloc_select_rejects_a_problem_beyond_its_scratch():
     rc = _native.lib().hsa_select_noalloc(ctypes.byref(prob), fake, fake, fake, fake, fake, None)
     assert rc == _native.HSA_ERR_WORKSPACE
     assert b"static scratch" in _native.lib().hsa_last_error()
+
+
+def test_noalloc_timeout_is_reported_by_its_status_reader():
+    """A device-side timeout inside hsa_select_noalloc lands in the static
+    scratch's status word; hsa_noalloc_status reports it (the test flag makes
+    the scoring kernel's wait run out, see tests/test_failure_gpu.py), and the
+    next call is clean and equal to hsa_select."""
+    torch.cuda.set_device(0)
+    p = CASES[1]
+    inp = make_inputs(p, seed=12, device="cuda")
+    Q, K, W = inp["Q"], inp["K"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    st = torch.cuda.current_stream().cuda_stream
+    ref_idx, ref_score, ref_keff = hsa.select(Q, L, p.S, p.k, p.tau, p.q_pos0, Tkv=p.Tkv)
+    out = (torch.empty_like(ref_idx), torch.empty_like(ref_score), torch.empty_like(ref_keff))
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, Q.dtype,
+                            _native.HSA_FLAG_TEST_STALL)
+    rc = _native.lib().hsa_select_noalloc(ctypes.byref(prob), ctypes.c_void_p(Q.data_ptr()),
+                                          ctypes.c_void_p(L.data_ptr()), ctypes.c_void_p(out[0].data_ptr()),
+                                          ctypes.c_void_p(out[1].data_ptr()), ctypes.c_void_p(out[2].data_ptr()), st)
+    assert rc == _native.HSA_OK
+    assert _native.lib().hsa_noalloc_status(st) == _native.HSA_ERR_TIMEOUT
+    assert _native.lib().hsa_noalloc_status(st) == _native.HSA_OK   # read and cleared
+    assert _noalloc_call(p, Q, L, out) == _native.HSA_OK
+    assert _native.lib().hsa_noalloc_status(st) == _native.HSA_OK
+    assert torch.equal(out[0], ref_idx) and torch.equal(out[2], ref_keff) and torch.equal(out[1], ref_score)
