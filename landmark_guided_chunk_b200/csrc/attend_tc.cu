@@ -47,8 +47,8 @@ constexpr int D = 128;           // head dim of this kernel
 constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
 constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
-constexpr int TB = 4096;         // tokens per phase
-constexpr int NB = 2;            // phases per batch (= per launch)
+constexpr int TB = 16384;        // tokens per phase (larger phases fill the per-chunk tiles better)
+constexpr int NB = 1;            // phases per batch (= per launch)
 constexpr int NT_ATT = 512;      // warps 0-1 Q producers, 2 MMA, 3 K/V loader, 4-7 softmax, 8-15 O drain
 constexpr int NPROD = 64;        // producer threads (two tile rows each)
 

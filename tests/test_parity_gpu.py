@@ -297,3 +297,26 @@ def test_attend_skips_and_reports_out_of_range_selection():
         hsa.device_status(ws)
     hsa.attend(Q, K, V, idx, sc, ke, p.S, p.k, ws=ws)
     hsa.device_status(ws)
+
+
+@pytest.mark.parametrize("nchunks", [1000, 5000])
+def test_scoring_prefill_continuation_over_a_long_context(nchunks):
+    """A prefill continuation (128 new queries after a long cached context) on the
+    tcgen05 scoring kernel: few M-tiles, each scanning thousands of chunks in many
+    N-slices.  Checked on every row."""
+    p = Problem(B=1, Tq=128, Tkv=64 * nchunks + 7, H=8, Hkv=2, d=128, S=64, k=16, tau=0.0,
+                q_pos0=64 * nchunks + 7 - 128, dtype="bf16")
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, torch.bfloat16)
+    assert hsa.plan(prob)["select"][0] == "tensor"
+    inp = make_inputs(p, seed=13, device="cuda")
+    Q, K, W = inp["Q"], inp["K"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    idx, score, keff = hsa.select(Q, L, p.S, p.k, p.tau, p.q_pos0, Tkv=p.Tkv)
+    torch.cuda.synchronize()
+    rb, rt = _rows_all(p)
+    orc = oracle.select(Q.cpu().reshape(p.B * p.Tq, p.H, p.d), rb, rt + p.q_pos0, L.double().cpu().numpy(), p.S,
+                        p.k, p.tau, p.H, want_all=True)
+    ncand = np.minimum((rt + p.q_pos0) // p.S, p.C)
+    sel = parity.check_selection(idx.reshape(-1, p.Hkv, p.k).cpu().numpy(), score.reshape(-1, p.Hkv, p.k).cpu().numpy(),
+                                 keff.reshape(-1, p.Hkv).cpu().numpy(), orc, ncand, p.k, p.tau)
+    assert sel["ties"] <= max(2, sel["exact"] // 100)
