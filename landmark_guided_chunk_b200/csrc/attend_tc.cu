@@ -47,7 +47,7 @@ constexpr int D = 128;           // head dim of this kernel
 constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
 constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
-constexpr int TB = 16384;        // tokens per phase (larger phases fill the per-chunk tiles better)
+constexpr int TB = 16384;        // tokens per phase (larger phases fill the per-chunk tiles better; a multiple of HT)
 constexpr int NB = 1;            // phases per batch (= per launch)
 constexpr int NT_ATT = 512;      // warps 0-1 Q producers, 2 MMA, 3 K/V loader, 4-7 softmax, 8-15 O drain
 constexpr int NPROD = 64;        // producer threads (two tile rows each)
@@ -222,6 +222,106 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
         const int pos = a.boff[u] + atomicAdd(&a.bcursor[u], 1);
         a.pairs[pos] = (t << 5) | i;
         a.pair_w[pos] = a.w8[row * a.kmax + i];
+    }
+}
+
+// The same two steps with the rows of one CTA taken as HT consecutive tokens of one
+// (b, kv head) -- all in one phase, since HT divides TB -- so that a CTA counts its
+// pairs per chunk in a shared-memory histogram and touches each of its buckets'
+// global counters once, instead of once per pair.  Used when the histogram of C
+// counters fits in shared memory (two of them for the scatter).
+constexpr int HT = 256;                 // tokens per CTA
+constexpr int HIST_MAX_C = 16384;       // chunks whose counters fit in shared memory
+
+__device__ __forceinline__ bool hist_row(const AttTcArgs &a, int &b, int &j, int &t, long long &row) {
+    const int tb = (a.Tq + HT - 1) / HT;
+    const int blk = (int)blockIdx.x;
+    const int bj = blk / tb;
+    b = bj / a.Hkv;
+    j = bj % a.Hkv;
+    t = (blk % tb) * HT + (int)threadIdx.x;
+    row = ((long long)b * a.Tq + t) * a.Hkv + j;
+    return t < a.Tq;
+}
+
+__global__ void __launch_bounds__(HT) att_count_hist_kernel(AttTcArgs a) {
+    extern __shared__ int hist[];   // [C]
+    for (int c = threadIdx.x; c < a.C; c += HT) hist[c] = 0;
+    __syncthreads();
+    int b, j, t;
+    long long row;
+    const bool live = hist_row(a, b, j, t, row);
+    if (live) {
+        int ke = a.keff[row];
+        if (ke < 0 || ke > a.kmax) {
+            atomicOr(a.status, DEV_BAD_INDEX);
+            ke = ke < 0 ? 0 : a.kmax;
+        }
+        const int nc = ncand_of(a, t);
+        const int32_t *ri = a.idx + row * a.kmax;
+        const float *rs = a.score + row * a.kmax;
+        float m = -INFINITY;
+        for (int i = 0; i < ke; ++i) m = fmaxf(m, rs[i]);
+        float z = 0.f;
+        for (int i = 0; i < ke; ++i) z += expf(rs[i] - m);
+        for (int i = 0; i < ke; ++i) {
+            a.w8[row * a.kmax + i] = expf(rs[i] - m) / z;
+            const int c = ri[i];
+            if (c < 0 || c >= nc) {
+                atomicOr(a.status, DEV_BAD_INDEX);
+                continue;
+            }
+            atomicAdd(&hist[c], 1);
+        }
+    }
+    __syncthreads();
+    const int tb = (a.Tq + HT - 1) / HT;
+    const int t0 = ((int)blockIdx.x % tb) * HT;
+    const int bj = (int)blockIdx.x / tb;
+    const long long p = (long long)bj * a.ntb + t0 / TB;
+    for (int c = threadIdx.x; c < a.C; c += HT)
+        if (hist[c] > 0) atomicAdd(&a.bcount[p * a.C + c], hist[c]);
+}
+
+__global__ void __launch_bounds__(HT) att_scatter_hist_kernel(AttTcArgs a) {
+    extern __shared__ int sh[];   // [C] counts, then cursors; [C] bucket bases
+    int *cnt = sh, *basep = sh + a.C;
+    for (int c = threadIdx.x; c < a.C; c += HT) cnt[c] = 0;
+    __syncthreads();
+    int b, j, t;
+    long long row;
+    const bool live = hist_row(a, b, j, t, row);
+    int ke = 0, nc = 0;
+    if (live) {
+        ke = a.keff[row];
+        ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
+        nc = ncand_of(a, t);
+        for (int i = 0; i < ke; ++i) {
+            const int c = a.idx[row * a.kmax + i];
+            if (c >= 0 && c < nc) atomicAdd(&cnt[c], 1);
+        }
+    }
+    __syncthreads();
+    const int tb = (a.Tq + HT - 1) / HT;
+    const int bj = (int)blockIdx.x / tb;
+    const long long p = (long long)bj * a.ntb + (((int)blockIdx.x % tb) * HT) / TB;
+    for (int c = threadIdx.x; c < a.C; c += HT) {
+        const int n = cnt[c];
+        if (n > 0) {
+            const long long u = p * a.C + c;
+            basep[c] = a.boff[u] + atomicAdd(&a.bcursor[u], n);   // this CTA's range in the bucket
+        }
+        cnt[c] = 0;
+    }
+    __syncthreads();
+    if (live) {
+        for (int i = 0; i < ke; ++i) {
+            const int c = a.idx[row * a.kmax + i];
+            if (c < 0 || c >= nc) continue;
+            const int pos = basep[c] + atomicAdd(&cnt[c], 1);
+            a.pairs[pos] = (t << 5) | i;
+            a.pair_w[pos] = a.w8[row * a.kmax + i];
+        }
     }
 }
 
@@ -751,11 +851,25 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     if (e == cudaSuccess) e = cudaMemsetAsync(bf.ring, 0, L.ring_bytes, st);
     if (e != cudaSuccess) return e;
     const int rows_blocks = (int)((p.rows + 255) / 256);
-    att_count_kernel<<<rows_blocks, 256, 0, st>>>(a);
+    const bool hist = p.C <= HIST_MAX_C;
+    const int hist_blocks = p.B * p.Hkv * ((p.Tq + HT - 1) / HT);
+    if (hist) {
+        if ((e = cudaFuncSetAttribute(att_scatter_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(2 * p.C * sizeof(int)))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(att_count_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(p.C * sizeof(int)))) != cudaSuccess)
+            return e;
+        att_count_hist_kernel<<<hist_blocks, HT, p.C * sizeof(int), st>>>(a);
+    } else {
+        att_count_kernel<<<rows_blocks, 256, 0, st>>>(a);
+    }
     att_scan1_kernel<<<L.nblk, 1024, 0, st>>>(a);
     att_scan2_kernel<<<1, 1024, 0, st>>>(a, L.nblk);
     att_tiles_kernel<<<(L.nbucket + 255) / 256, 256, 0, st>>>(a);
-    att_scatter_kernel<<<rows_blocks, 256, 0, st>>>(a);
+    if (hist)
+        att_scatter_hist_kernel<<<hist_blocks, HT, 2 * p.C * sizeof(int), st>>>(a);
+    else
+        att_scatter_kernel<<<rows_blocks, 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // K and V as 3D (d, Hkv, B*Tcap): box (64, 1, S) = S rows of 128 B

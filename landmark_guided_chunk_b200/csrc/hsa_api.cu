@@ -5,11 +5,21 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace hsa {
 
 static thread_local char g_err[512] = "";
+
+// An NVTX range around each launching entry point, named after it, so that a
+// timeline (nsys, ncu's range filters) shows the library's calls.  Header-only
+// NVTX: without an attached tool a range costs a null check.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
 
 hsa_status_t fail(hsa_status_t s, const char *fmt, ...) {
     va_list ap;
@@ -254,6 +264,7 @@ hsa_status_t hsa_plan(const hsa_problem_t *prob, hsa_plan_t *plan) {
 }
 
 hsa_status_t hsa_landmarks(const hsa_problem_t *prob, const void *K, const void *W_L, void *L, void *stream) {
+    NvtxRange nvtx_("hsa_landmarks");
     Prob p;
     HSA_TRY(validate(prob, &p));
     const bool any = (long long)p.B * p.C > 0;
@@ -266,6 +277,7 @@ hsa_status_t hsa_landmarks(const hsa_problem_t *prob, const void *K, const void 
 
 hsa_status_t hsa_landmarks_refined(const hsa_problem_t *prob, const void *K, const void *W_L, const void *W_q,
                                    const void *W_k, const void *W_v, void *L, void *stream) {
+    NvtxRange nvtx_("hsa_landmarks_refined");
     Prob p;
     HSA_TRY(validate(prob, &p));
     if (p.flags & HSA_FLAG_QUEST) return fail(HSA_ERR_INVALID_ARG, "the refiner makes landmarks, not Quest summaries");
@@ -282,6 +294,7 @@ hsa_status_t hsa_landmarks_refined(const hsa_problem_t *prob, const void *K, con
 
 hsa_status_t hsa_decode_append(const hsa_problem_t *prob, const void *k_new, const void *v_new, void *K, void *V,
                                const void *W_L, void *L, void *stream) {
+    NvtxRange nvtx_("hsa_decode_append");
     Prob p;
     HSA_TRY(validate(prob, &p));
     if (p.B > 0 && p.Tkv >= p.Tcap)
@@ -310,6 +323,7 @@ hsa_status_t hsa_decode_append(const hsa_problem_t *prob, const void *k_new, con
 
 hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L, int32_t *idx, float *score,
                         int32_t *keff, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange nvtx_("hsa_select");
     Prob p;
     HSA_TRY(validate(prob, &p));
     const bool rows = p.rows > 0;
@@ -328,6 +342,7 @@ hsa_status_t hsa_select(const hsa_problem_t *prob, const void *Q, const void *L,
 
 hsa_status_t hsa_attend(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const int32_t *idx,
                         const float *score, const int32_t *keff, void *O, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange nvtx_("hsa_attend");
     Prob p;
     HSA_TRY(validate(prob, &p));
     const bool rows = p.rows > 0;
@@ -349,6 +364,7 @@ hsa_status_t hsa_attend(const hsa_problem_t *prob, const void *Q, const void *K,
 hsa_status_t hsa_attend_partials(const hsa_problem_t *prob, const void *Q, const void *K, const void *V,
                                  const int32_t *idx, const int32_t *keff, float *o_part, void *ws, size_t ws_bytes,
                                  void *stream) {
+    NvtxRange nvtx_("hsa_attend_partials");
     Prob p;
     HSA_TRY(validate(prob, &p));
     if (p.rows > 0 && !attend_gather_supported(p))
@@ -373,6 +389,7 @@ hsa_status_t hsa_attend_partials(const hsa_problem_t *prob, const void *Q, const
 hsa_status_t hsa_merge_partials(const hsa_problem_t *prob, int nshard, const float *score, const int32_t *idx,
                                 const int32_t *keff, const float *o_part, void *O, int32_t *idx_out,
                                 float *score_out, int32_t *keff_out, void *stream) {
+    NvtxRange nvtx_("hsa_merge_partials");
     Prob p;
     HSA_TRY(validate(prob, &p));
     if (nshard < 1) return fail(HSA_ERR_INVALID_ARG, "nshard=%d", nshard);
@@ -393,6 +410,7 @@ hsa_status_t hsa_merge_partials(const hsa_problem_t *prob, int nshard, const flo
 hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const void *W_L,
                          void *L, int32_t *idx, float *score, int32_t *keff, void *O, void *ws, size_t ws_bytes,
                          void *stream) {
+    NvtxRange nvtx_("hsa_forward");
     Prob p;
     HSA_TRY(validate(prob, &p));
     const bool rows = p.rows > 0;
@@ -440,6 +458,7 @@ hsa_status_t hsa_backward_workspace_size(const hsa_problem_t *prob, size_t *byte
 hsa_status_t hsa_backward(const hsa_problem_t *prob, const void *Q, const void *K, const void *V, const void *W_L,
                           const void *L, const int32_t *idx, const float *score, const int32_t *keff, const void *dO,
                           float *dQ, float *dK, float *dV, float *dW_L, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange nvtx_("hsa_backward");
     Prob p;
     HSA_TRY(validate(prob, &p));
     if (p.flags & HSA_FLAG_QUEST) return fail(HSA_ERR_UNSUPPORTED, "backward of Quest scoring is not implemented");

@@ -8,6 +8,8 @@
 // cudaGetSymbolAddress (with that device current) and passed to the kernels.
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace hsa {
@@ -42,8 +44,19 @@ hsa_status_t scratch_on_current_device(void **out) {
 
 using namespace hsa;
 
+static hsa_status_t select_noalloc_impl(const hsa_problem_t *prob, const void *Q, const void *L, int32_t *idx,
+                                        float *score, int32_t *keff, void *stream);
+
 extern "C" HSA_API hsa_status_t hsa_select_noalloc(const hsa_problem_t *prob, const void *Q, const void *L,
                                                    int32_t *idx, float *score, int32_t *keff, void *stream) {
+    nvtxRangePushA("hsa_select_noalloc");
+    const hsa_status_t r = select_noalloc_impl(prob, Q, L, idx, score, keff, stream);
+    nvtxRangePop();
+    return r;
+}
+
+static hsa_status_t select_noalloc_impl(const hsa_problem_t *prob, const void *Q, const void *L, int32_t *idx,
+                                        float *score, int32_t *keff, void *stream) {
     Prob p;
     hsa_status_t s = validate(prob, &p);
     if (s != HSA_OK) return s;
