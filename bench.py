@@ -644,7 +644,10 @@ def run_decode(args, world, rank, local, pk, name="decode_1m"):
                         "frac": round(gbs / pk["hbm_gbs"], 4), "bytes_per_step": scan + gather},
            "stages": stages,
            "l2": "512 MiB written then read before every step and before each stage timed alone", "paths": plan,
-           "gpu_launches_per_step": plan["select"][1] + plan["attend"][1]}
+           "gpu_launches_per_step": plan["select"][1] + (0 if plan["forward_fused"] else plan["attend"][1]),
+           "fused": ("one cooperative launch: the scan, then each row's chunk gather as soon as its selection "
+                     "is published; the stages above are the same work as two separate calls")
+           if plan["forward_fused"] else None}
     if name == "decode_1m":
         res["loop"] = decode_loop(p, hsa, Q, K, V, W, L, O, ws, st, world)
     if name == "decode_16m" and p.B == 1:

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define HSA_ABI_VERSION 4
+#define HSA_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define HSA_API __attribute__((visibility("default")))
@@ -270,7 +270,11 @@ HSA_API hsa_status_t hsa_merge_partials(const hsa_problem_t *p, int nshard, cons
  * The whole path: hsa_landmarks (unless HSA_FLAG_LANDMARKS_READY), then
  * hsa_select, then hsa_attend.  L is an output (or an input with the flag).
  * idx, score and keff may each be NULL.  The selection then lives only in the
- * workspace.
+ * workspace.  For decode shapes (one query per sequence over a long context,
+ * hsa_plan_t.forward_fused = 1) the selection and the attention run as one
+ * cooperative launch: each row's chunks are gathered as soon as its selection
+ * is complete, while other rows are still being scored.  The results are
+ * those of hsa_select followed by hsa_attend (O up to fp32 summation order).
  */
 HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                          const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
@@ -337,12 +341,15 @@ typedef enum {
 typedef struct {
     int32_t landmark_path, select_path, attend_path;        /* hsa_path_t */
     int32_t landmark_kernels, select_kernels, attend_kernels; /* kernel launches per call of each stage */
+    int32_t forward_fused;   /* 1: hsa_forward runs selection and attention as one launch (select_kernels
+                                counts it; the attention stage adds none) */
 } hsa_plan_t;
 
 /*
  * Which kernels hsa_landmarks / hsa_select / hsa_attend launch for problem *p
  * (a pure function of the problem; nothing is launched).  hsa_forward launches
- * the sum of the three (minus the landmark stage with HSA_FLAG_LANDMARKS_READY).
+ * the sum of the three (minus the landmark stage with HSA_FLAG_LANDMARKS_READY,
+ * and minus attend_kernels when forward_fused is 1).
  */
 HSA_API hsa_status_t hsa_plan(const hsa_problem_t *p, hsa_plan_t *plan);
 
@@ -351,6 +358,13 @@ HSA_API const char *hsa_status_string(hsa_status_t s);
 
 /* Detail of the last failing call on this host thread (which argument, which CUDA error). */
 HSA_API const char *hsa_last_error(void);
+
+/* 1 if the loaded library is the debug build (compiled with HSA_DEBUG): every
+ * kernel checks the indices it derives itself -- gathered token and chunk
+ * indices, TMA coordinates, accumulator offsets -- and a failed check is
+ * recorded in the status word (hsa_get_device_status: HSA_ERR_CUDA, "internal
+ * index check") with the index clamped into its range.  0 for release builds. */
+HSA_API int hsa_debug_checks(void);
 
 /* HSA_ABI_VERSION of the loaded library. */
 HSA_API int hsa_abi_version(void);

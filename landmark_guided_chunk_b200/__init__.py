@@ -43,7 +43,8 @@ def plan(prob: hsa_problem_t) -> dict:
     names = _native.PATH_NAMES
     return {"landmarks": (names[pl.landmark_path], pl.landmark_kernels),
             "select": (names[pl.select_path], pl.select_kernels),
-            "attend": (names[pl.attend_path], pl.attend_kernels)}
+            "attend": (names[pl.attend_path], pl.attend_kernels),
+            "forward_fused": bool(pl.forward_fused)}
 
 
 def kmax_of(k: int, tau: float) -> int:

@@ -10,7 +10,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libhsa_b200.so")
+# HSA_DEBUG=1 selects the debug build (every kernel-derived index checked on the device)
+DEBUG = os.environ.get("HSA_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libhsa_b200_debug.so" if DEBUG else "libhsa_b200.so")
 
 HSA_OK, HSA_ERR_INVALID_ARG, HSA_ERR_UNSUPPORTED, HSA_ERR_WORKSPACE, HSA_ERR_CUDA, HSA_ERR_TIMEOUT = range(6)
 HSA_F32, HSA_BF16 = 0, 1
@@ -22,7 +24,8 @@ HSA_FLAG_QUEST = 8
 EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version",
             "hsa_select_noalloc", "hsa_decode_append", "hsa_attend_partials", "hsa_merge_partials",
-            "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status", "hsa_landmarks_refined")
+            "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status", "hsa_landmarks_refined",
+            "hsa_debug_checks")
 PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor", 4: "mma_split"}
 
 
@@ -37,7 +40,8 @@ class hsa_problem_t(ctypes.Structure):
 class hsa_plan_t(ctypes.Structure):
     _fields_ = [("landmark_path", ctypes.c_int32), ("select_path", ctypes.c_int32),
                 ("attend_path", ctypes.c_int32), ("landmark_kernels", ctypes.c_int32),
-                ("select_kernels", ctypes.c_int32), ("attend_kernels", ctypes.c_int32)]
+                ("select_kernels", ctypes.c_int32), ("attend_kernels", ctypes.c_int32),
+                ("forward_fused", ctypes.c_int32)]
 
 
 class HSAError(RuntimeError):
@@ -56,7 +60,7 @@ def lib() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(f"HSA CUDA library not built: {LIB_PATH} is missing "
-                           "(run landmark_guided_chunk_b200/build.py or __graft_entry__.build())")
+                           "(run landmark_guided_chunk_b200/build.py [--debug] or __graft_entry__.build())")
     L = ctypes.CDLL(LIB_PATH)
     P, Z, I32p, Fp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
     prob = ctypes.POINTER(hsa_problem_t)
@@ -81,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.hsa_last_error.restype = ctypes.c_char_p
     L.hsa_abi_version.argtypes = []
     L.hsa_abi_version.restype = ctypes.c_int
+    L.hsa_debug_checks.argtypes = []
+    L.hsa_debug_checks.restype = ctypes.c_int
     for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
               "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc", "hsa_decode_append",
               "hsa_attend_partials", "hsa_merge_partials", "hsa_backward_workspace_size", "hsa_backward",

@@ -3,6 +3,10 @@
 Each csrc/*.cu file is compiled to an object under _build/ (in parallel, skipped
 when up to date), then the objects are linked into one shared library with the
 CUDA runtime linked statically.  The library depends on no torch symbol.
+
+build(debug=True) makes libhsa_b200_debug.so from the same sources with
+-DHSA_DEBUG: the kernels then check every index they derive themselves (see
+dbg_clamp in csrc/common.cuh).  The binding loads it when HSA_DEBUG=1 is set.
 """
 from __future__ import annotations
 
@@ -18,6 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(ROOT, "_build", "obj")
 LIB = os.path.join(PKG, "libhsa_b200.so")
+DEBUG_OBJDIR = os.path.join(ROOT, "_build", "obj_debug")
+DEBUG_LIB = os.path.join(PKG, "libhsa_b200_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE,
@@ -42,10 +48,10 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
-    obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+def _compile(src: str, verbose_ptxas: bool, debug: bool = False) -> str:
+    obj = os.path.join(DEBUG_OBJDIR if debug else OBJDIR, os.path.basename(src) + ".o")
     if _stale(obj, [src] + _headers() + [__file__]):
-        cmd = [_nvcc(), *ARCH, *CFLAGS, "-c", src, "-o", obj]
+        cmd = [_nvcc(), *ARCH, *CFLAGS, *(["-DHSA_DEBUG"] if debug else []), "-c", src, "-o", obj]
         if verbose_ptxas:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,23 +62,24 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    os.makedirs(OBJDIR, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    objdir, lib = (DEBUG_OBJDIR, DEBUG_LIB) if debug else (OBJDIR, LIB)
+    os.makedirs(objdir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     if force:
-        for o in glob.glob(os.path.join(OBJDIR, "*.o")):
+        for o in glob.glob(os.path.join(objdir, "*.o")):
             os.remove(o)
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    if force or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, debug), srcs))
+    if force or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [_nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -519,7 +519,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 const bool valid = mm[h] < T.n;
                 const char *src = reinterpret_cast<const char *>(Q);
                 if (valid) {
-                    const int t = pr[h] >> 5;
+                    const int t0 = (T.p % a.ntb) * TB;   // the tile's phase: tokens t0 .. t0 + TB - 1
+                    const int t = (int)dbg_clamp(pr[h] >> 5, t0, min(a.Tq, t0 + TB), a.status);
                     src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
                 }
                 const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
@@ -551,12 +552,14 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 if (e.x == prev_p && e.y == prev_c) continue;
                 prev_p = e.x;
                 prev_c = e.y;
-                const int bj = e.x / a.ntb, Tb = bj / a.Hkv, Tj = bj % a.Hkv;
+                const int bj = (int)dbg_clamp(e.x / a.ntb, 0, (long long)a.B * a.Hkv, a.status);
+                const int Tb = bj / a.Hkv, Tj = bj % a.Hkv;
+                const int cz = (int)dbg_clamp(e.y, 0, a.C, a.status);   // the bucket's chunk
                 const int skv = nload % a.nskv, ikv = nload / a.nskv;
                 if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
                 mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
                 uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
-                const int z = Tb * a.Tcap + e.y * S;
+                const int z = Tb * a.Tcap + cz * S;
                 tma_load_3d(dk, &tmK, 0, Tj, z, &bar->kv_full[skv]);
                 tma_load_3d(dk + kv_bytes, &tmK, 64, Tj, z, &bar->kv_full[skv]);
                 tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, Tj, z, &bar->kv_full[skv]);
@@ -722,7 +725,11 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             // destinations of the staging rows this lane will reduce (rows rr*4 + lane/8 of the warp)
             int dstoff[8];
 #pragma unroll
-            for (int rr = 0; rr < 8; ++rr) dstoff[rr] = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
+            for (int rr = 0; rr < 8; ++rr) {
+                // -1 (padding) or the start of a row of the phase's accumulator slot
+                const int o = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
+                dstoff[rr] = o < 0 ? -1 : (int)dbg_clamp(o, 0, (long long)(TB - 1) * a.G * D + 1, a.status);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->info_empty[si]);
             if (!(ok = mbar_wait(&bar->l_full[b], k & 1, abort, a.status))) break;

@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(NT_BWD, 1)
         if (threadIdx.x < RT) {
             const int rr = threadIdx.x;
             if (rr < nrow) {
-                const int pc = a.pairs[tr.y + rr / a.G], g = rr % a.G;
+                const int pc = (int)dbg_clamp(a.pairs[tr.y + rr / a.G], 0, a.rows * a.kmax, a.status), g = rr % a.G;
                 const long long bt = (long long)(pc / a.kmax) / a.Hkv;
                 s_qoff[rr] = (bt * a.H + (long long)cj * a.G + g) * D;
                 s_w[rr] = a.w[pc];
@@ -704,7 +704,7 @@ __global__ void __launch_bounds__(BT_ROWS, 1)
         w_o = 0.f;
         e_o = -1;
         if (r < nrow) {
-            const int pc = a.pairs[tr.y + r / a.G], g = r % a.G;
+            const int pc = (int)dbg_clamp(a.pairs[tr.y + r / a.G], 0, a.rows * a.kmax, a.status), g = r % a.G;
             const long long bt = (long long)(pc / a.kmax) / a.Hkv;
             qoff = (bt * a.H + (long long)j * a.G + g) * D;
             w_o = a.w[pc];
@@ -1057,7 +1057,7 @@ __global__ void __launch_bounds__(NT_W, 1)
             float w = 0.f;
             int e = -1;
             if (pr < tr.z * a.G) {
-                const int pc = a.pairs[tr.y + pr / a.G], g = pr % a.G;
+                const int pc = (int)dbg_clamp(a.pairs[tr.y + pr / a.G], 0, a.rows * a.kmax, a.status), g = pr % a.G;
                 w = a.pair_w[tr.y + pr / a.G];
                 const long long bt = (long long)(pc / a.kmax) / a.Hkv;
                 qoff = (bt * a.H + (long long)bucket_pos(a, tr.x).j * a.G + g) * D;

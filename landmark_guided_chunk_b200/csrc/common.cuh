@@ -50,6 +50,9 @@ struct WsLayout {
     size_t sel_cnt;      // split select (tensor-core scan): per-row completion counters, right after the header
     size_t att_cnt;      // gather attend: per-row completion counters, right after the header
     size_t att_acc;      // gather attend: per-row fp32 accumulators (rows x G x d), right after the counters
+    size_t dec_ready;    // fused decode step: publication slots (rows int32), zeroed with the status word
+    size_t dec_ctr;      // fused decode step: rows published, units claimed (2 int32), zeroed likewise
+    bool fused_decode;   // hsa_forward runs the decode scan and the gather as one launch
     size_t clear_bytes;  // bytes from the workspace start zeroed before every call (status word, counters)
     size_t total;
     int nsplit, chunks_per_split;
@@ -76,6 +79,28 @@ constexpr uint32_t DEV_OK = 0;
 constexpr uint32_t DEV_TIMEOUT = 1;      // a bounded wait expired
 constexpr uint32_t DEV_BAD_INDEX = 2;    // hsa_attend got a chunk index / keff outside its row's range
 constexpr uint32_t DEV_INTERNAL = 4;     // a kernel's own slot/index check failed; the access was skipped
+
+// Debug builds (compiled with -DHSA_DEBUG into libhsa_b200_debug.so) check the
+// indices a kernel derives itself before it uses them: gathered token and
+// chunk indices, TMA coordinates, accumulator offsets.  An index outside its
+// range is recorded in the status word (DEV_INTERNAL, HSA_ERR_CUDA from
+// hsa_get_device_status) and clamped into the range, so the access stays
+// inside its tensor and no wait is left without its data.  Release builds
+// compile the checks away.
+#ifdef HSA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ long long dbg_clamp(long long x, long long lo, long long hi, uint32_t *status) {
+    if constexpr (kDebugChecks) {
+        if (x < lo || x >= hi) {
+            atomicOr(status, DEV_INTERNAL);
+            return x < lo ? lo : hi - 1;
+        }
+    }
+    return x;
+}
 
 // ---------------------------------------------------------------------------- element access
 
@@ -280,6 +305,13 @@ void select_stream_shape(const Prob &p, int sms, int *grid, int *maxe);
 cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
                                  int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
                                  cudaStream_t st);
+// The fused decode step: the stream scan, then (same launch, cooperative) the chunk
+// gather of each published row (select_stream.cu).  grid is the scan's grid.
+bool decode_fused_supported(const Prob &p, int grid, int sms);
+cudaError_t launch_decode_fused(const Prob &p, const void *Q, const void *K, const void *V, const void *L,
+                                int32_t *idx, float *score, int32_t *keff, void *O, float2 *lists, int32_t *cnt,
+                                int32_t *ready, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
+                                int grid, int maxe, cudaStream_t st);
 // part != null: partial mode (o_i of every (row, slot) into part [rows][kmax][G][d]; no fusion, O unused)
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,
                                  const float *score, const int32_t *keff, void *O, float *acc, int32_t *cnt,

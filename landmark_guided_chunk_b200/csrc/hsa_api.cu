@@ -85,6 +85,12 @@ WsLayout ws_layout(const Prob &p) {
         w.att_cnt = take(rows * sizeof(int32_t));
         w.att_acc = take(rows * (size_t)p.G * p.d * sizeof(float));
     }
+    // Decode with both of those kernels: hsa_forward fuses them into one launch.
+    w.fused_decode = w.stream_select && w.gather_attend && decode_fused_supported(p, w.stream_grid, device_sms());
+    if (w.fused_decode) {
+        w.dec_ready = take(rows * sizeof(int32_t));
+        w.dec_ctr = take(2 * sizeof(int32_t));
+    }
     w.clear_bytes = off > 256 ? off : sizeof(uint32_t);
     w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
     w.sel_score = take(rows * p.kmax * sizeof(float));
@@ -133,6 +139,7 @@ WsLayout ws_layout(const Prob &p) {
     w.plan.attend_kernels = rows == 0 ? 0
                             : w.tc_attend ? attend_tc_launches(w.att)
                                           : (w.split_attend && !w.gather_attend ? 2 : 1);
+    w.plan.forward_fused = w.fused_decode ? 1 : 0;
     return w;
 }
 
@@ -232,6 +239,8 @@ using namespace hsa;
 extern "C" {
 
 int hsa_abi_version(void) { return HSA_ABI_VERSION; }
+
+int hsa_debug_checks(void) { return kDebugChecks ? 1 : 0; }
 
 const char *hsa_last_error(void) { return g_err; }
 
@@ -438,6 +447,17 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     int32_t *sidx = idx ? idx : reinterpret_cast<int32_t *>(wsb + w.sel_idx);
     float *ssc = score ? score : reinterpret_cast<float *>(wsb + w.sel_score);
     int32_t *skf = keff ? keff : reinterpret_cast<int32_t *>(wsb + w.sel_keff);
+    if (w.fused_decode && p.C > 0) {
+        e = launch_decode_fused(p, Q, K, V, L, sidx, ssc, skf, O, reinterpret_cast<float2 *>(wsb + w.split_lists),
+                                reinterpret_cast<int32_t *>(wsb + w.sel_cnt), reinterpret_cast<int32_t *>(wsb + w.dec_ready),
+                                reinterpret_cast<int32_t *>(wsb + w.dec_ctr), reinterpret_cast<int32_t *>(wsb + w.att_cnt),
+                                reinterpret_cast<float *>(wsb + w.att_acc), reinterpret_cast<uint32_t *>(wsb + w.hdr),
+                                w.stream_grid, w.stream_maxe, st);
+        if (e != cudaErrorCooperativeLaunchTooLarge)
+            return e == cudaSuccess ? HSA_OK : cuda_fail(e, "fused decode kernel launch");
+        // the device cannot hold every CTA at once right now: the same two kernels, one after the other
+        cudaGetLastError();
+    }
     e = run_selection(p, w, Q, L, sidx, ssc, skf, wsb, st);
     if (e != cudaSuccess) return cuda_fail(e, "selection kernel launch");
     e = launch_attend(p, w, Q, K, V, sidx, ssc, skf, O, wsb, st);
@@ -502,7 +522,7 @@ hsa_status_t hsa_get_device_status(void *ws, size_t ws_bytes, void *stream) {
     if (word & DEV_TIMEOUT) return fail(HSA_ERR_TIMEOUT, "device-status word 0x%x: a bounded device wait expired", word);
     if (word & DEV_INTERNAL)
         return fail(HSA_ERR_CUDA, "device-status word 0x%x: a kernel's internal index check failed (the access was "
-                    "skipped; results of that call are incomplete)", word);
+                    "skipped or, in the debug build, clamped; results of that call are incomplete)", word);
     return fail(HSA_ERR_INVALID_ARG, "device-status word 0x%x: hsa_attend got a keff or chunk index outside "
                 "its row's candidates (those slots were skipped)", word);
 }

@@ -21,15 +21,30 @@
 // one list per (row, CTA), and the CTA that completes a row (per-row counter,
 // zeroed with the status word) merges the row's lists and writes its
 // selection, with the router's k_eff.
+//
+// Fused decode step (hsa_forward): the same launch then does the chunk
+// attention and the fusion.  The warp that completes a row publishes it
+// (release store of row + 1 into the next slot of a publication list), and
+// once a CTA's scan is done all of its warps become gather workers with one
+// K/V stage each, carved from the now idle ring: a worker claims the next
+// (publication slot, kept slot) unit from a global counter, waits (bounded)
+// until that slot is published, stages the chunk's K and V by TMA and adds
+// w_i * o_i / l_i into the row's fp32 accumulator; whoever finishes a row's
+// last kept slot converts it to bf16 O.  Rows published early are gathered
+// while the slowest CTAs still scan, and the gather needs no launch of its
+// own.  Workers wait only on rows, and rows depend only on the scan, so the
+// launch is cooperative (every CTA resident) and cannot deadlock.
 #include <algorithm>
 
 #include "common.cuh"
+#include "decode_mma.cuh"
 #include "sm100.cuh"
 
 namespace hsa {
 namespace {
 
 using namespace sm100;
+using namespace decode;
 
 constexpr int TCH = 64;    // chunks per tile
 constexpr int NCW = 6;     // consumer warps
@@ -49,6 +64,15 @@ struct StreamArgs {
     int grid, maxe;       // CTAs; list slots per row
     float tau;
     uint32_t *status;
+    int rows;             // B * Hkv (one query per sequence)
+    // fused decode step only
+    int B, Tcap, nunits, nwg;   // units = rows * kmax; gather workers per CTA
+    float scale;                // 1/sqrt(d)
+    int32_t *ready;             // [rows] publication slots: row + 1, 0 until published
+    int32_t *ctr;               // [0] rows published, [1] units claimed
+    int32_t *att_cnt;           // [rows] kept slots gathered per row
+    float *acc;                 // [rows][G][d] fp32 accumulators
+    __nv_bfloat16 *O;
 };
 
 struct __align__(8) StreamBars {
@@ -62,6 +86,33 @@ __device__ __forceinline__ bool in_range(long long x, long long n, uint32_t *sta
     if (x >= 0 && x < n) return true;
     atomicOr(status, DEV_INTERNAL);
     return false;
+}
+
+__device__ __forceinline__ void st_release_gpu(int32_t *p, int v) {
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Wait until publication slot *p is set; 0 if the wait expired or another
+// CTA's wait did (the status word carries DEV_TIMEOUT).
+__device__ __forceinline__ int wait_published(const int32_t *p, uint32_t *status, volatile int *abort) {
+    int v = ld_acquire_gpu(p);
+    if (v != 0) return v;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(128);
+        if ((v = ld_acquire_gpu(p)) != 0) return v;
+        if (*abort || (__ldcv(status) & DEV_TIMEOUT)) return 0;
+        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            *abort = 1;
+            atomicOr(status, DEV_TIMEOUT);
+            return 0;
+        }
+    }
 }
 
 // Order-preserving unsigned code of a float (for atomicMax on scores).
@@ -79,36 +130,124 @@ __device__ __forceinline__ int cta_of(const StreamArgs &a, long long T) {
     return (int)(((T + 1) * a.grid - 1) / a.total);
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-// 16-byte chunk j of row u in a box of 128-byte rows written with the 128-byte swizzle
-__device__ __forceinline__ uint32_t swz(uint32_t box, int u, int j) {
-    return box + (uint32_t)u * 128u + ((uint32_t)(j ^ (u & 7)) << 4);
+// ---------------------------------------------------------------------------- fused gather phase
+// Bytes of one gather worker's stage: a chunk's K and V, D/64 boxes of S rows each.
+template <int D, int S>
+constexpr int gather_stage_bytes() {
+    return 2 * (D / 64) * S * 128;
 }
 
-template <int D>
+// The gather phase of the fused decode step (all of a CTA's warps, after its
+// scan): claim units, wait for their rows, stage the chunks, accumulate.
+template <int D, int S>
+__device__ __forceinline__ void gather_phase(const StreamArgs &a, uint8_t *base, uint64_t *gbar, volatile int *abort,
+                                             const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                             const __nv_bfloat16 *__restrict__ Q, const int32_t *idx,
+                                             const float *score, const int32_t *keff) {
+    constexpr int NB = D / 64, BOX = S * 128, STAGE = gather_stage_bytes<D, S>();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= a.nwg) return;
+    uint8_t *stage = base + (size_t)warp * STAGE;
+    uint64_t *mbk = &gbar[2 * warp], *mbv = &gbar[2 * warp + 1];
+    uint32_t phase = 0;                    // parity of the next K (and V) load
+    bool pend_k = false, pend_v = false;   // copies issued and not yet consumed
+    while (!*abort) {
+        int u = 0;
+        if (lane == 0) u = atomicAdd(&a.ctr[1], 1);
+        u = __shfl_sync(FULL, u, 0);
+        if (u >= a.nunits) break;
+        const int pos = u / a.kmax, i = u - pos * a.kmax;
+        int rv = 0;
+        if (lane == 0) rv = wait_published(&a.ready[pos], a.status, abort);
+        rv = __shfl_sync(FULL, rv, 0);
+        if (rv == 0 || !in_range(rv - 1, a.rows, a.status)) break;
+        const int row = rv - 1;
+        const int j = row % a.Hkv, b = row / a.Hkv;
+        const size_t qrow = ((size_t)b * a.H + (size_t)j * a.G) * D;   // Q [B][1][H][d]
+        // one round trip: keff, the slot's chunk, the row's retrieval scores, Q fragments
+        int ke = 0, c = 0;
+        if (lane == 0) {
+            ke = __ldcg(&keff[row]);
+            c = __ldcg(&idx[(size_t)row * a.kmax + i]);
+        }
+        const float sv = lane < a.kmax ? __ldcg(&score[(size_t)row * a.kmax + lane]) : -INFINITY;
+        uint32_t qa[D / 16][4];
+        load_q_frags<D>(Q + qrow, a.G, qa);
+        ke = __shfl_sync(FULL, ke, 0);
+        c = __shfl_sync(FULL, c, 0);
+        if (i >= ke) {
+            if (ke == 0 && i == 0)   // no candidates: the output is zero
+                for (int e = lane; e < a.G * D; e += 32) a.O[qrow + e] = __float2bfloat16(0.f);
+            continue;
+        }
+        const bool cok = in_range(c, a.ncand, a.status);
+        if (cok && lane == 0) {
+            const int z = b * a.Tcap + c * S;
+            mbar_expect_tx(mbk, (uint32_t)(NB * BOX));
+            mbar_expect_tx(mbv, (uint32_t)(NB * BOX));
+#pragma unroll
+            for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + kb * BOX, &tmK, 64 * kb, j, z, mbk);
+#pragma unroll
+            for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + (NB + kb) * BOX, &tmV, 64 * kb, j, z, mbv);
+        }
+        if (cok) pend_k = pend_v = true;
+        // this slot's fusion weight: softmax over the row's kept retrieval scores
+        const float xs = lane < ke ? sv : -INFINITY;
+        const float m = warp_max(xs);
+        const float ex = lane < ke ? expf(xs - m) : 0.f;
+        const float w = __shfl_sync(FULL, ex, i) / warp_sum(ex);
+        if (cok) {
+            bool ok = mbar_wait(mbk, phase, abort, a.status);
+            if (ok) pend_k = false;
+            if (!__all_sync(FULL, ok)) break;
+            const uint32_t sk = smem_u32(stage);
+            float *racc = a.acc + (size_t)row * a.G * D;
+            auto wait_v = [&]() {
+                bool v = mbar_wait(mbv, phase, abort, a.status);
+                if (v) pend_v = false;
+                return __all_sync(FULL, v);
+            };
+            if (!chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, w, 0,
+                                     [&](int g, int col, float x, float y) { red_add2(racc + (size_t)g * D + col, x, y); },
+                                     wait_v))
+                break;
+            phase ^= 1u;   // both copies consumed
+        }
+        // this slot is done; whoever completes the row converts its accumulator to O
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&a.att_cnt[row], 1) == ke - 1;
+        if (__shfl_sync(FULL, last, 0)) {
+            __threadfence();
+            acc_to_bf16(a.acc + (size_t)row * a.G * D, a.O + qrow, a.G * D);
+        }
+        __syncwarp();   // the stage is free for the next unit
+    }
+    // after an expired wait: let the copies still in flight land before the CTA exits
+    if (lane == 0 && pend_k) mbar_drain(mbk, phase);
+    if (lane == 0 && pend_v) mbar_drain(mbv, phase);
+}
+
+constexpr int WL_BYTES = RMAX * NCW * 16 * (int)sizeof(float2);   // the consumer warps' lists
+
+// S is the chunk length of the fused gather phase (0: selection only).
+template <int D, int S>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
-    select_stream_kernel(const __grid_constant__ CUtensorMap tmL, const __nv_bfloat16 *__restrict__ Q,
+    select_stream_kernel(const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __nv_bfloat16 *__restrict__ Q,
                          float2 *__restrict__ lists, int32_t *__restrict__ idx, float *__restrict__ score,
                          int32_t *__restrict__ keff, int32_t *__restrict__ cnt, StreamArgs a) {
+    constexpr bool FUSE = S > 0;
     constexpr int NB = D / 64;          // boxes per tile
     constexpr int BOXB = TCH * 128;     // bytes of one box
     constexpr int STB = NB * BOXB;      // bytes of one stage
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ StreamBars bar;
-    __shared__ float2 wl[RMAX][NCW][16];   // each consumer warp's list per row slot
+    __shared__ __align__(8) uint64_t gbar[FUSE ? 2 * (NCW + 1) : 1];   // gather: K and V barrier per worker
+    // each consumer warp's list per row slot, after the ring (the gather stages may cover both)
+    float2 (*wl)[NCW][16] = reinterpret_cast<float2 (*)[NCW][16]>(base + (size_t)NST * STB);
     __shared__ unsigned s_floor[RMAX];     // best k-th score any warp's list has reached, per row slot
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int x = (int)blockIdx.x;
@@ -121,6 +260,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             mbar_init(&bar.full[s], 1);
             mbar_init(&bar.empty[s], 1);
         }
+        if constexpr (FUSE)
+            for (int s = 0; s < 2 * (NCW + 1); ++s) mbar_init(&gbar[s], 1);
         bar.abort = 0;
         fence_mbar_init();
     }
@@ -137,8 +278,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             for (; k < ntile; ++k) {
                 const int s = k % NST, u = k / NST;
                 if (u > 0 && !(ok = mbar_wait(&bar.empty[s], (u - 1) & 1, &bar.abort, a.status))) break;
-                const long long T = lo + k, row = T / a.tpr;
-                const int y = (int)(row * a.Lc + (T % a.tpr) * TCH);
+                const long long T = lo + k, row = dbg_clamp(T / a.tpr, 0, a.rows, a.status);
+                const int y = (int)(row * a.Lc + dbg_clamp((T % a.tpr) * TCH, 0, a.ncand, a.status));
                 mbar_expect_tx(&bar.full[s], (uint32_t)STB);
 #pragma unroll
                 for (int kb = 0; kb < NB; ++kb)
@@ -221,49 +362,68 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 
     // ---- per row slot: merge the consumer warps' lists, publish the CTA's list;
     // the CTA that completes the row merges the row's lists and writes the row
-    if (ntile == 0 || bar.abort) return;
-    const int nrows = (int)((hi - 1) / a.tpr - r_lo + 1);
-    if (warp >= nrows || !in_range(warp, RMAX, a.status)) return;
-    const long long row = r_lo + warp;
-    float v = lane < 16 ? wl[warp][0][lane].x : -INFINITY;
-    int id = lane < 16 ? __float_as_int(wl[warp][0][lane].y) : INT32_MAX;
-    if (lane >= a.kmax) {
-        v = -INFINITY;
-        id = INT32_MAX;
-    }
-    for (int w2 = 1; w2 < NCW; ++w2) {
-        const float2 e = lane < 16 ? wl[warp][w2][lane] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
-        list_merge16(v, id, e.x, __float_as_int(e.y), a.kmax, lane);
-    }
-    const long long T0 = row * a.tpr;
-    const int x0 = cta_of(a, T0), x1 = cta_of(a, T0 + a.tpr - 1);
-    float2 *rl = lists + row * (long long)a.maxe * a.kmax;
-    if (!in_range(x - x0, a.maxe, a.status) || !in_range(x1 - x0, a.maxe, a.status)) return;
-    if (lane < a.kmax) rl[(x - x0) * a.kmax + lane] = make_float2(v, __int_as_float(id));
-    __threadfence();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(&cnt[row], 1) == x1 - x0;
-    if (!__shfl_sync(FULL, last, 0)) return;
-    __threadfence();
-    list_init(v, id);
-    // the row's lists, eight in flight per round trip (then merged in order)
-    const int ne = x1 - x0 + 1;
-    for (int e0 = 0; e0 < ne; e0 += 8) {
-        float2 f[8];
+    auto finish_row = [&]() {
+        if (ntile == 0 || bar.abort) return;
+        const int nrows = (int)((hi - 1) / a.tpr - r_lo + 1);
+        if (warp >= nrows || !in_range(warp, RMAX, a.status)) return;
+        const long long row = r_lo + warp;
+        float v = lane < 16 ? wl[warp][0][lane].x : -INFINITY;
+        int id = lane < 16 ? __float_as_int(wl[warp][0][lane].y) : INT32_MAX;
+        if (lane >= a.kmax) {
+            v = -INFINITY;
+            id = INT32_MAX;
+        }
+        for (int w2 = 1; w2 < NCW; ++w2) {
+            const float2 e = lane < 16 ? wl[warp][w2][lane] : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+            list_merge16(v, id, e.x, __float_as_int(e.y), a.kmax, lane);
+        }
+        const long long T0 = row * a.tpr;
+        const int x0 = cta_of(a, T0), x1 = cta_of(a, T0 + a.tpr - 1);
+        float2 *rl = lists + row * (long long)a.maxe * a.kmax;
+        if (!in_range(x - x0, a.maxe, a.status) || !in_range(x1 - x0, a.maxe, a.status)) return;
+        if (lane < a.kmax) rl[(x - x0) * a.kmax + lane] = make_float2(v, __int_as_float(id));
+        __threadfence();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&cnt[row], 1) == x1 - x0;
+        if (!__shfl_sync(FULL, last, 0)) return;
+        __threadfence();
+        list_init(v, id);
+        // the row's lists, eight in flight per round trip (then merged in order)
+        const int ne = x1 - x0 + 1;
+        for (int e0 = 0; e0 < ne; e0 += 8) {
+            float2 f[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            f[u] = (e0 + u < ne && lane < a.kmax) ? __ldcg(rl + (e0 + u) * a.kmax + lane)
-                                                  : make_float2(-INFINITY, __int_as_float(INT32_MAX));
+            for (int u = 0; u < 8; ++u)
+                f[u] = (e0 + u < ne && lane < a.kmax) ? __ldcg(rl + (e0 + u) * a.kmax + lane)
+                                                      : make_float2(-INFINITY, __int_as_float(INT32_MAX));
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            if (e0 + u < ne) list_merge16(v, id, f[u].x, __float_as_int(f[u].y), a.kmax, lane);
+            for (int u = 0; u < 8; ++u)
+                if (e0 + u < ne) list_merge16(v, id, f[u].x, __float_as_int(f[u].y), a.kmax, lane);
+        }
+        const int ke = list_keff(v, a.ncand, a.k, a.kmax, a.tau);
+        if (lane < a.kmax) {
+            idx[row * a.kmax + lane] = lane < ke ? id : -1;
+            score[row * a.kmax + lane] = lane < ke ? v : -INFINITY;
+        }
+        if (lane == 0) keff[row] = ke;
+        if constexpr (FUSE) {
+            // publish the row: every lane's selection writes, then the slot
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                const int pos = atomicAdd(&a.ctr[0], 1);
+                if (in_range(pos, a.rows, a.status)) st_release_gpu(&a.ready[pos], (int)row + 1);
+            }
+        }
+    };
+    finish_row();
+    if constexpr (FUSE) {
+        // the ring and the lists are free: they become the gather stages (TMA
+        // writes after this CTA's generic accesses to the same shared memory)
+        fence_proxy_async_smem();
+        __syncthreads();
+        gather_phase<D, S>(a, base, gbar, &bar.abort, tmK, tmV, Q, idx, score, keff);
     }
-    const int ke = list_keff(v, a.ncand, a.k, a.kmax, a.tau);
-    if (lane < a.kmax) {
-        idx[row * a.kmax + lane] = lane < ke ? id : -1;
-        score[row * a.kmax + lane] = lane < ke ? v : -INFINITY;
-    }
-    if (lane == 0) keff[row] = ke;
 }
 
 }  // namespace
@@ -291,10 +451,8 @@ void select_stream_shape(const Prob &p, int sms, int *grid, int *maxe) {
     *maxe = (int)e;
 }
 
-cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
-                                 int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
-                                 cudaStream_t st) {
-    StreamArgs a;
+static StreamArgs stream_args(const Prob &p, uint32_t *status, int grid, int maxe) {
+    StreamArgs a{};
     a.Tq = p.Tq;
     a.H = p.H;
     a.Hkv = p.Hkv;
@@ -306,29 +464,117 @@ cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, in
     a.kmax = p.kmax;
     a.ncand = (int)std::min<long long>(p.q_pos0 / p.S, p.C);
     a.tpr = (a.ncand + TCH - 1) / TCH;
+    a.rows = (int)p.rows;
     a.total = p.rows * (long long)a.tpr;
     a.grid = grid;
     a.maxe = maxe;
     a.tau = p.tau;
     a.status = status;
+    return a;
+}
+
+static size_t ring_smem(int d) { return 1024 + (size_t)NST * (d / 64) * TCH * 128 + WL_BYTES; }
+
+cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, int32_t *idx, float *score,
+                                 int32_t *keff, float2 *lists, int32_t *cnt, uint32_t *status, int grid, int maxe,
+                                 cudaStream_t st) {
+    StreamArgs a = stream_args(p, status, grid, maxe);
     CUtensorMap ml;
     cudaError_t e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, TCH);
     if (e != cudaSuccess) return e;
-    const size_t smem = 1024 + (size_t)NST * (p.d / 64) * TCH * 128;
+    const size_t smem = ring_smem(p.d);
+    // the K/V map arguments are unused without the gather phase
     if (p.d == 128) {
-        if ((e = cudaFuncSetAttribute(select_stream_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(select_stream_kernel<128, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
-        select_stream_kernel<128><<<grid, (NCW + 1) * 32, smem, st>>>(ml, (const __nv_bfloat16 *)Q, lists, idx, score,
-                                                                      keff, cnt, a);
+        select_stream_kernel<128, 0><<<grid, (NCW + 1) * 32, smem, st>>>(ml, ml, ml, (const __nv_bfloat16 *)Q, lists,
+                                                                         idx, score, keff, cnt, a);
     } else {
-        if ((e = cudaFuncSetAttribute(select_stream_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(select_stream_kernel<64, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smem)) != cudaSuccess)
             return e;
-        select_stream_kernel<64><<<grid, (NCW + 1) * 32, smem, st>>>(ml, (const __nv_bfloat16 *)Q, lists, idx, score,
-                                                                     keff, cnt, a);
+        select_stream_kernel<64, 0><<<grid, (NCW + 1) * 32, smem, st>>>(ml, ml, ml, (const __nv_bfloat16 *)Q, lists,
+                                                                        idx, score, keff, cnt, a);
     }
     return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------- fused decode step
+
+bool decode_fused_supported(const Prob &p, int grid, int sms) {
+    // one CTA per SM (the ring's shared memory), all resident at once
+    return select_stream_supported(p) && !(p.flags & HSA_FLAG_QUEST) && grid <= sms && p.rows * p.kmax < (1ll << 31);
+}
+
+template <int D, int S>
+static cudaError_t launch_fused_ds(StreamArgs a, const CUtensorMap &ml, const CUtensorMap &mk, const CUtensorMap &mv,
+                                   const void *Q, float2 *lists, int32_t *idx, float *score, int32_t *keff,
+                                   int32_t *cnt, cudaStream_t st) {
+    auto kern = select_stream_kernel<D, S>;
+    cudaError_t e;
+    int dev = 0, optin = 0;
+    cudaFuncAttributes fa;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    constexpr size_t STAGE = gather_stage_bytes<D, S>();
+    const long long room = (long long)optin - (long long)fa.sharedSizeBytes - 1024;
+    int nwg = (int)std::min<long long>(NCW + 1, room / (long long)STAGE);
+    if (nwg < 1) return cudaErrorInvalidConfiguration;
+    a.nwg = nwg;
+    const size_t smem = std::max(ring_smem(D), 1024 + (size_t)nwg * STAGE);
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    const __nv_bfloat16 *q = (const __nv_bfloat16 *)Q;
+    void *args[] = {(void *)&ml, (void *)&mk, (void *)&mv, (void *)&q, (void *)&lists, (void *)&idx,
+                    (void *)&score, (void *)&keff, (void *)&cnt, (void *)&a};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.grid);
+    cfg.blockDim = dim3((NCW + 1) * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // every CTA resident: gather workers wait on other CTAs' rows
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void *>(kern), args);
+}
+
+cudaError_t launch_decode_fused(const Prob &p, const void *Q, const void *K, const void *V, const void *L,
+                                int32_t *idx, float *score, int32_t *keff, void *O, float2 *lists, int32_t *cnt,
+                                int32_t *ready, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
+                                int grid, int maxe, cudaStream_t st) {
+    StreamArgs a = stream_args(p, status, grid, maxe);
+    a.B = p.B;
+    a.Tcap = p.Tcap;
+    a.nunits = (int)(p.rows * p.kmax);
+    a.scale = 1.0f / sqrtf((float)p.d);
+    a.ready = ready;
+    a.ctr = ctr;
+    a.att_cnt = att_cnt;
+    a.acc = acc;
+    a.O = (__nv_bfloat16 *)O;
+    CUtensorMap ml, mk, mv;
+    cudaError_t e = make_tmap_2d(&ml, L, (uint64_t)p.d, (uint64_t)p.B * p.Hkv * p.Lc, 64, TCH);
+    if (e != cudaSuccess) return e;
+    // K and V as 3D (d, Hkv, B*Tcap): box (64, 1, S) = S rows of 128 bytes, 128-byte swizzle
+    const uint64_t dims[3] = {(uint64_t)p.d, (uint64_t)p.Hkv, (uint64_t)p.B * p.Tcap};
+    const uint64_t strides[2] = {(uint64_t)p.d * 2, (uint64_t)p.Hkv * p.d * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)p.S};
+    if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
+#define HSA_FUSED(D_, S_)                                                                                   \
+    if (p.d == D_ && p.S == S_) return launch_fused_ds<D_, S_>(a, ml, mk, mv, Q, lists, idx, score, keff, cnt, st);
+    HSA_FUSED(128, 64)
+    HSA_FUSED(128, 32)
+    HSA_FUSED(128, 128)
+    HSA_FUSED(64, 64)
+    HSA_FUSED(64, 32)
+    HSA_FUSED(64, 128)
+#undef HSA_FUSED
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace hsa

@@ -180,23 +180,25 @@ __global__ void __launch_bounds__(256, 1)
             for (int tau = blockIdx.x; tau < a.ntiles && ok; tau += gridDim.x) {
                 const Tile T = tile_of<NT>(a, tau);
                 if (T.nslices == 0) continue;
-                const int y = T.b * a.Tq + T.t0;
+                const int y = (int)dbg_clamp(T.b * a.Tq + T.t0, 0, (long long)a.B * a.Tq, a.status);   // query row
+                const int qj = (int)dbg_clamp(T.j, 0, a.Hkv, a.status);
                 for (int kb = 0; kb < a.nkb; ++kb) {
                     if (ta > 0 && !(ok = mbar_wait(&bar->a_empty[kb], (ta - 1) & 1, abort, a.status, a.wait_ns))) break;
                     mbar_expect_tx(&bar->a_full[kb], (uint32_t)BOX);
-                    tma_load_2d(sA + (size_t)kb * BOX, &tmQ, T.j * a.G * a.d + kb * 64, y, &bar->a_full[kb]);
+                    tma_load_2d(sA + (size_t)kb * BOX, &tmQ, qj * a.G * a.d + kb * 64, y, &bar->a_full[kb]);
                     kb_part = kb + 1;
                 }
                 if (!ok) break;
                 ++ta;
                 kb_part = 0;
-                const int ly = (T.b * a.Hkv + T.j) * a.Lc;
+                const int ly = (T.b * a.Hkv + qj) * a.Lc;   // the (b, kv head) landmark list
                 for (int n = 0; n < T.nslices; ++n, ++g) {
                     const int s = g % NSTAGE, i = g / NSTAGE;
                     if (i > 0 && !(ok = mbar_wait(&bar->b_empty[s], (i - 1) & 1, abort, a.status, a.wait_ns))) break;
                     mbar_expect_tx(&bar->b_full[s], (uint32_t)(a.dkb * BOXB));
                     for (int kd = 0; kd < a.dkb; ++kd)
-                        tma_load_2d(sB + (size_t)(s * a.dkb + kd) * BOXB, &tmL, kd * 64, ly + n * NT, &bar->b_full[s]);
+                        tma_load_2d(sB + (size_t)(s * a.dkb + kd) * BOXB, &tmL, kd * 64,
+                                    ly + (int)dbg_clamp(n * NT, 0, a.C, a.status), &bar->b_full[s]);
                 }
             }
             // wind down: every load issued has landed before the CTA may exit

@@ -24,7 +24,23 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.EXPORTED)
-    assert lib.hsa_abi_version() == 4
+    assert lib.hsa_abi_version() == 5
+    assert lib.hsa_debug_checks() == (1 if _native.DEBUG else 0)
+
+
+def test_debug_library_exports_every_declared_symbol():
+    """The HSA_DEBUG build (device-side index checks) has the same ABI and says so."""
+    path = os.path.join(ROOT, "landmark_guided_chunk_b200", "libhsa_b200_debug.so")
+    if not os.path.exists(path):
+        from landmark_guided_chunk_b200 import build
+        build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(dbg, n), n
+    dbg.hsa_abi_version.restype = ctypes.c_int
+    dbg.hsa_debug_checks.restype = ctypes.c_int
+    assert dbg.hsa_abi_version() == 5
+    assert dbg.hsa_debug_checks() == 1
 
 
 def test_status_strings():

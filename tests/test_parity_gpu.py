@@ -121,6 +121,9 @@ def test_tensor_core_paths_are_the_ones_planned():
     # long decode scans in bf16: the streaming mma.sync scan with the merge folded in
     assert tuple(_plan(workload("decode_1m"))["select"]) == ("mma_split", 1)
     assert tuple(_plan(DECODE_SMALL[3])["select"]) == ("mma_split", 1)
+    # hsa_forward runs the decode scan and the gather as one launch; prefill does not fuse
+    assert _plan(workload("decode_1m"))["forward_fused"] and _plan(workload("decode_16m"))["forward_fused"]
+    assert not _plan(workload("prefill_bf16"))["forward_fused"]
 
 
 DECODE_SMALL = [
@@ -269,6 +272,37 @@ def test_full_decode_workload(name):
             for j in range(p.Hkv):
                 assert c in idx[b, 0, j, :keff[b, 0, j]], f"planted chunk {c} missed (b={b}, kv={j})"
     del r
+    torch.cuda.empty_cache()
+
+
+FUSED = [q for q in DECODE_SMALL if q.name in ("decode_split", "decode_router", "decode_s32_g8")]
+
+
+@pytest.mark.parametrize("p", FUSED + [workload("decode_1m")], ids=lambda p: p.name)
+def test_fused_decode_step_equals_select_then_attend(p):
+    """The fused decode launch (scan, then each published row's gather) gives
+    the selection of hsa_select bit for bit and the O of hsa_attend on it (up
+    to the order of the fp32 accumulator additions), on the same workspace
+    called repeatedly (its publication slots and counters are reset per call)."""
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, torch.bfloat16,
+                            hsa._native.HSA_FLAG_LANDMARKS_READY)
+    assert hsa.plan(prob)["forward_fused"], hsa.plan(prob)
+    inp = make_inputs(p, seed=11, device="cuda")
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
+    L = hsa.landmarks(K, W, p.S)
+    ws = hsa.alloc_workspace(prob)
+    idx, sc, ke = hsa.select(Q, L, p.S, p.k, p.tau, p.q_pos0, Tkv=p.Tkv, ws=ws)
+    O_ref = hsa.attend(Q, K, V, idx, sc, ke, p.S, p.k, p.tau, p.q_pos0, ws=ws)
+    hsa.device_status(ws)
+    for rep in range(3):
+        O, _, idx2, sc2, ke2 = hsa.forward(Q, K, V, None, p.S, p.k, p.tau, p.q_pos0, L=L, landmarks_ready=True,
+                                           return_selection=True, ws=ws)
+        hsa.device_status(ws)
+        assert torch.equal(idx2, idx) and torch.equal(ke2, ke) and torch.equal(sc2, sc), f"repeat {rep}"
+        err = (O.float() - O_ref.float()).abs().max().item()
+        scale = O_ref.float().abs().max().item()
+        assert err <= 2 ** -7 * max(scale, 1.0), f"repeat {rep}: fused O differs by {err} (max |O| {scale})"
+    del inp, Q, K, V, L, ws
     torch.cuda.empty_cache()
 
 
