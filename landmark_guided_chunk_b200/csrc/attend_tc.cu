@@ -43,7 +43,6 @@ namespace {
 
 using namespace sm100;
 
-constexpr int D = 128;           // head dim of this kernel
 constexpr int MROWS = 128;       // M of every tile (TOK tokens x G heads)
 constexpr int SCAN_BLK = 4096;   // elements per first-level scan block
 constexpr int PITCH = 36;        // staging row pitch (floats) for a 32-column slice
@@ -69,7 +68,8 @@ struct AttTcArgs {
     int32_t *pairs;              // [rows * kmax]  (t << 5) | slot
     float *pair_w;               // [rows * kmax]  fusion weight of each pair
     int4 *tiles;                 // (phase, chunk, first pair, pairs in tile)
-    float *ringbuf;              // [2*NB][TB][G][D]
+    float *ringbuf;              // [2*NB][TB][G][d]
+    int d;                       // head dim (64 or 128)
     uint32_t *status;
 };
 
@@ -83,9 +83,9 @@ __device__ __forceinline__ int phase_of(const AttTcArgs &a, int b, int j, int t)
 }
 
 // ring slot of phase p
-__device__ __forceinline__ float *slot_of(const AttTcArgs &a, int p) {
+__device__ __forceinline__ float *slot_of(const AttTcArgs &a, int p) {   // accumulator rows of d floats
     const int s = ((p / NB) & 1) * NB + (p % NB);
-    return a.ringbuf + (size_t)s * TB * a.G * D;
+    return a.ringbuf + (size_t)s * TB * a.G * a.d;
 }
 
 // ---------------------------------------------------------------------------- helper kernels
@@ -376,9 +376,12 @@ __device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
 
 // Rows (token, head) of the phases in batch `bt`: accumulators -> bf16 O,
 // accumulators zeroed.  Warps of the whole grid take groups of 8 consecutive
-// rows (8 loads in flight per lane).
+// rows (2*D float4, D/16 loads in flight per lane).
+template <int D>
 __device__ void finalize_batch(const AttTcArgs &a, __nv_bfloat16 *__restrict__ O, int bt, int gwarp, int nwarps,
                                int lane) {
+    constexpr int RV = D / 4;            // float4 per row
+    constexpr int NU = 8 * RV / 32;      // float4 per lane per group of 8 rows
     const int p0 = bt * NB, p1 = min(a.nphase, p0 + NB);
     const int rows_per_phase = TB * a.G;   // a multiple of 8
     const long long ngroups = (long long)(p1 - p0) * rows_per_phase / 8;
@@ -388,37 +391,41 @@ __device__ void finalize_batch(const AttTcArgs &a, __nv_bfloat16 *__restrict__ O
         const int rr0 = (int)(e0 % rows_per_phase);
         const int bj = p / a.ntb, tbi = p % a.ntb;
         const int b = bj / a.Hkv, j = bj % a.Hkv;
-        float4 *acc = reinterpret_cast<float4 *>(slot_of(a, p) + (size_t)rr0 * D) + lane;
-        float4 v[8];
+        float4 *acc = reinterpret_cast<float4 *>(slot_of(a, p) + (size_t)rr0 * D);
+        float4 v[NU];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(acc + u * (D / 4));
+        for (int u = 0; u < NU; ++u) v[u] = __ldcg(acc + lane + 32 * u);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int rr = rr0 + u;
+        for (int u = 0; u < NU; ++u) {
+            const int e = lane + 32 * u;   // float4 e of the group: row rr0 + e / RV, columns 4 (e % RV) ..
+            const int rr = rr0 + e / RV;
             const int t = tbi * TB + rr / a.G, g = rr % a.G;
-            __stcg(acc + u * (D / 4), make_float4(0.f, 0.f, 0.f, 0.f));
+            __stcg(acc + e, make_float4(0.f, 0.f, 0.f, 0.f));
             if (t < a.Tq) {
                 __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y), hi = __floats2bfloat162_rn(v[u].z, v[u].w);
                 uint2 pk;
                 pk.x = *reinterpret_cast<uint32_t *>(&lo);
                 pk.y = *reinterpret_cast<uint32_t *>(&hi);
-                reinterpret_cast<uint2 *>(O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + g) * D)[lane] = pk;
+                reinterpret_cast<uint2 *>(O + (((size_t)b * a.Tq + t) * a.H + (size_t)j * a.G + g) * D)[e % RV] = pk;
             }
         }
     }
 }
 
+template <int D>
 __global__ void __launch_bounds__(NT_ATT, 1)
     att_main_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __nv_bfloat16 *__restrict__ Q, __nv_bfloat16 *__restrict__ O, AttTcArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.S;
+    constexpr int NBX = D / 64;                            // 64-column boxes per row of Q, K, V
+    constexpr int QTILE = MROWS * D * 2;                   // one Q tile: NBX boxes of 128 rows x 128 B
     const int kv_bytes = S * 128;                          // one 64-column box of S rows
     const int p_bytes = (S / 64) * 16384;                  // one P tile
-    uint8_t *sQ = base;                                    // nsq x 32 KB
-    uint8_t *sKV = sQ + (size_t)a.nsq * 32768;             // nskv x (K: 2 boxes, V: 2 boxes)
-    uint8_t *sP = sKV + (size_t)a.nskv * 4 * kv_bytes;     // 2 P buffers x p_bytes
+    uint8_t *sQ = base;                                    // nsq x QTILE
+    uint8_t *sKV = sQ + (size_t)a.nsq * QTILE;             // nskv x (K: NBX boxes, V: NBX boxes)
+    uint8_t *sP = sKV + (size_t)a.nskv * 2 * NBX * kv_bytes;   // 2 P buffers x p_bytes
     float *stg = reinterpret_cast<float *>(sP + 2 * (size_t)p_bytes);   // 8 O warps x 32 x PITCH
     TileRows *info = reinterpret_cast<TileRows *>(stg + 8 * 32 * PITCH);      // NINFO stages
     AttBars *bar = reinterpret_cast<AttBars *>(info + NINFO);
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 
     // finalise the previous batch (its slots are not touched by this batch's tiles)
     if (a.batch > 0)
-        finalize_batch(a, O, a.batch - 1, blockIdx.x * (NT_ATT / 32) + warp, gridDim.x * (NT_ATT / 32), lane);
+        finalize_batch<D>(a, O, a.batch - 1, blockIdx.x * (NT_ATT / 32) + warp, gridDim.x * (NT_ATT / 32), lane);
     if (a.batch >= a.nbatch) return;
 
     if (threadIdx.x == 0) {
@@ -523,9 +530,9 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                     const int t = (int)dbg_clamp(pr[h] >> 5, t0, min(a.Tq, t0 + TB), a.status);
                     src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
                 }
-                const uint32_t dq = smem_u32(sQ + sq * 32768) + (r >> 3) * 1024 + (r & 7) * 128;
+                const uint32_t dq = smem_u32(sQ + sq * QTILE) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
+                for (int x = 0; x < D / 8; ++x) {
                     const int kb = x >> 3, cx = x & 7;
                     cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
                 }
@@ -557,13 +564,14 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 const int cz = (int)dbg_clamp(e.y, 0, a.C, a.status);   // the bucket's chunk
                 const int skv = nload % a.nskv, ikv = nload / a.nskv;
                 if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
-                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(4 * kv_bytes));
-                uint8_t *dk = sKV + (size_t)skv * 4 * kv_bytes;
+                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(2 * NBX * kv_bytes));
+                uint8_t *dk = sKV + (size_t)skv * 2 * NBX * kv_bytes;
                 const int z = Tb * a.Tcap + cz * S;
-                tma_load_3d(dk, &tmK, 0, Tj, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + kv_bytes, &tmK, 64, Tj, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + 2 * kv_bytes, &tmV, 0, Tj, z, &bar->kv_full[skv]);
-                tma_load_3d(dk + 3 * kv_bytes, &tmV, 64, Tj, z, &bar->kv_full[skv]);
+#pragma unroll
+                for (int kb = 0; kb < NBX; ++kb) {
+                    tma_load_3d(dk + kb * kv_bytes, &tmK, 64 * kb, Tj, z, &bar->kv_full[skv]);
+                    tma_load_3d(dk + (NBX + kb) * kv_bytes, &tmV, 64 * kb, Tj, z, &bar->kv_full[skv]);
+                }
                 ++nload;
             }
             // wind down: the K/V loads issued have all landed
@@ -603,10 +611,10 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 }
                 tc_fence_after();
                 const uint32_t s_tmem = tmem + (i & 1) * 128;
-                const uint32_t qa = smem_u32(sQ + sq * 32768);
-                const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 4 * kv_bytes);
+                const uint32_t qa = smem_u32(sQ + sq * QTILE);
+                const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t a_addr = qa + (kk >> 2) * 16384 + (kk & 3) * 32;
                     const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + (kk & 3) * 32;
                     umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
@@ -632,7 +640,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                 const int skv = li % a.nskv;
                 const uint32_t o_tmem = tmem + 256 + b * 128;
                 const uint32_t pa = smem_u32(sP + b * p_bytes);
-                const uint32_t vb = smem_u32(sKV + (size_t)skv * 4 * kv_bytes) + 2 * kv_bytes;
+                const uint32_t vb = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes) + NBX * kv_bytes;
                 for (int kk = 0; kk < S / 16; ++kk) {
                     // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
                     // V: MN-major, keys kk*16..+15 are two 8-row groups starting (kk*16)*128 B
@@ -708,7 +716,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             if (lane == 0) mbar_arrive(&bar->l_full[b]);
         }
     } else if (warp >= 8) {
-        // ------------------------------------------------------------ O drain: thread = tile row, 64 of its columns
+        // ------------------------------------------------------------ O drain: thread = tile row, D/2 of its columns
         const int ew = warp & 3;               // TMEM lane quadrant
         const int hf = (warp - 8) >> 2;        // column half
         const int r = ew * 32 + lane;
@@ -741,12 +749,12 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             if (!(ok = mbar_wait(&bar->o_full[b], k & 1, abort, a.status))) break;
             tc_fence_after();
             float *acc_slot = slot_of(a, Tp) + 4 * (lane & 7);
-            const uint32_t o_base = tmem + lane_off + 256 + b * 128 + hf * 64;
-            for (int q = 0; q < 2; ++q) {
+            const uint32_t o_base = tmem + lane_off + 256 + b * 128 + hf * (D / 2);
+            for (int q = 0; q < D / 64; ++q) {
                 uint32_t orr[32];
                 tmem_ld32(o_base + q * 32, orr);
                 tmem_wait_ld();
-                if (q == 1) {
+                if (q == D / 64 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&bar->o_empty[b]);
@@ -758,7 +766,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
                         make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
                                     __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
                 __syncwarp();
-                const int col = hf * 64 + q * 32;
+                const int col = hf * (D / 2) + q * 32;
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
                     if (dstoff[rr] >= 0) {
@@ -784,7 +792,8 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 // ---------------------------------------------------------------------------- host side
 
 bool attend_tc_supported(const Prob &p) {
-    if (!(p.dtype == HSA_BF16 && p.d == D && (p.S == 64 || p.S == 128) && p.G <= 16 && (32 % p.G) == 0 &&
+    // G need not divide the 128 tile rows: a tile holds floor(128 / G) tokens and the last rows are padding
+    if (!(p.dtype == HSA_BF16 && (p.d == 64 || p.d == 128) && (p.S == 64 || p.S == 128) && p.G <= 16 &&
           p.C >= 1 && p.Tq >= 1 && p.kmax <= 32 && p.Tq < (1 << 26) && (long long)p.B * p.Tcap < (1ll << 31)))
         return false;
     // the second scan level is one block of 1024 threads over SCAN_BLK-bucket blocks
@@ -806,7 +815,7 @@ AttTcLayout attend_tc_layout(const Prob &p) {
     const size_t pairs = (size_t)p.rows * p.kmax;
     L.max_tiles = pairs / L.tok + (size_t)L.nbucket + 1;
     L.counter_ints = 2 * (size_t)L.nbucket;
-    L.ring_bytes = (size_t)L.ring * TB * p.G * D * sizeof(float);
+    L.ring_bytes = (size_t)L.ring * TB * p.G * p.d * sizeof(float);
     return L;
 }
 
@@ -832,9 +841,10 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.ntb = L.ntb;
     a.nphase = L.nphase;
     a.nbucket = L.nbucket;
-    // S=64: double-buffered Q and K/V (~200 KB of smem); S=128: single
-    a.nsq = p.S <= 64 ? 2 : 1;
-    a.nskv = p.S <= 64 ? 2 : 1;
+    // double-buffered Q and K/V where shared memory allows (d=128, S=128: single, ~200 KB)
+    a.nsq = (p.S <= 64 || p.d == 64) ? 2 : 1;
+    a.nskv = (p.S <= 64 || p.d == 64) ? 2 : 1;
+    a.d = p.d;
     a.nbatch = (L.nphase + NB - 1) / NB;
     a.q_pos0 = p.q_pos0;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)p.d);
@@ -886,17 +896,18 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     const uint32_t box[3] = {64, 1, (uint32_t)p.S};
     if ((e = make_tmap_3d(&mk, K, dims, strides, box)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mv, V, dims, strides, box)) != cudaSuccess) return e;
-    const size_t smem = 1024 + (size_t)a.nsq * 32768 + (size_t)a.nskv * 4 * p.S * 128 + 2 * (size_t)(p.S / 64) * 16384 +
-                        8 * 32 * PITCH * sizeof(float) + NINFO * sizeof(TileRows) + sizeof(AttBars);
-    if ((e = cudaFuncSetAttribute(att_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-        cudaSuccess)
+    const size_t smem = 1024 + (size_t)a.nsq * 128 * p.d * 2 + (size_t)a.nskv * 2 * (p.d / 64) * p.S * 128 +
+                        2 * (size_t)(p.S / 64) * 16384 + 8 * 32 * PITCH * sizeof(float) + NINFO * sizeof(TileRows) +
+                        sizeof(AttBars);
+    auto kern = p.d == 64 ? att_main_kernel<64> : att_main_kernel<128>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
         return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     for (int bt = 0; bt <= a.nbatch; ++bt) {
         a.batch = bt;
-        att_main_kernel<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
+        kern<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -87,6 +87,19 @@ SMALL = [
 ]
 
 
+# shapes on the tensor-core attention beyond prefill_bf16's: group sizes that do not divide the 128
+# rows of a tile (padding rows), and head dim 64
+ODD_GROUPS = [
+    Problem(B=2, Tq=64 * 33 + 21, Tkv=64 * 33 + 21, H=8, Hkv=2, d=64, S=64, k=8, dtype="bf16", name="bf16_d64_s64"),
+    Problem(B=1, Tq=128 * 14 + 77, Tkv=128 * 14 + 77, H=12, Hkv=2, d=64, S=128, k=6, tau=0.05, dtype="bf16",
+            name="bf16_d64_s128_g6"),
+    Problem(B=1, Tq=64 * 30 + 11, Tkv=64 * 30 + 11, H=12, Hkv=2, d=128, S=64, k=8, dtype="bf16", name="bf16_g6"),
+    Problem(B=2, Tq=64 * 17 + 40, Tkv=64 * 17 + 40, H=6, Hkv=2, d=128, S=64, k=5, dtype="bf16", name="bf16_g3"),
+    Problem(B=2, Tq=128 * 12 + 3, Tkv=128 * 12 + 3, H=12, Hkv=1, d=128, S=128, k=4, tau=0.05, dtype="bf16",
+            name="bf16_g12_router"),
+]
+
+
 def _plan(p: Problem, simt=False):
     return hsa.plan(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau,
                                      torch.bfloat16 if p.dtype == "bf16" else torch.float32,
@@ -99,6 +112,13 @@ def test_small_prefill_all_rows(p):
     assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
     print(f"{p.name}: end-to-end selection mismatch vs the oracle's own landmarks: {r['e2e_mismatch']:.4f}")
     assert r["e2e_mismatch"] <= 0.05
+
+
+@pytest.mark.parametrize("p", ODD_GROUPS, ids=lambda p: p.name)
+def test_tensor_attention_other_shapes(p):
+    assert _plan(p)["attend"][0] == "tensor"
+    r = run_case(p)
+    assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
 
 
 @pytest.mark.parametrize("p", [q for q in SMALL if q.dtype == "bf16"], ids=lambda p: p.name)
