@@ -50,8 +50,8 @@ struct WsLayout {
     size_t sel_cnt;      // split select (tensor-core scan): per-row completion counters, right after the header
     size_t att_cnt;      // gather attend: per-row completion counters, right after the header
     size_t att_acc;      // gather attend: per-row fp32 accumulators (rows x G x d), right after the counters
-    size_t dec_ready;    // fused decode step: publication slots (rows int32), zeroed with the status word
-    size_t dec_ctr;      // fused decode step: rows published, units claimed (2 int32), zeroed likewise
+    size_t dec_desc;     // fused decode step: unit descriptors (rows x kmax x 8 B), zeroed with the status word
+    size_t dec_ctr;      // fused decode step: units claimed (int32), zeroed likewise
     bool fused_decode;   // hsa_forward runs the decode scan and the gather as one launch
     size_t clear_bytes;  // bytes from the workspace start zeroed before every call (status word, counters)
     size_t total;
@@ -310,7 +310,7 @@ cudaError_t launch_select_stream(const Prob &p, const void *Q, const void *L, in
 bool decode_fused_supported(const Prob &p, int grid, int sms);
 cudaError_t launch_decode_fused(const Prob &p, const void *Q, const void *K, const void *V, const void *L,
                                 int32_t *idx, float *score, int32_t *keff, void *O, float2 *lists, int32_t *cnt,
-                                int32_t *ready, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
+                                unsigned long long *desc, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
                                 int grid, int maxe, cudaStream_t st);
 // part != null: partial mode (o_i of every (row, slot) into part [rows][kmax][G][d]; no fusion, O unused)
 cudaError_t launch_attend_gather(const Prob &p, const void *Q, const void *K, const void *V, const int32_t *idx,

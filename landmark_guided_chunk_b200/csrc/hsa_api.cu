@@ -88,8 +88,8 @@ WsLayout ws_layout(const Prob &p) {
     // Decode with both of those kernels: hsa_forward fuses them into one launch.
     w.fused_decode = w.stream_select && w.gather_attend && decode_fused_supported(p, w.stream_grid, device_sms());
     if (w.fused_decode) {
-        w.dec_ready = take(rows * sizeof(int32_t));
-        w.dec_ctr = take(2 * sizeof(int32_t));
+        w.dec_desc = take(rows * (size_t)p.kmax * sizeof(unsigned long long));
+        w.dec_ctr = take(sizeof(int32_t));
     }
     w.clear_bytes = off > 256 ? off : sizeof(uint32_t);
     w.sel_idx = take(rows * p.kmax * sizeof(int32_t));
@@ -449,7 +449,7 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     int32_t *skf = keff ? keff : reinterpret_cast<int32_t *>(wsb + w.sel_keff);
     if (w.fused_decode && p.C > 0) {
         e = launch_decode_fused(p, Q, K, V, L, sidx, ssc, skf, O, reinterpret_cast<float2 *>(wsb + w.split_lists),
-                                reinterpret_cast<int32_t *>(wsb + w.sel_cnt), reinterpret_cast<int32_t *>(wsb + w.dec_ready),
+                                reinterpret_cast<int32_t *>(wsb + w.sel_cnt), reinterpret_cast<unsigned long long *>(wsb + w.dec_desc),
                                 reinterpret_cast<int32_t *>(wsb + w.dec_ctr), reinterpret_cast<int32_t *>(wsb + w.att_cnt),
                                 reinterpret_cast<float *>(wsb + w.att_acc), reinterpret_cast<uint32_t *>(wsb + w.hdr),
                                 w.stream_grid, w.stream_maxe, st);

@@ -23,14 +23,14 @@
 // selection, with the router's k_eff.
 //
 // Fused decode step (hsa_forward): the same launch then does the chunk
-// attention and the fusion.  The warp that completes a row publishes it
-// (release store of row + 1 into the next slot of a publication list), and
-// once a CTA's scan is done all of its warps become gather workers with one
-// K/V stage each, carved from the now idle ring: a worker claims the next
-// (publication slot, kept slot) unit from a global counter, waits (bounded)
-// until that slot is published, stages the chunk's K and V by TMA and adds
-// w_i * o_i / l_i into the row's fp32 accumulator; whoever finishes a row's
-// last kept slot converts it to bf16 O.  Rows published early are gathered
+// attention and the fusion.  The warp that completes a row publishes, per
+// kept slot i, a unit descriptor (chunk + 1, fusion weight w_i) with a
+// release store (empty slots get a marker), and once a CTA's scan is done all
+// of its warps become gather workers with one K/V stage each, carved from the
+// now idle ring: a worker claims the next (row, slot) unit from a global
+// counter, loads the row's query heads, waits (bounded) for the descriptor,
+// stages the chunk's K and V by TMA and adds w_i * o_i / l_i into the row's
+// fp32 accumulator; whoever finishes a row's last slot converts it to bf16 O.  Rows published early are gathered
 // while the slowest CTAs still scan, and the gather needs no launch of its
 // own.  Workers wait only on rows, and rows depend only on the scan, so the
 // launch is cooperative (every CTA resident) and cannot deadlock.
@@ -68,8 +68,8 @@ struct StreamArgs {
     // fused decode step only
     int B, Tcap, nunits, nwg;   // units = rows * kmax; gather workers per CTA
     float scale;                // 1/sqrt(d)
-    int32_t *ready;             // [rows] publication slots: row + 1, 0 until published
-    int32_t *ctr;               // [0] rows published, [1] units claimed
+    unsigned long long *desc;   // [rows][kmax] unit descriptors: (chunk + 1) << 32 | bits(w), EMPTY_SLOT, 0 until published
+    int32_t *ctr;               // [0] units claimed
     int32_t *att_cnt;           // [rows] kept slots gathered per row
     float *acc;                 // [rows][G][d] fp32 accumulators
     __nv_bfloat16 *O;
@@ -88,24 +88,26 @@ __device__ __forceinline__ bool in_range(long long x, long long n, uint32_t *sta
     return false;
 }
 
-__device__ __forceinline__ void st_release_gpu(int32_t *p, int v) {
-    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void st_release_gpu64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_acquire_gpu64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
+constexpr unsigned long long EMPTY_SLOT = 0xffffffff00000000ull;   // a published slot past the row's keff
 
-// Wait until publication slot *p is set; 0 if the wait expired or another
+// Wait until unit descriptor *p is published; 0 if the wait expired or another
 // CTA's wait did (the status word carries DEV_TIMEOUT).
-__device__ __forceinline__ int wait_published(const int32_t *p, uint32_t *status, volatile int *abort) {
-    int v = ld_acquire_gpu(p);
+__device__ __forceinline__ unsigned long long wait_published(const unsigned long long *p, uint32_t *status,
+                                                             volatile int *abort) {
+    unsigned long long v = ld_acquire_gpu64(p);
     if (v != 0) return v;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         __nanosleep(128);
-        if ((v = ld_acquire_gpu(p)) != 0) return v;
+        if ((v = ld_acquire_gpu64(p)) != 0) return v;
         if (*abort || (__ldcv(status) & DEV_TIMEOUT)) return 0;
         if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
             *abort = 1;
@@ -138,12 +140,11 @@ constexpr int gather_stage_bytes() {
 }
 
 // The gather phase of the fused decode step (all of a CTA's warps, after its
-// scan): claim units, wait for their rows, stage the chunks, accumulate.
+// scan): claim units, wait for their descriptors, stage the chunks, accumulate.
 template <int D, int S>
 __device__ __forceinline__ void gather_phase(const StreamArgs &a, uint8_t *base, uint64_t *gbar, volatile int *abort,
                                              const CUtensorMap &tmK, const CUtensorMap &tmV,
-                                             const __nv_bfloat16 *__restrict__ Q, const int32_t *idx,
-                                             const float *score, const int32_t *keff) {
+                                             const __nv_bfloat16 *__restrict__ Q) {
     constexpr int NB = D / 64, BOX = S * 128, STAGE = gather_stage_bytes<D, S>();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp >= a.nwg) return;
@@ -153,74 +154,58 @@ __device__ __forceinline__ void gather_phase(const StreamArgs &a, uint8_t *base,
     bool pend_k = false, pend_v = false;   // copies issued and not yet consumed
     while (!*abort) {
         int u = 0;
-        if (lane == 0) u = atomicAdd(&a.ctr[1], 1);
+        if (lane == 0) u = atomicAdd(&a.ctr[0], 1);
         u = __shfl_sync(FULL, u, 0);
         if (u >= a.nunits) break;
-        const int pos = u / a.kmax, i = u - pos * a.kmax;
-        int rv = 0;
-        if (lane == 0) rv = wait_published(&a.ready[pos], a.status, abort);
-        rv = __shfl_sync(FULL, rv, 0);
-        if (rv == 0 || !in_range(rv - 1, a.rows, a.status)) break;
-        const int row = rv - 1;
+        const int row = u / a.kmax;
         const int j = row % a.Hkv, b = row / a.Hkv;
         const size_t qrow = ((size_t)b * a.H + (size_t)j * a.G) * D;   // Q [B][1][H][d]
-        // one round trip: keff, the slot's chunk, the row's retrieval scores, Q fragments
-        int ke = 0, c = 0;
-        if (lane == 0) {
-            ke = __ldcg(&keff[row]);
-            c = __ldcg(&idx[(size_t)row * a.kmax + i]);
-        }
-        const float sv = lane < a.kmax ? __ldcg(&score[(size_t)row * a.kmax + lane]) : -INFINITY;
+        // the group's query heads while the row's selection may still be in progress
         uint32_t qa[D / 16][4];
         load_q_frags<D>(Q + qrow, a.G, qa);
-        ke = __shfl_sync(FULL, ke, 0);
-        c = __shfl_sync(FULL, c, 0);
-        if (i >= ke) {
-            if (ke == 0 && i == 0)   // no candidates: the output is zero
-                for (int e = lane; e < a.G * D; e += 32) a.O[qrow + e] = __float2bfloat16(0.f);
-            continue;
-        }
-        const bool cok = in_range(c, a.ncand, a.status);
-        if (cok && lane == 0) {
-            const int z = b * a.Tcap + c * S;
-            mbar_expect_tx(mbk, (uint32_t)(NB * BOX));
-            mbar_expect_tx(mbv, (uint32_t)(NB * BOX));
+        unsigned long long dv = 0;
+        if (lane == 0) dv = wait_published(&a.desc[u], a.status, abort);
+        dv = __shfl_sync(FULL, dv, 0);
+        if (dv == 0) break;
+        if (dv != EMPTY_SLOT) {
+            const int c = (int)(dv >> 32) - 1;
+            const float w = __uint_as_float((uint32_t)dv);
+            if (in_range(c, a.ncand, a.status)) {
+                if (lane == 0) {
+                    const int z = b * a.Tcap + c * S;
+                    mbar_expect_tx(mbk, (uint32_t)(NB * BOX));
+                    mbar_expect_tx(mbv, (uint32_t)(NB * BOX));
 #pragma unroll
-            for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + kb * BOX, &tmK, 64 * kb, j, z, mbk);
+                    for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + kb * BOX, &tmK, 64 * kb, j, z, mbk);
 #pragma unroll
-            for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + (NB + kb) * BOX, &tmV, 64 * kb, j, z, mbv);
+                    for (int kb = 0; kb < NB; ++kb) tma_load_3d(stage + (NB + kb) * BOX, &tmV, 64 * kb, j, z, mbv);
+                }
+                pend_k = pend_v = true;
+                bool ok = mbar_wait(mbk, phase, abort, a.status);
+                if (ok) pend_k = false;
+                if (!__all_sync(FULL, ok)) break;
+                const uint32_t sk = smem_u32(stage);
+                float *racc = a.acc + (size_t)row * a.G * D;
+                auto wait_v = [&]() {
+                    bool v = mbar_wait(mbv, phase, abort, a.status);
+                    if (v) pend_v = false;
+                    return __all_sync(FULL, v);
+                };
+                if (!chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, w, 0,
+                                         [&](int g, int col, float x, float y) { red_add2(racc + (size_t)g * D + col, x, y); },
+                                         wait_v))
+                    break;
+                phase ^= 1u;   // both copies consumed
+            }
         }
-        if (cok) pend_k = pend_v = true;
-        // this slot's fusion weight: softmax over the row's kept retrieval scores
-        const float xs = lane < ke ? sv : -INFINITY;
-        const float m = warp_max(xs);
-        const float ex = lane < ke ? expf(xs - m) : 0.f;
-        const float w = __shfl_sync(FULL, ex, i) / warp_sum(ex);
-        if (cok) {
-            bool ok = mbar_wait(mbk, phase, abort, a.status);
-            if (ok) pend_k = false;
-            if (!__all_sync(FULL, ok)) break;
-            const uint32_t sk = smem_u32(stage);
-            float *racc = a.acc + (size_t)row * a.G * D;
-            auto wait_v = [&]() {
-                bool v = mbar_wait(mbv, phase, abort, a.status);
-                if (v) pend_v = false;
-                return __all_sync(FULL, v);
-            };
-            if (!chunk_unit<D, S, D>(sk, sk + NB * BOX, qa, a.G, a.scale, w, 0,
-                                     [&](int g, int col, float x, float y) { red_add2(racc + (size_t)g * D + col, x, y); },
-                                     wait_v))
-                break;
-            phase ^= 1u;   // both copies consumed
-        }
-        // this slot is done; whoever completes the row converts its accumulator to O
+        // this slot is done (empty ones too); whoever completes the row's kmax slots converts it to O
         __threadfence();
         __syncwarp();
         int last = 0;
-        if (lane == 0) last = atomicAdd(&a.att_cnt[row], 1) == ke - 1;
+        if (lane == 0) last = atomicAdd(&a.att_cnt[row], 1) == a.kmax - 1;
         if (__shfl_sync(FULL, last, 0)) {
             __threadfence();
-            acc_to_bf16(a.acc + (size_t)row * a.G * D, a.O + qrow, a.G * D);
+            acc_to_bf16(a.acc + (size_t)row * a.G * D, a.O + qrow, a.G * D);   // zeros for a row without candidates
         }
         __syncwarp();   // the stage is free for the next unit
     }
@@ -407,13 +392,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         }
         if (lane == 0) keff[row] = ke;
         if constexpr (FUSE) {
-            // publish the row: every lane's selection writes, then the slot
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) {
-                const int pos = atomicAdd(&a.ctr[0], 1);
-                if (in_range(pos, a.rows, a.status)) st_release_gpu(&a.ready[pos], (int)row + 1);
-            }
+            // publish each slot's unit: its chunk and its fusion weight (softmax of the kept scores)
+            const float m = __shfl_sync(FULL, v, 0);   // the list is sorted: the row's best score
+            const float ex = lane < ke ? expf(v - m) : 0.f;
+            const float w = ex / warp_sum(ex);
+            if (lane < a.kmax)
+                st_release_gpu64(&a.desc[row * a.kmax + lane],
+                                 lane < ke ? ((unsigned long long)(uint32_t)(id + 1) << 32) | __float_as_uint(w)
+                                           : EMPTY_SLOT);
         }
     };
     finish_row();
@@ -422,7 +408,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         // writes after this CTA's generic accesses to the same shared memory)
         fence_proxy_async_smem();
         __syncthreads();
-        gather_phase<D, S>(a, base, gbar, &bar.abort, tmK, tmV, Q, idx, score, keff);
+        gather_phase<D, S>(a, base, gbar, &bar.abort, tmK, tmV, Q);
     }
 }
 
@@ -544,14 +530,14 @@ static cudaError_t launch_fused_ds(StreamArgs a, const CUtensorMap &ml, const CU
 
 cudaError_t launch_decode_fused(const Prob &p, const void *Q, const void *K, const void *V, const void *L,
                                 int32_t *idx, float *score, int32_t *keff, void *O, float2 *lists, int32_t *cnt,
-                                int32_t *ready, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
+                                unsigned long long *desc, int32_t *ctr, int32_t *att_cnt, float *acc, uint32_t *status,
                                 int grid, int maxe, cudaStream_t st) {
     StreamArgs a = stream_args(p, status, grid, maxe);
     a.B = p.B;
     a.Tcap = p.Tcap;
     a.nunits = (int)(p.rows * p.kmax);
     a.scale = 1.0f / sqrtf((float)p.d);
-    a.ready = ready;
+    a.desc = desc;
     a.ctr = ctr;
     a.att_cnt = att_cnt;
     a.acc = acc;
