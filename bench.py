@@ -283,6 +283,24 @@ def run_router(args, world, rank, local, pk):
     return out
 
 
+def run_prefill_line(args, world, rank, local, pk, name):
+    """Another prefill workload (prefill_bf16_d64: the prefill_bf16 shapes at head
+    dim 64) through the same forward: time per stage, tokens/s, roofline."""
+    dev = torch.device("cuda", local)
+    ps = PrefillSetup(name, args.seed + rank, dev)
+    p = ps.p
+    steps = max(1, min(args.steps, 10))
+    ms, stage_ms, keff_sum, _ = ps.time_stages(steps, args.warmup, world)
+    stages_out, roof = ps.roofline(stage_ms, keff_sum, pk)
+    out = {"workload": f"{p.name}: B{p.B} T{p.Tq} H{p.H} Hkv{p.Hkv} d{p.d} S{p.S} k{p.k}",
+           "ms_per_forward": round(ms, 4), "steps": steps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
+           "stages": stages_out, "roofline": roof,
+           "gpu_launches": steps * sum(ps.plan[x][1] for x in ("landmarks", "select", "attend"))}
+    del ps
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_variants(args, world, rank, local, pk):
     """The two selection variants on the prefill_bf16 shapes, each stage timed
     with CUDA events over back-to-back forwards: Quest block scoring
@@ -475,6 +493,8 @@ def run_b200(args, world, rank, local):
     torch.cuda.empty_cache()
     if not args.no_router and args.workload == "prefill_bf16":
         out["router_bf16"] = run_router(args, world, rank, local, pk)
+    if not args.no_d64 and args.workload == "prefill_bf16":
+        out["prefill_bf16_d64"] = run_prefill_line(args, world, rank, local, pk, "prefill_bf16_d64")
     if not args.no_variants and args.workload == "prefill_bf16":
         out["variants"] = run_variants(args, world, rank, local, pk)
     if not args.no_decode:
@@ -945,6 +965,7 @@ def main():
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass line")
     ap.add_argument("--no-router", action="store_true", help="skip the gap-router prefill line (router_bf16)")
     ap.add_argument("--no-variants", action="store_true", help="skip the selection-variant lines (Quest, refiner)")
+    ap.add_argument("--no-d64", action="store_true", help="skip the head-dim-64 prefill line (prefill_bf16_d64)")
     ap.add_argument("--case", action="store_true",
                     help="single-case driver for profiler captures (see run_case); prints no JSON line")
     ap.add_argument("--iters", type=int, default=3, help="--case: iterations")

@@ -88,6 +88,8 @@ WORKLOADS = {
     "decode_1m": _decode("decode_1m", 8, 1 << 20, 32, 8, 128, 64, 16, planted=8),
     "router_bf16": _prefill("router_bf16", 1, 131072, 32, 8, 128, 128, 8, "bf16", tau=0.02),
     "decode_16m": _decode("decode_16m", 1, 1 << 24, 32, 8, 128, 64, 16, planted=4),
+    # prefill_bf16 at head dim 64 (the tensor-core attention's other width)
+    "prefill_bf16_d64": _prefill("prefill_bf16_d64", 1, 65536, 32, 8, 64, 64, 16, "bf16"),
 }
 
 

@@ -132,7 +132,7 @@ def test_small_prefill_cuda_core_path(p):
 
 def test_tensor_core_paths_are_the_ones_planned():
     # many rows in bf16: tcgen05 scoring and chunk-major tcgen05 attention
-    for name in ("prefill_bf16", "router_bf16"):
+    for name in ("prefill_bf16", "router_bf16", "prefill_bf16_d64"):
         assert _plan(workload(name))["select"][0] == "tensor"
         assert _plan(workload(name))["attend"][0] == "tensor"
     assert _plan(SMALL[1])["select"][0] == "tensor"
@@ -268,7 +268,7 @@ def test_device_status_is_clear_after_calls():
 
 # ------------------------------------------------------------------- full workloads (sampled rows)
 
-@pytest.mark.parametrize("name", ["prefill_bf16", "router_bf16"])
+@pytest.mark.parametrize("name", ["prefill_bf16", "router_bf16", "prefill_bf16_d64"])
 def test_full_prefill_workload_sampled_rows(name):
     p = workload(name)
     r = run_case(p, rows=_rows_sampled(p, 192))
