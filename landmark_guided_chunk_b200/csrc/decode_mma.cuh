@@ -43,11 +43,6 @@ __device__ __forceinline__ uint32_t swz(uint32_t box, int u, int j) {
     return box + (uint32_t)u * 128u + ((uint32_t)(j ^ (u & 7)) << 4);
 }
 
-// Release/acquire fence at GPU scope: paired through a relaxed atomic counter
-// (writes, fence, atomicAdd  ->  atomicAdd, fence, reads), it orders a hand-off
-// between CTAs without the sequentially consistent fence __threadfence() is.
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 __device__ __forceinline__ void red_add2(float *addr, float x, float y) {
     asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(x), "f"(y) : "memory");
 }

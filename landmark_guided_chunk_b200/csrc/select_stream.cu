@@ -199,12 +199,12 @@ __device__ __forceinline__ void gather_phase(const StreamArgs &a, uint8_t *base,
             }
         }
         // this slot is done (empty ones too); whoever completes the row's kmax slots converts it to O
-        fence_acq_rel_gpu();
+        __threadfence();
         __syncwarp();
         int last = 0;
         if (lane == 0) last = atomicAdd(&a.att_cnt[row], 1) == a.kmax - 1;
         if (__shfl_sync(FULL, last, 0)) {
-            fence_acq_rel_gpu();
+            __threadfence();
             acc_to_bf16(a.acc + (size_t)row * a.G * D, a.O + qrow, a.G * D);   // zeros for a row without candidates
         }
         __syncwarp();   // the stage is free for the next unit
@@ -367,23 +367,22 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         float2 *rl = lists + row * (long long)a.maxe * a.kmax;
         if (!in_range(x - x0, a.maxe, a.status) || !in_range(x1 - x0, a.maxe, a.status)) return;
         if (lane < a.kmax) rl[(x - x0) * a.kmax + lane] = make_float2(v, __int_as_float(id));
-        fence_acq_rel_gpu();
-        __syncwarp();
+        __threadfence();
         int last = 0;
         if (lane == 0) last = atomicAdd(&cnt[row], 1) == x1 - x0;
         if (!__shfl_sync(FULL, last, 0)) return;
-        fence_acq_rel_gpu();
+        __threadfence();
         list_init(v, id);
-        // the row's lists, sixteen in flight per round trip (then merged in order)
+        // the row's lists, eight in flight per round trip (then merged in order)
         const int ne = x1 - x0 + 1;
-        for (int e0 = 0; e0 < ne; e0 += 16) {
-            float2 f[16];
+        for (int e0 = 0; e0 < ne; e0 += 8) {
+            float2 f[8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
+            for (int u = 0; u < 8; ++u)
                 f[u] = (e0 + u < ne && lane < a.kmax) ? __ldcg(rl + (e0 + u) * a.kmax + lane)
                                                       : make_float2(-INFINITY, __int_as_float(INT32_MAX));
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
+            for (int u = 0; u < 8; ++u)
                 if (e0 + u < ne) list_merge16(v, id, f[u].x, __float_as_int(f[u].y), a.kmax, lane);
         }
         const int ke = list_keff(v, a.ncand, a.k, a.kmax, a.tau);
