@@ -360,7 +360,7 @@ def run_variants(args, world, rank, local, pk):
     sum_bytes = k_bytes + p.B * p.Hkv * p.C * 2 * p.d * es
     out["quest"] = {
         "ms_per_forward": round(total, 4), "tokens_per_s": round(p.B * p.Tq * world / (total * 1e-3), 1),
-        "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3), "plan": {k2: list(v) for k2, v in qplan.items()},
+        "keff_mean": round(keff_sum / (p.B * p.Tq * p.Hkv), 3), "plan": {k2: (list(v) if isinstance(v, tuple) else v) for k2, v in qplan.items()},
         "stages": {
             "summaries": {"ms": round(ms["summaries"], 4), "bound": "hbm", "unit": "GB/s",
                           "achieved": round(sum_bytes / (ms["summaries"] * 1e-3) / 1e9, 1),
