@@ -30,10 +30,11 @@
 // now idle ring: a worker claims the next (row, slot) unit from a global
 // counter, loads the row's query heads, waits (bounded) for the descriptor,
 // stages the chunk's K and V by TMA and adds w_i * o_i / l_i into the row's
-// fp32 accumulator; whoever finishes a row's last slot converts it to bf16 O.  Rows published early are gathered
-// while the slowest CTAs still scan, and the gather needs no launch of its
-// own.  Workers wait only on rows, and rows depend only on the scan, so the
-// launch is cooperative (every CTA resident) and cannot deadlock.
+// fp32 accumulator; whoever finishes a row's last slot converts it to bf16 O.
+// Rows published early are gathered while the slowest CTAs still scan, and the
+// gather needs no launch of its own.  Workers wait only on rows, and rows
+// depend only on the scan, so the launch is cooperative (every CTA resident)
+// and cannot deadlock.
 #include <algorithm>
 
 #include "common.cuh"
