@@ -187,3 +187,28 @@ def test_quest_flag_host_rules():
     # the refiner needs every weight
     assert _native.lib().hsa_landmarks_refined(ctypes.byref(plain), fake, fake, fake, None, fake, fake, None) == \
         _native.HSA_ERR_INVALID_ARG
+
+
+def test_fused_decode_plan_host_rules():
+    """hsa_forward fuses the decode scan and the gather only for decode-shaped bf16 problems
+    with long contexts that both kernels support, never under Quest scoring, and the
+    fused plan adds no attention launch.  The workspace grows by the unit descriptors."""
+    from landmark_guided_chunk_b200.inputs import workload
+    bf16 = torch_bf16()
+
+    def plan_of(p, flags=0):
+        return hsa.plan(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, bf16, flags))
+
+    for name in ("decode_1m", "decode_16m"):
+        pl = plan_of(workload(name))
+        assert pl["forward_fused"] and pl["select"] == ("mma_split", 1) and pl["attend"] == ("mma_split", 1)
+        assert not plan_of(workload(name), _native.HSA_FLAG_QUEST)["forward_fused"]
+        assert not plan_of(workload(name), _native.HSA_FLAG_SIMT)["forward_fused"]
+    assert not plan_of(workload("prefill_bf16"))["forward_fused"]
+    # a short context (under 2048 candidate chunks) takes the per-row scan: no fusion
+    short = workload("decode_1m").with_(Tkv=64 * 1500, q_pos0=64 * 1500)
+    assert not plan_of(short)["forward_fused"]
+    # the fused layout holds one 8-byte descriptor per (row, slot) on top of the unfused one
+    p = workload("decode_1m")
+    fused = hsa.workspace_size(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, bf16))
+    assert fused >= p.B * p.Hkv * p.k * 8
