@@ -244,6 +244,31 @@ __device__ __forceinline__ bool hist_row(const AttTcArgs &a, int &b, int &j, int
     return t < a.Tq;
 }
 
+// A row's kept slots: chunk indices, and scores or weights.  Rows of kmax
+// 4-byte entries start on 16-byte boundaries when kmax is a multiple of 4 (the
+// buffers are 16-byte aligned), and are then read as 16-byte vectors.
+__device__ __forceinline__ void load_row_slots(const int32_t *idx, const float *val, int ke, int kmax,
+                                               int (&c)[MAX_KMAX], float (&x)[MAX_KMAX]) {
+    if ((kmax & 3) == 0) {
+#pragma unroll
+        for (int q = 0; q < MAX_KMAX / 4; ++q) {
+            if (4 * q < ke) {
+                const int4 ci = reinterpret_cast<const int4 *>(idx)[q];
+                const float4 xv = reinterpret_cast<const float4 *>(val)[q];
+                c[4 * q] = ci.x, c[4 * q + 1] = ci.y, c[4 * q + 2] = ci.z, c[4 * q + 3] = ci.w;
+                x[4 * q] = xv.x, x[4 * q + 1] = xv.y, x[4 * q + 2] = xv.z, x[4 * q + 3] = xv.w;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) {
+                c[i] = idx[i];
+                x[i] = val[i];
+            }
+    }
+}
+
 __global__ void __launch_bounds__(HT) att_count_hist_kernel(AttTcArgs a) {
     extern __shared__ int hist[];   // [C]
     for (int c = threadIdx.x; c < a.C; c += HT) hist[c] = 0;
@@ -258,20 +283,41 @@ __global__ void __launch_bounds__(HT) att_count_hist_kernel(AttTcArgs a) {
             ke = ke < 0 ? 0 : a.kmax;
         }
         const int nc = ncand_of(a, t);
-        const int32_t *ri = a.idx + row * a.kmax;
-        const float *rs = a.score + row * a.kmax;
+        int ci[MAX_KMAX];
+        float sv[MAX_KMAX];
+        load_row_slots(a.idx + row * a.kmax, a.score + row * a.kmax, ke, a.kmax, ci, sv);
+        // fusion weights: softmax of the kept scores
         float m = -INFINITY;
-        for (int i = 0; i < ke; ++i) m = fmaxf(m, rs[i]);
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) m = fmaxf(m, sv[i]);
         float z = 0.f;
-        for (int i = 0; i < ke; ++i) z += expf(rs[i] - m);
-        for (int i = 0; i < ke; ++i) {
-            a.w8[row * a.kmax + i] = expf(rs[i] - m) / z;
-            const int c = ri[i];
-            if (c < 0 || c >= nc) {
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) {
+                sv[i] = expf(sv[i] - m);
+                z += sv[i];
+            }
+        float *w = a.w8 + row * a.kmax;
+        if ((a.kmax & 3) == 0) {
+#pragma unroll
+            for (int q = 0; q < MAX_KMAX / 4; ++q)
+                if (4 * q < ke)
+                    reinterpret_cast<float4 *>(w)[q] =
+                        make_float4(sv[4 * q] / z, sv[4 * q + 1] / z, sv[4 * q + 2] / z, sv[4 * q + 3] / z);
+        } else {
+#pragma unroll
+            for (int i = 0; i < MAX_KMAX; ++i)
+                if (i < ke) w[i] = sv[i] / z;
+        }
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i) {
+            if (i >= ke) continue;
+            if (ci[i] < 0 || ci[i] >= nc) {
                 atomicOr(a.status, DEV_BAD_INDEX);
                 continue;
             }
-            atomicAdd(&hist[c], 1);
+            atomicAdd(&hist[ci[i]], 1);
         }
     }
     __syncthreads();
@@ -292,14 +338,16 @@ __global__ void __launch_bounds__(HT) att_scatter_hist_kernel(AttTcArgs a) {
     long long row;
     const bool live = hist_row(a, b, j, t, row);
     int ke = 0, nc = 0;
+    int ci[MAX_KMAX];
+    float wv[MAX_KMAX];
     if (live) {
         ke = a.keff[row];
         ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
         nc = ncand_of(a, t);
-        for (int i = 0; i < ke; ++i) {
-            const int c = a.idx[row * a.kmax + i];
-            if (c >= 0 && c < nc) atomicAdd(&cnt[c], 1);
-        }
+        load_row_slots(a.idx + row * a.kmax, a.w8 + row * a.kmax, ke, a.kmax, ci, wv);
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke && ci[i] >= 0 && ci[i] < nc) atomicAdd(&cnt[ci[i]], 1);
     }
     __syncthreads();
     const int tb = (a.Tq + HT - 1) / HT;
@@ -315,12 +363,12 @@ __global__ void __launch_bounds__(HT) att_scatter_hist_kernel(AttTcArgs a) {
     }
     __syncthreads();
     if (live) {
-        for (int i = 0; i < ke; ++i) {
-            const int c = a.idx[row * a.kmax + i];
-            if (c < 0 || c >= nc) continue;
-            const int pos = basep[c] + atomicAdd(&cnt[c], 1);
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i) {
+            if (i >= ke || ci[i] < 0 || ci[i] >= nc) continue;
+            const int pos = basep[ci[i]] + atomicAdd(&cnt[ci[i]], 1);
             a.pairs[pos] = (t << 5) | i;
-            a.pair_w[pos] = a.w8[row * a.kmax + i];
+            a.pair_w[pos] = wv[i];
         }
     }
 }
