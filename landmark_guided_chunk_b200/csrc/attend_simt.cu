@@ -299,9 +299,8 @@ cudaError_t launch_attend(const Prob &p, const WsLayout &w, const void *Q, const
     if (p.rows == 0) return cudaSuccess;
     if (w.tc_attend) {
         AttTcBuffers bf;
-        bf.w8 = reinterpret_cast<float *>(ws + w.att_w8);
-        bf.pairs = reinterpret_cast<int32_t *>(ws + w.att_pairs);
-        bf.pair_w = reinterpret_cast<float *>(ws + w.att_pair_w);
+        bf.w8 = w.att.hist ? nullptr : reinterpret_cast<float *>(ws + w.att_w8);
+        bf.pairs = reinterpret_cast<int2 *>(ws + w.att_pairs);
         bf.counters = reinterpret_cast<int32_t *>(ws + w.att_counters);
         bf.boff = reinterpret_cast<int32_t *>(ws + w.att_boff);
         bf.btile = reinterpret_cast<int32_t *>(ws + w.att_btile);

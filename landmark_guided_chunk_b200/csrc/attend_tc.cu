@@ -61,12 +61,11 @@ struct AttTcArgs {
     const int32_t *idx;
     const float *score;
     const int32_t *keff;
-    float *w8;                   // [rows][kmax] fusion weights
+    float *w8;                   // [rows][kmax] fusion weights (per-pair-atomics path only)
     int32_t *bcount, *bcursor;   // [nbucket]
     int32_t *boff, *btile;       // [nbucket + 1]
     int32_t *blk;                // [2 * nblk] first-level block totals
-    int32_t *pairs;              // [rows * kmax]  (t << 5) | slot
-    float *pair_w;               // [rows * kmax]  fusion weight of each pair
+    int2 *pairs;                 // [rows * kmax]  ((t << 5) | slot, bits of the pair's fusion weight), bucketed
     int4 *tiles;                 // (phase, chunk, first pair, pairs in tile)
     float *ringbuf;              // [2*NB][TB][G][d]
     int d;                       // head dim (64 or 128)
@@ -220,8 +219,7 @@ __global__ void att_scatter_kernel(AttTcArgs a) {
         if (c < 0 || c >= nc) continue;
         const long long u = (long long)p * a.C + c;
         const int pos = a.boff[u] + atomicAdd(&a.bcursor[u], 1);
-        a.pairs[pos] = (t << 5) | i;
-        a.pair_w[pos] = a.w8[row * a.kmax + i];
+        a.pairs[pos] = make_int2((t << 5) | i, __float_as_int(a.w8[row * a.kmax + i]));
     }
 }
 
@@ -244,7 +242,7 @@ __device__ __forceinline__ bool hist_row(const AttTcArgs &a, int &b, int &j, int
     return t < a.Tq;
 }
 
-// A row's kept slots: chunk indices, and scores or weights.  Rows of kmax
+// A row's kept slots: chunk indices, and (val non-null) their scores.  Rows of kmax
 // 4-byte entries start on 16-byte boundaries when kmax is a multiple of 4 (the
 // buffers are 16-byte aligned), and are then read as 16-byte vectors.
 __device__ __forceinline__ void load_row_slots(const int32_t *idx, const float *val, int ke, int kmax,
@@ -254,9 +252,11 @@ __device__ __forceinline__ void load_row_slots(const int32_t *idx, const float *
         for (int q = 0; q < MAX_KMAX / 4; ++q) {
             if (4 * q < ke) {
                 const int4 ci = reinterpret_cast<const int4 *>(idx)[q];
-                const float4 xv = reinterpret_cast<const float4 *>(val)[q];
                 c[4 * q] = ci.x, c[4 * q + 1] = ci.y, c[4 * q + 2] = ci.z, c[4 * q + 3] = ci.w;
-                x[4 * q] = xv.x, x[4 * q + 1] = xv.y, x[4 * q + 2] = xv.z, x[4 * q + 3] = xv.w;
+                if (val != nullptr) {
+                    const float4 xv = reinterpret_cast<const float4 *>(val)[q];
+                    x[4 * q] = xv.x, x[4 * q + 1] = xv.y, x[4 * q + 2] = xv.z, x[4 * q + 3] = xv.w;
+                }
             }
         }
     } else {
@@ -264,7 +264,7 @@ __device__ __forceinline__ void load_row_slots(const int32_t *idx, const float *
         for (int i = 0; i < MAX_KMAX; ++i)
             if (i < ke) {
                 c[i] = idx[i];
-                x[i] = val[i];
+                if (val != nullptr) x[i] = val[i];
             }
     }
 }
@@ -284,32 +284,8 @@ __global__ void __launch_bounds__(HT) att_count_hist_kernel(AttTcArgs a) {
         }
         const int nc = ncand_of(a, t);
         int ci[MAX_KMAX];
-        float sv[MAX_KMAX];
-        load_row_slots(a.idx + row * a.kmax, a.score + row * a.kmax, ke, a.kmax, ci, sv);
-        // fusion weights: softmax of the kept scores
-        float m = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < MAX_KMAX; ++i)
-            if (i < ke) m = fmaxf(m, sv[i]);
-        float z = 0.f;
-#pragma unroll
-        for (int i = 0; i < MAX_KMAX; ++i)
-            if (i < ke) {
-                sv[i] = expf(sv[i] - m);
-                z += sv[i];
-            }
-        float *w = a.w8 + row * a.kmax;
-        if ((a.kmax & 3) == 0) {
-#pragma unroll
-            for (int q = 0; q < MAX_KMAX / 4; ++q)
-                if (4 * q < ke)
-                    reinterpret_cast<float4 *>(w)[q] =
-                        make_float4(sv[4 * q] / z, sv[4 * q + 1] / z, sv[4 * q + 2] / z, sv[4 * q + 3] / z);
-        } else {
-#pragma unroll
-            for (int i = 0; i < MAX_KMAX; ++i)
-                if (i < ke) w[i] = sv[i] / z;
-        }
+        float unused[MAX_KMAX];
+        load_row_slots(a.idx + row * a.kmax, nullptr, ke, a.kmax, ci, unused);
 #pragma unroll
         for (int i = 0; i < MAX_KMAX; ++i) {
             if (i >= ke) continue;
@@ -344,7 +320,22 @@ __global__ void __launch_bounds__(HT) att_scatter_hist_kernel(AttTcArgs a) {
         ke = a.keff[row];
         ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
         nc = ncand_of(a, t);
-        load_row_slots(a.idx + row * a.kmax, a.w8 + row * a.kmax, ke, a.kmax, ci, wv);
+        load_row_slots(a.idx + row * a.kmax, a.score + row * a.kmax, ke, a.kmax, ci, wv);
+        // fusion weights: softmax of the kept scores
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) m = fmaxf(m, wv[i]);
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) {
+                wv[i] = expf(wv[i] - m);
+                z += wv[i];
+            }
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) wv[i] /= z;
 #pragma unroll
         for (int i = 0; i < MAX_KMAX; ++i)
             if (i < ke && ci[i] >= 0 && ci[i] < nc) atomicAdd(&cnt[ci[i]], 1);
@@ -367,8 +358,7 @@ __global__ void __launch_bounds__(HT) att_scatter_hist_kernel(AttTcArgs a) {
         for (int i = 0; i < MAX_KMAX; ++i) {
             if (i >= ke || ci[i] < 0 || ci[i] >= nc) continue;
             const int pos = basep[ci[i]] + atomicAdd(&cnt[ci[i]], 1);
-            a.pairs[pos] = (t << 5) | i;
-            a.pair_w[pos] = wv[i];
+            a.pairs[pos] = make_int2((t << 5) | i, __float_as_int(wv[i]));
         }
     }
 }
@@ -542,8 +532,9 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const bool v = tau < tile_hi && mm[h] < T.n;
-            pr[h] = v ? a.pairs[T.start + mm[h]] : 0;
-            pw[h] = v ? a.pair_w[T.start + mm[h]] : 0.f;
+            const int2 e = v ? a.pairs[T.start + mm[h]] : make_int2(0, 0);
+            pr[h] = e.x;
+            pw[h] = __int_as_float(e.y);
         }
         for (; tau < tile_hi && ok; ++i) {
             // prefetch the next tile while this one is issued
@@ -589,8 +580,9 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const bool v = tau_n < tile_hi && mm[h] < Tn.n;
-                pr[h] = v ? a.pairs[Tn.start + mm[h]] : 0;
-                pw[h] = v ? a.pair_w[Tn.start + mm[h]] : 0.f;
+                const int2 e = v ? a.pairs[Tn.start + mm[h]] : make_int2(0, 0);
+                pr[h] = e.x;
+                pw[h] = __int_as_float(e.y);
             }
             T = Tn;
             tau = tau_n;
@@ -860,6 +852,7 @@ AttTcLayout attend_tc_layout(const Prob &p) {
     L.nblk = (L.nbucket + SCAN_BLK - 1) / SCAN_BLK;
     L.tok = MROWS / p.G;
     L.ring = 2 * NB;
+    L.hist = p.C <= HIST_MAX_C;
     const size_t pairs = (size_t)p.rows * p.kmax;
     L.max_tiles = pairs / L.tok + (size_t)L.nbucket + 1;
     L.counter_ints = 2 * (size_t)L.nbucket;
@@ -906,7 +899,6 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.btile = bf.btile;
     a.blk = bf.blk;
     a.pairs = bf.pairs;
-    a.pair_w = bf.pair_w;
     a.tiles = bf.tiles;
     a.ringbuf = bf.ring;
     a.status = bf.status;
@@ -916,7 +908,7 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     if (e == cudaSuccess) e = cudaMemsetAsync(bf.ring, 0, L.ring_bytes, st);
     if (e != cudaSuccess) return e;
     const int rows_blocks = (int)((p.rows + 255) / 256);
-    const bool hist = p.C <= HIST_MAX_C;
+    const bool hist = L.hist;
     const int hist_blocks = p.B * p.Hkv * ((p.Tq + HT - 1) / HT);
     if (hist) {
         if ((e = cudaFuncSetAttribute(att_scatter_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -30,12 +30,14 @@ struct Prob {
 // Sizes of the chunk-major tensor-core attention's workspace pieces.
 struct AttTcLayout {
     int tb, ntb, nsub, nphase, nbucket, nblk, tok, ring;
+    bool hist;   // buckets counted through shared-memory histograms (C small enough); else per-pair atomics
     size_t max_tiles, counter_ints, ring_bytes;
 };
 
 struct AttTcBuffers {
-    float *w8, *pair_w;
-    int32_t *pairs, *counters, *boff, *btile, *blk;
+    float *w8;                 // per-pair-atomics path only: fusion weights [rows][kmax]
+    int2 *pairs;               // bucketed (token << 5 | slot, fusion weight bits)
+    int32_t *counters, *boff, *btile, *blk;
     int4 *tiles;
     float *ring;
     uint32_t *status;
@@ -61,7 +63,7 @@ struct WsLayout {
     AttTcLayout att;
     bool quest;          // Quest scoring: the select fields above describe quest_select_view(p)
     size_t quest_q;      // Quest scoring: the transformed query rows (quest_qprep_bytes)
-    size_t att_w8, att_pairs, att_pair_w, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
+    size_t att_w8, att_pairs, att_counters, att_boff, att_btile, att_blk, att_tiles, att_ring;
     hsa_plan_t plan;     // kernel paths and launch counts per stage
 };
 

@@ -112,9 +112,8 @@ WsLayout ws_layout(const Prob &p) {
     if (w.split_attend && !w.gather_attend) w.partials = take(rows * (size_t)p.kmax * p.G * p.d * sizeof(float));
     if (w.tc_attend) {
         w.att = attend_tc_layout(p);
-        w.att_w8 = take(rows * p.kmax * sizeof(float));
-        w.att_pairs = take(rows * p.kmax * sizeof(int32_t));
-        w.att_pair_w = take(rows * p.kmax * sizeof(float));
+        if (!w.att.hist) w.att_w8 = take(rows * p.kmax * sizeof(float));
+        w.att_pairs = take(rows * p.kmax * sizeof(int2));
         w.att_counters = take(w.att.counter_ints * sizeof(int32_t));
         w.att_boff = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
         w.att_btile = take(((size_t)w.att.nbucket + 1) * sizeof(int32_t));
