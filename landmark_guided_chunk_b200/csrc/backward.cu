@@ -193,6 +193,134 @@ __global__ void bwd_scatter_kernel(BwdArgs a) {
     }
 }
 
+// The same two steps with the rows of one CTA taken as BHT consecutive tokens
+// of one (b, kv head): the CTA counts its pairs per chunk in a shared-memory
+// histogram and touches each of its buckets' global counters once, instead of
+// once per pair.  Used when the C counters (two arrays for the scatter) fit in
+// shared memory.  Rows are read as 16-byte vectors when kmax is a multiple of 4.
+constexpr int BHT = 256;
+constexpr int BHIST_MAX_C = 16384;
+
+__device__ __forceinline__ bool bhist_row(const BwdArgs &a, int &b, int &j, int &t, long long &r) {
+    const int tb = (a.Tq + BHT - 1) / BHT;
+    const int bj = (int)blockIdx.x / tb;
+    b = bj / a.Hkv;
+    j = bj % a.Hkv;
+    t = ((int)blockIdx.x % tb) * BHT + (int)threadIdx.x;
+    r = ((long long)b * a.Tq + t) * a.Hkv + j;
+    return t < a.Tq;
+}
+
+// A row's first ke slots of an int and a float array (rows of kmax entries).
+__device__ __forceinline__ void bwd_row_slots(const int32_t *ip, const float *fp, int ke, int kmax,
+                                              int (&c)[MAX_KMAX], float (&x)[MAX_KMAX]) {
+    if ((kmax & 3) == 0) {
+#pragma unroll
+        for (int q = 0; q < MAX_KMAX / 4; ++q)
+            if (4 * q < ke) {
+                const int4 ci = reinterpret_cast<const int4 *>(ip)[q];
+                const float4 xv = reinterpret_cast<const float4 *>(fp)[q];
+                c[4 * q] = ci.x, c[4 * q + 1] = ci.y, c[4 * q + 2] = ci.z, c[4 * q + 3] = ci.w;
+                x[4 * q] = xv.x, x[4 * q + 1] = xv.y, x[4 * q + 2] = xv.z, x[4 * q + 3] = xv.w;
+            }
+    } else {
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) {
+                c[i] = ip[i];
+                x[i] = fp[i];
+            }
+    }
+}
+
+__global__ void __launch_bounds__(BHT) bwd_prep_hist_kernel(BwdArgs a) {
+    extern __shared__ int hist[];   // [C]
+    for (int c = threadIdx.x; c < a.C; c += BHT) hist[c] = 0;
+    __syncthreads();
+    int b, j, t;
+    long long r;
+    if (bhist_row(a, b, j, t, r)) {
+        int ke = a.keff[r];
+        if (ke < 0 || ke > a.kmax) {
+            atomicOr(a.status, DEV_BAD_INDEX);
+            ke = ke < 0 ? 0 : a.kmax;
+        }
+        int ci[MAX_KMAX];
+        float sv[MAX_KMAX];
+        bwd_row_slots(a.idx + r * a.kmax, a.score + r * a.kmax, ke, a.kmax, ci, sv);
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) m = fmaxf(m, sv[i]);
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke) {
+                sv[i] = expf(sv[i] - m);
+                z += sv[i];
+            }
+        const long long nc = ncand_of(a, t);
+        float *wr = a.w + r * a.kmax;
+        for (int i = 0; i < a.kmax; ++i) wr[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i) {
+            if (i >= ke) continue;
+            wr[i] = sv[i] / z;
+            if (ci[i] < 0 || ci[i] >= nc) {
+                atomicOr(a.status, DEV_BAD_INDEX);
+                continue;
+            }
+            atomicAdd(&hist[ci[i]], 1);
+        }
+    }
+    __syncthreads();
+    const int tb = (a.Tq + BHT - 1) / BHT;
+    const long long bj = (int)blockIdx.x / tb;
+    for (int c = threadIdx.x; c < a.C; c += BHT)
+        if (hist[c] > 0) atomicAdd(a.bcount + bj * a.C + c, hist[c]);
+}
+
+__global__ void __launch_bounds__(BHT) bwd_scatter_hist_kernel(BwdArgs a) {
+    extern __shared__ int sh[];   // [C] counts, then cursors; [C] this CTA's base in each bucket
+    int *cnt = sh, *basep = sh + a.C;
+    for (int c = threadIdx.x; c < a.C; c += BHT) cnt[c] = 0;
+    __syncthreads();
+    int b, j, t;
+    long long r;
+    const bool live = bhist_row(a, b, j, t, r);
+    int ke = 0;
+    long long nc = 0;
+    int ci[MAX_KMAX];
+    float wv[MAX_KMAX];
+    if (live) {
+        ke = a.keff[r];
+        ke = ke < 0 ? 0 : (ke > a.kmax ? a.kmax : ke);
+        nc = ncand_of(a, t);
+        bwd_row_slots(a.idx + r * a.kmax, a.w + r * a.kmax, ke, a.kmax, ci, wv);
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i)
+            if (i < ke && ci[i] >= 0 && ci[i] < nc) atomicAdd(&cnt[ci[i]], 1);
+    }
+    __syncthreads();
+    const int tb = (a.Tq + BHT - 1) / BHT;
+    const long long bj = (int)blockIdx.x / tb;
+    for (int c = threadIdx.x; c < a.C; c += BHT) {
+        const int n = cnt[c];
+        if (n > 0) basep[c] = atomicAdd(a.bcount + bj * a.C + c, n);   // this CTA's run in the bucket
+        cnt[c] = 0;
+    }
+    __syncthreads();
+    if (live) {
+#pragma unroll
+        for (int i = 0; i < MAX_KMAX; ++i) {
+            if (i >= ke || ci[i] < 0 || ci[i] >= nc) continue;
+            const int pos = basep[ci[i]] + atomicAdd(&cnt[ci[i]], 1);
+            a.pairs[pos] = (int)(r * a.kmax + i);
+            a.pair_w[pos] = wv[i];
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------- chunk-major attention backward
 
 // 16 bytes of stored values -> fp32 in shared memory
@@ -434,6 +562,29 @@ __global__ void __launch_bounds__(NT_BWD, 1)
 
 constexpr int NT_FUSE = 256;   // 8 warps, one selection row each
 
+// CPL consecutive stored values of a row (this lane's columns) as fp32, one vector load.
+template <int CPL> __device__ __forceinline__ void load_cols(const float *p, float (&o)[CPL]) {
+    if constexpr (CPL == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        o[0] = v.x, o[1] = v.y, o[2] = v.z, o[3] = v.w;
+    } else {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
+        o[0] = v.x, o[1] = v.y;
+    }
+}
+template <int CPL> __device__ __forceinline__ void load_cols(const __nv_bfloat16 *p, float (&o)[CPL]) {
+    if constexpr (CPL == 4) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v.y));
+        o[0] = f0.x, o[1] = f0.y, o[2] = f1.x, o[3] = f1.y;
+    } else {
+        const uint32_t v = __ldg(reinterpret_cast<const unsigned int *>(p));
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+        o[0] = f0.x, o[1] = f0.y;
+    }
+}
+
 // Per selection row: dw_i = sum_h e_hi, ds_i = w_i (dw_i - sum w dw); then
 // dQ_h += sum_i ds_i L_ci for every head of the group, dL_ci += ds_i sum_h q_h.
 template <typename T, int D>
@@ -469,24 +620,43 @@ __global__ void __launch_bounds__(NT_FUSE) bwd_fuse_kernel(BwdArgs a, int Lc, co
 #pragma unroll
     for (int x = 0; x < CPL; ++x) qs[x] = 0.f;
     const T *qrow = Q + (bt * a.H + (long long)j * a.G) * D + lane * CPL;
-    for (int g = 0; g < a.G; ++g)
+    for (int g0 = 0; g0 < a.G; g0 += 4) {   // four heads' loads in flight, summed in head order
+        float qv[4][CPL];
 #pragma unroll
-        for (int x = 0; x < CPL; ++x) qs[x] += to_f32(qrow[(long long)g * D + x]);
+        for (int h = 0; h < 4; ++h)
+            if (g0 + h < a.G) load_cols<CPL>(qrow + (long long)(g0 + h) * D, qv[h]);
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            if (g0 + h < a.G)
+#pragma unroll
+                for (int x = 0; x < CPL; ++x) qs[x] += qv[h][x];
+    }
     float dq[CPL];
 #pragma unroll
     for (int x = 0; x < CPL; ++x) dq[x] = 0.f;
-    for (int i = 0; i < ke; ++i) {
-        const float dsi = __shfl_sync(FULL, ds, i);
-        const int ci = __shfl_sync(FULL, c, i);
-        if (ci < 0) continue;   // warp-uniform
-        const T *lrow = L + (((long long)b * a.Hkv + j) * Lc + ci) * D + lane * CPL;
-        Cols<CPL> o;
+    // the kept chunks' landmark rows eight at a time (their loads in flight together), in slot order
+    for (int i0 = 0; i0 < ke; i0 += 8) {
+        float lv[8][CPL], dsv[8];
+        int civ[8];
 #pragma unroll
-        for (int x = 0; x < CPL; ++x) {
-            dq[x] = fmaf(dsi, to_f32(lrow[x]), dq[x]);
-            o.v[x] = dsi * qs[x];
+        for (int q = 0; q < 8; ++q) {
+            const int i = i0 + q;
+            dsv[q] = __shfl_sync(FULL, ds, i & 31);
+            civ[q] = __shfl_sync(FULL, c, i & 31);
+            if (i < ke && civ[q] >= 0)   // warp-uniform
+                load_cols<CPL>(L + (((long long)b * a.Hkv + j) * Lc + civ[q]) * D + lane * CPL, lv[q]);
         }
-        o.red(a.dL + (((long long)b * a.Hkv + j) * a.C + ci) * D + lane * CPL);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (i0 + q >= ke || civ[q] < 0) continue;   // warp-uniform
+            Cols<CPL> o;
+#pragma unroll
+            for (int x = 0; x < CPL; ++x) {
+                dq[x] = fmaf(dsv[q], lv[q][x], dq[x]);
+                o.v[x] = dsv[q] * qs[x];
+            }
+            o.red(a.dL + (((long long)b * a.Hkv + j) * a.C + civ[q]) * D + lane * CPL);
+        }
     }
     Cols<CPL> o;
 #pragma unroll
@@ -544,7 +714,18 @@ __global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T 
         if (!__syncthreads_or(v != 0.f)) continue;   // never kept by any row: nothing to add
         const long long row0 = ((long long)b * a.Tcap + (long long)c * a.S) * a.Hkv + j;
         float ps = 0.f, pm = 0.f;
-        for (int u = part; u < a.S; u += PARTS) ps += to_f32(K[(row0 + (long long)u * a.Hkv) * D + xcol]);
+        // this thread's column of the chunk's keys, eight rows' loads in flight (summed in row order)
+        for (int u0 = part; u0 < a.S; u0 += 8 * PARTS) {
+            float kv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int u = u0 + q * PARTS;
+                kv[q] = u < a.S ? to_f32(K[(row0 + (long long)u * a.Hkv) * D + xcol]) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (u0 + q * PARTS < a.S) ps += kv[q];
+        }
         for (int f = part; f < D; f += PARTS) pm = fmaf(sdl[f], sW[xcol * WP + f], pm);
         spart[part * D + xcol] = ps;
         __syncthreads();
@@ -562,10 +743,19 @@ __global__ void __launch_bounds__(NT_LM) bwd_landmark_kernel(BwdArgs a, const T 
             sdm[threadIdx.x] = m / (float)a.S;
         }
         __syncthreads();
-        for (int i = threadIdx.x; i < a.S * D; i += NT_LM) {
-            const int u = i / D, x = i - u * D;
-            float *p = dK + (row0 + (long long)u * a.Hkv) * D + x;
-            *p += sdm[x];
+        // the keys' gradients += dL_c W_L^T / S, eight read-modify-writes in flight per thread
+        for (int i0 = threadIdx.x; i0 < a.S * D; i0 += 8 * NT_LM) {
+            float kv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int i = i0 + q * NT_LM, u = i / D, x = i - u * D;
+                kv[q] = i < a.S * D ? dK[(row0 + (long long)u * a.Hkv) * D + x] : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int i = i0 + q * NT_LM, u = i / D, x = i - u * D;
+                if (i < a.S * D) dK[(row0 + (long long)u * a.Hkv) * D + x] = kv[q] + sdm[x];
+            }
         }
 #pragma unroll
         for (int q = 0; q < XPW; ++q) {
@@ -1418,11 +1608,25 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     a.dL = reinterpret_cast<float *>(ws + w.dL);
     a.status = reinterpret_cast<uint32_t *>(ws + w.hdr);
     const unsigned row_grid = (unsigned)((p.rows + 255) / 256);
-    bwd_prep_kernel<<<row_grid, 256, 0, st>>>(a);
+    const bool hist = p.C <= BHIST_MAX_C;
+    const unsigned hist_grid = (unsigned)(p.B * p.Hkv * ((p.Tq + BHT - 1) / BHT));
+    if (hist) {
+        if ((e = cudaFuncSetAttribute(bwd_prep_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(p.C * sizeof(int)))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwd_scatter_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(2 * p.C * sizeof(int)))) != cudaSuccess)
+            return e;
+        bwd_prep_hist_kernel<<<hist_grid, BHT, p.C * sizeof(int), st>>>(a);
+    } else {
+        bwd_prep_kernel<<<row_grid, 256, 0, st>>>(a);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_scan_kernel<<<1, NT_SCAN, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_scatter_kernel<<<row_grid, 256, 0, st>>>(a);
+    if (hist)
+        bwd_scatter_hist_kernel<<<hist_grid, BHT, 2 * p.C * sizeof(int), st>>>(a);
+    else
+        bwd_scatter_kernel<<<row_grid, 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int grid = (int)(w.max_tiles < sms ? w.max_tiles : sms);
     const bool bf = p.dtype == HSA_BF16;
