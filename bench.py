@@ -550,12 +550,12 @@ def run_backward(args, p, hsa, Q, K, V, W, L, idx, score, keff, keff_sum, st, wo
     pk = peaks()
     roof = ({"bound": "tensor", "achieved": round(ach, 2), "unit": "TFLOP/s", "peak": pk["bf16_tflops_sustained"],
              "frac": round(ach / pk["bf16_tflops_sustained"], 4),
-             "peak_source": f"{pk['source']} (sustained bf16); whole backward call, 6 kernels"} if tc else
+             "peak_source": f"{pk['source']} (sustained bf16); whole backward call, 7 kernels"} if tc else
             {"bound": "alu", "achieved": round(ach, 2), "unit": "TFLOP/s", "peak": round(FFMA_PEAK_TFLOPS, 1),
              "frac": round(ach / FFMA_PEAK_TFLOPS, 4),
              "peak_source": "fp32 FMA lanes x clocks.max.sm (CUDA-core path)"})
     return {"ms": round(ms, 3), "steps": nsteps, "tokens_per_s": round(p.B * p.Tq * world / (ms * 1e-3), 1),
-            "kernels": 6, "path": "tensor" if tc else "simt",
+            "kernels": 7, "path": "tensor" if tc else "simt",
             "exchange": "all-reduce (sum) of dW_L, d x d fp32, over the ranks" if world > 1 else "none (one rank)",
             "dtype": "bf16 operands, fp32 accumulation" if tc else "f32", "roofline": roof}
 

@@ -56,6 +56,7 @@ struct BwdArgs {
     float *e;                   // [rows][kmax][G]  dO_h . o_hi
     int32_t *bcount;            // [nbucket] pair counts, then scatter cursors
     int32_t *boff;              // [nbucket + 1] first pair of each bucket
+    int32_t *btile;             // [nbucket + 1] first tile of each bucket
     int32_t *pairs;             // [rows * kmax] row * kmax + slot, bucket-major
     float *pair_w;              // [rows * kmax] fusion weight of each pair, bucket-major
     int4 *tiles;                // (bucket, first pair, pairs, 0)
@@ -111,8 +112,9 @@ __global__ void bwd_prep_kernel(BwdArgs a) {
 }
 
 // Exclusive scans of pair counts and tile counts over the buckets, in blocks
-// of NT_SCAN with a running carry; each bucket also writes its tile records
-// and turns its count into the scatter cursor.
+// of NT_SCAN with a running carry; each bucket's count becomes its scatter
+// cursor.  The tile records are written by bwd_tiles_kernel, one thread per
+// bucket over the whole grid.
 __global__ void __launch_bounds__(NT_SCAN) bwd_scan_kernel(BwdArgs a) {
     __shared__ int wp[NT_SCAN / 32], wt[NT_SCAN / 32];
     __shared__ int carry_p, carry_t;
@@ -158,9 +160,8 @@ __global__ void __launch_bounds__(NT_SCAN) bwd_scan_kernel(BwdArgs a) {
         const int et = carry_t + (warp ? wt[warp - 1] : 0) + it - nt;
         if (i < a.nbucket) {
             a.boff[i] = ep;
+            a.btile[i] = et;
             a.bcount[i] = ep;   // scatter cursor
-            for (int q = 0; q < nt; ++q)
-                a.tiles[et + q] = make_int4((int)i, ep + q * a.pt, min(a.pt, cnt - q * a.pt), 0);
         }
         __syncthreads();
         if (threadIdx.x == NT_SCAN - 1) {
@@ -171,8 +172,17 @@ __global__ void __launch_bounds__(NT_SCAN) bwd_scan_kernel(BwdArgs a) {
     }
     if (threadIdx.x == 0) {
         a.boff[a.nbucket] = carry_p;
+        a.btile[a.nbucket] = carry_t;
         *a.ntiles = carry_t;
     }
+}
+
+// Each bucket's tile records: (bucket, first pair, pairs, 0), pt pairs per tile.
+__global__ void bwd_tiles_kernel(BwdArgs a) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.nbucket) return;
+    const int ep = a.boff[i], cnt = a.boff[i + 1] - ep, et = a.btile[i], nt = a.btile[i + 1] - et;
+    for (int q = 0; q < nt; ++q) a.tiles[et + q] = make_int4((int)i, ep + q * a.pt, min(a.pt, cnt - q * a.pt), 0);
 }
 
 __global__ void bwd_scatter_kernel(BwdArgs a) {
@@ -619,44 +629,31 @@ __global__ void __launch_bounds__(NT_FUSE) bwd_fuse_kernel(BwdArgs a, int Lc, co
     float qs[CPL];
 #pragma unroll
     for (int x = 0; x < CPL; ++x) qs[x] = 0.f;
+    // (one row at a time: the kernel relies on occupancy, eight CTAs of low register use per SM,
+    // to hide the loads' latency; batching them in registers measured slower)
     const T *qrow = Q + (bt * a.H + (long long)j * a.G) * D + lane * CPL;
-    for (int g0 = 0; g0 < a.G; g0 += 4) {   // four heads' loads in flight, summed in head order
-        float qv[4][CPL];
+    for (int g = 0; g < a.G; ++g) {
+        float qv[CPL];
+        load_cols<CPL>(qrow + (long long)g * D, qv);
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
-            if (g0 + h < a.G) load_cols<CPL>(qrow + (long long)(g0 + h) * D, qv[h]);
-#pragma unroll
-        for (int h = 0; h < 4; ++h)
-            if (g0 + h < a.G)
-#pragma unroll
-                for (int x = 0; x < CPL; ++x) qs[x] += qv[h][x];
+        for (int x = 0; x < CPL; ++x) qs[x] += qv[x];
     }
     float dq[CPL];
 #pragma unroll
     for (int x = 0; x < CPL; ++x) dq[x] = 0.f;
-    // the kept chunks' landmark rows eight at a time (their loads in flight together), in slot order
-    for (int i0 = 0; i0 < ke; i0 += 8) {
-        float lv[8][CPL], dsv[8];
-        int civ[8];
+    for (int i = 0; i < ke; ++i) {
+        const float dsi = __shfl_sync(FULL, ds, i);
+        const int ci = __shfl_sync(FULL, c, i);
+        if (ci < 0) continue;   // warp-uniform
+        float lv[CPL];
+        load_cols<CPL>(L + (((long long)b * a.Hkv + j) * Lc + ci) * D + lane * CPL, lv);
+        Cols<CPL> o;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int i = i0 + q;
-            dsv[q] = __shfl_sync(FULL, ds, i & 31);
-            civ[q] = __shfl_sync(FULL, c, i & 31);
-            if (i < ke && civ[q] >= 0)   // warp-uniform
-                load_cols<CPL>(L + (((long long)b * a.Hkv + j) * Lc + civ[q]) * D + lane * CPL, lv[q]);
+        for (int x = 0; x < CPL; ++x) {
+            dq[x] = fmaf(dsi, lv[x], dq[x]);
+            o.v[x] = dsi * qs[x];
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (i0 + q >= ke || civ[q] < 0) continue;   // warp-uniform
-            Cols<CPL> o;
-#pragma unroll
-            for (int x = 0; x < CPL; ++x) {
-                dq[x] = fmaf(dsv[q], lv[q][x], dq[x]);
-                o.v[x] = dsv[q] * qs[x];
-            }
-            o.red(a.dL + (((long long)b * a.Hkv + j) * a.C + civ[q]) * D + lane * CPL);
-        }
+        o.red(a.dL + (((long long)b * a.Hkv + j) * a.C + ci) * D + lane * CPL);
     }
     Cols<CPL> o;
 #pragma unroll
@@ -1551,6 +1548,7 @@ BwdLayout backward_layout(const Prob &p) {
     w.w = take(pairs * sizeof(float));
     w.e = take(pairs * p.G * sizeof(float));
     w.boff = take(((size_t)w.nbucket + 1) * sizeof(int32_t));
+    w.btile = take(((size_t)w.nbucket + 1) * sizeof(int32_t));
     w.pairs = take(pairs * sizeof(int32_t));
     w.pair_w = take(pairs * sizeof(float));
     w.tiles = take((size_t)w.max_tiles * sizeof(int4));
@@ -1563,7 +1561,7 @@ bool backward_supported(const Prob &p) {
     return (long long)p.rows * p.kmax * p.G < (1ll << 31) && w.max_tiles < (1ll << 31) && p.G <= RT;
 }
 
-int backward_launches(const Prob &p) { return p.rows > 0 && p.C > 0 ? 6 : 0; }
+int backward_launches(const Prob &p) { return p.rows > 0 && p.C > 0 ? 7 : 0; }
 
 cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms, const void *Q, const void *K,
                             const void *V, const void *W, const void *L, const int32_t *idx, const float *score,
@@ -1601,6 +1599,7 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     a.e = reinterpret_cast<float *>(ws + w.e);
     a.bcount = reinterpret_cast<int32_t *>(ws + w.bcount);
     a.boff = reinterpret_cast<int32_t *>(ws + w.boff);
+    a.btile = reinterpret_cast<int32_t *>(ws + w.btile);
     a.pairs = reinterpret_cast<int32_t *>(ws + w.pairs);
     a.pair_w = reinterpret_cast<float *>(ws + w.pair_w);
     a.tiles = reinterpret_cast<int4 *>(ws + w.tiles);
@@ -1622,6 +1621,8 @@ cudaError_t launch_backward(const Prob &p, const BwdLayout &w, char *ws, int sms
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     bwd_scan_kernel<<<1, NT_SCAN, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    bwd_tiles_kernel<<<(unsigned)((w.nbucket + 255) / 256), 256, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (hist)
         bwd_scatter_hist_kernel<<<hist_grid, BHT, 2 * p.C * sizeof(int), st>>>(a);

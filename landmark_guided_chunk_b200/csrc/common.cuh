@@ -343,7 +343,7 @@ cudaError_t launch_quest_qprep(const Prob &p, const void *Q, void *Qp, cudaStrea
 
 // Backward (backward.cu): workspace layout, support check, kernel count, launch.
 struct BwdLayout {
-    size_t hdr, bcount, dL, clear_bytes, w, e, boff, pairs, pair_w, tiles, total;
+    size_t hdr, bcount, dL, clear_bytes, w, e, boff, btile, pairs, pair_w, tiles, total;
     long long nbucket, max_tiles;
     int pt;    // pairs per tile
     bool tc;   // tensor-core attention backward (bf16, d 128, S 64 / 128)
