@@ -208,6 +208,10 @@ def test_fused_decode_plan_host_rules():
     # a short context (under 2048 candidate chunks) takes the per-row scan: no fusion
     short = workload("decode_1m").with_(Tkv=64 * 1500, q_pos0=64 * 1500)
     assert not plan_of(short)["forward_fused"]
+    # so many rows that the scan needs more CTAs than there are SMs: they could not all be resident
+    # at once, so the scan and the gather stay two launches
+    wide = workload("decode_1m").with_(B=64, Tkv=64 * 4096, q_pos0=64 * 4096)
+    assert plan_of(wide)["select"][0] == "mma_split" and not plan_of(wide)["forward_fused"]
     # the fused layout holds one 8-byte descriptor per (row, slot) on top of the unfused one
     p = workload("decode_1m")
     fused = hsa.workspace_size(hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, bf16))
