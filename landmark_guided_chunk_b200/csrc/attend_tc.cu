@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(NT_ATT, 1)
 
     if (warp < 2) {
         // ------------------------------------------------------------ producers: Q gather (rows r, r+64), K/V TMA
+        __shared__ const char *rowsrc[MROWS];   // this tile's row sources (each warp writes and reads its own rows)
         int rr[2], mm[2], gg[2], pr[2];
         float pw[2];
 #pragma unroll
@@ -559,21 +560,51 @@ __global__ void __launch_bounds__(NT_ATT, 1)
             }
             const int sq = i % a.nsq, iq = i / a.nsq;
             if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
+            // the tile's Q rows: row r of the tile is head gg of token pr >> 5 (padding rows zero-filled)
+            const char *srcs[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int r = rr[h];
-                const bool valid = mm[h] < T.n;
-                const char *src = reinterpret_cast<const char *>(Q);
-                if (valid) {
+                srcs[h] = nullptr;
+                if (mm[h] < T.n) {
                     const int t0 = (T.p % a.ntb) * TB;   // the tile's phase: tokens t0 .. t0 + TB - 1
                     const int t = (int)dbg_clamp(pr[h] >> 5, t0, min(a.Tq, t0 + TB), a.status);
-                    src += ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
+                    srcs[h] = reinterpret_cast<const char *>(Q) +
+                              ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
                 }
-                const uint32_t dq = smem_u32(sQ + sq * QTILE) + (r >> 3) * 1024 + (r & 7) * 128;
+            }
+            const uint32_t qbase = smem_u32(sQ + sq * QTILE);
+            if constexpr (D == 128) {
+                // each thread puts its two rows' sources in the warp's table; then every copy
+                // instruction takes four rows x 128 bytes, each 8-lane group one whole 128-byte line
 #pragma unroll
-                for (int x = 0; x < D / 8; ++x) {
-                    const int kb = x >> 3, cx = x & 7;
-                    cp_async16(dq + kb * 16384 + ((cx ^ (r & 7)) << 4), src + (valid ? x * 16 : 0), valid ? 16u : 0u);
+                for (int h = 0; h < 2; ++h) rowsrc[rr[h]] = srcs[h];
+                __syncwarp();
+                const int cx = lane & 7;
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+#pragma unroll
+                    for (int g4 = 0; g4 < 8; ++g4) {
+                        const int r = warp * 32 + blk * NPROD + g4 * 4 + (lane >> 3);
+                        const char *s = rowsrc[r];
+                        const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128 + ((cx ^ (r & 7)) << 4);
+#pragma unroll
+                        for (int kb = 0; kb < D / 64; ++kb)
+                            cp_async16(dq + kb * 16384, s != nullptr ? s + kb * 128 + cx * 16 : reinterpret_cast<const char *>(Q),
+                                       s != nullptr ? 16u : 0u);
+                    }
+                }
+                __syncwarp();   // the table is rewritten for the next tile only after every lane has read it
+            } else {
+                // 128-byte rows: each thread copies its own two rows (the table measured slower here)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = rr[h];
+                    const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int x = 0; x < D / 8; ++x)
+                        cp_async16(dq + ((x ^ (r & 7)) << 4),
+                                   srcs[h] != nullptr ? srcs[h] + x * 16 : reinterpret_cast<const char *>(Q),
+                                   srcs[h] != nullptr ? 16u : 0u);
                 }
             }
             cp_async_arrive(&bar->q_full[sq]);
