@@ -788,14 +788,25 @@ def dram_traffic(stage: str, path: str):
     ent = d.get(f"{stage}:{path}")
     if not ent:
         return None
-    import hashlib
-    h = hashlib.sha256()
-    for src in ent.get("sources", []):
-        with open(os.path.join(ROOT, src), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest()[:16] != ent.get("source_hash"):
+    if source_digest(ent.get("sources", [])) != ent.get("source_hash"):
         return None
     return ent.get("bytes_per_launch")
+
+
+def source_digest(paths) -> str:
+    """Digest of the code in the given source files, with // comments and blank
+    lines left out: a capture stays valid across comment-only edits, and any
+    change to the code itself invalidates it."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for src in paths:
+        with open(os.path.join(ROOT, src)) as fh:
+            for line in fh:
+                code = re.sub(r"//.*$", "", line).rstrip()
+                if code.strip():
+                    h.update(code.encode() + b"\n")
+    return h.hexdigest()[:16]
 
 
 # --------------------------------------------------------------------------- CPU baseline (oracle)

@@ -13,12 +13,15 @@
 //     P  = exp(S - rowmax), l = sum P      softmax warps, P -> smem (bf16)
 //     O  = P . V_c                          tcgen05, M128 x N=d x K=S, TMEM
 //     O_acc[t][h] += (w_slot / l) * O       O-drain warps, fp32 vector reductions (red.v4)
-// Roles (16 warps, 4 per SM sub-partition so each may hold 128 registers):
-// two producer warps gather the tile's Q rows (cp.async) and issue the K/V TMA
-// loads, one thread issues the MMAs, four softmax warps (one per TMEM lane
-// quadrant) and eight O-drain warps (two per quadrant, 64 columns each) take
-// every tile.  S, P and O are double-buffered by tile parity, so the drain of
-// tile i overlaps the softmax of tile i+1 and the QK product of tile i+2.
+// The kernel is a template on the head dim (D = 64 or 128).  Roles (16 warps,
+// 4 per SM sub-partition so each may hold 128 registers): two producer warps
+// gather the tile's Q rows (cp.async; for D = 128 through a per-warp table of
+// row addresses, so that each 8-lane group copies one whole 128-byte line),
+// one loader warp issues the K/V TMA loads, one thread issues the MMAs, four
+// softmax warps (one per TMEM lane quadrant) and eight O-drain warps (two per
+// quadrant, D/2 columns each) take every tile.  S, P and O are double-buffered
+// by tile parity, so the drain of tile i overlaps the softmax of tile i+1 and
+// the QK product of tile i+2.
 // Since w is known before the attention, the cross-chunk fusion is linear and
 // needs no rescaling.
 //
@@ -31,9 +34,9 @@
 // tiles of batch beta, whose slots differ.  The kernel boundary is the only
 // synchronisation, so no CTA ever waits for another.
 //
-// Helper kernels (before the batches): count pairs per (phase, chunk) bucket
-// and compute the fusion weights; two-level exclusive scan of pair and tile
-// counts; tile list; scatter of the pairs into their buckets.
+// Helper kernels (before the batches): count pairs per (phase, chunk) bucket;
+// two-level exclusive scan of pair and tile counts; tile list; scatter of the
+// pairs, each with its fusion weight, into their buckets.
 #include "common.cuh"
 #include "sm100.cuh"
 
