@@ -12,14 +12,15 @@
  * k for rows whose top-k cut is nearly tied.
  *
  * Conventions shared by every entry point:
- *   - All tensor arguments are DEVICE pointers.  The caller allocates them, and
- *     also the workspace.  The library never allocates, keeps no global
+ *   - All tensor arguments are DEVICE pointers, except the tensors of
+ *     hsa_forward_host, which live in host memory.  The caller allocates them,
+ *     and also the workspace.  The library never allocates, keeps no global
  *     mutable state, and is safe to call from several host threads on
  *     different streams, each with its own workspace.
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL =
  *     the legacy default stream).  Host-side validation runs before any launch.
  *     An invalid call launches nothing and returns a status.
- *   - Layouts (row-major, contiguous, every pointer 16-byte aligned):
+ *   - Layouts (row-major, contiguous, every device pointer 16-byte aligned):
  *       Q, O   [B][Tq][H][d]       K, V  [B][Tcap][Hkv][d]
  *       W_L    [d][d]  (row = input dim: landmark = mean_row * W_L)
  *       L      [B][Hkv][Ccap][d],  C = floor(Tkv / S) of them valid
@@ -62,7 +63,7 @@
 extern "C" {
 #endif
 
-#define HSA_ABI_VERSION 5
+#define HSA_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define HSA_API __attribute__((visibility("default")))
@@ -279,6 +280,32 @@ HSA_API hsa_status_t hsa_merge_partials(const hsa_problem_t *p, int nshard, cons
 HSA_API hsa_status_t hsa_forward(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
                          const void *W_L, void *L, int32_t *idx, float *score, int32_t *keff,
                          void *O, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * hsa_forward for a caller whose tensors live in HOST memory.  On `stream` it
+ * enqueues the copies of the inputs into the device buffer `dev`, the whole
+ * forward of hsa_forward there (landmarks, selection, chunk attention and
+ * fusion), and the copy of O back to host memory; each copy is one
+ * cudaMemcpyAsync.  Host layouts are those of hsa_forward: Q and O
+ * [B][Tq][H][d], K and V [B][Tcap][Hkv][d] (copied whole), W_L [d][d] (not
+ * read under HSA_FLAG_QUEST).  A host pointer may be NULL only where
+ * hsa_forward would not read the tensor (e.g. K and V with no chunks); host
+ * pointers need no alignment.
+ * dev: a device buffer of hsa_forward_host_bytes(p) bytes, 256-byte aligned,
+ * that receives the device copies of Q, K, V, W_L, the landmarks and O; it is
+ * the caller's and may be reused once the stream has passed this call.  ws:
+ * the workspace of hsa_workspace_size(p).  Every argument is checked before
+ * anything is enqueued.  The call returns once the work is enqueued: O is
+ * complete when the stream reaches this point, and the host buffers must stay
+ * valid until then.  With page-locked host memory the copies are
+ * asynchronous, so calls on several streams (each with its own dev and ws)
+ * overlap one call's uploads with another's compute and download.
+ * HSA_FLAG_LANDMARKS_READY is refused: the landmarks are made here from K.
+ */
+HSA_API hsa_status_t hsa_forward_host_bytes(const hsa_problem_t *p, size_t *bytes);
+HSA_API hsa_status_t hsa_forward_host(const hsa_problem_t *p, const void *Q, const void *K, const void *V,
+                                      const void *W_L, void *O, void *dev, size_t dev_bytes, void *ws,
+                                      size_t ws_bytes, void *stream);
 
 /*
  * Backward pass: gradients of the method with respect to Q, K, V and W_L,

@@ -21,8 +21,8 @@ from . import _native
 from ._native import HSAError, hsa_problem_t
 
 __all__ = ["make_problem", "plan", "workspace_size", "alloc_workspace", "landmarks", "landmarks_refined",
-           "quest_summaries", "select", "select_noalloc", "attend",
-           "forward", "decode_append", "attend_partials", "merge_partials", "device_status", "HSAError",
+           "quest_summaries", "select", "select_noalloc", "attend", "forward", "forward_host",
+           "forward_host_bytes", "decode_append", "attend_partials", "merge_partials", "device_status", "HSAError",
            "hsa_problem_t", "kmax_of", "backward", "backward_workspace_size"]
 
 _DT = {torch.float32: _native.HSA_F32, torch.bfloat16: _native.HSA_BF16}
@@ -232,6 +232,41 @@ def forward(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, L=None, landmarks_ready=False
                                             _stream(Q)), "hsa_forward")
     if return_selection:
         return (O, L) + sel
+    return O
+
+
+def forward_host_bytes(prob: hsa_problem_t) -> int:
+    """hsa_forward_host_bytes: device bytes that hsa_forward_host keeps its copies in."""
+    n = ctypes.c_size_t(0)
+    _native.check(_native.lib().hsa_forward_host_bytes(ctypes.byref(prob), ctypes.byref(n)), "hsa_forward_host_bytes")
+    return int(n.value)
+
+
+def forward_host(Q, K, V, W_L, S, k, tau=0.0, q_pos0=0, O=None, dev=None, ws=None, stream=None, quest=False,
+                 device=None):
+    """hsa_forward_host: the whole forward on HOST tensors (CPU, contiguous; page-locked ones make the
+    copies asynchronous).  Q [B,Tq,H,d], K and V [B,Tcap,Hkv,d], W_L [d,d] (None with quest).  Returns
+    O (a CPU tensor, written when `stream` reaches the call: synchronize before reading it).  dev and
+    ws are device uint8 buffers of forward_host_bytes(prob) and workspace_size(prob) bytes, made on
+    `device` (default: the current CUDA device) when None; calls in flight on different streams need
+    their own.  stream: a torch.cuda.Stream (default: the device's current stream)."""
+    for t in (Q, K, V, W_L, O):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("forward_host takes contiguous host (CPU) tensors")
+    B, Tq, H, d = Q.shape
+    Tcap, Hkv = K.shape[1], K.shape[2]
+    prob = _prob_from(Q, Tcap, Hkv, S, k, tau, q_pos0, _native.HSA_FLAG_QUEST if quest else 0, Tcap)
+    dev_t = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if dev is None:
+        dev = torch.empty(max(256, forward_host_bytes(prob)), dtype=torch.uint8, device=dev_t)
+    if ws is None:
+        ws = alloc_workspace(prob, dev_t)
+    if O is None:
+        O = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned())
+    st = stream if stream is not None else torch.cuda.current_stream(dev_t)
+    _native.check(_native.lib().hsa_forward_host(ctypes.byref(prob), _p(Q), _p(K), _p(V), _p(W_L), _p(O),
+                                                 _p(dev), dev.numel(), _p(ws), ws.numel(), st.cuda_stream),
+                  "hsa_forward_host")
     return O
 
 

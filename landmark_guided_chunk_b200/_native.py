@@ -25,7 +25,7 @@ EXPORTED = ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "
             "hsa_get_device_status", "hsa_plan", "hsa_status_string", "hsa_last_error", "hsa_abi_version",
             "hsa_select_noalloc", "hsa_decode_append", "hsa_attend_partials", "hsa_merge_partials",
             "hsa_backward_workspace_size", "hsa_backward", "hsa_noalloc_status", "hsa_landmarks_refined",
-            "hsa_debug_checks")
+            "hsa_debug_checks", "hsa_forward_host_bytes", "hsa_forward_host")
 PATH_NAMES = {0: "none", 1: "simt_rows", 2: "simt_split", 3: "tensor", 4: "mma_split"}
 
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.hsa_select.argtypes = [prob, P, P, I32p, Fp, I32p, P, Z, P]
     L.hsa_attend.argtypes = [prob, P, P, P, I32p, Fp, I32p, P, P, Z, P]
     L.hsa_forward.argtypes = [prob, P, P, P, P, P, I32p, Fp, I32p, P, P, Z, P]
+    L.hsa_forward_host_bytes.argtypes = [prob, ctypes.POINTER(ctypes.c_size_t)]
+    L.hsa_forward_host.argtypes = [prob, P, P, P, P, P, P, Z, P, Z, P]
     L.hsa_get_device_status.argtypes = [P, Z, P]
     L.hsa_plan.argtypes = [prob, ctypes.POINTER(hsa_plan_t)]
     L.hsa_select_noalloc.argtypes = [prob, P, P, I32p, Fp, I32p, P]
@@ -90,7 +92,7 @@ def lib() -> ctypes.CDLL:
     for f in ("hsa_workspace_size", "hsa_landmarks", "hsa_select", "hsa_attend", "hsa_forward",
               "hsa_get_device_status", "hsa_plan", "hsa_select_noalloc", "hsa_decode_append",
               "hsa_attend_partials", "hsa_merge_partials", "hsa_backward_workspace_size", "hsa_backward",
-              "hsa_noalloc_status", "hsa_landmarks_refined"):
+              "hsa_noalloc_status", "hsa_landmarks_refined", "hsa_forward_host_bytes", "hsa_forward_host"):
         getattr(L, f).restype = ctypes.c_int
     _lib = L
     return L

@@ -231,6 +231,37 @@ static hsa_status_t clear_status(char *ws, const WsLayout &w, cudaStream_t st) {
     return e == cudaSuccess ? HSA_OK : cuda_fail(e, "clearing the device-status word");
 }
 
+// Device copies that hsa_forward_host keeps in the caller's buffer: byte
+// offsets (256-aligned) and sizes of Q, K, V, W_L, the landmarks and O.
+struct HostLayout {
+    size_t q, k, v, w, l, o, total;
+    size_t q_bytes, kv_bytes, w_bytes, l_bytes;
+};
+
+static HostLayout host_layout(const Prob &p) {
+    const size_t es = p.dtype == HSA_BF16 ? 2 : 4;
+    const bool quest = (p.flags & HSA_FLAG_QUEST) != 0;
+    HostLayout h{};
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        const size_t o = off;
+        off += (n + 255) & ~size_t(255);
+        return o;
+    };
+    h.q_bytes = (size_t)p.B * p.Tq * p.H * p.d * es;
+    h.kv_bytes = (size_t)p.B * p.Tcap * p.Hkv * p.d * es;
+    h.w_bytes = quest ? 0 : (size_t)p.d * p.d * es;
+    h.l_bytes = (size_t)p.B * p.Hkv * p.Lc * (quest ? 2 : 1) * p.d * es;
+    h.q = take(h.q_bytes);
+    h.k = take(h.kv_bytes);
+    h.v = take(h.kv_bytes);
+    h.w = take(h.w_bytes);
+    h.l = take(h.l_bytes);
+    h.o = take(h.q_bytes);
+    h.total = off > 256 ? off : 256;
+    return h;
+}
+
 }  // namespace hsa
 
 using namespace hsa;
@@ -461,6 +492,60 @@ hsa_status_t hsa_forward(const hsa_problem_t *prob, const void *Q, const void *K
     if (e != cudaSuccess) return cuda_fail(e, "selection kernel launch");
     e = launch_attend(p, w, Q, K, V, sidx, ssc, skf, O, wsb, st);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+    return HSA_OK;
+}
+
+hsa_status_t hsa_forward_host_bytes(const hsa_problem_t *prob, size_t *bytes) {
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (!bytes) return fail(HSA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = host_layout(p).total;
+    return HSA_OK;
+}
+
+hsa_status_t hsa_forward_host(const hsa_problem_t *prob, const void *Q, const void *K, const void *V,
+                              const void *W_L, void *O, void *dev, size_t dev_bytes, void *ws, size_t ws_bytes,
+                              void *stream) {
+    NvtxRange nvtx_("hsa_forward_host");
+    Prob p;
+    HSA_TRY(validate(prob, &p));
+    if (p.flags & HSA_FLAG_LANDMARKS_READY)
+        return fail(HSA_ERR_INVALID_ARG, "hsa_forward_host makes the landmarks from K: HSA_FLAG_LANDMARKS_READY "
+                    "is not accepted (use hsa_forward)");
+    // the host tensors hsa_forward will read (landmarks are always made here)
+    const bool rows = p.rows > 0;
+    const bool chunks = (long long)p.B * p.C > 0;
+    const bool need_k = (rows && p.C > 0) || chunks;
+    const bool need_v = rows && p.C > 0;
+    const bool need_w = chunks && !(p.flags & HSA_FLAG_QUEST);
+    if (rows && !Q) return fail(HSA_ERR_INVALID_ARG, "Q is NULL");
+    if (need_k && !K) return fail(HSA_ERR_INVALID_ARG, "K is NULL");
+    if (need_v && !V) return fail(HSA_ERR_INVALID_ARG, "V is NULL");
+    if (need_w && !W_L) return fail(HSA_ERR_INVALID_ARG, "W_L is NULL");
+    if (rows && !O) return fail(HSA_ERR_INVALID_ARG, "O is NULL");
+    const HostLayout h = host_layout(p);
+    if (!dev) return fail(HSA_ERR_INVALID_ARG, "device buffer is NULL");
+    if ((uintptr_t)dev & 255u) return fail(HSA_ERR_INVALID_ARG, "device buffer is not 256-byte aligned");
+    if (dev_bytes < h.total)
+        return fail(HSA_ERR_INVALID_ARG, "device buffer has %zu bytes, needs %zu", dev_bytes, h.total);
+    HSA_TRY(check_ws(ws_layout(p), ws, ws_bytes));
+    cudaStream_t st = (cudaStream_t)stream;
+    char *db = (char *)dev;
+    cudaError_t e = cudaSuccess;
+    auto up = [&](size_t off, const void *src, size_t n, bool needed) {
+        if (e == cudaSuccess && needed && n > 0) e = cudaMemcpyAsync(db + off, src, n, cudaMemcpyHostToDevice, st);
+    };
+    up(h.q, Q, h.q_bytes, rows);
+    up(h.k, K, h.kv_bytes, need_k);
+    up(h.v, V, h.kv_bytes, need_v);
+    up(h.w, W_L, h.w_bytes, need_w);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy of the inputs");
+    HSA_TRY(hsa_forward(prob, db + h.q, db + h.k, db + h.v, db + h.w, db + h.l, nullptr, nullptr, nullptr, db + h.o,
+                        ws, ws_bytes, stream));
+    if (rows && h.q_bytes > 0) {
+        e = cudaMemcpyAsync(O, db + h.o, h.q_bytes, cudaMemcpyDeviceToHost, st);
+        if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy of O");
+    }
     return HSA_OK;
 }
 

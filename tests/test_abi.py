@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_native.EXPORTED)
-    assert lib.hsa_abi_version() == 5
+    assert lib.hsa_abi_version() == 6
     assert lib.hsa_debug_checks() == (1 if _native.DEBUG else 0)
 
 
@@ -39,7 +39,7 @@ def test_debug_library_exports_every_declared_symbol():
         assert hasattr(dbg, n), n
     dbg.hsa_abi_version.restype = ctypes.c_int
     dbg.hsa_debug_checks.restype = ctypes.c_int
-    assert dbg.hsa_abi_version() == 5
+    assert dbg.hsa_abi_version() == 6
     assert dbg.hsa_debug_checks() == 1
 
 
@@ -108,6 +108,50 @@ def test_forward_validates_pointers_before_launch():
     assert b"workspace" in _native.lib().hsa_last_error()
     ready = _prob(flags=_native.HSA_FLAG_LANDMARKS_READY)
     assert _call_forward(ready, W=None, L=None) == _native.HSA_ERR_INVALID_ARG   # L is required
+
+
+def _host_bytes(prob):
+    n = ctypes.c_size_t()
+    assert _native.lib().hsa_forward_host_bytes(ctypes.byref(prob), ctypes.byref(n)) == _native.HSA_OK
+    return n.value
+
+
+def test_forward_host_bytes_is_the_sum_of_its_aligned_copies():
+    """Q, K, V, W_L, the landmarks and O, each rounded up to 256 bytes (bf16: 2 bytes an element)."""
+    up = lambda n: (n + 255) // 256 * 256
+    B, T, H, Hkv, d, S = 2, 1000, 4, 2, 64, 64
+    q = B * T * H * d * 2
+    kv = B * 1024 * Hkv * d * 2                                           # K and V copied whole (Tcap = 1024)
+    lm = B * Hkv * (1024 // S) * d * 2
+    p = _prob(B=B, Tq=T, Tkv=T, H=H, Hkv=Hkv, d=d, S=S, kv_cap=1024)
+    assert _host_bytes(p) == up(q) + 2 * up(kv) + up(d * d * 2) + up(lm) + up(q)
+    quest = _prob(B=B, Tq=T, Tkv=T, H=H, Hkv=Hkv, d=d, S=S, kv_cap=1024, flags=_native.HSA_FLAG_QUEST)
+    assert _host_bytes(quest) == up(q) + 2 * up(kv) + up(2 * lm) + up(q)  # no W_L, summaries of width 2d
+    assert _host_bytes(_prob(B=0)) == 64 * 64 * 2                          # W_L alone
+
+
+def _call_forward_host(prob, Q=16, K=16, V=16, W=16, O=16, dev=256, dev_bytes=None, ws=256, ws_bytes=1 << 30):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)
+    dev_bytes = _host_bytes(prob) if dev_bytes is None else dev_bytes
+    return _native.lib().hsa_forward_host(ctypes.byref(prob), P(Q), P(K), P(V), P(W), P(O), P(dev), dev_bytes,
+                                          P(ws), ws_bytes, None)
+
+
+def test_forward_host_validates_before_enqueueing():
+    """Fake, never-dereferenced addresses: every call below must fail in host validation."""
+    p = _prob()
+    for kw in (dict(Q=None), dict(K=None), dict(V=None), dict(W=None), dict(O=None), dict(dev=None),
+               dict(dev=272), dict(dev_bytes=_host_bytes(p) - 1)):
+        assert _call_forward_host(p, **kw) == _native.HSA_ERR_INVALID_ARG, kw
+    assert b"device buffer" in _native.lib().hsa_last_error()
+    assert _call_forward_host(p, ws=None) == _native.HSA_ERR_WORKSPACE
+    assert _call_forward_host(p, ws_bytes=64) == _native.HSA_ERR_WORKSPACE
+    ready = _prob(flags=_native.HSA_FLAG_LANDMARKS_READY)
+    assert _call_forward_host(ready) == _native.HSA_ERR_INVALID_ARG
+    assert b"LANDMARKS_READY" in _native.lib().hsa_last_error()
+    quest = _prob(flags=_native.HSA_FLAG_QUEST)                            # Quest reads no W_L ...
+    assert _call_forward_host(quest, W=None, dev=None) == _native.HSA_ERR_INVALID_ARG
+    assert b"device buffer" in _native.lib().hsa_last_error()             # ... so only the buffer is missing
 
 
 def _call_append(prob, kn=16, vn=16, K=16, V=16, W=16, L=16):

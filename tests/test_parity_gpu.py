@@ -36,7 +36,7 @@ def _oracle_L(p: Problem, inp):
     return oracle.landmarks_stored(K.cpu(), W.cpu(), p.S, p.dtype)
 
 
-def run_case(p: Problem, rows=None, seed=0, landmarks_first=False, force_simt=False):
+def run_case(p: Problem, rows=None, seed=0, landmarks_first=False, force_simt=False, host=False):
     torch.manual_seed(seed)
     inp = make_inputs(p, seed=seed, device="cuda")
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W_L"]
@@ -48,6 +48,13 @@ def run_case(p: Problem, rows=None, seed=0, landmarks_first=False, force_simt=Fa
         O, L, idx, score, keff = hsa.forward(Q, K, V, W, p.S, p.k, p.tau, p.q_pos0, return_selection=True,
                                              force_simt=force_simt)
     torch.cuda.synchronize()
+    if host:
+        # the same forward from page-locked host buffers (hsa_forward_host): its O is the one checked
+        Qh, Kh, Vh, Wh = (x.cpu().pin_memory() for x in (Q, K, V, W))
+        Oh = hsa.forward_host(Qh, Kh, Vh, Wh, p.S, p.k, p.tau, p.q_pos0)
+        torch.cuda.synchronize()
+        assert not Oh.is_cuda
+        O = Oh.cuda()
     L_orc = _oracle_L(p, inp)
     lm = parity.check_landmarks(L, L_orc)
     rb, rt = rows if rows is not None else _rows_all(p)
@@ -112,6 +119,42 @@ def test_small_prefill_all_rows(p):
     assert r["sel"]["ties"] <= max(2, r["sel"]["exact"] // 200)
     print(f"{p.name}: end-to-end selection mismatch vs the oracle's own landmarks: {r['e2e_mismatch']:.4f}")
     assert r["e2e_mismatch"] <= 0.05
+
+
+@pytest.mark.parametrize("p", SMALL[:3], ids=lambda p: p.name)
+def test_forward_from_host_buffers(p):
+    """hsa_forward_host: inputs copied up, the whole forward, O copied down, all on one stream;
+    O checked against the oracle like the device-buffer forward's."""
+    run_case(p, host=True)
+
+
+def test_forward_host_calls_in_flight_on_three_streams():
+    """Six hsa_forward_host calls on three streams, each stream with its own device buffer and
+    workspace, so one call's uploads overlap another's compute and download: each O equals the
+    device-buffer forward of its own inputs (up to the order of the fp32 accumulator additions)."""
+    p = SMALL[1]
+    prob = hsa.make_problem(p.B, p.Tq, p.Tkv, p.H, p.Hkv, p.d, p.S, p.k, p.q_pos0, p.tau, torch.bfloat16)
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    devs = [torch.empty(hsa.forward_host_bytes(prob), dtype=torch.uint8, device="cuda") for _ in streams]
+    wss = [hsa.alloc_workspace(prob) for _ in streams]
+    host_in, outs, expect = [], [], []
+    for seed in range(6):
+        inp = make_inputs(p, seed=100 + seed, device="cuda")
+        dev_in = (inp["Q"], inp["K"], inp["V"], inp["W_L"])
+        expect.append(hsa.forward(*dev_in, p.S, p.k, p.tau, p.q_pos0).float().cpu())
+        host_in.append(tuple(x.cpu().pin_memory() for x in dev_in))
+    torch.cuda.synchronize()
+    for i, (Qh, Kh, Vh, Wh) in enumerate(host_in):
+        j = i % 3
+        outs.append(hsa.forward_host(Qh, Kh, Vh, Wh, p.S, p.k, p.tau, p.q_pos0, dev=devs[j], ws=wss[j],
+                                     stream=streams[j]))
+    torch.cuda.synchronize()
+    for O, E in zip(outs, expect):
+        # one bf16 ulp of the element, plus the fp32 summation-order error of up to kmax terms of |w o| < 8
+        tol = 2.0 ** -7 * E.abs() + 16 * 8 * 2.0 ** -24
+        assert torch.all((O.float() - E).abs() <= tol), (O.float() - E).abs().max()
+    for ws in wss:
+        hsa.device_status(ws)
 
 
 @pytest.mark.parametrize("p", ODD_GROUPS, ids=lambda p: p.name)
