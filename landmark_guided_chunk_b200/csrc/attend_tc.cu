@@ -28,20 +28,11 @@
 // Accumulators.  The pairs are grouped into phases of TB tokens of one (b, kv
 // head), and the tiles are ordered phase-major.  The phases are processed in
 // batches of NB, one kernel launch per batch.  A batch reduces into NB
-// accumulator slots of a ring, which stays resident in L2.  Two orders:
-//  - early (two slots): launch beta first finalises batch beta-1 (its slots ->
-//    bf16 O, slots zeroed), every warp of every CTA taking a share, then runs
-//    the tiles of batch beta, whose slots differ.  The kernel boundary is the
-//    only synchronisation;
-//  - late (three slots): launch beta runs its tiles, then finalises batch
-//    beta-1.  Launches after the first are programmatic dependent launches: a
-//    CTA starts on its SM as soon as the previous launch's CTA there has
-//    exited, so one launch's slowest CTAs overlap the next launch's tiles.  The
-//    finalisation waits for the previous launch to complete; the tiles of
-//    batch beta wait only for a counter saying that slot beta % 3, last used by
-//    batch beta - 3, has been finalised by every CTA (by then it almost always
-//    has, so that wait returns at once).
-// Each shape takes the order that measured faster.
+// accumulator slots of a ring of 2*NB, which stays resident in L2.  Launch
+// beta first finalises batch beta-1 (its slots -> bf16 O, slots zeroed).  Every
+// warp of every CTA takes a share of that, and then the CTA moves on to the
+// tiles of batch beta, whose slots differ.  The kernel boundary is the only
+// synchronisation, so no CTA ever waits for another.
 //
 // Helper kernels (before the batches): count pairs per (phase, chunk) bucket;
 // two-level exclusive scan of pair and tile counts; tile list; scatter of the
@@ -79,10 +70,7 @@ struct AttTcArgs {
     int32_t *blk;                // [2 * nblk] first-level block totals
     int2 *pairs;                 // [rows * kmax]  ((t << 5) | slot, bits of the pair's fusion weight), bucketed
     int4 *tiles;                 // (phase, chunk, first pair, pairs in tile)
-    float *ringbuf;              // [ring*NB][TB][G][d]
-    int ring;                    // accumulator slots (in batches): batch q accumulates into slot q % ring
-    int late;                    // 1: each launch finalises the previous batch after its own tiles (see the kernel)
-    int32_t *fin_cnt;            // [nbatch + 1]: CTAs that have finalised batch q (and zeroed its slot); late only
+    float *ringbuf;              // [2*NB][TB][G][d]
     int d;                       // head dim (64 or 128)
     uint32_t *status;
 };
@@ -98,7 +86,7 @@ __device__ __forceinline__ int phase_of(const AttTcArgs &a, int b, int j, int t)
 
 // ring slot of phase p
 __device__ __forceinline__ float *slot_of(const AttTcArgs &a, int p) {   // accumulator rows of d floats
-    const int s = ((p / NB) % a.ring) * NB + (p % NB);
+    const int s = ((p / NB) & 1) * NB + (p % NB);
     return a.ringbuf + (size_t)s * TB * a.G * a.d;
 }
 
@@ -427,26 +415,6 @@ __device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
                  : "memory");
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Bounded wait until *cnt >= target.  False (abort set, DEV_TIMEOUT recorded) if the limit expired.
-__device__ bool wait_count(const int32_t *cnt, int target, volatile int *abort, uint32_t *status) {
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_gpu(cnt) < target) {
-        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-            *abort = 1;
-            atomicOr(status, DEV_TIMEOUT);
-            return false;
-        }
-        __nanosleep(256);
-    }
-    return true;
-}
-
 // Rows (token, head) of the phases in batch `bt`: accumulators -> bf16 O,
 // accumulators zeroed.  Warps of the whole grid take groups of 8 consecutive
 // rows (2*D float4, D/16 loads in flight per lane).
@@ -505,411 +473,391 @@ __global__ void __launch_bounds__(NT_ATT, 1)
     volatile int *abort = &bar->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // One launch per batch q.  Early order (a.late == 0, two slots): the launch first finalises batch
-    // q - 1, whose slot batch q does not touch, then runs its tiles; the kernel boundary is the only
-    // synchronisation.  Late order (three slots): the launch runs its tiles, then finalises batch q - 1.
-    // Launches after the first are then programmatic dependent launches: a CTA of launch q starts on
-    // its SM as soon as the CTA of launch q - 1 there has exited, so one launch's slowest CTAs overlap
-    // the next launch's tiles.  Batch q accumulates into slot q % 3, last used by batch q - 3, which
-    // launch q - 2 finalised and zeroed: its counter says when every CTA has done so.  Only the
-    // finalisation waits for the whole previous launch (griddepcontrol.wait).
-    if (a.late) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (!a.late && a.batch > 0)
+    // finalise the previous batch (its slots are not touched by this batch's tiles)
+    if (a.batch > 0)
         finalize_batch<D>(a, O, a.batch - 1, blockIdx.x * (NT_ATT / 32) + warp, gridDim.x * (NT_ATT / 32), lane);
-    if (a.batch < a.nbatch) {
-        if (threadIdx.x == 0) {
-            for (int s = 0; s < 2; ++s) {
-                mbar_init(&bar->q_full[s], NPROD);
-                mbar_init(&bar->q_empty[s], 1);
-                mbar_init(&bar->kv_full[s], 1);
-                mbar_init(&bar->kv_empty[s], 1);
-                mbar_init(&bar->s_full[s], 1);
-                mbar_init(&bar->p_full[s], 4);
-                mbar_init(&bar->p_empty[s], 1);
-                mbar_init(&bar->o_full[s], 1);
-                mbar_init(&bar->o_empty[s], 8);
-                mbar_init(&bar->l_full[s], 4);
-                mbar_init(&bar->l_empty[s], 8);
-            }
-            for (int s = 0; s < NINFO; ++s) {
-                mbar_init(&bar->info_full[s], NPROD);
-                mbar_init(&bar->info_empty[s], 8);
-            }
-            mbar_init(&bar->done, 1);
-            bar->abort = 0;
-            const int p0 = a.batch * NB, p1 = min(a.nphase, p0 + NB);
-            bar->tile_lo = a.btile[p0 * a.C];
-            bar->tile_hi = a.btile[p1 * a.C];
-            if (a.late && a.batch >= a.ring) wait_count(&a.fin_cnt[a.batch - a.ring], (int)gridDim.x, abort, a.status);
-            fence_mbar_init();
-        }
-        if (warp == 2) {
-            tmem_alloc(&bar->tmem_base, 512);
-            tmem_relinquish();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        const uint32_t tmem = bar->tmem_base;
-        // TMEM columns: S buffers at 0 and 128, O buffers at 256 and 384 (buffer = tile index & 1)
-        // each CTA takes a contiguous range of the batch's tiles, so the tiles of one
-        // bucket (same chunk) mostly stay together and share one K/V load
-        const int per = (bar->tile_hi - bar->tile_lo + (int)gridDim.x - 1) / (int)gridDim.x;
-        const int tile_lo = min(bar->tile_hi, bar->tile_lo + (int)blockIdx.x * per);
-        const int tile_hi = min(bar->tile_hi, tile_lo + per);
+    if (a.batch >= a.nbatch) return;
 
-        if (*abort) {
-            // the slot was not released in time (DEV_TIMEOUT recorded): no tile is processed
-        } else if (warp < 2) {
-            // ------------------------------------------------------------ producers: Q gather (rows r, r+64), K/V TMA
-            __shared__ const char *rowsrc[MROWS];   // this tile's row sources (each warp writes and reads its own rows)
-            int rr[2], mm[2], gg[2], pr[2];
-            float pw[2];
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar->q_full[s], NPROD);
+            mbar_init(&bar->q_empty[s], 1);
+            mbar_init(&bar->kv_full[s], 1);
+            mbar_init(&bar->kv_empty[s], 1);
+            mbar_init(&bar->s_full[s], 1);
+            mbar_init(&bar->p_full[s], 4);
+            mbar_init(&bar->p_empty[s], 1);
+            mbar_init(&bar->o_full[s], 1);
+            mbar_init(&bar->o_empty[s], 8);
+            mbar_init(&bar->l_full[s], 4);
+            mbar_init(&bar->l_empty[s], 8);
+        }
+        for (int s = 0; s < NINFO; ++s) {
+            mbar_init(&bar->info_full[s], NPROD);
+            mbar_init(&bar->info_empty[s], 8);
+        }
+        mbar_init(&bar->done, 1);
+        bar->abort = 0;
+        const int p0 = a.batch * NB, p1 = min(a.nphase, p0 + NB);
+        bar->tile_lo = a.btile[p0 * a.C];
+        bar->tile_hi = a.btile[p1 * a.C];
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&bar->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+    // TMEM columns: S buffers at 0 and 128, O buffers at 256 and 384 (buffer = tile index & 1)
+    // each CTA takes a contiguous range of the batch's tiles, so the tiles of one
+    // bucket (same chunk) mostly stay together and share one K/V load
+    const int per = (bar->tile_hi - bar->tile_lo + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int tile_lo = min(bar->tile_hi, bar->tile_lo + (int)blockIdx.x * per);
+    const int tile_hi = min(bar->tile_hi, tile_lo + per);
+
+    if (warp < 2) {
+        // ------------------------------------------------------------ producers: Q gather (rows r, r+64), K/V TMA
+        __shared__ const char *rowsrc[MROWS];   // this tile's row sources (each warp writes and reads its own rows)
+        int rr[2], mm[2], gg[2], pr[2];
+        float pw[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                rr[h] = threadIdx.x + h * NPROD;
-                mm[h] = rr[h] / a.G;
-                gg[h] = rr[h] % a.G;
+        for (int h = 0; h < 2; ++h) {
+            rr[h] = threadIdx.x + h * NPROD;
+            mm[h] = rr[h] / a.G;
+            gg[h] = rr[h] % a.G;
+        }
+        int i = 0;
+        bool ok = true;
+        int tau = tile_lo;
+        TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const bool v = tau < tile_hi && mm[h] < T.n;
+            const int2 e = v ? a.pairs[T.start + mm[h]] : make_int2(0, 0);
+            pr[h] = e.x;
+            pw[h] = __int_as_float(e.y);
+        }
+        for (; tau < tile_hi && ok; ++i) {
+            // prefetch the next tile while this one is issued
+            const int tau_n = tau + 1;
+            TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
+            // row info for the O drain (its slot is free once the drain of tile i - NINFO read it)
+            {
+                const int si = i % NINFO, ii = i / NINFO;
+                if (ii > 0 && !(ok = mbar_wait(&bar->info_empty[si], (ii - 1) & 1, abort, a.status))) break;
+                TileRows &ri = info[si];
+                if (threadIdx.x == 0) {
+                    ri.p = T.p;
+                    ri.n = T.n;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const bool v = mm[h] < T.n;
+                    ri.off[rr[h]] = v ? (((pr[h] >> 5) - (T.p % a.ntb) * TB) * a.G + gg[h]) * D : -1;
+                    ri.w[rr[h]] = v ? pw[h] : 0.f;
+                }
+                mbar_arrive(&bar->info_full[si]);
             }
-            int i = 0;
-            bool ok = true;
-            int tau = tile_lo;
-            TileInfo T = tau < tile_hi ? tile_info(a, tau) : TileInfo{};
+            const int sq = i % a.nsq, iq = i / a.nsq;
+            if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
+            // the tile's Q rows: row r of the tile is head gg of token pr >> 5 (padding rows zero-filled)
+            const char *srcs[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const bool v = tau < tile_hi && mm[h] < T.n;
-                const int2 e = v ? a.pairs[T.start + mm[h]] : make_int2(0, 0);
+                srcs[h] = nullptr;
+                if (mm[h] < T.n) {
+                    const int t0 = (T.p % a.ntb) * TB;   // the tile's phase: tokens t0 .. t0 + TB - 1
+                    const int t = (int)dbg_clamp(pr[h] >> 5, t0, min(a.Tq, t0 + TB), a.status);
+                    srcs[h] = reinterpret_cast<const char *>(Q) +
+                              ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
+                }
+            }
+            const uint32_t qbase = smem_u32(sQ + sq * QTILE);
+            if constexpr (D == 128) {
+                // each thread puts its two rows' sources in the warp's table; then every copy
+                // instruction takes four rows x 128 bytes, each 8-lane group one whole 128-byte line
+#pragma unroll
+                for (int h = 0; h < 2; ++h) rowsrc[rr[h]] = srcs[h];
+                __syncwarp();
+                const int cx = lane & 7;
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+#pragma unroll
+                    for (int g4 = 0; g4 < 8; ++g4) {
+                        const int r = warp * 32 + blk * NPROD + g4 * 4 + (lane >> 3);
+                        const char *s = rowsrc[r];
+                        const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128 + ((cx ^ (r & 7)) << 4);
+#pragma unroll
+                        for (int kb = 0; kb < D / 64; ++kb)
+                            cp_async16(dq + kb * 16384, s != nullptr ? s + kb * 128 + cx * 16 : reinterpret_cast<const char *>(Q),
+                                       s != nullptr ? 16u : 0u);
+                    }
+                }
+                __syncwarp();   // the table is rewritten for the next tile only after every lane has read it
+            } else {
+                // 128-byte rows: each thread copies its own two rows (the table measured slower here)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = rr[h];
+                    const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int x = 0; x < D / 8; ++x)
+                        cp_async16(dq + ((x ^ (r & 7)) << 4),
+                                   srcs[h] != nullptr ? srcs[h] + x * 16 : reinterpret_cast<const char *>(Q),
+                                   srcs[h] != nullptr ? 16u : 0u);
+                }
+            }
+            cp_async_arrive(&bar->q_full[sq]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const bool v = tau_n < tile_hi && mm[h] < Tn.n;
+                const int2 e = v ? a.pairs[Tn.start + mm[h]] : make_int2(0, 0);
                 pr[h] = e.x;
                 pw[h] = __int_as_float(e.y);
             }
-            for (; tau < tile_hi && ok; ++i) {
-                // prefetch the next tile while this one is issued
-                const int tau_n = tau + 1;
-                TileInfo Tn = tau_n < tile_hi ? tile_info(a, tau_n) : TileInfo{};
-                // row info for the O drain (its slot is free once the drain of tile i - NINFO read it)
-                {
-                    const int si = i % NINFO, ii = i / NINFO;
-                    if (ii > 0 && !(ok = mbar_wait(&bar->info_empty[si], (ii - 1) & 1, abort, a.status))) break;
-                    TileRows &ri = info[si];
-                    if (threadIdx.x == 0) {
-                        ri.p = T.p;
-                        ri.n = T.n;
-                    }
+            T = Tn;
+            tau = tau_n;
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ K/V loader: one TMA load per bucket run
+        // (consecutive tiles of one (phase, chunk) share a load), as far ahead as the stages allow
+        if (lane == 0) {
+            int nload = 0, prev_p = -1, prev_c = -1;
+            bool ok = true;
+            for (int tau = tile_lo; tau < tile_hi && ok; ++tau) {
+                const int4 e = a.tiles[tau];
+                if (e.x == prev_p && e.y == prev_c) continue;
+                prev_p = e.x;
+                prev_c = e.y;
+                const int bj = (int)dbg_clamp(e.x / a.ntb, 0, (long long)a.B * a.Hkv, a.status);
+                const int Tb = bj / a.Hkv, Tj = bj % a.Hkv;
+                const int cz = (int)dbg_clamp(e.y, 0, a.C, a.status);   // the bucket's chunk
+                const int skv = nload % a.nskv, ikv = nload / a.nskv;
+                if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
+                mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(2 * NBX * kv_bytes));
+                uint8_t *dk = sKV + (size_t)skv * 2 * NBX * kv_bytes;
+                const int z = Tb * a.Tcap + cz * S;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const bool v = mm[h] < T.n;
-                        ri.off[rr[h]] = v ? (((pr[h] >> 5) - (T.p % a.ntb) * TB) * a.G + gg[h]) * D : -1;
-                        ri.w[rr[h]] = v ? pw[h] : 0.f;
-                    }
-                    mbar_arrive(&bar->info_full[si]);
+                for (int kb = 0; kb < NBX; ++kb) {
+                    tma_load_3d(dk + kb * kv_bytes, &tmK, 64 * kb, Tj, z, &bar->kv_full[skv]);
+                    tma_load_3d(dk + (NBX + kb) * kv_bytes, &tmV, 64 * kb, Tj, z, &bar->kv_full[skv]);
                 }
-                const int sq = i % a.nsq, iq = i / a.nsq;
-                if (iq > 0 && !(ok = mbar_wait(&bar->q_empty[sq], (iq - 1) & 1, abort, a.status))) break;
-                // the tile's Q rows: row r of the tile is head gg of token pr >> 5 (padding rows zero-filled)
-                const char *srcs[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    srcs[h] = nullptr;
-                    if (mm[h] < T.n) {
-                        const int t0 = (T.p % a.ntb) * TB;   // the tile's phase: tokens t0 .. t0 + TB - 1
-                        const int t = (int)dbg_clamp(pr[h] >> 5, t0, min(a.Tq, t0 + TB), a.status);
-                        srcs[h] = reinterpret_cast<const char *>(Q) +
-                                  ((((size_t)T.b * a.Tq + t) * a.H + (size_t)T.j * a.G + gg[h]) * D) * 2;
-                    }
-                }
-                const uint32_t qbase = smem_u32(sQ + sq * QTILE);
-                if constexpr (D == 128) {
-                    // each thread puts its two rows' sources in the warp's table; then every copy
-                    // instruction takes four rows x 128 bytes, each 8-lane group one whole 128-byte line
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) rowsrc[rr[h]] = srcs[h];
-                    __syncwarp();
-                    const int cx = lane & 7;
-#pragma unroll
-                    for (int blk = 0; blk < 2; ++blk) {
-#pragma unroll
-                        for (int g4 = 0; g4 < 8; ++g4) {
-                            const int r = warp * 32 + blk * NPROD + g4 * 4 + (lane >> 3);
-                            const char *s = rowsrc[r];
-                            const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128 + ((cx ^ (r & 7)) << 4);
-#pragma unroll
-                            for (int kb = 0; kb < D / 64; ++kb)
-                                cp_async16(dq + kb * 16384, s != nullptr ? s + kb * 128 + cx * 16 : reinterpret_cast<const char *>(Q),
-                                           s != nullptr ? 16u : 0u);
-                        }
-                    }
-                    __syncwarp();   // the table is rewritten for the next tile only after every lane has read it
-                } else {
-                    // 128-byte rows: each thread copies its own two rows (the table measured slower here)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int r = rr[h];
-                        const uint32_t dq = qbase + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                        for (int x = 0; x < D / 8; ++x)
-                            cp_async16(dq + ((x ^ (r & 7)) << 4),
-                                       srcs[h] != nullptr ? srcs[h] + x * 16 : reinterpret_cast<const char *>(Q),
-                                       srcs[h] != nullptr ? 16u : 0u);
-                    }
-                }
-                cp_async_arrive(&bar->q_full[sq]);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const bool v = tau_n < tile_hi && mm[h] < Tn.n;
-                    const int2 e = v ? a.pairs[Tn.start + mm[h]] : make_int2(0, 0);
-                    pr[h] = e.x;
-                    pw[h] = __int_as_float(e.y);
-                }
-                T = Tn;
-                tau = tau_n;
+                ++nload;
             }
-            asm volatile("cp.async.wait_all;" ::: "memory");
-        } else if (warp == 3) {
-            // ------------------------------------------------------------ K/V loader: one TMA load per bucket run
-            // (consecutive tiles of one (phase, chunk) share a load), as far ahead as the stages allow
-            if (lane == 0) {
-                int nload = 0, prev_p = -1, prev_c = -1;
-                bool ok = true;
-                for (int tau = tile_lo; tau < tile_hi && ok; ++tau) {
-                    const int4 e = a.tiles[tau];
-                    if (e.x == prev_p && e.y == prev_c) continue;
-                    prev_p = e.x;
-                    prev_c = e.y;
-                    const int bj = (int)dbg_clamp(e.x / a.ntb, 0, (long long)a.B * a.Hkv, a.status);
-                    const int Tb = bj / a.Hkv, Tj = bj % a.Hkv;
-                    const int cz = (int)dbg_clamp(e.y, 0, a.C, a.status);   // the bucket's chunk
-                    const int skv = nload % a.nskv, ikv = nload / a.nskv;
-                    if (ikv > 0 && !(ok = mbar_wait(&bar->kv_empty[skv], (ikv - 1) & 1, abort, a.status))) break;
-                    mbar_expect_tx(&bar->kv_full[skv], (uint32_t)(2 * NBX * kv_bytes));
-                    uint8_t *dk = sKV + (size_t)skv * 2 * NBX * kv_bytes;
-                    const int z = Tb * a.Tcap + cz * S;
-#pragma unroll
-                    for (int kb = 0; kb < NBX; ++kb) {
-                        tma_load_3d(dk + kb * kv_bytes, &tmK, 64 * kb, Tj, z, &bar->kv_full[skv]);
-                        tma_load_3d(dk + (NBX + kb) * kv_bytes, &tmV, 64 * kb, Tj, z, &bar->kv_full[skv]);
-                    }
+            // wind down: the K/V loads issued have all landed
+            for (int s = 0; s < a.nskv && s < nload; ++s)
+                mbar_drain(&bar->kv_full[s], ((nload - 1 - s) / a.nskv) & 1);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ MMA issuer
+        // With two K/V stages QK(i+1) is issued before PV(i), so the next tile's softmax
+        // overlaps this one's PV; with one stage the order is QK(i), PV(i), ...
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
+            const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
+            const int n_mine = tile_hi - tile_lo;
+            // K/V load index of each tile, derived from the tile records exactly as the loader does;
+            // the records come four tiles ahead, so their L2 round trips stay off this loop
+            int key_p = -1, key_c = -1, nload = 0;
+            auto load_of = [&](int4 e) -> int {   // call with the records of tiles 0, 1, 2, ... in order
+                if (e.x != key_p || e.y != key_c) {
+                    key_p = e.x;
+                    key_c = e.y;
                     ++nload;
                 }
-                // wind down: the K/V loads issued have all landed
-                for (int s = 0; s < a.nskv && s < nload; ++s)
-                    mbar_drain(&bar->kv_full[s], ((nload - 1 - s) / a.nskv) & 1);
-            }
-        } else if (warp == 2) {
-            // ------------------------------------------------------------ MMA issuer
-            // With two K/V stages QK(i+1) is issued before PV(i), so the next tile's softmax
-            // overlaps this one's PV; with one stage the order is QK(i), PV(i), ...
-            if (lane == 0) {
-                const uint32_t idesc_s = idesc_bf16_f32(MROWS, S, 0, 0);
-                const uint32_t idesc_o = idesc_bf16_f32(MROWS, D, 0, 1);
-                const int n_mine = tile_hi - tile_lo;
-                // K/V load index of each tile, derived from the tile records exactly as the loader does;
-                // the records come four tiles ahead, so their L2 round trips stay off this loop
-                int key_p = -1, key_c = -1, nload = 0;
-                auto load_of = [&](int4 e) -> int {   // call with the records of tiles 0, 1, 2, ... in order
-                    if (e.x != key_p || e.y != key_c) {
-                        key_p = e.x;
-                        key_c = e.y;
-                        ++nload;
-                    }
-                    return nload - 1;
-                };
-                auto rec = [&](int t) -> int4 { return t < n_mine ? a.tiles[tile_lo + t] : make_int4(-1, -1, 0, 0); };
-                int4 w1 = rec(1), w2 = rec(2), w3 = rec(3), w4 = rec(4);
-                int waited_load = -1;   // last load whose kv_full has been waited on
-                // QK(i) writes S buffer i & 1, whose previous tile (i - 2) the softmax has released
-                // through p_full before PV(i - 2) was issued, which precedes this call.
-                auto issue_qk = [&](int i, int li) -> bool {
-                    const int sq = i % a.nsq, iq = i / a.nsq, skv = li % a.nskv, ikv = li / a.nskv;
-                    if (!mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status)) return false;
-                    if (li != waited_load) {
-                        if (!mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status)) return false;
-                        waited_load = li;
-                    }
-                    tc_fence_after();
-                    const uint32_t s_tmem = tmem + (i & 1) * 128;
-                    const uint32_t qa = smem_u32(sQ + sq * QTILE);
-                    const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t a_addr = qa + (kk >> 2) * 16384 + (kk & 3) * 32;
-                        const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + (kk & 3) * 32;
-                        umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
-                    }
-                    umma_commit(&bar->s_full[i & 1]);
-                    umma_commit(&bar->q_empty[sq]);
-                    return true;
-                };
-                const bool early = a.nskv >= 2;
-                int li = n_mine > 0 ? load_of(rec(0)) : 0;
-                bool ok = n_mine > 0 ? issue_qk(0, li) : true;
-                for (int i = 0; i < n_mine && ok; ++i) {
-                    const int b = i & 1, k = i >> 1;
-                    const int li_next = i + 1 < n_mine ? load_of(w1) : -1;
-                    w1 = w2;
-                    w2 = w3;
-                    w3 = w4;
-                    w4 = rec(i + 5);
-                    if (early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
-                    if (!(ok = mbar_wait(&bar->p_full[b], k & 1, abort, a.status))) break;
-                    if (k > 0 && !(ok = mbar_wait(&bar->o_empty[b], (k - 1) & 1, abort, a.status))) break;
-                    tc_fence_after();
-                    const int skv = li % a.nskv;
-                    const uint32_t o_tmem = tmem + 256 + b * 128;
-                    const uint32_t pa = smem_u32(sP + b * p_bytes);
-                    const uint32_t vb = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes) + NBX * kv_bytes;
-                    for (int kk = 0; kk < S / 16; ++kk) {
-                        // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
-                        // V: MN-major, keys kk*16..+15 are two 8-row groups starting (kk*16)*128 B
-                        // into each 64-dim box; the two boxes are kv_bytes apart.
-                        const uint32_t a_addr = pa + (kk >> 2) * 16384 + (kk & 3) * 32;
-                        const uint32_t b_addr = vb + kk * 16 * 128;
-                        umma_bf16(o_tmem, desc_kmajor_sw128(a_addr), desc_mnmajor_sw128(b_addr, kv_bytes, 1024), idesc_o,
-                                  kk != 0);
-                    }
-                    umma_commit(&bar->o_full[b]);
-                    umma_commit(&bar->p_empty[b]);
-                    // the K/V stage is free once the last tile of its load is done
-                    if (li_next != li) umma_commit(&bar->kv_empty[skv]);
-                    if (!early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
-                    li = li_next;
+                return nload - 1;
+            };
+            auto rec = [&](int t) -> int4 { return t < n_mine ? a.tiles[tile_lo + t] : make_int4(-1, -1, 0, 0); };
+            int4 w1 = rec(1), w2 = rec(2), w3 = rec(3), w4 = rec(4);
+            int waited_load = -1;   // last load whose kv_full has been waited on
+            // QK(i) writes S buffer i & 1, whose previous tile (i - 2) the softmax has released
+            // through p_full before PV(i - 2) was issued, which precedes this call.
+            auto issue_qk = [&](int i, int li) -> bool {
+                const int sq = i % a.nsq, iq = i / a.nsq, skv = li % a.nskv, ikv = li / a.nskv;
+                if (!mbar_wait(&bar->q_full[sq], iq & 1, abort, a.status)) return false;
+                if (li != waited_load) {
+                    if (!mbar_wait(&bar->kv_full[skv], ikv & 1, abort, a.status)) return false;
+                    waited_load = li;
                 }
-                umma_commit(&bar->done);
-                mbar_drain(&bar->done, 0);
-            }
-        } else if (warp >= 4 && warp < 8) {
-            // ------------------------------------------------------------ softmax: thread = tile row, every tile
-            const int ew = warp & 3;               // TMEM lane quadrant
-            const int r = ew * 32 + lane;
-            const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
-            bool ok = true;
-            for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
-                const int b = i & 1, k = i >> 1;
-                if (!(ok = mbar_wait(&bar->s_full[b], k & 1, abort, a.status))) break;
                 tc_fence_after();
-                const uint32_t s_base = tmem + lane_off + b * 128;
-                uint8_t *myP = sP + b * p_bytes;
-                float l = 0.f;
-                uint32_t sr[32];
-                float mx = -INFINITY;
-                for (int q = 0; q < S / 32; ++q) {
-                    tmem_ld32(s_base + q * 32, sr);
-                    tmem_wait_ld();
+                const uint32_t s_tmem = tmem + (i & 1) * 128;
+                const uint32_t qa = smem_u32(sQ + sq * QTILE);
+                const uint32_t kb0 = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t a_addr = qa + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t b_addr = kb0 + (kk >> 2) * kv_bytes + (kk & 3) * 32;
+                    umma_bf16(s_tmem, desc_kmajor_sw128(a_addr), desc_kmajor_sw128(b_addr), idesc_s, kk != 0);
                 }
-                // P buffer b is free once PV(i - 2) has read it
-                if (k > 0 && !(ok = mbar_wait(&bar->p_empty[b], (k - 1) & 1, abort, a.status))) break;
-                for (int q = 0; q < S / 32; ++q) {
-                    tmem_ld32(s_base + q * 32, sr);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float p0 = exp2f((__uint_as_float(sr[2 * e]) - mx) * a.scale_log2);
-                        const float p1 = exp2f((__uint_as_float(sr[2 * e + 1]) - mx) * a.scale_log2);
-                        __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                        // the MMA sees the rounded probabilities: normalise by their sum
-                        const float2 hf = __bfloat1622float2(h);
-                        l += hf.x + hf.y;
-                        pk[e] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                    uint8_t *prow = myP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const int cx = (q & 1) * 4 + x;
-                        *reinterpret_cast<uint4 *>(prow + ((cx ^ (r & 7)) << 4)) =
-                            make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->p_full[b]);
-                // row sum for the O drain of this tile
-                if (k > 0 && !(ok = mbar_wait(&bar->l_empty[b], (k - 1) & 1, abort, a.status))) break;
-                bar->l[b][r] = l;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->l_full[b]);
-            }
-        } else if (warp >= 8) {
-            // ------------------------------------------------------------ O drain: thread = tile row, D/2 of its columns
-            const int ew = warp & 3;               // TMEM lane quadrant
-            const int hf = (warp - 8) >> 2;        // column half
-            const int r = ew * 32 + lane;
-            const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
-            float *wst = stg + (warp - 8) * 32 * PITCH;
-            bool ok = true;
-            for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
+                umma_commit(&bar->s_full[i & 1]);
+                umma_commit(&bar->q_empty[sq]);
+                return true;
+            };
+            const bool early = a.nskv >= 2;
+            int li = n_mine > 0 ? load_of(rec(0)) : 0;
+            bool ok = n_mine > 0 ? issue_qk(0, li) : true;
+            for (int i = 0; i < n_mine && ok; ++i) {
                 const int b = i & 1, k = i >> 1;
-                const int si = i % NINFO;
-                if (!(ok = mbar_wait(&bar->info_full[si], (i / NINFO) & 1, abort, a.status))) break;
-                const int Tp = info[si].p;
-                const int myoff = info[si].off[r];
-                const float w = info[si].w[r];
-                // destinations of the staging rows this lane will reduce (rows rr*4 + lane/8 of the warp)
-                int dstoff[8];
+                const int li_next = i + 1 < n_mine ? load_of(w1) : -1;
+                w1 = w2;
+                w2 = w3;
+                w3 = w4;
+                w4 = rec(i + 5);
+                if (early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
+                if (!(ok = mbar_wait(&bar->p_full[b], k & 1, abort, a.status))) break;
+                if (k > 0 && !(ok = mbar_wait(&bar->o_empty[b], (k - 1) & 1, abort, a.status))) break;
+                tc_fence_after();
+                const int skv = li % a.nskv;
+                const uint32_t o_tmem = tmem + 256 + b * 128;
+                const uint32_t pa = smem_u32(sP + b * p_bytes);
+                const uint32_t vb = smem_u32(sKV + (size_t)skv * 2 * NBX * kv_bytes) + NBX * kv_bytes;
+                for (int kk = 0; kk < S / 16; ++kk) {
+                    // P: K-major, k-block kk/4 (64 keys each), 32 B per K=16 step inside it.
+                    // V: MN-major, keys kk*16..+15 are two 8-row groups starting (kk*16)*128 B
+                    // into each 64-dim box; the two boxes are kv_bytes apart.
+                    const uint32_t a_addr = pa + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t b_addr = vb + kk * 16 * 128;
+                    umma_bf16(o_tmem, desc_kmajor_sw128(a_addr), desc_mnmajor_sw128(b_addr, kv_bytes, 1024), idesc_o,
+                              kk != 0);
+                }
+                umma_commit(&bar->o_full[b]);
+                umma_commit(&bar->p_empty[b]);
+                // the K/V stage is free once the last tile of its load is done
+                if (li_next != li) umma_commit(&bar->kv_empty[skv]);
+                if (!early && li_next >= 0 && !(ok = issue_qk(i + 1, li_next))) break;
+                li = li_next;
+            }
+            umma_commit(&bar->done);
+            mbar_drain(&bar->done, 0);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ softmax: thread = tile row, every tile
+        const int ew = warp & 3;               // TMEM lane quadrant
+        const int r = ew * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
+        bool ok = true;
+        for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
+            const int b = i & 1, k = i >> 1;
+            if (!(ok = mbar_wait(&bar->s_full[b], k & 1, abort, a.status))) break;
+            tc_fence_after();
+            const uint32_t s_base = tmem + lane_off + b * 128;
+            uint8_t *myP = sP + b * p_bytes;
+            float l = 0.f;
+            uint32_t sr[32];
+            float mx = -INFINITY;
+            for (int q = 0; q < S / 32; ++q) {
+                tmem_ld32(s_base + q * 32, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[e]));
+            }
+            // P buffer b is free once PV(i - 2) has read it
+            if (k > 0 && !(ok = mbar_wait(&bar->p_empty[b], (k - 1) & 1, abort, a.status))) break;
+            for (int q = 0; q < S / 32; ++q) {
+                tmem_ld32(s_base + q * 32, sr);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = exp2f((__uint_as_float(sr[2 * e]) - mx) * a.scale_log2);
+                    const float p1 = exp2f((__uint_as_float(sr[2 * e + 1]) - mx) * a.scale_log2);
+                    __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    // the MMA sees the rounded probabilities: normalise by their sum
+                    const float2 hf = __bfloat1622float2(h);
+                    l += hf.x + hf.y;
+                    pk[e] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                uint8_t *prow = myP + (q >> 1) * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int cx = (q & 1) * 4 + x;
+                    *reinterpret_cast<uint4 *>(prow + ((cx ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->p_full[b]);
+            // row sum for the O drain of this tile
+            if (k > 0 && !(ok = mbar_wait(&bar->l_empty[b], (k - 1) & 1, abort, a.status))) break;
+            bar->l[b][r] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->l_full[b]);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ O drain: thread = tile row, D/2 of its columns
+        const int ew = warp & 3;               // TMEM lane quadrant
+        const int hf = (warp - 8) >> 2;        // column half
+        const int r = ew * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
+        float *wst = stg + (warp - 8) * 32 * PITCH;
+        bool ok = true;
+        for (int i = 0; tile_lo + i < tile_hi && ok; ++i) {
+            const int b = i & 1, k = i >> 1;
+            const int si = i % NINFO;
+            if (!(ok = mbar_wait(&bar->info_full[si], (i / NINFO) & 1, abort, a.status))) break;
+            const int Tp = info[si].p;
+            const int myoff = info[si].off[r];
+            const float w = info[si].w[r];
+            // destinations of the staging rows this lane will reduce (rows rr*4 + lane/8 of the warp)
+            int dstoff[8];
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                // -1 (padding) or the start of a row of the phase's accumulator slot
+                const int o = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
+                dstoff[rr] = o < 0 ? -1 : (int)dbg_clamp(o, 0, (long long)(TB - 1) * a.G * D + 1, a.status);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->info_empty[si]);
+            if (!(ok = mbar_wait(&bar->l_full[b], k & 1, abort, a.status))) break;
+            const float l = bar->l[b][r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->l_empty[b]);
+            const float f = myoff >= 0 ? w / l : 0.f;
+            // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
+            if (!(ok = mbar_wait(&bar->o_full[b], k & 1, abort, a.status))) break;
+            tc_fence_after();
+            float *acc_slot = slot_of(a, Tp) + 4 * (lane & 7);
+            const uint32_t o_base = tmem + lane_off + 256 + b * 128 + hf * (D / 2);
+            for (int q = 0; q < D / 64; ++q) {
+                uint32_t orr[32];
+                tmem_ld32(o_base + q * 32, orr);
+                tmem_wait_ld();
+                if (q == D / 64 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bar->o_empty[b]);
+                }
+                float *mine = wst + lane * PITCH;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(mine + e) =
+                        make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
+                                    __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
+                __syncwarp();
+                const int col = hf * (D / 2) + q * 32;
 #pragma unroll
                 for (int rr = 0; rr < 8; ++rr) {
-                    // -1 (padding) or the start of a row of the phase's accumulator slot
-                    const int o = info[si].off[ew * 32 + rr * 4 + (lane >> 3)];
-                    dstoff[rr] = o < 0 ? -1 : (int)dbg_clamp(o, 0, (long long)(TB - 1) * a.G * D + 1, a.status);
+                    if (dstoff[rr] >= 0) {
+                        const int lr = rr * 4 + (lane >> 3);
+                        red_add_v4(acc_slot + dstoff[rr] + col,
+                                   *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
+                    }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->info_empty[si]);
-                if (!(ok = mbar_wait(&bar->l_full[b], k & 1, abort, a.status))) break;
-                const float l = bar->l[b][r];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->l_empty[b]);
-                const float f = myoff >= 0 ? w / l : 0.f;
-                // O row -> (w/l) * O, reduced into the phase's accumulator slot 32 columns at a time
-                if (!(ok = mbar_wait(&bar->o_full[b], k & 1, abort, a.status))) break;
-                tc_fence_after();
-                float *acc_slot = slot_of(a, Tp) + 4 * (lane & 7);
-                const uint32_t o_base = tmem + lane_off + 256 + b * 128 + hf * (D / 2);
-                for (int q = 0; q < D / 64; ++q) {
-                    uint32_t orr[32];
-                    tmem_ld32(o_base + q * 32, orr);
-                    tmem_wait_ld();
-                    if (q == D / 64 - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&bar->o_empty[b]);
-                    }
-                    float *mine = wst + lane * PITCH;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(mine + e) =
-                            make_float4(__uint_as_float(orr[e]) * f, __uint_as_float(orr[e + 1]) * f,
-                                        __uint_as_float(orr[e + 2]) * f, __uint_as_float(orr[e + 3]) * f);
-                    __syncwarp();
-                    const int col = hf * (D / 2) + q * 32;
-#pragma unroll
-                    for (int rr = 0; rr < 8; ++rr) {
-                        if (dstoff[rr] >= 0) {
-                            const int lr = rr * 4 + (lane >> 3);
-                            red_add_v4(acc_slot + dstoff[rr] + col,
-                                       *reinterpret_cast<const float4 *>(wst + lr * PITCH + 4 * (lane & 7)));
-                        }
-                    }
-                    __syncwarp();
-                }
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 2) {
-            tc_fence_after();
-            tmem_dealloc(tmem, 512);
-        }
     }
-    if (a.late && a.batch > 0) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        finalize_batch<D>(a, O, a.batch - 1, blockIdx.x * (NT_ATT / 32) + warp, gridDim.x * (NT_ATT / 32), lane);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
-            atomicAdd(&a.fin_cnt[a.batch - 1], 1);
-        }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -937,15 +885,11 @@ AttTcLayout attend_tc_layout(const Prob &p) {
     L.nbucket = L.nphase * p.C;
     L.nblk = (L.nbucket + SCAN_BLK - 1) / SCAN_BLK;
     L.tok = MROWS / p.G;
-    // late order (three slots, launches overlapped) where it measured faster; the early order for
-    // d = 128, S = 64, where the finalisation's traffic overlapping other CTAs' tiles cost more
-    // than the overlapped tails saved
-    L.late = !(p.d == 128 && p.S == 64);
-    L.ring = (L.late ? 3 : 2) * NB;
+    L.ring = 2 * NB;
     L.hist = p.C <= HIST_MAX_C;
     const size_t pairs = (size_t)p.rows * p.kmax;
     L.max_tiles = pairs / L.tok + (size_t)L.nbucket + 1;
-    L.counter_ints = 2 * (size_t)L.nbucket + (size_t)(L.nphase + NB - 1) / NB + 1;   // bucket counts, cursors, fin_cnt
+    L.counter_ints = 2 * (size_t)L.nbucket;
     L.ring_bytes = (size_t)L.ring * TB * p.G * p.d * sizeof(float);
     return L;
 }
@@ -991,9 +935,6 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     a.pairs = bf.pairs;
     a.tiles = bf.tiles;
     a.ringbuf = bf.ring;
-    a.ring = L.ring / NB;
-    a.late = L.late ? 1 : 0;
-    a.fin_cnt = bf.counters + 2 * (size_t)L.nbucket;
     a.status = bf.status;
 
     // bucket counters and the accumulator ring start at zero on every call
@@ -1038,22 +979,10 @@ cudaError_t launch_attend_tc(const Prob &p, const AttTcLayout &L, const AttTcBuf
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // launch 0 follows the helper kernels in stream order; in the late order each later launch may start
-    // while the one before it finishes (programmatic dependent launch; the kernel waits where it must)
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sms);
-    cfg.blockDim = dim3(NT_ATT);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
     for (int bt = 0; bt <= a.nbatch; ++bt) {
         a.batch = bt;
-        cfg.attrs = L.late && bt > 0 ? pdl : nullptr;
-        cfg.numAttrs = L.late && bt > 0 ? 1 : 0;
-        if ((e = cudaLaunchKernelEx(&cfg, kern, mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a)) != cudaSuccess)
-            return e;
+        kern<<<sms, NT_ATT, smem, st>>>(mk, mv, (const __nv_bfloat16 *)Q, (__nv_bfloat16 *)O, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -31,7 +31,6 @@ struct Prob {
 struct AttTcLayout {
     int tb, ntb, nsub, nphase, nbucket, nblk, tok, ring;
     bool hist;   // buckets counted through shared-memory histograms (C small enough); else per-pair atomics
-    bool late;   // launches finalise the previous batch after their own tiles (three accumulator slots)
     size_t max_tiles, counter_ints, ring_bytes;
 };
 
